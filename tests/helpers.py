@@ -1,0 +1,25 @@
+"""Shared test helpers: converting synthetic weights for the oracle, tolerances."""
+from __future__ import annotations
+
+import numpy as np
+
+from synth import to_f64
+
+
+def oracle_weights(w: dict) -> dict:
+    """float64 copies of a synth weight dict (exact upcast of bf16/fp32 values)."""
+    return {
+        "embed": to_f64(w["embed"]),
+        "final_norm": to_f64(w["final_norm"]),
+        "layers": [{k: to_f64(v) for k, v in lw.items()} for lw in w["layers"]],
+    }
+
+
+def rel_l2(a, b) -> float:
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+
+
+def max_abs(a, b) -> float:
+    return float(np.max(np.abs(np.asarray(a, dtype=np.float64) - np.asarray(b, dtype=np.float64))))
