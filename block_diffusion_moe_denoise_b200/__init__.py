@@ -1,0 +1,182 @@
+"""B200-native block-diffusion MoE denoising step.
+
+The product is libdg.so, a C-ABI library of sm_100a kernels (include/dg.h,
+include/dg_ops.h).  This module is its thin Python binding: it marshals torch
+device tensors (used only for device memory and streams) into the C calls,
+with the same names.  Every step of the pass runs in the library's kernels;
+if the library is not built the import of `DG` fails loudly.
+"""
+from __future__ import annotations
+
+import ctypes as C
+
+import torch
+
+from . import _ffi
+from ._ffi import DGError, check, dg_config, dg_layer_weights, dg_weights  # noqa: F401
+
+__all__ = ["DG", "DGError", "config_struct", "philox_tokens", "route_topk"]
+
+
+def _ptr(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return C.c_void_p(stream.cuda_stream)
+
+
+def config_struct(cfg) -> dg_config:
+    """dg_config from a synth.ModelConfig-like object."""
+    return dg_config(cfg.n_layers, cfg.d_model, cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim, cfg.n_experts,
+                     cfg.top_k, cfg.ffn_expert, cfg.ffn_shared, cfg.vocab, cfg.canvas, cfg.max_steps,
+                     cfg.min_accept, cfg.entropy_thresh, cfg.rope_theta, cfg.norm_eps)
+
+
+def philox_tokens(seed: int, block: int, step: int, request: int, pos0: int, n: int, vocab: int,
+                  out: torch.Tensor, stream=None) -> None:
+    check(_ffi.load().dg_op_philox_tokens(seed, block, step, request, pos0, n, vocab, _ptr(out), _stream(stream)),
+          "dg_op_philox_tokens")
+
+
+def route_topk(logits: torch.Tensor, k: int, idx: torch.Tensor, w: torch.Tensor, stream=None) -> None:
+    T, E = logits.shape
+    check(_ffi.load().dg_op_route_topk(_ptr(logits), T, E, k, _ptr(idx), _ptr(w), _stream(stream)),
+          "dg_op_route_topk")
+
+
+class DG:
+    """A libdg handle bound to caller-owned torch tensors (weights, workspace)."""
+
+    def __init__(self, cfg, weights: dict, max_requests: int, kv_capacity: int, device="cuda", stream=None):
+        lib = _ffi.load()
+        self.lib = lib
+        self.cfg = cfg
+        self.c_cfg = config_struct(cfg)
+        self.weights = weights            # keep the tensors alive
+        self.stream = stream or torch.cuda.current_stream(device)
+        layers = (dg_layer_weights * cfg.n_layers)()
+        for i, lw in enumerate(weights["layers"]):
+            layers[i] = dg_layer_weights(*[lw[n].data_ptr() for n in (
+                "attn_norm", "w_qkv", "w_o", "ffn_norm", "w_router", "w_gate", "w_up", "w_down", "ws_gate",
+                "ws_up", "ws_down")])
+        self._layers = layers
+        self.c_w = dg_weights(weights["embed"].data_ptr(), weights["final_norm"].data_ptr(), layers)
+        nbytes = lib.dg_workspace_size(C.byref(self.c_cfg), max_requests, kv_capacity)
+        if nbytes == 0:
+            raise DGError(-1, "dg_workspace_size")
+        self.workspace = torch.empty(nbytes + 1024, dtype=torch.uint8, device=device)
+        base = self.workspace.data_ptr()
+        self._ws_off = (-base) % 1024
+        h = C.c_void_p()
+        check(lib.dg_init(C.byref(self.c_cfg), C.byref(self.c_w), max_requests, kv_capacity,
+                          C.c_void_p(base + self._ws_off), nbytes, C.c_void_p(self.stream.cuda_stream),
+                          C.byref(h)), "dg_init")
+        self.h = h
+        self.max_requests = max_requests
+        self.kv_capacity = kv_capacity
+
+    def close(self):
+        if getattr(self, "h", None):
+            self.lib.dg_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # ---- the C ABI, same names ----
+    def prefill(self, req: int, tokens: torch.Tensor):
+        check(self.lib.dg_prefill(self.h, req, _ptr(tokens), tokens.numel()), "dg_prefill")
+
+    def set_kv(self, req: int, layer: int, pos0: int, k: torch.Tensor, v: torch.Tensor):
+        check(self.lib.dg_set_kv(self.h, req, layer, pos0, k.shape[1], _ptr(k), _ptr(v)), "dg_set_kv")
+
+    def get_kv(self, req: int, layer: int, pos0: int, n: int):
+        c = self.cfg
+        k = torch.empty((c.n_kv_heads, n, c.head_dim), dtype=torch.bfloat16, device=self.workspace.device)
+        v = torch.empty_like(k)
+        check(self.lib.dg_get_kv(self.h, req, layer, pos0, n, _ptr(k), _ptr(v)), "dg_get_kv")
+        return k, v
+
+    def set_kv_len(self, req: int, n: int):
+        check(self.lib.dg_set_kv_len(self.h, req, n), "dg_set_kv_len")
+
+    def kv_len(self, req: int) -> int:
+        return self.lib.dg_kv_len(self.h, req)
+
+    def open_canvas(self, req: int, seed: int, block: int):
+        check(self.lib.dg_open_canvas(self.h, req, seed, block), "dg_open_canvas")
+
+    def denoise_step(self, reqs, d_remaining: torch.Tensor | None = None):
+        arr = (C.c_int * len(reqs))(*reqs)
+        check(self.lib.dg_denoise_step(self.h, len(reqs), arr, _ptr(d_remaining)), "dg_denoise_step")
+
+    def read_remaining(self, req: int) -> int:
+        r = C.c_int32()
+        check(self.lib.dg_read_remaining(self.h, req, C.byref(r)), "dg_read_remaining")
+        return r.value
+
+    def commit_block(self, req: int):
+        check(self.lib.dg_commit_block(self.h, req), "dg_commit_block")
+
+    def generate(self, req: int, prompt_host: torch.Tensor, n_out: int, seed: int, out_host: torch.Tensor):
+        n_blocks = n_out // self.cfg.canvas
+        steps = (C.c_int * max(1, n_blocks))()
+        check(self.lib.dg_generate(self.h, req, C.c_void_p(prompt_host.data_ptr()), prompt_host.numel(), n_out, seed,
+                                   C.c_void_p(out_host.data_ptr()), steps), "dg_generate")
+        return list(steps)[:n_blocks]
+
+    def get_canvas(self, req: int):
+        dev = self.workspace.device
+        C_ = self.cfg.canvas
+        tok = torch.empty(C_, dtype=torch.int32, device=dev)
+        mask = torch.empty(C_, dtype=torch.uint8, device=dev)
+        stats = torch.empty((C_, 4), dtype=torch.float32, device=dev)
+        am = torch.empty(C_, dtype=torch.int32, device=dev)
+        check(self.lib.dg_get_canvas(self.h, req, _ptr(tok), _ptr(mask), _ptr(stats), _ptr(am)), "dg_get_canvas")
+        return tok, mask, stats, am
+
+    def set_canvas(self, req: int, tokens: torch.Tensor, mask: torch.Tensor, step: int):
+        check(self.lib.dg_set_canvas(self.h, req, _ptr(tokens), _ptr(mask), step), "dg_set_canvas")
+
+    def sync(self):
+        check(self.lib.dg_sync(self.h), "dg_sync")
+
+    # ---- operation-level entry points ----
+    def op_route_group(self, idx: torch.Tensor, w: torch.Tensor):
+        T = idx.shape[0]
+        dev = idx.device
+        E = self.cfg.n_experts
+        counts = torch.empty(E, dtype=torch.int32, device=dev)
+        offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+        perm = torch.empty(idx.numel(), dtype=torch.int32, device=dev)
+        check(self.lib.dg_op_route_group(self.h, _ptr(idx), _ptr(w), T, _ptr(counts), _ptr(offsets), _ptr(perm)),
+              "dg_op_route_group")
+        return counts, offsets, perm
+
+    def op_sample(self, req: int, entropy, logconf, argmax, step: int):
+        check(self.lib.dg_op_sample(self.h, req, _ptr(entropy), _ptr(logconf), _ptr(argmax), step), "dg_op_sample")
+
+    def op_lm_head(self, x: torch.Tensor, want_logits: bool = False):
+        T = x.shape[0]
+        dev = x.device
+        stats = torch.empty((T, 4), dtype=torch.float32, device=dev)
+        am = torch.empty(T, dtype=torch.int32, device=dev)
+        logits = torch.empty((T, self.cfg.vocab), dtype=torch.float32, device=dev) if want_logits else None
+        check(self.lib.dg_op_lm_head(self.h, _ptr(x), T, _ptr(stats), _ptr(am), _ptr(logits)), "dg_op_lm_head")
+        return stats, am, logits
+
+    def debug_forward(self, req: int, tokens: torch.Tensor, n_layers: int):
+        check(self.lib.dg_debug_forward(self.h, req, _ptr(tokens), tokens.numel(), n_layers), "dg_debug_forward")
+
+    def debug_buffer(self, name: str, dtype: torch.dtype, shape=None) -> torch.Tensor:
+        off, nb = C.c_size_t(), C.c_size_t()
+        check(self.lib.dg_debug_buffer(self.h, name.encode(), C.byref(off), C.byref(nb)), "dg_debug_buffer")
+        o = self._ws_off + off.value
+        t = self.workspace[o: o + nb.value].view(dtype)
+        return t if shape is None else t[: int(torch.tensor(shape).prod())].view(*shape)

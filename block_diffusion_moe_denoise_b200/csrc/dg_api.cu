@@ -1,0 +1,793 @@
+// Host side of libdg: workspace planning, TMA descriptors, the decoder pass
+// orchestration (prefill / denoising step / commit / generate) and the C ABI.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <map>
+#include <string>
+#include <utility>
+
+#include "dg_internal.h"
+
+using namespace dg;
+
+namespace {
+
+constexpr size_t kAlign = 1024;
+constexpr int kLmGridMax = 256;
+constexpr int kSplitCap = 8;
+
+struct LayerMaps {
+  CUtensorMap qkv, o, gate, up, down, sgate, sup, sdown;
+};
+
+struct ReqState {
+  long long kv_len = 0;
+  int block = 0;
+  int step = 0;
+  unsigned long long seed = 0;
+  bool open = false;
+  int last_slot = 0;
+};
+
+// Offsets of every buffer inside the caller's workspace.
+struct Plan {
+  std::map<std::string, std::pair<size_t, size_t>> buf;
+  size_t total = 0;
+  size_t add(const char* name, size_t bytes) {
+    const size_t off = (total + kAlign - 1) / kAlign * kAlign;
+    buf[name] = {off, bytes};
+    total = off + bytes;
+    return off;
+  }
+};
+
+bool config_ok(const dg_config* c) {
+  if (!c) return false;
+  if (c->n_layers < 1 || c->d_model < 256 || c->d_model % 256 != 0) return false;
+  if (!(c->head_dim == 64 || c->head_dim == 128 || c->head_dim == 256)) return false;
+  if (c->n_kv_heads < 1 || c->n_q_heads < 1 || c->n_q_heads % c->n_kv_heads != 0) return false;
+  if (((c->n_q_heads + 2 * c->n_kv_heads) * c->head_dim) % 256 != 0) return false;
+  if ((c->n_q_heads * c->head_dim) % 64 != 0) return false;
+  if (c->n_experts < 1 || c->n_experts > 256 || c->top_k < 1 || c->top_k > 8 || c->top_k > c->n_experts) return false;
+  if (c->ffn_expert < 64 || c->ffn_expert % 64 != 0 || c->ffn_shared < 64 || c->ffn_shared % 64 != 0) return false;
+  if (c->vocab < 256 || c->vocab % 256 != 0) return false;
+  if (c->canvas < 1 || c->canvas > 256) return false;
+  if (c->max_steps < 1 || c->min_accept < 0) return false;
+  return true;
+}
+
+void make_plan(const dg_config* c, int max_req, long long cap, Plan* p) {
+  const int T = max_req * c->canvas;
+  const int Tcap = (T + 127) / 128 * 128;
+  const long long rows = (long long)T * c->top_k;
+  const int D = c->head_dim, d = c->d_model;
+  const long long n_nt = c->n_experts + (rows + 63) / 64;
+  p->add("err", 64);
+  p->add("kv", (size_t)max_req * c->n_layers * 2 * c->n_kv_heads * (size_t)cap * D * 2);
+  p->add("x", (size_t)Tcap * d * 4);
+  p->add("hn", (size_t)Tcap * d * 2);
+  p->add("q", (size_t)c->n_q_heads * Tcap * D * 2);
+  p->add("o", (size_t)Tcap * c->n_q_heads * D * 2);
+  p->add("u", (size_t)Tcap * d * 2);
+  p->add("idx", (size_t)T * c->top_k * 4);
+  p->add("w", (size_t)T * c->top_k * 4);
+  p->add("counts", (size_t)c->n_experts * 4);
+  p->add("offsets", (size_t)(c->n_experts + 1) * 4);
+  p->add("pair_row", (size_t)rows * 4);
+  p->add("row_token", (size_t)rows * 4);
+  p->add("row_weight", (size_t)rows * 4);
+  p->add("row_pair", (size_t)rows * 4);
+  p->add("tile_counts", 64);
+  p->add("egu_tiles", (size_t)n_nt * (c->ffn_expert / 64) * 16);
+  p->add("ed_tiles", (size_t)n_nt * (d / 128) * 16);
+  p->add("xp", (size_t)rows * d * 2);
+  p->add("hp", (size_t)rows * c->ffn_expert * 2);
+  p->add("yp", (size_t)rows * d * 4);
+  p->add("hs", (size_t)Tcap * c->ffn_shared * 2);
+  p->add("attn_o", (size_t)kSplitCap * c->n_q_heads * Tcap * D * 4);
+  p->add("attn_ml", (size_t)kSplitCap * c->n_q_heads * Tcap * 8);
+  p->add("lm_part", (size_t)kLmGridMax * Tcap * 16);
+  p->add("stats", (size_t)Tcap * 16);
+  p->add("argmax", (size_t)Tcap * 4);
+  p->add("canvas", (size_t)max_req * c->canvas * 4);
+  p->add("mask", (size_t)max_req * c->canvas);
+  p->add("remaining", (size_t)max_req * 4);
+  p->add("tok_pos", (size_t)Tcap * 4);
+  p->add("tok_req", (size_t)Tcap * 4);
+  p->add("inv_freq", (size_t)D / 2 * 8);
+  p->add("prompt", (size_t)cap * 4);
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor [rows, K] (K contiguous) read in boxes of 64 x box_rows with
+// the 128-byte swizzle; rows past the end read as zeros.
+bool make_map(CUtensorMap* m, const void* base, long long K, long long rows, int box_rows) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  if ((reinterpret_cast<uintptr_t>(base) & 15) != 0 || (K * 2) % 16 != 0) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+struct dg_handle {
+  dg_config cfg;
+  int max_req = 0;
+  long long cap = 0;
+  cudaStream_t st = nullptr;
+  int num_sms = 0;
+  int T_max = 0, Tcap = 0;
+  const bf16* embed = nullptr;
+  const float* final_norm = nullptr;
+  std::vector<dg_layer_weights> lw;
+  uint8_t* ws = nullptr;
+  Plan plan;
+  int egu_cap = 0, ed_cap = 0;
+  long long kv_req_stride = 0, kv_layer_stride = 0;
+  std::vector<LayerMaps> maps;
+  CUtensorMap tm_hn, tm_o, tm_u, tm_xp, tm_hp, tm_hs, tm_embed;
+  ReqState req[DG_MAX_REQUESTS];
+
+  template <class T>
+  T* B(const char* name) const {
+    return reinterpret_cast<T*>(ws + plan.buf.at(name).first);
+  }
+};
+
+#define CK(expr)                              \
+  do {                                        \
+    cudaError_t e__ = (expr);                 \
+    if (e__ != cudaSuccess) return DG_E_CUDA; \
+  } while (0)
+
+namespace {
+
+// One decoder pass over s.n slots of s.Tr tokens.  n_layers layers; when
+// `qkv_only_last` the last layer runs only its K/V projection (nothing reads
+// the rest: commit and prefill); `want_lm` adds the final norm + LM head.
+int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layers, bool qkv_only_last, bool want_lm,
+             float* logits) {
+  const dg_config& c = h->cfg;
+  const int T = s.n * s.Tr;
+  const int d = c.d_model, D = c.head_dim, k = c.top_k;
+  cudaStream_t st = h->st;
+  int* err = h->B<int>("err");
+  float* x = h->B<float>("x");
+  bf16* hn = h->B<bf16>("hn");
+  CK(run_embed(ids, s, h->embed, c.vocab, d, x, h->B<int>("tok_pos"), h->B<int>("tok_req"), err, st));
+  for (int l = 0; l < n_layers; ++l) {
+    const dg_layer_weights& w = h->lw[l];
+    const LayerMaps& m = h->maps[l];
+    bf16* kv_l = h->B<bf16>("kv") + (size_t)l * h->kv_layer_stride;
+    CK(run_rmsnorm(x, (const float*)w.attn_norm, T, d, c.norm_eps, hn, st));
+    QkvArgs qa;
+    qa.tm_x = &h->tm_hn;
+    qa.tm_w = &m.qkv;
+    qa.T = T;
+    qa.d = d;
+    qa.rows = (c.n_q_heads + 2 * c.n_kv_heads) * D;
+    qa.D = D;
+    qa.Hq = c.n_q_heads;
+    qa.Hkv = c.n_kv_heads;
+    qa.q_T = h->Tcap;
+    qa.kv_cap = (int)h->cap;
+    qa.num_sms = h->num_sms;
+    qa.kv_req_stride = h->kv_req_stride;
+    qa.tok_pos = h->B<int>("tok_pos");
+    qa.tok_req = h->B<int>("tok_req");
+    qa.inv_freq = h->B<double>("inv_freq");
+    qa.q = h->B<bf16>("q");
+    qa.kv = kv_l;
+    qa.err = err;
+    CK(run_qkv(qa, st));
+    if (qkv_only_last && l == c.n_layers - 1) break;
+
+    AttnArgs aa;
+    aa.q = h->B<bf16>("q");
+    aa.q_T = h->Tcap;
+    aa.o = h->B<bf16>("o");
+    aa.kv = kv_l;
+    aa.req_stride = h->kv_req_stride;
+    aa.cap = h->cap;
+    aa.Hq = c.n_q_heads;
+    aa.Hkv = c.n_kv_heads;
+    aa.D = D;
+    aa.Tr = s.Tr;
+    aa.n_slots = s.n;
+    int max_keys = 0;
+    for (int i = 0; i < DG_MAX_REQUESTS; ++i) {
+      aa.req[i] = i < s.n ? s.req[i] : 0;
+      aa.n_keys[i] = i < s.n ? s.pos0[i] + s.Tr : 0;
+      if (aa.n_keys[i] > max_keys) max_keys = aa.n_keys[i];
+    }
+    const int G = c.n_q_heads / c.n_kv_heads;
+    const int base_ctas = ((G * s.Tr + 63) / 64) * c.n_kv_heads * s.n;
+    int split = (h->num_sms + base_ctas - 1) / base_ctas;
+    const int max_by_keys = max_keys / 256 > 0 ? max_keys / 256 : 1;
+    if (split > max_by_keys) split = max_by_keys;
+    if (split > kSplitCap) split = kSplitCap;
+    if (split < 1) split = 1;
+    aa.n_split = split;
+    aa.part_o = h->B<float>("attn_o");
+    aa.part_ml = h->B<float2>("attn_ml");
+    aa.scale = 1.0f / sqrtf((float)D);
+    CK(run_attention(aa, st));
+
+    OprojArgs oa;
+    oa.tm_w = &m.o;
+    oa.tm_o = &h->tm_o;
+    oa.T = T;
+    oa.d = d;
+    oa.K = c.n_q_heads * D;
+    oa.num_sms = h->num_sms;
+    oa.x = x;
+    oa.err = err;
+    CK(run_oproj(oa, st));
+
+    CK(run_router(x, (const float*)w.ffn_norm, c.norm_eps, (const bf16*)w.w_router, T, d, c.n_experts, k,
+                  h->B<bf16>("u"), h->B<int>("idx"), h->B<float>("w"), err, st));
+    GroupArgs ga;
+    ga.idx = h->B<int>("idx");
+    ga.w = h->B<float>("w");
+    ga.T = T;
+    ga.k = k;
+    ga.E = c.n_experts;
+    ga.FJ = c.ffn_expert / 64;
+    ga.MD = d / 128;
+    ga.egu_cap = h->egu_cap;
+    ga.ed_cap = h->ed_cap;
+    ga.counts = h->B<int>("counts");
+    ga.offsets = h->B<int>("offsets");
+    ga.pair_row = h->B<int>("pair_row");
+    ga.row_token = h->B<int>("row_token");
+    ga.row_weight = h->B<float>("row_weight");
+    ga.row_pair = h->B<int>("row_pair");
+    ga.egu_tiles = h->B<int4>("egu_tiles");
+    ga.egu_count = h->B<int>("tile_counts");
+    ga.ed_tiles = h->B<int4>("ed_tiles");
+    ga.ed_count = h->B<int>("tile_counts") + 1;
+    ga.err = err;
+    CK(run_group(ga, st));
+    CK(run_gather(h->B<bf16>("u"), h->B<int>("row_token"), T * k, d, h->B<bf16>("xp"), st));
+
+    ExpertArgs ea;
+    ea.tm_gate = &m.gate;
+    ea.tm_up = &m.up;
+    ea.tm_xp = &h->tm_xp;
+    ea.tm_down = &m.down;
+    ea.tm_hp = &h->tm_hp;
+    ea.d = d;
+    ea.fe = c.ffn_expert;
+    ea.num_sms = h->num_sms;
+    ea.egu_tiles = h->B<int4>("egu_tiles");
+    ea.egu_count = h->B<int>("tile_counts");
+    ea.ed_tiles = h->B<int4>("ed_tiles");
+    ea.ed_count = h->B<int>("tile_counts") + 1;
+    ea.counts = h->B<int>("counts");
+    ea.offsets = h->B<int>("offsets");
+    ea.row_weight = h->B<float>("row_weight");
+    ea.hp = h->B<bf16>("hp");
+    ea.yp = h->B<float>("yp");
+    ea.err = err;
+    CK(run_experts(ea, st));
+
+    SharedArgs sa;
+    sa.tm_u = &h->tm_u;
+    sa.tm_gate = &m.sgate;
+    sa.tm_up = &m.sup;
+    sa.tm_down = &m.sdown;
+    sa.tm_hs = &h->tm_hs;
+    sa.T = T;
+    sa.d = d;
+    sa.fs = c.ffn_shared;
+    sa.k = k;
+    sa.num_sms = h->num_sms;
+    sa.hs = h->B<bf16>("hs");
+    sa.x = x;
+    sa.yp = h->B<float>("yp");
+    sa.pair_row = h->B<int>("pair_row");
+    sa.err = err;
+    CK(run_shared(sa, st));
+  }
+  if (want_lm) {
+    CK(run_rmsnorm(x, h->final_norm, T, d, c.norm_eps, hn, st));
+    LmArgs la;
+    la.tm_x = &h->tm_hn;
+    la.tm_embed = &h->tm_embed;
+    la.T = T;
+    la.d = d;
+    la.num_sms = h->num_sms < kLmGridMax ? h->num_sms : kLmGridMax;
+    la.V = c.vocab;
+    la.part = h->B<float4>("lm_part");
+    la.logits = logits;
+    la.err = err;
+    int grid = 0;
+    CK(run_lm_head(la, &grid, st));
+    CK(run_lm_combine(h->B<float4>("lm_part"), grid, (T + 127) / 128, T, h->B<float>("stats"), h->B<int>("argmax"),
+                      err, st));
+  }
+  return DG_OK;
+}
+
+bool req_ok(const dg_handle* h, int r) { return h && r >= 0 && r < h->max_req; }
+
+}  // namespace
+
+extern "C" {
+
+size_t dg_workspace_size(const dg_config* cfg, int max_requests, int64_t kv_capacity) {
+  if (!config_ok(cfg) || max_requests < 1 || max_requests > DG_MAX_REQUESTS || kv_capacity < cfg->canvas) return 0;
+  Plan p;
+  make_plan(cfg, max_requests, kv_capacity, &p);
+  return p.total;
+}
+
+const char* dg_strerror(int code) {
+  switch (code) {
+    case DG_OK: return "ok";
+    case DG_E_ARG: return "invalid argument or unsupported shape";
+    case DG_E_STATE: return "call not valid in the current request state";
+    case DG_E_CAPACITY: return "KV capacity or workspace too small";
+    case DG_E_CUDA: return "CUDA runtime error";
+    case DG_E_DEVICE: return "a kernel reported a device-side error";
+    case DG_E_UNSUPPORTED: return "no sm_100 device";
+    default: return "unknown error";
+  }
+}
+
+int dg_init(const dg_config* cfg, const dg_weights* wts, int max_requests, int64_t kv_capacity, void* workspace,
+            size_t workspace_bytes, void* stream, dg_handle** out) {
+  if (!out) return DG_E_ARG;
+  *out = nullptr;
+  if (!config_ok(cfg) || !wts || !wts->embed || !wts->final_norm || !wts->layers || !workspace) return DG_E_ARG;
+  if (max_requests < 1 || max_requests > DG_MAX_REQUESTS || kv_capacity < cfg->canvas) return DG_E_ARG;
+  if (kv_capacity > (1ll << 30)) return DG_E_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0) return DG_E_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DG_E_CUDA;
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return DG_E_CUDA;
+  if (prop.major != 10) return DG_E_UNSUPPORTED;
+  if ((size_t)prop.sharedMemPerBlockOptin < gemm_smem_bytes_max()) return DG_E_UNSUPPORTED;
+
+  dg_handle* h = new dg_handle();
+  h->cfg = *cfg;
+  h->max_req = max_requests;
+  h->cap = kv_capacity;
+  h->st = static_cast<cudaStream_t>(stream);
+  h->num_sms = prop.multiProcessorCount;
+  h->T_max = max_requests * cfg->canvas;
+  h->Tcap = (h->T_max + 127) / 128 * 128;
+  h->embed = static_cast<const bf16*>(wts->embed);
+  h->final_norm = static_cast<const float*>(wts->final_norm);
+  h->lw.assign(wts->layers, wts->layers + cfg->n_layers);
+  make_plan(cfg, max_requests, kv_capacity, &h->plan);
+  if (workspace_bytes < h->plan.total) {
+    delete h;
+    return DG_E_CAPACITY;
+  }
+  h->ws = static_cast<uint8_t*>(workspace);
+  const dg_config& c = h->cfg;
+  const int d = c.d_model, D = c.head_dim;
+  h->kv_layer_stride = 2ll * c.n_kv_heads * kv_capacity * D;
+  h->kv_req_stride = h->kv_layer_stride * c.n_layers;
+  const long long rows = (long long)h->T_max * c.top_k;
+  const long long n_nt = c.n_experts + (rows + 63) / 64;
+  h->egu_cap = (int)(n_nt * (c.ffn_expert / 64));
+  h->ed_cap = (int)(n_nt * (d / 128));
+
+  bool ok = true;
+  const int qkv_rows = (c.n_q_heads + 2 * c.n_kv_heads) * D;
+  const long long E = c.n_experts;
+  h->maps.resize(c.n_layers);
+  for (int l = 0; l < c.n_layers && ok; ++l) {
+    const dg_layer_weights& w = h->lw[l];
+    LayerMaps& m = h->maps[l];
+    ok = ok && w.attn_norm && w.ffn_norm && w.w_router;
+    ok = ok && make_map(&m.qkv, w.w_qkv, d, qkv_rows, 256);
+    ok = ok && make_map(&m.o, w.w_o, (long long)c.n_q_heads * D, d, 128);
+    ok = ok && make_map(&m.gate, w.w_gate, d, E * c.ffn_expert, 64);
+    ok = ok && make_map(&m.up, w.w_up, d, E * c.ffn_expert, 64);
+    ok = ok && make_map(&m.down, w.w_down, c.ffn_expert, E * d, 128);
+    ok = ok && make_map(&m.sgate, w.ws_gate, d, c.ffn_shared, 64);
+    ok = ok && make_map(&m.sup, w.ws_up, d, c.ffn_shared, 64);
+    ok = ok && make_map(&m.sdown, w.ws_down, c.ffn_shared, d, 128);
+  }
+  ok = ok && make_map(&h->tm_hn, h->B<bf16>("hn"), d, h->Tcap, 128);
+  ok = ok && make_map(&h->tm_o, h->B<bf16>("o"), (long long)c.n_q_heads * D, h->Tcap, 128);
+  ok = ok && make_map(&h->tm_u, h->B<bf16>("u"), d, h->Tcap, 128);
+  ok = ok && make_map(&h->tm_xp, h->B<bf16>("xp"), d, rows, 64);
+  ok = ok && make_map(&h->tm_hp, h->B<bf16>("hp"), c.ffn_expert, rows, 64);
+  ok = ok && make_map(&h->tm_hs, h->B<bf16>("hs"), c.ffn_shared, h->Tcap, 128);
+  ok = ok && make_map(&h->tm_embed, h->embed, d, c.vocab, 256);
+  if (!ok) {
+    delete h;
+    return DG_E_ARG;
+  }
+  // RoPE inverse frequencies theta^(-2i/D), computed in double
+  std::vector<double> inv(D / 2);
+  for (int i = 0; i < D / 2; ++i) inv[i] = pow((double)c.rope_theta, -2.0 * i / (double)D);
+  if (cudaMemcpyAsync(h->B<double>("inv_freq"), inv.data(), inv.size() * 8, cudaMemcpyHostToDevice, h->st) !=
+          cudaSuccess ||
+      cudaMemsetAsync(h->B<int>("err"), 0, 64, h->st) != cudaSuccess ||
+      cudaMemsetAsync(h->B<int>("remaining"), 0, (size_t)max_requests * 4, h->st) != cudaSuccess ||
+      cudaStreamSynchronize(h->st) != cudaSuccess) {
+    delete h;
+    return DG_E_CUDA;
+  }
+  *out = h;
+  return DG_OK;
+}
+
+void dg_destroy(dg_handle* h) { delete h; }
+
+int64_t dg_kv_len(const dg_handle* h, int req) { return req_ok(h, req) ? h->req[req].kv_len : -1; }
+
+int dg_set_kv(dg_handle* h, int req, int layer, int64_t pos0, int64_t n, const void* d_k, const void* d_v) {
+  if (!req_ok(h, req) || layer < 0 || layer >= h->cfg.n_layers || pos0 < 0 || n < 0 || !d_k || !d_v) return DG_E_ARG;
+  if (pos0 + n > h->cap) return DG_E_CAPACITY;
+  bf16* ck = h->B<bf16>("kv") + req * h->kv_req_stride + layer * h->kv_layer_stride;
+  bf16* cv = ck + (size_t)h->cfg.n_kv_heads * h->cap * h->cfg.head_dim;
+  CK(run_kv_copy(ck, cv, h->cfg.n_kv_heads, h->cap, h->cfg.head_dim, pos0, n, (const bf16*)d_k, (const bf16*)d_v,
+                 nullptr, nullptr, h->st));
+  return DG_OK;
+}
+
+int dg_get_kv(dg_handle* h, int req, int layer, int64_t pos0, int64_t n, void* d_k, void* d_v) {
+  if (!req_ok(h, req) || layer < 0 || layer >= h->cfg.n_layers || pos0 < 0 || n < 0 || !d_k || !d_v) return DG_E_ARG;
+  if (pos0 + n > h->cap) return DG_E_CAPACITY;
+  bf16* ck = h->B<bf16>("kv") + req * h->kv_req_stride + layer * h->kv_layer_stride;
+  bf16* cv = ck + (size_t)h->cfg.n_kv_heads * h->cap * h->cfg.head_dim;
+  CK(run_kv_copy(ck, cv, h->cfg.n_kv_heads, h->cap, h->cfg.head_dim, pos0, n, nullptr, nullptr, (bf16*)d_k,
+                 (bf16*)d_v, h->st));
+  return DG_OK;
+}
+
+int dg_set_kv_len(dg_handle* h, int req, int64_t len) {
+  if (!req_ok(h, req) || len < 0) return DG_E_ARG;
+  if (h->req[req].open) return DG_E_STATE;
+  if (len > h->cap) return DG_E_CAPACITY;
+  h->req[req].kv_len = len;
+  return DG_OK;
+}
+
+int dg_prefill(dg_handle* h, int req, const int32_t* d_tokens, int n) {
+  if (!req_ok(h, req) || n < 0 || (n > 0 && !d_tokens)) return DG_E_ARG;
+  ReqState& r = h->req[req];
+  if (r.open) return DG_E_STATE;
+  if (r.kv_len + n > h->cap) return DG_E_CAPACITY;
+  const int seg = h->cfg.canvas;
+  for (int s0 = 0; s0 < n; s0 += seg) {
+    const int len = n - s0 < seg ? n - s0 : seg;
+    SlotInfo s;
+    memset(&s, 0, sizeof(s));
+    s.n = 1;
+    s.Tr = len;
+    s.req[0] = req;
+    s.pos0[0] = (int)r.kv_len;
+    const int* ids[1] = {d_tokens + s0};
+    int rc = run_pass(h, ids, s, h->cfg.n_layers, true, false, nullptr);
+    if (rc != DG_OK) return rc;
+    r.kv_len += len;
+  }
+  return DG_OK;
+}
+
+int dg_open_canvas(dg_handle* h, int req, uint64_t seed, int block) {
+  if (!req_ok(h, req) || block < 0) return DG_E_ARG;
+  ReqState& r = h->req[req];
+  if (r.kv_len + h->cfg.canvas > h->cap) return DG_E_CAPACITY;
+  const int C = h->cfg.canvas;
+  CK(run_philox_tokens(seed, block, 0, req, 0, C, h->cfg.vocab, h->B<int>("canvas") + (size_t)req * C,
+                       h->B<unsigned char>("mask") + (size_t)req * C, h->st));
+  CK(cudaMemsetAsync(h->B<int>("remaining") + req, 0, 4, h->st));
+  r.open = true;
+  r.seed = seed;
+  r.block = block;
+  r.step = 0;
+  return DG_OK;
+}
+
+static int sample_slots(dg_handle* h, int n_req, const int* reqs, const float* entropy, const float* logconf,
+                        int stride, const int* argmax, const int* steps) {
+  const dg_config& c = h->cfg;
+  SampleArgs a;
+  memset(&a, 0, sizeof(a));
+  a.n_slots = n_req;
+  a.canvas = c.canvas;
+  a.vocab = c.vocab;
+  a.min_accept = c.min_accept;
+  a.max_steps = c.max_steps;
+  a.thr = c.entropy_thresh;
+  for (int i = 0; i < n_req; ++i) {
+    const ReqState& r = h->req[reqs[i]];
+    a.req[i] = reqs[i];
+    a.block[i] = r.block;
+    a.step[i] = steps[i];
+    a.seed[i] = r.seed;
+  }
+  a.entropy = entropy;
+  a.logconf = logconf;
+  a.stride = stride;
+  a.argmax = argmax;
+  a.canvas_tok = h->B<int>("canvas");
+  a.mask = h->B<unsigned char>("mask");
+  a.remaining = h->B<int>("remaining");
+  a.err = h->B<int>("err");
+  CK(run_sample(a, h->st));
+  return DG_OK;
+}
+
+int dg_denoise_step(dg_handle* h, int n_req, const int* reqs, int32_t* d_remaining) {
+  if (!h || n_req < 1 || n_req > h->max_req || !reqs) return DG_E_ARG;
+  for (int i = 0; i < n_req; ++i) {
+    if (!req_ok(h, reqs[i])) return DG_E_ARG;
+    for (int j = 0; j < i; ++j)
+      if (reqs[j] == reqs[i]) return DG_E_ARG;
+    if (!h->req[reqs[i]].open) return DG_E_STATE;
+  }
+  const int C = h->cfg.canvas;
+  SlotInfo s;
+  memset(&s, 0, sizeof(s));
+  s.n = n_req;
+  s.Tr = C;
+  const int* ids[DG_MAX_REQUESTS];
+  int steps[DG_MAX_REQUESTS];
+  for (int i = 0; i < n_req; ++i) {
+    s.req[i] = reqs[i];
+    s.pos0[i] = (int)h->req[reqs[i]].kv_len;
+    ids[i] = h->B<int>("canvas") + (size_t)reqs[i] * C;
+    steps[i] = h->req[reqs[i]].step + 1;
+  }
+  int rc = run_pass(h, ids, s, h->cfg.n_layers, false, true, nullptr);
+  if (rc != DG_OK) return rc;
+  float* stats = h->B<float>("stats");
+  rc = sample_slots(h, n_req, reqs, stats, stats + 1, 4, h->B<int>("argmax"), steps);
+  if (rc != DG_OK) return rc;
+  for (int i = 0; i < n_req; ++i) {
+    h->req[reqs[i]].step = steps[i];
+    h->req[reqs[i]].last_slot = i;
+    if (d_remaining)
+      CK(cudaMemcpyAsync(d_remaining + i, h->B<int>("remaining") + reqs[i], 4, cudaMemcpyDeviceToDevice, h->st));
+  }
+  return DG_OK;
+}
+
+int dg_read_remaining(dg_handle* h, int req, int32_t* remaining) {
+  if (!req_ok(h, req) || !remaining) return DG_E_ARG;
+  CK(cudaMemcpyAsync(remaining, h->B<int>("remaining") + req, 4, cudaMemcpyDeviceToHost, h->st));
+  CK(cudaStreamSynchronize(h->st));
+  return DG_OK;
+}
+
+int dg_commit_block(dg_handle* h, int req) {
+  if (!req_ok(h, req)) return DG_E_ARG;
+  ReqState& r = h->req[req];
+  if (!r.open) return DG_E_STATE;
+  const int C = h->cfg.canvas;
+  SlotInfo s;
+  memset(&s, 0, sizeof(s));
+  s.n = 1;
+  s.Tr = C;
+  s.req[0] = req;
+  s.pos0[0] = (int)r.kv_len;
+  const int* ids[1] = {h->B<int>("canvas") + (size_t)req * C};
+  int rc = run_pass(h, ids, s, h->cfg.n_layers, true, false, nullptr);
+  if (rc != DG_OK) return rc;
+  r.kv_len += C;
+  r.open = false;
+  return DG_OK;
+}
+
+int dg_sync(dg_handle* h) {
+  if (!h) return DG_E_ARG;
+  CK(cudaStreamSynchronize(h->st));
+  int e = 0;
+  CK(cudaMemcpy(&e, h->B<int>("err"), 4, cudaMemcpyDeviceToHost));
+  if (e != 0) {
+    cudaMemset(h->B<int>("err"), 0, 4);
+    return DG_E_DEVICE;
+  }
+  return DG_OK;
+}
+
+int dg_generate(dg_handle* h, int req, const int32_t* h_prompt, int n_prompt, int n_out, uint64_t seed,
+                int32_t* h_out, int* steps_taken) {
+  if (!req_ok(h, req) || n_prompt < 0 || (n_prompt > 0 && !h_prompt) || n_out < 0 || !h_out) return DG_E_ARG;
+  const int C = h->cfg.canvas;
+  if (n_out % C != 0) return DG_E_ARG;
+  ReqState& r = h->req[req];
+  if (r.open || r.kv_len != 0) return DG_E_STATE;
+  if ((long long)n_prompt + n_out > h->cap) return DG_E_CAPACITY;
+  int* prompt = h->B<int>("prompt");
+  if (n_prompt > 0) CK(cudaMemcpyAsync(prompt, h_prompt, (size_t)n_prompt * 4, cudaMemcpyHostToDevice, h->st));
+  int rc = dg_prefill(h, req, prompt, n_prompt);
+  if (rc != DG_OK) return rc;
+  for (int b = 0; b < n_out / C; ++b) {
+    rc = dg_open_canvas(h, req, seed, b);
+    if (rc != DG_OK) return rc;
+    int steps = 0;
+    int32_t rem = 1;
+    while (rem > 0) {
+      rc = dg_denoise_step(h, 1, &req, nullptr);
+      if (rc != DG_OK) return rc;
+      ++steps;
+      rc = dg_read_remaining(h, req, &rem);
+      if (rc != DG_OK) return rc;
+      if (steps >= h->cfg.max_steps && rem > 0) return DG_E_DEVICE;
+    }
+    if (steps_taken) steps_taken[b] = steps;
+    CK(cudaMemcpyAsync(h_out + (size_t)b * C, h->B<int>("canvas") + (size_t)req * C, (size_t)C * 4,
+                       cudaMemcpyDeviceToHost, h->st));
+    rc = dg_commit_block(h, req);
+    if (rc != DG_OK) return rc;
+  }
+  return dg_sync(h);
+}
+
+int dg_get_canvas(dg_handle* h, int req, int32_t* d_tokens, uint8_t* d_mask, float* d_stats, int32_t* d_argmax) {
+  if (!req_ok(h, req)) return DG_E_ARG;
+  const int C = h->cfg.canvas;
+  const ReqState& r = h->req[req];
+  if (d_tokens)
+    CK(cudaMemcpyAsync(d_tokens, h->B<int>("canvas") + (size_t)req * C, (size_t)C * 4, cudaMemcpyDeviceToDevice,
+                       h->st));
+  if (d_mask)
+    CK(cudaMemcpyAsync(d_mask, h->B<unsigned char>("mask") + (size_t)req * C, (size_t)C, cudaMemcpyDeviceToDevice,
+                       h->st));
+  if (d_stats)
+    CK(cudaMemcpyAsync(d_stats, h->B<float>("stats") + (size_t)r.last_slot * C * 4, (size_t)C * 16,
+                       cudaMemcpyDeviceToDevice, h->st));
+  if (d_argmax)
+    CK(cudaMemcpyAsync(d_argmax, h->B<int>("argmax") + (size_t)r.last_slot * C, (size_t)C * 4,
+                       cudaMemcpyDeviceToDevice, h->st));
+  return DG_OK;
+}
+
+int dg_set_canvas(dg_handle* h, int req, const int32_t* d_tokens, const uint8_t* d_mask, int step) {
+  if (!req_ok(h, req) || step < 0) return DG_E_ARG;
+  ReqState& r = h->req[req];
+  if (!r.open) return DG_E_STATE;
+  const int C = h->cfg.canvas;
+  if (d_tokens)
+    CK(cudaMemcpyAsync(h->B<int>("canvas") + (size_t)req * C, d_tokens, (size_t)C * 4, cudaMemcpyDeviceToDevice,
+                       h->st));
+  if (d_mask)
+    CK(cudaMemcpyAsync(h->B<unsigned char>("mask") + (size_t)req * C, d_mask, (size_t)C, cudaMemcpyDeviceToDevice,
+                       h->st));
+  r.step = step;
+  return DG_OK;
+}
+
+// ---- operation-level entry points ----
+
+int dg_op_philox_tokens(uint64_t seed, int block, int step, int request, int64_t pos0, int64_t n, int vocab,
+                        int32_t* d_out, void* stream) {
+  if (n < 0 || vocab < 1 || block < 0 || step < 0 || request < 0 || pos0 < 0 || (n > 0 && !d_out)) return DG_E_ARG;
+  CK(run_philox_tokens(seed, block, step, request, pos0, n, vocab, d_out, nullptr, static_cast<cudaStream_t>(stream)));
+  return DG_OK;
+}
+
+int dg_op_route_topk(const float* d_logits, int T, int E, int k, int32_t* d_idx, float* d_w, void* stream) {
+  if (T < 0 || E < 1 || E > 256 || k < 1 || k > 8 || k > E || (T > 0 && (!d_logits || !d_idx || !d_w))) return DG_E_ARG;
+  CK(run_topk(d_logits, T, E, k, d_idx, d_w, static_cast<cudaStream_t>(stream)));
+  return DG_OK;
+}
+
+int dg_op_route_group(dg_handle* h, const int32_t* d_idx, const float* d_w, int T, int32_t* d_counts,
+                      int32_t* d_offsets, int32_t* d_perm) {
+  if (!h || T < 1 || T > h->T_max || !d_idx || !d_w) return DG_E_ARG;
+  const dg_config& c = h->cfg;
+  GroupArgs ga;
+  ga.idx = d_idx;
+  ga.w = d_w;
+  ga.T = T;
+  ga.k = c.top_k;
+  ga.E = c.n_experts;
+  ga.FJ = c.ffn_expert / 64;
+  ga.MD = c.d_model / 128;
+  ga.egu_cap = h->egu_cap;
+  ga.ed_cap = h->ed_cap;
+  ga.counts = h->B<int>("counts");
+  ga.offsets = h->B<int>("offsets");
+  ga.pair_row = h->B<int>("pair_row");
+  ga.row_token = h->B<int>("row_token");
+  ga.row_weight = h->B<float>("row_weight");
+  ga.row_pair = h->B<int>("row_pair");
+  ga.egu_tiles = h->B<int4>("egu_tiles");
+  ga.egu_count = h->B<int>("tile_counts");
+  ga.ed_tiles = h->B<int4>("ed_tiles");
+  ga.ed_count = h->B<int>("tile_counts") + 1;
+  ga.err = h->B<int>("err");
+  CK(run_group(ga, h->st));
+  if (d_counts)
+    CK(cudaMemcpyAsync(d_counts, ga.counts, (size_t)c.n_experts * 4, cudaMemcpyDeviceToDevice, h->st));
+  if (d_offsets)
+    CK(cudaMemcpyAsync(d_offsets, ga.offsets, (size_t)(c.n_experts + 1) * 4, cudaMemcpyDeviceToDevice, h->st));
+  if (d_perm)
+    CK(cudaMemcpyAsync(d_perm, ga.row_pair, (size_t)T * c.top_k * 4, cudaMemcpyDeviceToDevice, h->st));
+  return DG_OK;
+}
+
+int dg_op_sample(dg_handle* h, int req, const float* d_entropy, const float* d_logconf, const int32_t* d_argmax,
+                 int step) {
+  if (!req_ok(h, req) || !d_entropy || !d_logconf || !d_argmax || step < 1) return DG_E_ARG;
+  if (!h->req[req].open) return DG_E_STATE;
+  int steps[1] = {step};
+  int rc = sample_slots(h, 1, &req, d_entropy, d_logconf, 1, d_argmax, steps);
+  if (rc == DG_OK) h->req[req].step = step;
+  return rc;
+}
+
+int dg_op_lm_head(dg_handle* h, const float* d_x, int T, float* d_stats, int32_t* d_argmax, float* d_logits) {
+  if (!h || T < 1 || T > h->T_max || !d_x) return DG_E_ARG;
+  const dg_config& c = h->cfg;
+  float* x = h->B<float>("x");
+  CK(cudaMemcpyAsync(x, d_x, (size_t)T * c.d_model * 4, cudaMemcpyDeviceToDevice, h->st));
+  CK(run_rmsnorm(x, h->final_norm, T, c.d_model, c.norm_eps, h->B<bf16>("hn"), h->st));
+  LmArgs la;
+  la.tm_x = &h->tm_hn;
+  la.tm_embed = &h->tm_embed;
+  la.T = T;
+  la.d = c.d_model;
+  la.num_sms = h->num_sms < kLmGridMax ? h->num_sms : kLmGridMax;
+  la.V = c.vocab;
+  la.part = h->B<float4>("lm_part");
+  la.logits = d_logits;
+  la.err = h->B<int>("err");
+  int grid = 0;
+  CK(run_lm_head(la, &grid, h->st));
+  CK(run_lm_combine(la.part, grid, (T + 127) / 128, T, h->B<float>("stats"), h->B<int>("argmax"), la.err, h->st));
+  if (d_stats) CK(cudaMemcpyAsync(d_stats, h->B<float>("stats"), (size_t)T * 16, cudaMemcpyDeviceToDevice, h->st));
+  if (d_argmax) CK(cudaMemcpyAsync(d_argmax, h->B<int>("argmax"), (size_t)T * 4, cudaMemcpyDeviceToDevice, h->st));
+  return DG_OK;
+}
+
+int dg_debug_forward(dg_handle* h, int req, const int32_t* d_tokens, int T, int n_layers) {
+  if (!req_ok(h, req) || !d_tokens || T < 1 || T > h->cfg.canvas || n_layers < 1 || n_layers > h->cfg.n_layers)
+    return DG_E_ARG;
+  const ReqState& r = h->req[req];
+  if (r.kv_len + T > h->cap) return DG_E_CAPACITY;
+  SlotInfo s;
+  memset(&s, 0, sizeof(s));
+  s.n = 1;
+  s.Tr = T;
+  s.req[0] = req;
+  s.pos0[0] = (int)r.kv_len;
+  const int* ids[1] = {d_tokens};
+  return run_pass(h, ids, s, n_layers, false, n_layers == h->cfg.n_layers, nullptr);
+}
+
+int dg_debug_buffer(const dg_handle* h, const char* name, size_t* offset, size_t* bytes) {
+  if (!h || !name) return DG_E_ARG;
+  auto it = h->plan.buf.find(name);
+  if (it == h->plan.buf.end()) return DG_E_ARG;
+  if (offset) *offset = it->second.first;
+  if (bytes) *bytes = it->second.second;
+  return DG_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,154 @@
+// Internal declarations shared by the libdg translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <vector>
+
+#include "../../include/dg.h"
+#include "../../include/dg_ops.h"
+
+namespace dg {
+
+using bf16 = __nv_bfloat16;
+
+// ---- arguments of the tcgen05 GEMM launchers (gemm_ops.cu) ----
+struct QkvArgs {
+  const CUtensorMap* tm_x;  // normed tokens [Tcap, d]
+  const CUtensorMap* tm_w;  // w_qkv
+  int T, d, rows, D, Hq, Hkv, q_T, kv_cap, num_sms;
+  long long kv_req_stride;
+  const int* tok_pos;
+  const int* tok_req;
+  const double* inv_freq;
+  bf16* q;
+  bf16* kv;
+  int* err;
+};
+struct OprojArgs {
+  const CUtensorMap* tm_w;
+  const CUtensorMap* tm_o;
+  int T, d, K, num_sms;
+  float* x;
+  int* err;
+};
+struct ExpertArgs {
+  const CUtensorMap *tm_gate, *tm_up, *tm_xp, *tm_down, *tm_hp;
+  int d, fe, num_sms;
+  const int4* egu_tiles;
+  const int* egu_count;
+  const int4* ed_tiles;
+  const int* ed_count;
+  const int* counts;
+  const int* offsets;
+  const float* row_weight;
+  bf16* hp;
+  float* yp;
+  int* err;
+};
+struct SharedArgs {
+  const CUtensorMap *tm_u, *tm_gate, *tm_up, *tm_down, *tm_hs;
+  int T, d, fs, k, num_sms;
+  bf16* hs;
+  float* x;
+  const float* yp;
+  const int* pair_row;
+  int* err;
+};
+struct LmArgs {
+  const CUtensorMap* tm_x;
+  const CUtensorMap* tm_embed;
+  int T, d, num_sms;
+  long long V;
+  float4* part;
+  float* logits;
+  int* err;
+};
+
+cudaError_t run_qkv(const QkvArgs& a, cudaStream_t st);
+cudaError_t run_oproj(const OprojArgs& a, cudaStream_t st);
+cudaError_t run_experts(const ExpertArgs& a, cudaStream_t st);
+cudaError_t run_shared(const SharedArgs& a, cudaStream_t st);
+cudaError_t run_lm_head(const LmArgs& a, int* grid_out, cudaStream_t st);
+size_t gemm_smem_bytes_max();
+
+// ---- small kernels (kernels.cu) ----
+struct SlotInfo {
+  int n;                       // slots (requests) in this pass
+  int Tr;                      // tokens per slot
+  int req[DG_MAX_REQUESTS];    // request of each slot
+  int pos0[DG_MAX_REQUESTS];   // position of the slot's first token
+};
+
+// ids[slot] points at the slot's Tr token ids
+cudaError_t run_embed(const int* const* ids, const SlotInfo& s, const bf16* embed, int V, int d, float* x, int* tok_pos,
+                      int* tok_req, int* err, cudaStream_t st);
+cudaError_t run_rmsnorm(const float* x, const float* g, int T, int d, float eps, bf16* out, cudaStream_t st);
+cudaError_t run_router(const float* x, const float* g, float eps, const bf16* wr, int T, int d, int E, int k,
+                       bf16* u, int* idx, float* w, int* err, cudaStream_t st);
+cudaError_t run_topk(const float* logits, int T, int E, int k, int* idx, float* w, cudaStream_t st);
+struct GroupArgs {
+  const int* idx;
+  const float* w;
+  int T, k, E, FJ, MD, egu_cap, ed_cap;
+  int* counts;
+  int* offsets;
+  int* pair_row;
+  int* row_token;
+  float* row_weight;
+  int* row_pair;
+  int4* egu_tiles;
+  int* egu_count;
+  int4* ed_tiles;
+  int* ed_count;
+  int* err;
+};
+cudaError_t run_group(const GroupArgs& a, cudaStream_t st);
+cudaError_t run_gather(const bf16* u, const int* row_token, int rows, int d, bf16* xp, cudaStream_t st);
+cudaError_t run_lm_combine(const float4* part, int G, int MT, int T, float* stats, int* argmax, int* err,
+                           cudaStream_t st);
+struct SampleArgs {
+  int n_slots, canvas, vocab, min_accept, max_steps;
+  float thr;
+  int req[DG_MAX_REQUESTS];
+  int block[DG_MAX_REQUESTS];
+  int step[DG_MAX_REQUESTS];
+  unsigned long long seed[DG_MAX_REQUESTS];
+  const float* entropy;   // [slot*canvas + i] * stride
+  const float* logconf;   // [slot*canvas + i] * stride
+  int stride;             // floats between consecutive positions
+  const int* argmax;      // [slot*canvas + i]
+  int* canvas_tok;        // [req][canvas]
+  unsigned char* mask;    // [req][canvas]
+  int* remaining;         // [req]
+  int* err;
+};
+cudaError_t run_sample(const SampleArgs& a, cudaStream_t st);
+cudaError_t run_philox_tokens(unsigned long long seed, int block, int step, int request, long long pos0, long long n,
+                              int vocab, int* out, unsigned char* mask_clear, cudaStream_t st);
+cudaError_t run_kv_copy(bf16* cache_k, bf16* cache_v, int Hkv, long long cap, int D, long long pos0, long long n,
+                        const bf16* k_in, const bf16* v_in, bf16* k_out, bf16* v_out, cudaStream_t st);
+
+// ---- attention (attention.cu) ----
+struct AttnArgs {
+  const bf16* q;     // [Hq][q_T][D]
+  int q_T;
+  bf16* o;           // [T][Hq*D]
+  const bf16* kv;    // this layer's K block of request 0
+  long long req_stride;
+  long long cap;
+  int Hq, Hkv, D, Tr, n_slots;
+  int req[DG_MAX_REQUESTS];
+  int n_keys[DG_MAX_REQUESTS];
+  int n_split;       // key splits (1 = direct)
+  float* part_o;     // [n_split][Hq][q_T][D]
+  float2* part_ml;   // [n_split][Hq][q_T]
+  float scale;
+};
+cudaError_t run_attention(const AttnArgs& a, cudaStream_t st);
+int attention_split_cap();
+
+}  // namespace dg

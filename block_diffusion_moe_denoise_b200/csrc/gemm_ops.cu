@@ -1,0 +1,653 @@
+// The dense contractions of the denoising pass on the tcgen05 GEMM engine,
+// each with its epilogue fused:
+//   qkv     RMSNorm'd tokens x W_qkv^T, rotate-half RoPE on q/k, q -> [Hq][T][D],
+//           k/v -> KV cache slots of the canvas (or prefill segment)
+//   oproj   x += O W_o^T                               (weights as the 128-row operand)
+//   egu     routed experts, gate|up for 64 hidden units per tile, SwiGLU in the
+//           epilogue (weights as the 128-row operand, the expert's tokens as N)
+//   ed      routed experts, down projection scaled by the pair's routing weight
+//   sgu     shared expert gate|up + SwiGLU (tokens as the 128-row operand)
+//   sd      shared expert down + sum of the token's routed outputs + residual
+//   lm      tied LM head with per-row online max / argmax / sum e^(z-m) /
+//           sum e^(z-m)(z-m) so the logits are never written
+// Structure of a decoder layer and the MoE: DiffusionGemma pages ("26B MoE
+// Architecture, but Only 3.8B Activated"; "The speed numbers and the hardware
+// they require": 128 experts, 8 active plus one shared expert).
+#include "dg_internal.h"
+#include "umma_gemm.cuh"
+
+namespace dg {
+
+DG_DEVINL void store_bf16x16(__nv_bfloat16* dst, const float* v) {
+  uint4 a, b;
+  a.x = pack_bf16x2(v[0], v[1]);
+  a.y = pack_bf16x2(v[2], v[3]);
+  a.z = pack_bf16x2(v[4], v[5]);
+  a.w = pack_bf16x2(v[6], v[7]);
+  b.x = pack_bf16x2(v[8], v[9]);
+  b.y = pack_bf16x2(v[10], v[11]);
+  b.z = pack_bf16x2(v[12], v[13]);
+  b.w = pack_bf16x2(v[14], v[15]);
+  reinterpret_cast<uint4*>(dst)[0] = a;
+  reinterpret_cast<uint4*>(dst)[1] = b;
+}
+
+// ---------------------------------------------------------------------------
+// QKV projection + RoPE + KV-cache write
+// ---------------------------------------------------------------------------
+struct P_QKV : ProblemBase {
+  static constexpr int BN = 256, STAGES = 4, B_STAGE = BN * 128, TMEM_COLS = 512;
+  struct Params {
+    CUtensorMap tmA;  // normed tokens [Tcap, d]
+    CUtensorMap tmB;  // w_qkv [(Hq+2Hkv)*D, d]
+    int T, nk, MT, NT, D, Hq, Hkv, q_T, kv_cap;
+    long long kv_req_stride;
+    const int* tok_pos;
+    const int* tok_req;
+    const double* inv_freq;  // [D/2]
+    __nv_bfloat16* q;
+    __nv_bfloat16* kv;  // this layer's K block of request 0; V follows after Hkv*cap*D
+    int* err;
+  };
+  DG_DEVINL static void prefetch(const Params& p) {
+    tma_prefetch_desc(&p.tmA);
+    tma_prefetch_desc(&p.tmB);
+  }
+  DG_DEVINL static int num_tiles(const Params& p) { return p.MT * p.NT; }
+  DG_DEVINL static Tile tile(const Params& p, int v) {
+    Tile t;
+    t.valid = 1;
+    t.nk = p.nk;
+    t.n_mma = BN;
+    t.a = v % p.MT;  // token tile
+    t.b = v / p.MT;  // 256-row block of W_qkv
+    return t;
+  }
+  DG_DEVINL static uint32_t tx_bytes(const Params&, const Tile&) { return kAStage + B_STAGE; }
+  DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
+    tma_load_2d(sa, &p.tmA, kb * 64, t.a * 128, bar);
+    tma_load_2d(sb, &p.tmB, kb * 64, t.b * 256, bar);
+  }
+  DG_DEVINL static void epilogue(const Params& p, const Tile& t, uint32_t taddr, int, int, int row, uint8_t*) {
+    const int tok = t.a * 128 + row;
+    const bool ok = tok < p.T;
+    const int pos = ok ? p.tok_pos[tok] : 0;
+    const int req = ok ? p.tok_req[tok] : 0;
+    const int D = p.D, half = D >> 1;
+    for (int hh = 0; hh < 256 / D; ++hh) {
+      const int r0 = t.b * 256 + hh * D;
+      const uint32_t col0 = (uint32_t)(hh * D);
+      int kind, head;
+      if (r0 < p.Hq * D) {
+        kind = 0;
+        head = r0 / D;
+      } else if (r0 < (p.Hq + p.Hkv) * D) {
+        kind = 1;
+        head = (r0 - p.Hq * D) / D;
+      } else {
+        kind = 2;
+        head = (r0 - (p.Hq + p.Hkv) * D) / D;
+      }
+      __nv_bfloat16* dst;
+      if (kind == 0)
+        dst = p.q + ((size_t)head * p.q_T + tok) * D;
+      else
+        dst = p.kv + (size_t)req * p.kv_req_stride +
+              ((size_t)(kind == 2 ? p.Hkv : 0) + head) * (size_t)p.kv_cap * D + (size_t)pos * D;
+      if (kind == 2) {
+        for (int c = 0; c < D; c += 16) {
+          float v[16];
+          tmem_ld16(taddr + col0 + c, v);
+          if (ok) store_bf16x16(dst + c, v);
+        }
+      } else {
+        for (int i0 = 0; i0 < half; i0 += 16) {
+          float x1[16], x2[16];
+          tmem_ld16(taddr + col0 + i0, x1);
+          tmem_ld16(taddr + col0 + half + i0, x2);
+          if (ok) {
+            float y1[16], y2[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              // angle in fp64, reduced to [-pi, pi] before the fp32 sincos
+              double a = (double)pos * p.inv_freq[i0 + i];
+              a -= rint(a * 0.15915494309189535) * 6.283185307179586;
+              float s, c;
+              sincosf((float)a, &s, &c);
+              y1[i] = x1[i] * c - x2[i] * s;
+              y2[i] = x2[i] * c + x1[i] * s;
+            }
+            store_bf16x16(dst + i0, y1);
+            store_bf16x16(dst + half + i0, y2);
+          }
+        }
+      }
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------
+// Output projection + residual: x[t, f] += sum_c O[t, c] W_o[f, c]
+// ---------------------------------------------------------------------------
+struct P_OPROJ : ProblemBase {
+  static constexpr int BN = 128, STAGES = 6, B_STAGE = BN * 128, TMEM_COLS = 256;
+  struct Params {
+    CUtensorMap tmA;  // w_o [d, Hq*D]
+    CUtensorMap tmB;  // O [Tcap, Hq*D]
+    int T, nk, MT, NT, d;
+    float* x;
+    int* err;
+  };
+  DG_DEVINL static void prefetch(const Params& p) {
+    tma_prefetch_desc(&p.tmA);
+    tma_prefetch_desc(&p.tmB);
+  }
+  DG_DEVINL static int num_tiles(const Params& p) { return p.MT * p.NT; }
+  DG_DEVINL static Tile tile(const Params& p, int v) {
+    Tile t;
+    t.valid = 1;
+    t.nk = p.nk;
+    t.b = v % p.NT;  // token tile
+    t.a = v / p.NT;  // 128 output features
+    t.n_mma = round_up16(min(128, p.T - t.b * 128));
+    return t;
+  }
+  DG_DEVINL static uint32_t tx_bytes(const Params&, const Tile&) { return kAStage + B_STAGE; }
+  DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
+    tma_load_2d(sa, &p.tmA, kb * 64, t.a * 128, bar);
+    tma_load_2d(sb, &p.tmB, kb * 64, t.b * 128, bar);
+  }
+  DG_DEVINL static void epilogue(const Params& p, const Tile& t, uint32_t taddr, int, int, int row, uint8_t*) {
+    const int f = t.a * 128 + row;
+    for (int c0 = 0; c0 < t.n_mma; c0 += 16) {
+      float v[16];
+      tmem_ld16(taddr + c0, v);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int tok = t.b * 128 + c0 + j;
+        if (tok < p.T) p.x[(size_t)tok * p.d + f] += v[j];
+      }
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------
+// Routed experts, gate|up + SwiGLU.  Tile (e, j, nt): hidden units j*64..+63 of
+// expert e for its tokens nt*64..+63 (rows of the expert-grouped buffer).
+// A rows 0..63 = W_gate rows, 64..127 = W_up rows of the same hidden units.
+// ---------------------------------------------------------------------------
+struct P_EGU : ProblemBase {
+  static constexpr int BN = 64, STAGES = 8, B_STAGE = BN * 128, TMEM_COLS = 128;
+  static constexpr int EP_SMEM = 64 * 17 * 4;
+  struct Params {
+    CUtensorMap tmG;  // w_gate as [E*fe, d]
+    CUtensorMap tmU;  // w_up   as [E*fe, d]
+    CUtensorMap tmX;  // expert-grouped tokens [rows_cap, d]
+    int nk, fe;
+    const int4* tiles;
+    const int* n_tiles;
+    const int* counts;
+    const int* offsets;
+    __nv_bfloat16* hp;  // [rows_cap, fe]
+    int* err;
+  };
+  DG_DEVINL static void prefetch(const Params& p) {
+    tma_prefetch_desc(&p.tmG);
+    tma_prefetch_desc(&p.tmU);
+    tma_prefetch_desc(&p.tmX);
+  }
+  DG_DEVINL static int num_tiles(const Params& p) { return *p.n_tiles; }
+  DG_DEVINL static Tile tile(const Params& p, int v) {
+    const int4 tt = p.tiles[v];
+    Tile t;
+    t.a = tt.x;  // expert
+    t.b = tt.y;  // hidden-unit block
+    const int nt = tt.z;
+    const int n_valid = min(64, p.counts[t.a] - nt * 64);
+    t.valid = n_valid > 0;
+    t.c = n_valid;
+    t.d = p.offsets[t.a] + nt * 64;  // first grouped row
+    t.nk = p.nk;
+    t.n_mma = round_up16(n_valid);
+    return t;
+  }
+  DG_DEVINL static uint32_t tx_bytes(const Params&, const Tile&) { return kAStage + B_STAGE; }
+  DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
+    const int r = t.a * p.fe + t.b * 64;
+    tma_load_2d(sa, &p.tmG, kb * 64, r, bar);
+    tma_load_2d(sa + 64 * 128, &p.tmU, kb * 64, r, bar);
+    tma_load_2d(sb, &p.tmX, kb * 64, t.d, bar);
+  }
+  DG_DEVINL static void epilogue(const Params& p, const Tile& t, uint32_t taddr, int, int, int row, uint8_t* ep) {
+    float* xch = reinterpret_cast<float*>(ep);
+    for (int c0 = 0; c0 < t.n_mma; c0 += 16) {
+      float v[16];
+      tmem_ld16(taddr + c0, v);
+      if (row >= 64) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) xch[(row - 64) * 17 + i] = v[i];
+      }
+      named_bar_sync(1, 128);
+      if (row < 64) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int c = c0 + i;
+          if (c < t.c) {
+            const float h = silu_f(v[i]) * xch[row * 17 + i];
+            p.hp[(size_t)(t.d + c) * p.fe + t.b * 64 + row] = f2bf(h);
+          }
+        }
+      }
+      named_bar_sync(1, 128);
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------
+// Routed experts, down projection.  Tile (e, m, nt): output features m*128..+127
+// of expert e for its grouped rows nt*64..+63; each row scaled by its gate weight.
+// ---------------------------------------------------------------------------
+struct P_ED : ProblemBase {
+  static constexpr int BN = 64, STAGES = 8, B_STAGE = BN * 128, TMEM_COLS = 128;
+  struct Params {
+    CUtensorMap tmW;  // w_down as [E*d, fe]
+    CUtensorMap tmH;  // hidden [rows_cap, fe]
+    int nk, d;
+    const int4* tiles;
+    const int* n_tiles;
+    const int* counts;
+    const int* offsets;
+    const float* row_weight;
+    float* yp;  // [rows_cap, d]
+    int* err;
+  };
+  DG_DEVINL static void prefetch(const Params& p) {
+    tma_prefetch_desc(&p.tmW);
+    tma_prefetch_desc(&p.tmH);
+  }
+  DG_DEVINL static int num_tiles(const Params& p) { return *p.n_tiles; }
+  DG_DEVINL static Tile tile(const Params& p, int v) {
+    const int4 tt = p.tiles[v];
+    Tile t;
+    t.a = tt.x;  // expert
+    t.b = tt.y;  // 128-feature block
+    const int nt = tt.z;
+    const int n_valid = min(64, p.counts[t.a] - nt * 64);
+    t.valid = n_valid > 0;
+    t.c = n_valid;
+    t.d = p.offsets[t.a] + nt * 64;
+    t.nk = p.nk;
+    t.n_mma = round_up16(n_valid);
+    return t;
+  }
+  DG_DEVINL static uint32_t tx_bytes(const Params&, const Tile&) { return kAStage + B_STAGE; }
+  DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
+    tma_load_2d(sa, &p.tmW, kb * 64, t.a * p.d + t.b * 128, bar);
+    tma_load_2d(sb, &p.tmH, kb * 64, t.d, bar);
+  }
+  DG_DEVINL static void epilogue(const Params& p, const Tile& t, uint32_t taddr, int, int, int row, uint8_t*) {
+    const int f = t.b * 128 + row;
+    for (int c0 = 0; c0 < t.n_mma; c0 += 16) {
+      float v[16];
+      tmem_ld16(taddr + c0, v);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int c = c0 + i;
+        if (c < t.c) {
+          const int r = t.d + c;
+          p.yp[(size_t)r * p.d + f] = p.row_weight[r] * v[i];
+        }
+      }
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------
+// Shared expert gate|up + SwiGLU.  Tile (mt, j): tokens mt*128..+127, hidden
+// units j*64..+63; B rows 0..63 = gate rows, 64..127 = up rows.
+// ---------------------------------------------------------------------------
+struct P_SGU : ProblemBase {
+  static constexpr int BN = 128, STAGES = 6, B_STAGE = BN * 128, TMEM_COLS = 256;
+  struct Params {
+    CUtensorMap tmX;  // normed tokens [Tcap, d]
+    CUtensorMap tmG;  // ws_gate [fs, d]
+    CUtensorMap tmU;  // ws_up [fs, d]
+    int T, nk, MT, FJ, fs;
+    __nv_bfloat16* hs;  // [Tcap, fs]
+    int* err;
+  };
+  DG_DEVINL static void prefetch(const Params& p) {
+    tma_prefetch_desc(&p.tmX);
+    tma_prefetch_desc(&p.tmG);
+    tma_prefetch_desc(&p.tmU);
+  }
+  DG_DEVINL static int num_tiles(const Params& p) { return p.MT * p.FJ; }
+  DG_DEVINL static Tile tile(const Params& p, int v) {
+    Tile t;
+    t.valid = 1;
+    t.nk = p.nk;
+    t.n_mma = BN;
+    t.a = v % p.MT;
+    t.b = v / p.MT;
+    return t;
+  }
+  DG_DEVINL static uint32_t tx_bytes(const Params&, const Tile&) { return kAStage + B_STAGE; }
+  DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
+    tma_load_2d(sa, &p.tmX, kb * 64, t.a * 128, bar);
+    tma_load_2d(sb, &p.tmG, kb * 64, t.b * 64, bar);
+    tma_load_2d(sb + 64 * 128, &p.tmU, kb * 64, t.b * 64, bar);
+  }
+  DG_DEVINL static void epilogue(const Params& p, const Tile& t, uint32_t taddr, int, int, int row, uint8_t*) {
+    const int tok = t.a * 128 + row;
+    const bool ok = tok < p.T;
+    for (int c0 = 0; c0 < 64; c0 += 16) {
+      float g[16], u[16];
+      tmem_ld16(taddr + c0, g);
+      tmem_ld16(taddr + 64 + c0, u);
+      if (ok) {
+        float h[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) h[i] = silu_f(g[i]) * u[i];
+        store_bf16x16(p.hs + (size_t)tok * p.fs + t.b * 64 + c0, h);
+      }
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------
+// Shared expert down + routed combine + residual:
+//   x[t, f] += (Hs W_sd^T)[t, f] + sum_j Yp[row(t, j), f]
+// ---------------------------------------------------------------------------
+struct P_SD : ProblemBase {
+  static constexpr int BN = 128, STAGES = 6, B_STAGE = BN * 128, TMEM_COLS = 256;
+  struct Params {
+    CUtensorMap tmW;  // ws_down [d, fs]
+    CUtensorMap tmH;  // Hs [Tcap, fs]
+    int T, nk, MT, NT, d, k;
+    float* x;
+    const float* yp;
+    const int* pair_row;
+    int* err;
+  };
+  DG_DEVINL static void prefetch(const Params& p) {
+    tma_prefetch_desc(&p.tmW);
+    tma_prefetch_desc(&p.tmH);
+  }
+  DG_DEVINL static int num_tiles(const Params& p) { return p.MT * p.NT; }
+  DG_DEVINL static Tile tile(const Params& p, int v) {
+    Tile t;
+    t.valid = 1;
+    t.nk = p.nk;
+    t.b = v % p.NT;
+    t.a = v / p.NT;
+    t.n_mma = round_up16(min(128, p.T - t.b * 128));
+    return t;
+  }
+  DG_DEVINL static uint32_t tx_bytes(const Params&, const Tile&) { return kAStage + B_STAGE; }
+  DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
+    tma_load_2d(sa, &p.tmW, kb * 64, t.a * 128, bar);
+    tma_load_2d(sb, &p.tmH, kb * 64, t.b * 128, bar);
+  }
+  DG_DEVINL static void epilogue(const Params& p, const Tile& t, uint32_t taddr, int, int, int row, uint8_t*) {
+    const int f = t.a * 128 + row;
+    for (int c0 = 0; c0 < t.n_mma; c0 += 16) {
+      float v[16];
+      tmem_ld16(taddr + c0, v);
+#pragma unroll 4
+      for (int i = 0; i < 16; ++i) {
+        const int tok = t.b * 128 + c0 + i;
+        if (tok < p.T) {
+          float s = v[i];
+          for (int j = 0; j < p.k; ++j) s += p.yp[(size_t)p.pair_row[tok * p.k + j] * p.d + f];
+          p.x[(size_t)tok * p.d + f] += s;
+        }
+      }
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------
+// LM head with fused online statistics.  Tile (mt, vt): tokens mt*128..+127,
+// vocab rows vt*256..+255.  Each epilogue thread owns one token row and keeps,
+// per token tile, the running (max m, argmax a, s = sum e^(z-m),
+// t = sum e^(z-m)(z-m)) in shared memory across the CTA's tiles; the CTA's
+// partial is written at the end and merged across CTAs by k_lm_combine.
+// ---------------------------------------------------------------------------
+struct LmStat {
+  float m, s, t;
+  int a;
+};
+
+struct P_LM : ProblemBase {
+  static constexpr int BN = 256, STAGES = 4, B_STAGE = BN * 128, TMEM_COLS = 512;
+  static constexpr int MT_MAX = 8;
+  static constexpr int EP_SMEM = MT_MAX * 128 * (int)sizeof(LmStat);
+  struct Params {
+    CUtensorMap tmX;  // final-normed tokens [Tcap, d]
+    CUtensorMap tmE;  // embedding [V, d]
+    int T, nk, MT, NV;
+    long long V;
+    float4* part;    // [gridDim.x][MT*128]
+    float* logits;   // optional [T, V]
+    int* err;
+  };
+  DG_DEVINL static void prefetch(const Params& p) {
+    tma_prefetch_desc(&p.tmX);
+    tma_prefetch_desc(&p.tmE);
+  }
+  DG_DEVINL static int num_tiles(const Params& p) { return p.MT * p.NV; }
+  DG_DEVINL static Tile tile(const Params& p, int v) {
+    Tile t;
+    t.valid = 1;
+    t.nk = p.nk;
+    t.n_mma = BN;
+    t.a = v % p.MT;
+    t.b = v / p.MT;
+    return t;
+  }
+  DG_DEVINL static uint32_t tx_bytes(const Params&, const Tile&) { return kAStage + B_STAGE; }
+  DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
+    tma_load_2d(sa, &p.tmX, kb * 64, t.a * 128, bar);
+    tma_load_2d(sb, &p.tmE, kb * 64, t.b * 256, bar);
+  }
+  DG_DEVINL static void epilogue_init(const Params& p, int row, uint8_t* ep) {
+    LmStat* st = reinterpret_cast<LmStat*>(ep);
+    for (int mt = 0; mt < p.MT; ++mt) st[mt * 128 + row] = LmStat{-INFINITY, 0.f, 0.f, 0x7fffffff};
+  }
+  DG_DEVINL static void epilogue(const Params& p, const Tile& t, uint32_t taddr, int, int, int row, uint8_t* ep) {
+    LmStat* st = reinterpret_cast<LmStat*>(ep);
+    LmStat r = st[t.a * 128 + row];
+    const int tok = t.a * 128 + row;
+    const bool ok = tok < p.T;
+    constexpr float kLog2e = 1.4426950408889634f;
+    for (int c0 = 0; c0 < 256; c0 += 32) {
+      float z[32];
+      tmem_ld16(taddr + c0, z);
+      tmem_ld16(taddr + c0 + 16, z + 16);
+      if (p.logits != nullptr && ok) {
+        float* dst = p.logits + (size_t)tok * p.V + (size_t)t.b * 256 + c0;
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(z[i], z[i + 1], z[i + 2], z[i + 3]);
+      }
+      float cm = z[0];
+      int ca = 0;
+#pragma unroll
+      for (int i = 1; i < 32; ++i)
+        if (z[i] > cm) {
+          cm = z[i];
+          ca = i;
+        }
+      if (cm > r.m) {
+        if (r.s > 0.f) {
+          const float f = exp2f((r.m - cm) * kLog2e);
+          r.t = f * (r.t + (r.m - cm) * r.s);
+          r.s *= f;
+        }
+        r.m = cm;
+        r.a = t.b * 256 + c0 + ca;
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float dz = z[i] - r.m;
+        const float e = exp2f(dz * kLog2e);
+        r.s += e;
+        r.t = fmaf(e, dz, r.t);
+      }
+    }
+    st[t.a * 128 + row] = r;
+  }
+  DG_DEVINL static void finish(const Params& p, int row, uint8_t* ep) {
+    const LmStat* st = reinterpret_cast<const LmStat*>(ep);
+    for (int mt = 0; mt < p.MT; ++mt) {
+      const LmStat r = st[mt * 128 + row];
+      p.part[((size_t)blockIdx.x * p.MT + mt) * 128 + row] = make_float4(r.m, r.s, r.t, __int_as_float(r.a));
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------
+// host launchers
+// ---------------------------------------------------------------------------
+template <class P>
+static cudaError_t launch_gemm(const typename P::Params& p, int grid, cudaStream_t st) {
+  static bool configured = false;
+  const size_t smem = GemmSmem<P>::total;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(k_umma_gemm<P>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  if (grid <= 0) return cudaSuccess;
+  k_umma_gemm<P><<<grid, 192, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+static int grid_for(int tiles, int sms) { return tiles < sms ? tiles : sms; }
+
+cudaError_t run_qkv(const QkvArgs& a, cudaStream_t st) {
+  P_QKV::Params p;
+  p.tmA = *a.tm_x;
+  p.tmB = *a.tm_w;
+  p.T = a.T;
+  p.nk = a.d / 64;
+  p.MT = (a.T + 127) / 128;
+  p.NT = a.rows / 256;
+  p.D = a.D;
+  p.Hq = a.Hq;
+  p.Hkv = a.Hkv;
+  p.q_T = a.q_T;
+  p.kv_cap = a.kv_cap;
+  p.kv_req_stride = a.kv_req_stride;
+  p.tok_pos = a.tok_pos;
+  p.tok_req = a.tok_req;
+  p.inv_freq = a.inv_freq;
+  p.q = a.q;
+  p.kv = a.kv;
+  p.err = a.err;
+  return launch_gemm<P_QKV>(p, grid_for(p.MT * p.NT, a.num_sms), st);
+}
+
+cudaError_t run_oproj(const OprojArgs& a, cudaStream_t st) {
+  P_OPROJ::Params p;
+  p.tmA = *a.tm_w;
+  p.tmB = *a.tm_o;
+  p.T = a.T;
+  p.nk = a.K / 64;
+  p.MT = a.d / 128;
+  p.NT = (a.T + 127) / 128;
+  p.d = a.d;
+  p.x = a.x;
+  p.err = a.err;
+  return launch_gemm<P_OPROJ>(p, grid_for(p.MT * p.NT, a.num_sms), st);
+}
+
+cudaError_t run_experts(const ExpertArgs& a, cudaStream_t st) {
+  P_EGU::Params g;
+  g.tmG = *a.tm_gate;
+  g.tmU = *a.tm_up;
+  g.tmX = *a.tm_xp;
+  g.nk = a.d / 64;
+  g.fe = a.fe;
+  g.tiles = a.egu_tiles;
+  g.n_tiles = a.egu_count;
+  g.counts = a.counts;
+  g.offsets = a.offsets;
+  g.hp = a.hp;
+  g.err = a.err;
+  cudaError_t e = launch_gemm<P_EGU>(g, a.num_sms, st);
+  if (e != cudaSuccess) return e;
+  P_ED::Params dn;
+  dn.tmW = *a.tm_down;
+  dn.tmH = *a.tm_hp;
+  dn.nk = a.fe / 64;
+  dn.d = a.d;
+  dn.tiles = a.ed_tiles;
+  dn.n_tiles = a.ed_count;
+  dn.counts = a.counts;
+  dn.offsets = a.offsets;
+  dn.row_weight = a.row_weight;
+  dn.yp = a.yp;
+  dn.err = a.err;
+  return launch_gemm<P_ED>(dn, a.num_sms, st);
+}
+
+cudaError_t run_shared(const SharedArgs& a, cudaStream_t st) {
+  P_SGU::Params g;
+  g.tmX = *a.tm_u;
+  g.tmG = *a.tm_gate;
+  g.tmU = *a.tm_up;
+  g.T = a.T;
+  g.nk = a.d / 64;
+  g.MT = (a.T + 127) / 128;
+  g.FJ = a.fs / 64;
+  g.fs = a.fs;
+  g.hs = a.hs;
+  g.err = a.err;
+  cudaError_t e = launch_gemm<P_SGU>(g, grid_for(g.MT * g.FJ, a.num_sms), st);
+  if (e != cudaSuccess) return e;
+  P_SD::Params dn;
+  dn.tmW = *a.tm_down;
+  dn.tmH = *a.tm_hs;
+  dn.T = a.T;
+  dn.nk = a.fs / 64;
+  dn.MT = a.d / 128;
+  dn.NT = (a.T + 127) / 128;
+  dn.d = a.d;
+  dn.k = a.k;
+  dn.x = a.x;
+  dn.yp = a.yp;
+  dn.pair_row = a.pair_row;
+  dn.err = a.err;
+  return launch_gemm<P_SD>(dn, grid_for(dn.MT * dn.NT, a.num_sms), st);
+}
+
+cudaError_t run_lm_head(const LmArgs& a, int* grid_out, cudaStream_t st) {
+  P_LM::Params p;
+  p.tmX = *a.tm_x;
+  p.tmE = *a.tm_embed;
+  p.T = a.T;
+  p.nk = a.d / 64;
+  p.MT = (a.T + 127) / 128;
+  p.NV = (int)(a.V / 256);
+  p.V = a.V;
+  p.part = a.part;
+  p.logits = a.logits;
+  p.err = a.err;
+  if (p.MT > P_LM::MT_MAX) return cudaErrorInvalidValue;
+  const int grid = grid_for(p.MT * p.NV, a.num_sms);
+  *grid_out = grid;
+  return launch_gemm<P_LM>(p, grid, st);
+}
+
+size_t gemm_smem_bytes_max() {
+  size_t m = GemmSmem<P_QKV>::total;
+  m = m > GemmSmem<P_OPROJ>::total ? m : GemmSmem<P_OPROJ>::total;
+  m = m > GemmSmem<P_EGU>::total ? m : GemmSmem<P_EGU>::total;
+  m = m > GemmSmem<P_ED>::total ? m : GemmSmem<P_ED>::total;
+  m = m > GemmSmem<P_SGU>::total ? m : GemmSmem<P_SGU>::total;
+  m = m > GemmSmem<P_SD>::total ? m : GemmSmem<P_SD>::total;
+  m = m > GemmSmem<P_LM>::total ? m : GemmSmem<P_LM>::total;
+  return m;
+}
+
+}  // namespace dg

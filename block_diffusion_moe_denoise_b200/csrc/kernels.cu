@@ -1,0 +1,534 @@
+// CUDA-core kernels of the denoising pass: everything that is not a dense
+// contraction.  Warp-shuffle reductions, 16-byte vector loads/stores.
+#include <float.h>
+
+#include "common.cuh"
+#include "dg_internal.h"
+
+namespace dg {
+
+// ---------------------------------------------------------------------------
+// Embedding gather: x[t, :] = E[id_t, :] (fp32 residual stream), and each
+// token's absolute position and request.
+// ---------------------------------------------------------------------------
+struct EmbedParams {
+  SlotInfo s;
+  const int* ids[DG_MAX_REQUESTS];
+};
+
+__global__ void k_embed(EmbedParams p, const bf16* __restrict__ embed, int V, int d, float* __restrict__ x,
+                        int* tok_pos, int* tok_req, int* err) {
+  const int t = blockIdx.x;
+  const int slot = t / p.s.Tr;
+  const int i = t - slot * p.s.Tr;
+  int id = p.ids[slot][i];
+  if (id < 0 || id >= V) {
+    if (threadIdx.x == 0) atomicOr(err, DG_DEVERR_TOKEN);
+    id = 0;
+  }
+  if (threadIdx.x == 0) {
+    tok_pos[t] = p.s.pos0[slot] + i;
+    tok_req[t] = p.s.req[slot];
+  }
+  const uint4* src = reinterpret_cast<const uint4*>(embed + (size_t)id * d);
+  float4* dst = reinterpret_cast<float4*>(x + (size_t)t * d);
+  for (int c = threadIdx.x; c < d / 8; c += blockDim.x) {
+    const uint4 v = src[c];
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+    const float2 a = __bfloat1622float2(h[0]), b = __bfloat1622float2(h[1]);
+    const float2 e = __bfloat1622float2(h[2]), f = __bfloat1622float2(h[3]);
+    dst[2 * c] = make_float4(a.x, a.y, b.x, b.y);
+    dst[2 * c + 1] = make_float4(e.x, e.y, f.x, f.y);
+  }
+}
+
+cudaError_t run_embed(const int* const* ids, const SlotInfo& s, const bf16* embed, int V, int d, float* x,
+                      int* tok_pos, int* tok_req, int* err, cudaStream_t st) {
+  EmbedParams p;
+  p.s = s;
+  for (int i = 0; i < DG_MAX_REQUESTS; ++i) p.ids[i] = i < s.n ? ids[i] : nullptr;
+  const int T = s.n * s.Tr;
+  if (T == 0) return cudaSuccess;
+  k_embed<<<T, 128, 0, st>>>(p, embed, V, d, x, tok_pos, tok_req, err);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// RMSNorm: out = bf16(x / sqrt(mean(x^2) + eps) * g), one warp per row.
+// ---------------------------------------------------------------------------
+__global__ void k_rmsnorm(const float* __restrict__ x, const float* __restrict__ g, int T, int d, float eps,
+                          bf16* __restrict__ out) {
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= T) return;
+  const float4* xr = reinterpret_cast<const float4*>(x + (size_t)row * d);
+  float ss = 0.f;
+  for (int c = lane; c < d / 4; c += 32) {
+    const float4 v = xr[c];
+    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  }
+  ss = warp_sum(ss);
+  const float rs = rsqrtf(ss / (float)d + eps);
+  const float4* g4 = reinterpret_cast<const float4*>(g);
+  uint2* o = reinterpret_cast<uint2*>(out + (size_t)row * d);
+  for (int c = lane; c < d / 4; c += 32) {
+    const float4 v = xr[c];
+    const float4 w = g4[c];
+    o[c] = make_uint2(pack_bf16x2(v.x * rs * w.x, v.y * rs * w.y), pack_bf16x2(v.z * rs * w.z, v.w * rs * w.w));
+  }
+}
+
+cudaError_t run_rmsnorm(const float* x, const float* g, int T, int d, float eps, bf16* out, cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+  k_rmsnorm<<<(T + 7) / 8, 256, 0, st>>>(x, g, T, d, eps, out);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Router top-k: one warp per token over E <= 256 fp32 logits.  Picks the k
+// largest in descending order (ties to the lower expert id) and the softmax of
+// the picked logits.
+// ---------------------------------------------------------------------------
+DG_DEVINL void topk_warp(const float* vals, int E, int k, int* idx_out, float* w_out) {
+  const int lane = threadIdx.x & 31;
+  float v[8];
+  unsigned taken = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int e = lane + 32 * j;
+    v[j] = e < E ? vals[e] : -INFINITY;
+    if (e >= E) taken |= 1u << j;
+  }
+  float sel_v[8];
+  int sel_i[8];
+  for (int r = 0; r < k; ++r) {
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = lane + 32 * j;
+      if (!(taken & (1u << j)) && (v[j] > bv || (v[j] == bv && e < bi))) {
+        bv = v[j];
+        bi = e;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ov > bv || (ov == bv && oi < bi)) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    if (bi != 0x7fffffff && (bi & 31) == lane) taken |= 1u << (bi >> 5);
+    sel_v[r] = bv;
+    sel_i[r] = bi;
+  }
+  if (lane == 0) {
+    float sum = 0.f, e[8];
+    for (int r = 0; r < k; ++r) {
+      e[r] = expf(sel_v[r] - sel_v[0]);
+      sum += e[r];
+    }
+    for (int r = 0; r < k; ++r) {
+      idx_out[r] = sel_i[r];
+      w_out[r] = e[r] / sum;
+    }
+  }
+}
+
+__global__ void k_topk(const float* __restrict__ logits, int T, int E, int k, int* idx, float* w) {
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  topk_warp(logits + (size_t)t * E, E, k, idx + (size_t)t * k, w + (size_t)t * k);
+}
+
+cudaError_t run_topk(const float* logits, int T, int E, int k, int* idx, float* w, cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+  k_topk<<<(T + 7) / 8, 256, 0, st>>>(logits, T, E, k, idx, w);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// FFN RMSNorm + router logits (fp32 accumulate of bf16 inputs) + top-k.
+// kRouterTok tokens per CTA so the router weight is read once per CTA.
+// ---------------------------------------------------------------------------
+constexpr int kRouterTok = 4;
+
+__global__ void __launch_bounds__(256) k_router(const float* __restrict__ x, const float* __restrict__ g, float eps,
+                                                const bf16* __restrict__ wr, int T, int d, int E, int k,
+                                                bf16* __restrict__ u, int* idx, float* w) {
+  extern __shared__ float rsm[];
+  float* su = rsm;                       // [kRouterTok][d]
+  float* sl = rsm + kRouterTok * d;      // [kRouterTok][E]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t0 = blockIdx.x * kRouterTok;
+  if (warp < kRouterTok) {
+    const int t = t0 + warp;
+    float* dst = su + warp * d;
+    if (t < T) {
+      const float4* xr = reinterpret_cast<const float4*>(x + (size_t)t * d);
+      float ss = 0.f;
+      for (int c = lane; c < d / 4; c += 32) {
+        const float4 v = xr[c];
+        ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+      }
+      ss = warp_sum(ss);
+      const float rs = rsqrtf(ss / (float)d + eps);
+      const float4* g4 = reinterpret_cast<const float4*>(g);
+      uint2* uo = reinterpret_cast<uint2*>(u + (size_t)t * d);
+      for (int c = lane; c < d / 4; c += 32) {
+        const float4 v = xr[c];
+        const float4 gg = g4[c];
+        const uint32_t lo = pack_bf16x2(v.x * rs * gg.x, v.y * rs * gg.y);
+        const uint32_t hi = pack_bf16x2(v.z * rs * gg.z, v.w * rs * gg.w);
+        uo[c] = make_uint2(lo, hi);
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&lo));
+        const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hi));
+        reinterpret_cast<float4*>(dst)[c] = make_float4(a.x, a.y, b.x, b.y);
+      }
+    } else {
+      for (int c = lane; c < d; c += 32) dst[c] = 0.f;
+    }
+  }
+  __syncthreads();
+  for (int e = warp; e < E; e += 8) {
+    float acc[kRouterTok];
+#pragma unroll
+    for (int tt = 0; tt < kRouterTok; ++tt) acc[tt] = 0.f;
+    const bf16* wrow = wr + (size_t)e * d;
+    for (int c = lane * 8; c < d; c += 256) {
+      const uint4 wv = *reinterpret_cast<const uint4*>(wrow + c);
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&wv);
+      float wf[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f2 = __bfloat1622float2(h[i]);
+        wf[2 * i] = f2.x;
+        wf[2 * i + 1] = f2.y;
+      }
+#pragma unroll
+      for (int tt = 0; tt < kRouterTok; ++tt) {
+        const float* s = su + tt * d + c;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[tt] = fmaf(s[i], wf[i], acc[tt]);
+      }
+    }
+#pragma unroll
+    for (int tt = 0; tt < kRouterTok; ++tt) {
+      const float r = warp_sum(acc[tt]);
+      if (lane == 0) sl[tt * E + e] = r;
+    }
+  }
+  __syncthreads();
+  if (warp < kRouterTok && t0 + warp < T) {
+    const int t = t0 + warp;
+    topk_warp(sl + warp * E, E, k, idx + (size_t)t * k, w + (size_t)t * k);
+  }
+}
+
+cudaError_t run_router(const float* x, const float* g, float eps, const bf16* wr, int T, int d, int E, int k, bf16* u,
+                       int* idx, float* w, int*, cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+  const size_t smem = (size_t)kRouterTok * (d + E) * sizeof(float);
+  static size_t configured = 0;
+  if (smem > configured) {
+    cudaError_t e = cudaFuncSetAttribute(k_router, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    configured = smem;
+  }
+  k_router<<<(T + kRouterTok - 1) / kRouterTok, 256, smem, st>>>(x, g, eps, wr, T, d, E, k, u, idx, w);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Expert grouping (single CTA): per-expert counts, exclusive offsets, the row
+// of every (token, slot) pair in expert-grouped order (tokens ascending inside
+// an expert, via per-expert token bitmasks), and the GEMM tile lists.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024) k_group(GroupArgs a) {
+  extern __shared__ int gsm[];
+  const int E = a.E, T = a.T, k = a.k;
+  const int MW = (T + 31) >> 5;
+  int* cnt = gsm;                 // [E]
+  int* off = cnt + E;             // [E+1]
+  int* toff = off + E + 1;        // [E+1]
+  unsigned* mask = reinterpret_cast<unsigned*>(toff + E + 1);  // [E][MW]
+  const int tid = threadIdx.x;
+  for (int i = tid; i < E; i += blockDim.x) cnt[i] = 0;
+  for (int i = tid; i < E * MW; i += blockDim.x) mask[i] = 0u;
+  __syncthreads();
+  const int P = T * k;
+  for (int p = tid; p < P; p += blockDim.x) {
+    const int e = a.idx[p];
+    const int t = p / k;
+    if (e < 0 || e >= E) {
+      atomicOr(a.err, DG_DEVERR_TOKEN);
+      continue;
+    }
+    atomicAdd(&cnt[e], 1);
+    atomicOr(&mask[e * MW + (t >> 5)], 1u << (t & 31));
+  }
+  __syncthreads();
+  if (tid == 0) {
+    off[0] = 0;
+    toff[0] = 0;
+    for (int e = 0; e < E; ++e) {
+      off[e + 1] = off[e] + cnt[e];
+      toff[e + 1] = toff[e] + (cnt[e] + 63) / 64;
+    }
+    const int egu = toff[E] * a.FJ, ed = toff[E] * a.MD;
+    if (egu > a.egu_cap || ed > a.ed_cap) atomicOr(a.err, DG_DEVERR_CAPACITY);
+    *a.egu_count = min(egu, a.egu_cap);
+    *a.ed_count = min(ed, a.ed_cap);
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += blockDim.x) {
+    a.counts[e] = cnt[e];
+    a.offsets[e] = off[e];
+  }
+  if (tid == 0) a.offsets[E] = off[E];
+  for (int p = tid; p < P; p += blockDim.x) {
+    const int e = a.idx[p];
+    if (e < 0 || e >= E) continue;
+    const int t = p / k;
+    const unsigned* m = mask + e * MW;
+    int rank = __popc(m[t >> 5] & ((1u << (t & 31)) - 1u));
+    for (int wi = 0; wi < (t >> 5); ++wi) rank += __popc(m[wi]);
+    const int row = off[e] + rank;
+    a.pair_row[p] = row;
+    a.row_token[row] = t;
+    a.row_weight[row] = a.w[p];
+    a.row_pair[row] = p;
+  }
+  for (int e = tid; e < E; e += blockDim.x) {
+    const int n_nt = toff[e + 1] - toff[e];
+    for (int nt = 0; nt < n_nt; ++nt) {
+      const int base_g = (toff[e] + nt) * a.FJ;
+      for (int j = 0; j < a.FJ; ++j)
+        if (base_g + j < a.egu_cap) a.egu_tiles[base_g + j] = make_int4(e, j, nt, 0);
+      const int base_d = (toff[e] + nt) * a.MD;
+      for (int m = 0; m < a.MD; ++m)
+        if (base_d + m < a.ed_cap) a.ed_tiles[base_d + m] = make_int4(e, m, nt, 0);
+    }
+  }
+}
+
+cudaError_t run_group(const GroupArgs& a, cudaStream_t st) {
+  const int MW = (a.T + 31) >> 5;
+  const size_t smem = (size_t)(3 * a.E + 2 + a.E * MW) * sizeof(int);
+  static size_t configured = 0;
+  if (smem > configured) {
+    cudaError_t e = cudaFuncSetAttribute(k_group, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    configured = smem;
+  }
+  k_group<<<1, 1024, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Gather token rows into expert-grouped order: xp[row] = u[row_token[row]].
+// ---------------------------------------------------------------------------
+__global__ void k_gather(const bf16* __restrict__ u, const int* __restrict__ row_token, int rows, int d,
+                         bf16* __restrict__ xp) {
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const uint4* src = reinterpret_cast<const uint4*>(u + (size_t)row_token[row] * d);
+  uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)row * d);
+  for (int c = lane; c < d / 8; c += 32) dst[c] = src[c];
+}
+
+cudaError_t run_gather(const bf16* u, const int* row_token, int rows, int d, bf16* xp, cudaStream_t st) {
+  if (rows == 0) return cudaSuccess;
+  k_gather<<<(rows + 7) / 8, 256, 0, st>>>(u, row_token, rows, d, xp);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Merge of the LM head's per-CTA partials, in CTA order:
+//   m = max, s = sum e^(z-m), t = sum e^(z-m)(z-m), argmax lowest id on ties.
+//   logZ = m + ln s, H = ln s - t/s, logconf = -ln s.
+// ---------------------------------------------------------------------------
+__global__ void k_lm_combine(const float4* __restrict__ part, int G, int MT, int T, float* stats, int* argmax,
+                             int* err) {
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= T) return;
+  float m = -INFINITY, s = 0.f, tt = 0.f;
+  int a = 0x7fffffff;
+  const size_t stride = (size_t)MT * 128;
+  for (int c = 0; c < G; ++c) {
+    const float4 v = part[(size_t)c * stride + t];
+    const float mc = v.x, sc = v.y, tc = v.z;
+    const int ac = __float_as_int(v.w);
+    if (!(sc > 0.f)) {
+      if (sc != sc) atomicOr(err, DG_DEVERR_NAN);
+      continue;
+    }
+    if (s == 0.f) {
+      m = mc;
+      s = sc;
+      tt = tc;
+      a = ac;
+    } else if (mc > m) {
+      const float f = expf(m - mc);
+      tt = f * (tt + (m - mc) * s) + tc;
+      s = f * s + sc;
+      m = mc;
+      a = ac;
+    } else {
+      const float f = expf(mc - m);
+      tt += f * (tc + (mc - m) * sc);
+      s += f * sc;
+      if (mc == m && ac < a) a = ac;
+    }
+  }
+  const float ls = logf(s);
+  float4 o = make_float4(ls - tt / s, -ls, m, m + ls);
+  if (!(s > 0.f) || o.x != o.x) atomicOr(err, DG_DEVERR_NAN);
+  reinterpret_cast<float4*>(stats)[t] = o;
+  argmax[t] = a;
+}
+
+cudaError_t run_lm_combine(const float4* part, int G, int MT, int T, float* stats, int* argmax, int* err,
+                           cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+  k_lm_combine<<<(T + 127) / 128, 128, 0, st>>>(part, G, MT, T, stats, argmax, err);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Philox-4x32-10 (Salmon et al., SC'11): ten rounds of two 32x32->64-bit
+// multiplies with the high halves XORed into the odd words and the round key,
+// key bumped by the Weyl constants between rounds.
+// ---------------------------------------------------------------------------
+DG_DEVINL uint32_t philox_word0(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3, uint32_t k0, uint32_t k1) {
+  constexpr uint32_t M0 = 0xD2511F53u, M1 = 0xCD9E8D57u, W0 = 0x9E3779B9u, W1 = 0xBB67AE85u;
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    if (r > 0) {
+      k0 += W0;
+      k1 += W1;
+    }
+    const uint32_t lo0 = M0 * c0, hi0 = __umulhi(M0, c0);
+    const uint32_t lo1 = M1 * c2, hi1 = __umulhi(M1, c2);
+    const uint32_t n0 = hi1 ^ c1 ^ k0, n2 = hi0 ^ c3 ^ k1;
+    c0 = n0;
+    c1 = lo1;
+    c2 = n2;
+    c3 = lo0;
+  }
+  return c0;
+}
+
+DG_DEVINL int renoise_token(unsigned long long seed, int block, int step, uint32_t pos, int request, int vocab) {
+  const uint32_t x0 = philox_word0(pos, (uint32_t)step, (uint32_t)block, (uint32_t)request, (uint32_t)seed,
+                                   (uint32_t)(seed >> 32));
+  return (int)(((unsigned long long)x0 * (unsigned long long)vocab) >> 32);
+}
+
+__global__ void k_philox_tokens(unsigned long long seed, int block, int step, int request, long long pos0, long long n,
+                                int vocab, int* out, unsigned char* mask_clear) {
+  const long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  out[i] = renoise_token(seed, block, step, (uint32_t)(pos0 + i), request, vocab);
+  if (mask_clear) mask_clear[i] = 0;
+}
+
+cudaError_t run_philox_tokens(unsigned long long seed, int block, int step, int request, long long pos0, long long n,
+                              int vocab, int* out, unsigned char* mask_clear, cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  k_philox_tokens<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(seed, block, step, request, pos0, n, vocab, out,
+                                                               mask_clear);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Accept / freeze / re-noise rule, one CTA per canvas, one thread per position.
+// ---------------------------------------------------------------------------
+__global__ void k_sample(SampleArgs a) {
+  extern __shared__ float ssm[];
+  float* lc_s = ssm;                                             // [canvas]
+  int* un_s = reinterpret_cast<int*>(ssm + a.canvas);            // [canvas]
+  const int slot = blockIdx.x;
+  const int req = a.req[slot];
+  const int i = threadIdx.x;
+  const int C = a.canvas;
+  const bool valid = i < C;
+  const size_t p = (size_t)slot * C + i;
+  int acc = 1;
+  float H = 0.f, lc = -INFINITY;
+  int am = 0;
+  if (valid) {
+    acc = a.mask[(size_t)req * C + i] ? 1 : 0;
+    H = a.entropy[p * a.stride];
+    lc = a.logconf[p * a.stride];
+    am = a.argmax[p];
+    if (H != H || lc != lc) atomicOr(a.err, DG_DEVERR_NAN);
+    lc_s[i] = lc;
+    un_s[i] = !acc;
+  }
+  const int nU = __syncthreads_count(valid && !acc);
+  const int n_top = min(a.min_accept, nU);
+  const bool force = a.step[slot] >= a.max_steps;
+  int rank = 0;
+  if (valid && !acc) {
+    for (int j = 0; j < C; ++j) {
+      const float o = lc_s[j];
+      rank += (un_s[j] && (o > lc || (o == lc && j < i))) ? 1 : 0;
+    }
+  }
+  const bool take = valid && !acc && (force || H <= a.thr || rank < n_top);
+  if (take) {
+    if (am < 0 || am >= a.vocab) {
+      atomicOr(a.err, DG_DEVERR_TOKEN);
+      am = 0;
+    }
+    a.canvas_tok[(size_t)req * C + i] = am;
+    a.mask[(size_t)req * C + i] = 1;
+  } else if (valid && !acc) {
+    a.canvas_tok[(size_t)req * C + i] =
+        renoise_token(a.seed[slot], a.block[slot], a.step[slot], (uint32_t)i, req, a.vocab);
+  }
+  const int rem = __syncthreads_count(valid && !acc && !take);
+  if (i == 0) a.remaining[req] = rem;
+}
+
+cudaError_t run_sample(const SampleArgs& a, cudaStream_t st) {
+  if (a.n_slots == 0) return cudaSuccess;
+  const int threads = (a.canvas + 31) / 32 * 32;
+  k_sample<<<a.n_slots, threads, (size_t)a.canvas * 8, st>>>(a);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// KV copy between the cache layout [Hkv][cap][D] and a dense [Hkv][n][D].
+// ---------------------------------------------------------------------------
+__global__ void k_kv_copy(bf16* cache_k, bf16* cache_v, int Hkv, long long cap, int D, long long pos0, long long n,
+                          const bf16* k_in, const bf16* v_in, bf16* k_out, bf16* v_out) {
+  const long long r = blockIdx.x;  // (head, i)
+  const int head = (int)(r / n);
+  const long long i = r - (long long)head * n;
+  const size_t cache_off = ((size_t)head * cap + pos0 + i) * D;
+  const size_t dense_off = ((size_t)head * n + i) * D;
+  for (int c = threadIdx.x; c < D / 8; c += blockDim.x) {
+    if (k_in) {
+      reinterpret_cast<uint4*>(cache_k + cache_off)[c] = reinterpret_cast<const uint4*>(k_in + dense_off)[c];
+      reinterpret_cast<uint4*>(cache_v + cache_off)[c] = reinterpret_cast<const uint4*>(v_in + dense_off)[c];
+    } else {
+      reinterpret_cast<uint4*>(k_out + dense_off)[c] = reinterpret_cast<const uint4*>(cache_k + cache_off)[c];
+      reinterpret_cast<uint4*>(v_out + dense_off)[c] = reinterpret_cast<const uint4*>(cache_v + cache_off)[c];
+    }
+  }
+}
+
+cudaError_t run_kv_copy(bf16* cache_k, bf16* cache_v, int Hkv, long long cap, int D, long long pos0, long long n,
+                        const bf16* k_in, const bf16* v_in, bf16* k_out, bf16* v_out, cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  k_kv_copy<<<(unsigned)(Hkv * n), 32, 0, st>>>(cache_k, cache_v, Hkv, cap, D, pos0, n, k_in, v_in, k_out, v_out);
+  return cudaGetLastError();
+}
+
+}  // namespace dg

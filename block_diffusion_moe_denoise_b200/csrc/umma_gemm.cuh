@@ -1,0 +1,171 @@
+// Persistent, warp-specialised tcgen05 GEMM engine for sm_100a.
+//
+//   D[128 x N] = A[128 x K] * B[N x K]^T      (bf16 operands, fp32 accumulator in TMEM)
+//
+// Both operands are K-major tiles staged in shared memory by TMA with the
+// 128-byte swizzle, 64 bf16 (one 128-byte row) per k-block.  Roles:
+//   warp 0 (one lane)   TMA producer: fills a STAGES-deep ring of (A, B) tiles
+//   warp 1 (one lane)   MMA issuer: 4 x tcgen05.mma (K = 16 each) per k-block,
+//                       tcgen05.commit frees the ring slot / signals the accumulator
+//   warps 2..5          epilogue: tcgen05.ld of the accumulator rows they own
+//                       (warp w reads TMEM lanes 32*(w%4) .. +31) and the fused
+//                       problem-specific epilogue
+// The accumulator is double-buffered in TMEM (2 x BN columns) so the epilogue
+// of one tile overlaps the main loop of the next.  Tiles are assigned
+// statically (tile v to CTA v mod gridDim.x), so every role walks the same list.
+//
+// A problem class P supplies: BN, STAGES, B_STAGE (bytes), EP_SMEM (bytes),
+// TMEM_COLS, Params, num_tiles(), tile(), tx_bytes(), load(), epilogue(),
+// finish().  Every wait is bounded (see mbar_wait_bounded).
+#pragma once
+
+#include "common.cuh"
+
+namespace dg {
+
+struct Tile {
+  int valid;
+  int nk;     // k-blocks of 64
+  int n_mma;  // MMA N (multiple of 16, <= BN)
+  int a, b, c, d, e;  // problem-specific coordinates
+};
+
+constexpr int kAStage = 128 * 128;  // 128 rows x 128 bytes
+
+template <class P>
+struct GemmSmem {
+  static constexpr int kStages = P::STAGES;
+  static constexpr size_t a_off = 0;
+  static constexpr size_t b_off = a_off + (size_t)kStages * kAStage;
+  static constexpr size_t ep_off = b_off + (size_t)kStages * P::B_STAGE;
+  static constexpr size_t bar_off = (ep_off + P::EP_SMEM + 15) & ~(size_t)15;
+  static constexpr size_t misc_off = bar_off + (2 * kStages + 4) * 8;
+  static constexpr size_t total = misc_off + 16 + 1024;  // + alignment slack
+};
+
+template <class P>
+__global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ typename P::Params p) {
+  using S = GemmSmem<P>;
+  extern __shared__ uint8_t dyn_smem[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~(uintptr_t)1023);
+  uint8_t* sA = base + S::a_off;
+  uint8_t* sB = base + S::b_off;
+  uint8_t* ep_smem = base + S::ep_off;
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + S::bar_off);
+  uint64_t* empty = full + P::STAGES;
+  uint64_t* tfull = empty + P::STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + S::misc_off);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(base + S::misc_off + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < P::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 0 && lane == 0) P::prefetch(p);
+  if (warp == 1) tmem_alloc(tmem_slot, P::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int n_tiles = P::num_tiles(p);
+  int* err = p.err;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      for (int v = blockIdx.x; v < n_tiles; v += gridDim.x) {
+        const Tile t = P::tile(p, v);
+        if (!t.valid) continue;
+        const uint32_t tx = P::tx_bytes(p, t);
+        bool ok = true;
+        for (int kb = 0; kb < t.nk; ++kb) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, err)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[stage], tx);
+          P::load(p, t, kb, smem_u32(sA + (size_t)stage * kAStage), smem_u32(sB + (size_t)stage * P::B_STAGE),
+                  &full[stage]);
+          if (++stage == P::STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+      for (int v = blockIdx.x; v < n_tiles; v += gridDim.x) {
+        const Tile t = P::tile(p, v);
+        if (!t.valid) continue;
+        if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1, abort_flag, err)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + acc * P::BN;
+        const uint32_t idesc = umma_idesc_bf16(128, (uint32_t)t.n_mma);
+        bool ok = true;
+        for (int kb = 0; kb < t.nk; ++kb) {
+          if (!mbar_wait_bounded(&full[stage], phase, abort_flag, err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + (size_t)stage * kAStage);
+          const uint32_t b0 = smem_u32(sB + (size_t)stage * P::B_STAGE);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            umma_bf16(d_tmem, umma_sdesc_k128(a0 + 32 * k), umma_sdesc_k128(b0 + 32 * k), idesc,
+                      (kb | k) != 0 ? 1u : 0u);
+          umma_commit(&empty[stage]);
+          if (++stage == P::STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1;
+      }
+    }
+  } else {
+    const int q = warp & 3;            // TMEM lane quadrant of this warp
+    const int row = q * 32 + lane;     // accumulator row (M index) owned by this thread
+    P::epilogue_init(p, row, ep_smem);
+    uint32_t acc = 0, acc_phase = 0;
+    for (int v = blockIdx.x; v < n_tiles; v += gridDim.x) {
+      const Tile t = P::tile(p, v);
+      if (!t.valid) continue;
+      if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, err)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + acc * P::BN;
+      P::epilogue(p, t, taddr, q, lane, row, ep_smem);
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1;
+    }
+    P::finish(p, row, ep_smem);
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, P::TMEM_COLS);
+}
+
+// Default no-op hooks for problems that need none.
+struct ProblemBase {
+  static constexpr int EP_SMEM = 0;
+  template <class Params>
+  DG_DEVINL static void epilogue_init(const Params&, int, uint8_t*) {}
+  template <class Params>
+  DG_DEVINL static void finish(const Params&, int, uint8_t*) {}
+};
+
+DG_DEVINL int round_up16(int n) { return (n + 15) & ~15; }
+
+}  // namespace dg

@@ -1,0 +1,68 @@
+/*
+ * dg_ops.h -- operation-level entry points of libdg, used to check each step
+ * of the denoising pass on its own.  Same conventions as dg.h (caller-owned
+ * device pointers, asynchronous on the handle's stream unless stated, DG_OK or
+ * a negative DG_E_* code).
+ */
+#ifndef DG_OPS_H_
+#define DG_OPS_H_
+
+#include "dg.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Philox-4x32-10 re-noise draw (Salmon et al., SC'11, "Parallel Random Numbers:
+ * As Easy as 1, 2, 3"): d_out[i] = floor(x0 * vocab / 2^32) where x0 is the
+ * first output word for key (seed mod 2^32, seed >> 32) and counter
+ * (pos0 + i, step, block, request).  Standalone (no handle); stream may be NULL. */
+int dg_op_philox_tokens(uint64_t seed, int block, int step, int request, int64_t pos0, int64_t n, int vocab,
+                        int32_t* d_out, void* stream);
+
+/* Router selection from given fp32 logits [T, E] (device): top_k experts per
+ * token in descending logit order (ties to the lower expert id) and the
+ * softmax of the selected logits (the full softmax renormalised over the k
+ * picks).  d_idx [T, k] int32, d_w [T, k] f32.  Standalone; stream may be NULL. */
+int dg_op_route_topk(const float* d_logits, int T, int E, int k, int32_t* d_idx, float* d_w, void* stream);
+
+/* Grouping of (token, slot) pairs by expert, with the handle's workspace as
+ * scratch: from d_idx [T, k] computes counts [E], exclusive offsets [E+1] and
+ * d_perm [T*k] = t*k + j in expert order, tokens ascending inside an expert.
+ * T <= max_requests * canvas. */
+int dg_op_route_group(dg_handle* h, const int32_t* d_idx, const float* d_w, int T, int32_t* d_counts,
+                      int32_t* d_offsets, int32_t* d_perm);
+
+/* The accept / re-noise rule for request `req` from given per-position
+ * statistics (device, [canvas] each): entropy (nats), logconf (log max-prob)
+ * and argmax.  Uses the request's open canvas, mask, seed and block; `step` is
+ * the step number (1-based).  Updates canvas, mask, remaining. */
+int dg_op_sample(dg_handle* h, int req, const float* d_entropy, const float* d_logconf, const int32_t* d_argmax,
+                 int step);
+
+/* Final RMSNorm + tied LM head + fused statistics on given fp32 hidden rows
+ * d_x [T, d]: per row argmax, max logit, log-partition, entropy, logconf into
+ * d_stats [T][4] = (entropy, logconf, max, logZ) and d_argmax [T].  If d_logits
+ * is not NULL the fp32 logits [T, vocab] are written too. */
+int dg_op_lm_head(dg_handle* h, const float* d_x, int T, float* d_stats, int32_t* d_argmax, float* d_logits);
+
+/* Run the decoder over `T` tokens (device ids) of request `req` at positions
+ * [L, L+T) without advancing L, stopping after `n_layers` layers (the K/V of
+ * those layers are written to the cache slots).  The intermediates of the last
+ * layer run stay in the workspace; dg_debug_buffer locates them. */
+int dg_debug_forward(dg_handle* h, int req, const int32_t* d_tokens, int T, int n_layers);
+
+/* Byte offset and size, inside the workspace, of a named internal buffer:
+ * "x" f32 [T, d] residual stream; "hn" bf16 [T, d] normed input of the last
+ * projection; "q" bf16 [Hq, Tcap, D]; "o" bf16 [T, Hq*D]; "u" bf16 [T, d];
+ * "idx" i32 [T, k]; "w" f32 [T, k]; "counts" i32 [E]; "offsets" i32 [E+1];
+ * "pair_row" i32 [T*k]; "row_pair" i32 [T*k]; "hp" bf16 [T*k, fe];
+ * "yp" f32 [T*k, d]; "hs" bf16 [T, fs]; "stats" f32 [Tcap][4];
+ * "argmax" i32 [Tcap]; "canvas" i32 [max_req, canvas]; "mask" u8 [...];
+ * "remaining" i32 [max_req].  Returns DG_E_ARG for an unknown name. */
+int dg_debug_buffer(const dg_handle* h, const char* name, size_t* offset, size_t* bytes);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DG_OPS_H_ */

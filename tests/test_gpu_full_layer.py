@@ -1,0 +1,127 @@
+"""GPU vs oracle at the full synthetic shape: one decoder layer (d 2816, 16/8
+heads of 256, 128 experts top-8 + shared 2112, vocab 262144) over a 256-token
+canvas with a 4096-token synthetic KV prefix, in the same launch configuration
+as the benchmark (1 request, 256 canvas tokens)."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import layers as OL
+from oracle.model import Oracle, Trace
+from oracle import sampler as OS
+from synth import LAYER, make_kv_prefix, make_weights, to_f64
+
+from .gpu_common import LOGIT_MAX_ABS, REL_L2, np64, rel_l2, routing_match
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+CFG = LAYER
+L_PREFIX = 4096
+
+
+@pytest.fixture(scope="module")
+def setup():
+    import block_diffusion_moe_denoise_b200 as dgm
+    w = make_weights(CFG, seed=0, device="cuda")
+    k, v = make_kv_prefix(CFG, L_PREFIX, seed=1, device="cuda")
+    h = dgm.DG(CFG, w, max_requests=1, kv_capacity=L_PREFIX + CFG.canvas)
+    h.set_kv(0, 0, 0, k, v)
+    h.set_kv_len(0, L_PREFIX)
+    h.open_canvas(0, 2, 0)
+    tok, _, _, _ = h.get_canvas(0)
+    h.debug_forward(0, tok, 1)                 # the whole 1-layer pass incl. LM head
+    h.sync()
+    ow = {"embed": to_f64(w["embed"]), "final_norm": to_f64(w["final_norm"]),
+          "layers": [{n: to_f64(t) for n, t in w["layers"][0].items()}]}
+    ora = Oracle(CFG, ow)
+    cache = ora.new_cache(L_PREFIX + CFG.canvas)
+    cache.K[0][:, :L_PREFIX] = to_f64(k)
+    cache.V[0][:, :L_PREFIX] = to_f64(v)
+    cache.length = L_PREFIX
+    tr = Trace()
+    ora.forward(tok.cpu().numpy().astype(np.int64), cache, want_stats=False, trace=tr)
+    yield dict(h=h, w=w, ora=ora, tr=tr.layers[0], tok=tok, cache=cache)
+    h.close()
+
+
+def test_canvas_init_is_philox(setup):
+    ref, _ = OS.init_canvas(CFG.canvas, seed=2, block=0, vocab=CFG.vocab)
+    np.testing.assert_array_equal(setup["tok"].cpu().numpy(), ref)
+
+
+def test_attention_path(setup):
+    h, rec = setup["h"], setup["tr"]
+    T, d, Hq, D = CFG.canvas, CFG.d_model, CFG.n_q_heads, CFG.head_dim
+    Tcap = 256
+    q = np64(h.debug_buffer("q", torch.bfloat16, (Hq, Tcap, D))).transpose(1, 0, 2)
+    assert rel_l2(q, rec["q"]) < REL_L2
+    kk, vv = h.get_kv(0, 0, L_PREFIX, T)
+    assert rel_l2(np64(kk).transpose(1, 0, 2), rec["k"]) < REL_L2
+    assert rel_l2(np64(vv).transpose(1, 0, 2), rec["v"]) < REL_L2
+    o = np64(h.debug_buffer("o", torch.bfloat16, (Tcap, Hq * D)))
+    assert rel_l2(o, rec["o"].reshape(T, Hq * D)) < REL_L2
+    assert rel_l2(np64(h.debug_buffer("u", torch.bfloat16, (Tcap, d))), rec["u"]) < REL_L2
+
+
+def test_moe_path(setup):
+    h, rec, ora = setup["h"], setup["tr"], setup["ora"]
+    T, d, k = CFG.canvas, CFG.d_model, CFG.top_k
+    idx = h.debug_buffer("idx", torch.int32, (T, k)).cpu().numpy()
+    same = routing_match(idx, rec["idx"])
+    assert same.mean() >= 0.95, same.mean()
+    counts = h.debug_buffer("counts", torch.int32, (CFG.n_experts,)).cpu().numpy()
+    assert counts.sum() == T * k and (counts == np.bincount(idx.ravel(), minlength=CFG.n_experts)).all()
+    pair_row = h.debug_buffer("pair_row", torch.int32, (T * k,)).cpu().numpy()
+    yp = np64(h.debug_buffer("yp", torch.float32, (T * k, d)))
+    W = ora.layer(0)
+    rng = np.random.default_rng(0)
+    got, ref = [], []
+    for t in rng.choice(np.nonzero(same)[0], 24, replace=False):
+        for j in range(k):
+            e = idx[t, j]
+            jj = list(rec["idx"][t]).index(e)
+            hid = OL.silu(rec["u"][t] @ W["w_gate"][e].T) * (rec["u"][t] @ W["w_up"][e].T)
+            got.append(yp[pair_row[t * k + j]])
+            ref.append(rec["w"][t, jj] * (hid @ W["w_down"][e].T))
+    assert rel_l2(got, ref) < REL_L2
+    hs = np64(h.debug_buffer("hs", torch.bfloat16, (256, CFG.ffn_shared)))
+    assert rel_l2(hs, OL.silu(rec["u"] @ W["ws_gate"].T) * (rec["u"] @ W["ws_up"].T)) < REL_L2
+    x = np64(h.debug_buffer("x", torch.float32, (256, d)))
+    assert rel_l2(x[same], rec["x_out"][same]) < REL_L2
+
+
+def test_lm_head_sampled_rows(setup):
+    h, rec, ora = setup["h"], setup["tr"], setup["ora"]
+    stats = h.debug_buffer("stats", torch.float32, (256, 4)).cpu().numpy().astype(np.float64)
+    am = h.debug_buffer("argmax", torch.int32, (256,)).cpu().numpy()
+    rows = np.random.default_rng(1).choice(256, 24, replace=False)
+    xn = OL.rms_norm(rec["x_out"][rows], ora.final_norm, CFG.norm_eps)
+    ref = OL.lm_head_stats(xn, ora.embed)
+    assert np.max(np.abs(stats[rows, 2] - ref["max"])) < LOGIT_MAX_ABS
+    assert np.max(np.abs(stats[rows, 3] - ref["logZ"])) < LOGIT_MAX_ABS
+    assert rel_l2(stats[rows, 0], ref["entropy"]) < REL_L2
+    srt = np.sort(ref["logits"], axis=-1)
+    sure = srt[:, -1] - srt[:, -2] > 1e-2
+    np.testing.assert_array_equal(am[rows][sure], ref["argmax"][sure])
+
+
+def test_public_step_matches_debug_pass(setup):
+    """dg_denoise_step on the same canvas reproduces the pass bit for bit and
+    applies the rule to its statistics: the 22 most confident positions are
+    frozen to their argmax, every other position is re-drawn."""
+    h = setup["h"]
+    before = h.debug_buffer("stats", torch.float32, (256, 4)).clone()
+    h.denoise_step([0])
+    tok, mask, stats, am = h.get_canvas(0)
+    h.sync()
+    assert torch.equal(stats, before)
+    assert h.read_remaining(0) == 256 - 22
+    lc = stats[:, 1].cpu().numpy()
+    m = mask.cpu().numpy().astype(bool)
+    assert m.sum() == 22 and (stats[:, 0].cpu().numpy() > 1.0).all()
+    order = sorted(range(256), key=lambda i: (-lc[i], i))
+    assert set(np.nonzero(m)[0]) == set(order[:22])
+    np.testing.assert_array_equal(tok.cpu().numpy()[m], am.cpu().numpy()[m])
+    t = tok.cpu().numpy()
+    assert t.min() >= 0 and t.max() < CFG.vocab

@@ -1,0 +1,136 @@
+"""Bit-exact parity of the integer / selection kernels against the oracle, on
+identical fp32 inputs: Philox re-noise draws, router top-k, expert grouping,
+canvas initialisation and the accept / re-noise rule."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import layers as OL
+from oracle import philox as OP
+from oracle import sampler as OS
+from synth import TINY, make_weights
+
+from .gpu_common import to_device
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+
+@pytest.fixture(scope="module")
+def dgmod():
+    import block_diffusion_moe_denoise_b200 as dgm
+    return dgm
+
+
+@pytest.fixture(scope="module")
+def tiny_handle(dgmod):
+    w = to_device(make_weights(TINY, seed=0))
+    h = dgmod.DG(TINY, w, max_requests=4, kv_capacity=1024)
+    yield h
+    h.close()
+
+
+@pytest.mark.parametrize("seed,block,step,req_id,vocab", [
+    (0, 0, 0, 0, 2048), (1234, 3, 12, 0, 262144), (2**40 + 7, 1, 5, 3, 262144), (99, 2, 1, 1, 1000)])
+def test_philox_tokens_bitwise(dgmod, seed, block, step, req_id, vocab):
+    n = 1_000_000 if vocab == 262144 and seed == 1234 else 65536
+    out = torch.empty(n, dtype=torch.int32, device="cuda")
+    dgmod.philox_tokens(seed, block, step, req_id, 0, n, vocab, out)
+    torch.cuda.synchronize()
+    ref = OP.renoise_tokens(seed, block, step, np.arange(n), vocab, req_id)
+    np.testing.assert_array_equal(out.cpu().numpy(), ref)
+
+
+def test_route_topk_bitwise(dgmod):
+    rng = np.random.default_rng(0)
+    for T, E, k in ((256, 128, 8), (1024, 128, 8), (37, 16, 2), (5, 256, 8)):
+        logits = rng.normal(size=(T, E)).astype(np.float32)
+        logits[: T // 4, : E // 2] = np.round(logits[: T // 4, : E // 2], 1)   # many exact ties
+        logits[0, :] = 0.5                                                    # all tied
+        d = torch.from_numpy(logits).cuda()
+        idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+        w = torch.empty((T, k), dtype=torch.float32, device="cuda")
+        dgmod.route_topk(d, k, idx, w)
+        torch.cuda.synchronize()
+        ridx, rw = OL.route(logits.astype(np.float64), k)
+        np.testing.assert_array_equal(idx.cpu().numpy(), ridx)
+        np.testing.assert_allclose(w.cpu().numpy(), rw, rtol=2e-6, atol=1e-7)
+
+
+def test_route_group_bitwise(tiny_handle):
+    rng = np.random.default_rng(1)
+    E, k = TINY.n_experts, TINY.top_k
+    for T in (256, 1024, 1, 77):
+        logits = rng.normal(size=(T, E))
+        if T == 77:
+            logits[:, 3] += 10.0                     # one expert takes every token
+        idx, w = OL.route(logits, k)
+        counts, offsets, perm = tiny_handle.op_route_group(
+            torch.from_numpy(idx.astype(np.int32)).cuda(), torch.from_numpy(w.astype(np.float32)).cuda())
+        torch.cuda.synchronize()
+        rc, ro, rp, _ = OL.histogram_and_permutation(idx, E)
+        np.testing.assert_array_equal(counts.cpu().numpy(), rc)
+        np.testing.assert_array_equal(offsets.cpu().numpy(), ro)
+        np.testing.assert_array_equal(perm.cpu().numpy(), rp)
+        tiny_handle.sync()
+
+
+def test_open_canvas_bitwise(tiny_handle):
+    tiny_handle.set_kv_len(2, 0)
+    tiny_handle.open_canvas(2, 1234, 3)
+    tok, mask, _, _ = tiny_handle.get_canvas(2)
+    torch.cuda.synchronize()
+    ref, racc = OS.init_canvas(TINY.canvas, seed=1234, block=3, vocab=TINY.vocab, request=2)
+    np.testing.assert_array_equal(tok.cpu().numpy(), ref)
+    assert not mask.cpu().numpy().any() and not racc.any()
+
+
+def _rand_stats(rng, n, vocab, low_entropy=0):
+    H = rng.uniform(2.0, 8.0, size=n).astype(np.float32)
+    if low_entropy:
+        H[rng.choice(n, low_entropy, replace=False)] = rng.uniform(0.0, 1.0, size=low_entropy)
+        H[0] = np.float32(1.0)                                    # exactly at the threshold
+    lc = np.round(rng.normal(-5.0, 0.3, size=n), 2).astype(np.float32)   # ties in logconf
+    am = rng.integers(0, vocab, size=n).astype(np.int32)
+    return H, lc, am
+
+
+@pytest.mark.parametrize("low_entropy", [0, 30])
+def test_sampler_bitwise_full_canvas(tiny_handle, low_entropy):
+    """Twelve steps of the rule from identical fp32 statistics: canvas, mask and
+    remaining match the oracle exactly, and the canvas converges."""
+    C, V = TINY.canvas, TINY.vocab
+    req, seed = 1, 77
+    tiny_handle.set_kv_len(req, 0)
+    tiny_handle.open_canvas(req, seed, 0)
+    canvas, acc = OS.init_canvas(C, seed=seed, block=0, vocab=V, request=req)
+    rng = np.random.default_rng(2 + low_entropy)
+    for step in range(1, TINY.max_steps + 1):
+        H, lc, am = _rand_stats(rng, C, V, low_entropy if step == 1 else 0)
+        tiny_handle.op_sample(req, torch.from_numpy(H).cuda(), torch.from_numpy(lc).cuda(),
+                              torch.from_numpy(am).cuda(), step)
+        canvas, acc, rem = OS.sample_step(canvas, acc, am, H.astype(np.float64), lc.astype(np.float64), seed=seed,
+                                          block=0, step=step, vocab=V, entropy_thresh=TINY.entropy_thresh,
+                                          min_accept=TINY.min_accept, max_steps=TINY.max_steps, request=req)
+        tok, mask, _, _ = tiny_handle.get_canvas(req)
+        np.testing.assert_array_equal(tok.cpu().numpy(), canvas)
+        np.testing.assert_array_equal(mask.cpu().numpy().astype(bool), acc)
+        assert tiny_handle.read_remaining(req) == rem
+        if rem == 0:
+            break
+    assert rem == 0
+    tiny_handle.sync()
+
+
+def test_sampler_step_cap_forces_acceptance(tiny_handle):
+    C, V = TINY.canvas, TINY.vocab
+    req = 3
+    tiny_handle.set_kv_len(req, 0)
+    tiny_handle.open_canvas(req, 5, 1)
+    rng = np.random.default_rng(9)
+    H, lc, am = _rand_stats(rng, C, V)
+    tiny_handle.op_sample(req, torch.from_numpy(H).cuda(), torch.from_numpy(lc).cuda(), torch.from_numpy(am).cuda(),
+                          TINY.max_steps)
+    tok, mask, _, _ = tiny_handle.get_canvas(req)
+    assert mask.cpu().numpy().all() and tiny_handle.read_remaining(req) == 0
+    np.testing.assert_array_equal(tok.cpu().numpy(), am)
