@@ -1,0 +1,450 @@
+#!/usr/bin/env python
+"""Benchmark of the block-diffusion MoE denoising path on one B200 per process.
+
+Workload (default "generate"): the full synthetic 30-layer MoE stack (d 2816,
+16/8 heads of 256, 128 experts top-8 + shared 2112, vocab 262144; bf16 random
+weights, N(0, 0.02)), batch 1, a 4096-token uniform-random prompt prefilled
+into the KV cache, then 256-token canvases.  One benchmark step is one canvas:
+open (Philox init), denoising steps until every position is accepted (12 with
+the >=22-most-confident rule), commit.  Canvases cycle through blocks 0..3 at
+KV positions 4096, 4352, 4608, 4864 (4096 in / 1024 out), the KV length being
+reset to 4096 every fourth canvas.
+
+  value       output tokens/s of the whole job (inputs resident in HBM),
+              device-timed with CUDA events, max over ranks
+  e2e         the same metric through dg_generate with pinned host buffers
+              (prompt copied in, 1024 output ids copied out, prefill included)
+  roofline    the dominant kernel (routed-expert gate/up GEMM) against the
+              measured HBM copy bandwidth
+  cpu_baseline  the fp64 oracle on the host cores, on a bounded sample
+
+`--impl reference` times the oracle alone (the reference arm of this build).
+Multi-GPU: independent replicas, one per rank (no data-path collective).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+PROMPT = 4096
+N_OUT = 1024
+SEED = 1234
+METRIC = "output tok/s at batch 1 (4096 in / 1024 out), full synthetic 30-layer MoE stack; ms/denoise step"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=8)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="generate", choices=["generate", "layer"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# peaks and clocks
+# ---------------------------------------------------------------------------
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained"), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class ClockSampler:
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str):
+        self.uuid = uuid
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9 or (self.uuid and self.uuid not in f[0]):
+                continue
+            try:
+                rows.append((float(f[1]), float(f[2]), float(f[3]), f[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        loaded = [r for r in rows if r[2] > 250.0] or rows
+        sm = sorted(r[0] for r in loaded)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[3]) if v.lower() == "active"})
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(loaded), "power_w_max": max(r[2] for r in rows)}
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work
+# ---------------------------------------------------------------------------
+def expert_gate_up_bytes(cfg, n_touched: int, T: int) -> float:
+    """Bytes one routed-expert gate|up launch must move: the gate and up
+    weights of every expert some token is routed to, the grouped token rows
+    read, the SwiGLU hidden rows written."""
+    w = n_touched * 2 * cfg.ffn_expert * cfg.d_model * 2
+    rows = T * cfg.top_k
+    return w + rows * cfg.d_model * 2 + rows * cfg.ffn_expert * 2
+
+
+def step_work(cfg, kv_len: int, T: int, n_touched: int):
+    """(bytes, flops) of one denoising step: every weight of the touched
+    experts and all dense weights once, the KV prefix read, per-token FLOPs."""
+    d, D = cfg.d_model, cfg.head_dim
+    attn_w = cfg.qkv_rows * d + d * cfg.n_q_heads * D
+    per_layer_w = attn_w + n_touched * 3 * cfg.ffn_expert * d + 3 * cfg.ffn_shared * d + cfg.n_experts * d
+    weights = (cfg.n_layers * per_layer_w + cfg.vocab * d) * 2
+    kv = cfg.n_layers * 2 * cfg.n_kv_heads * (kv_len + T) * D * 2
+    act = cfg.n_layers * T * (cfg.top_k * (3 * d + cfg.ffn_expert) * 2 + 12 * d * 4)
+    active = cfg.active_params_per_token()
+    flops = 2 * T * active + cfg.n_layers * 4 * cfg.n_q_heads * T * (kv_len + T) * D
+    return weights + kv + act, flops
+
+
+# ---------------------------------------------------------------------------
+# oracle baseline (host cores)
+# ---------------------------------------------------------------------------
+def oracle_sample(reps: int = 1, warm: int = 0):
+    """Time the fp64 oracle on a bounded sample of the workload: one of the 30
+    layers of a denoising step over a 256-token canvas with a 4096-token
+    prefix, plus the LM head over 1/16 of the vocabulary; scaled to a canvas
+    (12 steps of 30 layers + LM head, one 30-layer commit)."""
+    import numpy as np
+    from oracle import layers as OL
+    from oracle.model import Oracle
+    from synth import FULL, make_kv_prefix, make_layer, make_tokens, to_f64
+    from synth.weights import _normal_bf16, tensor_seed
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [os.cpu_count()])
+    except Exception:
+        threads = os.cpu_count()
+    cfg1 = FULL.with_(n_layers=1)
+    lw = {k: to_f64(v) for k, v in make_layer(FULL, 0, seed=0).items()}
+    embed = _normal_bf16((FULL.vocab, FULL.d_model), tensor_seed(0, -1, "embed"), "cpu", 0.02)
+    tok = make_tokens(FULL, 256, seed=2, name="canvas").numpy().astype(np.int64)
+    k, v = make_kv_prefix(FULL, PROMPT, seed=1)
+    Vs = FULL.vocab // 16
+    emb_rows = to_f64(embed[: Vs])
+    ora = Oracle(cfg1, {"embed": to_f64(embed), "final_norm": np.ones(FULL.d_model), "layers": [lw]})
+    times = []
+    for it in range(warm + reps):
+        cache = ora.new_cache(PROMPT + 256)
+        cache.K[0][:, :PROMPT] = to_f64(k)
+        cache.V[0][:, :PROMPT] = to_f64(v)
+        cache.length = PROMPT
+        t0 = time.perf_counter()
+        from oracle.model import Trace
+        tr = Trace()
+        ora.forward(tok, cache, want_stats=False, trace=tr)
+        t1 = time.perf_counter()
+        xn = OL.rms_norm(tr.layers[0]["x_out"], np.ones(FULL.d_model), FULL.norm_eps)
+        OL.lm_head_stats(xn, emb_rows)
+        t2 = time.perf_counter()
+        if it >= warm:
+            t_layer, t_lm = t1 - t0, (t2 - t1) * 16
+            t_step = FULL.n_layers * t_layer + t_lm
+            t_canvas = 12 * t_step + FULL.n_layers * t_layer
+            times.append((256.0 / t_canvas, t_canvas, t_step, t1 - t0 + t2 - t1))
+    tok_s = sum(t[0] for t in times) / len(times)
+    return {"value": tok_s, "unit": "tok/s", "cores": threads, "kind": "oracle",
+            "sample": "fp64 oracle: 1 of 30 layers of one denoising step (256-token canvas, 4096-token KV prefix) "
+                      "+ LM head on 1/16 of the vocab, scaled to 12 steps + 1 commit per 256-token canvas",
+            "ms_per_denoise_step": 1e3 * sum(t[2] for t in times) / len(times),
+            "ms_per_canvas": 1e3 * sum(t[1] for t in times) / len(times),
+            "sample_seconds": sum(t[3] for t in times) / len(times)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (replicas)
+# ---------------------------------------------------------------------------
+def dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# the reference arm: the oracle, as it stands, on the host cores
+# ---------------------------------------------------------------------------
+def run_reference(args, world):
+    from synth import FULL
+    s = oracle_sample(reps=args.steps, warm=args.warmup)
+    line = {"impl": "reference", "metric": METRIC, "value": s["value"], "unit": "tok/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": s["ms_per_canvas"],
+            "ms_per_denoise_step": s["ms_per_denoise_step"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(FULL, "generate", world),
+            "cpu_baseline": {k: s[k] for k in ("value", "unit", "cores", "kind", "sample")},
+            "e2e": {"value": s["value"], "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(cfg, workload, world):
+    if workload == "layer":
+        name = ("layer: one decoder layer at full shape + LM head over 262144, one denoising step, "
+                "4096-token synthetic KV prefix, 256-token canvas, batch 1")
+    else:
+        name = ("generate: 30 layers d2816, 16q/8kv heads x256, 128 experts top-8 + shared 2112, vocab 262144, "
+                "4096-token prompt prefilled, canvases of 256 (12 steps + commit), blocks 0-3, batch 1")
+    return {"workload": name, "canvas": cfg.canvas, "kv_prefix": PROMPT, "batch": 1,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": "inputs larger than L2: every step streams ~50 GB of weights (no flush needed)"}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def main():
+    args = parse()
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, world)
+        return
+    import torch
+
+    import block_diffusion_moe_denoise_b200 as dgm
+    from synth import FULL, LAYER, make_kv_prefix, make_tokens, make_weights
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    cfg = FULL if args.workload == "generate" else LAYER
+    hbm_gbs, bf16_tf, bf16_tf_sus, peak_kind = measured_peaks()
+
+    w = make_weights(cfg, seed=0, device=dev)
+    torch.cuda.synchronize()
+    cap = PROMPT + N_OUT if args.workload == "generate" else PROMPT + cfg.canvas
+    h = dgm.DG(cfg, w, max_requests=1, kv_capacity=cap, device=dev)
+    st = h.stream
+    prompt = make_tokens(cfg, PROMPT, seed=0)
+
+    def ev():
+        e = torch.cuda.Event(enable_timing=True)
+        e.record(st)
+        return e
+
+    seg_steps, seg_commit, steps_per = [], [], []
+    if args.workload == "generate":
+        t0e = ev()
+        h.prefill(0, prompt.to(dev))
+        t1e = ev()
+        h.sync()
+        prefill_ms = t0e.elapsed_time(t1e)
+
+        def one_step(i, record=False):
+            b = i % 4
+            if b == 0:
+                h.set_kv_len(0, PROMPT)
+            h.open_canvas(0, SEED, b)
+            e0 = ev() if record else None
+            n = 0
+            while True:
+                h.denoise_step([0])
+                n += 1
+                if h.read_remaining(0) == 0:
+                    break
+            e1 = ev() if record else None
+            h.commit_block(0)
+            e2 = ev() if record else None
+            if record:
+                seg_steps.append((e0, e1))
+                seg_commit.append((e1, e2))
+                steps_per.append(n)
+    else:
+        k, v = make_kv_prefix(cfg, PROMPT, seed=1, device=dev)
+        h.set_kv(0, 0, 0, k, v)
+        h.set_kv_len(0, PROMPT)
+        prefill_ms = None
+
+        def one_step(i, record=False):
+            if i % cfg.max_steps == 0:
+                h.open_canvas(0, SEED, 0)
+            e0 = ev() if record else None
+            h.denoise_step([0])
+            e1 = ev() if record else None
+            if record:
+                seg_steps.append((e0, e1))
+                steps_per.append(1)
+
+    for i in range(args.warmup):
+        one_step(i)
+    h.sync()
+    barrier(world)
+    torch.cuda.synchronize()
+    launches0 = h.launch_count()
+    uuid = str(torch.cuda.get_device_properties(dev).uuid) if hasattr(torch.cuda.get_device_properties(dev), "uuid") else ""
+    with ClockSampler(uuid) as clk:
+        start = ev()
+        for i in range(args.steps):
+            one_step(args.warmup + i, record=True)
+        end = ev()
+        torch.cuda.synchronize()
+    barrier(world)
+    elapsed = start.elapsed_time(end)
+    launches = h.launch_count() - launches0
+    h.sync()
+    elapsed_max = max_over_ranks(elapsed, world)
+    toks_per_step = cfg.canvas if args.workload == "generate" else cfg.canvas / 12.0
+    value = world * toks_per_step * args.steps / (elapsed_max / 1e3)
+    step_ms = sum(a.elapsed_time(b) for a, b in seg_steps)
+    n_steps = sum(steps_per)
+    ms_denoise = step_ms / n_steps
+    commit_ms = sum(a.elapsed_time(b) for a, b in seg_commit) / max(1, len(seg_commit))
+
+    # kernel-class breakdown: one more profiled step (events on the library stream)
+    h.profile(-1)
+    h.profile(1)
+    one_step(args.warmup + args.steps, record=False)
+    h.profile(0)
+    prof = h.profile_read()
+    counts = h.debug_buffer("counts", torch.int32, (cfg.n_experts,)).cpu()
+    n_touched = int((counts > 0).sum())
+    T = cfg.canvas
+    egu_ms, egu_n = prof["experts_gate_up"]
+    egu_bytes = expert_gate_up_bytes(cfg, n_touched, T)
+    egu_avg_ms = egu_ms / max(1, egu_n)
+    achieved = egu_bytes / (egu_avg_ms * 1e-3) / 1e9
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "experts_gate_up_traffic.json")
+    if os.path.exists(tpath):
+        try:
+            tj = json.load(open(tpath))
+            import hashlib
+            src = open(os.path.join(ROOT, "block_diffusion_moe_denoise_b200", "csrc", "gemm_ops.cu"), "rb").read()
+            src += open(os.path.join(ROOT, "block_diffusion_moe_denoise_b200", "csrc", "umma_gemm.cuh"), "rb").read()
+            if tj.get("source_sha256") == hashlib.sha256(src).hexdigest():
+                traffic = tj["bytes_per_launch"]
+        except Exception:
+            traffic = None
+    total_prof = sum(v[0] for v in prof.values()) or 1.0
+    kernels = {k: {"ms": round(v[0], 4), "launches": v[1], "share": round(v[0] / total_prof, 4)}
+               for k, v in prof.items() if v[1] > 0}
+    sbytes, sflops = step_work(cfg, PROMPT + 384 if args.workload == "generate" else PROMPT, T, n_touched)
+    t_roof_ms = max(sbytes / (hbm_gbs * 1e9), sflops / (bf16_tf * 1e12)) * 1e3
+
+    e2e = None
+    if args.workload == "generate" and not args.no_e2e:
+        ph = prompt.to(torch.int32).pin_memory()
+        out = torch.empty(N_OUT, dtype=torch.int32).pin_memory()
+        h.set_kv_len(0, 0)
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        gen_steps = h.generate(0, ph, N_OUT, SEED, out)
+        t1 = time.perf_counter()
+        e2e_val = max_over_ranks(t1 - t0, world)
+        nb = N_OUT // cfg.canvas
+        e2e = {"value": world * N_OUT / e2e_val, "unit": "tok/s", "h2d_bytes_per_step": PROMPT * 4 // nb,
+               "d2h_bytes_per_step": cfg.canvas * 4 + 4 * (sum(gen_steps) // nb),
+               "scope": "dg_generate with pinned host buffers: prompt H2D + prefill + 4 canvases + output D2H",
+               "steps_per_canvas": gen_steps}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        s = oracle_sample()
+        cpu = {k: s[k] for k in ("value", "unit", "cores", "kind", "sample")}
+
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tok/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": elapsed_max / args.steps,
+        "ms_per_denoise_step": ms_denoise,
+        "ms_per_commit": commit_ms,
+        "steps_per_canvas": steps_per[:8],
+        "prefill_ms": prefill_ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,0.02) bf16 weights, uniform token ids)",
+        "config": workload_config(cfg, args.workload, world),
+        "roofline": {"kernel": "experts_gate_up (routed-expert gate|up GEMM + SwiGLU)", "bound": "hbm",
+                     "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s", "frac": achieved / hbm_gbs,
+                     "traffic": traffic, "algorithmic_bytes_per_launch": egu_bytes,
+                     "avg_launch_ms": egu_avg_ms, "peak_source": f"{peak_kind} HBM copy (MEASURED_PEAKS.json)"},
+        "step_roofline": {"bytes": sbytes, "flops": sflops, "bound": "hbm" if sbytes / hbm_gbs > sflops / bf16_tf / 1e3
+                          else "tensor", "t_roof_ms": t_roof_ms, "frac": t_roof_ms / ms_denoise,
+                          "experts_touched_per_layer": n_touched},
+        "kernels": kernels,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    h.close()
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

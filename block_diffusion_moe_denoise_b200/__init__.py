@@ -171,6 +171,24 @@ class DG:
         check(self.lib.dg_op_lm_head(self.h, _ptr(x), T, _ptr(stats), _ptr(am), _ptr(logits)), "dg_op_lm_head")
         return stats, am, logits
 
+    KERNEL_CLASSES = ("embed", "rmsnorm", "qkv", "attention", "oproj", "router", "group", "gather",
+                      "experts_gate_up", "experts_down", "shared_gate_up", "shared_down", "lm_head", "lm_combine",
+                      "sample", "other")
+
+    def profile(self, enable: int):
+        check(self.lib.dg_profile(self.h, enable), "dg_profile")
+
+    def profile_read(self) -> dict:
+        out = {}
+        for k in self.KERNEL_CLASSES:
+            ms, n = C.c_double(), C.c_int64()
+            check(self.lib.dg_profile_read(self.h, k.encode(), C.byref(ms), C.byref(n)), "dg_profile_read")
+            out[k] = (ms.value, n.value)
+        return out
+
+    def launch_count(self) -> int:
+        return self.lib.dg_launch_count(self.h)
+
     def debug_forward(self, req: int, tokens: torch.Tensor, n_layers: int):
         check(self.lib.dg_debug_forward(self.h, req, _ptr(tokens), tokens.numel(), n_layers), "dg_debug_forward")
 

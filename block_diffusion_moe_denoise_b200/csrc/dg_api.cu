@@ -133,8 +133,55 @@ bool make_map(CUtensorMap* m, const void* base, long long K, long long rows, int
 
 }  // namespace
 
+// Opt-in per-kernel-class timing with CUDA events recorded on the handle's
+// stream around each launch (dg_profile); a launch counter is always kept.
+struct KernelProfiler {
+  bool on = false;
+  std::vector<std::pair<int, std::pair<cudaEvent_t, cudaEvent_t>>> pending;
+  std::vector<cudaEvent_t> pool;
+  double total_ms[16] = {0};
+  long long count[16] = {0};
+  cudaEvent_t get() {
+    if (!pool.empty()) {
+      cudaEvent_t e = pool.back();
+      pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+  }
+  void flush() {
+    for (auto& r : pending) {
+      cudaEventSynchronize(r.second.second);
+      float ms = 0.f;
+      cudaEventElapsedTime(&ms, r.second.first, r.second.second);
+      total_ms[r.first] += ms;
+      count[r.first] += 1;
+      pool.push_back(r.second.first);
+      pool.push_back(r.second.second);
+    }
+    pending.clear();
+  }
+  ~KernelProfiler() {
+    for (auto& r : pending) {
+      cudaEventDestroy(r.second.first);
+      cudaEventDestroy(r.second.second);
+    }
+    for (auto e : pool) cudaEventDestroy(e);
+  }
+};
+
+const char* const kKernelClass[] = {"embed", "rmsnorm", "qkv", "attention", "oproj", "router", "group", "gather",
+                                    "experts_gate_up", "experts_down", "shared_gate_up", "shared_down", "lm_head",
+                                    "lm_combine", "sample", "other"};
+enum KClass { K_EMBED, K_RMSNORM, K_QKV, K_ATTN, K_OPROJ, K_ROUTER, K_GROUP, K_GATHER, K_EGU, K_ED, K_SGU, K_SD,
+              K_LM, K_LMC, K_SAMPLE, K_OTHER };
+
 struct dg_handle {
   dg_config cfg;
+  KernelProfiler prof;
+  long long launches = 0;
   int max_req = 0;
   long long cap = 0;
   cudaStream_t st = nullptr;
@@ -163,6 +210,24 @@ struct dg_handle {
     if (e__ != cudaSuccess) return DG_E_CUDA; \
   } while (0)
 
+// Launch `expr` (n kernels of class `cls`), counting it and, when profiling,
+// bracketing it with events on the handle's stream.
+#define LAUNCH(h, cls, n, expr)                                              \
+  do {                                                                       \
+    cudaEvent_t e0__ = nullptr, e1__ = nullptr;                              \
+    if ((h)->prof.on) {                                                      \
+      e0__ = (h)->prof.get();                                                \
+      e1__ = (h)->prof.get();                                                \
+      cudaEventRecord(e0__, (h)->st);                                        \
+    }                                                                        \
+    CK(expr);                                                                \
+    (h)->launches += (n);                                                    \
+    if ((h)->prof.on) {                                                      \
+      cudaEventRecord(e1__, (h)->st);                                        \
+      (h)->prof.pending.push_back({(int)(cls), {e0__, e1__}});               \
+    }                                                                        \
+  } while (0)
+
 namespace {
 
 // One decoder pass over s.n slots of s.Tr tokens.  n_layers layers; when
@@ -177,12 +242,12 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
   int* err = h->B<int>("err");
   float* x = h->B<float>("x");
   bf16* hn = h->B<bf16>("hn");
-  CK(run_embed(ids, s, h->embed, c.vocab, d, x, h->B<int>("tok_pos"), h->B<int>("tok_req"), err, st));
+  LAUNCH(h, K_EMBED, 1, run_embed(ids, s, h->embed, c.vocab, d, x, h->B<int>("tok_pos"), h->B<int>("tok_req"), err, st));
   for (int l = 0; l < n_layers; ++l) {
     const dg_layer_weights& w = h->lw[l];
     const LayerMaps& m = h->maps[l];
     bf16* kv_l = h->B<bf16>("kv") + (size_t)l * h->kv_layer_stride;
-    CK(run_rmsnorm(x, (const float*)w.attn_norm, T, d, c.norm_eps, hn, st));
+    LAUNCH(h, K_RMSNORM, 1, run_rmsnorm(x, (const float*)w.attn_norm, T, d, c.norm_eps, hn, st));
     QkvArgs qa;
     qa.tm_x = &h->tm_hn;
     qa.tm_w = &m.qkv;
@@ -202,7 +267,7 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     qa.q = h->B<bf16>("q");
     qa.kv = kv_l;
     qa.err = err;
-    CK(run_qkv(qa, st));
+    LAUNCH(h, K_QKV, 1, run_qkv(qa, st));
     if (qkv_only_last && l == c.n_layers - 1) break;
 
     AttnArgs aa;
@@ -234,7 +299,7 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     aa.part_o = h->B<float>("attn_o");
     aa.part_ml = h->B<float2>("attn_ml");
     aa.scale = 1.0f / sqrtf((float)D);
-    CK(run_attention(aa, st));
+    LAUNCH(h, K_ATTN, aa.n_split > 1 ? 2 : 1, run_attention(aa, st));
 
     OprojArgs oa;
     oa.tm_w = &m.o;
@@ -245,10 +310,11 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     oa.num_sms = h->num_sms;
     oa.x = x;
     oa.err = err;
-    CK(run_oproj(oa, st));
+    LAUNCH(h, K_OPROJ, 1, run_oproj(oa, st));
 
-    CK(run_router(x, (const float*)w.ffn_norm, c.norm_eps, (const bf16*)w.w_router, T, d, c.n_experts, k,
-                  h->B<bf16>("u"), h->B<int>("idx"), h->B<float>("w"), err, st));
+    LAUNCH(h, K_ROUTER, 1,
+           run_router(x, (const float*)w.ffn_norm, c.norm_eps, (const bf16*)w.w_router, T, d, c.n_experts, k,
+                      h->B<bf16>("u"), h->B<int>("idx"), h->B<float>("w"), err, st));
     GroupArgs ga;
     ga.idx = h->B<int>("idx");
     ga.w = h->B<float>("w");
@@ -270,8 +336,8 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     ga.ed_tiles = h->B<int4>("ed_tiles");
     ga.ed_count = h->B<int>("tile_counts") + 1;
     ga.err = err;
-    CK(run_group(ga, st));
-    CK(run_gather(h->B<bf16>("u"), h->B<int>("row_token"), T * k, d, h->B<bf16>("xp"), st));
+    LAUNCH(h, K_GROUP, 1, run_group(ga, st));
+    LAUNCH(h, K_GATHER, 1, run_gather(h->B<bf16>("u"), h->B<int>("row_token"), T * k, d, h->B<bf16>("xp"), st));
 
     ExpertArgs ea;
     ea.tm_gate = &m.gate;
@@ -292,7 +358,8 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     ea.hp = h->B<bf16>("hp");
     ea.yp = h->B<float>("yp");
     ea.err = err;
-    CK(run_experts(ea, st));
+    LAUNCH(h, K_EGU, 1, run_experts_gate_up(ea, st));
+    LAUNCH(h, K_ED, 1, run_experts_down(ea, st));
 
     SharedArgs sa;
     sa.tm_u = &h->tm_u;
@@ -310,10 +377,11 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     sa.yp = h->B<float>("yp");
     sa.pair_row = h->B<int>("pair_row");
     sa.err = err;
-    CK(run_shared(sa, st));
+    LAUNCH(h, K_SGU, 1, run_shared_gate_up(sa, st));
+    LAUNCH(h, K_SD, 1, run_shared_down(sa, st));
   }
   if (want_lm) {
-    CK(run_rmsnorm(x, h->final_norm, T, d, c.norm_eps, hn, st));
+    LAUNCH(h, K_RMSNORM, 1, run_rmsnorm(x, h->final_norm, T, d, c.norm_eps, hn, st));
     LmArgs la;
     la.tm_x = &h->tm_hn;
     la.tm_embed = &h->tm_embed;
@@ -325,9 +393,10 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     la.logits = logits;
     la.err = err;
     int grid = 0;
-    CK(run_lm_head(la, &grid, st));
-    CK(run_lm_combine(h->B<float4>("lm_part"), grid, (T + 127) / 128, T, h->B<float>("stats"), h->B<int>("argmax"),
-                      err, st));
+    LAUNCH(h, K_LM, 1, run_lm_head(la, &grid, st));
+    LAUNCH(h, K_LMC, 1,
+           run_lm_combine(h->B<float4>("lm_part"), grid, (T + 127) / 128, T, h->B<float>("stats"),
+                          h->B<int>("argmax"), err, st));
   }
   return DG_OK;
 }
@@ -501,8 +570,9 @@ int dg_open_canvas(dg_handle* h, int req, uint64_t seed, int block) {
   ReqState& r = h->req[req];
   if (r.kv_len + h->cfg.canvas > h->cap) return DG_E_CAPACITY;
   const int C = h->cfg.canvas;
-  CK(run_philox_tokens(seed, block, 0, req, 0, C, h->cfg.vocab, h->B<int>("canvas") + (size_t)req * C,
-                       h->B<unsigned char>("mask") + (size_t)req * C, h->st));
+  LAUNCH(h, K_OTHER, 1,
+         run_philox_tokens(seed, block, 0, req, 0, C, h->cfg.vocab, h->B<int>("canvas") + (size_t)req * C,
+                           h->B<unsigned char>("mask") + (size_t)req * C, h->st));
   CK(cudaMemsetAsync(h->B<int>("remaining") + req, 0, 4, h->st));
   r.open = true;
   r.seed = seed;
@@ -537,7 +607,7 @@ static int sample_slots(dg_handle* h, int n_req, const int* reqs, const float* e
   a.mask = h->B<unsigned char>("mask");
   a.remaining = h->B<int>("remaining");
   a.err = h->B<int>("err");
-  CK(run_sample(a, h->st));
+  LAUNCH(h, K_SAMPLE, 1, run_sample(a, h->st));
   return DG_OK;
 }
 
@@ -780,6 +850,34 @@ int dg_debug_forward(dg_handle* h, int req, const int32_t* d_tokens, int T, int 
   const int* ids[1] = {d_tokens};
   return run_pass(h, ids, s, n_layers, false, n_layers == h->cfg.n_layers, nullptr);
 }
+
+int dg_profile(dg_handle* h, int enable) {
+  if (!h) return DG_E_ARG;
+  h->prof.flush();
+  if (enable < 0) {
+    for (int i = 0; i < 16; ++i) {
+      h->prof.total_ms[i] = 0.0;
+      h->prof.count[i] = 0;
+    }
+    return DG_OK;
+  }
+  h->prof.on = enable != 0;
+  return DG_OK;
+}
+
+int dg_profile_read(dg_handle* h, const char* kernel, double* total_ms, int64_t* launches) {
+  if (!h || !kernel) return DG_E_ARG;
+  h->prof.flush();
+  for (int i = 0; i < 16; ++i)
+    if (strcmp(kernel, kKernelClass[i]) == 0) {
+      if (total_ms) *total_ms = h->prof.total_ms[i];
+      if (launches) *launches = h->prof.count[i];
+      return DG_OK;
+    }
+  return DG_E_ARG;
+}
+
+int64_t dg_launch_count(const dg_handle* h) { return h ? h->launches : -1; }
 
 int dg_debug_buffer(const dg_handle* h, const char* name, size_t* offset, size_t* bytes) {
   if (!h || !name) return DG_E_ARG;

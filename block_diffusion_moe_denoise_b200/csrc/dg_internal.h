@@ -70,8 +70,10 @@ struct LmArgs {
 
 cudaError_t run_qkv(const QkvArgs& a, cudaStream_t st);
 cudaError_t run_oproj(const OprojArgs& a, cudaStream_t st);
-cudaError_t run_experts(const ExpertArgs& a, cudaStream_t st);
-cudaError_t run_shared(const SharedArgs& a, cudaStream_t st);
+cudaError_t run_experts_gate_up(const ExpertArgs& a, cudaStream_t st);
+cudaError_t run_experts_down(const ExpertArgs& a, cudaStream_t st);
+cudaError_t run_shared_gate_up(const SharedArgs& a, cudaStream_t st);
+cudaError_t run_shared_down(const SharedArgs& a, cudaStream_t st);
 cudaError_t run_lm_head(const LmArgs& a, int* grid_out, cudaStream_t st);
 size_t gemm_smem_bytes_max();
 

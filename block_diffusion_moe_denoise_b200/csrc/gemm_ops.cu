@@ -561,7 +561,7 @@ cudaError_t run_oproj(const OprojArgs& a, cudaStream_t st) {
   return launch_gemm<P_OPROJ>(p, grid_for(p.MT * p.NT, a.num_sms), st);
 }
 
-cudaError_t run_experts(const ExpertArgs& a, cudaStream_t st) {
+cudaError_t run_experts_gate_up(const ExpertArgs& a, cudaStream_t st) {
   P_EGU::Params g;
   g.tmG = *a.tm_gate;
   g.tmU = *a.tm_up;
@@ -574,8 +574,10 @@ cudaError_t run_experts(const ExpertArgs& a, cudaStream_t st) {
   g.offsets = a.offsets;
   g.hp = a.hp;
   g.err = a.err;
-  cudaError_t e = launch_gemm<P_EGU>(g, a.num_sms, st);
-  if (e != cudaSuccess) return e;
+  return launch_gemm<P_EGU>(g, a.num_sms, st);
+}
+
+cudaError_t run_experts_down(const ExpertArgs& a, cudaStream_t st) {
   P_ED::Params dn;
   dn.tmW = *a.tm_down;
   dn.tmH = *a.tm_hp;
@@ -591,7 +593,7 @@ cudaError_t run_experts(const ExpertArgs& a, cudaStream_t st) {
   return launch_gemm<P_ED>(dn, a.num_sms, st);
 }
 
-cudaError_t run_shared(const SharedArgs& a, cudaStream_t st) {
+cudaError_t run_shared_gate_up(const SharedArgs& a, cudaStream_t st) {
   P_SGU::Params g;
   g.tmX = *a.tm_u;
   g.tmG = *a.tm_gate;
@@ -603,8 +605,10 @@ cudaError_t run_shared(const SharedArgs& a, cudaStream_t st) {
   g.fs = a.fs;
   g.hs = a.hs;
   g.err = a.err;
-  cudaError_t e = launch_gemm<P_SGU>(g, grid_for(g.MT * g.FJ, a.num_sms), st);
-  if (e != cudaSuccess) return e;
+  return launch_gemm<P_SGU>(g, grid_for(g.MT * g.FJ, a.num_sms), st);
+}
+
+cudaError_t run_shared_down(const SharedArgs& a, cudaStream_t st) {
   P_SD::Params dn;
   dn.tmW = *a.tm_down;
   dn.tmH = *a.tm_hs;

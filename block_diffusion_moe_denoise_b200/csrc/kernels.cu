@@ -151,7 +151,8 @@ cudaError_t run_topk(const float* logits, int T, int E, int k, int* idx, float* 
 }
 
 // ---------------------------------------------------------------------------
-// FFN RMSNorm + router logits (fp32 accumulate of bf16 inputs) + top-k.
+// FFN RMSNorm + router logits (fp32 normalised row x bf16 router weights,
+// fp32 accumulation) + top-k.
 // kRouterTok tokens per CTA so the router weight is read once per CTA.
 // ---------------------------------------------------------------------------
 constexpr int kRouterTok = 4;
@@ -184,9 +185,9 @@ __global__ void __launch_bounds__(256) k_router(const float* __restrict__ x, con
         const uint32_t lo = pack_bf16x2(v.x * rs * gg.x, v.y * rs * gg.y);
         const uint32_t hi = pack_bf16x2(v.z * rs * gg.z, v.w * rs * gg.w);
         uo[c] = make_uint2(lo, hi);
-        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&lo));
-        const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hi));
-        reinterpret_cast<float4*>(dst)[c] = make_float4(a.x, a.y, b.x, b.y);
+        // the router reads the fp32 normalised row (the experts read the bf16 copy)
+        reinterpret_cast<float4*>(dst)[c] =
+            make_float4(v.x * rs * gg.x, v.y * rs * gg.y, v.z * rs * gg.z, v.w * rs * gg.w);
       }
     } else {
       for (int c = lane; c < d; c += 32) dst[c] = 0.f;

@@ -62,6 +62,18 @@ int dg_debug_forward(dg_handle* h, int req, const int32_t* d_tokens, int T, int 
  * "remaining" i32 [max_req].  Returns DG_E_ARG for an unknown name. */
 int dg_debug_buffer(const dg_handle* h, const char* name, size_t* offset, size_t* bytes);
 
+/* Per-kernel-class timing: enable=1 records a CUDA event pair on the handle's
+ * stream around every launch of the pass, enable=0 stops, enable=-1 clears the
+ * totals.  dg_profile_read (synchronising) returns the summed elapsed ms and
+ * launch count of one class: "embed", "rmsnorm", "qkv", "attention", "oproj",
+ * "router", "group", "gather", "experts_gate_up", "experts_down",
+ * "shared_gate_up", "shared_down", "lm_head", "lm_combine", "sample", "other". */
+int dg_profile(dg_handle* h, int enable);
+int dg_profile_read(dg_handle* h, const char* kernel, double* total_ms, int64_t* launches);
+
+/* Kernels launched by this handle so far (always counted). */
+int64_t dg_launch_count(const dg_handle* h);
+
 #ifdef __cplusplus
 }
 #endif

@@ -39,3 +39,49 @@ def rel_l2(a, b) -> float:
 def routing_match(gpu_idx: np.ndarray, ora_idx: np.ndarray) -> np.ndarray:
     """Tokens whose selected experts agree (same set; order may differ only on exact ties)."""
     return np.array([set(a.tolist()) == set(b.tolist()) for a, b in zip(gpu_idx, ora_idx)])
+
+
+# Routing ambiguity.  Top-k routing is discontinuous: a token whose k-th and
+# (k+1)-th router logits are nearly tied can pick a different expert on the GPU
+# than in the oracle (the GPU's residual stream carries bf16 rounding of every
+# earlier GEMM input, about 1e-3 relative, i.e. router-logit noise of ~4e-4 at
+# d=256 and ~1.2e-3 at d=2816), which moves that token's hidden state by tens
+# of percent.  Such tokens are identified from the ORACLE's own router logits
+# (gap below ROUTER_GAP, >= 4 sigma of that noise), excluded from value
+# comparisons and counted; everywhere else routing must agree exactly.
+ROUTER_GAP = 5e-3
+
+
+def router_gap(router_logits: np.ndarray, k: int) -> np.ndarray:
+    s = np.sort(router_logits, axis=-1)
+    return s[:, -k] - s[:, -k - 1]
+
+
+def ambiguous_tokens(trace_layers, k: int, upto: int | None = None) -> np.ndarray:
+    """Tokens whose oracle routing is near a tie in any of the first `upto` layers."""
+    recs = trace_layers if upto is None else trace_layers[:upto]
+    amb = np.zeros(recs[0]["router_logits"].shape[0], dtype=bool)
+    for rec in recs:
+        amb |= router_gap(rec["router_logits"], k) < ROUTER_GAP
+    return amb
+
+
+def oracle_prefill_traced(ora, cache, tokens):
+    """The oracle's prefill, segment by segment, keeping each segment's trace;
+    returns the per-token ambiguity over the layers that feed the K/V."""
+    from oracle.model import Trace
+    tokens = np.asarray(tokens, dtype=np.int64)
+    seg = ora.cfg.canvas
+    amb = []
+    for s0 in range(0, tokens.shape[0], seg):
+        part = tokens[s0: s0 + seg]
+        tr = Trace()
+        ora.forward(part, cache, want_stats=False, trace=tr)
+        cache.length += part.shape[0]
+        amb.append(ambiguous_tokens(tr.layers, ora.cfg.top_k, ora.cfg.n_layers - 1))
+    return np.concatenate(amb)
+
+
+def kv_rel_l2(gpu_kv: np.ndarray, ora_kv: np.ndarray, keep: np.ndarray) -> float:
+    """gpu/ora as [Hkv, n, D]; compare positions where keep is True."""
+    return rel_l2(gpu_kv[:, keep], ora_kv[:, keep])

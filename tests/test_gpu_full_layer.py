@@ -11,7 +11,7 @@ from oracle.model import Oracle, Trace
 from oracle import sampler as OS
 from synth import LAYER, make_kv_prefix, make_weights, to_f64
 
-from .gpu_common import LOGIT_MAX_ABS, REL_L2, np64, rel_l2, routing_match
+from .gpu_common import LOGIT_MAX_ABS, REL_L2, ambiguous_tokens, np64, rel_l2, routing_match
 
 pytestmark = [pytest.mark.gpu,
               pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
@@ -69,7 +69,9 @@ def test_moe_path(setup):
     T, d, k = CFG.canvas, CFG.d_model, CFG.top_k
     idx = h.debug_buffer("idx", torch.int32, (T, k)).cpu().numpy()
     same = routing_match(idx, rec["idx"])
-    assert same.mean() >= 0.95, same.mean()
+    amb = ambiguous_tokens([rec], k)
+    assert same[~amb].all(), np.nonzero(~same & ~amb)
+    print(f"full layer: {amb.sum()} routing-ambiguous tokens, {(~same).sum()} re-routed")
     counts = h.debug_buffer("counts", torch.int32, (CFG.n_experts,)).cpu().numpy()
     assert counts.sum() == T * k and (counts == np.bincount(idx.ravel(), minlength=CFG.n_experts)).all()
     pair_row = h.debug_buffer("pair_row", torch.int32, (T * k,)).cpu().numpy()
@@ -95,7 +97,8 @@ def test_lm_head_sampled_rows(setup):
     h, rec, ora = setup["h"], setup["tr"], setup["ora"]
     stats = h.debug_buffer("stats", torch.float32, (256, 4)).cpu().numpy().astype(np.float64)
     am = h.debug_buffer("argmax", torch.int32, (256,)).cpu().numpy()
-    rows = np.random.default_rng(1).choice(256, 24, replace=False)
+    amb = ambiguous_tokens([rec], CFG.top_k)
+    rows = np.random.default_rng(1).choice(np.nonzero(~amb)[0], 24, replace=False)
     xn = OL.rms_norm(rec["x_out"][rows], ora.final_norm, CFG.norm_eps)
     ref = OL.lm_head_stats(xn, ora.embed)
     assert np.max(np.abs(stats[rows, 2] - ref["max"])) < LOGIT_MAX_ABS

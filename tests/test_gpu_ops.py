@@ -76,7 +76,6 @@ def test_route_group_bitwise(tiny_handle):
 
 
 def test_open_canvas_bitwise(tiny_handle):
-    tiny_handle.set_kv_len(2, 0)
     tiny_handle.open_canvas(2, 1234, 3)
     tok, mask, _, _ = tiny_handle.get_canvas(2)
     torch.cuda.synchronize()
@@ -100,8 +99,7 @@ def test_sampler_bitwise_full_canvas(tiny_handle, low_entropy):
     """Twelve steps of the rule from identical fp32 statistics: canvas, mask and
     remaining match the oracle exactly, and the canvas converges."""
     C, V = TINY.canvas, TINY.vocab
-    req, seed = 1, 77
-    tiny_handle.set_kv_len(req, 0)
+    req, seed = 1, 77 + low_entropy
     tiny_handle.open_canvas(req, seed, 0)
     canvas, acc = OS.init_canvas(C, seed=seed, block=0, vocab=V, request=req)
     rng = np.random.default_rng(2 + low_entropy)
@@ -125,7 +123,6 @@ def test_sampler_bitwise_full_canvas(tiny_handle, low_entropy):
 def test_sampler_step_cap_forces_acceptance(tiny_handle):
     C, V = TINY.canvas, TINY.vocab
     req = 3
-    tiny_handle.set_kv_len(req, 0)
     tiny_handle.open_canvas(req, 5, 1)
     rng = np.random.default_rng(9)
     H, lc, am = _rand_stats(rng, C, V)

@@ -10,7 +10,8 @@ from oracle import layers as OL
 from oracle.model import Oracle, Trace
 from synth import TINY, make_tokens, make_weights
 
-from .gpu_common import LOGIT_MAX_ABS, REL_L2, np64, rel_l2, routing_match, to_device
+from .gpu_common import (LOGIT_MAX_ABS, REL_L2, ambiguous_tokens, kv_rel_l2, np64, oracle_prefill_traced, rel_l2,
+                         routing_match, to_device)
 from .helpers import oracle_weights
 
 pytestmark = [pytest.mark.gpu,
@@ -40,12 +41,14 @@ def test_prefill_kv_matches_oracle(model, n_prompt):
     h.prefill(0, prompt.cuda())
     h.sync()
     cache = ora.new_cache(n_prompt)
-    ora.prefill(cache, prompt.numpy())
+    amb = oracle_prefill_traced(ora, cache, prompt.numpy())
     assert h.kv_len(0) == n_prompt
+    keep = ~amb
+    print(f"prefill {n_prompt}: {amb.sum()} routing-ambiguous tokens excluded")
     for l in range(CFG.n_layers):
         k, v = h.get_kv(0, l, 0, n_prompt)
-        assert rel_l2(np64(k), cache.K[l][:, :n_prompt]) < REL_L2
-        assert rel_l2(np64(v), cache.V[l][:, :n_prompt]) < REL_L2
+        assert kv_rel_l2(np64(k), cache.K[l][:, :n_prompt], keep) < REL_L2
+        assert kv_rel_l2(np64(v), cache.V[l][:, :n_prompt], keep) < REL_L2
     h.close()
 
 
@@ -59,7 +62,7 @@ def test_layer_intermediates(model, T):
     h.prefill(0, prompt.cuda())
     cache = ora.new_cache(128 + 256)
     ora.prefill(cache, prompt.numpy())
-    toks = make_tokens(CFG, T, seed=2, name="canvas")
+    toks = make_tokens(CFG, T, seed=2, name="canvas")  # noqa: E501
     h.debug_forward(0, toks.cuda(), 1)
     h.sync()
     tr = Trace()
@@ -81,7 +84,8 @@ def test_layer_intermediates(model, T):
     idx = h.debug_buffer("idx", torch.int32, (T, k)).cpu().numpy()
     wts = h.debug_buffer("w", torch.float32, (T, k)).cpu().numpy()
     same = routing_match(idx, rec["idx"])
-    assert same.mean() >= 0.97, same.mean()
+    amb = ambiguous_tokens([rec], k)
+    assert same[~amb].all(), np.nonzero(~same & ~amb)
     for t in np.nonzero(same)[0]:
         for j in range(k):
             jj = list(rec["idx"][t]).index(idx[t, j])
@@ -108,6 +112,7 @@ def test_layer_intermediates(model, T):
     assert rel_l2(hs, ref_hs) < REL_L2
     x = np64(h.debug_buffer("x", torch.float32, (Tcap, d))[:T])
     assert rel_l2(x[same], rec["x_out"][same]) < REL_L2
+    print(f"layer T={T}: {amb.sum()} ambiguous, {(~same).sum()} re-routed tokens")
     h.close()
 
 
@@ -144,18 +149,29 @@ def test_lm_head_logits_and_fused_stats(model):
     h.close()
 
 
-def _decisions_agree(ora_stats, ora_prev_acc, ora_acc, gpu_acc, cfg):
+def _decisions_agree(ora_stats, ora_prev_acc, ora_acc, gpu_acc, cfg, amb):
     """Positions where the accept decision differs must be near a decision
     boundary of the oracle: top-1 margin <= 1e-2, logconf within 1e-2 of the
-    min_accept-th value among unaccepted positions, or entropy within 1e-2 of
-    the threshold.  Returns (n_compared, n_excluded, n_bad)."""
+    min_accept-th value among unaccepted positions, entropy within 1e-2 of
+    the threshold, or routing-ambiguous in the oracle.  Any position whose
+    decision flips also shifts the rank cut by one, so the position ranked
+    next to the cut is on the boundary too.  Returns (n_compared, n_excluded,
+    n_bad)."""
     U = ~ora_prev_acc
     lc = ora_stats["logconf"]
     srt = np.sort(ora_stats["logits"], axis=-1)
     margin = srt[:, -1] - srt[:, -2]
     cut = np.sort(lc[U])[::-1][min(cfg.min_accept, U.sum()) - 1] if U.any() else 0.0
     near = (margin <= 1e-2) | (np.abs(lc - cut) <= 1e-2) | (np.abs(ora_stats["entropy"] - cfg.entropy_thresh) <= 1e-2)
+    near |= amb
     diff = (ora_acc != gpu_acc) & U
+    m = int((diff & near).sum())
+    if m:
+        n_top = min(cfg.min_accept, int(U.sum()))
+        order = sorted(np.nonzero(U)[0].tolist(), key=lambda i: (-lc[i], i))
+        rank = np.full(lc.shape[0], 10 ** 9)
+        rank[order] = np.arange(len(order))
+        near |= (rank >= n_top - m) & (rank < n_top + m)
     return int(U.sum()), int((near & U).sum()), int((diff & ~near).sum())
 
 
@@ -177,7 +193,10 @@ def test_teacher_forced_denoising_steps(model):
     excluded = 0
     for step in range(1, CFG.max_steps + 1):
         prev = acc.copy()
-        ncanvas, nacc, rem, st = ora.denoise_step(cache, canvas, acc, seed=seed, block=0, step=step)
+        tr = Trace()
+        st = ora.forward(canvas, cache, trace=tr)
+        amb = ambiguous_tokens(tr.layers, CFG.top_k)
+        ncanvas, nacc, rem, st = ora.denoise_step(cache, canvas, acc, seed=seed, block=0, step=step, stats=st)
         h.set_canvas(0, torch.from_numpy(canvas.astype(np.int32)).cuda(),
                      torch.from_numpy(acc.astype(np.uint8)).cuda(), step - 1)
         h.denoise_step([0])
@@ -185,16 +204,16 @@ def test_teacher_forced_denoising_steps(model):
         h.sync()
         gtok, gmask = gtok.cpu().numpy(), gmask.cpu().numpy().astype(bool)
         gs = gstats.cpu().numpy().astype(np.float64)
-        assert np.max(np.abs(gs[:, 2] - st["max"])) < LOGIT_MAX_ABS
-        assert rel_l2(gs[:, 0], st["entropy"]) < REL_L2
-        n, nex, bad = _decisions_agree(st, prev, nacc, gmask, CFG)
+        assert np.max(np.abs(gs[~amb, 2] - st["max"][~amb])) < LOGIT_MAX_ABS
+        assert rel_l2(gs[~amb, 0], st["entropy"][~amb]) < REL_L2
+        n, nex, bad = _decisions_agree(st, prev, nacc, gmask, CFG, amb)
         assert bad == 0, (step, bad)
         excluded += nex
         both_rej = ~nacc & ~gmask
         np.testing.assert_array_equal(gtok[both_rej], ncanvas[both_rej])     # Philox re-noise, bitwise
         both_acc_new = nacc & gmask & ~prev
         srt = np.sort(st["logits"], axis=-1)
-        sure = both_acc_new & (srt[:, -1] - srt[:, -2] > 1e-2)
+        sure = both_acc_new & (srt[:, -1] - srt[:, -2] > 1e-2) & ~amb
         np.testing.assert_array_equal(gtok[sure], ncanvas[sure])
         canvas, acc = ncanvas, nacc
         if rem == 0:
@@ -221,14 +240,16 @@ def test_commit_equals_prefill_and_oracle(model):
     h.sync()
     assert h.kv_len(0) == h.kv_len(1) == 384
     cache = ora.new_cache(384)
-    ora.prefill(cache, prompt.numpy())
-    ora.commit(cache, block.numpy())
+    amb_p = oracle_prefill_traced(ora, cache, prompt.numpy())
+    amb_c = oracle_prefill_traced(ora, cache, block.numpy())      # commit == prefill of the block
+    keep = ~amb_c
+    print(f"commit: {amb_c.sum()} routing-ambiguous block tokens excluded ({amb_p.sum()} in the prompt)")
     for l in range(CFG.n_layers):
         k0, v0 = h.get_kv(0, l, 0, 384)
         k1, v1 = h.get_kv(1, l, 0, 384)
         assert torch.equal(k0, k1) and torch.equal(v0, v1)
-        assert rel_l2(np64(k0)[:, 128:], cache.K[l][:, 128:384]) < REL_L2
-        assert rel_l2(np64(v0)[:, 128:], cache.V[l][:, 128:384]) < REL_L2
+        assert kv_rel_l2(np64(k0)[:, 128:], cache.K[l][:, 128:384], keep) < REL_L2
+        assert kv_rel_l2(np64(v0)[:, 128:], cache.V[l][:, 128:384], keep) < REL_L2
     h.close()
 
 
