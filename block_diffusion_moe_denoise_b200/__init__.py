@@ -15,7 +15,7 @@ import torch
 from . import _ffi
 from ._ffi import DGError, check, dg_config, dg_layer_weights, dg_weights  # noqa: F401
 
-__all__ = ["DG", "DGError", "config_struct", "philox_tokens", "route_topk"]
+__all__ = ["DG", "DGError", "config_struct", "lm_head_noalloc", "philox_tokens", "route_topk"]
 
 
 def _ptr(t):
@@ -45,6 +45,16 @@ def route_topk(logits: torch.Tensor, k: int, idx: torch.Tensor, w: torch.Tensor,
     T, E = logits.shape
     check(_ffi.load().dg_op_route_topk(_ptr(logits), T, E, k, _ptr(idx), _ptr(w), _stream(stream)),
           "dg_op_route_topk")
+
+
+def lm_head_noalloc(x: torch.Tensor, final_norm: torch.Tensor, embed: torch.Tensor, norm_eps: float,
+                    stats: torch.Tensor, argmax: torch.Tensor, err: torch.Tensor | None = None, stream=None) -> None:
+    """dg_op_lm_head_noalloc: LM-head statistics with the library's built-in
+    scratch (no workspace, no allocation inside)."""
+    T, d = x.shape
+    check(_ffi.load().dg_op_lm_head_noalloc(_ptr(x), _ptr(final_norm), _ptr(embed), T, d, embed.shape[0], norm_eps,
+                                            _ptr(stats), _ptr(argmax), _ptr(err), _stream(stream)),
+          "dg_op_lm_head_noalloc")
 
 
 class DG:

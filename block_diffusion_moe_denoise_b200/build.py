@@ -8,7 +8,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libdg.so")
-SOURCES = ["dg_api.cu", "gemm_ops.cu", "kernels.cu", "attention.cu"]
+SOURCES = ["dg_api.cu", "gemm_ops.cu", "kernels.cu", "attention.cu", "noalloc.cu"]
 HEADERS = ["common.cuh", "umma_gemm.cuh", "dg_internal.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

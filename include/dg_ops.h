@@ -74,6 +74,34 @@ int dg_profile_read(dg_handle* h, const char* kernel, double* total_ms, int64_t*
 /* Kernels launched by this handle so far (always counted). */
 int64_t dg_launch_count(const dg_handle* h);
 
+/* LM-head statistics for callers that cannot allocate device memory.  (No
+ * counterpart in the pages: this is a deployment variant of dg_op_lm_head.)
+ * Some callers have no workspace to give and must not call cudaMalloc: a
+ * serving runtime whose caching allocator already owns all free HBM, or a
+ * latency-critical loop where cudaMalloc's implicit device synchronisation is
+ * not acceptable.  This entry point needs no handle and allocates nothing: it
+ * runs the same final RMSNorm + tied LM head + fused statistics kernels as
+ * dg_op_lm_head with their scratch (normalised bf16 rows and per-CTA partial
+ * statistics) in a fixed 3 MiB array inside the library, which every GPU that
+ * loads the library holds until the process exits.
+ *   d_x [T, d_model] f32 hidden rows, d_final_norm [d_model] f32 gain,
+ *   d_embed [vocab, d_model] bf16 (the tied embedding), all 16-byte aligned;
+ *   outputs d_stats [T][4] = (entropy, logconf, max logit, log-partition) and
+ *   d_argmax [T]; d_err (may be NULL) receives the device error word
+ *   (0 = ok; cleared by each call).  Asynchronous on `stream`.
+ * Limits: 1 <= T <= DG_NOALLOC_MAX_TOKENS, 64 <= d_model <=
+ * DG_NOALLOC_MAX_DMODEL with d_model % 64 == 0, vocab % 256 == 0; anything
+ * else returns DG_E_ARG before any work is enqueued.  The first call on a
+ * device resolves the array's address on that device and must come before any
+ * stream capture.  All calls share the array and it keeps the last call's
+ * contents (nothing in it needs to start at zero); calls that overlap on the
+ * GPU race on it, so the caller must serialise them. */
+#define DG_NOALLOC_MAX_TOKENS 256
+#define DG_NOALLOC_MAX_DMODEL 4096
+int dg_op_lm_head_noalloc(const float* d_x, const float* d_final_norm, const void* d_embed, int T, int d_model,
+                          int vocab, float norm_eps, float* d_stats, int32_t* d_argmax, int32_t* d_err,
+                          void* stream);
+
 #ifdef __cplusplus
 }
 #endif
