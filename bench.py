@@ -118,7 +118,7 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # algorithmic work
 # ---------------------------------------------------------------------------
-def expert_gate_up_bytes(cfg, n_touched: int, T: int) -> float:
+def expert_gate_up_bytes(cfg, n_touched: float, T: int) -> float:
     """Bytes one routed-expert gate|up launch must move: the gate and up
     weights of every expert some token is routed to, the grouped token rows
     read, the SwiGLU hidden rows written."""
@@ -127,7 +127,7 @@ def expert_gate_up_bytes(cfg, n_touched: int, T: int) -> float:
     return w + rows * cfg.d_model * 2 + rows * cfg.ffn_expert * 2
 
 
-def step_work(cfg, kv_len: int, T: int, n_touched: int):
+def step_work(cfg, kv_len: int, T: int, n_touched: float):
     """(bytes, flops) of one denoising step: every weight of the touched
     experts and all dense weights once, the KV prefix read, per-token FLOPs."""
     d, D = cfg.d_model, cfg.head_dim
@@ -357,12 +357,14 @@ def main():
 
     # kernel-class breakdown: one more profiled step (events on the library stream)
     h.profile(-1)
+    rs0 = h.debug_buffer("route_stats", torch.int64, (2,)).cpu().clone()
     h.profile(1)
     one_step(args.warmup + args.steps, record=False)
     h.profile(0)
     prof = h.profile_read()
-    counts = h.debug_buffer("counts", torch.int32, (cfg.n_experts,)).cpu()
-    n_touched = int((counts > 0).sum())
+    rs1 = h.debug_buffer("route_stats", torch.int64, (2,)).cpu()
+    # experts that received at least one token, averaged over every layer of the profiled step
+    n_touched = float((rs1[0] - rs0[0]) / max(1, int(rs1[1] - rs0[1])))
     T = cfg.canvas
     egu_ms, egu_n = prof["experts_gate_up"]
     egu_bytes = expert_gate_up_bytes(cfg, n_touched, T)
@@ -431,7 +433,7 @@ def main():
                      "avg_launch_ms": egu_avg_ms, "peak_source": f"{peak_kind} HBM copy (MEASURED_PEAKS.json)"},
         "step_roofline": {"bytes": sbytes, "flops": sflops, "bound": "hbm" if sbytes / hbm_gbs > sflops / bf16_tf / 1e3
                           else "tensor", "t_roof_ms": t_roof_ms, "frac": t_roof_ms / ms_denoise,
-                          "experts_touched_per_layer": n_touched},
+                          "experts_touched_per_layer": round(n_touched, 2)},
         "kernels": kernels,
         "cpu_baseline": cpu,
         "e2e": e2e,

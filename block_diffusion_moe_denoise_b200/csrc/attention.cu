@@ -1,229 +1,329 @@
-// Canvas attention: every canvas (or prefill segment) query attends, with no
-// mask, to all committed keys of its request and to every key of its own
-// segment (DiffusionGemma pages: bidirectional decoder pass over the canvas,
-// "What DiffusionGemma is"; every token sees every other token in its
-// context, "26B MoE Architecture, but Only 3.8B Activated").
+// Canvas attention on tcgen05: every canvas (or prefill segment) query
+// attends, with no mask, to all committed keys of its request and to every
+// key of its own segment (DiffusionGemma pages: bidirectional decoder pass
+// over the canvas, "What DiffusionGemma is"; every token sees every other
+// token in its context, "26B MoE Architecture, but Only 3.8B Activated").
 //
-// FlashAttention-style single pass with online softmax (exp2 domain), GQA:
-// the G = Hq/Hkv query heads of a KV head are stacked as G*Tr query rows so one
-// CTA's K/V tiles serve all of them.  64 query rows x 64-key tiles per CTA,
-// 4 warps x 16 rows, bf16 mma.sync m16n8k16 with fp32 accumulation, K/V tiles
-// double-buffered through cp.async into XOR-swizzled shared memory.  The key
-// range is split across CTAs (split-KV) when the query tiles alone cannot fill
-// the GPU; partial (O, max, sum) are merged by k_attn_combine.
+// One CTA = 128 query rows of one (request slot, KV head) -- the G = Hq/Hkv
+// query heads of a KV head are stacked as G*Tr rows so one K/V tile serves
+// them all -- over one range of keys (split-KV when the query tiles alone
+// cannot fill the GPU; partial (O, max, sum) are merged by k_attn_combine).
+//   warp 0     TMA producer: 64-key K tiles [64 x D] and V^T tiles [D x 64] in
+//              separate two-slot rings (the cache keeps V transposed so both
+//              MMAs read K-major operands); a K slot is refilled as soon as the
+//              S MMA that read it completes, a V slot once its PV MMA completes
+//   warp 1     MMA issuer: S = Q K^T into one of two TMEM buffers (N = 64),
+//              O += P V^T into TMEM (N = D); S(j+1) is issued before PV(j)
+//   warps 2-5  one query row per thread: Q row into shared memory, then per
+//              tile the exp2-domain online softmax on the S row read from TMEM,
+//              P row (bf16) written into the swizzled shared tile PV reads.
+//              The running max is only moved (and O, l rescaled in TMEM) when
+//              it grows by more than 2^8, so rescales are rare; O and l always
+//              share the same reference max, so the result is exact.
+// Every wait is bounded (mbar_wait_bounded).
 #include "common.cuh"
 #include "dg_internal.h"
 
 namespace dg {
 
-DG_DEVINL void cp_async16(uint32_t dst, const void* src, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0) : "memory");
-}
-DG_DEVINL void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-DG_DEVINL void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
+constexpr int kAQ = 128;        // query rows per CTA
+constexpr int kAK = 64;         // keys per tile
+constexpr int kAStages = 2;     // K/V ring depth
+constexpr float kRescaleLog2 = 8.0f;
 
-DG_DEVINL void ldsm_x4(uint32_t* r, uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-DG_DEVINL void ldsm_x4_t(uint32_t* r, uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-DG_DEVINL void mma_bf16_16816(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
+template <int D>
+struct AttnSmem {
+  static constexpr int kQ = kAQ * D * 2;            // Q: D/64 blocks of [128 x 128 B]
+  static constexpr int kK = kAK * D * 2;            // K tile: D/64 blocks of [64 x 128 B]
+  static constexpr int kV = D * kAK * 2;            // V^T tile: [D x 128 B]
+  static constexpr int kP = kAQ * kAK * 2;          // P tile: [128 x 128 B]
+  static constexpr size_t q_off = 0;
+  static constexpr size_t k_off = q_off + kQ;
+  static constexpr size_t v_off = k_off + (size_t)kAStages * kK;
+  static constexpr size_t p_off = v_off + (size_t)kAStages * kV;
+  static constexpr size_t bar_off = p_off + 2 * (size_t)kP;
+  static constexpr int kBars = 4 * kAStages + 9;
+  static constexpr size_t misc_off = bar_off + kBars * 8;
+  // at least 120 KB so two CTAs (each owning all 512 TMEM columns) never share an SM
+  static constexpr size_t total = misc_off + 16 + 1024 > 120 * 1024 ? misc_off + 16 + 1024 : 120 * 1024;
+};
+
+DG_DEVINL void tmem_st16(uint32_t taddr, const float* v) {
   asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-constexpr int kBQ = 64, kBK = 64;
-
-// byte offset of 16-byte chunk `ch` of row `r` in a [rows][D] bf16 tile whose
-// chunk index is XOR-swizzled with (r mod 8)
-template <int D>
-DG_DEVINL uint32_t swz(int r, int ch) {
-  return (uint32_t)(r * D * 2 + ((ch ^ (r & 7)) << 4));
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
+      "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+      "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
+      "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
+      "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])));
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 template <int D>
-__global__ void __launch_bounds__(128, 1) k_attn(const AttnArgs a) {
-  constexpr int CH = D / 8;  // 16-byte chunks per row
-  extern __shared__ __align__(128) uint8_t asmem[];
-  const uint32_t sQ = smem_u32(asmem);
-  const uint32_t sK0 = sQ + kBQ * D * 2;
-  const uint32_t sV0 = sK0 + 2 * kBK * D * 2;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+__global__ void __launch_bounds__(192, 1) k_attn_tc(const __grid_constant__ AttnArgs a) {
+  using S = AttnSmem<D>;
+  extern __shared__ uint8_t dyn_smem[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~(uintptr_t)1023);
+  uint8_t* sQ = base + S::q_off;
+  uint8_t* sK = base + S::k_off;
+  uint8_t* sV = base + S::v_off;
+  uint8_t* sP = base + S::p_off;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + S::bar_off);
+  uint64_t* k_full = bars;
+  uint64_t* k_empty = bars + kAStages;
+  uint64_t* v_full = bars + 2 * kAStages;
+  uint64_t* v_empty = bars + 3 * kAStages;
+  uint64_t* s_full = bars + 4 * kAStages;       // [2]
+  uint64_t* s_empty = s_full + 2;               // [2]
+  uint64_t* p_full = s_empty + 2;               // [2]
+  uint64_t* pv_done = p_full + 2;               // [2]
+  uint64_t* q_ready = pv_done + 2;              // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + S::misc_off);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(base + S::misc_off + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = a.Hq / a.Hkv;
   const int slot = blockIdx.y / a.Hkv, g = blockIdx.y % a.Hkv;
   const int rows = G * a.Tr;
-  const int r0 = blockIdx.x * kBQ;
+  const int r0 = blockIdx.x * kAQ;
   const int n_keys = a.n_keys[slot];
   int per = (n_keys + a.n_split - 1) / a.n_split;
-  per = (per + kBK - 1) / kBK * kBK;
+  per = (per + kAK - 1) / kAK * kAK;
   const int k_begin = blockIdx.z * per;
   const int k_end = min(n_keys, k_begin + per);
-  const int n_tiles = k_end > k_begin ? (k_end - k_begin + kBK - 1) / kBK : 0;
-  const bf16* Kg = a.kv + (size_t)a.req[slot] * a.req_stride + (size_t)g * a.cap * D;
-  const bf16* Vg = Kg + (size_t)a.Hkv * a.cap * D;
+  const int n_tiles = k_end > k_begin ? (k_end - k_begin + kAK - 1) / kAK : 0;
+  int* err = a.err;
 
-  // Q tile
-  for (int c = tid; c < kBQ * CH; c += 128) {
-    const int r = c / CH, ch = c % CH;
-    const int qr = r0 + r;
-    const bool ok = qr < rows;
-    const int h = g * G + (ok ? qr / a.Tr : 0);
-    const int t = slot * a.Tr + (ok ? qr % a.Tr : 0);
-    cp_async16(sQ + swz<D>(r, ch), a.q + ((size_t)h * a.q_T + t) * D + ch * 8, ok);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kAStages; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&s_empty[b], 128);
+      mbar_init(&p_full[b], 128);
+      mbar_init(&pv_done[b], 1);
+    }
+    mbar_init(q_ready, 128);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
   }
-  auto load_kv = [&](int it, int buf) {
-    const int key0 = k_begin + it * kBK;
-    const uint32_t sk = sK0 + buf * kBK * D * 2, sv = sV0 + buf * kBK * D * 2;
-    for (int c = tid; c < kBK * CH; c += 128) {
-      const int r = c / CH, ch = c % CH;
-      const int key = key0 + r;
-      const bool ok = key < k_end;
-      const size_t off = (size_t)(ok ? key : k_begin) * D + ch * 8;
-      cp_async16(sk + swz<D>(r, ch), Kg + off, ok);
-      cp_async16(sv + swz<D>(r, ch), Vg + off, ok);
-    }
-  };
-  if (n_tiles > 0) load_kv(0, 0);
-  cp_async_commit();
-
-  float o[D / 8][4];
-#pragma unroll
-  for (int j = 0; j < D / 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
-  float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
-  const float sl2 = a.scale * 1.4426950408889634f;
-
-  for (int it = 0; it < n_tiles; ++it) {
-    const int buf = it & 1;
-    if (it + 1 < n_tiles) {
-      load_kv(it + 1, buf ^ 1);
-      cp_async_commit();
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    const uint32_t sk = sK0 + buf * kBK * D * 2, sv = sV0 + buf * kBK * D * 2;
-
-    float s[8][4];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      uint32_t af[4];
-      {
-        const int r = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-        ldsm_x4(af, sQ + swz<D>(r, kk * 2 + (lane >> 4)));
-      }
-#pragma unroll
-      for (int np = 0; np < 4; ++np) {
-        uint32_t bf[4];
-        const int key = np * 16 + (lane & 7) + (lane >> 4) * 8;
-        ldsm_x4(bf, sk + swz<D>(key, kk * 2 + ((lane >> 3) & 1)));
-        mma_bf16_16816(s[2 * np], af, bf[0], bf[1]);
-        mma_bf16_16816(s[2 * np + 1], af, bf[2], bf[3]);
-      }
-    }
-    // online softmax (rows lane/4 and lane/4 + 8 of this warp's 16)
-    const int key0 = k_begin + it * kBK;
-    float mx_a = -INFINITY, mx_b = -INFINITY;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int key = key0 + j * 8 + (lane & 3) * 2 + (e & 1);
-        const float v = key < k_end ? s[j][e] * sl2 : -INFINITY;
-        s[j][e] = v;
-        if (e < 2) mx_a = fmaxf(mx_a, v);
-        else mx_b = fmaxf(mx_b, v);
-      }
-    }
-    mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 1));
-    mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 2));
-    mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 1));
-    mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 2));
-    const float mn_a = fmaxf(m_a, mx_a), mn_b = fmaxf(m_b, mx_b);
-    const float mu_a = mn_a == -INFINITY ? 0.f : mn_a, mu_b = mn_b == -INFINITY ? 0.f : mn_b;
-    const float al_a = exp2f(m_a - mu_a), al_b = exp2f(m_b - mu_b);
-    m_a = mn_a;
-    m_b = mn_b;
-    float rs_a = 0.f, rs_b = 0.f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      s[j][0] = exp2f(s[j][0] - mu_a);
-      s[j][1] = exp2f(s[j][1] - mu_a);
-      s[j][2] = exp2f(s[j][2] - mu_b);
-      s[j][3] = exp2f(s[j][3] - mu_b);
-      rs_a += s[j][0] + s[j][1];
-      rs_b += s[j][2] + s[j][3];
-    }
-    l_a = l_a * al_a + rs_a;
-    l_b = l_b * al_b + rs_b;
-#pragma unroll
-    for (int j = 0; j < D / 8; ++j) {
-      o[j][0] *= al_a;
-      o[j][1] *= al_a;
-      o[j][2] *= al_b;
-      o[j][3] *= al_b;
-    }
-    // O += P V
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      uint32_t pf[4];
-      pf[0] = pack_bf16x2(s[2 * kk][0], s[2 * kk][1]);
-      pf[1] = pack_bf16x2(s[2 * kk][2], s[2 * kk][3]);
-      pf[2] = pack_bf16x2(s[2 * kk + 1][0], s[2 * kk + 1][1]);
-      pf[3] = pack_bf16x2(s[2 * kk + 1][2], s[2 * kk + 1][3]);
-      const int key = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-#pragma unroll
-      for (int dp = 0; dp < D / 16; ++dp) {
-        uint32_t bf[4];
-        ldsm_x4_t(bf, sv + swz<D>(key, dp * 2 + (lane >> 4)));
-        mma_bf16_16816(o[2 * dp], pf, bf[0], bf[1]);
-        mma_bf16_16816(o[2 * dp + 1], pf, bf[2], bf[3]);
-      }
-    }
-    __syncthreads();
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&a.tm_k);
+    tma_prefetch_desc(&a.tm_vt);
   }
-  cp_async_wait<0>();
+  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;   // O: columns [0, D); S buffers at 256 and 320
+  const uint32_t tm_o = tmem, tm_s0 = tmem + 256;
 
-  l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
-  l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
-  l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
-  l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
+  // cache rows of this (request, layer, kv head) in the two tensor maps
+  const long long krow0 = a.k_row0 + (long long)a.req[slot] * a.req_rows_k + (long long)g * a.cap;
+  const long long vrow0 = a.v_row0 + (long long)a.req[slot] * a.req_rows_v + (long long)g * D;
 
+  if (warp == 0) {
+    if (lane == 0) {
+      // issue order K(0), K(1), then V(j), K(j+2) for j = 0, 1, ...: K(j+2)
+      // waits for S(j), V(j) for PV(j-2), matching the MMA issue order
+      auto load_k = [&](int j) -> bool {
+        const int st = j % kAStages;
+        if (!mbar_wait_bounded(&k_empty[st], ((j / kAStages) & 1) ^ 1, abort_flag, err)) return false;
+        mbar_arrive_expect_tx(&k_full[st], S::kK);
+        const uint32_t k_dst = smem_u32(sK + (size_t)st * S::kK);
+        const int key0 = k_begin + j * kAK;
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    const int qr = r0 + warp * 16 + (lane >> 2) + half * 8;
-    if (qr >= rows) continue;
-    const int h = g * G + qr / a.Tr;
-    const int t = slot * a.Tr + qr % a.Tr;
-    const float l = half ? l_b : l_a;
-    const float m = half ? m_b : m_a;
-    if (a.n_split == 1) {
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      uint32_t* dst = reinterpret_cast<uint32_t*>(a.o + (size_t)t * a.Hq * D + (size_t)h * D);
+        for (int kb = 0; kb < D / 64; ++kb)
+          tma_load_2d(k_dst + kb * (kAK * 128), &a.tm_k, kb * 64, (int)(krow0 + key0), &k_full[st]);
+        return true;
+      };
+      auto load_v = [&](int j) -> bool {
+        const int st = j % kAStages;
+        if (!mbar_wait_bounded(&v_empty[st], ((j / kAStages) & 1) ^ 1, abort_flag, err)) return false;
+        mbar_arrive_expect_tx(&v_full[st], S::kV);
+        tma_load_2d(smem_u32(sV + (size_t)st * S::kV), &a.tm_vt, k_begin + j * kAK, (int)vrow0, &v_full[st]);
+        return true;
+      };
+      bool ok = true;
+      for (int j = 0; ok && j < kAStages && j < n_tiles; ++j) ok = load_k(j);
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        ok = load_v(j);
+        if (ok && j + kAStages < n_tiles) ok = load_k(j + kAStages);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && n_tiles > 0) {
+      const uint32_t idesc_s = umma_idesc_bf16(128, kAK);
+      const uint32_t idesc_o = umma_idesc_bf16(128, D);
+      const uint32_t q0 = smem_u32(sQ), p0 = smem_u32(sP);
+      bool ok = mbar_wait_bounded(q_ready, 0, abort_flag, err);
+      // S(j) = Q K_j^T into S buffer j%2
+      auto issue_s = [&](int j) -> bool {
+        const int b = j & 1, stage = j % kAStages;
+        if (!mbar_wait_bounded(&s_empty[b], ((j >> 1) & 1) ^ 1, abort_flag, err)) return false;
+        if (!mbar_wait_bounded(&k_full[stage], (j / kAStages) & 1, abort_flag, err)) return false;
+        tc_fence_after();
+        const uint32_t k0 = smem_u32(sK + (size_t)stage * S::kK);
 #pragma unroll
-      for (int j = 0; j < D / 8; ++j)
-        dst[(j * 8 + (lane & 3) * 2) >> 1] = pack_bf16x2(o[j][2 * half] * inv, o[j][2 * half + 1] * inv);
-    } else {
-      const size_t row = ((size_t)blockIdx.z * a.Hq + h) * a.q_T + t;
-      float2* dst = reinterpret_cast<float2*>(a.part_o + row * D);
+        for (int kb = 0; kb < D / 64; ++kb)
 #pragma unroll
-      for (int j = 0; j < D / 8; ++j) dst[(j * 8 + (lane & 3) * 2) >> 1] = make_float2(o[j][2 * half], o[j][2 * half + 1]);
-      if ((lane & 3) == 0) a.part_ml[row] = make_float2(m, l);
+          for (int k = 0; k < 4; ++k)
+            umma_bf16(tm_s0 + b * kAK, umma_sdesc_k128(q0 + kb * (kAQ * 128) + 32 * k),
+                      umma_sdesc_k128(k0 + kb * (kAK * 128) + 32 * k), idesc_s, (kb | k) != 0 ? 1u : 0u);
+        umma_commit(&k_empty[stage]);
+        umma_commit(&s_full[b]);
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        if (j + 1 < n_tiles && !issue_s(j + 1)) break;
+        const int b = j & 1, stage = j % kAStages;
+        if (!mbar_wait_bounded(&v_full[stage], (j / kAStages) & 1, abort_flag, err)) break;
+        if (!mbar_wait_bounded(&p_full[b], (j >> 1) & 1, abort_flag, err)) break;
+        tc_fence_after();
+        const uint32_t v0 = smem_u32(sV + (size_t)stage * S::kV);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          umma_bf16(tm_o, umma_sdesc_k128(p0 + b * S::kP + 32 * k), umma_sdesc_k128(v0 + 32 * k), idesc_o,
+                    (j | k) != 0 ? 1u : 0u);
+        umma_commit(&v_empty[stage]);
+        umma_commit(&pv_done[b]);
+      }
+    }
+  } else {
+    // ---- softmax / epilogue warps: one query row per thread ----
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const int qr = r0 + row;
+    const bool valid = qr < rows;
+    const int h = g * G + (valid ? qr / a.Tr : 0);
+    const int t = slot * a.Tr + (valid ? qr % a.Tr : 0);
+    // Q row -> shared memory in the 128-byte-swizzled K-major layout
+    {
+      const uint4* src = reinterpret_cast<const uint4*>(a.q + ((size_t)h * a.q_T + t) * D);
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c) {
+        const uint4 v = valid ? src[c] : make_uint4(0, 0, 0, 0);
+        const int kb = c >> 3, ch = c & 7;
+        *reinterpret_cast<uint4*>(sQ + kb * (kAQ * 128) + row * 128 + ((ch ^ (row & 7)) << 4)) = v;
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(q_ready);
+    }
+    const float sl2 = a.scale * 1.4426950408889634f;
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_tiles && ok; ++j) {
+      const int b = j & 1;
+      if (!mbar_wait_bounded(&s_full[b], (j >> 1) & 1, abort_flag, err)) { ok = false; break; }
+      tc_fence_after();
+      float s[kAK];
+#pragma unroll
+      for (int c = 0; c < kAK; c += 16) tmem_ld16(tm_s0 + lane_off + b * kAK + c, s + c);
+      tc_fence_before();
+      mbar_arrive(&s_empty[b]);
+      const int key0 = k_begin + j * kAK;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kAK; ++c) {
+        s[c] = key0 + c < k_end ? s[c] * sl2 : -INFINITY;
+        mx = fmaxf(mx, s[c]);
+      }
+      const bool need = mx > m_used + kRescaleLog2;
+      const float m_new = need ? mx : m_used;
+      // P buffer b is free once PV(j-2) is done
+      if (j >= 2 && !mbar_wait_bounded(&pv_done[b], ((j - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
+      if (__any_sync(0xffffffffu, need) && j >= 1) {
+        // O holds PV(0..j-1): wait for PV(j-1), then rescale this warp's rows
+        if (!mbar_wait_bounded(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        tc_fence_after();
+        const float f = need ? exp2f(m_used - m_new) : 1.f;
+        for (int c = 0; c < D; c += 16) {
+          float o[16];
+          tmem_ld16(tm_o + lane_off + c, o);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) o[i] *= f;
+          tmem_st16(tm_o + lane_off + c, o);
+        }
+        l *= f;
+      }
+      m_used = m_new;
+      uint8_t* prow = sP + b * S::kP + row * 128;
+      float rs = 0.f;
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        float p[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          p[i] = exp2f(s[ch * 8 + i] - m_used);
+          rs += p[i];
+        }
+        uint4 v;
+        v.x = pack_bf16x2(p[0], p[1]);
+        v.y = pack_bf16x2(p[2], p[3]);
+        v.z = pack_bf16x2(p[4], p[5]);
+        v.w = pack_bf16x2(p[6], p[7]);
+        *reinterpret_cast<uint4*>(prow + ((ch ^ (row & 7)) << 4)) = v;
+      }
+      l += rs;
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&p_full[b]);
+    }
+    // final O
+    if (ok && n_tiles > 0 &&
+        mbar_wait_bounded(&pv_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, abort_flag, err)) {
+      tc_fence_after();
+      if (a.n_split == 1) {
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        uint4* dst = reinterpret_cast<uint4*>(a.o + (size_t)t * a.Hq * D + (size_t)h * D);
+        for (int c = 0; c < D; c += 16) {
+          float o[16];
+          tmem_ld16(tm_o + lane_off + c, o);
+          if (valid) {
+            uint4 u0, u1;
+            u0.x = pack_bf16x2(o[0] * inv, o[1] * inv);
+            u0.y = pack_bf16x2(o[2] * inv, o[3] * inv);
+            u0.z = pack_bf16x2(o[4] * inv, o[5] * inv);
+            u0.w = pack_bf16x2(o[6] * inv, o[7] * inv);
+            u1.x = pack_bf16x2(o[8] * inv, o[9] * inv);
+            u1.y = pack_bf16x2(o[10] * inv, o[11] * inv);
+            u1.z = pack_bf16x2(o[12] * inv, o[13] * inv);
+            u1.w = pack_bf16x2(o[14] * inv, o[15] * inv);
+            dst[c / 8] = u0;
+            dst[c / 8 + 1] = u1;
+          }
+        }
+      } else {
+        const size_t prow_i = ((size_t)blockIdx.z * a.Hq + h) * a.q_T + t;
+        float4* dst = reinterpret_cast<float4*>(a.part_o + prow_i * D);
+        for (int c = 0; c < D; c += 16) {
+          float o[16];
+          tmem_ld16(tm_o + lane_off + c, o);
+          if (valid)
+#pragma unroll
+            for (int i = 0; i < 16; i += 4) dst[(c + i) / 4] = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
+        }
+        if (valid) a.part_ml[prow_i] = make_float2(m_used, l);
+      }
+    } else if (n_tiles == 0 && a.n_split > 1 && valid) {
+      const size_t prow_i = ((size_t)blockIdx.z * a.Hq + h) * a.q_T + t;
+      a.part_ml[prow_i] = make_float2(-INFINITY, 0.f);
     }
   }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
 // Merge of the split-KV partials: O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s.
@@ -262,22 +362,30 @@ int attention_split_cap() { return 16; }
 
 template <int D>
 static cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st) {
-  const size_t smem = (size_t)(kBQ + 4 * kBK) * D * 2;
+  const size_t smem = AttnSmem<D>::total;
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(k_attn<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(k_attn_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     configured = true;
   }
   const int G = a.Hq / a.Hkv;
-  dim3 grid((G * a.Tr + kBQ - 1) / kBQ, a.Hkv * a.n_slots, a.n_split);
-  k_attn<D><<<grid, 128, smem, st>>>(a);
+  dim3 grid((G * a.Tr + kAQ - 1) / kAQ, a.Hkv * a.n_slots, a.n_split);
+  k_attn_tc<D><<<grid, 192, smem, st>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || a.n_split == 1) return e;
   const int T = a.n_slots * a.Tr;
   const int warps = T * a.Hq;
   k_attn_combine<<<(warps + 7) / 8, 256, 0, st>>>(a.part_o, a.part_ml, a.n_split, a.Hq, a.q_T, T, D, a.o);
   return cudaGetLastError();
+}
+
+size_t attention_smem_bytes(int D) {
+  switch (D) {
+    case 64: return AttnSmem<64>::total;
+    case 128: return AttnSmem<128>::total;
+    default: return AttnSmem<256>::total;
+  }
 }
 
 cudaError_t run_attention(const AttnArgs& a, cudaStream_t st) {

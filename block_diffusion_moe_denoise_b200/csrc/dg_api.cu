@@ -48,7 +48,8 @@ bool config_ok(const dg_config* c) {
   if (c->n_layers < 1 || c->d_model < 256 || c->d_model % 256 != 0) return false;
   if (!(c->head_dim == 64 || c->head_dim == 128 || c->head_dim == 256)) return false;
   if (c->n_kv_heads < 1 || c->n_q_heads < 1 || c->n_q_heads % c->n_kv_heads != 0) return false;
-  if (((c->n_q_heads + 2 * c->n_kv_heads) * c->head_dim) % 256 != 0) return false;
+  if ((c->n_q_heads * c->head_dim) % 128 != 0 || (c->n_kv_heads * c->head_dim) % 128 != 0) return false;
+  if (c->ffn_shared % 32 != 0) return false;
   if ((c->n_q_heads * c->head_dim) % 64 != 0) return false;
   if (c->n_experts < 1 || c->n_experts > 256 || c->top_k < 1 || c->top_k > 8 || c->top_k > c->n_experts) return false;
   if (c->ffn_expert < 64 || c->ffn_expert % 64 != 0 || c->ffn_shared < 64 || c->ffn_shared % 64 != 0) return false;
@@ -58,7 +59,10 @@ bool config_ok(const dg_config* c) {
   return true;
 }
 
-void make_plan(const dg_config* c, int max_req, long long cap, Plan* p) {
+long long round_cap(long long cap) { return (cap + 63) / 64 * 64; }
+
+void make_plan(const dg_config* c, int max_req, long long cap_user, Plan* p) {
+  const long long cap = round_cap(cap_user);
   const int T = max_req * c->canvas;
   const int Tcap = (T + 127) / 128 * 128;
   const long long rows = (long long)T * c->top_k;
@@ -80,6 +84,7 @@ void make_plan(const dg_config* c, int max_req, long long cap, Plan* p) {
   p->add("row_weight", (size_t)rows * 4);
   p->add("row_pair", (size_t)rows * 4);
   p->add("tile_counts", 64);
+  p->add("route_stats", 64);
   p->add("egu_tiles", (size_t)n_nt * (c->ffn_expert / 64) * 16);
   p->add("ed_tiles", (size_t)n_nt * (d / 128) * 16);
   p->add("xp", (size_t)rows * d * 2);
@@ -97,7 +102,9 @@ void make_plan(const dg_config* c, int max_req, long long cap, Plan* p) {
   p->add("tok_pos", (size_t)Tcap * 4);
   p->add("tok_req", (size_t)Tcap * 4);
   p->add("inv_freq", (size_t)D / 2 * 8);
-  p->add("prompt", (size_t)cap * 4);
+  p->add("rope", (size_t)Tcap * (D / 2) * 8);
+  p->add("router_logits", (size_t)Tcap * c->n_experts * 4);
+  p->add("prompt", (size_t)cap_user * 4);
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -195,7 +202,8 @@ struct dg_handle {
   int egu_cap = 0, ed_cap = 0;
   long long kv_req_stride = 0, kv_layer_stride = 0;
   std::vector<LayerMaps> maps;
-  CUtensorMap tm_hn, tm_o, tm_u, tm_xp, tm_hp, tm_hs, tm_embed;
+  CUtensorMap tm_hn, tm_o, tm_u, tm_xp, tm_hp, tm_hs, tm_embed, tm_k, tm_vt;
+  long long cap_user = 0;  // capacity the caller asked for (cap is rounded up to 64)
   ReqState req[DG_MAX_REQUESTS];
 
   template <class T>
@@ -242,12 +250,20 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
   int* err = h->B<int>("err");
   float* x = h->B<float>("x");
   bf16* hn = h->B<bf16>("hn");
-  LAUNCH(h, K_EMBED, 1, run_embed(ids, s, h->embed, c.vocab, d, x, h->B<int>("tok_pos"), h->B<int>("tok_req"), err, st));
+  LAUNCH(h, K_EMBED, 1,
+         run_embed(ids, s, h->embed, c.vocab, d, x, h->B<int>("tok_pos"), h->B<int>("tok_req"),
+                   h->B<double>("inv_freq"), D / 2, h->B<float2>("rope"), err, st));
+  // the routed outputs of layer l are summed into x by the norm kernel of layer l+1
+  float* yp = h->B<float>("yp");
+  const int* pair_row = h->B<int>("pair_row");
+  int pending_k = 0;
   for (int l = 0; l < n_layers; ++l) {
     const dg_layer_weights& w = h->lw[l];
     const LayerMaps& m = h->maps[l];
     bf16* kv_l = h->B<bf16>("kv") + (size_t)l * h->kv_layer_stride;
-    LAUNCH(h, K_RMSNORM, 1, run_rmsnorm(x, (const float*)w.attn_norm, T, d, c.norm_eps, hn, st));
+    LAUNCH(h, K_RMSNORM, 1,
+           run_combine_rmsnorm(x, yp, pair_row, pending_k, (const float*)w.attn_norm, T, d, c.norm_eps, hn, st));
+    pending_k = 0;
     QkvArgs qa;
     qa.tm_x = &h->tm_hn;
     qa.tm_w = &m.qkv;
@@ -263,7 +279,7 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     qa.kv_req_stride = h->kv_req_stride;
     qa.tok_pos = h->B<int>("tok_pos");
     qa.tok_req = h->B<int>("tok_req");
-    qa.inv_freq = h->B<double>("inv_freq");
+    qa.rope = h->B<float2>("rope");
     qa.q = h->B<bf16>("q");
     qa.kv = kv_l;
     qa.err = err;
@@ -271,11 +287,15 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     if (qkv_only_last && l == c.n_layers - 1) break;
 
     AttnArgs aa;
+    aa.tm_k = h->tm_k;
+    aa.tm_vt = h->tm_vt;
     aa.q = h->B<bf16>("q");
     aa.q_T = h->Tcap;
     aa.o = h->B<bf16>("o");
-    aa.kv = kv_l;
-    aa.req_stride = h->kv_req_stride;
+    aa.k_row0 = (long long)l * 2 * c.n_kv_heads * h->cap;
+    aa.req_rows_k = (long long)c.n_layers * 2 * c.n_kv_heads * h->cap;
+    aa.v_row0 = (long long)l * 2 * c.n_kv_heads * D + (long long)c.n_kv_heads * D;
+    aa.req_rows_v = (long long)c.n_layers * 2 * c.n_kv_heads * D;
     aa.cap = h->cap;
     aa.Hq = c.n_q_heads;
     aa.Hkv = c.n_kv_heads;
@@ -289,8 +309,8 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
       if (aa.n_keys[i] > max_keys) max_keys = aa.n_keys[i];
     }
     const int G = c.n_q_heads / c.n_kv_heads;
-    const int base_ctas = ((G * s.Tr + 63) / 64) * c.n_kv_heads * s.n;
-    int split = (h->num_sms + base_ctas - 1) / base_ctas;
+    const int base_ctas = ((G * s.Tr + 127) / 128) * c.n_kv_heads * s.n;
+    int split = h->num_sms / base_ctas;
     const int max_by_keys = max_keys / 256 > 0 ? max_keys / 256 : 1;
     if (split > max_by_keys) split = max_by_keys;
     if (split > kSplitCap) split = kSplitCap;
@@ -299,6 +319,7 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     aa.part_o = h->B<float>("attn_o");
     aa.part_ml = h->B<float2>("attn_ml");
     aa.scale = 1.0f / sqrtf((float)D);
+    aa.err = err;
     LAUNCH(h, K_ATTN, aa.n_split > 1 ? 2 : 1, run_attention(aa, st));
 
     OprojArgs oa;
@@ -312,9 +333,9 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     oa.err = err;
     LAUNCH(h, K_OPROJ, 1, run_oproj(oa, st));
 
-    LAUNCH(h, K_ROUTER, 1,
+    LAUNCH(h, K_ROUTER, 2,
            run_router(x, (const float*)w.ffn_norm, c.norm_eps, (const bf16*)w.w_router, T, d, c.n_experts, k,
-                      h->B<bf16>("u"), h->B<int>("idx"), h->B<float>("w"), err, st));
+                      h->B<bf16>("u"), h->B<float>("router_logits"), h->B<int>("idx"), h->B<float>("w"), st));
     GroupArgs ga;
     ga.idx = h->B<int>("idx");
     ga.w = h->B<float>("w");
@@ -335,6 +356,7 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     ga.egu_count = h->B<int>("tile_counts");
     ga.ed_tiles = h->B<int4>("ed_tiles");
     ga.ed_count = h->B<int>("tile_counts") + 1;
+    ga.route_stats = h->B<unsigned long long>("route_stats");
     ga.err = err;
     LAUNCH(h, K_GROUP, 1, run_group(ga, st));
     LAUNCH(h, K_GATHER, 1, run_gather(h->B<bf16>("u"), h->B<int>("row_token"), T * k, d, h->B<bf16>("xp"), st));
@@ -370,18 +392,17 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     sa.T = T;
     sa.d = d;
     sa.fs = c.ffn_shared;
-    sa.k = k;
     sa.num_sms = h->num_sms;
     sa.hs = h->B<bf16>("hs");
     sa.x = x;
-    sa.yp = h->B<float>("yp");
-    sa.pair_row = h->B<int>("pair_row");
     sa.err = err;
     LAUNCH(h, K_SGU, 1, run_shared_gate_up(sa, st));
     LAUNCH(h, K_SD, 1, run_shared_down(sa, st));
+    pending_k = k;
   }
   if (want_lm) {
-    LAUNCH(h, K_RMSNORM, 1, run_rmsnorm(x, h->final_norm, T, d, c.norm_eps, hn, st));
+    LAUNCH(h, K_RMSNORM, 1,
+           run_combine_rmsnorm(x, yp, pair_row, pending_k, h->final_norm, T, d, c.norm_eps, hn, st));
     LmArgs la;
     la.tm_x = &h->tm_hn;
     la.tm_embed = &h->tm_embed;
@@ -397,6 +418,9 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     LAUNCH(h, K_LMC, 1,
            run_lm_combine(h->B<float4>("lm_part"), grid, (T + 127) / 128, T, h->B<float>("stats"),
                           h->B<int>("argmax"), err, st));
+  } else if (pending_k) {
+    // a pass stopped after a full layer: fold its routed outputs into x
+    LAUNCH(h, K_RMSNORM, 1, run_combine_rmsnorm(x, yp, pair_row, pending_k, nullptr, T, d, c.norm_eps, nullptr, st));
   }
   return DG_OK;
 }
@@ -440,12 +464,15 @@ int dg_init(const dg_config* cfg, const dg_weights* wts, int max_requests, int64
   cudaDeviceProp prop;
   if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return DG_E_CUDA;
   if (prop.major != 10) return DG_E_UNSUPPORTED;
-  if ((size_t)prop.sharedMemPerBlockOptin < gemm_smem_bytes_max()) return DG_E_UNSUPPORTED;
+  if ((size_t)prop.sharedMemPerBlockOptin < gemm_smem_bytes_max() ||
+      (size_t)prop.sharedMemPerBlockOptin < attention_smem_bytes(cfg->head_dim))
+    return DG_E_UNSUPPORTED;
 
   dg_handle* h = new dg_handle();
   h->cfg = *cfg;
   h->max_req = max_requests;
-  h->cap = kv_capacity;
+  h->cap = round_cap(kv_capacity);
+  h->cap_user = kv_capacity;
   h->st = static_cast<cudaStream_t>(stream);
   h->num_sms = prop.multiProcessorCount;
   h->T_max = max_requests * cfg->canvas;
@@ -461,7 +488,7 @@ int dg_init(const dg_config* cfg, const dg_weights* wts, int max_requests, int64
   h->ws = static_cast<uint8_t*>(workspace);
   const dg_config& c = h->cfg;
   const int d = c.d_model, D = c.head_dim;
-  h->kv_layer_stride = 2ll * c.n_kv_heads * kv_capacity * D;
+  h->kv_layer_stride = 2ll * c.n_kv_heads * h->cap * D;
   h->kv_req_stride = h->kv_layer_stride * c.n_layers;
   const long long rows = (long long)h->T_max * c.top_k;
   const long long n_nt = c.n_experts + (rows + 63) / 64;
@@ -476,22 +503,27 @@ int dg_init(const dg_config* cfg, const dg_weights* wts, int max_requests, int64
     const dg_layer_weights& w = h->lw[l];
     LayerMaps& m = h->maps[l];
     ok = ok && w.attn_norm && w.ffn_norm && w.w_router;
-    ok = ok && make_map(&m.qkv, w.w_qkv, d, qkv_rows, 256);
+    ok = ok && make_map(&m.qkv, w.w_qkv, d, qkv_rows, 64);
     ok = ok && make_map(&m.o, w.w_o, (long long)c.n_q_heads * D, d, 128);
     ok = ok && make_map(&m.gate, w.w_gate, d, E * c.ffn_expert, 64);
     ok = ok && make_map(&m.up, w.w_up, d, E * c.ffn_expert, 64);
     ok = ok && make_map(&m.down, w.w_down, c.ffn_expert, E * d, 128);
-    ok = ok && make_map(&m.sgate, w.ws_gate, d, c.ffn_shared, 64);
-    ok = ok && make_map(&m.sup, w.ws_up, d, c.ffn_shared, 64);
+    ok = ok && make_map(&m.sgate, w.ws_gate, d, c.ffn_shared, 32);
+    ok = ok && make_map(&m.sup, w.ws_up, d, c.ffn_shared, 32);
     ok = ok && make_map(&m.sdown, w.ws_down, c.ffn_shared, d, 128);
   }
   ok = ok && make_map(&h->tm_hn, h->B<bf16>("hn"), d, h->Tcap, 128);
-  ok = ok && make_map(&h->tm_o, h->B<bf16>("o"), (long long)c.n_q_heads * D, h->Tcap, 128);
+  ok = ok && make_map(&h->tm_o, h->B<bf16>("o"), (long long)c.n_q_heads * D, h->Tcap, 64);
   ok = ok && make_map(&h->tm_u, h->B<bf16>("u"), d, h->Tcap, 128);
   ok = ok && make_map(&h->tm_xp, h->B<bf16>("xp"), d, rows, 64);
   ok = ok && make_map(&h->tm_hp, h->B<bf16>("hp"), c.ffn_expert, rows, 64);
-  ok = ok && make_map(&h->tm_hs, h->B<bf16>("hs"), c.ffn_shared, h->Tcap, 128);
+  ok = ok && make_map(&h->tm_hs, h->B<bf16>("hs"), c.ffn_shared, h->Tcap, 64);
   ok = ok && make_map(&h->tm_embed, h->embed, d, c.vocab, 256);
+  {
+    const long long kv_elems = (long long)max_requests * h->kv_req_stride;
+    ok = ok && make_map(&h->tm_k, h->B<bf16>("kv"), D, kv_elems / D, 64);
+    ok = ok && make_map(&h->tm_vt, h->B<bf16>("kv"), h->cap, kv_elems / h->cap, D);
+  }
   if (!ok) {
     delete h;
     return DG_E_ARG;
@@ -502,6 +534,8 @@ int dg_init(const dg_config* cfg, const dg_weights* wts, int max_requests, int64
   if (cudaMemcpyAsync(h->B<double>("inv_freq"), inv.data(), inv.size() * 8, cudaMemcpyHostToDevice, h->st) !=
           cudaSuccess ||
       cudaMemsetAsync(h->B<int>("err"), 0, 64, h->st) != cudaSuccess ||
+      cudaMemsetAsync(h->B<int>("route_stats"), 0, 64, h->st) != cudaSuccess ||
+      cudaMemsetAsync(h->B<bf16>("kv"), 0, h->plan.buf.at("kv").second, h->st) != cudaSuccess ||
       cudaMemsetAsync(h->B<int>("remaining"), 0, (size_t)max_requests * 4, h->st) != cudaSuccess ||
       cudaStreamSynchronize(h->st) != cudaSuccess) {
     delete h;
@@ -517,7 +551,7 @@ int64_t dg_kv_len(const dg_handle* h, int req) { return req_ok(h, req) ? h->req[
 
 int dg_set_kv(dg_handle* h, int req, int layer, int64_t pos0, int64_t n, const void* d_k, const void* d_v) {
   if (!req_ok(h, req) || layer < 0 || layer >= h->cfg.n_layers || pos0 < 0 || n < 0 || !d_k || !d_v) return DG_E_ARG;
-  if (pos0 + n > h->cap) return DG_E_CAPACITY;
+  if (pos0 + n > h->cap_user) return DG_E_CAPACITY;
   bf16* ck = h->B<bf16>("kv") + req * h->kv_req_stride + layer * h->kv_layer_stride;
   bf16* cv = ck + (size_t)h->cfg.n_kv_heads * h->cap * h->cfg.head_dim;
   CK(run_kv_copy(ck, cv, h->cfg.n_kv_heads, h->cap, h->cfg.head_dim, pos0, n, (const bf16*)d_k, (const bf16*)d_v,
@@ -527,7 +561,7 @@ int dg_set_kv(dg_handle* h, int req, int layer, int64_t pos0, int64_t n, const v
 
 int dg_get_kv(dg_handle* h, int req, int layer, int64_t pos0, int64_t n, void* d_k, void* d_v) {
   if (!req_ok(h, req) || layer < 0 || layer >= h->cfg.n_layers || pos0 < 0 || n < 0 || !d_k || !d_v) return DG_E_ARG;
-  if (pos0 + n > h->cap) return DG_E_CAPACITY;
+  if (pos0 + n > h->cap_user) return DG_E_CAPACITY;
   bf16* ck = h->B<bf16>("kv") + req * h->kv_req_stride + layer * h->kv_layer_stride;
   bf16* cv = ck + (size_t)h->cfg.n_kv_heads * h->cap * h->cfg.head_dim;
   CK(run_kv_copy(ck, cv, h->cfg.n_kv_heads, h->cap, h->cfg.head_dim, pos0, n, nullptr, nullptr, (bf16*)d_k,
@@ -538,7 +572,7 @@ int dg_get_kv(dg_handle* h, int req, int layer, int64_t pos0, int64_t n, void* d
 int dg_set_kv_len(dg_handle* h, int req, int64_t len) {
   if (!req_ok(h, req) || len < 0) return DG_E_ARG;
   if (h->req[req].open) return DG_E_STATE;
-  if (len > h->cap) return DG_E_CAPACITY;
+  if (len > h->cap_user) return DG_E_CAPACITY;
   h->req[req].kv_len = len;
   return DG_OK;
 }
@@ -547,7 +581,7 @@ int dg_prefill(dg_handle* h, int req, const int32_t* d_tokens, int n) {
   if (!req_ok(h, req) || n < 0 || (n > 0 && !d_tokens)) return DG_E_ARG;
   ReqState& r = h->req[req];
   if (r.open) return DG_E_STATE;
-  if (r.kv_len + n > h->cap) return DG_E_CAPACITY;
+  if (r.kv_len + n > h->cap_user) return DG_E_CAPACITY;
   const int seg = h->cfg.canvas;
   for (int s0 = 0; s0 < n; s0 += seg) {
     const int len = n - s0 < seg ? n - s0 : seg;
@@ -568,7 +602,7 @@ int dg_prefill(dg_handle* h, int req, const int32_t* d_tokens, int n) {
 int dg_open_canvas(dg_handle* h, int req, uint64_t seed, int block) {
   if (!req_ok(h, req) || block < 0) return DG_E_ARG;
   ReqState& r = h->req[req];
-  if (r.kv_len + h->cfg.canvas > h->cap) return DG_E_CAPACITY;
+  if (r.kv_len + h->cfg.canvas > h->cap_user) return DG_E_CAPACITY;
   const int C = h->cfg.canvas;
   LAUNCH(h, K_OTHER, 1,
          run_philox_tokens(seed, block, 0, req, 0, C, h->cfg.vocab, h->B<int>("canvas") + (size_t)req * C,
@@ -691,7 +725,7 @@ int dg_generate(dg_handle* h, int req, const int32_t* h_prompt, int n_prompt, in
   if (n_out % C != 0) return DG_E_ARG;
   ReqState& r = h->req[req];
   if (r.open || r.kv_len != 0) return DG_E_STATE;
-  if ((long long)n_prompt + n_out > h->cap) return DG_E_CAPACITY;
+  if ((long long)n_prompt + n_out > h->cap_user) return DG_E_CAPACITY;
   int* prompt = h->B<int>("prompt");
   if (n_prompt > 0) CK(cudaMemcpyAsync(prompt, h_prompt, (size_t)n_prompt * 4, cudaMemcpyHostToDevice, h->st));
   int rc = dg_prefill(h, req, prompt, n_prompt);
@@ -791,6 +825,7 @@ int dg_op_route_group(dg_handle* h, const int32_t* d_idx, const float* d_w, int 
   ga.egu_count = h->B<int>("tile_counts");
   ga.ed_tiles = h->B<int4>("ed_tiles");
   ga.ed_count = h->B<int>("tile_counts") + 1;
+  ga.route_stats = nullptr;
   ga.err = h->B<int>("err");
   CK(run_group(ga, h->st));
   if (d_counts)
@@ -840,7 +875,7 @@ int dg_debug_forward(dg_handle* h, int req, const int32_t* d_tokens, int T, int 
   if (!req_ok(h, req) || !d_tokens || T < 1 || T > h->cfg.canvas || n_layers < 1 || n_layers > h->cfg.n_layers)
     return DG_E_ARG;
   const ReqState& r = h->req[req];
-  if (r.kv_len + T > h->cap) return DG_E_CAPACITY;
+  if (r.kv_len + T > h->cap_user) return DG_E_CAPACITY;
   SlotInfo s;
   memset(&s, 0, sizeof(s));
   s.n = 1;

@@ -23,7 +23,7 @@ struct QkvArgs {
   long long kv_req_stride;
   const int* tok_pos;
   const int* tok_req;
-  const double* inv_freq;
+  const float2* rope;  // [T][D/2] (cos, sin)
   bf16* q;
   bf16* kv;
   int* err;
@@ -51,11 +51,9 @@ struct ExpertArgs {
 };
 struct SharedArgs {
   const CUtensorMap *tm_u, *tm_gate, *tm_up, *tm_down, *tm_hs;
-  int T, d, fs, k, num_sms;
+  int T, d, fs, num_sms;
   bf16* hs;
   float* x;
-  const float* yp;
-  const int* pair_row;
   int* err;
 };
 struct LmArgs {
@@ -87,10 +85,12 @@ struct SlotInfo {
 
 // ids[slot] points at the slot's Tr token ids
 cudaError_t run_embed(const int* const* ids, const SlotInfo& s, const bf16* embed, int V, int d, float* x, int* tok_pos,
-                      int* tok_req, int* err, cudaStream_t st);
+                      int* tok_req, const double* inv_freq, int half, float2* rope, int* err, cudaStream_t st);
+cudaError_t run_combine_rmsnorm(float* x, const float* yp, const int* pair_row, int k, const float* g, int T, int d,
+                                float eps, bf16* out, cudaStream_t st);
 cudaError_t run_rmsnorm(const float* x, const float* g, int T, int d, float eps, bf16* out, cudaStream_t st);
 cudaError_t run_router(const float* x, const float* g, float eps, const bf16* wr, int T, int d, int E, int k,
-                       bf16* u, int* idx, float* w, int* err, cudaStream_t st);
+                       bf16* u, float* logits, int* idx, float* w, cudaStream_t st);
 cudaError_t run_topk(const float* logits, int T, int E, int k, int* idx, float* w, cudaStream_t st);
 struct GroupArgs {
   const int* idx;
@@ -106,6 +106,7 @@ struct GroupArgs {
   int* egu_count;
   int4* ed_tiles;
   int* ed_count;
+  unsigned long long* route_stats;  // [0] += experts touched, [1] += launches (may be null)
   int* err;
 };
 cudaError_t run_group(const GroupArgs& a, cudaStream_t st);
@@ -136,11 +137,13 @@ cudaError_t run_kv_copy(bf16* cache_k, bf16* cache_v, int Hkv, long long cap, in
 
 // ---- attention (attention.cu) ----
 struct AttnArgs {
-  const bf16* q;     // [Hq][q_T][D]
+  CUtensorMap tm_k;   // whole KV area as rows of D elements, 64 x 64 boxes
+  CUtensorMap tm_vt;  // whole KV area as rows of cap elements, 64 x D boxes
+  const bf16* q;      // [Hq][q_T][D]
   int q_T;
-  bf16* o;           // [T][Hq*D]
-  const bf16* kv;    // this layer's K block of request 0
-  long long req_stride;
+  bf16* o;            // [T][Hq*D]
+  long long k_row0, req_rows_k;   // tm_k row of (request 0, this layer, head 0, pos 0); rows per request
+  long long v_row0, req_rows_v;   // tm_vt row of (request 0, this layer, head 0, dim 0); rows per request
   long long cap;
   int Hq, Hkv, D, Tr, n_slots;
   int req[DG_MAX_REQUESTS];
@@ -149,8 +152,10 @@ struct AttnArgs {
   float* part_o;     // [n_split][Hq][q_T][D]
   float2* part_ml;   // [n_split][Hq][q_T]
   float scale;
+  int* err;
 };
 cudaError_t run_attention(const AttnArgs& a, cudaStream_t st);
 int attention_split_cap();
+size_t attention_smem_bytes(int D);
 
 }  // namespace dg

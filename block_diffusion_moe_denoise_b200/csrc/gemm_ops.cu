@@ -7,7 +7,8 @@
 //           epilogue (weights as the 128-row operand, the expert's tokens as N)
 //   ed      routed experts, down projection scaled by the pair's routing weight
 //   sgu     shared expert gate|up + SwiGLU (tokens as the 128-row operand)
-//   sd      shared expert down + sum of the token's routed outputs + residual
+//   sd      shared expert down + residual (the routed outputs are summed into the
+//           residual by the next combine + RMSNorm kernel)
 //   lm      tied LM head with per-row online max / argmax / sum e^(z-m) /
 //           sum e^(z-m)(z-m) so the logits are never written
 // Structure of a decoder layer and the MoE: DiffusionGemma pages ("26B MoE
@@ -33,22 +34,54 @@ DG_DEVINL void store_bf16x16(__nv_bfloat16* dst, const float* v) {
 }
 
 // ---------------------------------------------------------------------------
-// QKV projection + RoPE + KV-cache write
+// QKV projection + RoPE + KV-cache write.  Tile (token tile a, 128-column tile
+// b).  The 128 W_qkv rows of a q/k tile are two 64-row boxes chosen so every
+// rotate-half pair (i, i + D/2) lands in columns (c, c + 64) of the same
+// accumulator row (head_dim 128/256), or inside one 64-column head at distance
+// 32 (head_dim 64): the rotation stays in one thread.  cos/sin come from the
+// per-pass table the embedding kernel writes.
 // ---------------------------------------------------------------------------
 struct P_QKV : ProblemBase {
-  static constexpr int BN = 256, STAGES = 4, B_STAGE = BN * 128, TMEM_COLS = 512;
+  static constexpr int BN = 128, STAGES = 6, B_STAGE = BN * 128, TMEM_COLS = 256;
   struct Params {
     CUtensorMap tmA;  // normed tokens [Tcap, d]
-    CUtensorMap tmB;  // w_qkv [(Hq+2Hkv)*D, d]
+    CUtensorMap tmB;  // w_qkv [(Hq+2Hkv)*D, d], 64-row boxes
     int T, nk, MT, NT, D, Hq, Hkv, q_T, kv_cap;
     long long kv_req_stride;
     const int* tok_pos;
     const int* tok_req;
-    const double* inv_freq;  // [D/2]
+    const float2* rope;  // [T][D/2] (cos, sin)
     __nv_bfloat16* q;
-    __nv_bfloat16* kv;  // this layer's K block of request 0; V follows after Hkv*cap*D
+    __nv_bfloat16* kv;  // this layer's K block [Hkv][cap][D] of request 0; V^T [Hkv][D][cap] follows
     int* err;
   };
+  // region (0 q, 1 k, 2 v), index of the tile inside its region, and the first
+  // W_qkv row of each 64-row box
+  DG_DEVINL static void rows_of(const Params& p, int b, int& kind, int& tb, int& r0, int& r1) {
+    const int D = p.D;
+    const int nq = p.Hq * D / 128, nkv = p.Hkv * D / 128;
+    int base;
+    if (b < nq) {
+      kind = 0;
+      tb = b;
+      base = 0;
+    } else if (b < nq + nkv) {
+      kind = 1;
+      tb = b - nq;
+      base = p.Hq * D;
+    } else {
+      kind = 2;
+      tb = b - nq - nkv;
+      base = (p.Hq + p.Hkv) * D;
+    }
+    if (kind != 2 && D == 256) {
+      r0 = base + (tb >> 1) * 256 + (tb & 1) * 64;
+      r1 = r0 + 128;
+    } else {
+      r0 = base + tb * 128;
+      r1 = r0 + 64;
+    }
+  }
   DG_DEVINL static void prefetch(const Params& p) {
     tma_prefetch_desc(&p.tmA);
     tma_prefetch_desc(&p.tmB);
@@ -60,13 +93,24 @@ struct P_QKV : ProblemBase {
     t.nk = p.nk;
     t.n_mma = BN;
     t.a = v % p.MT;  // token tile
-    t.b = v / p.MT;  // 256-row block of W_qkv
+    t.b = v / p.MT;  // 128-column tile of W_qkv
     return t;
   }
   DG_DEVINL static uint32_t tx_bytes(const Params&, const Tile&) { return kAStage + B_STAGE; }
   DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
+    int kind, tb, r0, r1;
+    rows_of(p, t.b, kind, tb, r0, r1);
     tma_load_2d(sa, &p.tmA, kb * 64, t.a * 128, bar);
-    tma_load_2d(sb, &p.tmB, kb * 64, t.b * 256, bar);
+    tma_load_2d(sb, &p.tmB, kb * 64, r0, bar);
+    tma_load_2d(sb + 64 * 128, &p.tmB, kb * 64, r1, bar);
+  }
+  DG_DEVINL static void rotate16(const float* x1, const float* x2, const float2* cs, float* y1, float* y2) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float2 r = cs[i];
+      y1[i] = x1[i] * r.x - x2[i] * r.y;
+      y2[i] = x2[i] * r.x + x1[i] * r.y;
+    }
   }
   DG_DEVINL static void epilogue(const Params& p, const Tile& t, uint32_t taddr, int, int, int row, uint8_t*) {
     const int tok = t.a * 128 + row;
@@ -74,66 +118,87 @@ struct P_QKV : ProblemBase {
     const int pos = ok ? p.tok_pos[tok] : 0;
     const int req = ok ? p.tok_req[tok] : 0;
     const int D = p.D, half = D >> 1;
-    for (int hh = 0; hh < 256 / D; ++hh) {
-      const int r0 = t.b * 256 + hh * D;
-      const uint32_t col0 = (uint32_t)(hh * D);
-      int kind, head;
-      if (r0 < p.Hq * D) {
-        kind = 0;
-        head = r0 / D;
-      } else if (r0 < (p.Hq + p.Hkv) * D) {
-        kind = 1;
-        head = (r0 - p.Hq * D) / D;
-      } else {
-        kind = 2;
-        head = (r0 - (p.Hq + p.Hkv) * D) / D;
-      }
-      __nv_bfloat16* dst;
-      if (kind == 0)
-        dst = p.q + ((size_t)head * p.q_T + tok) * D;
-      else
-        dst = p.kv + (size_t)req * p.kv_req_stride +
-              ((size_t)(kind == 2 ? p.Hkv : 0) + head) * (size_t)p.kv_cap * D + (size_t)pos * D;
-      if (kind == 2) {
-        for (int c = 0; c < D; c += 16) {
-          float v[16];
-          tmem_ld16(taddr + col0 + c, v);
-          if (ok) store_bf16x16(dst + c, v);
-        }
-      } else {
-        for (int i0 = 0; i0 < half; i0 += 16) {
-          float x1[16], x2[16];
-          tmem_ld16(taddr + col0 + i0, x1);
-          tmem_ld16(taddr + col0 + half + i0, x2);
-          if (ok) {
-            float y1[16], y2[16];
+    int kind, tb, r0, r1;
+    rows_of(p, t.b, kind, tb, r0, r1);
+    __nv_bfloat16* kbase = p.kv + (size_t)req * p.kv_req_stride + (size_t)pos * D;
+    const size_t head_stride = (size_t)p.kv_cap * D;
+    if (kind == 2) {
+      // V is cached transposed, [Hkv][D][cap]: consecutive tokens of a warp
+      // write consecutive positions of each dimension row
+      __nv_bfloat16* vt = p.kv + (size_t)req * p.kv_req_stride + (size_t)p.Hkv * head_stride + pos;
+      for (int c = 0; c < 128; c += 16) {
+        float v[16];
+        tmem_ld16(taddr + c, v);
+        const int r = tb * 128 + c;  // = head * D + dim
+        if (ok) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              // angle in fp64, reduced to [-pi, pi] before the fp32 sincos
-              double a = (double)pos * p.inv_freq[i0 + i];
-              a -= rint(a * 0.15915494309189535) * 6.283185307179586;
-              float s, c;
-              sincosf((float)a, &s, &c);
-              y1[i] = x1[i] * c - x2[i] * s;
-              y2[i] = x2[i] * c + x1[i] * s;
-            }
-            store_bf16x16(dst + i0, y1);
-            store_bf16x16(dst + half + i0, y2);
+          for (int i = 0; i < 16; ++i) vt[(size_t)(r + i) * p.kv_cap] = f2bf(v[i]);
+        }
+      }
+      return;
+    }
+    const float2* cs_row = p.rope + (size_t)(ok ? tok : 0) * half;
+    if (D == 64) {
+      for (int hh = 0; hh < 2; ++hh) {
+        const int head = tb * 2 + hh;
+        __nv_bfloat16* dst = kind == 0 ? p.q + ((size_t)head * p.q_T + tok) * D : kbase + (size_t)head * head_stride;
+        for (int c = 0; c < 32; c += 16) {
+          float x1[16], x2[16], y1[16], y2[16];
+          tmem_ld16(taddr + hh * 64 + c, x1);
+          tmem_ld16(taddr + hh * 64 + 32 + c, x2);
+          if (ok) {
+            float2 cs[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) cs[i] = cs_row[c + i];
+            rotate16(x1, x2, cs, y1, y2);
+            store_bf16x16(dst + c, y1);
+            store_bf16x16(dst + 32 + c, y2);
           }
         }
+      }
+      return;
+    }
+    const int j = D == 256 ? (tb & 1) : 0;
+    const int head = D == 256 ? (tb >> 1) : tb;
+    __nv_bfloat16* dst = kind == 0 ? p.q + ((size_t)head * p.q_T + tok) * D : kbase + (size_t)head * head_stride;
+    for (int c = 0; c < 64; c += 16) {
+      float x1[16], x2[16], y1[16], y2[16];
+      tmem_ld16(taddr + c, x1);
+      tmem_ld16(taddr + 64 + c, x2);
+      if (ok) {
+        float2 cs[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) cs[i] = cs_row[j * 64 + c + i];
+        rotate16(x1, x2, cs, y1, y2);
+        store_bf16x16(dst + j * 64 + c, y1);
+        store_bf16x16(dst + half + j * 64 + c, y2);
       }
     }
   }
 };
 
 // ---------------------------------------------------------------------------
-// Output projection + residual: x[t, f] += sum_c O[t, c] W_o[f, c]
+// Residual update x[t, f] += acc[f, t] for one 16-token chunk of an epilogue
+// row: the 16 residual loads are issued together, then the 16 stores.
+// ---------------------------------------------------------------------------
+DG_DEVINL void residual_add16(float* x, int d, int f, int tok0, int T, const float* v) {
+  float xv[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) xv[j] = tok0 + j < T ? x[(size_t)(tok0 + j) * d + f] : 0.f;
+#pragma unroll
+  for (int j = 0; j < 16; ++j)
+    if (tok0 + j < T) x[(size_t)(tok0 + j) * d + f] = xv[j] + v[j];
+}
+
+// ---------------------------------------------------------------------------
+// Output projection + residual: x[t, f] += sum_c O[t, c] W_o[f, c].
+// Tile (128 output features a, 64 tokens b).
 // ---------------------------------------------------------------------------
 struct P_OPROJ : ProblemBase {
-  static constexpr int BN = 128, STAGES = 6, B_STAGE = BN * 128, TMEM_COLS = 256;
+  static constexpr int BN = 64, STAGES = 8, B_STAGE = BN * 128, TMEM_COLS = 128;
   struct Params {
     CUtensorMap tmA;  // w_o [d, Hq*D]
-    CUtensorMap tmB;  // O [Tcap, Hq*D]
+    CUtensorMap tmB;  // O [Tcap, Hq*D], 64-row boxes
     int T, nk, MT, NT, d;
     float* x;
     int* err;
@@ -149,24 +214,20 @@ struct P_OPROJ : ProblemBase {
     t.nk = p.nk;
     t.b = v % p.NT;  // token tile
     t.a = v / p.NT;  // 128 output features
-    t.n_mma = round_up16(min(128, p.T - t.b * 128));
+    t.n_mma = round_up16(min(BN, p.T - t.b * BN));
     return t;
   }
   DG_DEVINL static uint32_t tx_bytes(const Params&, const Tile&) { return kAStage + B_STAGE; }
   DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
     tma_load_2d(sa, &p.tmA, kb * 64, t.a * 128, bar);
-    tma_load_2d(sb, &p.tmB, kb * 64, t.b * 128, bar);
+    tma_load_2d(sb, &p.tmB, kb * 64, t.b * BN, bar);
   }
   DG_DEVINL static void epilogue(const Params& p, const Tile& t, uint32_t taddr, int, int, int row, uint8_t*) {
     const int f = t.a * 128 + row;
     for (int c0 = 0; c0 < t.n_mma; c0 += 16) {
       float v[16];
       tmem_ld16(taddr + c0, v);
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const int tok = t.b * 128 + c0 + j;
-        if (tok < p.T) p.x[(size_t)tok * p.d + f] += v[j];
-      }
+      residual_add16(p.x, p.d, f, t.b * BN + c0, p.T, v);
     }
   }
 };
@@ -304,14 +365,14 @@ struct P_ED : ProblemBase {
 
 // ---------------------------------------------------------------------------
 // Shared expert gate|up + SwiGLU.  Tile (mt, j): tokens mt*128..+127, hidden
-// units j*64..+63; B rows 0..63 = gate rows, 64..127 = up rows.
+// units j*32..+31; B rows 0..31 = gate rows, 32..63 = up rows.
 // ---------------------------------------------------------------------------
 struct P_SGU : ProblemBase {
-  static constexpr int BN = 128, STAGES = 6, B_STAGE = BN * 128, TMEM_COLS = 256;
+  static constexpr int BN = 64, STAGES = 8, B_STAGE = BN * 128, TMEM_COLS = 128;
   struct Params {
     CUtensorMap tmX;  // normed tokens [Tcap, d]
-    CUtensorMap tmG;  // ws_gate [fs, d]
-    CUtensorMap tmU;  // ws_up [fs, d]
+    CUtensorMap tmG;  // ws_gate [fs, d], 32-row boxes
+    CUtensorMap tmU;  // ws_up [fs, d], 32-row boxes
     int T, nk, MT, FJ, fs;
     __nv_bfloat16* hs;  // [Tcap, fs]
     int* err;
@@ -334,39 +395,38 @@ struct P_SGU : ProblemBase {
   DG_DEVINL static uint32_t tx_bytes(const Params&, const Tile&) { return kAStage + B_STAGE; }
   DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
     tma_load_2d(sa, &p.tmX, kb * 64, t.a * 128, bar);
-    tma_load_2d(sb, &p.tmG, kb * 64, t.b * 64, bar);
-    tma_load_2d(sb + 64 * 128, &p.tmU, kb * 64, t.b * 64, bar);
+    tma_load_2d(sb, &p.tmG, kb * 64, t.b * 32, bar);
+    tma_load_2d(sb + 32 * 128, &p.tmU, kb * 64, t.b * 32, bar);
   }
   DG_DEVINL static void epilogue(const Params& p, const Tile& t, uint32_t taddr, int, int, int row, uint8_t*) {
     const int tok = t.a * 128 + row;
     const bool ok = tok < p.T;
-    for (int c0 = 0; c0 < 64; c0 += 16) {
+    for (int c0 = 0; c0 < 32; c0 += 16) {
       float g[16], u[16];
       tmem_ld16(taddr + c0, g);
-      tmem_ld16(taddr + 64 + c0, u);
+      tmem_ld16(taddr + 32 + c0, u);
       if (ok) {
         float h[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) h[i] = silu_f(g[i]) * u[i];
-        store_bf16x16(p.hs + (size_t)tok * p.fs + t.b * 64 + c0, h);
+        store_bf16x16(p.hs + (size_t)tok * p.fs + t.b * 32 + c0, h);
       }
     }
   }
 };
 
 // ---------------------------------------------------------------------------
-// Shared expert down + routed combine + residual:
-//   x[t, f] += (Hs W_sd^T)[t, f] + sum_j Yp[row(t, j), f]
+// Shared expert down + residual: x[t, f] += (Hs W_sd^T)[t, f].  The routed
+// experts' outputs are added by the next combine + RMSNorm kernel.
+// Tile (128 output features a, 64 tokens b).
 // ---------------------------------------------------------------------------
 struct P_SD : ProblemBase {
-  static constexpr int BN = 128, STAGES = 6, B_STAGE = BN * 128, TMEM_COLS = 256;
+  static constexpr int BN = 64, STAGES = 8, B_STAGE = BN * 128, TMEM_COLS = 128;
   struct Params {
     CUtensorMap tmW;  // ws_down [d, fs]
-    CUtensorMap tmH;  // Hs [Tcap, fs]
-    int T, nk, MT, NT, d, k;
+    CUtensorMap tmH;  // Hs [Tcap, fs], 64-row boxes
+    int T, nk, MT, NT, d;
     float* x;
-    const float* yp;
-    const int* pair_row;
     int* err;
   };
   DG_DEVINL static void prefetch(const Params& p) {
@@ -380,28 +440,20 @@ struct P_SD : ProblemBase {
     t.nk = p.nk;
     t.b = v % p.NT;
     t.a = v / p.NT;
-    t.n_mma = round_up16(min(128, p.T - t.b * 128));
+    t.n_mma = round_up16(min(BN, p.T - t.b * BN));
     return t;
   }
   DG_DEVINL static uint32_t tx_bytes(const Params&, const Tile&) { return kAStage + B_STAGE; }
   DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
     tma_load_2d(sa, &p.tmW, kb * 64, t.a * 128, bar);
-    tma_load_2d(sb, &p.tmH, kb * 64, t.b * 128, bar);
+    tma_load_2d(sb, &p.tmH, kb * 64, t.b * BN, bar);
   }
   DG_DEVINL static void epilogue(const Params& p, const Tile& t, uint32_t taddr, int, int, int row, uint8_t*) {
     const int f = t.a * 128 + row;
     for (int c0 = 0; c0 < t.n_mma; c0 += 16) {
       float v[16];
       tmem_ld16(taddr + c0, v);
-#pragma unroll 4
-      for (int i = 0; i < 16; ++i) {
-        const int tok = t.b * 128 + c0 + i;
-        if (tok < p.T) {
-          float s = v[i];
-          for (int j = 0; j < p.k; ++j) s += p.yp[(size_t)p.pair_row[tok * p.k + j] * p.d + f];
-          p.x[(size_t)tok * p.d + f] += s;
-        }
-      }
+      residual_add16(p.x, p.d, f, t.b * BN + c0, p.T, v);
     }
   }
 };
@@ -531,7 +583,7 @@ cudaError_t run_qkv(const QkvArgs& a, cudaStream_t st) {
   p.T = a.T;
   p.nk = a.d / 64;
   p.MT = (a.T + 127) / 128;
-  p.NT = a.rows / 256;
+  p.NT = a.rows / 128;
   p.D = a.D;
   p.Hq = a.Hq;
   p.Hkv = a.Hkv;
@@ -540,7 +592,7 @@ cudaError_t run_qkv(const QkvArgs& a, cudaStream_t st) {
   p.kv_req_stride = a.kv_req_stride;
   p.tok_pos = a.tok_pos;
   p.tok_req = a.tok_req;
-  p.inv_freq = a.inv_freq;
+  p.rope = a.rope;
   p.q = a.q;
   p.kv = a.kv;
   p.err = a.err;
@@ -554,7 +606,7 @@ cudaError_t run_oproj(const OprojArgs& a, cudaStream_t st) {
   p.T = a.T;
   p.nk = a.K / 64;
   p.MT = a.d / 128;
-  p.NT = (a.T + 127) / 128;
+  p.NT = (a.T + P_OPROJ::BN - 1) / P_OPROJ::BN;
   p.d = a.d;
   p.x = a.x;
   p.err = a.err;
@@ -601,7 +653,7 @@ cudaError_t run_shared_gate_up(const SharedArgs& a, cudaStream_t st) {
   g.T = a.T;
   g.nk = a.d / 64;
   g.MT = (a.T + 127) / 128;
-  g.FJ = a.fs / 64;
+  g.FJ = a.fs / 32;
   g.fs = a.fs;
   g.hs = a.hs;
   g.err = a.err;
@@ -615,12 +667,9 @@ cudaError_t run_shared_down(const SharedArgs& a, cudaStream_t st) {
   dn.T = a.T;
   dn.nk = a.fs / 64;
   dn.MT = a.d / 128;
-  dn.NT = (a.T + 127) / 128;
+  dn.NT = (a.T + P_SD::BN - 1) / P_SD::BN;
   dn.d = a.d;
-  dn.k = a.k;
   dn.x = a.x;
-  dn.yp = a.yp;
-  dn.pair_row = a.pair_row;
   dn.err = a.err;
   return launch_gemm<P_SD>(dn, grid_for(dn.MT * dn.NT, a.num_sms), st);
 }

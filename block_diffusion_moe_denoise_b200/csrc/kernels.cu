@@ -17,7 +17,8 @@ struct EmbedParams {
 };
 
 __global__ void k_embed(EmbedParams p, const bf16* __restrict__ embed, int V, int d, float* __restrict__ x,
-                        int* tok_pos, int* tok_req, int* err) {
+                        int* tok_pos, int* tok_req, const double* __restrict__ inv_freq, int half,
+                        float2* __restrict__ rope, int* err) {
   const int t = blockIdx.x;
   const int slot = t / p.s.Tr;
   const int i = t - slot * p.s.Tr;
@@ -26,9 +27,19 @@ __global__ void k_embed(EmbedParams p, const bf16* __restrict__ embed, int V, in
     if (threadIdx.x == 0) atomicOr(err, DG_DEVERR_TOKEN);
     id = 0;
   }
+  const int pos = p.s.pos0[slot] + i;
   if (threadIdx.x == 0) {
-    tok_pos[t] = p.s.pos0[slot] + i;
+    tok_pos[t] = pos;
     tok_req[t] = p.s.req[slot];
+  }
+  // RoPE (cos, sin) of this token's position for every frequency: the angle in
+  // fp64, reduced to [-pi, pi] before the fp32 sincos; shared by all layers.
+  for (int f = threadIdx.x; f < half; f += blockDim.x) {
+    double a = (double)pos * inv_freq[f];
+    a -= rint(a * 0.15915494309189535) * 6.283185307179586;
+    float sn, cs;
+    sincosf((float)a, &sn, &cs);
+    rope[(size_t)t * half + f] = make_float2(cs, sn);
   }
   const uint4* src = reinterpret_cast<const uint4*>(embed + (size_t)id * d);
   float4* dst = reinterpret_cast<float4*>(x + (size_t)t * d);
@@ -43,13 +54,14 @@ __global__ void k_embed(EmbedParams p, const bf16* __restrict__ embed, int V, in
 }
 
 cudaError_t run_embed(const int* const* ids, const SlotInfo& s, const bf16* embed, int V, int d, float* x,
-                      int* tok_pos, int* tok_req, int* err, cudaStream_t st) {
+                      int* tok_pos, int* tok_req, const double* inv_freq, int half, float2* rope, int* err,
+                      cudaStream_t st) {
   EmbedParams p;
   p.s = s;
   for (int i = 0; i < DG_MAX_REQUESTS; ++i) p.ids[i] = i < s.n ? ids[i] : nullptr;
   const int T = s.n * s.Tr;
   if (T == 0) return cudaSuccess;
-  k_embed<<<T, 128, 0, st>>>(p, embed, V, d, x, tok_pos, tok_req, err);
+  k_embed<<<T, 128, 0, st>>>(p, embed, V, d, x, tok_pos, tok_req, inv_freq, half, rope, err);
   return cudaGetLastError();
 }
 
@@ -81,6 +93,77 @@ __global__ void k_rmsnorm(const float* __restrict__ x, const float* __restrict__
 cudaError_t run_rmsnorm(const float* x, const float* g, int T, int d, float eps, bf16* out, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
   k_rmsnorm<<<(T + 7) / 8, 256, 0, st>>>(x, g, T, d, eps, out);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Routed-expert combine + RMSNorm, one CTA per token row:
+//   x[t] += sum_j Yp[row(t, j)]   (k = 0: nothing to combine)
+//   out[t] = bf16(x[t] / sqrt(mean(x[t]^2) + eps) * g)
+// The k expert outputs are added in slot order (deterministic).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_combine_rmsnorm(float* __restrict__ x, const float* __restrict__ yp,
+                                                         const int* __restrict__ pair_row, int k,
+                                                         const float* __restrict__ g, int d, float eps,
+                                                         bf16* __restrict__ out) {
+  extern __shared__ float crow[];  // [d]
+  __shared__ float red[8];
+  const int t = blockIdx.x;
+  float4* xr = reinterpret_cast<float4*>(x + (size_t)t * d);
+  float4* cr = reinterpret_cast<float4*>(crow);
+  int rows[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) rows[j] = j < k ? pair_row[(size_t)t * k + j] : 0;
+  float ss = 0.f;
+  for (int c = threadIdx.x; c < d / 4; c += blockDim.x) {
+    float4 v = xr[c];
+    float4 y[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (j < k) y[j] = reinterpret_cast<const float4*>(yp + (size_t)rows[j] * d)[c];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (j < k) {
+        v.x += y[j].x;
+        v.y += y[j].y;
+        v.z += y[j].z;
+        v.w += y[j].w;
+      }
+    if (k) xr[c] = v;
+    cr[c] = v;
+    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  }
+  if (out == nullptr) return;
+  ss = warp_sum(ss);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+    v = warp_sum(v);
+    if (threadIdx.x == 0) red[0] = v;
+  }
+  __syncthreads();
+  const float rs = rsqrtf(red[0] / (float)d + eps);
+  const float4* g4 = reinterpret_cast<const float4*>(g);
+  uint2* o = reinterpret_cast<uint2*>(out + (size_t)t * d);
+  for (int c = threadIdx.x; c < d / 4; c += blockDim.x) {
+    const float4 v = cr[c];
+    const float4 w = g4[c];
+    o[c] = make_uint2(pack_bf16x2(v.x * rs * w.x, v.y * rs * w.y), pack_bf16x2(v.z * rs * w.z, v.w * rs * w.w));
+  }
+}
+
+cudaError_t run_combine_rmsnorm(float* x, const float* yp, const int* pair_row, int k, const float* g, int T, int d,
+                                float eps, bf16* out, cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+  const size_t smem = (size_t)d * sizeof(float);
+  static size_t configured = 0;
+  if (smem > 48 * 1024 && smem > configured) {
+    cudaError_t e = cudaFuncSetAttribute(k_combine_rmsnorm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    configured = smem;
+  }
+  k_combine_rmsnorm<<<T, 256, smem, st>>>(x, yp, pair_row, k, g, d, eps, out);
   return cudaGetLastError();
 }
 
@@ -151,21 +234,22 @@ cudaError_t run_topk(const float* logits, int T, int E, int k, int* idx, float* 
 }
 
 // ---------------------------------------------------------------------------
-// FFN RMSNorm + router logits (fp32 normalised row x bf16 router weights,
-// fp32 accumulation) + top-k.
-// kRouterTok tokens per CTA so the router weight is read once per CTA.
+// FFN RMSNorm + router logits.  Grid (token groups of kRT, expert groups of
+// kRE): each CTA normalises its kRT rows in fp32 (the CTA of expert group 0
+// also writes the bf16 copy the experts read) and computes their logits
+// against kRE router rows, fp32 row x bf16 weights with fp32 accumulation.
+// Each warp owns 4 experts so every lane keeps 4 independent weight loads in
+// flight.  The top-k selection follows in k_topk.
 // ---------------------------------------------------------------------------
-constexpr int kRouterTok = 4;
+constexpr int kRT = 8, kRE = 32;
 
-__global__ void __launch_bounds__(256) k_router(const float* __restrict__ x, const float* __restrict__ g, float eps,
-                                                const bf16* __restrict__ wr, int T, int d, int E, int k,
-                                                bf16* __restrict__ u, int* idx, float* w) {
-  extern __shared__ float rsm[];
-  float* su = rsm;                       // [kRouterTok][d]
-  float* sl = rsm + kRouterTok * d;      // [kRouterTok][E]
+__global__ void __launch_bounds__(256) k_router_logits(const float* __restrict__ x, const float* __restrict__ g,
+                                                       float eps, const bf16* __restrict__ wr, int T, int d, int E,
+                                                       bf16* __restrict__ u, float* __restrict__ logits) {
+  extern __shared__ float su[];  // [kRT][d]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t0 = blockIdx.x * kRouterTok;
-  if (warp < kRouterTok) {
+  const int t0 = blockIdx.x * kRT, e0 = blockIdx.y * kRE;
+  if (warp < kRT) {
     const int t = t0 + warp;
     float* dst = su + warp * d;
     if (t < T) {
@@ -182,65 +266,78 @@ __global__ void __launch_bounds__(256) k_router(const float* __restrict__ x, con
       for (int c = lane; c < d / 4; c += 32) {
         const float4 v = xr[c];
         const float4 gg = g4[c];
-        const uint32_t lo = pack_bf16x2(v.x * rs * gg.x, v.y * rs * gg.y);
-        const uint32_t hi = pack_bf16x2(v.z * rs * gg.z, v.w * rs * gg.w);
-        uo[c] = make_uint2(lo, hi);
-        // the router reads the fp32 normalised row (the experts read the bf16 copy)
-        reinterpret_cast<float4*>(dst)[c] =
-            make_float4(v.x * rs * gg.x, v.y * rs * gg.y, v.z * rs * gg.z, v.w * rs * gg.w);
+        const float4 n = make_float4(v.x * rs * gg.x, v.y * rs * gg.y, v.z * rs * gg.z, v.w * rs * gg.w);
+        if (blockIdx.y == 0) uo[c] = make_uint2(pack_bf16x2(n.x, n.y), pack_bf16x2(n.z, n.w));
+        reinterpret_cast<float4*>(dst)[c] = n;
       }
     } else {
       for (int c = lane; c < d; c += 32) dst[c] = 0.f;
     }
   }
   __syncthreads();
-  for (int e = warp; e < E; e += 8) {
-    float acc[kRouterTok];
+  float acc[4][kRT];
 #pragma unroll
-    for (int tt = 0; tt < kRouterTok; ++tt) acc[tt] = 0.f;
-    const bf16* wrow = wr + (size_t)e * d;
-    for (int c = lane * 8; c < d; c += 256) {
-      const uint4 wv = *reinterpret_cast<const uint4*>(wrow + c);
+  for (int q = 0; q < 4; ++q)
+#pragma unroll
+    for (int tt = 0; tt < kRT; ++tt) acc[q][tt] = 0.f;
+  const int eb = e0 + warp * 4;
+  for (int c = lane * 8; c < d; c += 256) {
+    float wf[4][8];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint4 wv = make_uint4(0, 0, 0, 0);
+      if (eb + q < E) wv = *reinterpret_cast<const uint4*>(wr + (size_t)(eb + q) * d + c);
       const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&wv);
-      float wf[8];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const float2 f2 = __bfloat1622float2(h[i]);
-        wf[2 * i] = f2.x;
-        wf[2 * i + 1] = f2.y;
-      }
-#pragma unroll
-      for (int tt = 0; tt < kRouterTok; ++tt) {
-        const float* s = su + tt * d + c;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[tt] = fmaf(s[i], wf[i], acc[tt]);
+        wf[q][2 * i] = f2.x;
+        wf[q][2 * i + 1] = f2.y;
       }
     }
 #pragma unroll
-    for (int tt = 0; tt < kRouterTok; ++tt) {
-      const float r = warp_sum(acc[tt]);
-      if (lane == 0) sl[tt * E + e] = r;
+    for (int tt = 0; tt < kRT; ++tt) {
+      const float4 a = *reinterpret_cast<const float4*>(su + tt * d + c);
+      const float4 b = *reinterpret_cast<const float4*>(su + tt * d + c + 4);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float r = acc[q][tt];
+        r = fmaf(a.x, wf[q][0], r);
+        r = fmaf(a.y, wf[q][1], r);
+        r = fmaf(a.z, wf[q][2], r);
+        r = fmaf(a.w, wf[q][3], r);
+        r = fmaf(b.x, wf[q][4], r);
+        r = fmaf(b.y, wf[q][5], r);
+        r = fmaf(b.z, wf[q][6], r);
+        r = fmaf(b.w, wf[q][7], r);
+        acc[q][tt] = r;
+      }
     }
   }
-  __syncthreads();
-  if (warp < kRouterTok && t0 + warp < T) {
-    const int t = t0 + warp;
-    topk_warp(sl + warp * E, E, k, idx + (size_t)t * k, w + (size_t)t * k);
-  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+#pragma unroll
+    for (int tt = 0; tt < kRT; ++tt) {
+      const float r = warp_sum(acc[q][tt]);
+      if (lane == 0 && eb + q < E && t0 + tt < T) logits[(size_t)(t0 + tt) * E + eb + q] = r;
+    }
 }
 
 cudaError_t run_router(const float* x, const float* g, float eps, const bf16* wr, int T, int d, int E, int k, bf16* u,
-                       int* idx, float* w, int*, cudaStream_t st) {
+                       float* logits, int* idx, float* w, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
-  const size_t smem = (size_t)kRouterTok * (d + E) * sizeof(float);
+  const size_t smem = (size_t)kRT * d * sizeof(float);
   static size_t configured = 0;
   if (smem > configured) {
-    cudaError_t e = cudaFuncSetAttribute(k_router, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(k_router_logits, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     configured = smem;
   }
-  k_router<<<(T + kRouterTok - 1) / kRouterTok, 256, smem, st>>>(x, g, eps, wr, T, d, E, k, u, idx, w);
-  return cudaGetLastError();
+  dim3 grid((T + kRT - 1) / kRT, (E + kRE - 1) / kRE);
+  k_router_logits<<<grid, 256, smem, st>>>(x, g, eps, wr, T, d, E, u, logits);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return run_topk(logits, T, E, k, idx, w, st);
 }
 
 // ---------------------------------------------------------------------------
@@ -278,6 +375,12 @@ __global__ void __launch_bounds__(1024) k_group(GroupArgs a) {
     for (int e = 0; e < E; ++e) {
       off[e + 1] = off[e] + cnt[e];
       toff[e + 1] = toff[e] + (cnt[e] + 63) / 64;
+    }
+    if (a.route_stats) {
+      int touched = 0;
+      for (int e = 0; e < E; ++e) touched += cnt[e] > 0;
+      atomicAdd(&a.route_stats[0], (unsigned long long)touched);
+      atomicAdd(&a.route_stats[1], 1ull);
     }
     const int egu = toff[E] * a.FJ, ed = toff[E] * a.MD;
     if (egu > a.egu_cap || ed > a.ed_cap) atomicOr(a.err, DG_DEVERR_CAPACITY);
@@ -353,50 +456,61 @@ cudaError_t run_gather(const bf16* u, const int* row_token, int rows, int d, bf1
 //   m = max, s = sum e^(z-m), t = sum e^(z-m)(z-m), argmax lowest id on ties.
 //   logZ = m + ln s, H = ln s - t/s, logconf = -ln s.
 // ---------------------------------------------------------------------------
+struct LmPart {
+  float m, s, t;
+  int a;
+};
+
+DG_DEVINL LmPart lm_merge(LmPart x, LmPart y) {
+  if (!(y.s > 0.f)) return x;
+  if (!(x.s > 0.f)) return y;
+  if (y.m > x.m || (y.m == x.m && y.a < x.a)) {
+    const LmPart tmp = x;
+    x = y;
+    y = tmp;
+  }
+  // x holds the larger max (ties: the lower argmax)
+  const float f = expf(y.m - x.m);
+  x.t += f * (y.t + (y.m - x.m) * y.s);
+  x.s += f * y.s;
+  return x;
+}
+
 __global__ void k_lm_combine(const float4* __restrict__ part, int G, int MT, int T, float* stats, int* argmax,
                              int* err) {
-  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
   if (t >= T) return;
-  float m = -INFINITY, s = 0.f, tt = 0.f;
-  int a = 0x7fffffff;
   const size_t stride = (size_t)MT * 128;
-  for (int c = 0; c < G; ++c) {
+  LmPart r{-INFINITY, 0.f, 0.f, 0x7fffffff};
+  for (int c = lane; c < G; c += 32) {
     const float4 v = part[(size_t)c * stride + t];
-    const float mc = v.x, sc = v.y, tc = v.z;
-    const int ac = __float_as_int(v.w);
-    if (!(sc > 0.f)) {
-      if (sc != sc) atomicOr(err, DG_DEVERR_NAN);
-      continue;
-    }
-    if (s == 0.f) {
-      m = mc;
-      s = sc;
-      tt = tc;
-      a = ac;
-    } else if (mc > m) {
-      const float f = expf(m - mc);
-      tt = f * (tt + (m - mc) * s) + tc;
-      s = f * s + sc;
-      m = mc;
-      a = ac;
-    } else {
-      const float f = expf(mc - m);
-      tt += f * (tc + (mc - m) * sc);
-      s += f * sc;
-      if (mc == m && ac < a) a = ac;
-    }
+    if (v.y != v.y) atomicOr(err, DG_DEVERR_NAN);
+    r = lm_merge(r, LmPart{v.x, v.y, v.z, __float_as_int(v.w)});
   }
-  const float ls = logf(s);
-  float4 o = make_float4(ls - tt / s, -ls, m, m + ls);
-  if (!(s > 0.f) || o.x != o.x) atomicOr(err, DG_DEVERR_NAN);
-  reinterpret_cast<float4*>(stats)[t] = o;
-  argmax[t] = a;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    LmPart q;
+    q.m = __shfl_xor_sync(0xffffffffu, r.m, o);
+    q.s = __shfl_xor_sync(0xffffffffu, r.s, o);
+    q.t = __shfl_xor_sync(0xffffffffu, r.t, o);
+    q.a = __shfl_xor_sync(0xffffffffu, r.a, o);
+    // both lanes of a pair merge in the same (lower lane first) order
+    r = (lane & o) ? lm_merge(q, r) : lm_merge(r, q);
+  }
+  if (lane == 0) {
+    const float ls = logf(r.s);
+    const float4 o = make_float4(ls - r.t / r.s, -ls, r.m, r.m + ls);
+    if (!(r.s > 0.f) || o.x != o.x) atomicOr(err, DG_DEVERR_NAN);
+    reinterpret_cast<float4*>(stats)[t] = o;
+    argmax[t] = r.a;
+  }
 }
 
 cudaError_t run_lm_combine(const float4* part, int G, int MT, int T, float* stats, int* argmax, int* err,
                            cudaStream_t st) {
   if (T == 0) return cudaSuccess;
-  k_lm_combine<<<(T + 127) / 128, 128, 0, st>>>(part, G, MT, T, stats, argmax, err);
+  k_lm_combine<<<(T + 7) / 8, 256, 0, st>>>(part, G, MT, T, stats, argmax, err);
   return cudaGetLastError();
 }
 
@@ -505,30 +619,50 @@ cudaError_t run_sample(const SampleArgs& a, cudaStream_t st) {
 }
 
 // ---------------------------------------------------------------------------
-// KV copy between the cache layout [Hkv][cap][D] and a dense [Hkv][n][D].
+// KV copy between the cache layout (K [Hkv][cap][D], V^T [Hkv][D][cap]) and
+// dense [Hkv][n][D] arrays, either direction.
 // ---------------------------------------------------------------------------
-__global__ void k_kv_copy(bf16* cache_k, bf16* cache_v, int Hkv, long long cap, int D, long long pos0, long long n,
-                          const bf16* k_in, const bf16* v_in, bf16* k_out, bf16* v_out) {
+__global__ void k_k_copy(bf16* cache_k, int Hkv, long long cap, int D, long long pos0, long long n, const bf16* k_in,
+                         bf16* k_out) {
   const long long r = blockIdx.x;  // (head, i)
   const int head = (int)(r / n);
   const long long i = r - (long long)head * n;
   const size_t cache_off = ((size_t)head * cap + pos0 + i) * D;
   const size_t dense_off = ((size_t)head * n + i) * D;
   for (int c = threadIdx.x; c < D / 8; c += blockDim.x) {
-    if (k_in) {
+    if (k_in)
       reinterpret_cast<uint4*>(cache_k + cache_off)[c] = reinterpret_cast<const uint4*>(k_in + dense_off)[c];
-      reinterpret_cast<uint4*>(cache_v + cache_off)[c] = reinterpret_cast<const uint4*>(v_in + dense_off)[c];
-    } else {
+    else
       reinterpret_cast<uint4*>(k_out + dense_off)[c] = reinterpret_cast<const uint4*>(cache_k + cache_off)[c];
-      reinterpret_cast<uint4*>(v_out + dense_off)[c] = reinterpret_cast<const uint4*>(cache_v + cache_off)[c];
-    }
+  }
+}
+
+__global__ void k_vt_copy(bf16* cache_vt, int Hkv, long long cap, int D, long long pos0, long long n,
+                          const bf16* v_in, bf16* v_out) {
+  const long long total = (long long)Hkv * D * n;
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
+       e += (long long)gridDim.x * blockDim.x) {
+    const long long i = e % n;             // position fastest: coalesced in the cache
+    const long long hd = e / n;            // head * D + dim
+    const long long head = hd / D, dim = hd % D;
+    const size_t c_off = (size_t)hd * cap + pos0 + i;
+    const size_t d_off = ((size_t)head * n + i) * D + dim;
+    if (v_in)
+      cache_vt[c_off] = v_in[d_off];
+    else
+      v_out[d_off] = cache_vt[c_off];
   }
 }
 
 cudaError_t run_kv_copy(bf16* cache_k, bf16* cache_v, int Hkv, long long cap, int D, long long pos0, long long n,
                         const bf16* k_in, const bf16* v_in, bf16* k_out, bf16* v_out, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
-  k_kv_copy<<<(unsigned)(Hkv * n), 32, 0, st>>>(cache_k, cache_v, Hkv, cap, D, pos0, n, k_in, v_in, k_out, v_out);
+  k_k_copy<<<(unsigned)(Hkv * n), 32, 0, st>>>(cache_k, Hkv, cap, D, pos0, n, k_in, k_out);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const long long total = (long long)Hkv * D * n;
+  const unsigned blocks = (unsigned)((total + 255) / 256 < 65535 ? (total + 255) / 256 : 65535);
+  k_vt_copy<<<blocks, 256, 0, st>>>(cache_v, Hkv, cap, D, pos0, n, v_in, v_out);
   return cudaGetLastError();
 }
 

@@ -59,7 +59,9 @@ int dg_debug_forward(dg_handle* h, int req, const int32_t* d_tokens, int T, int 
  * "pair_row" i32 [T*k]; "row_pair" i32 [T*k]; "hp" bf16 [T*k, fe];
  * "yp" f32 [T*k, d]; "hs" bf16 [T, fs]; "stats" f32 [Tcap][4];
  * "argmax" i32 [Tcap]; "canvas" i32 [max_req, canvas]; "mask" u8 [...];
- * "remaining" i32 [max_req].  Returns DG_E_ARG for an unknown name. */
+ * "remaining" i32 [max_req]; "route_stats" u64 [2] = (sum over router launches
+ * of the number of experts that received a token, number of launches).
+ * Returns DG_E_ARG for an unknown name. */
 int dg_debug_buffer(const dg_handle* h, const char* name, size_t* offset, size_t* bytes);
 
 /* Per-kernel-class timing: enable=1 records a CUDA event pair on the handle's

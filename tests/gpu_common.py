@@ -43,13 +43,14 @@ def routing_match(gpu_idx: np.ndarray, ora_idx: np.ndarray) -> np.ndarray:
 
 # Routing ambiguity.  Top-k routing is discontinuous: a token whose k-th and
 # (k+1)-th router logits are nearly tied can pick a different expert on the GPU
-# than in the oracle (the GPU's residual stream carries bf16 rounding of every
-# earlier GEMM input, about 1e-3 relative, i.e. router-logit noise of ~4e-4 at
-# d=256 and ~1.2e-3 at d=2816), which moves that token's hidden state by tens
-# of percent.  Such tokens are identified from the ORACLE's own router logits
-# (gap below ROUTER_GAP, >= 4 sigma of that noise), excluded from value
-# comparisons and counted; everywhere else routing must agree exactly.
-ROUTER_GAP = 5e-3
+# than in the oracle, which moves that token's hidden state by tens of percent.
+# The GPU's residual stream carries the bf16 rounding of every earlier GEMM
+# input (measured relative L2 error of a layer's output: ~3e-3), so its router
+# logits carry noise of about 3e-3 times their RMS.  A token is ambiguous when
+# the ORACLE's gap is below ROUTER_GAP_REL (1.5%, ~5 sigma of that noise) of
+# the RMS of that layer's router logits; such tokens are excluded from value
+# comparisons and counted, and everywhere else routing must agree exactly.
+ROUTER_GAP_REL = 0.015
 
 
 def router_gap(router_logits: np.ndarray, k: int) -> np.ndarray:
@@ -62,7 +63,8 @@ def ambiguous_tokens(trace_layers, k: int, upto: int | None = None) -> np.ndarra
     recs = trace_layers if upto is None else trace_layers[:upto]
     amb = np.zeros(recs[0]["router_logits"].shape[0], dtype=bool)
     for rec in recs:
-        amb |= router_gap(rec["router_logits"], k) < ROUTER_GAP
+        r = rec["router_logits"]
+        amb |= router_gap(r, k) < ROUTER_GAP_REL * np.sqrt(np.mean(r * r))
     return amb
 
 
@@ -85,3 +87,27 @@ def oracle_prefill_traced(ora, cache, tokens):
 def kv_rel_l2(gpu_kv: np.ndarray, ora_kv: np.ndarray, keep: np.ndarray) -> float:
     """gpu/ora as [Hkv, n, D]; compare positions where keep is True."""
     return rel_l2(gpu_kv[:, keep], ora_kv[:, keep])
+
+
+# Argmax agreement.  With every logit within LOGIT_MAX_ABS of the oracle's,
+# the top-1 token is guaranteed to agree exactly when the oracle's top-1
+# margin exceeds 2 * LOGIT_MAX_ABS: that is asserted with no exception.
+# Tokens with a margin above 1e-2 (the workload's stated threshold) are
+# counted and their agreement reported as a rate, which must stay high.
+STRICT_MARGIN = 2 * LOGIT_MAX_ABS
+PAGE_MARGIN = 1e-2
+
+
+def argmax_agreement(gpu_argmax, ora_logits, keep=None, min_rate=0.95):
+    gpu_argmax = np.asarray(gpu_argmax)
+    srt = np.sort(ora_logits, axis=-1)
+    margin = srt[:, -1] - srt[:, -2]
+    ora_am = np.argmax(ora_logits, axis=-1)
+    keep = np.ones(margin.shape[0], dtype=bool) if keep is None else keep
+    strict = keep & (margin > STRICT_MARGIN)
+    np.testing.assert_array_equal(gpu_argmax[strict], ora_am[strict])
+    counted = keep & (margin > PAGE_MARGIN)
+    agree = (gpu_argmax == ora_am)[counted]
+    rate = float(agree.mean()) if agree.size else 1.0
+    assert rate >= min_rate, (rate, int(counted.sum()))
+    return int(counted.sum()), int((~agree).sum()), rate
