@@ -121,6 +121,8 @@ __global__ void __launch_bounds__(192, 1) k_attn_tc(const __grid_constant__ Attn
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_trigger();
+  pdl_wait();
   const uint32_t tmem = *tmem_slot;   // O: columns [0, D); S buffers at 256 and 320
   const uint32_t tm_o = tmem, tm_s0 = tmem + 256;
 
@@ -327,38 +329,63 @@ __global__ void __launch_bounds__(192, 1) k_attn_tc(const __grid_constant__ Attn
 }
 
 // Merge of the split-KV partials: O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s.
+// One warp per (token, head); lane s reads split s's (max, sum), each lane then
+// owns 8 consecutive output elements and loads every split's values at once.
+constexpr int kMaxSplits = 8;
+
 __global__ void k_attn_combine(const float* __restrict__ part_o, const float2* __restrict__ part_ml, int n_split,
                                int Hq, int q_T, int T, int D, bf16* __restrict__ o) {
+  pdl_trigger();
+  pdl_wait();
   const int w = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (w >= T * Hq) return;
   const int t = w / Hq, h = w % Hq;
-  float M = -INFINITY;
-  for (int s = 0; s < n_split; ++s) {
-    const float2 ml = part_ml[((size_t)s * Hq + h) * q_T + t];
-    if (ml.y > 0.f) M = fmaxf(M, ml.x);
-  }
-  float L = 0.f;
-  float wts[16];
-  for (int s = 0; s < n_split; ++s) {
-    const float2 ml = part_ml[((size_t)s * Hq + h) * q_T + t];
-    wts[s] = ml.y > 0.f ? exp2f(ml.x - M) : 0.f;
-    L += wts[s] * ml.y;
-  }
-  const float inv = L > 0.f ? 1.f / L : 0.f;
-  for (int c = lane * 2; c < D; c += 64) {
-    float ax = 0.f, ay = 0.f;
-    for (int s = 0; s < n_split; ++s) {
-      if (wts[s] == 0.f) continue;
-      const float2 v = *reinterpret_cast<const float2*>(part_o + (((size_t)s * Hq + h) * q_T + t) * D + c);
-      ax += wts[s] * v.x;
-      ay += wts[s] * v.y;
+  float2 ml = make_float2(-INFINITY, 0.f);
+  if (lane < n_split) ml = part_ml[((size_t)lane * Hq + h) * q_T + t];
+  float M = ml.y > 0.f ? ml.x : -INFINITY;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  const float wl = ml.y > 0.f ? exp2f(ml.x - M) : 0.f;
+  float L = wl * ml.y;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+  float wts[kMaxSplits];
+#pragma unroll
+  for (int s = 0; s < kMaxSplits; ++s) wts[s] = __shfl_sync(0xffffffffu, wl, s);
+  const int c = lane * 8;
+  if (c >= D) return;
+  float4 va[kMaxSplits], vb[kMaxSplits];
+#pragma unroll
+  for (int s = 0; s < kMaxSplits; ++s)
+    if (s < n_split && wts[s] != 0.f) {
+      const float4* src = reinterpret_cast<const float4*>(part_o + (((size_t)s * Hq + h) * q_T + t) * D + c);
+      va[s] = src[0];
+      vb[s] = src[1];
     }
-    *reinterpret_cast<uint32_t*>(o + (size_t)t * Hq * D + (size_t)h * D + c) = pack_bf16x2(ax * inv, ay * inv);
-  }
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int s = 0; s < kMaxSplits; ++s)
+    if (s < n_split && wts[s] != 0.f) {
+      acc[0] += wts[s] * va[s].x;
+      acc[1] += wts[s] * va[s].y;
+      acc[2] += wts[s] * va[s].z;
+      acc[3] += wts[s] * va[s].w;
+      acc[4] += wts[s] * vb[s].x;
+      acc[5] += wts[s] * vb[s].y;
+      acc[6] += wts[s] * vb[s].z;
+      acc[7] += wts[s] * vb[s].w;
+    }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  uint4 u;
+  u.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+  u.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+  u.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
+  u.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
+  *reinterpret_cast<uint4*>(o + (size_t)t * Hq * D + (size_t)h * D + c) = u;
 }
 
-int attention_split_cap() { return 16; }
+int attention_split_cap() { return kMaxSplits; }
 
 template <int D>
 static cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st) {
@@ -371,12 +398,18 @@ static cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st) {
   }
   const int G = a.Hq / a.Hkv;
   dim3 grid((G * a.Tr + kAQ - 1) / kAQ, a.Hkv * a.n_slots, a.n_split);
-  k_attn_tc<D><<<grid, 192, smem, st>>>(a);
+  {
+    const cudaError_t e_ = launch_pdl(k_attn_tc<D>, dim3(grid), dim3(192), smem, st, a);
+    if (e_ != cudaSuccess) return e_;
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || a.n_split == 1) return e;
   const int T = a.n_slots * a.Tr;
   const int warps = T * a.Hq;
-  k_attn_combine<<<(warps + 7) / 8, 256, 0, st>>>(a.part_o, a.part_ml, a.n_split, a.Hq, a.q_T, T, D, a.o);
+  {
+    const cudaError_t e_ = launch_pdl(k_attn_combine, dim3((warps + 7) / 8), dim3(256), 0, st, a.part_o, a.part_ml, a.n_split, a.Hq, a.q_T, T, D, a.o);
+    if (e_ != cudaSuccess) return e_;
+  }
   return cudaGetLastError();
 }
 

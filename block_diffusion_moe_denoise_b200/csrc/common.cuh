@@ -22,6 +22,15 @@ enum : int {
 // single kernel; after it the kernel records DG_DEVERR_TIMEOUT and unwinds.
 #define DG_WAIT_LIMIT_NS 2000000000ull
 
+// Programmatic dependent launch: every kernel of the pass is launched so that
+// it may start while its predecessor in the stream drains.  A kernel lets its
+// successor be scheduled (pdl_trigger) and then waits for the predecessor to
+// complete and its writes to be visible (pdl_wait) before touching anything
+// the predecessor produced.  Every CTA waits unconditionally, so completion
+// stays transitive along the stream.
+DG_DEVINL void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+DG_DEVINL void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 DG_DEVINL uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -185,6 +194,12 @@ DG_DEVINL void named_bar_sync(int id, int nthreads) {
 // misc
 // ---------------------------------------------------------------------------
 DG_DEVINL float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+DG_DEVINL int warp_sum_int(int v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;

@@ -49,7 +49,6 @@ bool config_ok(const dg_config* c) {
   if (!(c->head_dim == 64 || c->head_dim == 128 || c->head_dim == 256)) return false;
   if (c->n_kv_heads < 1 || c->n_q_heads < 1 || c->n_q_heads % c->n_kv_heads != 0) return false;
   if ((c->n_q_heads * c->head_dim) % 128 != 0 || (c->n_kv_heads * c->head_dim) % 128 != 0) return false;
-  if (c->ffn_shared % 32 != 0) return false;
   if ((c->n_q_heads * c->head_dim) % 64 != 0) return false;
   if (c->n_experts < 1 || c->n_experts > 256 || c->top_k < 1 || c->top_k > 8 || c->top_k > c->n_experts) return false;
   if (c->ffn_expert < 64 || c->ffn_expert % 64 != 0 || c->ffn_shared < 64 || c->ffn_shared % 64 != 0) return false;
@@ -104,6 +103,9 @@ void make_plan(const dg_config* c, int max_req, long long cap_user, Plan* p) {
   p->add("inv_freq", (size_t)D / 2 * 8);
   p->add("rope", (size_t)Tcap * (D / 2) * 8);
   p->add("router_logits", (size_t)Tcap * c->n_experts * 4);
+  p->add("part", (size_t)kMaxPartSplits * Tcap * d * 4);
+  p->add("route_mask", (size_t)2 * c->n_experts * ((T + 31) / 32) * 4);
+  p->add("un", (size_t)Tcap * d * 4);
   p->add("prompt", (size_t)cap_user * 4);
 }
 
@@ -205,6 +207,7 @@ struct dg_handle {
   CUtensorMap tm_hn, tm_o, tm_u, tm_xp, tm_hp, tm_hs, tm_embed, tm_k, tm_vt;
   long long cap_user = 0;  // capacity the caller asked for (cap is rounded up to 64)
   ReqState req[DG_MAX_REQUESTS];
+  int mask_flip = 0;  // which of the two routing bitmask buffers the next layer uses
 
   template <class T>
   T* B(const char* name) const {
@@ -253,17 +256,22 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
   LAUNCH(h, K_EMBED, 1,
          run_embed(ids, s, h->embed, c.vocab, d, x, h->B<int>("tok_pos"), h->B<int>("tok_req"),
                    h->B<double>("inv_freq"), D / 2, h->B<float2>("rope"), err, st));
-  // the routed outputs of layer l are summed into x by the norm kernel of layer l+1
+  // the routed outputs and the shared-expert partials of layer l are summed
+  // into x by the norm kernel of layer l+1 (or the final norm)
   float* yp = h->B<float>("yp");
   const int* pair_row = h->B<int>("pair_row");
-  int pending_k = 0;
+  float* part = h->B<float>("part");
+  int pending_k = 0, pending_parts = 0;
+  const int so = wpart_splits(d, T, c.n_q_heads * D, h->num_sms);
+  const int ss = wpart_splits(d, T, c.ffn_shared, h->num_sms);
   for (int l = 0; l < n_layers; ++l) {
     const dg_layer_weights& w = h->lw[l];
     const LayerMaps& m = h->maps[l];
     bf16* kv_l = h->B<bf16>("kv") + (size_t)l * h->kv_layer_stride;
     LAUNCH(h, K_RMSNORM, 1,
-           run_combine_rmsnorm(x, yp, pair_row, pending_k, (const float*)w.attn_norm, T, d, c.norm_eps, hn, st));
-    pending_k = 0;
+           run_residual_norm(x, yp, pair_row, pending_k, part, pending_parts, h->Tcap, (const float*)w.attn_norm, T,
+                             d, c.norm_eps, hn, nullptr, st));
+    pending_k = pending_parts = 0;
     QkvArgs qa;
     qa.tm_x = &h->tm_hn;
     qa.tm_w = &m.qkv;
@@ -322,20 +330,25 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     aa.err = err;
     LAUNCH(h, K_ATTN, aa.n_split > 1 ? 2 : 1, run_attention(aa, st));
 
-    OprojArgs oa;
+    WpartArgs oa;
     oa.tm_w = &m.o;
-    oa.tm_o = &h->tm_o;
+    oa.tm_x = &h->tm_o;
     oa.T = T;
+    oa.Tcap = h->Tcap;
     oa.d = d;
     oa.K = c.n_q_heads * D;
+    oa.splits = so;
     oa.num_sms = h->num_sms;
-    oa.x = x;
+    oa.part = part;
     oa.err = err;
-    LAUNCH(h, K_OPROJ, 1, run_oproj(oa, st));
-
-    LAUNCH(h, K_ROUTER, 2,
-           run_router(x, (const float*)w.ffn_norm, c.norm_eps, (const bf16*)w.w_router, T, d, c.n_experts, k,
-                      h->B<bf16>("u"), h->B<float>("router_logits"), h->B<int>("idx"), h->B<float>("w"), st));
+    LAUNCH(h, K_OPROJ, 1, run_wpart(oa, st));
+    // x += attention output projection; FFN RMSNorm -> bf16 rows (experts) and fp32 rows (router)
+    LAUNCH(h, K_RMSNORM, 1,
+           run_residual_norm(x, nullptr, nullptr, 0, part, so, h->Tcap, (const float*)w.ffn_norm, T, d, c.norm_eps,
+                             h->B<bf16>("u"), h->B<float>("un"), st));
+    LAUNCH(h, K_ROUTER, 1,
+           run_router_logits(h->B<float>("un"), (const bf16*)w.w_router, T, d, c.n_experts,
+                             h->B<float>("router_logits"), st));
     GroupArgs ga;
     ga.idx = h->B<int>("idx");
     ga.w = h->B<float>("w");
@@ -358,8 +371,15 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     ga.ed_count = h->B<int>("tile_counts") + 1;
     ga.route_stats = h->B<unsigned long long>("route_stats");
     ga.err = err;
-    LAUNCH(h, K_GROUP, 1, run_group(ga, st));
-    LAUNCH(h, K_GATHER, 1, run_gather(h->B<bf16>("u"), h->B<int>("row_token"), T * k, d, h->B<bf16>("xp"), st));
+    {
+      const size_t mw = (size_t)c.n_experts * ((h->T_max + 31) / 32);
+      unsigned* masks = h->B<unsigned>("route_mask");
+      unsigned* cur = masks + (size_t)h->mask_flip * mw;
+      unsigned* nxt = masks + (size_t)(h->mask_flip ^ 1) * mw;
+      h->mask_flip ^= 1;
+      LAUNCH(h, K_GROUP, 2,
+             run_route(h->B<float>("router_logits"), h->B<bf16>("u"), d, h->B<bf16>("xp"), cur, nxt, ga, st));
+    }
 
     ExpertArgs ea;
     ea.tm_gate = &m.gate;
@@ -378,7 +398,7 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     ea.offsets = h->B<int>("offsets");
     ea.row_weight = h->B<float>("row_weight");
     ea.hp = h->B<bf16>("hp");
-    ea.yp = h->B<float>("yp");
+    ea.yp = yp;
     ea.err = err;
     LAUNCH(h, K_EGU, 1, run_experts_gate_up(ea, st));
     LAUNCH(h, K_ED, 1, run_experts_down(ea, st));
@@ -387,22 +407,32 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     sa.tm_u = &h->tm_u;
     sa.tm_gate = &m.sgate;
     sa.tm_up = &m.sup;
-    sa.tm_down = &m.sdown;
-    sa.tm_hs = &h->tm_hs;
     sa.T = T;
     sa.d = d;
     sa.fs = c.ffn_shared;
     sa.num_sms = h->num_sms;
     sa.hs = h->B<bf16>("hs");
-    sa.x = x;
     sa.err = err;
     LAUNCH(h, K_SGU, 1, run_shared_gate_up(sa, st));
-    LAUNCH(h, K_SD, 1, run_shared_down(sa, st));
+    WpartArgs da;
+    da.tm_w = &m.sdown;
+    da.tm_x = &h->tm_hs;
+    da.T = T;
+    da.Tcap = h->Tcap;
+    da.d = d;
+    da.K = c.ffn_shared;
+    da.splits = ss;
+    da.num_sms = h->num_sms;
+    da.part = part;
+    da.err = err;
+    LAUNCH(h, K_SD, 1, run_wpart(da, st));
     pending_k = k;
+    pending_parts = ss;
   }
   if (want_lm) {
     LAUNCH(h, K_RMSNORM, 1,
-           run_combine_rmsnorm(x, yp, pair_row, pending_k, h->final_norm, T, d, c.norm_eps, hn, st));
+           run_residual_norm(x, yp, pair_row, pending_k, part, pending_parts, h->Tcap, h->final_norm, T, d,
+                             c.norm_eps, hn, nullptr, st));
     LmArgs la;
     la.tm_x = &h->tm_hn;
     la.tm_embed = &h->tm_embed;
@@ -418,9 +448,11 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     LAUNCH(h, K_LMC, 1,
            run_lm_combine(h->B<float4>("lm_part"), grid, (T + 127) / 128, T, h->B<float>("stats"),
                           h->B<int>("argmax"), err, st));
-  } else if (pending_k) {
-    // a pass stopped after a full layer: fold its routed outputs into x
-    LAUNCH(h, K_RMSNORM, 1, run_combine_rmsnorm(x, yp, pair_row, pending_k, nullptr, T, d, c.norm_eps, nullptr, st));
+  } else if (pending_k || pending_parts) {
+    // a pass stopped after a full layer: fold its expert outputs into x
+    LAUNCH(h, K_RMSNORM, 1,
+           run_residual_norm(x, yp, pair_row, pending_k, part, pending_parts, h->Tcap, nullptr, T, d, c.norm_eps,
+                             nullptr, nullptr, st));
   }
   return DG_OK;
 }
@@ -508,16 +540,16 @@ int dg_init(const dg_config* cfg, const dg_weights* wts, int max_requests, int64
     ok = ok && make_map(&m.gate, w.w_gate, d, E * c.ffn_expert, 64);
     ok = ok && make_map(&m.up, w.w_up, d, E * c.ffn_expert, 64);
     ok = ok && make_map(&m.down, w.w_down, c.ffn_expert, E * d, 128);
-    ok = ok && make_map(&m.sgate, w.ws_gate, d, c.ffn_shared, 32);
-    ok = ok && make_map(&m.sup, w.ws_up, d, c.ffn_shared, 32);
+    ok = ok && make_map(&m.sgate, w.ws_gate, d, c.ffn_shared, 64);
+    ok = ok && make_map(&m.sup, w.ws_up, d, c.ffn_shared, 64);
     ok = ok && make_map(&m.sdown, w.ws_down, c.ffn_shared, d, 128);
   }
   ok = ok && make_map(&h->tm_hn, h->B<bf16>("hn"), d, h->Tcap, 128);
-  ok = ok && make_map(&h->tm_o, h->B<bf16>("o"), (long long)c.n_q_heads * D, h->Tcap, 64);
+  ok = ok && make_map(&h->tm_o, h->B<bf16>("o"), (long long)c.n_q_heads * D, h->Tcap, 256);
   ok = ok && make_map(&h->tm_u, h->B<bf16>("u"), d, h->Tcap, 128);
   ok = ok && make_map(&h->tm_xp, h->B<bf16>("xp"), d, rows, 64);
   ok = ok && make_map(&h->tm_hp, h->B<bf16>("hp"), c.ffn_expert, rows, 64);
-  ok = ok && make_map(&h->tm_hs, h->B<bf16>("hs"), c.ffn_shared, h->Tcap, 64);
+  ok = ok && make_map(&h->tm_hs, h->B<bf16>("hs"), c.ffn_shared, h->Tcap, 256);
   ok = ok && make_map(&h->tm_embed, h->embed, d, c.vocab, 256);
   {
     const long long kv_elems = (long long)max_requests * h->kv_req_stride;
@@ -535,6 +567,7 @@ int dg_init(const dg_config* cfg, const dg_weights* wts, int max_requests, int64
           cudaSuccess ||
       cudaMemsetAsync(h->B<int>("err"), 0, 64, h->st) != cudaSuccess ||
       cudaMemsetAsync(h->B<int>("route_stats"), 0, 64, h->st) != cudaSuccess ||
+      cudaMemsetAsync(h->B<int>("route_mask"), 0, h->plan.buf.at("route_mask").second, h->st) != cudaSuccess ||
       cudaMemsetAsync(h->B<bf16>("kv"), 0, h->plan.buf.at("kv").second, h->st) != cudaSuccess ||
       cudaMemsetAsync(h->B<int>("remaining"), 0, (size_t)max_requests * 4, h->st) != cudaSuccess ||
       cudaStreamSynchronize(h->st) != cudaSuccess) {
@@ -806,8 +839,8 @@ int dg_op_route_group(dg_handle* h, const int32_t* d_idx, const float* d_w, int 
   if (!h || T < 1 || T > h->T_max || !d_idx || !d_w) return DG_E_ARG;
   const dg_config& c = h->cfg;
   GroupArgs ga;
-  ga.idx = d_idx;
-  ga.w = d_w;
+  ga.idx = const_cast<int*>(d_idx);
+  ga.w = const_cast<float*>(d_w);
   ga.T = T;
   ga.k = c.top_k;
   ga.E = c.n_experts;

@@ -15,6 +15,23 @@ namespace dg {
 
 using bf16 = __nv_bfloat16;
 
+// Launch with programmatic stream serialization (see pdl_trigger / pdl_wait).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // ---- arguments of the tcgen05 GEMM launchers (gemm_ops.cu) ----
 struct QkvArgs {
   const CUtensorMap* tm_x;  // normed tokens [Tcap, d]
@@ -28,11 +45,12 @@ struct QkvArgs {
   bf16* kv;
   int* err;
 };
-struct OprojArgs {
-  const CUtensorMap* tm_w;
-  const CUtensorMap* tm_o;
-  int T, d, K, num_sms;
-  float* x;
+constexpr int kMaxPartSplits = 8;
+struct WpartArgs {
+  const CUtensorMap* tm_w;  // weights [d, K], 128-row boxes
+  const CUtensorMap* tm_x;  // activations [Tcap, K], 256-row boxes
+  int T, Tcap, d, K, splits, num_sms;
+  float* part;              // [splits][Tcap][d]
   int* err;
 };
 struct ExpertArgs {
@@ -50,10 +68,9 @@ struct ExpertArgs {
   int* err;
 };
 struct SharedArgs {
-  const CUtensorMap *tm_u, *tm_gate, *tm_up, *tm_down, *tm_hs;
+  const CUtensorMap *tm_u, *tm_gate, *tm_up;
   int T, d, fs, num_sms;
   bf16* hs;
-  float* x;
   int* err;
 };
 struct LmArgs {
@@ -67,11 +84,11 @@ struct LmArgs {
 };
 
 cudaError_t run_qkv(const QkvArgs& a, cudaStream_t st);
-cudaError_t run_oproj(const OprojArgs& a, cudaStream_t st);
+int wpart_splits(int d, int T, int K, int num_sms);
+cudaError_t run_wpart(const WpartArgs& a, cudaStream_t st);
 cudaError_t run_experts_gate_up(const ExpertArgs& a, cudaStream_t st);
 cudaError_t run_experts_down(const ExpertArgs& a, cudaStream_t st);
 cudaError_t run_shared_gate_up(const SharedArgs& a, cudaStream_t st);
-cudaError_t run_shared_down(const SharedArgs& a, cudaStream_t st);
 cudaError_t run_lm_head(const LmArgs& a, int* grid_out, cudaStream_t st);
 size_t gemm_smem_bytes_max();
 
@@ -86,15 +103,18 @@ struct SlotInfo {
 // ids[slot] points at the slot's Tr token ids
 cudaError_t run_embed(const int* const* ids, const SlotInfo& s, const bf16* embed, int V, int d, float* x, int* tok_pos,
                       int* tok_req, const double* inv_freq, int half, float2* rope, int* err, cudaStream_t st);
-cudaError_t run_combine_rmsnorm(float* x, const float* yp, const int* pair_row, int k, const float* g, int T, int d,
-                                float eps, bf16* out, cudaStream_t st);
+// x[t] += sum_j yp[pair_row[t*k+j]] + sum_s part[s][t]; then (if an output is
+// given) the RMSNorm of x[t] with gain g as bf16 and/or fp32
+cudaError_t run_residual_norm(float* x, const float* yp, const int* pair_row, int k, const float* part, int n_part,
+                              int Tcap, const float* g, int T, int d, float eps, bf16* out, float* out_f32,
+                              cudaStream_t st);
 cudaError_t run_rmsnorm(const float* x, const float* g, int T, int d, float eps, bf16* out, cudaStream_t st);
-cudaError_t run_router(const float* x, const float* g, float eps, const bf16* wr, int T, int d, int E, int k,
-                       bf16* u, float* logits, int* idx, float* w, cudaStream_t st);
+// router logits [T, E] from fp32 normalised rows un [T, d]
+cudaError_t run_router_logits(const float* un, const bf16* wr, int T, int d, int E, float* logits, cudaStream_t st);
 cudaError_t run_topk(const float* logits, int T, int E, int k, int* idx, float* w, cudaStream_t st);
 struct GroupArgs {
-  const int* idx;
-  const float* w;
+  int* idx;     // [T, k] selected experts (read by run_group, written by run_route)
+  float* w;     // [T, k] gate weights (read by run_group, written by run_route)
   int T, k, E, FJ, MD, egu_cap, ed_cap;
   int* counts;
   int* offsets;
@@ -110,6 +130,10 @@ struct GroupArgs {
   int* err;
 };
 cudaError_t run_group(const GroupArgs& a, cudaStream_t st);
+// top-k selection from logits (token bitmasks in `mask`, zeroed beforehand), then
+// the grouping above plus the gather of u rows into xp; clears `mask_next`
+cudaError_t run_route(const float* logits, const bf16* u, int d, bf16* xp, unsigned* mask, unsigned* mask_next,
+                      const GroupArgs& a, cudaStream_t st);
 cudaError_t run_gather(const bf16* u, const int* row_token, int rows, int d, bf16* xp, cudaStream_t st);
 cudaError_t run_lm_combine(const float4* part, int G, int MT, int T, float* stats, int* argmax, int* err,
                            cudaStream_t st);

@@ -2,13 +2,12 @@
 // each with its epilogue fused:
 //   qkv     RMSNorm'd tokens x W_qkv^T, rotate-half RoPE on q/k, q -> [Hq][T][D],
 //           k/v -> KV cache slots of the canvas (or prefill segment)
-//   oproj   x += O W_o^T                               (weights as the 128-row operand)
+//   wpart   split-K weight-row GEMM to fp32 partials (output projection and
+//           shared-expert down projection; reduced by the residual + norm kernel)
 //   egu     routed experts, gate|up for 64 hidden units per tile, SwiGLU in the
 //           epilogue (weights as the 128-row operand, the expert's tokens as N)
 //   ed      routed experts, down projection scaled by the pair's routing weight
 //   sgu     shared expert gate|up + SwiGLU (tokens as the 128-row operand)
-//   sd      shared expert down + residual (the routed outputs are summed into the
-//           residual by the next combine + RMSNorm kernel)
 //   lm      tied LM head with per-row online max / argmax / sum e^(z-m) /
 //           sum e^(z-m)(z-m) so the logits are never written
 // Structure of a decoder layer and the MoE: DiffusionGemma pages ("26B MoE
@@ -104,6 +103,20 @@ struct P_QKV : ProblemBase {
     tma_load_2d(sb, &p.tmB, kb * 64, r0, bar);
     tma_load_2d(sb + 64 * 128, &p.tmB, kb * 64, r1, bar);
   }
+  DG_DEVINL static void epilogue_prefetch(const Params& p, const Tile& t, int row) {
+    const int tok = t.a * 128 + row;
+    if (tok >= p.T) return;
+    prefetch_l1(p.tok_pos + tok);
+    prefetch_l1(p.tok_req + tok);
+    int kind, tb, r0, r1;
+    rows_of(p, t.b, kind, tb, r0, r1);
+    if (kind == 2) return;
+    const int half = p.D >> 1;
+    const int j = p.D == 256 ? (tb & 1) : 0;
+    const char* cs = reinterpret_cast<const char*>(p.rope + (size_t)tok * half + (p.D == 64 ? 0 : j * 64));
+    const int bytes = (p.D == 64 ? 32 : 64) * 8;
+    for (int o = 0; o < bytes; o += 128) prefetch_l1(cs + o);
+  }
   DG_DEVINL static void rotate16(const float* x1, const float* x2, const float2* cs, float* y1, float* y2) {
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
@@ -178,56 +191,57 @@ struct P_QKV : ProblemBase {
 };
 
 // ---------------------------------------------------------------------------
-// Residual update x[t, f] += acc[f, t] for one 16-token chunk of an epilogue
-// row: the 16 residual loads are issued together, then the 16 stores.
+// Split-K weight-row GEMM with fp32 partial output, shared by the output
+// projection and the shared expert's down projection:
+//   part[s][t][f] = sum_{c in K-slice s} X[t, c] W[f, c]
+// Tile (128 output features a, 256 tokens b, K-slice s).  N = 256 keeps the
+// tensor core fed (the weight slice read per MMA is amortised over all
+// tokens); the K split gives enough CTAs.  The slices are summed, in slice
+// order, into the residual stream by the next residual + norm kernel.
 // ---------------------------------------------------------------------------
-DG_DEVINL void residual_add16(float* x, int d, int f, int tok0, int T, const float* v) {
-  float xv[16];
-#pragma unroll
-  for (int j = 0; j < 16; ++j) xv[j] = tok0 + j < T ? x[(size_t)(tok0 + j) * d + f] : 0.f;
-#pragma unroll
-  for (int j = 0; j < 16; ++j)
-    if (tok0 + j < T) x[(size_t)(tok0 + j) * d + f] = xv[j] + v[j];
-}
-
-// ---------------------------------------------------------------------------
-// Output projection + residual: x[t, f] += sum_c O[t, c] W_o[f, c].
-// Tile (128 output features a, 64 tokens b).
-// ---------------------------------------------------------------------------
-struct P_OPROJ : ProblemBase {
-  static constexpr int BN = 64, STAGES = 8, B_STAGE = BN * 128, TMEM_COLS = 128;
+struct P_WPART : ProblemBase {
+  static constexpr int BN = 256, STAGES = 4, B_STAGE = BN * 128, TMEM_COLS = 512;
   struct Params {
-    CUtensorMap tmA;  // w_o [d, Hq*D]
-    CUtensorMap tmB;  // O [Tcap, Hq*D], 64-row boxes
-    int T, nk, MT, NT, d;
-    float* x;
+    CUtensorMap tmA;  // weights [d, K], 128-row boxes
+    CUtensorMap tmB;  // activations [Tcap, K], 256-row boxes
+    int T, nk, MT, NT, S, Tcap, d;
+    float* part;  // [S][Tcap][d]
     int* err;
   };
   DG_DEVINL static void prefetch(const Params& p) {
     tma_prefetch_desc(&p.tmA);
     tma_prefetch_desc(&p.tmB);
   }
-  DG_DEVINL static int num_tiles(const Params& p) { return p.MT * p.NT; }
+  DG_DEVINL static int num_tiles(const Params& p) { return p.MT * p.NT * p.S; }
   DG_DEVINL static Tile tile(const Params& p, int v) {
     Tile t;
-    t.valid = 1;
-    t.nk = p.nk;
-    t.b = v % p.NT;  // token tile
-    t.a = v / p.NT;  // 128 output features
+    t.a = v % p.MT;              // feature tile
+    const int rest = v / p.MT;
+    t.b = rest % p.NT;           // token tile
+    t.c = rest / p.NT;           // K slice
+    const int per = (p.nk + p.S - 1) / p.S;
+    t.d = t.c * per;             // first k-block
+    t.nk = min(per, p.nk - t.d);
+    t.valid = t.nk > 0;
     t.n_mma = round_up16(min(BN, p.T - t.b * BN));
     return t;
   }
   DG_DEVINL static uint32_t tx_bytes(const Params&, const Tile&) { return kAStage + B_STAGE; }
   DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
-    tma_load_2d(sa, &p.tmA, kb * 64, t.a * 128, bar);
-    tma_load_2d(sb, &p.tmB, kb * 64, t.b * BN, bar);
+    tma_load_2d(sa, &p.tmA, (t.d + kb) * 64, t.a * 128, bar);
+    tma_load_2d(sb, &p.tmB, (t.d + kb) * 64, t.b * BN, bar);
   }
   DG_DEVINL static void epilogue(const Params& p, const Tile& t, uint32_t taddr, int, int, int row, uint8_t*) {
     const int f = t.a * 128 + row;
+    float* dst = p.part + (size_t)t.c * p.Tcap * p.d + f;
     for (int c0 = 0; c0 < t.n_mma; c0 += 16) {
       float v[16];
       tmem_ld16(taddr + c0, v);
-      residual_add16(p.x, p.d, f, t.b * BN + c0, p.T, v);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int tok = t.b * BN + c0 + j;
+        if (tok < p.T) dst[(size_t)tok * p.d] = v[j];
+      }
     }
   }
 };
@@ -365,14 +379,14 @@ struct P_ED : ProblemBase {
 
 // ---------------------------------------------------------------------------
 // Shared expert gate|up + SwiGLU.  Tile (mt, j): tokens mt*128..+127, hidden
-// units j*32..+31; B rows 0..31 = gate rows, 32..63 = up rows.
+// units j*64..+63; B rows 0..63 = gate rows, 64..127 = up rows.
 // ---------------------------------------------------------------------------
 struct P_SGU : ProblemBase {
-  static constexpr int BN = 64, STAGES = 8, B_STAGE = BN * 128, TMEM_COLS = 128;
+  static constexpr int BN = 128, STAGES = 6, B_STAGE = BN * 128, TMEM_COLS = 256;
   struct Params {
     CUtensorMap tmX;  // normed tokens [Tcap, d]
-    CUtensorMap tmG;  // ws_gate [fs, d], 32-row boxes
-    CUtensorMap tmU;  // ws_up [fs, d], 32-row boxes
+    CUtensorMap tmG;  // ws_gate [fs, d], 64-row boxes
+    CUtensorMap tmU;  // ws_up [fs, d], 64-row boxes
     int T, nk, MT, FJ, fs;
     __nv_bfloat16* hs;  // [Tcap, fs]
     int* err;
@@ -395,65 +409,22 @@ struct P_SGU : ProblemBase {
   DG_DEVINL static uint32_t tx_bytes(const Params&, const Tile&) { return kAStage + B_STAGE; }
   DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
     tma_load_2d(sa, &p.tmX, kb * 64, t.a * 128, bar);
-    tma_load_2d(sb, &p.tmG, kb * 64, t.b * 32, bar);
-    tma_load_2d(sb + 32 * 128, &p.tmU, kb * 64, t.b * 32, bar);
+    tma_load_2d(sb, &p.tmG, kb * 64, t.b * 64, bar);
+    tma_load_2d(sb + 64 * 128, &p.tmU, kb * 64, t.b * 64, bar);
   }
   DG_DEVINL static void epilogue(const Params& p, const Tile& t, uint32_t taddr, int, int, int row, uint8_t*) {
     const int tok = t.a * 128 + row;
     const bool ok = tok < p.T;
-    for (int c0 = 0; c0 < 32; c0 += 16) {
+    for (int c0 = 0; c0 < 64; c0 += 16) {
       float g[16], u[16];
       tmem_ld16(taddr + c0, g);
-      tmem_ld16(taddr + 32 + c0, u);
+      tmem_ld16(taddr + 64 + c0, u);
       if (ok) {
         float h[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) h[i] = silu_f(g[i]) * u[i];
-        store_bf16x16(p.hs + (size_t)tok * p.fs + t.b * 32 + c0, h);
+        store_bf16x16(p.hs + (size_t)tok * p.fs + t.b * 64 + c0, h);
       }
-    }
-  }
-};
-
-// ---------------------------------------------------------------------------
-// Shared expert down + residual: x[t, f] += (Hs W_sd^T)[t, f].  The routed
-// experts' outputs are added by the next combine + RMSNorm kernel.
-// Tile (128 output features a, 64 tokens b).
-// ---------------------------------------------------------------------------
-struct P_SD : ProblemBase {
-  static constexpr int BN = 64, STAGES = 8, B_STAGE = BN * 128, TMEM_COLS = 128;
-  struct Params {
-    CUtensorMap tmW;  // ws_down [d, fs]
-    CUtensorMap tmH;  // Hs [Tcap, fs], 64-row boxes
-    int T, nk, MT, NT, d;
-    float* x;
-    int* err;
-  };
-  DG_DEVINL static void prefetch(const Params& p) {
-    tma_prefetch_desc(&p.tmW);
-    tma_prefetch_desc(&p.tmH);
-  }
-  DG_DEVINL static int num_tiles(const Params& p) { return p.MT * p.NT; }
-  DG_DEVINL static Tile tile(const Params& p, int v) {
-    Tile t;
-    t.valid = 1;
-    t.nk = p.nk;
-    t.b = v % p.NT;
-    t.a = v / p.NT;
-    t.n_mma = round_up16(min(BN, p.T - t.b * BN));
-    return t;
-  }
-  DG_DEVINL static uint32_t tx_bytes(const Params&, const Tile&) { return kAStage + B_STAGE; }
-  DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
-    tma_load_2d(sa, &p.tmW, kb * 64, t.a * 128, bar);
-    tma_load_2d(sb, &p.tmH, kb * 64, t.b * BN, bar);
-  }
-  DG_DEVINL static void epilogue(const Params& p, const Tile& t, uint32_t taddr, int, int, int row, uint8_t*) {
-    const int f = t.a * 128 + row;
-    for (int c0 = 0; c0 < t.n_mma; c0 += 16) {
-      float v[16];
-      tmem_ld16(taddr + c0, v);
-      residual_add16(p.x, p.d, f, t.b * BN + c0, p.T, v);
     }
   }
 };
@@ -570,8 +541,7 @@ static cudaError_t launch_gemm(const typename P::Params& p, int grid, cudaStream
     configured = true;
   }
   if (grid <= 0) return cudaSuccess;
-  k_umma_gemm<P><<<grid, 192, smem, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(k_umma_gemm<P>, dim3(grid), dim3(192), smem, st, p);
 }
 
 static int grid_for(int tiles, int sms) { return tiles < sms ? tiles : sms; }
@@ -599,18 +569,30 @@ cudaError_t run_qkv(const QkvArgs& a, cudaStream_t st) {
   return launch_gemm<P_QKV>(p, grid_for(p.MT * p.NT, a.num_sms), st);
 }
 
-cudaError_t run_oproj(const OprojArgs& a, cudaStream_t st) {
-  P_OPROJ::Params p;
+// K split so that feature tiles x token tiles x splits fills the GPU once.
+int wpart_splits(int d, int T, int K, int num_sms) {
+  const int tiles = (d / 128) * ((T + 255) / 256);
+  int s = num_sms / tiles;
+  const int nk = K / 64;
+  if (s > nk) s = nk;
+  if (s > kMaxPartSplits) s = kMaxPartSplits;
+  return s < 1 ? 1 : s;
+}
+
+cudaError_t run_wpart(const WpartArgs& a, cudaStream_t st) {
+  P_WPART::Params p;
   p.tmA = *a.tm_w;
-  p.tmB = *a.tm_o;
+  p.tmB = *a.tm_x;
   p.T = a.T;
   p.nk = a.K / 64;
   p.MT = a.d / 128;
-  p.NT = (a.T + P_OPROJ::BN - 1) / P_OPROJ::BN;
+  p.NT = (a.T + P_WPART::BN - 1) / P_WPART::BN;
+  p.S = a.splits;
+  p.Tcap = a.Tcap;
   p.d = a.d;
-  p.x = a.x;
+  p.part = a.part;
   p.err = a.err;
-  return launch_gemm<P_OPROJ>(p, grid_for(p.MT * p.NT, a.num_sms), st);
+  return launch_gemm<P_WPART>(p, grid_for(p.MT * p.NT * p.S, a.num_sms), st);
 }
 
 cudaError_t run_experts_gate_up(const ExpertArgs& a, cudaStream_t st) {
@@ -653,25 +635,11 @@ cudaError_t run_shared_gate_up(const SharedArgs& a, cudaStream_t st) {
   g.T = a.T;
   g.nk = a.d / 64;
   g.MT = (a.T + 127) / 128;
-  g.FJ = a.fs / 32;
+  g.FJ = a.fs / 64;
   g.fs = a.fs;
   g.hs = a.hs;
   g.err = a.err;
   return launch_gemm<P_SGU>(g, grid_for(g.MT * g.FJ, a.num_sms), st);
-}
-
-cudaError_t run_shared_down(const SharedArgs& a, cudaStream_t st) {
-  P_SD::Params dn;
-  dn.tmW = *a.tm_down;
-  dn.tmH = *a.tm_hs;
-  dn.T = a.T;
-  dn.nk = a.fs / 64;
-  dn.MT = a.d / 128;
-  dn.NT = (a.T + P_SD::BN - 1) / P_SD::BN;
-  dn.d = a.d;
-  dn.x = a.x;
-  dn.err = a.err;
-  return launch_gemm<P_SD>(dn, grid_for(dn.MT * dn.NT, a.num_sms), st);
 }
 
 cudaError_t run_lm_head(const LmArgs& a, int* grid_out, cudaStream_t st) {
@@ -694,11 +662,10 @@ cudaError_t run_lm_head(const LmArgs& a, int* grid_out, cudaStream_t st) {
 
 size_t gemm_smem_bytes_max() {
   size_t m = GemmSmem<P_QKV>::total;
-  m = m > GemmSmem<P_OPROJ>::total ? m : GemmSmem<P_OPROJ>::total;
+  m = m > GemmSmem<P_WPART>::total ? m : GemmSmem<P_WPART>::total;
   m = m > GemmSmem<P_EGU>::total ? m : GemmSmem<P_EGU>::total;
   m = m > GemmSmem<P_ED>::total ? m : GemmSmem<P_ED>::total;
   m = m > GemmSmem<P_SGU>::total ? m : GemmSmem<P_SGU>::total;
-  m = m > GemmSmem<P_SD>::total ? m : GemmSmem<P_SD>::total;
   m = m > GemmSmem<P_LM>::total ? m : GemmSmem<P_LM>::total;
   return m;
 }

@@ -19,6 +19,8 @@ struct EmbedParams {
 __global__ void k_embed(EmbedParams p, const bf16* __restrict__ embed, int V, int d, float* __restrict__ x,
                         int* tok_pos, int* tok_req, const double* __restrict__ inv_freq, int half,
                         float2* __restrict__ rope, int* err) {
+  pdl_trigger();
+  pdl_wait();
   const int t = blockIdx.x;
   const int slot = t / p.s.Tr;
   const int i = t - slot * p.s.Tr;
@@ -61,7 +63,10 @@ cudaError_t run_embed(const int* const* ids, const SlotInfo& s, const bf16* embe
   for (int i = 0; i < DG_MAX_REQUESTS; ++i) p.ids[i] = i < s.n ? ids[i] : nullptr;
   const int T = s.n * s.Tr;
   if (T == 0) return cudaSuccess;
-  k_embed<<<T, 128, 0, st>>>(p, embed, V, d, x, tok_pos, tok_req, inv_freq, half, rope, err);
+  {
+    const cudaError_t e_ = launch_pdl(k_embed, dim3(T), dim3(128), 0, st, p, embed, V, d, x, tok_pos, tok_req, inv_freq, half, rope, err);
+    if (e_ != cudaSuccess) return e_;
+  }
   return cudaGetLastError();
 }
 
@@ -70,6 +75,8 @@ cudaError_t run_embed(const int* const* ids, const SlotInfo& s, const bf16* embe
 // ---------------------------------------------------------------------------
 __global__ void k_rmsnorm(const float* __restrict__ x, const float* __restrict__ g, int T, int d, float eps,
                           bf16* __restrict__ out) {
+  pdl_trigger();
+  pdl_wait();
   const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= T) return;
@@ -92,20 +99,27 @@ __global__ void k_rmsnorm(const float* __restrict__ x, const float* __restrict__
 
 cudaError_t run_rmsnorm(const float* x, const float* g, int T, int d, float eps, bf16* out, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
-  k_rmsnorm<<<(T + 7) / 8, 256, 0, st>>>(x, g, T, d, eps, out);
+  {
+    const cudaError_t e_ = launch_pdl(k_rmsnorm, dim3((T + 7) / 8), dim3(256), 0, st, x, g, T, d, eps, out);
+    if (e_ != cudaSuccess) return e_;
+  }
   return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------
-// Routed-expert combine + RMSNorm, one CTA per token row:
-//   x[t] += sum_j Yp[row(t, j)]   (k = 0: nothing to combine)
-//   out[t] = bf16(x[t] / sqrt(mean(x[t]^2) + eps) * g)
-// The k expert outputs are added in slot order (deterministic).
+// Residual update + RMSNorm, one CTA per token row:
+//   x[t] += sum_j Yp[row(t, j)] + sum_s part[s][t]
+//   out[t] = bf16(x[t] / sqrt(mean(x[t]^2) + eps) * g), out_f32[t] likewise in fp32
+// The routed experts' outputs (slot order) and the split-K partials (slice
+// order) are added in a fixed order, so the result is deterministic.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) k_combine_rmsnorm(float* __restrict__ x, const float* __restrict__ yp,
-                                                         const int* __restrict__ pair_row, int k,
-                                                         const float* __restrict__ g, int d, float eps,
-                                                         bf16* __restrict__ out) {
+__global__ void __launch_bounds__(256) k_residual_norm(float* __restrict__ x, const float* __restrict__ yp,
+                                                       const int* __restrict__ pair_row, int k,
+                                                       const float* __restrict__ part, int n_part, size_t part_stride,
+                                                       const float* __restrict__ g, int d, float eps,
+                                                       bf16* __restrict__ out, float* __restrict__ out_f32) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ float crow[];  // [d]
   __shared__ float red[8];
   const int t = blockIdx.x;
@@ -117,10 +131,13 @@ __global__ void __launch_bounds__(256) k_combine_rmsnorm(float* __restrict__ x, 
   float ss = 0.f;
   for (int c = threadIdx.x; c < d / 4; c += blockDim.x) {
     float4 v = xr[c];
-    float4 y[8];
+    float4 y[8], q[kMaxPartSplits];
 #pragma unroll
     for (int j = 0; j < 8; ++j)
       if (j < k) y[j] = reinterpret_cast<const float4*>(yp + (size_t)rows[j] * d)[c];
+#pragma unroll
+    for (int j = 0; j < kMaxPartSplits; ++j)
+      if (j < n_part) q[j] = reinterpret_cast<const float4*>(part + j * part_stride + (size_t)t * d)[c];
 #pragma unroll
     for (int j = 0; j < 8; ++j)
       if (j < k) {
@@ -129,11 +146,19 @@ __global__ void __launch_bounds__(256) k_combine_rmsnorm(float* __restrict__ x, 
         v.z += y[j].z;
         v.w += y[j].w;
       }
-    if (k) xr[c] = v;
+#pragma unroll
+    for (int j = 0; j < kMaxPartSplits; ++j)
+      if (j < n_part) {
+        v.x += q[j].x;
+        v.y += q[j].y;
+        v.z += q[j].z;
+        v.w += q[j].w;
+      }
+    if (k || n_part) xr[c] = v;
     cr[c] = v;
     ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
   }
-  if (out == nullptr) return;
+  if (out == nullptr && out_f32 == nullptr) return;
   ss = warp_sum(ss);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
   __syncthreads();
@@ -145,25 +170,32 @@ __global__ void __launch_bounds__(256) k_combine_rmsnorm(float* __restrict__ x, 
   __syncthreads();
   const float rs = rsqrtf(red[0] / (float)d + eps);
   const float4* g4 = reinterpret_cast<const float4*>(g);
-  uint2* o = reinterpret_cast<uint2*>(out + (size_t)t * d);
   for (int c = threadIdx.x; c < d / 4; c += blockDim.x) {
     const float4 v = cr[c];
     const float4 w = g4[c];
-    o[c] = make_uint2(pack_bf16x2(v.x * rs * w.x, v.y * rs * w.y), pack_bf16x2(v.z * rs * w.z, v.w * rs * w.w));
+    const float4 n = make_float4(v.x * rs * w.x, v.y * rs * w.y, v.z * rs * w.z, v.w * rs * w.w);
+    if (out)
+      reinterpret_cast<uint2*>(out + (size_t)t * d)[c] = make_uint2(pack_bf16x2(n.x, n.y), pack_bf16x2(n.z, n.w));
+    if (out_f32) reinterpret_cast<float4*>(out_f32 + (size_t)t * d)[c] = n;
   }
 }
 
-cudaError_t run_combine_rmsnorm(float* x, const float* yp, const int* pair_row, int k, const float* g, int T, int d,
-                                float eps, bf16* out, cudaStream_t st) {
+cudaError_t run_residual_norm(float* x, const float* yp, const int* pair_row, int k, const float* part, int n_part,
+                              int Tcap, const float* g, int T, int d, float eps, bf16* out, float* out_f32,
+                              cudaStream_t st) {
   if (T == 0) return cudaSuccess;
+  if (n_part > kMaxPartSplits || k > 8) return cudaErrorInvalidValue;
   const size_t smem = (size_t)d * sizeof(float);
   static size_t configured = 0;
   if (smem > 48 * 1024 && smem > configured) {
-    cudaError_t e = cudaFuncSetAttribute(k_combine_rmsnorm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(k_residual_norm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     configured = smem;
   }
-  k_combine_rmsnorm<<<T, 256, smem, st>>>(x, yp, pair_row, k, g, d, eps, out);
+  {
+    const cudaError_t e_ = launch_pdl(k_residual_norm, dim3(T), dim3(256), smem, st, x, yp, pair_row, k, part, n_part, (size_t)Tcap * d, g, d, eps, out, out_f32);
+    if (e_ != cudaSuccess) return e_;
+  }
   return cudaGetLastError();
 }
 
@@ -222,6 +254,8 @@ DG_DEVINL void topk_warp(const float* vals, int E, int k, int* idx_out, float* w
 }
 
 __global__ void k_topk(const float* __restrict__ logits, int T, int E, int k, int* idx, float* w) {
+  pdl_trigger();
+  pdl_wait();
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;
   topk_warp(logits + (size_t)t * E, E, k, idx + (size_t)t * k, w + (size_t)t * k);
@@ -229,70 +263,77 @@ __global__ void k_topk(const float* __restrict__ logits, int T, int E, int k, in
 
 cudaError_t run_topk(const float* logits, int T, int E, int k, int* idx, float* w, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
-  k_topk<<<(T + 7) / 8, 256, 0, st>>>(logits, T, E, k, idx, w);
+  {
+    const cudaError_t e_ = launch_pdl(k_topk, dim3((T + 7) / 8), dim3(256), 0, st, logits, T, E, k, idx, w);
+    if (e_ != cudaSuccess) return e_;
+  }
   return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------
-// FFN RMSNorm + router logits.  Grid (token groups of kRT, expert groups of
-// kRE): each CTA normalises its kRT rows in fp32 (the CTA of expert group 0
-// also writes the bf16 copy the experts read) and computes their logits
-// against kRE router rows, fp32 row x bf16 weights with fp32 accumulation.
-// Each warp owns 4 experts so every lane keeps 4 independent weight loads in
-// flight.  The top-k selection follows in k_topk.
+// Router logits from the fp32 normalised rows: grid (token groups of kRT,
+// expert groups of kRE); fp32 row x bf16 router weights, fp32 accumulation.
+// Each warp owns 2 experts for all kRT tokens of the CTA.
 // ---------------------------------------------------------------------------
-constexpr int kRT = 8, kRE = 32;
+constexpr int kRT = 8, kRE = 16;
 
-__global__ void __launch_bounds__(256) k_router_logits(const float* __restrict__ x, const float* __restrict__ g,
-                                                       float eps, const bf16* __restrict__ wr, int T, int d, int E,
-                                                       bf16* __restrict__ u, float* __restrict__ logits) {
+__global__ void __launch_bounds__(256) k_router_logits(const float* __restrict__ un, const bf16* __restrict__ wr,
+                                                       int T, int d, int E, float* __restrict__ logits) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ float su[];  // [kRT][d]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t0 = blockIdx.x * kRT, e0 = blockIdx.y * kRE;
-  if (warp < kRT) {
-    const int t = t0 + warp;
-    float* dst = su + warp * d;
-    if (t < T) {
-      const float4* xr = reinterpret_cast<const float4*>(x + (size_t)t * d);
-      float ss = 0.f;
-      for (int c = lane; c < d / 4; c += 32) {
-        const float4 v = xr[c];
-        ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
-      }
-      ss = warp_sum(ss);
-      const float rs = rsqrtf(ss / (float)d + eps);
-      const float4* g4 = reinterpret_cast<const float4*>(g);
-      uint2* uo = reinterpret_cast<uint2*>(u + (size_t)t * d);
-      for (int c = lane; c < d / 4; c += 32) {
-        const float4 v = xr[c];
-        const float4 gg = g4[c];
-        const float4 n = make_float4(v.x * rs * gg.x, v.y * rs * gg.y, v.z * rs * gg.z, v.w * rs * gg.w);
-        if (blockIdx.y == 0) uo[c] = make_uint2(pack_bf16x2(n.x, n.y), pack_bf16x2(n.z, n.w));
-        reinterpret_cast<float4*>(dst)[c] = n;
-      }
-    } else {
-      for (int c = lane; c < d; c += 32) dst[c] = 0.f;
+  const int d4 = d / 4;
+  // stage the rows in batches of 8 independent 16-byte loads per thread
+  for (int base = threadIdx.x; base < kRT * d4; base += 8 * blockDim.x) {
+    float4 r[8];
+#pragma unroll
+    for (int b = 0; b < 8; ++b) {
+      const int i = base + b * blockDim.x;
+      const int tt = i / d4, c = i - tt * d4;
+      r[b] = (i < kRT * d4 && t0 + tt < T) ? reinterpret_cast<const float4*>(un + (size_t)(t0 + tt) * d)[c]
+                                           : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int b = 0; b < 8; ++b) {
+      const int i = base + b * blockDim.x;
+      if (i < kRT * d4) reinterpret_cast<float4*>(su)[i] = r[b];
     }
   }
   __syncthreads();
-  float acc[4][kRT];
+  const int eb = e0 + warp * 2;
+  // every weight this lane needs, loaded up front (all loads in flight at once)
+  constexpr int kMaxChunks = 16;  // d <= 4096
+  const int n_chunks = (d + 255) / 256;
+  uint4 wv[2][kMaxChunks];
 #pragma unroll
-  for (int q = 0; q < 4; ++q)
+  for (int i = 0; i < kMaxChunks; ++i)
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int c = lane * 8 + i * 256;
+      wv[q][i] = (i < n_chunks && c < d && eb + q < E)
+                     ? __ldg(reinterpret_cast<const uint4*>(wr + (size_t)(eb + q) * d + c))
+                     : make_uint4(0, 0, 0, 0);
+    }
+  float acc[2][kRT];
+#pragma unroll
+  for (int q = 0; q < 2; ++q)
 #pragma unroll
     for (int tt = 0; tt < kRT; ++tt) acc[q][tt] = 0.f;
-  const int eb = e0 + warp * 4;
-  for (int c = lane * 8; c < d; c += 256) {
-    float wf[4][8];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      uint4 wv = make_uint4(0, 0, 0, 0);
-      if (eb + q < E) wv = *reinterpret_cast<const uint4*>(wr + (size_t)(eb + q) * d + c);
-      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&wv);
+  for (int i = 0; i < kMaxChunks; ++i) {
+    const int c = lane * 8 + i * 256;
+    if (i >= n_chunks || c >= d) break;
+    float wf[2][8];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 f2 = __bfloat1622float2(h[i]);
-        wf[q][2 * i] = f2.x;
-        wf[q][2 * i + 1] = f2.y;
+    for (int q = 0; q < 2; ++q) {
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&wv[q][i]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f2 = __bfloat1622float2(h[j]);
+        wf[q][2 * j] = f2.x;
+        wf[q][2 * j + 1] = f2.y;
       }
     }
 #pragma unroll
@@ -300,7 +341,7 @@ __global__ void __launch_bounds__(256) k_router_logits(const float* __restrict__
       const float4 a = *reinterpret_cast<const float4*>(su + tt * d + c);
       const float4 b = *reinterpret_cast<const float4*>(su + tt * d + c + 4);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < 2; ++q) {
         float r = acc[q][tt];
         r = fmaf(a.x, wf[q][0], r);
         r = fmaf(a.y, wf[q][1], r);
@@ -315,7 +356,7 @@ __global__ void __launch_bounds__(256) k_router_logits(const float* __restrict__
     }
   }
 #pragma unroll
-  for (int q = 0; q < 4; ++q)
+  for (int q = 0; q < 2; ++q)
 #pragma unroll
     for (int tt = 0; tt < kRT; ++tt) {
       const float r = warp_sum(acc[q][tt]);
@@ -323,8 +364,7 @@ __global__ void __launch_bounds__(256) k_router_logits(const float* __restrict__
     }
 }
 
-cudaError_t run_router(const float* x, const float* g, float eps, const bf16* wr, int T, int d, int E, int k, bf16* u,
-                       float* logits, int* idx, float* w, cudaStream_t st) {
+cudaError_t run_router_logits(const float* un, const bf16* wr, int T, int d, int E, float* logits, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
   const size_t smem = (size_t)kRT * d * sizeof(float);
   static size_t configured = 0;
@@ -334,10 +374,11 @@ cudaError_t run_router(const float* x, const float* g, float eps, const bf16* wr
     configured = smem;
   }
   dim3 grid((T + kRT - 1) / kRT, (E + kRE - 1) / kRE);
-  k_router_logits<<<grid, 256, smem, st>>>(x, g, eps, wr, T, d, E, u, logits);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  return run_topk(logits, T, E, k, idx, w, st);
+  {
+    const cudaError_t e_ = launch_pdl(k_router_logits, dim3(grid), dim3(256), smem, st, un, wr, T, d, E, logits);
+    if (e_ != cudaSuccess) return e_;
+  }
+  return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------
@@ -346,6 +387,8 @@ cudaError_t run_router(const float* x, const float* g, float eps, const bf16* wr
 // an expert, via per-expert token bitmasks), and the GEMM tile lists.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024) k_group(GroupArgs a) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ int gsm[];
   const int E = a.E, T = a.T, k = a.k;
   const int MW = (T + 31) >> 5;
@@ -428,7 +471,194 @@ cudaError_t run_group(const GroupArgs& a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     configured = smem;
   }
-  k_group<<<1, 1024, smem, st>>>(a);
+  {
+    const cudaError_t e_ = launch_pdl(k_group, dim3(1), dim3(1024), smem, st, a);
+    if (e_ != cudaSuccess) return e_;
+  }
+  return cudaGetLastError();
+}
+
+// Exclusive scan of 8 consecutive values per lane across a warp (256 values);
+// rewrites vals8 with the exclusive prefixes and returns the total.
+DG_DEVINL int warp_excl_scan8(int* vals8, int lane) {
+  int run = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int v = vals8[i];
+    vals8[i] = run;
+    run += v;
+  }
+  int incl = run;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  const int base = incl - run;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) vals8[i] += base;
+  return __shfl_sync(0xffffffffu, incl, 31);
+}
+
+// ---------------------------------------------------------------------------
+// Routing, part 1: top-k of every token's logits (one warp per token); each
+// selected (token, expert) sets bit t of that expert's token bitmask.
+// ---------------------------------------------------------------------------
+__global__ void k_topk_mask(const float* __restrict__ logits, int T, int E, int k, int* idx, float* w,
+                            unsigned* __restrict__ mask, int MW) {
+  pdl_trigger();
+  pdl_wait();
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  int* it = idx + (size_t)t * k;
+  float* wt = w + (size_t)t * k;
+  topk_warp(logits + (size_t)t * E, E, k, it, wt);
+  __syncwarp();
+  const int lane = threadIdx.x & 31;
+  if (lane < k) {
+    const int e = it[lane];
+    if (e >= 0 && e < E) atomicOr(&mask[(size_t)e * MW + (t >> 5)], 1u << (t & 31));
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Routing, part 2 (every CTA): per-expert counts from the bitmasks and their
+// exclusive scans (tiny, recomputed by each CTA); CTA 0 publishes counts,
+// offsets, tile lists and statistics.  Each CTA then places its share of the
+// (token, slot) pairs -- row = offset[e] + number of earlier tokens routed to
+// e, so tokens ascend inside an expert -- and copies the token's normalised
+// row into the expert-grouped buffer.  It also clears the other mask buffer
+// (used by the previous layer, read by nobody now) for the next layer.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_group_gather(GroupArgs a, const unsigned* __restrict__ mask,
+                                                      unsigned* __restrict__ mask_next, int MW,
+                                                      const bf16* __restrict__ u, int d, bf16* __restrict__ xp) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ int cnt[256];
+  __shared__ int off[257];
+  __shared__ int toff[257];
+  const int E = a.E, T = a.T, k = a.k, P = T * k;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int e = tid; e < E; e += blockDim.x) {
+    int c = 0;
+    for (int wi = 0; wi < MW; ++wi) c += __popc(mask[(size_t)e * MW + wi]);
+    cnt[e] = c;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int v[8], tv[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = lane * 8 + i;
+      v[i] = e < E ? cnt[e] : 0;
+      tv[i] = e < E ? (cnt[e] + 63) / 64 : 0;
+    }
+    const int tot = warp_excl_scan8(v, lane);
+    const int ttot = warp_excl_scan8(tv, lane);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = lane * 8 + i;
+      if (e < E) {
+        off[e] = v[i];
+        toff[e] = tv[i];
+      }
+    }
+    if (lane == 0) {
+      off[E] = tot;
+      toff[E] = ttot;
+      if (blockIdx.x == 0) {
+        const int egu = ttot * a.FJ, ed = ttot * a.MD;
+        if (egu > a.egu_cap || ed > a.ed_cap || tot != P) atomicOr(a.err, DG_DEVERR_CAPACITY);
+        *a.egu_count = min(egu, a.egu_cap);
+        *a.ed_count = min(ed, a.ed_cap);
+      }
+    }
+  }
+  __syncthreads();
+  if (blockIdx.x == 0) {
+    int touched = 0;
+    for (int e = tid; e < E; e += blockDim.x) {
+      a.counts[e] = cnt[e];
+      a.offsets[e] = off[e];
+      touched += cnt[e] > 0;
+    }
+    if (tid == 0) a.offsets[E] = off[E];
+    if (a.route_stats) {
+      touched = warp_sum_int(touched);
+      if (lane == 0) atomicAdd(&a.route_stats[0], (unsigned long long)touched);
+      if (tid == 0) atomicAdd(&a.route_stats[1], 1ull);
+    }
+    for (int e = warp; e < E; e += blockDim.x >> 5) {
+      const int n_nt = toff[e + 1] - toff[e];
+      for (int i = lane; i < n_nt * (a.FJ + a.MD); i += 32) {
+        const int nt = i / (a.FJ + a.MD), r = i % (a.FJ + a.MD);
+        if (r < a.FJ) {
+          const int slot = (toff[e] + nt) * a.FJ + r;
+          if (slot < a.egu_cap) a.egu_tiles[slot] = make_int4(e, r, nt, 0);
+        } else {
+          const int slot = (toff[e] + nt) * a.MD + (r - a.FJ);
+          if (slot < a.ed_cap) a.ed_tiles[slot] = make_int4(e, r - a.FJ, nt, 0);
+        }
+      }
+    }
+  }
+  // clear the other mask buffer, sliced across CTAs
+  for (int i = blockIdx.x * blockDim.x + tid; i < E * MW; i += gridDim.x * blockDim.x) mask_next[i] = 0u;
+  // this CTA's pairs, one warp per pair
+  const int per = (P + gridDim.x - 1) / gridDim.x;
+  const int p0 = blockIdx.x * per, p1 = min(P, p0 + per);
+  for (int p = p0 + warp; p < p1; p += blockDim.x >> 5) {
+    const int e = a.idx[p];
+    const int t = p / k;
+    int rank = 0;
+    if (e >= 0 && e < E) {
+      const unsigned* m = mask + (size_t)e * MW;
+      const int wt = t >> 5;
+      for (int wi = lane; wi <= wt; wi += 32) {
+        const unsigned bits = wi < wt ? m[wi] : (m[wi] & ((1u << (t & 31)) - 1u));
+        rank += __popc(bits);
+      }
+      rank = warp_sum_int(rank);
+    }
+    const int row = (e >= 0 && e < E) ? off[e] + rank : 0;
+    if (lane == 0) {
+      a.pair_row[p] = row;
+      a.row_token[row] = t;
+      a.row_weight[row] = a.w[p];
+      a.row_pair[row] = p;
+    }
+    const uint4* src = reinterpret_cast<const uint4*>(u + (size_t)t * d);
+    uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)row * d);
+    const int n16 = d / 8;
+    for (int c0 = lane; c0 < n16; c0 += 32 * 4) {
+      uint4 r[4];
+#pragma unroll
+      for (int b = 0; b < 4; ++b)
+        if (c0 + b * 32 < n16) r[b] = src[c0 + b * 32];
+#pragma unroll
+      for (int b = 0; b < 4; ++b)
+        if (c0 + b * 32 < n16) dst[c0 + b * 32] = r[b];
+    }
+  }
+}
+
+cudaError_t run_route(const float* logits, const bf16* u, int d, bf16* xp, unsigned* mask, unsigned* mask_next,
+                      const GroupArgs& a, cudaStream_t st) {
+  if (a.T < 1 || a.T > 1024 || a.E > 256) return cudaErrorInvalidValue;
+  const int MW = (a.T + 31) >> 5;
+  {
+    const cudaError_t e_ = launch_pdl(k_topk_mask, dim3((a.T + 7) / 8), dim3(256), 0, st, logits, a.T, a.E, a.k, a.idx, a.w, mask, MW);
+    if (e_ != cudaSuccess) return e_;
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int P = a.T * a.k;
+  const int grid = (P + 7) / 8 < 148 ? (P + 7) / 8 : 148;
+  {
+    const cudaError_t e_ = launch_pdl(k_group_gather, dim3(grid), dim3(256), 0, st, a, mask, mask_next, MW, u, d, xp);
+    if (e_ != cudaSuccess) return e_;
+  }
   return cudaGetLastError();
 }
 
@@ -437,6 +667,8 @@ cudaError_t run_group(const GroupArgs& a, cudaStream_t st) {
 // ---------------------------------------------------------------------------
 __global__ void k_gather(const bf16* __restrict__ u, const int* __restrict__ row_token, int rows, int d,
                          bf16* __restrict__ xp) {
+  pdl_trigger();
+  pdl_wait();
   const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
@@ -447,7 +679,10 @@ __global__ void k_gather(const bf16* __restrict__ u, const int* __restrict__ row
 
 cudaError_t run_gather(const bf16* u, const int* row_token, int rows, int d, bf16* xp, cudaStream_t st) {
   if (rows == 0) return cudaSuccess;
-  k_gather<<<(rows + 7) / 8, 256, 0, st>>>(u, row_token, rows, d, xp);
+  {
+    const cudaError_t e_ = launch_pdl(k_gather, dim3((rows + 7) / 8), dim3(256), 0, st, u, row_token, rows, d, xp);
+    if (e_ != cudaSuccess) return e_;
+  }
   return cudaGetLastError();
 }
 
@@ -478,6 +713,8 @@ DG_DEVINL LmPart lm_merge(LmPart x, LmPart y) {
 
 __global__ void k_lm_combine(const float4* __restrict__ part, int G, int MT, int T, float* stats, int* argmax,
                              int* err) {
+  pdl_trigger();
+  pdl_wait();
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= T) return;
@@ -510,7 +747,10 @@ __global__ void k_lm_combine(const float4* __restrict__ part, int G, int MT, int
 cudaError_t run_lm_combine(const float4* part, int G, int MT, int T, float* stats, int* argmax, int* err,
                            cudaStream_t st) {
   if (T == 0) return cudaSuccess;
-  k_lm_combine<<<(T + 7) / 8, 256, 0, st>>>(part, G, MT, T, stats, argmax, err);
+  {
+    const cudaError_t e_ = launch_pdl(k_lm_combine, dim3((T + 7) / 8), dim3(256), 0, st, part, G, MT, T, stats, argmax, err);
+    if (e_ != cudaSuccess) return e_;
+  }
   return cudaGetLastError();
 }
 
@@ -546,6 +786,8 @@ DG_DEVINL int renoise_token(unsigned long long seed, int block, int step, uint32
 
 __global__ void k_philox_tokens(unsigned long long seed, int block, int step, int request, long long pos0, long long n,
                                 int vocab, int* out, unsigned char* mask_clear) {
+  pdl_trigger();
+  pdl_wait();
   const long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
   if (i >= n) return;
   out[i] = renoise_token(seed, block, step, (uint32_t)(pos0 + i), request, vocab);
@@ -555,8 +797,11 @@ __global__ void k_philox_tokens(unsigned long long seed, int block, int step, in
 cudaError_t run_philox_tokens(unsigned long long seed, int block, int step, int request, long long pos0, long long n,
                               int vocab, int* out, unsigned char* mask_clear, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
-  k_philox_tokens<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(seed, block, step, request, pos0, n, vocab, out,
+  {
+    const cudaError_t e_ = launch_pdl(k_philox_tokens, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, seed, block, step, request, pos0, n, vocab, out,
                                                                mask_clear);
+    if (e_ != cudaSuccess) return e_;
+  }
   return cudaGetLastError();
 }
 
@@ -564,6 +809,8 @@ cudaError_t run_philox_tokens(unsigned long long seed, int block, int step, int 
 // Accept / freeze / re-noise rule, one CTA per canvas, one thread per position.
 // ---------------------------------------------------------------------------
 __global__ void k_sample(SampleArgs a) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ float ssm[];
   float* lc_s = ssm;                                             // [canvas]
   int* un_s = reinterpret_cast<int*>(ssm + a.canvas);            // [canvas]
@@ -614,7 +861,10 @@ __global__ void k_sample(SampleArgs a) {
 cudaError_t run_sample(const SampleArgs& a, cudaStream_t st) {
   if (a.n_slots == 0) return cudaSuccess;
   const int threads = (a.canvas + 31) / 32 * 32;
-  k_sample<<<a.n_slots, threads, (size_t)a.canvas * 8, st>>>(a);
+  {
+    const cudaError_t e_ = launch_pdl(k_sample, dim3(a.n_slots), dim3(threads), (size_t)a.canvas * 8, st, a);
+    if (e_ != cudaSuccess) return e_;
+  }
   return cudaGetLastError();
 }
 
@@ -624,6 +874,8 @@ cudaError_t run_sample(const SampleArgs& a, cudaStream_t st) {
 // ---------------------------------------------------------------------------
 __global__ void k_k_copy(bf16* cache_k, int Hkv, long long cap, int D, long long pos0, long long n, const bf16* k_in,
                          bf16* k_out) {
+  pdl_trigger();
+  pdl_wait();
   const long long r = blockIdx.x;  // (head, i)
   const int head = (int)(r / n);
   const long long i = r - (long long)head * n;
@@ -639,6 +891,8 @@ __global__ void k_k_copy(bf16* cache_k, int Hkv, long long cap, int D, long long
 
 __global__ void k_vt_copy(bf16* cache_vt, int Hkv, long long cap, int D, long long pos0, long long n,
                           const bf16* v_in, bf16* v_out) {
+  pdl_trigger();
+  pdl_wait();
   const long long total = (long long)Hkv * D * n;
   for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
        e += (long long)gridDim.x * blockDim.x) {
@@ -657,12 +911,18 @@ __global__ void k_vt_copy(bf16* cache_vt, int Hkv, long long cap, int D, long lo
 cudaError_t run_kv_copy(bf16* cache_k, bf16* cache_v, int Hkv, long long cap, int D, long long pos0, long long n,
                         const bf16* k_in, const bf16* v_in, bf16* k_out, bf16* v_out, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
-  k_k_copy<<<(unsigned)(Hkv * n), 32, 0, st>>>(cache_k, Hkv, cap, D, pos0, n, k_in, k_out);
+  {
+    const cudaError_t e_ = launch_pdl(k_k_copy, dim3((unsigned)(Hkv * n)), dim3(32), 0, st, cache_k, Hkv, cap, D, pos0, n, k_in, k_out);
+    if (e_ != cudaSuccess) return e_;
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const long long total = (long long)Hkv * D * n;
   const unsigned blocks = (unsigned)((total + 255) / 256 < 65535 ? (total + 255) / 256 : 65535);
-  k_vt_copy<<<blocks, 256, 0, st>>>(cache_v, Hkv, cap, D, pos0, n, v_in, v_out);
+  {
+    const cudaError_t e_ = launch_pdl(k_vt_copy, dim3(blocks), dim3(256), 0, st, cache_v, Hkv, cap, D, pos0, n, v_in, v_out);
+    if (e_ != cudaSuccess) return e_;
+  }
   return cudaGetLastError();
 }
 

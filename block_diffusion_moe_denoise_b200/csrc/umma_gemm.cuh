@@ -16,7 +16,9 @@
 //
 // A problem class P supplies: BN, STAGES, B_STAGE (bytes), EP_SMEM (bytes),
 // TMEM_COLS, Params, num_tiles(), tile(), tx_bytes(), load(), epilogue(),
-// finish().  Every wait is bounded (see mbar_wait_bounded).
+// finish(), epilogue_prefetch() (called before the accumulator wait, so an
+// epilogue can pull its inputs into L1 while the main loop runs).  Every wait
+// is bounded (see mbar_wait_bounded).
 #pragma once
 
 #include "common.cuh"
@@ -79,6 +81,8 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_trigger();
+  pdl_wait();
   const uint32_t tmem = *tmem_slot;
   const int n_tiles = P::num_tiles(p);
   int* err = p.err;
@@ -138,6 +142,7 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
     for (int v = blockIdx.x; v < n_tiles; v += gridDim.x) {
       const Tile t = P::tile(p, v);
       if (!t.valid) continue;
+      P::epilogue_prefetch(p, t, row);
       if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, err)) break;
       tc_fence_after();
       const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + acc * P::BN;
@@ -164,7 +169,11 @@ struct ProblemBase {
   DG_DEVINL static void epilogue_init(const Params&, int, uint8_t*) {}
   template <class Params>
   DG_DEVINL static void finish(const Params&, int, uint8_t*) {}
+  template <class Params>
+  DG_DEVINL static void epilogue_prefetch(const Params&, const Tile&, int) {}
 };
+
+DG_DEVINL void prefetch_l1(const void* ptr) { asm volatile("prefetch.global.L1 [%0];" ::"l"(ptr)); }
 
 DG_DEVINL int round_up16(int n) { return (n + 15) & ~15; }
 
