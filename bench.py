@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--workload", default="generate", choices=["generate", "layer"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--canvas-vocab", type=int, default=0,
+                    help="layer workload: draw canvas ids from this many distinct tokens (concentrates routing)")
     return ap.parse_args()
 
 
@@ -219,13 +221,22 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """Max of a per-rank scalar over all ranks (device tensor for NCCL, host for gloo)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(tokens_per_rank: float, elapsed_ms_local: float, world: int) -> tuple[float, float]:
+    """Whole-job tokens/s of `world` replicas: every rank's tokens over the
+    slowest rank's device time.  Returns (tokens/s, max elapsed ms)."""
+    elapsed = max_over_ranks(elapsed_ms_local, world)
+    return world * tokens_per_rank / (elapsed / 1e3), elapsed
 
 
 # ---------------------------------------------------------------------------
@@ -320,9 +331,15 @@ def main():
         h.set_kv_len(0, PROMPT)
         prefill_ms = None
 
+        if args.canvas_vocab:
+            ids = torch.randint(0, args.canvas_vocab, (cfg.canvas,), generator=torch.Generator().manual_seed(3))
+            fixed_canvas = (ids * 977).to(torch.int32).to(dev)
+
         def one_step(i, record=False):
             if i % cfg.max_steps == 0:
                 h.open_canvas(0, SEED, 0)
+                if args.canvas_vocab:
+                    h.set_canvas(0, fixed_canvas, torch.zeros(cfg.canvas, dtype=torch.uint8, device=dev), 0)
             e0 = ev() if record else None
             h.denoise_step([0])
             e1 = ev() if record else None
@@ -347,9 +364,8 @@ def main():
     elapsed = start.elapsed_time(end)
     launches = h.launch_count() - launches0
     h.sync()
-    elapsed_max = max_over_ranks(elapsed, world)
     toks_per_step = cfg.canvas if args.workload == "generate" else cfg.canvas / 12.0
-    value = world * toks_per_step * args.steps / (elapsed_max / 1e3)
+    value, elapsed_max = job_throughput(toks_per_step * args.steps, elapsed, world)
     step_ms = sum(a.elapsed_time(b) for a, b in seg_steps)
     n_steps = sum(steps_per)
     ms_denoise = step_ms / n_steps

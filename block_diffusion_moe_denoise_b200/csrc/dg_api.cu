@@ -66,7 +66,7 @@ void make_plan(const dg_config* c, int max_req, long long cap_user, Plan* p) {
   const int Tcap = (T + 127) / 128 * 128;
   const long long rows = (long long)T * c->top_k;
   const int D = c->head_dim, d = c->d_model;
-  const long long n_nt = c->n_experts + (rows + 63) / 64;
+  const long long n_nt = c->n_experts + (rows + kExpertRows - 1) / kExpertRows;
   p->add("err", 64);
   p->add("kv", (size_t)max_req * c->n_layers * 2 * c->n_kv_heads * (size_t)cap * D * 2);
   p->add("x", (size_t)Tcap * d * 4);
@@ -523,7 +523,7 @@ int dg_init(const dg_config* cfg, const dg_weights* wts, int max_requests, int64
   h->kv_layer_stride = 2ll * c.n_kv_heads * h->cap * D;
   h->kv_req_stride = h->kv_layer_stride * c.n_layers;
   const long long rows = (long long)h->T_max * c.top_k;
-  const long long n_nt = c.n_experts + (rows + 63) / 64;
+  const long long n_nt = c.n_experts + (rows + kExpertRows - 1) / kExpertRows;
   h->egu_cap = (int)(n_nt * (c.ffn_expert / 64));
   h->ed_cap = (int)(n_nt * (d / 128));
 
@@ -547,8 +547,8 @@ int dg_init(const dg_config* cfg, const dg_weights* wts, int max_requests, int64
   ok = ok && make_map(&h->tm_hn, h->B<bf16>("hn"), d, h->Tcap, 128);
   ok = ok && make_map(&h->tm_o, h->B<bf16>("o"), (long long)c.n_q_heads * D, h->Tcap, 256);
   ok = ok && make_map(&h->tm_u, h->B<bf16>("u"), d, h->Tcap, 128);
-  ok = ok && make_map(&h->tm_xp, h->B<bf16>("xp"), d, rows, 64);
-  ok = ok && make_map(&h->tm_hp, h->B<bf16>("hp"), c.ffn_expert, rows, 64);
+  ok = ok && make_map(&h->tm_xp, h->B<bf16>("xp"), d, rows, kExpertRows);
+  ok = ok && make_map(&h->tm_hp, h->B<bf16>("hp"), c.ffn_expert, rows, kExpertRows);
   ok = ok && make_map(&h->tm_hs, h->B<bf16>("hs"), c.ffn_shared, h->Tcap, 256);
   ok = ok && make_map(&h->tm_embed, h->embed, d, c.vocab, 256);
   {

@@ -46,6 +46,7 @@ struct QkvArgs {
   int* err;
 };
 constexpr int kMaxPartSplits = 8;
+constexpr int kExpertRows = 64;  // token rows per routed-expert GEMM tile
 struct WpartArgs {
   const CUtensorMap* tm_w;  // weights [d, K], 128-row boxes
   const CUtensorMap* tm_x;  // activations [Tcap, K], 256-row boxes

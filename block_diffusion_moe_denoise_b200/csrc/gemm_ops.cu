@@ -252,12 +252,12 @@ struct P_WPART : ProblemBase {
 // A rows 0..63 = W_gate rows, 64..127 = W_up rows of the same hidden units.
 // ---------------------------------------------------------------------------
 struct P_EGU : ProblemBase {
-  static constexpr int BN = 64, STAGES = 8, B_STAGE = BN * 128, TMEM_COLS = 128;
+  static constexpr int BN = kExpertRows, STAGES = 8, B_STAGE = BN * 128, TMEM_COLS = 128;
   static constexpr int EP_SMEM = 64 * 17 * 4;
   struct Params {
     CUtensorMap tmG;  // w_gate as [E*fe, d]
     CUtensorMap tmU;  // w_up   as [E*fe, d]
-    CUtensorMap tmX;  // expert-grouped tokens [rows_cap, d]
+    CUtensorMap tmX;  // expert-grouped tokens [rows_cap, d], 64-row boxes
     int nk, fe;
     const int4* tiles;
     const int* n_tiles;
@@ -278,10 +278,10 @@ struct P_EGU : ProblemBase {
     t.a = tt.x;  // expert
     t.b = tt.y;  // hidden-unit block
     const int nt = tt.z;
-    const int n_valid = min(64, p.counts[t.a] - nt * 64);
+    const int n_valid = min(BN, p.counts[t.a] - nt * BN);
     t.valid = n_valid > 0;
     t.c = n_valid;
-    t.d = p.offsets[t.a] + nt * 64;  // first grouped row
+    t.d = p.offsets[t.a] + nt * BN;  // first grouped row
     t.nk = p.nk;
     t.n_mma = round_up16(n_valid);
     return t;
@@ -323,10 +323,10 @@ struct P_EGU : ProblemBase {
 // of expert e for its grouped rows nt*64..+63; each row scaled by its gate weight.
 // ---------------------------------------------------------------------------
 struct P_ED : ProblemBase {
-  static constexpr int BN = 64, STAGES = 8, B_STAGE = BN * 128, TMEM_COLS = 128;
+  static constexpr int BN = kExpertRows, STAGES = 8, B_STAGE = BN * 128, TMEM_COLS = 128;
   struct Params {
     CUtensorMap tmW;  // w_down as [E*d, fe]
-    CUtensorMap tmH;  // hidden [rows_cap, fe]
+    CUtensorMap tmH;  // hidden [rows_cap, fe], 64-row boxes
     int nk, d;
     const int4* tiles;
     const int* n_tiles;
@@ -347,10 +347,10 @@ struct P_ED : ProblemBase {
     t.a = tt.x;  // expert
     t.b = tt.y;  // 128-feature block
     const int nt = tt.z;
-    const int n_valid = min(64, p.counts[t.a] - nt * 64);
+    const int n_valid = min(BN, p.counts[t.a] - nt * BN);
     t.valid = n_valid > 0;
     t.c = n_valid;
-    t.d = p.offsets[t.a] + nt * 64;
+    t.d = p.offsets[t.a] + nt * BN;
     t.nk = p.nk;
     t.n_mma = round_up16(n_valid);
     return t;

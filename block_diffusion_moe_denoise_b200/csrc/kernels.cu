@@ -417,7 +417,7 @@ __global__ void __launch_bounds__(1024) k_group(GroupArgs a) {
     toff[0] = 0;
     for (int e = 0; e < E; ++e) {
       off[e + 1] = off[e] + cnt[e];
-      toff[e + 1] = toff[e] + (cnt[e] + 63) / 64;
+      toff[e + 1] = toff[e] + (cnt[e] + kExpertRows - 1) / kExpertRows;
     }
     if (a.route_stats) {
       int touched = 0;
@@ -552,7 +552,7 @@ __global__ void __launch_bounds__(256) k_group_gather(GroupArgs a, const unsigne
     for (int i = 0; i < 8; ++i) {
       const int e = lane * 8 + i;
       v[i] = e < E ? cnt[e] : 0;
-      tv[i] = e < E ? (cnt[e] + 63) / 64 : 0;
+      tv[i] = e < E ? (cnt[e] + kExpertRows - 1) / kExpertRows : 0;
     }
     const int tot = warp_excl_scan8(v, lane);
     const int ttot = warp_excl_scan8(tv, lane);
