@@ -394,8 +394,11 @@ def main():
             import hashlib
             src = open(os.path.join(ROOT, "block_diffusion_moe_denoise_b200", "csrc", "gemm_ops.cu"), "rb").read()
             src += open(os.path.join(ROOT, "block_diffusion_moe_denoise_b200", "csrc", "umma_gemm.cuh"), "rb").read()
+            # The capture is a smaller case (one layer, 124 experts touched); DRAM
+            # traffic grows in proportion to the expert weights streamed, so it is
+            # scaled to this launch by its algorithmic bytes.
             if tj.get("source_sha256") == hashlib.sha256(src).hexdigest():
-                traffic = tj["bytes_per_launch"]
+                traffic = tj["traffic_per_algorithmic_byte"] * egu_bytes
         except Exception:
             traffic = None
     total_prof = sum(v[0] for v in prof.values()) or 1.0
