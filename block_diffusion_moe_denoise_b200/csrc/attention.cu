@@ -227,17 +227,31 @@ __global__ void __launch_bounds__(192, 1) k_attn_tc(const __grid_constant__ Attn
       if (!mbar_wait_bounded(&s_full[b], (j >> 1) & 1, abort_flag, err)) { ok = false; break; }
       tc_fence_after();
       float s[kAK];
+      {
+        uint32_t r[kAK / 16][16];
 #pragma unroll
-      for (int c = 0; c < kAK; c += 16) tmem_ld16(tm_s0 + lane_off + b * kAK + c, s + c);
+        for (int c = 0; c < kAK / 16; ++c) tmem_ld16_issue(tm_s0 + lane_off + b * kAK + c * 16, r[c]);
+#pragma unroll
+        for (int c = 0; c < kAK / 16; ++c) tmem_ld_wait16(r[c]);
+#pragma unroll
+        for (int c = 0; c < kAK / 16; ++c)
+#pragma unroll
+          for (int i = 0; i < 16; ++i) s[c * 16 + i] = __uint_as_float(r[c][i]);
+      }
       tc_fence_before();
       mbar_arrive(&s_empty[b]);
       const int key0 = k_begin + j * kAK;
-      float mx = -INFINITY;
+      if (key0 + kAK > k_end) {   // ragged last tile: keys past the range get no weight
 #pragma unroll
-      for (int c = 0; c < kAK; ++c) {
-        s[c] = key0 + c < k_end ? s[c] * sl2 : -INFINITY;
-        mx = fmaxf(mx, s[c]);
+        for (int c = 0; c < kAK; ++c)
+          if (key0 + c >= k_end) s[c] = -INFINITY;
       }
+      // raw-score max, then scaled (sl2 > 0 keeps the order); the tile has
+      // at least one key in range, so mx is finite
+      float mx = s[0];
+#pragma unroll
+      for (int c = 1; c < kAK; ++c) mx = fmaxf(mx, s[c]);
+      mx *= sl2;
       const bool need = mx > m_used + kRescaleLog2;
       const float m_new = need ? mx : m_used;
       // P buffer b is free once PV(j-2) is done
@@ -264,7 +278,7 @@ __global__ void __launch_bounds__(192, 1) k_attn_tc(const __grid_constant__ Attn
         float p[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          p[i] = exp2f(s[ch * 8 + i] - m_used);
+          p[i] = ex2_fast(fmaf(s[ch * 8 + i], sl2, -m_used));
           rs += p[i];
         }
         uint4 v;

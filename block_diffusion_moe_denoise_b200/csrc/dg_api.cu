@@ -19,7 +19,7 @@ constexpr int kLmGridMax = 256;
 constexpr int kSplitCap = 8;
 
 struct LayerMaps {
-  CUtensorMap qkv, o, gate, up, down, sgate, sup, sdown;
+  CUtensorMap qkv, o, gate, up, down, sgate, sup, sdown, router;
 };
 
 struct ReqState {
@@ -50,7 +50,8 @@ bool config_ok(const dg_config* c) {
   if (c->n_kv_heads < 1 || c->n_q_heads < 1 || c->n_q_heads % c->n_kv_heads != 0) return false;
   if ((c->n_q_heads * c->head_dim) % 128 != 0 || (c->n_kv_heads * c->head_dim) % 128 != 0) return false;
   if ((c->n_q_heads * c->head_dim) % 64 != 0) return false;
-  if (c->n_experts < 1 || c->n_experts > 256 || c->top_k < 1 || c->top_k > 8 || c->top_k > c->n_experts) return false;
+  if (c->n_experts < 16 || c->n_experts > 128 || c->n_experts % 16 != 0) return false;
+  if (c->top_k < 1 || c->top_k > 8 || c->top_k > c->n_experts) return false;
   if (c->ffn_expert < 64 || c->ffn_expert % 64 != 0 || c->ffn_shared < 64 || c->ffn_shared % 64 != 0) return false;
   if (c->vocab < 256 || c->vocab % 256 != 0) return false;
   if (c->canvas < 1 || c->canvas > 256) return false;
@@ -105,7 +106,6 @@ void make_plan(const dg_config* c, int max_req, long long cap_user, Plan* p) {
   p->add("router_logits", (size_t)Tcap * c->n_experts * 4);
   p->add("part", (size_t)kMaxPartSplits * Tcap * d * 4);
   p->add("route_mask", (size_t)2 * c->n_experts * ((T + 31) / 32) * 4);
-  p->add("un", (size_t)Tcap * d * 4);
   p->add("prompt", (size_t)cap_user * 4);
 }
 
@@ -270,7 +270,7 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     bf16* kv_l = h->B<bf16>("kv") + (size_t)l * h->kv_layer_stride;
     LAUNCH(h, K_RMSNORM, 1,
            run_residual_norm(x, yp, pair_row, pending_k, part, pending_parts, h->Tcap, (const float*)w.attn_norm, T,
-                             d, c.norm_eps, hn, nullptr, st));
+                             d, c.norm_eps, hn, st));
     pending_k = pending_parts = 0;
     QkvArgs qa;
     qa.tm_x = &h->tm_hn;
@@ -342,13 +342,36 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     oa.part = part;
     oa.err = err;
     LAUNCH(h, K_OPROJ, 1, run_wpart(oa, st));
-    // x += attention output projection; FFN RMSNorm -> bf16 rows (experts) and fp32 rows (router)
+    // x += attention output projection; FFN RMSNorm -> bf16 rows u
     LAUNCH(h, K_RMSNORM, 1,
            run_residual_norm(x, nullptr, nullptr, 0, part, so, h->Tcap, (const float*)w.ffn_norm, T, d, c.norm_eps,
-                             h->B<bf16>("u"), h->B<float>("un"), st));
-    LAUNCH(h, K_ROUTER, 1,
-           run_router_logits(h->B<float>("un"), (const bf16*)w.w_router, T, d, c.n_experts,
-                             h->B<float>("router_logits"), st));
+                             h->B<bf16>("u"), st));
+    const int MW = (h->T_max + 31) / 32;  // bitmask words per expert (fixed layout)
+    const size_t mw = (size_t)c.n_experts * MW;
+    unsigned* masks = h->B<unsigned>("route_mask");
+    unsigned* mask_cur = masks + (size_t)h->mask_flip * mw;
+    unsigned* mask_nxt = masks + (size_t)(h->mask_flip ^ 1) * mw;
+    h->mask_flip ^= 1;
+    // shared expert gate|up + router logits, top-k and token bitmasks
+    SharedArgs sa;
+    sa.tm_u = &h->tm_u;
+    sa.tm_gate = &m.sgate;
+    sa.tm_up = &m.sup;
+    sa.tm_router = &m.router;
+    sa.T = T;
+    sa.d = d;
+    sa.fs = c.ffn_shared;
+    sa.num_sms = h->num_sms;
+    sa.E = c.n_experts;
+    sa.k = k;
+    sa.MW = MW;
+    sa.hs = h->B<bf16>("hs");
+    sa.logits = h->B<float>("router_logits");
+    sa.idx = h->B<int>("idx");
+    sa.w = h->B<float>("w");
+    sa.mask = mask_cur;
+    sa.err = err;
+    LAUNCH(h, K_SGU, 1, run_shared_gate_up(sa, st));
     GroupArgs ga;
     ga.idx = h->B<int>("idx");
     ga.w = h->B<float>("w");
@@ -371,15 +394,7 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     ga.ed_count = h->B<int>("tile_counts") + 1;
     ga.route_stats = h->B<unsigned long long>("route_stats");
     ga.err = err;
-    {
-      const size_t mw = (size_t)c.n_experts * ((h->T_max + 31) / 32);
-      unsigned* masks = h->B<unsigned>("route_mask");
-      unsigned* cur = masks + (size_t)h->mask_flip * mw;
-      unsigned* nxt = masks + (size_t)(h->mask_flip ^ 1) * mw;
-      h->mask_flip ^= 1;
-      LAUNCH(h, K_GROUP, 2,
-             run_route(h->B<float>("router_logits"), h->B<bf16>("u"), d, h->B<bf16>("xp"), cur, nxt, ga, st));
-    }
+    LAUNCH(h, K_GROUP, 1, run_route(h->B<bf16>("u"), d, h->B<bf16>("xp"), mask_cur, mask_nxt, MW, ga, st));
 
     ExpertArgs ea;
     ea.tm_gate = &m.gate;
@@ -403,17 +418,6 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     LAUNCH(h, K_EGU, 1, run_experts_gate_up(ea, st));
     LAUNCH(h, K_ED, 1, run_experts_down(ea, st));
 
-    SharedArgs sa;
-    sa.tm_u = &h->tm_u;
-    sa.tm_gate = &m.sgate;
-    sa.tm_up = &m.sup;
-    sa.T = T;
-    sa.d = d;
-    sa.fs = c.ffn_shared;
-    sa.num_sms = h->num_sms;
-    sa.hs = h->B<bf16>("hs");
-    sa.err = err;
-    LAUNCH(h, K_SGU, 1, run_shared_gate_up(sa, st));
     WpartArgs da;
     da.tm_w = &m.sdown;
     da.tm_x = &h->tm_hs;
@@ -432,7 +436,7 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
   if (want_lm) {
     LAUNCH(h, K_RMSNORM, 1,
            run_residual_norm(x, yp, pair_row, pending_k, part, pending_parts, h->Tcap, h->final_norm, T, d,
-                             c.norm_eps, hn, nullptr, st));
+                             c.norm_eps, hn, st));
     LmArgs la;
     la.tm_x = &h->tm_hn;
     la.tm_embed = &h->tm_embed;
@@ -452,7 +456,7 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     // a pass stopped after a full layer: fold its expert outputs into x
     LAUNCH(h, K_RMSNORM, 1,
            run_residual_norm(x, yp, pair_row, pending_k, part, pending_parts, h->Tcap, nullptr, T, d, c.norm_eps,
-                             nullptr, nullptr, st));
+                             nullptr, st));
   }
   return DG_OK;
 }
@@ -540,8 +544,9 @@ int dg_init(const dg_config* cfg, const dg_weights* wts, int max_requests, int64
     ok = ok && make_map(&m.gate, w.w_gate, d, E * c.ffn_expert, 64);
     ok = ok && make_map(&m.up, w.w_up, d, E * c.ffn_expert, 64);
     ok = ok && make_map(&m.down, w.w_down, c.ffn_expert, E * d, 128);
-    ok = ok && make_map(&m.sgate, w.ws_gate, d, c.ffn_shared, 64);
-    ok = ok && make_map(&m.sup, w.ws_up, d, c.ffn_shared, 64);
+    ok = ok && make_map(&m.sgate, w.ws_gate, d, c.ffn_shared, 32);
+    ok = ok && make_map(&m.sup, w.ws_up, d, c.ffn_shared, 32);
+    ok = ok && make_map(&m.router, w.w_router, d, E, (int)E);
     ok = ok && make_map(&m.sdown, w.ws_down, c.ffn_shared, d, 128);
   }
   ok = ok && make_map(&h->tm_hn, h->B<bf16>("hn"), d, h->Tcap, 128);

@@ -69,9 +69,14 @@ struct ExpertArgs {
   int* err;
 };
 struct SharedArgs {
-  const CUtensorMap *tm_u, *tm_gate, *tm_up;
+  const CUtensorMap *tm_u, *tm_gate, *tm_up, *tm_router;
   int T, d, fs, num_sms;
+  int E, k, MW;       // router: experts (multiple of 16, <= 128), top-k, bitmask words per expert
   bf16* hs;
+  float* logits;      // [Tcap, E] router logits (kept for inspection)
+  int* idx;           // [T, k] picked experts
+  float* w;           // [T, k] their renormalised probabilities
+  unsigned* mask;     // [E][MW] per-expert token bitmasks, zero on entry
   int* err;
 };
 struct LmArgs {
@@ -107,15 +112,12 @@ cudaError_t run_embed(const int* const* ids, const SlotInfo& s, const bf16* embe
 // x[t] += sum_j yp[pair_row[t*k+j]] + sum_s part[s][t]; then (if an output is
 // given) the RMSNorm of x[t] with gain g as bf16 and/or fp32
 cudaError_t run_residual_norm(float* x, const float* yp, const int* pair_row, int k, const float* part, int n_part,
-                              int Tcap, const float* g, int T, int d, float eps, bf16* out, float* out_f32,
-                              cudaStream_t st);
+                              int Tcap, const float* g, int T, int d, float eps, bf16* out, cudaStream_t st);
 cudaError_t run_rmsnorm(const float* x, const float* g, int T, int d, float eps, bf16* out, cudaStream_t st);
-// router logits [T, E] from fp32 normalised rows un [T, d]
-cudaError_t run_router_logits(const float* un, const bf16* wr, int T, int d, int E, float* logits, cudaStream_t st);
 cudaError_t run_topk(const float* logits, int T, int E, int k, int* idx, float* w, cudaStream_t st);
 struct GroupArgs {
-  int* idx;     // [T, k] selected experts (read by run_group, written by run_route)
-  float* w;     // [T, k] gate weights (read by run_group, written by run_route)
+  int* idx;     // [T, k] selected experts (written by the router epilogue or the caller)
+  float* w;     // [T, k] gate weights
   int T, k, E, FJ, MD, egu_cap, ed_cap;
   int* counts;
   int* offsets;
@@ -131,9 +133,10 @@ struct GroupArgs {
   int* err;
 };
 cudaError_t run_group(const GroupArgs& a, cudaStream_t st);
-// top-k selection from logits (token bitmasks in `mask`, zeroed beforehand), then
-// the grouping above plus the gather of u rows into xp; clears `mask_next`
-cudaError_t run_route(const float* logits, const bf16* u, int d, bf16* xp, unsigned* mask, unsigned* mask_next,
+// the grouping above from the token bitmasks `mask` ([E][MW] words, MW fixed by
+// the workspace so the layout never changes between passes) the router epilogue
+// set, plus the gather of u rows into xp; clears all of `mask_next`
+cudaError_t run_route(const bf16* u, int d, bf16* xp, unsigned* mask, unsigned* mask_next, int MW,
                       const GroupArgs& a, cudaStream_t st);
 cudaError_t run_gather(const bf16* u, const int* row_token, int rows, int d, bf16* xp, cudaStream_t st);
 cudaError_t run_lm_combine(const float4* part, int G, int MT, int T, float* stats, int* argmax, int* err,

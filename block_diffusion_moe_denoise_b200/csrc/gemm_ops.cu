@@ -96,12 +96,19 @@ struct P_QKV : ProblemBase {
     return t;
   }
   DG_DEVINL static uint32_t tx_bytes(const Params&, const Tile&) { return kAStage + B_STAGE; }
-  DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
+  static constexpr bool PRELOAD = true;
+  DG_DEVINL static void load_w(const Params& p, const Tile& t, int kb, uint32_t, uint32_t sb, uint64_t* bar) {
     int kind, tb, r0, r1;
     rows_of(p, t.b, kind, tb, r0, r1);
-    tma_load_2d(sa, &p.tmA, kb * 64, t.a * 128, bar);
     tma_load_2d(sb, &p.tmB, kb * 64, r0, bar);
     tma_load_2d(sb + 64 * 128, &p.tmB, kb * 64, r1, bar);
+  }
+  DG_DEVINL static void load_x(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t, uint64_t* bar) {
+    tma_load_2d(sa, &p.tmA, kb * 64, t.a * 128, bar);
+  }
+  DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
+    load_x(p, t, kb, sa, sb, bar);
+    load_w(p, t, kb, sa, sb, bar);
   }
   DG_DEVINL static void epilogue_prefetch(const Params& p, const Tile& t, int row) {
     const int tok = t.a * 128 + row;
@@ -227,9 +234,16 @@ struct P_WPART : ProblemBase {
     return t;
   }
   DG_DEVINL static uint32_t tx_bytes(const Params&, const Tile&) { return kAStage + B_STAGE; }
-  DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
+  static constexpr bool PRELOAD = true;
+  DG_DEVINL static void load_w(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t, uint64_t* bar) {
     tma_load_2d(sa, &p.tmA, (t.d + kb) * 64, t.a * 128, bar);
+  }
+  DG_DEVINL static void load_x(const Params& p, const Tile& t, int kb, uint32_t, uint32_t sb, uint64_t* bar) {
     tma_load_2d(sb, &p.tmB, (t.d + kb) * 64, t.b * BN, bar);
+  }
+  DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
+    load_w(p, t, kb, sa, sb, bar);
+    load_x(p, t, kb, sa, sb, bar);
   }
   DG_DEVINL static void epilogue(const Params& p, const Tile& t, uint32_t taddr, int, int, int row, uint8_t*) {
     const int f = t.a * 128 + row;
@@ -378,52 +392,148 @@ struct P_ED : ProblemBase {
 };
 
 // ---------------------------------------------------------------------------
-// Shared expert gate|up + SwiGLU.  Tile (mt, j): tokens mt*128..+127, hidden
-// units j*64..+63; B rows 0..63 = gate rows, 64..127 = up rows.
+// Shared expert gate|up + SwiGLU, and the router, in one launch (both read the
+// FFN-normed token rows).  Tokens are the 128-row operand.
+//   router tile (mt):     N = E router rows; the epilogue thread owning a token
+//                         row picks its top-k experts (descending logit, ties to
+//                         the lower id), the softmax of the picked logits, and
+//                         sets the token's bit in each picked expert's bitmask
+//   shared tile (mt, j):  hidden units j*32..+31; B rows 0..31 = gate rows,
+//                         32..63 = up rows (N = 64, so 2 x 33 tiles fill the GPU)
+// Router tiles come first in the schedule: they have the longest main loop and
+// the grouping kernel that follows waits on them.
 // ---------------------------------------------------------------------------
 struct P_SGU : ProblemBase {
   static constexpr int BN = 128, STAGES = 6, B_STAGE = BN * 128, TMEM_COLS = 256;
+  static constexpr int kHid = 32;  // shared hidden units per tile
   struct Params {
     CUtensorMap tmX;  // normed tokens [Tcap, d]
-    CUtensorMap tmG;  // ws_gate [fs, d], 64-row boxes
-    CUtensorMap tmU;  // ws_up [fs, d], 64-row boxes
-    int T, nk, MT, FJ, fs;
+    CUtensorMap tmG;  // ws_gate [fs, d], 32-row boxes
+    CUtensorMap tmU;  // ws_up [fs, d], 32-row boxes
+    CUtensorMap tmR;  // w_router [E, d], E-row boxes
+    int T, nk, MT, FJ, fs, E, k, MW;
     __nv_bfloat16* hs;  // [Tcap, fs]
+    float* logits;      // [Tcap, E]
+    int* idx;           // [T, k]
+    float* w;           // [T, k]
+    unsigned* mask;     // [E][MW] token bitmasks (zero on entry)
     int* err;
   };
+  static constexpr bool PRELOAD = true;
   DG_DEVINL static void prefetch(const Params& p) {
     tma_prefetch_desc(&p.tmX);
     tma_prefetch_desc(&p.tmG);
     tma_prefetch_desc(&p.tmU);
+    tma_prefetch_desc(&p.tmR);
   }
-  DG_DEVINL static int num_tiles(const Params& p) { return p.MT * p.FJ; }
+  DG_DEVINL static int num_tiles(const Params& p) { return p.MT * (p.FJ + 1); }
   DG_DEVINL static Tile tile(const Params& p, int v) {
     Tile t;
     t.valid = 1;
     t.nk = p.nk;
-    t.n_mma = BN;
-    t.a = v % p.MT;
-    t.b = v / p.MT;
+    if (v < p.MT) {
+      t.a = v;
+      t.b = -1;  // router tile
+      t.n_mma = p.E;
+    } else {
+      t.a = (v - p.MT) % p.MT;
+      t.b = (v - p.MT) / p.MT;
+      t.n_mma = 2 * kHid;
+    }
     return t;
   }
-  DG_DEVINL static uint32_t tx_bytes(const Params&, const Tile&) { return kAStage + B_STAGE; }
-  DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
+  DG_DEVINL static uint32_t tx_bytes(const Params& p, const Tile& t) {
+    return kAStage + (t.b < 0 ? p.E : 2 * kHid) * 128;
+  }
+  DG_DEVINL static void load_w(const Params& p, const Tile& t, int kb, uint32_t, uint32_t sb, uint64_t* bar) {
+    if (t.b < 0) {
+      tma_load_2d(sb, &p.tmR, kb * 64, 0, bar);
+    } else {
+      tma_load_2d(sb, &p.tmG, kb * 64, t.b * kHid, bar);
+      tma_load_2d(sb + kHid * 128, &p.tmU, kb * 64, t.b * kHid, bar);
+    }
+  }
+  DG_DEVINL static void load_x(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t, uint64_t* bar) {
     tma_load_2d(sa, &p.tmX, kb * 64, t.a * 128, bar);
-    tma_load_2d(sb, &p.tmG, kb * 64, t.b * 64, bar);
-    tma_load_2d(sb + 64 * 128, &p.tmU, kb * 64, t.b * 64, bar);
+  }
+  DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
+    load_x(p, t, kb, sa, sb, bar);
+    load_w(p, t, kb, sa, sb, bar);
+  }
+  DG_DEVINL static void router_epilogue(const Params& p, int tok, uint32_t taddr) {
+    const bool ok = tok < p.T;
+    float tv[8];
+    int ti[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      tv[r] = -INFINITY;
+      ti[r] = 0x7fffffff;
+    }
+    for (int c0 = 0; c0 < p.E; c0 += 16) {
+      float z[16];
+      tmem_ld16(taddr + c0, z);
+      if (!ok) continue;
+      float4* lg = reinterpret_cast<float4*>(p.logits + (size_t)tok * p.E + c0);
+#pragma unroll
+      for (int i = 0; i < 16; i += 4) lg[i / 4] = make_float4(z[i], z[i + 1], z[i + 2], z[i + 3]);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        // experts arrive in ascending id order; a strict comparison keeps the
+        // earlier (lower) id ahead of an equal logit
+        float v = z[i];
+        int e = c0 + i;
+        if (v > tv[7]) {
+#pragma unroll
+          for (int r = 0; r < 8; ++r) {
+            if (v > tv[r]) {
+              const float fv = tv[r];
+              const int fi = ti[r];
+              tv[r] = v;
+              ti[r] = e;
+              v = fv;
+              e = fi;
+            }
+          }
+        }
+      }
+    }
+    if (!ok) return;
+    float ex[8], sum = 0.f;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      ex[r] = r < p.k ? expf(tv[r] - tv[0]) : 0.f;
+      sum += ex[r];
+    }
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      if (r < p.k) {
+        // fewer than k picks only happen with NaN logits
+        const bool valid = (unsigned)ti[r] < (unsigned)p.E;
+        p.idx[(size_t)tok * p.k + r] = valid ? ti[r] : -1;
+        p.w[(size_t)tok * p.k + r] = ex[r] / sum;
+        if (valid)
+          atomicOr(&p.mask[(size_t)ti[r] * p.MW + (tok >> 5)], 1u << (tok & 31));
+        else
+          atomicOr(p.err, DG_DEVERR_NAN);
+      }
+    }
   }
   DG_DEVINL static void epilogue(const Params& p, const Tile& t, uint32_t taddr, int, int, int row, uint8_t*) {
     const int tok = t.a * 128 + row;
+    if (t.b < 0) {
+      router_epilogue(p, tok, taddr);
+      return;
+    }
     const bool ok = tok < p.T;
-    for (int c0 = 0; c0 < 64; c0 += 16) {
+    for (int c0 = 0; c0 < kHid; c0 += 16) {
       float g[16], u[16];
       tmem_ld16(taddr + c0, g);
-      tmem_ld16(taddr + 64 + c0, u);
+      tmem_ld16(taddr + kHid + c0, u);
       if (ok) {
         float h[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) h[i] = silu_f(g[i]) * u[i];
-        store_bf16x16(p.hs + (size_t)tok * p.fs + t.b * 64 + c0, h);
+        store_bf16x16(p.hs + (size_t)tok * p.fs + t.b * kHid + c0, h);
       }
     }
   }
@@ -469,9 +579,16 @@ struct P_LM : ProblemBase {
     return t;
   }
   DG_DEVINL static uint32_t tx_bytes(const Params&, const Tile&) { return kAStage + B_STAGE; }
-  DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
-    tma_load_2d(sa, &p.tmX, kb * 64, t.a * 128, bar);
+  static constexpr bool PRELOAD = true;
+  DG_DEVINL static void load_w(const Params& p, const Tile& t, int kb, uint32_t, uint32_t sb, uint64_t* bar) {
     tma_load_2d(sb, &p.tmE, kb * 64, t.b * 256, bar);
+  }
+  DG_DEVINL static void load_x(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t, uint64_t* bar) {
+    tma_load_2d(sa, &p.tmX, kb * 64, t.a * 128, bar);
+  }
+  DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
+    load_x(p, t, kb, sa, sb, bar);
+    load_w(p, t, kb, sa, sb, bar);
   }
   DG_DEVINL static void epilogue_init(const Params& p, int row, uint8_t* ep) {
     LmStat* st = reinterpret_cast<LmStat*>(ep);
@@ -628,18 +745,27 @@ cudaError_t run_experts_down(const ExpertArgs& a, cudaStream_t st) {
 }
 
 cudaError_t run_shared_gate_up(const SharedArgs& a, cudaStream_t st) {
+  if (a.E < 16 || a.E > P_SGU::BN || a.E % 16 != 0 || a.k < 1 || a.k > 8) return cudaErrorInvalidValue;
   P_SGU::Params g;
   g.tmX = *a.tm_u;
   g.tmG = *a.tm_gate;
   g.tmU = *a.tm_up;
+  g.tmR = *a.tm_router;
   g.T = a.T;
   g.nk = a.d / 64;
   g.MT = (a.T + 127) / 128;
-  g.FJ = a.fs / 64;
+  g.FJ = a.fs / P_SGU::kHid;
   g.fs = a.fs;
+  g.E = a.E;
+  g.k = a.k;
+  g.MW = a.MW;
   g.hs = a.hs;
+  g.logits = a.logits;
+  g.idx = a.idx;
+  g.w = a.w;
+  g.mask = a.mask;
   g.err = a.err;
-  return launch_gemm<P_SGU>(g, grid_for(g.MT * g.FJ, a.num_sms), st);
+  return launch_gemm<P_SGU>(g, grid_for(g.MT * (g.FJ + 1), a.num_sms), st);
 }
 
 cudaError_t run_lm_head(const LmArgs& a, int* grid_out, cudaStream_t st) {

@@ -109,7 +109,7 @@ cudaError_t run_rmsnorm(const float* x, const float* g, int T, int d, float eps,
 // ---------------------------------------------------------------------------
 // Residual update + RMSNorm, one CTA per token row:
 //   x[t] += sum_j Yp[row(t, j)] + sum_s part[s][t]
-//   out[t] = bf16(x[t] / sqrt(mean(x[t]^2) + eps) * g), out_f32[t] likewise in fp32
+//   out[t] = bf16(x[t] / sqrt(mean(x[t]^2) + eps) * g)
 // The routed experts' outputs (slot order) and the split-K partials (slice
 // order) are added in a fixed order, so the result is deterministic.
 // ---------------------------------------------------------------------------
@@ -117,7 +117,7 @@ __global__ void __launch_bounds__(256) k_residual_norm(float* __restrict__ x, co
                                                        const int* __restrict__ pair_row, int k,
                                                        const float* __restrict__ part, int n_part, size_t part_stride,
                                                        const float* __restrict__ g, int d, float eps,
-                                                       bf16* __restrict__ out, float* __restrict__ out_f32) {
+                                                       bf16* __restrict__ out) {
   pdl_trigger();
   pdl_wait();
   extern __shared__ float crow[];  // [d]
@@ -158,7 +158,7 @@ __global__ void __launch_bounds__(256) k_residual_norm(float* __restrict__ x, co
     cr[c] = v;
     ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
   }
-  if (out == nullptr && out_f32 == nullptr) return;
+  if (out == nullptr) return;
   ss = warp_sum(ss);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
   __syncthreads();
@@ -174,15 +174,12 @@ __global__ void __launch_bounds__(256) k_residual_norm(float* __restrict__ x, co
     const float4 v = cr[c];
     const float4 w = g4[c];
     const float4 n = make_float4(v.x * rs * w.x, v.y * rs * w.y, v.z * rs * w.z, v.w * rs * w.w);
-    if (out)
-      reinterpret_cast<uint2*>(out + (size_t)t * d)[c] = make_uint2(pack_bf16x2(n.x, n.y), pack_bf16x2(n.z, n.w));
-    if (out_f32) reinterpret_cast<float4*>(out_f32 + (size_t)t * d)[c] = n;
+    reinterpret_cast<uint2*>(out + (size_t)t * d)[c] = make_uint2(pack_bf16x2(n.x, n.y), pack_bf16x2(n.z, n.w));
   }
 }
 
 cudaError_t run_residual_norm(float* x, const float* yp, const int* pair_row, int k, const float* part, int n_part,
-                              int Tcap, const float* g, int T, int d, float eps, bf16* out, float* out_f32,
-                              cudaStream_t st) {
+                              int Tcap, const float* g, int T, int d, float eps, bf16* out, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
   if (n_part > kMaxPartSplits || k > 8) return cudaErrorInvalidValue;
   const size_t smem = (size_t)d * sizeof(float);
@@ -193,7 +190,7 @@ cudaError_t run_residual_norm(float* x, const float* yp, const int* pair_row, in
     configured = smem;
   }
   {
-    const cudaError_t e_ = launch_pdl(k_residual_norm, dim3(T), dim3(256), smem, st, x, yp, pair_row, k, part, n_part, (size_t)Tcap * d, g, d, eps, out, out_f32);
+    const cudaError_t e_ = launch_pdl(k_residual_norm, dim3(T), dim3(256), smem, st, x, yp, pair_row, k, part, n_part, (size_t)Tcap * d, g, d, eps, out);
     if (e_ != cudaSuccess) return e_;
   }
   return cudaGetLastError();
@@ -265,117 +262,6 @@ cudaError_t run_topk(const float* logits, int T, int E, int k, int* idx, float* 
   if (T == 0) return cudaSuccess;
   {
     const cudaError_t e_ = launch_pdl(k_topk, dim3((T + 7) / 8), dim3(256), 0, st, logits, T, E, k, idx, w);
-    if (e_ != cudaSuccess) return e_;
-  }
-  return cudaGetLastError();
-}
-
-// ---------------------------------------------------------------------------
-// Router logits from the fp32 normalised rows: grid (token groups of kRT,
-// expert groups of kRE); fp32 row x bf16 router weights, fp32 accumulation.
-// Each warp owns 2 experts for all kRT tokens of the CTA.
-// ---------------------------------------------------------------------------
-constexpr int kRT = 8, kRE = 16;
-
-__global__ void __launch_bounds__(256) k_router_logits(const float* __restrict__ un, const bf16* __restrict__ wr,
-                                                       int T, int d, int E, float* __restrict__ logits) {
-  pdl_trigger();
-  pdl_wait();
-  extern __shared__ float su[];  // [kRT][d]
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t0 = blockIdx.x * kRT, e0 = blockIdx.y * kRE;
-  const int d4 = d / 4;
-  // stage the rows in batches of 8 independent 16-byte loads per thread
-  for (int base = threadIdx.x; base < kRT * d4; base += 8 * blockDim.x) {
-    float4 r[8];
-#pragma unroll
-    for (int b = 0; b < 8; ++b) {
-      const int i = base + b * blockDim.x;
-      const int tt = i / d4, c = i - tt * d4;
-      r[b] = (i < kRT * d4 && t0 + tt < T) ? reinterpret_cast<const float4*>(un + (size_t)(t0 + tt) * d)[c]
-                                           : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-#pragma unroll
-    for (int b = 0; b < 8; ++b) {
-      const int i = base + b * blockDim.x;
-      if (i < kRT * d4) reinterpret_cast<float4*>(su)[i] = r[b];
-    }
-  }
-  __syncthreads();
-  const int eb = e0 + warp * 2;
-  // every weight this lane needs, loaded up front (all loads in flight at once)
-  constexpr int kMaxChunks = 16;  // d <= 4096
-  const int n_chunks = (d + 255) / 256;
-  uint4 wv[2][kMaxChunks];
-#pragma unroll
-  for (int i = 0; i < kMaxChunks; ++i)
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      const int c = lane * 8 + i * 256;
-      wv[q][i] = (i < n_chunks && c < d && eb + q < E)
-                     ? __ldg(reinterpret_cast<const uint4*>(wr + (size_t)(eb + q) * d + c))
-                     : make_uint4(0, 0, 0, 0);
-    }
-  float acc[2][kRT];
-#pragma unroll
-  for (int q = 0; q < 2; ++q)
-#pragma unroll
-    for (int tt = 0; tt < kRT; ++tt) acc[q][tt] = 0.f;
-#pragma unroll
-  for (int i = 0; i < kMaxChunks; ++i) {
-    const int c = lane * 8 + i * 256;
-    if (i >= n_chunks || c >= d) break;
-    float wf[2][8];
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&wv[q][i]);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float2 f2 = __bfloat1622float2(h[j]);
-        wf[q][2 * j] = f2.x;
-        wf[q][2 * j + 1] = f2.y;
-      }
-    }
-#pragma unroll
-    for (int tt = 0; tt < kRT; ++tt) {
-      const float4 a = *reinterpret_cast<const float4*>(su + tt * d + c);
-      const float4 b = *reinterpret_cast<const float4*>(su + tt * d + c + 4);
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        float r = acc[q][tt];
-        r = fmaf(a.x, wf[q][0], r);
-        r = fmaf(a.y, wf[q][1], r);
-        r = fmaf(a.z, wf[q][2], r);
-        r = fmaf(a.w, wf[q][3], r);
-        r = fmaf(b.x, wf[q][4], r);
-        r = fmaf(b.y, wf[q][5], r);
-        r = fmaf(b.z, wf[q][6], r);
-        r = fmaf(b.w, wf[q][7], r);
-        acc[q][tt] = r;
-      }
-    }
-  }
-#pragma unroll
-  for (int q = 0; q < 2; ++q)
-#pragma unroll
-    for (int tt = 0; tt < kRT; ++tt) {
-      const float r = warp_sum(acc[q][tt]);
-      if (lane == 0 && eb + q < E && t0 + tt < T) logits[(size_t)(t0 + tt) * E + eb + q] = r;
-    }
-}
-
-cudaError_t run_router_logits(const float* un, const bf16* wr, int T, int d, int E, float* logits, cudaStream_t st) {
-  if (T == 0) return cudaSuccess;
-  const size_t smem = (size_t)kRT * d * sizeof(float);
-  static size_t configured = 0;
-  if (smem > configured) {
-    cudaError_t e = cudaFuncSetAttribute(k_router_logits, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    configured = smem;
-  }
-  dim3 grid((T + kRT - 1) / kRT, (E + kRE - 1) / kRE);
-  {
-    const cudaError_t e_ = launch_pdl(k_router_logits, dim3(grid), dim3(256), smem, st, un, wr, T, d, E, logits);
     if (e_ != cudaSuccess) return e_;
   }
   return cudaGetLastError();
@@ -501,28 +387,8 @@ DG_DEVINL int warp_excl_scan8(int* vals8, int lane) {
 }
 
 // ---------------------------------------------------------------------------
-// Routing, part 1: top-k of every token's logits (one warp per token); each
-// selected (token, expert) sets bit t of that expert's token bitmask.
-// ---------------------------------------------------------------------------
-__global__ void k_topk_mask(const float* __restrict__ logits, int T, int E, int k, int* idx, float* w,
-                            unsigned* __restrict__ mask, int MW) {
-  pdl_trigger();
-  pdl_wait();
-  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (t >= T) return;
-  int* it = idx + (size_t)t * k;
-  float* wt = w + (size_t)t * k;
-  topk_warp(logits + (size_t)t * E, E, k, it, wt);
-  __syncwarp();
-  const int lane = threadIdx.x & 31;
-  if (lane < k) {
-    const int e = it[lane];
-    if (e >= 0 && e < E) atomicOr(&mask[(size_t)e * MW + (t >> 5)], 1u << (t & 31));
-  }
-}
-
-// ---------------------------------------------------------------------------
-// Routing, part 2 (every CTA): per-expert counts from the bitmasks and their
+// Routing after the router GEMM (every CTA): per-expert counts from the token
+// bitmasks the router epilogue set and their
 // exclusive scans (tiny, recomputed by each CTA); CTA 0 publishes counts,
 // offsets, tile lists and statistics.  Each CTA then places its share of the
 // (token, slot) pairs -- row = offset[e] + number of earlier tokens routed to
@@ -643,16 +509,9 @@ __global__ void __launch_bounds__(256) k_group_gather(GroupArgs a, const unsigne
   }
 }
 
-cudaError_t run_route(const float* logits, const bf16* u, int d, bf16* xp, unsigned* mask, unsigned* mask_next,
+cudaError_t run_route(const bf16* u, int d, bf16* xp, unsigned* mask, unsigned* mask_next, int MW,
                       const GroupArgs& a, cudaStream_t st) {
-  if (a.T < 1 || a.T > 1024 || a.E > 256) return cudaErrorInvalidValue;
-  const int MW = (a.T + 31) >> 5;
-  {
-    const cudaError_t e_ = launch_pdl(k_topk_mask, dim3((a.T + 7) / 8), dim3(256), 0, st, logits, a.T, a.E, a.k, a.idx, a.w, mask, MW);
-    if (e_ != cudaSuccess) return e_;
-  }
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  if (a.T < 1 || a.T > 1024 || a.E > 256 || MW * 32 < a.T) return cudaErrorInvalidValue;
   const int P = a.T * a.k;
   const int grid = (P + 7) / 8 < 148 ? (P + 7) / 8 : 148;
   {

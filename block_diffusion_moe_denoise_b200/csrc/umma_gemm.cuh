@@ -17,8 +17,9 @@
 // A problem class P supplies: BN, STAGES, B_STAGE (bytes), EP_SMEM (bytes),
 // TMEM_COLS, Params, num_tiles(), tile(), tx_bytes(), load(), epilogue(),
 // finish(), epilogue_prefetch() (called before the accumulator wait, so an
-// epilogue can pull its inputs into L1 while the main loop runs).  Every wait
-// is bounded (see mbar_wait_bounded).
+// epilogue can pull its inputs into L1 while the main loop runs), and, with
+// PRELOAD, load_w()/load_x(): the weight and activation halves of load().
+// Every wait is bounded (see mbar_wait_bounded).
 #pragma once
 
 #include "common.cuh"
@@ -82,13 +83,32 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
   __syncthreads();
   tc_fence_after();
   pdl_trigger();
-  pdl_wait();
   const uint32_t tmem = *tmem_slot;
-  const int n_tiles = P::num_tiles(p);
   int* err = p.err;
 
   if (warp == 0) {
     if (lane == 0) {
+      // Weight tiles do not depend on the preceding kernel: for problems whose
+      // tile list is static (P::PRELOAD) the first ring slots of this CTA's
+      // first tile are filled with them before the dependency wait, so the
+      // weight stream starts while the predecessor drains.
+      int pre = 0;
+      if constexpr (P::PRELOAD) {
+        if ((int)blockIdx.x < P::num_tiles(p)) {
+          const Tile t0 = P::tile(p, blockIdx.x);
+          if (t0.valid) {
+            pre = t0.nk < P::STAGES ? t0.nk : P::STAGES;
+            const uint32_t tx = P::tx_bytes(p, t0);
+            for (int kb = 0; kb < pre; ++kb) {
+              mbar_arrive_expect_tx(&full[kb], tx);
+              P::load_w(p, t0, kb, smem_u32(sA + (size_t)kb * kAStage), smem_u32(sB + (size_t)kb * P::B_STAGE),
+                        &full[kb]);
+            }
+          }
+        }
+      }
+      pdl_wait();
+      const int n_tiles = P::num_tiles(p);
       uint32_t stage = 0, phase = 0;
       for (int v = blockIdx.x; v < n_tiles; v += gridDim.x) {
         const Tile t = P::tile(p, v);
@@ -96,16 +116,25 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
         const uint32_t tx = P::tx_bytes(p, t);
         bool ok = true;
         for (int kb = 0; kb < t.nk; ++kb) {
-          if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, err)) { ok = false; break; }
-          mbar_arrive_expect_tx(&full[stage], tx);
-          P::load(p, t, kb, smem_u32(sA + (size_t)stage * kAStage), smem_u32(sB + (size_t)stage * P::B_STAGE),
-                  &full[stage]);
+          const uint32_t sa = smem_u32(sA + (size_t)stage * kAStage), sb = smem_u32(sB + (size_t)stage * P::B_STAGE);
+          if (pre > 0) {  // slot already armed and holding its weight tile
+            --pre;
+            P::load_x(p, t, kb, sa, sb, &full[stage]);
+          } else {
+            if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, err)) { ok = false; break; }
+            mbar_arrive_expect_tx(&full[stage], tx);
+            P::load(p, t, kb, sa, sb, &full[stage]);
+          }
           if (++stage == P::STAGES) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
       }
+    } else {
+      pdl_wait();
     }
   } else if (warp == 1) {
+    pdl_wait();
+    const int n_tiles = P::num_tiles(p);
     if (lane == 0) {
       uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
       for (int v = blockIdx.x; v < n_tiles; v += gridDim.x) {
@@ -135,6 +164,8 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
       }
     }
   } else {
+    pdl_wait();
+    const int n_tiles = P::num_tiles(p);
     const int q = warp & 3;            // TMEM lane quadrant of this warp
     const int row = q * 32 + lane;     // accumulator row (M index) owned by this thread
     P::epilogue_init(p, row, ep_smem);
@@ -165,12 +196,17 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
 // Default no-op hooks for problems that need none.
 struct ProblemBase {
   static constexpr int EP_SMEM = 0;
+  static constexpr bool PRELOAD = false;  // true: static tiles, load_w / load_x split of load
   template <class Params>
   DG_DEVINL static void epilogue_init(const Params&, int, uint8_t*) {}
   template <class Params>
   DG_DEVINL static void finish(const Params&, int, uint8_t*) {}
   template <class Params>
   DG_DEVINL static void epilogue_prefetch(const Params&, const Tile&, int) {}
+  template <class Params>
+  DG_DEVINL static void load_w(const Params&, const Tile&, int, uint32_t, uint32_t, uint64_t*) {}
+  template <class Params>
+  DG_DEVINL static void load_x(const Params&, const Tile&, int, uint32_t, uint32_t, uint64_t*) {}
 };
 
 DG_DEVINL void prefetch_l1(const void* ptr) { asm volatile("prefetch.global.L1 [%0];" ::"l"(ptr)); }

@@ -58,7 +58,8 @@ extern "C" {
 /* Model shape and sampler knobs.  Supported shapes: d_model, ffn_expert and
  * ffn_shared multiples of 64 (d_model also of 128 and 256); head_dim 64, 128
  * or 256; (n_q_heads+2*n_kv_heads)*head_dim a multiple of 256; n_q_heads a
- * multiple of n_kv_heads; n_experts <= 256; top_k <= 8; vocab a multiple of
+ * multiple of n_kv_heads; n_experts a multiple of 16 up to 128 (the router
+ * is one tensor-core tile wide); top_k <= 8; vocab a multiple of
  * 256; canvas <= 256. */
 typedef struct dg_config {
   int n_layers, d_model, n_q_heads, n_kv_heads, head_dim;

@@ -97,6 +97,22 @@ def test_moe_path(setup):
     assert ex < REL_L2
 
 
+def test_router_epilogue(setup):
+    """The shared-expert GEMM's router tile: its fp32 logits against the
+    oracle's, and the top-k its epilogue picked against the oracle's routing
+    rule applied to those same logits (exact experts, ties to the lower id;
+    renormalised softmax weights to fp32 rounding)."""
+    h, rec = setup["h"], setup["tr"]
+    T, k, E = CFG.canvas, CFG.top_k, CFG.n_experts
+    gl = h.debug_buffer("router_logits", torch.float32, (256, E))[:T].cpu().numpy().astype(np.float64)
+    assert rel_l2(gl, rec["router_logits"]) < REL_L2
+    idx = h.debug_buffer("idx", torch.int32, (T, k)).cpu().numpy()
+    wts = h.debug_buffer("w", torch.float32, (T, k)).cpu().numpy()
+    ridx, rw = OL.route(gl, k)
+    np.testing.assert_array_equal(idx, ridx)
+    np.testing.assert_allclose(wts, rw, rtol=2e-6, atol=1e-7)
+
+
 def test_lm_head_sampled_rows(setup):
     h, rec, ora = setup["h"], setup["tr"], setup["ora"]
     stats = h.debug_buffer("stats", torch.float32, (256, 4)).cpu().numpy().astype(np.float64)

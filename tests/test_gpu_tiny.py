@@ -86,6 +86,12 @@ def test_layer_intermediates(model, T):
     same = routing_match(idx, rec["idx"])
     amb = ambiguous_tokens([rec], k)
     assert same[~amb].all(), np.nonzero(~same & ~amb)
+    # the router epilogue's top-k on the GPU's own fp32 logits follows the
+    # routing rule exactly
+    gl = h.debug_buffer("router_logits", torch.float32, (Tcap, CFG.n_experts))[:T].cpu().numpy().astype(np.float64)
+    ridx, rw = OL.route(gl, k)
+    np.testing.assert_array_equal(idx, ridx)
+    np.testing.assert_allclose(wts, rw, rtol=2e-6, atol=1e-7)
     for t in np.nonzero(same)[0]:
         for j in range(k):
             jj = list(rec["idx"][t]).index(idx[t, j])
