@@ -9,12 +9,13 @@
 // them all -- over one range of keys (split-KV when the query tiles alone
 // cannot fill the GPU; partial (O, max, sum) are merged by k_attn_combine).
 //   warp 0     TMA producer: 64-key K tiles [64 x D] and V^T tiles [D x 64] in
-//              separate two-slot rings (the cache keeps V transposed so both
+//              separate three-slot rings (the cache keeps V transposed so both
 //              MMAs read K-major operands); a K slot is refilled as soon as the
 //              S MMA that read it completes, a V slot once its PV MMA completes
-//   warp 1     MMA issuer: S = Q K^T into one of two TMEM buffers (N = 64),
-//              O += P V^T into TMEM (N = D); S(j+1) is issued before PV(j)
-//   warps 2-5  one query row per thread: Q row into shared memory, then per
+//   warp 1     MMA issuer: S = Q K^T into one of two TMEM buffers (N = 64, Q
+//              read from tensor memory), O += P V^T into TMEM (N = D); S(j+1)
+//              is issued before PV(j)
+//   warps 2-5  one query row per thread: Q row into tensor memory, then per
 //              tile the exp2-domain online softmax on the S row read from TMEM,
 //              P row (bf16) written into the swizzled shared tile PV reads.
 //              The running max is only moved (and O, l rescaled in TMEM) when
@@ -28,17 +29,19 @@ namespace dg {
 
 constexpr int kAQ = 128;        // query rows per CTA
 constexpr int kAK = 64;         // keys per tile
-constexpr int kAStages = 2;     // K/V ring depth
+constexpr int kAStages = 3;     // K/V ring depth
 constexpr float kRescaleLog2 = 8.0f;
+
+// Tensor memory (512 columns): O fp32 in [0, D), the two S buffers at 256 and
+// 320, Q (bf16 pairs, the A operand of S = Q K^T) in [384, 384 + D/2).
+constexpr uint32_t kTmS = 256, kTmQ = 384;
 
 template <int D>
 struct AttnSmem {
-  static constexpr int kQ = kAQ * D * 2;            // Q: D/64 blocks of [128 x 128 B]
   static constexpr int kK = kAK * D * 2;            // K tile: D/64 blocks of [64 x 128 B]
   static constexpr int kV = D * kAK * 2;            // V^T tile: [D x 128 B]
   static constexpr int kP = kAQ * kAK * 2;          // P tile: [128 x 128 B]
-  static constexpr size_t q_off = 0;
-  static constexpr size_t k_off = q_off + kQ;
+  static constexpr size_t k_off = 0;
   static constexpr size_t v_off = k_off + (size_t)kAStages * kK;
   static constexpr size_t p_off = v_off + (size_t)kAStages * kV;
   static constexpr size_t bar_off = p_off + 2 * (size_t)kP;
@@ -47,6 +50,7 @@ struct AttnSmem {
   // at least 120 KB so two CTAs (each owning all 512 TMEM columns) never share an SM
   static constexpr size_t total = misc_off + 16 + 1024 > 120 * 1024 ? misc_off + 16 + 1024 : 120 * 1024;
 };
+static_assert(AttnSmem<256>::total <= 227 * 1024, "attention shared memory exceeds the per-CTA limit");
 
 DG_DEVINL void tmem_st16(uint32_t taddr, const float* v) {
   asm volatile(
@@ -60,12 +64,22 @@ DG_DEVINL void tmem_st16(uint32_t taddr, const float* v) {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+DG_DEVINL void tmem_st16_raw(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+DG_DEVINL void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 template <int D>
 __global__ void __launch_bounds__(192, 1) k_attn_tc(const __grid_constant__ AttnArgs a) {
   using S = AttnSmem<D>;
   extern __shared__ uint8_t dyn_smem[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~(uintptr_t)1023);
-  uint8_t* sQ = base + S::q_off;
   uint8_t* sK = base + S::k_off;
   uint8_t* sV = base + S::v_off;
   uint8_t* sP = base + S::p_off;
@@ -123,8 +137,8 @@ __global__ void __launch_bounds__(192, 1) k_attn_tc(const __grid_constant__ Attn
   tc_fence_after();
   pdl_trigger();
   pdl_wait();
-  const uint32_t tmem = *tmem_slot;   // O: columns [0, D); S buffers at 256 and 320
-  const uint32_t tm_o = tmem, tm_s0 = tmem + 256;
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tm_o = tmem, tm_s0 = tmem + kTmS, tm_q = tmem + kTmQ;
 
   // cache rows of this (request, layer, kv head) in the two tensor maps
   const long long krow0 = a.k_row0 + (long long)a.req[slot] * a.req_rows_k + (long long)g * a.cap;
@@ -132,8 +146,8 @@ __global__ void __launch_bounds__(192, 1) k_attn_tc(const __grid_constant__ Attn
 
   if (warp == 0) {
     if (lane == 0) {
-      // issue order K(0), K(1), then V(j), K(j+2) for j = 0, 1, ...: K(j+2)
-      // waits for S(j), V(j) for PV(j-2), matching the MMA issue order
+      // issue order K(0..S-1), then V(j), K(j+S) for j = 0, 1, ... (S = ring
+      // depth): K(j+S) waits for S(j), V(j) for PV(j-S), matching the MMA order
       auto load_k = [&](int j) -> bool {
         const int st = j % kAStages;
         if (!mbar_wait_bounded(&k_empty[st], ((j / kAStages) & 1) ^ 1, abort_flag, err)) return false;
@@ -163,7 +177,7 @@ __global__ void __launch_bounds__(192, 1) k_attn_tc(const __grid_constant__ Attn
     if (lane == 0 && n_tiles > 0) {
       const uint32_t idesc_s = umma_idesc_bf16(128, kAK);
       const uint32_t idesc_o = umma_idesc_bf16(128, D);
-      const uint32_t q0 = smem_u32(sQ), p0 = smem_u32(sP);
+      const uint32_t p0 = smem_u32(sP);
       bool ok = mbar_wait_bounded(q_ready, 0, abort_flag, err);
       // S(j) = Q K_j^T into S buffer j%2
       auto issue_s = [&](int j) -> bool {
@@ -176,8 +190,8 @@ __global__ void __launch_bounds__(192, 1) k_attn_tc(const __grid_constant__ Attn
         for (int kb = 0; kb < D / 64; ++kb)
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            umma_bf16(tm_s0 + b * kAK, umma_sdesc_k128(q0 + kb * (kAQ * 128) + 32 * k),
-                      umma_sdesc_k128(k0 + kb * (kAK * 128) + 32 * k), idesc_s, (kb | k) != 0 ? 1u : 0u);
+            umma_bf16_ts(tm_s0 + b * kAK, tm_q + (uint32_t)(kb * 32 + k * 8),
+                         umma_sdesc_k128(k0 + kb * (kAK * 128) + 32 * k), idesc_s, (kb | k) != 0 ? 1u : 0u);
         umma_commit(&k_empty[stage]);
         umma_commit(&s_full[b]);
         return true;
@@ -207,16 +221,24 @@ __global__ void __launch_bounds__(192, 1) k_attn_tc(const __grid_constant__ Attn
     const bool valid = qr < rows;
     const int h = g * G + (valid ? qr / a.Tr : 0);
     const int t = slot * a.Tr + (valid ? qr % a.Tr : 0);
-    // Q row -> shared memory in the 128-byte-swizzled K-major layout
+    // Q row -> tensor memory lane `row`, bf16 pairs in columns kTmQ + [0, D/2)
     {
       const uint4* src = reinterpret_cast<const uint4*>(a.q + ((size_t)h * a.q_T + t) * D);
 #pragma unroll
-      for (int c = 0; c < D / 8; ++c) {
-        const uint4 v = valid ? src[c] : make_uint4(0, 0, 0, 0);
-        const int kb = c >> 3, ch = c & 7;
-        *reinterpret_cast<uint4*>(sQ + kb * (kAQ * 128) + row * 128 + ((ch ^ (row & 7)) << 4)) = v;
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[16];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint4 v = valid ? src[c * 4 + i] : make_uint4(0, 0, 0, 0);
+          r[4 * i] = v.x;
+          r[4 * i + 1] = v.y;
+          r[4 * i + 2] = v.z;
+          r[4 * i + 3] = v.w;
+        }
+        tmem_st16_raw(tm_q + lane_off + c * 16, r);
       }
-      fence_proxy_async_smem();
+      tmem_st_wait();
+      tc_fence_before();
       mbar_arrive(q_ready);
     }
     const float sl2 = a.scale * 1.4426950408889634f;

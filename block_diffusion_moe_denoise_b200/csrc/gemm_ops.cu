@@ -478,22 +478,22 @@ struct P_SGU : ProblemBase {
       for (int i = 0; i < 16; i += 4) lg[i / 4] = make_float4(z[i], z[i + 1], z[i + 2], z[i + 3]);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        // experts arrive in ascending id order; a strict comparison keeps the
-        // earlier (lower) id ahead of an equal logit
-        float v = z[i];
-        int e = c0 + i;
+        // Experts arrive in ascending id order; strict comparisons keep the
+        // earlier (lower) id ahead of an equal logit.  The list is sorted, so
+        // the comparisons are monotone in r and every slot's new value follows
+        // from the old list directly (no chain through the list).
+        const float v = z[i];
         if (v > tv[7]) {
+          bool gt[8];
 #pragma unroll
-          for (int r = 0; r < 8; ++r) {
-            if (v > tv[r]) {
-              const float fv = tv[r];
-              const int fi = ti[r];
-              tv[r] = v;
-              ti[r] = e;
-              v = fv;
-              e = fi;
-            }
+          for (int r = 0; r < 8; ++r) gt[r] = v > tv[r];
+#pragma unroll
+          for (int r = 7; r > 0; --r) {
+            tv[r] = gt[r] ? (gt[r - 1] ? tv[r - 1] : v) : tv[r];
+            ti[r] = gt[r] ? (gt[r - 1] ? ti[r - 1] : c0 + i) : ti[r];
           }
+          tv[0] = gt[0] ? v : tv[0];
+          ti[0] = gt[0] ? c0 + i : ti[0];
         }
       }
     }
