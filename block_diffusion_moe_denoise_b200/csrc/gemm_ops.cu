@@ -41,7 +41,7 @@ DG_DEVINL void store_bf16x16(__nv_bfloat16* dst, const float* v) {
 // per-pass table the embedding kernel writes.
 // ---------------------------------------------------------------------------
 struct P_QKV : ProblemBase {
-  static constexpr int BN = 128, STAGES = 6, B_STAGE = BN * 128, TMEM_COLS = 256;
+  static constexpr int BN = 128, STAGES = 3, KB = 2, B_STAGE = BN * 128, TMEM_COLS = 256;
   struct Params {
     CUtensorMap tmA;  // normed tokens [Tcap, d]
     CUtensorMap tmB;  // w_qkv [(Hq+2Hkv)*D, d], 64-row boxes
@@ -266,7 +266,7 @@ struct P_WPART : ProblemBase {
 // A rows 0..63 = W_gate rows, 64..127 = W_up rows of the same hidden units.
 // ---------------------------------------------------------------------------
 struct P_EGU : ProblemBase {
-  static constexpr int BN = kExpertRows, STAGES = 8, B_STAGE = BN * 128, TMEM_COLS = 128;
+  static constexpr int BN = kExpertRows, STAGES = 4, KB = 2, B_STAGE = BN * 128, TMEM_COLS = 128;
   static constexpr int EP_SMEM = 64 * 17 * 4;
   struct Params {
     CUtensorMap tmG;  // w_gate as [E*fe, d]
@@ -337,7 +337,7 @@ struct P_EGU : ProblemBase {
 // of expert e for its grouped rows nt*64..+63; each row scaled by its gate weight.
 // ---------------------------------------------------------------------------
 struct P_ED : ProblemBase {
-  static constexpr int BN = kExpertRows, STAGES = 8, B_STAGE = BN * 128, TMEM_COLS = 128;
+  static constexpr int BN = kExpertRows, STAGES = 4, KB = 2, B_STAGE = BN * 128, TMEM_COLS = 128;
   struct Params {
     CUtensorMap tmW;  // w_down as [E*d, fe]
     CUtensorMap tmH;  // hidden [rows_cap, fe], 64-row boxes
@@ -404,7 +404,7 @@ struct P_ED : ProblemBase {
 // the grouping kernel that follows waits on them.
 // ---------------------------------------------------------------------------
 struct P_SGU : ProblemBase {
-  static constexpr int BN = 128, STAGES = 6, B_STAGE = BN * 128, TMEM_COLS = 256;
+  static constexpr int BN = 128, STAGES = 3, KB = 2, B_STAGE = BN * 128, TMEM_COLS = 256;
   static constexpr int kHid = 32;  // shared hidden units per tile
   struct Params {
     CUtensorMap tmX;  // normed tokens [Tcap, d]

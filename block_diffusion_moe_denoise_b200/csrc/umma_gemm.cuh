@@ -3,7 +3,10 @@
 //   D[128 x N] = A[128 x K] * B[N x K]^T      (bf16 operands, fp32 accumulator in TMEM)
 //
 // Both operands are K-major tiles staged in shared memory by TMA with the
-// 128-byte swizzle, 64 bf16 (one 128-byte row) per k-block.  Roles:
+// 128-byte swizzle, 64 bf16 (one 128-byte row) per k-block.  A ring stage holds
+// P::KB consecutive k-blocks: every stage costs a pair of barrier round trips
+// (producer <-> MMA issuer), which dominates at small N, so small-N problems
+// take two k-blocks per stage.  Roles:
 //   warp 0 (one lane)   TMA producer: fills a STAGES-deep ring of (A, B) tiles
 //   warp 1 (one lane)   MMA issuer: 4 x tcgen05.mma (K = 16 each) per k-block,
 //                       tcgen05.commit frees the ring slot / signals the accumulator
@@ -14,7 +17,7 @@
 // of one tile overlaps the main loop of the next.  Tiles are assigned
 // statically (tile v to CTA v mod gridDim.x), so every role walks the same list.
 //
-// A problem class P supplies: BN, STAGES, B_STAGE (bytes), EP_SMEM (bytes),
+// A problem class P supplies: BN, STAGES, KB, B_STAGE (bytes per k-block), EP_SMEM (bytes),
 // TMEM_COLS, Params, num_tiles(), tile(), tx_bytes(), load(), epilogue(),
 // finish(), epilogue_prefetch() (called before the accumulator wait, so an
 // epilogue can pull its inputs into L1 while the main loop runs), and, with
@@ -38,9 +41,11 @@ constexpr int kAStage = 128 * 128;  // 128 rows x 128 bytes
 template <class P>
 struct GemmSmem {
   static constexpr int kStages = P::STAGES;
+  static constexpr size_t a_stage = (size_t)P::KB * kAStage;
+  static constexpr size_t b_stage = (size_t)P::KB * P::B_STAGE;
   static constexpr size_t a_off = 0;
-  static constexpr size_t b_off = a_off + (size_t)kStages * kAStage;
-  static constexpr size_t ep_off = b_off + (size_t)kStages * P::B_STAGE;
+  static constexpr size_t b_off = a_off + (size_t)kStages * a_stage;
+  static constexpr size_t ep_off = b_off + (size_t)kStages * b_stage;
   static constexpr size_t bar_off = (ep_off + P::EP_SMEM + 15) & ~(size_t)15;
   static constexpr size_t misc_off = bar_off + (2 * kStages + 4) * 8;
   static constexpr size_t total = misc_off + 16 + 1024;  // + alignment slack
@@ -92,17 +97,20 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
       // tile list is static (P::PRELOAD) the first ring slots of this CTA's
       // first tile are filled with them before the dependency wait, so the
       // weight stream starts while the predecessor drains.
-      int pre = 0;
+      int pre = 0;  // stages of the first tile armed before the wait
       if constexpr (P::PRELOAD) {
         if ((int)blockIdx.x < P::num_tiles(p)) {
           const Tile t0 = P::tile(p, blockIdx.x);
           if (t0.valid) {
-            pre = t0.nk < P::STAGES ? t0.nk : P::STAGES;
-            const uint32_t tx = P::tx_bytes(p, t0);
-            for (int kb = 0; kb < pre; ++kb) {
-              mbar_arrive_expect_tx(&full[kb], tx);
-              P::load_w(p, t0, kb, smem_u32(sA + (size_t)kb * kAStage), smem_u32(sB + (size_t)kb * P::B_STAGE),
-                        &full[kb]);
+            const int n_st = (t0.nk + P::KB - 1) / P::KB;
+            pre = n_st < P::STAGES ? n_st : P::STAGES;
+            for (int st = 0; st < pre; ++st) {
+              const int kb = st * P::KB;
+              const int nsub = t0.nk - kb < P::KB ? t0.nk - kb : P::KB;
+              mbar_arrive_expect_tx(&full[st], P::tx_bytes(p, t0) * (uint32_t)nsub);
+              for (int j = 0; j < nsub; ++j)
+                P::load_w(p, t0, kb + j, smem_u32(sA + st * S::a_stage + (size_t)j * kAStage),
+                          smem_u32(sB + st * S::b_stage + (size_t)j * P::B_STAGE), &full[st]);
             }
           }
         }
@@ -115,15 +123,21 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
         if (!t.valid) continue;
         const uint32_t tx = P::tx_bytes(p, t);
         bool ok = true;
-        for (int kb = 0; kb < t.nk; ++kb) {
-          const uint32_t sa = smem_u32(sA + (size_t)stage * kAStage), sb = smem_u32(sB + (size_t)stage * P::B_STAGE);
-          if (pre > 0) {  // slot already armed and holding its weight tile
+        for (int kb = 0; kb < t.nk; kb += P::KB) {
+          const int nsub = t.nk - kb < P::KB ? t.nk - kb : P::KB;
+          uint8_t* sa = sA + stage * S::a_stage;
+          uint8_t* sb = sB + stage * S::b_stage;
+          if (pre > 0) {  // slot already armed and holding its weight tiles
             --pre;
-            P::load_x(p, t, kb, sa, sb, &full[stage]);
+            for (int j = 0; j < nsub; ++j)
+              P::load_x(p, t, kb + j, smem_u32(sa + (size_t)j * kAStage), smem_u32(sb + (size_t)j * P::B_STAGE),
+                        &full[stage]);
           } else {
             if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, err)) { ok = false; break; }
-            mbar_arrive_expect_tx(&full[stage], tx);
-            P::load(p, t, kb, sa, sb, &full[stage]);
+            mbar_arrive_expect_tx(&full[stage], tx * (uint32_t)nsub);
+            for (int j = 0; j < nsub; ++j)
+              P::load(p, t, kb + j, smem_u32(sa + (size_t)j * kAStage), smem_u32(sb + (size_t)j * P::B_STAGE),
+                      &full[stage]);
           }
           if (++stage == P::STAGES) { stage = 0; phase ^= 1; }
         }
@@ -145,15 +159,21 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
         const uint32_t d_tmem = tmem + acc * P::BN;
         const uint32_t idesc = umma_idesc_bf16(128, (uint32_t)t.n_mma);
         bool ok = true;
-        for (int kb = 0; kb < t.nk; ++kb) {
+        for (int kb = 0; kb < t.nk; kb += P::KB) {
+          const int nsub = t.nk - kb < P::KB ? t.nk - kb : P::KB;
           if (!mbar_wait_bounded(&full[stage], phase, abort_flag, err)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(sA + (size_t)stage * kAStage);
-          const uint32_t b0 = smem_u32(sB + (size_t)stage * P::B_STAGE);
+          const uint32_t a0 = smem_u32(sA + stage * S::a_stage);
+          const uint32_t b0 = smem_u32(sB + stage * S::b_stage);
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            umma_bf16(d_tmem, umma_sdesc_k128(a0 + 32 * k), umma_sdesc_k128(b0 + 32 * k), idesc,
-                      (kb | k) != 0 ? 1u : 0u);
+          for (int j = 0; j < P::KB; ++j) {
+            if (j < nsub) {
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                umma_bf16(d_tmem, umma_sdesc_k128(a0 + j * kAStage + 32 * k),
+                          umma_sdesc_k128(b0 + j * P::B_STAGE + 32 * k), idesc, (kb | j | k) != 0 ? 1u : 0u);
+            }
+          }
           umma_commit(&empty[stage]);
           if (++stage == P::STAGES) { stage = 0; phase ^= 1; }
         }
@@ -197,6 +217,7 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
 struct ProblemBase {
   static constexpr int EP_SMEM = 0;
   static constexpr bool PRELOAD = false;  // true: static tiles, load_w / load_x split of load
+  static constexpr int KB = 1;            // k-blocks per ring stage
   template <class Params>
   DG_DEVINL static void epilogue_init(const Params&, int, uint8_t*) {}
   template <class Params>
