@@ -8,10 +8,11 @@
 // query heads of a KV head are stacked as G*Tr rows so one K/V tile serves
 // them all -- over one range of keys (split-KV when the query tiles alone
 // cannot fill the GPU; partial (O, max, sum) are merged by k_attn_combine).
-//   warp 0     TMA producer: 64-key K tiles [64 x D] and V^T tiles [D x 64] in
-//              separate three-slot rings (the cache keeps V transposed so both
-//              MMAs read K-major operands); a K slot is refilled as soon as the
-//              S MMA that read it completes, a V slot once its PV MMA completes
+//   warps 0, 6 TMA producers: 64-key K tiles [64 x D] (warp 0) and V^T tiles
+//              [D x 64] (warp 6) in separate three-slot rings (the cache keeps V
+//              transposed so both MMAs read K-major operands); a K slot is
+//              refilled as soon as the S MMA that read it completes, a V slot
+//              once its PV MMA completes
 //   warp 1     MMA issuer: S = Q K^T into one of two TMEM buffers (N = 64, Q
 //              read from tensor memory), O += P V^T into TMEM (N = D); S(j+1)
 //              is issued before PV(j)
@@ -31,6 +32,8 @@ constexpr int kAQ = 128;        // query rows per CTA
 constexpr int kAK = 64;         // keys per tile
 constexpr int kAStages = 3;     // K/V ring depth
 constexpr float kRescaleLog2 = 8.0f;
+constexpr int kVWarp = 6;                 // V^T producer
+constexpr int kAttnThreads = 32 * (kVWarp + 1);
 
 // Tensor memory (512 columns): O fp32 in [0, D), the two S buffers at 256 and
 // 320, Q (bf16 pairs, the A operand of S = Q K^T) in [384, 384 + D/2).
@@ -52,18 +55,6 @@ struct AttnSmem {
 };
 static_assert(AttnSmem<256>::total <= 227 * 1024, "attention shared memory exceeds the per-CTA limit");
 
-DG_DEVINL void tmem_st16(uint32_t taddr, const float* v) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
-          taddr),
-      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
-      "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
-      "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
-      "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
-      "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])));
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-
 DG_DEVINL void tmem_st16_raw(uint32_t taddr, const uint32_t* r) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
@@ -76,7 +67,7 @@ DG_DEVINL void tmem_st16_raw(uint32_t taddr, const uint32_t* r) {
 DG_DEVINL void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 template <int D>
-__global__ void __launch_bounds__(192, 1) k_attn_tc(const __grid_constant__ AttnArgs a) {
+__global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_constant__ AttnArgs a) {
   using S = AttnSmem<D>;
   extern __shared__ uint8_t dyn_smem[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~(uintptr_t)1023);
@@ -144,10 +135,9 @@ __global__ void __launch_bounds__(192, 1) k_attn_tc(const __grid_constant__ Attn
   const long long krow0 = a.k_row0 + (long long)a.req[slot] * a.req_rows_k + (long long)g * a.cap;
   const long long vrow0 = a.v_row0 + (long long)a.req[slot] * a.req_rows_v + (long long)g * D;
 
-  if (warp == 0) {
+  if (warp == 0 || warp == kVWarp) {
     if (lane == 0) {
-      // issue order K(0..S-1), then V(j), K(j+S) for j = 0, 1, ... (S = ring
-      // depth): K(j+S) waits for S(j), V(j) for PV(j-S), matching the MMA order
+      // K(j) waits for S(j - depth) to free its slot, V(j) for PV(j - depth)
       auto load_k = [&](int j) -> bool {
         const int st = j % kAStages;
         if (!mbar_wait_bounded(&k_empty[st], ((j / kAStages) & 1) ^ 1, abort_flag, err)) return false;
@@ -166,11 +156,13 @@ __global__ void __launch_bounds__(192, 1) k_attn_tc(const __grid_constant__ Attn
         tma_load_2d(smem_u32(sV + (size_t)st * S::kV), &a.tm_vt, k_begin + j * kAK, (int)vrow0, &v_full[st]);
         return true;
       };
+      // warp 0 streams K, the last warp V: a V load waits for PV(j - depth),
+      // which must not hold back the K stream (and the other way round)
       bool ok = true;
-      for (int j = 0; ok && j < kAStages && j < n_tiles; ++j) ok = load_k(j);
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        ok = load_v(j);
-        if (ok && j + kAStages < n_tiles) ok = load_k(j + kAStages);
+      if (warp == 0) {
+        for (int j = 0; ok && j < n_tiles; ++j) ok = load_k(j);
+      } else {
+        for (int j = 0; ok && j < n_tiles; ++j) ok = load_v(j);
       }
     }
   } else if (warp == 1) {
@@ -435,7 +427,7 @@ static cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st) {
   const int G = a.Hq / a.Hkv;
   dim3 grid((G * a.Tr + kAQ - 1) / kAQ, a.Hkv * a.n_slots, a.n_split);
   {
-    const cudaError_t e_ = launch_pdl(k_attn_tc<D>, dim3(grid), dim3(192), smem, st, a);
+    const cudaError_t e_ = launch_pdl(k_attn_tc<D>, dim3(grid), dim3(kAttnThreads), smem, st, a);
     if (e_ != cudaSuccess) return e_;
   }
   cudaError_t e = cudaGetLastError();

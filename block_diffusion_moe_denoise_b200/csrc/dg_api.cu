@@ -45,7 +45,7 @@ struct Plan {
 
 bool config_ok(const dg_config* c) {
   if (!c) return false;
-  if (c->n_layers < 1 || c->d_model < 256 || c->d_model % 256 != 0) return false;
+  if (c->n_layers < 1 || c->d_model < 256 || c->d_model > 4096 || c->d_model % 256 != 0) return false;
   if (!(c->head_dim == 64 || c->head_dim == 128 || c->head_dim == 256)) return false;
   if (c->n_kv_heads < 1 || c->n_q_heads < 1 || c->n_q_heads % c->n_kv_heads != 0) return false;
   if ((c->n_q_heads * c->head_dim) % 128 != 0 || (c->n_kv_heads * c->head_dim) % 128 != 0) return false;

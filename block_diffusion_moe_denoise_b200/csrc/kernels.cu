@@ -107,90 +107,93 @@ cudaError_t run_rmsnorm(const float* x, const float* g, int T, int d, float eps,
 }
 
 // ---------------------------------------------------------------------------
-// Residual update + RMSNorm, one CTA per token row:
+// Residual update + RMSNorm, one CTA per token row, 8 consecutive features per
+// thread so every input row is read with all loads in flight at once:
 //   x[t] += sum_j Yp[row(t, j)] + sum_s part[s][t]
 //   out[t] = bf16(x[t] / sqrt(mean(x[t]^2) + eps) * g)
 // The routed experts' outputs (slot order) and the split-K partials (slice
 // order) are added in a fixed order, so the result is deterministic.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) k_residual_norm(float* __restrict__ x, const float* __restrict__ yp,
-                                                       const int* __restrict__ pair_row, int k,
-                                                       const float* __restrict__ part, int n_part, size_t part_stride,
-                                                       const float* __restrict__ g, int d, float eps,
-                                                       bf16* __restrict__ out) {
+__global__ void __launch_bounds__(512) k_residual_norm(float* __restrict__ x, const float* __restrict__ yp,
+                                                        const int* __restrict__ pair_row, int k,
+                                                        const float* __restrict__ part, int n_part,
+                                                        size_t part_stride, const float* __restrict__ g, int d,
+                                                        float eps, bf16* __restrict__ out) {
   pdl_trigger();
   pdl_wait();
-  extern __shared__ float crow[];  // [d]
-  __shared__ float red[8];
+  __shared__ float red[32];
   const int t = blockIdx.x;
+  const int c = threadIdx.x * 2;  // first of this thread's two float4 columns
   float4* xr = reinterpret_cast<float4*>(x + (size_t)t * d);
-  float4* cr = reinterpret_cast<float4*>(crow);
   int rows[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) rows[j] = j < k ? pair_row[(size_t)t * k + j] : 0;
-  float ss = 0.f;
-  for (int c = threadIdx.x; c < d / 4; c += blockDim.x) {
-    float4 v = xr[c];
+  float4 v[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    v[h] = xr[c + h];
     float4 y[8], q[kMaxPartSplits];
 #pragma unroll
     for (int j = 0; j < 8; ++j)
-      if (j < k) y[j] = reinterpret_cast<const float4*>(yp + (size_t)rows[j] * d)[c];
+      if (j < k) y[j] = reinterpret_cast<const float4*>(yp + (size_t)rows[j] * d)[c + h];
 #pragma unroll
     for (int j = 0; j < kMaxPartSplits; ++j)
-      if (j < n_part) q[j] = reinterpret_cast<const float4*>(part + j * part_stride + (size_t)t * d)[c];
+      if (j < n_part) q[j] = reinterpret_cast<const float4*>(part + j * part_stride + (size_t)t * d)[c + h];
 #pragma unroll
     for (int j = 0; j < 8; ++j)
       if (j < k) {
-        v.x += y[j].x;
-        v.y += y[j].y;
-        v.z += y[j].z;
-        v.w += y[j].w;
+        v[h].x += y[j].x;
+        v[h].y += y[j].y;
+        v[h].z += y[j].z;
+        v[h].w += y[j].w;
       }
 #pragma unroll
     for (int j = 0; j < kMaxPartSplits; ++j)
       if (j < n_part) {
-        v.x += q[j].x;
-        v.y += q[j].y;
-        v.z += q[j].z;
-        v.w += q[j].w;
+        v[h].x += q[j].x;
+        v[h].y += q[j].y;
+        v[h].z += q[j].z;
+        v[h].w += q[j].w;
       }
-    if (k || n_part) xr[c] = v;
-    cr[c] = v;
-    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  }
+  if (k || n_part) {
+    xr[c] = v[0];
+    xr[c + 1] = v[1];
   }
   if (out == nullptr) return;
+  float ss = 0.f;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) ss += v[h].x * v[h].x + v[h].y * v[h].y + v[h].z * v[h].z + v[h].w * v[h].w;
   ss = warp_sum(ss);
+  const int nw = blockDim.x >> 5;
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
   __syncthreads();
   if (threadIdx.x < 32) {
-    float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
-    v = warp_sum(v);
-    if (threadIdx.x == 0) red[0] = v;
+    float r = threadIdx.x < nw ? red[threadIdx.x] : 0.f;
+    r = warp_sum(r);
+    if (threadIdx.x == 0) red[0] = r;
   }
   __syncthreads();
   const float rs = rsqrtf(red[0] / (float)d + eps);
   const float4* g4 = reinterpret_cast<const float4*>(g);
-  for (int c = threadIdx.x; c < d / 4; c += blockDim.x) {
-    const float4 v = cr[c];
-    const float4 w = g4[c];
-    const float4 n = make_float4(v.x * rs * w.x, v.y * rs * w.y, v.z * rs * w.z, v.w * rs * w.w);
-    reinterpret_cast<uint2*>(out + (size_t)t * d)[c] = make_uint2(pack_bf16x2(n.x, n.y), pack_bf16x2(n.z, n.w));
+  uint4 o;
+  {
+    const float4 w0 = g4[c], w1 = g4[c + 1];
+    o.x = pack_bf16x2(v[0].x * rs * w0.x, v[0].y * rs * w0.y);
+    o.y = pack_bf16x2(v[0].z * rs * w0.z, v[0].w * rs * w0.w);
+    o.z = pack_bf16x2(v[1].x * rs * w1.x, v[1].y * rs * w1.y);
+    o.w = pack_bf16x2(v[1].z * rs * w1.z, v[1].w * rs * w1.w);
   }
+  reinterpret_cast<uint4*>(out + (size_t)t * d)[threadIdx.x] = o;
 }
 
 cudaError_t run_residual_norm(float* x, const float* yp, const int* pair_row, int k, const float* part, int n_part,
                               int Tcap, const float* g, int T, int d, float eps, bf16* out, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
-  if (n_part > kMaxPartSplits || k > 8) return cudaErrorInvalidValue;
-  const size_t smem = (size_t)d * sizeof(float);
-  static size_t configured = 0;
-  if (smem > 48 * 1024 && smem > configured) {
-    cudaError_t e = cudaFuncSetAttribute(k_residual_norm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    configured = smem;
-  }
+  if (n_part > kMaxPartSplits || k > 8 || d % 256 != 0 || d > 4096) return cudaErrorInvalidValue;
   {
-    const cudaError_t e_ = launch_pdl(k_residual_norm, dim3(T), dim3(256), smem, st, x, yp, pair_row, k, part, n_part, (size_t)Tcap * d, g, d, eps, out);
+    const cudaError_t e_ = launch_pdl(k_residual_norm, dim3(T), dim3(d / 8), 0, st, x, yp, pair_row, k, part, n_part,
+                                      (size_t)Tcap * d, g, d, eps, out);
     if (e_ != cudaSuccess) return e_;
   }
   return cudaGetLastError();

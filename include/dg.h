@@ -56,7 +56,7 @@ extern "C" {
 #define DG_MAX_REQUESTS 8
 
 /* Model shape and sampler knobs.  Supported shapes: d_model, ffn_expert and
- * ffn_shared multiples of 64 (d_model also of 128 and 256); head_dim 64, 128
+ * ffn_shared multiples of 64 (d_model also of 128 and 256, at most 4096); head_dim 64, 128
  * or 256; (n_q_heads+2*n_kv_heads)*head_dim a multiple of 256; n_q_heads a
  * multiple of n_kv_heads; n_experts a multiple of 16 up to 128 (the router
  * is one tensor-core tile wide); top_k <= 8; vocab a multiple of
