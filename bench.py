@@ -355,10 +355,13 @@ def main():
     launches0 = h.launch_count()
     uuid = str(torch.cuda.get_device_properties(dev).uuid) if hasattr(torch.cuda.get_device_properties(dev), "uuid") else ""
     with ClockSampler(uuid) as clk:
+        # NVTX range "timed": lets a profiler restrict itself to the timed steps
+        torch.cuda.nvtx.range_push("timed")
         start = ev()
         for i in range(args.steps):
             one_step(args.warmup + i, record=True)
         end = ev()
+        torch.cuda.nvtx.range_pop()
         torch.cuda.synchronize()
     barrier(world)
     elapsed = start.elapsed_time(end)
