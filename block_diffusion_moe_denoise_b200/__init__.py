@@ -202,6 +202,12 @@ class DG:
     def debug_forward(self, req: int, tokens: torch.Tensor, n_layers: int):
         check(self.lib.dg_debug_forward(self.h, req, _ptr(tokens), tokens.numel(), n_layers), "dg_debug_forward")
 
+    def token_capacity(self) -> int:
+        """Rows of the per-pass token buffers (the middle extent of "q")."""
+        off, nb = C.c_size_t(), C.c_size_t()
+        check(self.lib.dg_debug_buffer(self.h, b"x", C.byref(off), C.byref(nb)), "dg_debug_buffer")
+        return nb.value // (self.cfg.d_model * 4)
+
     def debug_buffer(self, name: str, dtype: torch.dtype, shape=None) -> torch.Tensor:
         off, nb = C.c_size_t(), C.c_size_t()
         check(self.lib.dg_debug_buffer(self.h, name.encode(), C.byref(off), C.byref(nb)), "dg_debug_buffer")

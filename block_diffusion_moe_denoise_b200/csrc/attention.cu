@@ -93,7 +93,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
   const int rows = G * a.Tr;
   const int r0 = blockIdx.x * kAQ;
   const int n_keys = a.n_keys[slot];
-  int per = (n_keys + a.n_split - 1) / a.n_split;
+  const int n_split = a.slot_split[slot];
+  if ((int)blockIdx.z >= n_split) {  // this slot uses fewer key splits
+    pdl_trigger();
+    pdl_wait();
+    return;
+  }
+  int per = (n_keys + n_split - 1) / n_split;
   per = (per + kAK - 1) / kAK * kAK;
   const int k_begin = blockIdx.z * per;
   const int k_end = min(n_keys, k_begin + per);
@@ -311,7 +317,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
     if (ok && n_tiles > 0 &&
         mbar_wait_bounded(&pv_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, abort_flag, err)) {
       tc_fence_after();
-      if (a.n_split == 1) {
+      if (n_split == 1) {
         const float inv = l > 0.f ? 1.f / l : 0.f;
         uint4* dst = reinterpret_cast<uint4*>(a.o + (size_t)t * a.Hq * D + (size_t)h * D);
         for (int c = 0; c < D; c += 16) {
@@ -343,7 +349,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
         }
         if (valid) a.part_ml[prow_i] = make_float2(m_used, l);
       }
-    } else if (n_tiles == 0 && a.n_split > 1 && valid) {
+    } else if (n_tiles == 0 && n_split > 1 && valid) {
       const size_t prow_i = ((size_t)blockIdx.z * a.Hq + h) * a.q_T + t;
       a.part_ml[prow_i] = make_float2(-INFINITY, 0.f);
     }
@@ -359,16 +365,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
 // Merge of the split-KV partials: O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s.
 // One warp per (token, head); lane s reads split s's (max, sum), each lane then
 // owns 8 consecutive output elements and loads every split's values at once.
+// Tokens of slots that used a single split were written by the attention kernel.
 constexpr int kMaxSplits = 8;
 
-__global__ void k_attn_combine(const float* __restrict__ part_o, const float2* __restrict__ part_ml, int n_split,
-                               int Hq, int q_T, int T, int D, bf16* __restrict__ o) {
+struct SlotSplits {
+  int s[DG_MAX_REQUESTS];
+};
+
+__global__ void k_attn_combine(const float* __restrict__ part_o, const float2* __restrict__ part_ml,
+                               SlotSplits splits, int Tr, int Hq, int q_T, int T, int D, bf16* __restrict__ o) {
   pdl_trigger();
   pdl_wait();
   const int w = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (w >= T * Hq) return;
   const int t = w / Hq, h = w % Hq;
+  const int n_split = splits.s[t / Tr];
+  if (n_split == 1) return;  // written directly by the attention kernel
   float2 ml = make_float2(-INFINITY, 0.f);
   if (lane < n_split) ml = part_ml[((size_t)lane * Hq + h) * q_T + t];
   float M = ml.y > 0.f ? ml.x : -INFINITY;
@@ -434,8 +447,11 @@ static cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st) {
   if (e != cudaSuccess || a.n_split == 1) return e;
   const int T = a.n_slots * a.Tr;
   const int warps = T * a.Hq;
+  SlotSplits sp;
+  for (int i = 0; i < DG_MAX_REQUESTS; ++i) sp.s[i] = i < a.n_slots ? a.slot_split[i] : 1;
   {
-    const cudaError_t e_ = launch_pdl(k_attn_combine, dim3((warps + 7) / 8), dim3(256), 0, st, a.part_o, a.part_ml, a.n_split, a.Hq, a.q_T, T, D, a.o);
+    const cudaError_t e_ = launch_pdl(k_attn_combine, dim3((warps + 7) / 8), dim3(256), 0, st, a.part_o, a.part_ml, sp,
+                                      a.Tr, a.Hq, a.q_T, T, D, a.o);
     if (e_ != cudaSuccess) return e_;
   }
   return cudaGetLastError();
@@ -451,6 +467,8 @@ size_t attention_smem_bytes(int D) {
 
 cudaError_t run_attention(const AttnArgs& a, cudaStream_t st) {
   if (a.n_split < 1 || a.n_split > attention_split_cap()) return cudaErrorInvalidValue;
+  for (int i = 0; i < a.n_slots; ++i)
+    if (a.slot_split[i] < 1 || a.slot_split[i] > a.n_split) return cudaErrorInvalidValue;
   switch (a.D) {
     case 64: return launch_attn<64>(a, st);
     case 128: return launch_attn<128>(a, st);

@@ -17,6 +17,13 @@ namespace {
 constexpr size_t kAlign = 1024;
 constexpr int kLmGridMax = 256;
 constexpr int kSplitCap = 8;
+// A prefill pass carries up to this many consecutive 256-token segments of one
+// request (block-causal: each attends to the cache before it and to itself),
+// so the weights are streamed once per group instead of once per segment.
+constexpr int kPrefillSlots = 4;
+
+// Passes carry at most this many canvas-sized slots.
+int pass_slots(int max_req) { return max_req > kPrefillSlots ? max_req : kPrefillSlots; }
 
 struct LayerMaps {
   CUtensorMap qkv, o, gate, up, down, sgate, sup, sdown, router;
@@ -63,7 +70,7 @@ long long round_cap(long long cap) { return (cap + 63) / 64 * 64; }
 
 void make_plan(const dg_config* c, int max_req, long long cap_user, Plan* p) {
   const long long cap = round_cap(cap_user);
-  const int T = max_req * c->canvas;
+  const int T = pass_slots(max_req) * c->canvas;
   const int Tcap = (T + 127) / 128 * 128;
   const long long rows = (long long)T * c->top_k;
   const int D = c->head_dim, d = c->d_model;
@@ -262,8 +269,10 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
   const int* pair_row = h->B<int>("pair_row");
   float* part = h->B<float>("part");
   int pending_k = 0, pending_parts = 0;
-  const int so = wpart_splits(d, T, c.n_q_heads * D, h->num_sms);
-  const int ss = wpart_splits(d, T, c.ffn_shared, h->num_sms);
+  // K splits of the split-K projections are those of one slot, for the same
+  // reason as the attention key splits
+  const int so = wpart_splits(d, s.Tr, c.n_q_heads * D, h->num_sms);
+  const int ss = wpart_splits(d, s.Tr, c.ffn_shared, h->num_sms);
   for (int l = 0; l < n_layers; ++l) {
     const dg_layer_weights& w = h->lw[l];
     const LayerMaps& m = h->maps[l];
@@ -310,20 +319,26 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     aa.D = D;
     aa.Tr = s.Tr;
     aa.n_slots = s.n;
-    int max_keys = 0;
+    // Key splits are chosen per slot from that slot alone (enough CTAs for
+    // one slot to fill the GPU, at least 256 keys per split), so a segment's
+    // result does not depend on what else shares the pass.
+    const int G = c.n_q_heads / c.n_kv_heads;
+    const int slot_ctas = ((G * s.Tr + 127) / 128) * c.n_kv_heads;
+    aa.n_split = 1;
     for (int i = 0; i < DG_MAX_REQUESTS; ++i) {
       aa.req[i] = i < s.n ? s.req[i] : 0;
       aa.n_keys[i] = i < s.n ? s.pos0[i] + s.Tr : 0;
-      if (aa.n_keys[i] > max_keys) max_keys = aa.n_keys[i];
+      int split = 1;
+      if (i < s.n) {
+        split = h->num_sms / slot_ctas;
+        const int by_keys = aa.n_keys[i] / 256;
+        if (split > by_keys) split = by_keys;
+        if (split > kSplitCap) split = kSplitCap;
+        if (split < 1) split = 1;
+      }
+      aa.slot_split[i] = split;
+      if (split > aa.n_split) aa.n_split = split;
     }
-    const int G = c.n_q_heads / c.n_kv_heads;
-    const int base_ctas = ((G * s.Tr + 127) / 128) * c.n_kv_heads * s.n;
-    int split = h->num_sms / base_ctas;
-    const int max_by_keys = max_keys / 256 > 0 ? max_keys / 256 : 1;
-    if (split > max_by_keys) split = max_by_keys;
-    if (split > kSplitCap) split = kSplitCap;
-    if (split < 1) split = 1;
-    aa.n_split = split;
     aa.part_o = h->B<float>("attn_o");
     aa.part_ml = h->B<float2>("attn_ml");
     aa.scale = 1.0f / sqrtf((float)D);
@@ -511,7 +526,7 @@ int dg_init(const dg_config* cfg, const dg_weights* wts, int max_requests, int64
   h->cap_user = kv_capacity;
   h->st = static_cast<cudaStream_t>(stream);
   h->num_sms = prop.multiProcessorCount;
-  h->T_max = max_requests * cfg->canvas;
+  h->T_max = pass_slots(max_requests) * cfg->canvas;
   h->Tcap = (h->T_max + 127) / 128 * 128;
   h->embed = static_cast<const bf16*>(wts->embed);
   h->final_norm = static_cast<const float*>(wts->final_norm);
@@ -621,18 +636,27 @@ int dg_prefill(dg_handle* h, int req, const int32_t* d_tokens, int n) {
   if (r.open) return DG_E_STATE;
   if (r.kv_len + n > h->cap_user) return DG_E_CAPACITY;
   const int seg = h->cfg.canvas;
-  for (int s0 = 0; s0 < n; s0 += seg) {
-    const int len = n - s0 < seg ? n - s0 : seg;
+  const int group = h->T_max / seg;  // full segments per pass
+  int s0 = 0;
+  while (s0 < n) {
+    // consecutive full segments share a pass; a short last segment goes alone
+    const int full = (n - s0) / seg;
+    const int ns = full >= 1 ? (full < group ? full : group) : 1;
+    const int len = full >= 1 ? seg : n - s0;
     SlotInfo s;
     memset(&s, 0, sizeof(s));
-    s.n = 1;
+    s.n = ns;
     s.Tr = len;
-    s.req[0] = req;
-    s.pos0[0] = (int)r.kv_len;
-    const int* ids[1] = {d_tokens + s0};
+    const int* ids[DG_MAX_REQUESTS];
+    for (int i = 0; i < ns; ++i) {
+      s.req[i] = req;
+      s.pos0[i] = (int)r.kv_len + i * seg;
+      ids[i] = d_tokens + s0 + i * seg;
+    }
     int rc = run_pass(h, ids, s, h->cfg.n_layers, true, false, nullptr);
     if (rc != DG_OK) return rc;
-    r.kv_len += len;
+    r.kv_len += (long long)ns * len;
+    s0 += ns * len;
   }
   return DG_OK;
 }

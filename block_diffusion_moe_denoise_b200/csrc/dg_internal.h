@@ -110,7 +110,7 @@ struct SlotInfo {
 cudaError_t run_embed(const int* const* ids, const SlotInfo& s, const bf16* embed, int V, int d, float* x, int* tok_pos,
                       int* tok_req, const double* inv_freq, int half, float2* rope, int* err, cudaStream_t st);
 // x[t] += sum_j yp[pair_row[t*k+j]] + sum_s part[s][t]; then (if an output is
-// given) the RMSNorm of x[t] with gain g as bf16 and/or fp32
+// given) the RMSNorm of x[t] with gain g as bf16
 cudaError_t run_residual_norm(float* x, const float* yp, const int* pair_row, int k, const float* part, int n_part,
                               int Tcap, const float* g, int T, int d, float eps, bf16* out, cudaStream_t st);
 cudaError_t run_rmsnorm(const float* x, const float* g, int T, int d, float eps, bf16* out, cudaStream_t st);
@@ -176,7 +176,8 @@ struct AttnArgs {
   int Hq, Hkv, D, Tr, n_slots;
   int req[DG_MAX_REQUESTS];
   int n_keys[DG_MAX_REQUESTS];
-  int n_split;       // key splits (1 = direct)
+  int n_split;                         // largest key split over the slots
+  int slot_split[DG_MAX_REQUESTS];     // key splits of each slot (1 = direct output)
   float* part_o;     // [n_split][Hq][q_T][D]
   float2* part_ml;   // [n_split][Hq][q_T]
   float scale;

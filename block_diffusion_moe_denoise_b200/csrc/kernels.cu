@@ -408,10 +408,11 @@ __global__ void __launch_bounds__(256) k_group_gather(GroupArgs a, const unsigne
   __shared__ int off[257];
   __shared__ int toff[257];
   const int E = a.E, T = a.T, k = a.k, P = T * k;
+  const int used = (T + 31) >> 5;  // words of each expert's mask this pass can have set
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   for (int e = tid; e < E; e += blockDim.x) {
     int c = 0;
-    for (int wi = 0; wi < MW; ++wi) c += __popc(mask[(size_t)e * MW + wi]);
+    for (int wi = 0; wi < used; ++wi) c += __popc(mask[(size_t)e * MW + wi]);
     cnt[e] = c;
   }
   __syncthreads();

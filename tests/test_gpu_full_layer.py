@@ -53,17 +53,17 @@ def test_canvas_init_is_philox(setup):
 def test_attention_path(setup):
     h, rec = setup["h"], setup["tr"]
     T, d, Hq, D = CFG.canvas, CFG.d_model, CFG.n_q_heads, CFG.head_dim
-    Tcap = 256
-    q = np64(h.debug_buffer("q", torch.bfloat16, (Hq, Tcap, D))).transpose(1, 0, 2)
+    Tcap = h.token_capacity()
+    q = np64(h.debug_buffer("q", torch.bfloat16, (Hq, Tcap, D))[:, :T]).transpose(1, 0, 2)
     assert rel_l2(q, rec["q"]) < REL_L2
     kk, vv = h.get_kv(0, 0, L_PREFIX, T)
     assert rel_l2(np64(kk).transpose(1, 0, 2), rec["k"]) < REL_L2
     assert rel_l2(np64(vv).transpose(1, 0, 2), rec["v"]) < REL_L2
-    o = np64(h.debug_buffer("o", torch.bfloat16, (Tcap, Hq * D)))
+    o = np64(h.debug_buffer("o", torch.bfloat16, (T, Hq * D)))
     eo = rel_l2(o, rec["o"].reshape(T, Hq * D))
     print(f"full layer: rel-L2 of attention output {eo:.2e}")
     assert eo < REL_L2
-    assert rel_l2(np64(h.debug_buffer("u", torch.bfloat16, (Tcap, d))), rec["u"]) < REL_L2
+    assert rel_l2(np64(h.debug_buffer("u", torch.bfloat16, (T, d))), rec["u"]) < REL_L2
 
 
 def test_moe_path(setup):

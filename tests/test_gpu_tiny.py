@@ -32,11 +32,12 @@ def _handle(model, max_requests=2, cap=1024):
     return dgm.DG(CFG, wd, max_requests=max_requests, kv_capacity=cap)
 
 
-@pytest.mark.parametrize("n_prompt", [128, 200, 300])
+@pytest.mark.parametrize("n_prompt", [128, 200, 300, 1100])
 def test_prefill_kv_matches_oracle(model, n_prompt):
-    """Prefill in canvas-sized segments (ragged tails: 200, 256+44)."""
+    """Prefill in canvas-sized segments (ragged tails: 200, 256+44; 1100 = one
+    pass of four block-causal segments, then a 76-token segment)."""
     _, _, ora = model
-    h = _handle(model)
+    h = _handle(model, cap=1536)
     prompt = make_tokens(CFG, n_prompt, seed=n_prompt)
     h.prefill(0, prompt.cuda())
     h.sync()
@@ -50,6 +51,28 @@ def test_prefill_kv_matches_oracle(model, n_prompt):
         assert kv_rel_l2(np64(k), cache.K[l][:, :n_prompt], keep) < REL_L2
         assert kv_rel_l2(np64(v), cache.V[l][:, :n_prompt], keep) < REL_L2
     h.close()
+
+
+def test_batched_prefill_equals_segment_by_segment(model):
+    """Full segments are prefilled up to four per pass; the cache must equal,
+    bit for bit, the one built by feeding the same segments one call at a
+    time (every reduction order is fixed per segment)."""
+    n = 5 * CFG.canvas + 100
+    prompt = make_tokens(CFG, n, seed=7).cuda()
+    h1 = _handle(model, cap=2048)
+    h1.prefill(0, prompt)
+    h2 = _handle(model, cap=2048)
+    for s0 in range(0, n, CFG.canvas):
+        h2.prefill(0, prompt[s0:s0 + CFG.canvas])
+    h1.sync()
+    h2.sync()
+    assert h1.kv_len(0) == h2.kv_len(0) == n
+    for l in range(CFG.n_layers):
+        k1, v1 = h1.get_kv(0, l, 0, n)
+        k2, v2 = h2.get_kv(0, l, 0, n)
+        assert torch.equal(k1, k2) and torch.equal(v1, v2), f"layer {l}"
+    h1.close()
+    h2.close()
 
 
 @pytest.mark.parametrize("T", [256, 130])
@@ -69,7 +92,7 @@ def test_layer_intermediates(model, T):
     ora.forward(toks.numpy(), cache, want_stats=False, trace=tr, n_layers=1)
     rec = tr.layers[0]
     d, Hq, D, k = CFG.d_model, CFG.n_q_heads, CFG.head_dim, CFG.top_k
-    Tcap = (h.max_requests * CFG.canvas + 127) // 128 * 128
+    Tcap = h.token_capacity()
     hn = np64(h.debug_buffer("hn", torch.bfloat16, (Tcap, d))[:T])
     assert rel_l2(hn, rec["h"]) < REL_L2
     q = np64(h.debug_buffer("q", torch.bfloat16, (Hq, Tcap, D))[:, :T]).transpose(1, 0, 2)
