@@ -30,7 +30,8 @@ struct LayerMaps {
 };
 
 struct ReqState {
-  long long kv_len = 0;
+  long long kv_len = 0;  // committed length, including a pending block
+  bool pending = false;  // the last committed block's pass has not run yet (its tokens: "commit_tok")
   int block = 0;
   int step = 0;
   unsigned long long seed = 0;
@@ -104,6 +105,7 @@ void make_plan(const dg_config* c, int max_req, long long cap_user, Plan* p) {
   p->add("stats", (size_t)Tcap * 16);
   p->add("argmax", (size_t)Tcap * 4);
   p->add("canvas", (size_t)max_req * c->canvas * 4);
+  p->add("commit_tok", (size_t)max_req * c->canvas * 4);
   p->add("mask", (size_t)max_req * c->canvas);
   p->add("remaining", (size_t)max_req * 4);
   p->add("tok_pos", (size_t)Tcap * 4);
@@ -251,10 +253,13 @@ namespace {
 // One decoder pass over s.n slots of s.Tr tokens.  n_layers layers; when
 // `qkv_only_last` the last layer runs only its K/V projection (nothing reads
 // the rest: commit and prefill); `want_lm` adds the final norm + LM head.
+// One decoder pass over the slots of `s`.  With want_lm, the final norm and
+// the LM head run over the first lm_rows tokens only (lm_rows < 0: all).
 int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layers, bool qkv_only_last, bool want_lm,
-             float* logits) {
+             float* logits, int lm_rows = -1) {
   const dg_config& c = h->cfg;
   const int T = s.n * s.Tr;
+  const int TL = lm_rows < 0 ? T : lm_rows;
   const int d = c.d_model, D = c.head_dim, k = c.top_k;
   cudaStream_t st = h->st;
   int* err = h->B<int>("err");
@@ -450,12 +455,12 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
   }
   if (want_lm) {
     LAUNCH(h, K_RMSNORM, 1,
-           run_residual_norm(x, yp, pair_row, pending_k, part, pending_parts, h->Tcap, h->final_norm, T, d,
+           run_residual_norm(x, yp, pair_row, pending_k, part, pending_parts, h->Tcap, h->final_norm, TL, d,
                              c.norm_eps, hn, st));
     LmArgs la;
     la.tm_x = &h->tm_hn;
     la.tm_embed = &h->tm_embed;
-    la.T = T;
+    la.T = TL;
     la.d = d;
     la.num_sms = h->num_sms < kLmGridMax ? h->num_sms : kLmGridMax;
     la.V = c.vocab;
@@ -465,7 +470,7 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     int grid = 0;
     LAUNCH(h, K_LM, 1, run_lm_head(la, &grid, st));
     LAUNCH(h, K_LMC, 1,
-           run_lm_combine(h->B<float4>("lm_part"), grid, (T + 127) / 128, T, h->B<float>("stats"),
+           run_lm_combine(h->B<float4>("lm_part"), grid, (TL + 127) / 128, TL, h->B<float>("stats"),
                           h->B<int>("argmax"), err, st));
   } else if (pending_k || pending_parts) {
     // a pass stopped after a full layer: fold its expert outputs into x
@@ -477,6 +482,24 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
 }
 
 bool req_ok(const dg_handle* h, int r) { return h && r >= 0 && r < h->max_req; }
+
+// Run the pass of a committed block on its own (its K/V at [kv_len - canvas,
+// kv_len)) when nothing it could share a pass with is coming.
+int flush_commit(dg_handle* h, int req) {
+  ReqState& r = h->req[req];
+  if (!r.pending) return DG_OK;
+  const int C = h->cfg.canvas;
+  SlotInfo s;
+  memset(&s, 0, sizeof(s));
+  s.n = 1;
+  s.Tr = C;
+  s.req[0] = req;
+  s.pos0[0] = (int)(r.kv_len - C);
+  const int* ids[1] = {h->B<int>("commit_tok") + (size_t)req * C};
+  const int rc = run_pass(h, ids, s, h->cfg.n_layers, true, false, nullptr);
+  if (rc == DG_OK) r.pending = false;
+  return rc;
+}
 
 }  // namespace
 
@@ -605,6 +628,8 @@ int64_t dg_kv_len(const dg_handle* h, int req) { return req_ok(h, req) ? h->req[
 int dg_set_kv(dg_handle* h, int req, int layer, int64_t pos0, int64_t n, const void* d_k, const void* d_v) {
   if (!req_ok(h, req) || layer < 0 || layer >= h->cfg.n_layers || pos0 < 0 || n < 0 || !d_k || !d_v) return DG_E_ARG;
   if (pos0 + n > h->cap_user) return DG_E_CAPACITY;
+  const int rc = flush_commit(h, req);
+  if (rc != DG_OK) return rc;
   bf16* ck = h->B<bf16>("kv") + req * h->kv_req_stride + layer * h->kv_layer_stride;
   bf16* cv = ck + (size_t)h->cfg.n_kv_heads * h->cap * h->cfg.head_dim;
   CK(run_kv_copy(ck, cv, h->cfg.n_kv_heads, h->cap, h->cfg.head_dim, pos0, n, (const bf16*)d_k, (const bf16*)d_v,
@@ -615,6 +640,8 @@ int dg_set_kv(dg_handle* h, int req, int layer, int64_t pos0, int64_t n, const v
 int dg_get_kv(dg_handle* h, int req, int layer, int64_t pos0, int64_t n, void* d_k, void* d_v) {
   if (!req_ok(h, req) || layer < 0 || layer >= h->cfg.n_layers || pos0 < 0 || n < 0 || !d_k || !d_v) return DG_E_ARG;
   if (pos0 + n > h->cap_user) return DG_E_CAPACITY;
+  const int rc = flush_commit(h, req);
+  if (rc != DG_OK) return rc;
   bf16* ck = h->B<bf16>("kv") + req * h->kv_req_stride + layer * h->kv_layer_stride;
   bf16* cv = ck + (size_t)h->cfg.n_kv_heads * h->cap * h->cfg.head_dim;
   CK(run_kv_copy(ck, cv, h->cfg.n_kv_heads, h->cap, h->cfg.head_dim, pos0, n, nullptr, nullptr, (bf16*)d_k,
@@ -626,6 +653,8 @@ int dg_set_kv_len(dg_handle* h, int req, int64_t len) {
   if (!req_ok(h, req) || len < 0) return DG_E_ARG;
   if (h->req[req].open) return DG_E_STATE;
   if (len > h->cap_user) return DG_E_CAPACITY;
+  const int rc = flush_commit(h, req);
+  if (rc != DG_OK) return rc;
   h->req[req].kv_len = len;
   return DG_OK;
 }
@@ -635,6 +664,8 @@ int dg_prefill(dg_handle* h, int req, const int32_t* d_tokens, int n) {
   ReqState& r = h->req[req];
   if (r.open) return DG_E_STATE;
   if (r.kv_len + n > h->cap_user) return DG_E_CAPACITY;
+  int rc0 = flush_commit(h, req);
+  if (rc0 != DG_OK) return rc0;
   const int seg = h->cfg.canvas;
   const int group = h->T_max / seg;  // full segments per pass
   int s0 = 0;
@@ -716,20 +747,41 @@ int dg_denoise_step(dg_handle* h, int n_req, const int* reqs, int32_t* d_remaini
     if (!h->req[reqs[i]].open) return DG_E_STATE;
   }
   const int C = h->cfg.canvas;
+  // pending commits of these requests join the pass as extra slots after the
+  // canvases (block-causal: a committed block's keys end where its canvas's
+  // begin); the LM head covers the canvas slots only
+  int n_pend = 0;
+  for (int i = 0; i < n_req; ++i) n_pend += h->req[reqs[i]].pending ? 1 : 0;
+  if (n_req + n_pend > h->T_max / C || n_req + n_pend > DG_MAX_REQUESTS) {
+    for (int i = 0; i < n_req; ++i) {
+      const int rc0 = flush_commit(h, reqs[i]);
+      if (rc0 != DG_OK) return rc0;
+    }
+    n_pend = 0;
+  }
   SlotInfo s;
   memset(&s, 0, sizeof(s));
-  s.n = n_req;
+  s.n = n_req + n_pend;
   s.Tr = C;
   const int* ids[DG_MAX_REQUESTS];
   int steps[DG_MAX_REQUESTS];
+  int j = n_req;
   for (int i = 0; i < n_req; ++i) {
+    const ReqState& r = h->req[reqs[i]];
     s.req[i] = reqs[i];
-    s.pos0[i] = (int)h->req[reqs[i]].kv_len;
+    s.pos0[i] = (int)r.kv_len;
     ids[i] = h->B<int>("canvas") + (size_t)reqs[i] * C;
-    steps[i] = h->req[reqs[i]].step + 1;
+    steps[i] = r.step + 1;
+    if (r.pending) {
+      s.req[j] = reqs[i];
+      s.pos0[j] = (int)(r.kv_len - C);
+      ids[j] = h->B<int>("commit_tok") + (size_t)reqs[i] * C;
+      ++j;
+    }
   }
-  int rc = run_pass(h, ids, s, h->cfg.n_layers, false, true, nullptr);
+  int rc = run_pass(h, ids, s, h->cfg.n_layers, false, true, nullptr, n_req * C);
   if (rc != DG_OK) return rc;
+  for (int i = 0; i < n_req; ++i) h->req[reqs[i]].pending = false;
   float* stats = h->B<float>("stats");
   rc = sample_slots(h, n_req, reqs, stats, stats + 1, 4, h->B<int>("argmax"), steps);
   if (rc != DG_OK) return rc;
@@ -753,17 +805,17 @@ int dg_commit_block(dg_handle* h, int req) {
   if (!req_ok(h, req)) return DG_E_ARG;
   ReqState& r = h->req[req];
   if (!r.open) return DG_E_STATE;
-  const int C = h->cfg.canvas;
-  SlotInfo s;
-  memset(&s, 0, sizeof(s));
-  s.n = 1;
-  s.Tr = C;
-  s.req[0] = req;
-  s.pos0[0] = (int)r.kv_len;
-  const int* ids[1] = {h->B<int>("canvas") + (size_t)req * C};
-  int rc = run_pass(h, ids, s, h->cfg.n_layers, true, false, nullptr);
+  int rc = flush_commit(h, req);  // a block committed before this one without a step in between
   if (rc != DG_OK) return rc;
+  // The block's pass is deferred: it rides along with the request's next
+  // denoising step (one weight stream for both), or runs on its own as soon
+  // as another call needs the cache.  The tokens are kept aside because the
+  // next dg_open_canvas overwrites the canvas.
+  const int C = h->cfg.canvas;
+  CK(cudaMemcpyAsync(h->B<int>("commit_tok") + (size_t)req * C, h->B<int>("canvas") + (size_t)req * C, (size_t)C * 4,
+                     cudaMemcpyDeviceToDevice, h->st));
   r.kv_len += C;
+  r.pending = true;
   r.open = false;
   return DG_OK;
 }
@@ -786,7 +838,7 @@ int dg_generate(dg_handle* h, int req, const int32_t* h_prompt, int n_prompt, in
   const int C = h->cfg.canvas;
   if (n_out % C != 0) return DG_E_ARG;
   ReqState& r = h->req[req];
-  if (r.open || r.kv_len != 0) return DG_E_STATE;
+  if (r.open || r.kv_len != 0 || r.pending) return DG_E_STATE;
   if ((long long)n_prompt + n_out > h->cap_user) return DG_E_CAPACITY;
   int* prompt = h->B<int>("prompt");
   if (n_prompt > 0) CK(cudaMemcpyAsync(prompt, h_prompt, (size_t)n_prompt * 4, cudaMemcpyHostToDevice, h->st));
@@ -811,6 +863,8 @@ int dg_generate(dg_handle* h, int req, const int32_t* h_prompt, int n_prompt, in
     rc = dg_commit_block(h, req);
     if (rc != DG_OK) return rc;
   }
+  rc = flush_commit(h, req);
+  if (rc != DG_OK) return rc;
   return dg_sync(h);
 }
 
@@ -938,6 +992,8 @@ int dg_debug_forward(dg_handle* h, int req, const int32_t* d_tokens, int T, int 
     return DG_E_ARG;
   const ReqState& r = h->req[req];
   if (r.kv_len + T > h->cap_user) return DG_E_CAPACITY;
+  const int rc = flush_commit(h, req);
+  if (rc != DG_OK) return rc;
   SlotInfo s;
   memset(&s, 0, sizeof(s));
   s.n = 1;

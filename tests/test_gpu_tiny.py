@@ -75,6 +75,36 @@ def test_batched_prefill_equals_segment_by_segment(model):
     h2.close()
 
 
+def test_commit_rides_with_next_step(model):
+    """A committed block's pass runs inside the next canvas's first denoising
+    step (two block-causal slots of one request); that step's statistics and
+    the committed K/V must equal, bit for bit, those obtained when the commit
+    runs on its own first."""
+    def run(standalone):
+        h = _handle(model, max_requests=1, cap=1024)
+        h.prefill(0, make_tokens(CFG, 300, seed=21).cuda())
+        h.open_canvas(0, 5, 0)
+        for _ in range(CFG.max_steps):
+            h.denoise_step([0])
+            if h.read_remaining(0) == 0:
+                break
+        h.commit_block(0)
+        if standalone:
+            h.set_kv_len(0, h.kv_len(0))  # needs the cache: runs the commit pass now
+        h.open_canvas(0, 5, 1)
+        h.denoise_step([0])
+        _, _, st, am = h.get_canvas(0)
+        out = [st.clone(), am.clone()]
+        for l in range(CFG.n_layers):
+            out += [t.clone() for t in h.get_kv(0, l, 300, CFG.canvas)]
+        h.sync()
+        h.close()
+        return out
+    fused, alone = run(False), run(True)
+    for a, b in zip(fused, alone):
+        assert torch.equal(a, b)
+
+
 @pytest.mark.parametrize("T", [256, 130])
 def test_layer_intermediates(model, T):
     """One decoder layer over a canvas (and a ragged 130-token segment) after a
