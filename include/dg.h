@@ -112,13 +112,17 @@ const char* dg_strerror(int code);
 /* Append `n` prompt tokens (device int32 array) to request `req`'s KV cache:
  * the decoder runs over segments of `canvas` tokens counted from the first
  * token; each segment attends to all earlier positions and bidirectionally to
- * itself.  Fails with DG_E_STATE while a canvas is open, DG_E_CAPACITY if the
- * cache would overflow. */
+ * itself.  Up to four full segments share one decoder pass (block-causal
+ * slots), with a result bit-identical to one segment per call.  Fails with
+ * DG_E_STATE while a canvas is open, DG_E_CAPACITY if the cache would
+ * overflow. */
 int dg_prefill(dg_handle* h, int req, const int32_t* d_tokens, int n);
 
 /* Write synthetic committed K/V: positions [pos0, pos0+n) of layer `layer`
  * from device arrays k, v of shape [n_kv_heads, n, head_dim] bf16 (post-RoPE
- * keys).  Does not change the KV length. */
+ * keys).  Does not change the KV length.  Like dg_get_kv, dg_set_kv_len,
+ * dg_prefill and dg_debug_forward, it first runs a deferred commit pass of
+ * the request (see dg_commit_block). */
 int dg_set_kv(dg_handle* h, int req, int layer, int64_t pos0, int64_t n, const void* d_k, const void* d_v);
 /* Read back K/V of positions [pos0, pos0+n) into [n_kv_heads, n, head_dim] bf16. */
 int dg_get_kv(dg_handle* h, int req, int layer, int64_t pos0, int64_t n, void* d_k, void* d_v);
@@ -143,7 +147,12 @@ int dg_denoise_step(dg_handle* h, int n_req, const int* reqs, int32_t* d_remaini
 int dg_read_remaining(dg_handle* h, int req, int32_t* remaining);
 
 /* Commit request `req`'s converged canvas: the decoder runs over the final
- * canvas tokens at [L, L+canvas), writing their K/V, and L advances by canvas.
+ * canvas tokens at [L, L+canvas), writing their K/V, and L advances by canvas
+ * (dg_kv_len reports the new length at once).  The pass itself is deferred:
+ * it joins the request's next dg_denoise_step as an extra block-causal slot
+ * (one weight stream for both, bit-identical results), or runs on its own
+ * when a call that needs the cache comes first (dg_get_kv, dg_set_kv,
+ * dg_set_kv_len, dg_prefill, dg_debug_forward, the end of dg_generate).
  * DG_E_STATE if no canvas is open.  The caller decides convergence (remaining
  * == 0); committing earlier commits the current tokens as they are. */
 int dg_commit_block(dg_handle* h, int req);
