@@ -32,7 +32,9 @@ def config_struct(cfg) -> dg_config:
     """dg_config from a synth.ModelConfig-like object."""
     return dg_config(cfg.n_layers, cfg.d_model, cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim, cfg.n_experts,
                      cfg.top_k, cfg.ffn_expert, cfg.ffn_shared, cfg.vocab, cfg.canvas, cfg.max_steps,
-                     cfg.min_accept, cfg.entropy_thresh, cfg.rope_theta, cfg.norm_eps)
+                     cfg.min_accept, cfg.entropy_thresh, cfg.rope_theta, cfg.norm_eps,
+                     getattr(cfg, "sampler", 0), getattr(cfg, "entropy_budget", 0.1),
+                     getattr(cfg, "stop_entropy", 0.005))
 
 
 def philox_tokens(seed: int, block: int, step: int, request: int, pos0: int, n: int, vocab: int,

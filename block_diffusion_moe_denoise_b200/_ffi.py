@@ -17,7 +17,8 @@ class dg_config(C.Structure):
     _fields_ = [(n, C.c_int) for n in ("n_layers", "d_model", "n_q_heads", "n_kv_heads", "head_dim", "n_experts",
                                        "top_k", "ffn_expert", "ffn_shared", "vocab", "canvas", "max_steps",
                                        "min_accept")] + \
-               [("entropy_thresh", C.c_float), ("rope_theta", C.c_float), ("norm_eps", C.c_float)]
+               [("entropy_thresh", C.c_float), ("rope_theta", C.c_float), ("norm_eps", C.c_float),
+                ("sampler", C.c_int), ("entropy_budget", C.c_float), ("stop_entropy", C.c_float)]
 
 
 class dg_layer_weights(C.Structure):

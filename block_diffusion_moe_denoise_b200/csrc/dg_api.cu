@@ -64,6 +64,8 @@ bool config_ok(const dg_config* c) {
   if (c->vocab < 256 || c->vocab % 256 != 0) return false;
   if (c->canvas < 1 || c->canvas > 256) return false;
   if (c->max_steps < 1 || c->min_accept < 0) return false;
+  if (c->sampler != DG_SAMPLER_THRESHOLD && c->sampler != DG_SAMPLER_ENTROPY_BUDGET) return false;
+  if (c->sampler == DG_SAMPLER_ENTROPY_BUDGET && !(c->entropy_budget >= 0.f && c->stop_entropy >= 0.f)) return false;
   return true;
 }
 
@@ -106,6 +108,7 @@ void make_plan(const dg_config* c, int max_req, long long cap_user, Plan* p) {
   p->add("argmax", (size_t)Tcap * 4);
   p->add("canvas", (size_t)max_req * c->canvas * 4);
   p->add("commit_tok", (size_t)max_req * c->canvas * 4);
+  p->add("prev_argmax", (size_t)max_req * c->canvas * 4);
   p->add("mask", (size_t)max_req * c->canvas);
   p->add("remaining", (size_t)max_req * 4);
   p->add("tok_pos", (size_t)Tcap * 4);
@@ -719,6 +722,10 @@ static int sample_slots(dg_handle* h, int n_req, const int* reqs, const float* e
   a.min_accept = c.min_accept;
   a.max_steps = c.max_steps;
   a.thr = c.entropy_thresh;
+  a.mode = c.sampler;
+  a.budget = c.entropy_budget;
+  a.stop_entropy = c.stop_entropy;
+  a.prev_argmax = h->B<int>("prev_argmax");
   for (int i = 0; i < n_req; ++i) {
     const ReqState& r = h->req[reqs[i]];
     a.req[i] = reqs[i];

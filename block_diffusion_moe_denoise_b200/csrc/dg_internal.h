@@ -144,6 +144,9 @@ cudaError_t run_lm_combine(const float4* part, int G, int MT, int T, float* stat
 struct SampleArgs {
   int n_slots, canvas, vocab, min_accept, max_steps;
   float thr;
+  int mode;               // DG_SAMPLER_THRESHOLD or DG_SAMPLER_ENTROPY_BUDGET
+  float budget, stop_entropy;
+  int* prev_argmax;       // [req][canvas] argmax of the previous step (budget rule)
   int req[DG_MAX_REQUESTS];
   int block[DG_MAX_REQUESTS];
   int step[DG_MAX_REQUESTS];

@@ -670,6 +670,13 @@ cudaError_t run_philox_tokens(unsigned long long seed, int block, int step, int 
 
 // ---------------------------------------------------------------------------
 // Accept / freeze / re-noise rule, one CTA per canvas, one thread per position.
+// Threshold rule: accept an open position whose entropy is <= thr or that is
+// among the min_accept most confident open positions.  Entropy-budget rule
+// (the pages' default sampler, "How the sampler actually works"): accept the
+// open positions from most to least confident while their running entropy
+// stays within the budget (at least the first); accept them all once the
+// argmax of every open position repeats the previous step's and their mean
+// entropy is below stop_entropy.  Both accept everything at the step cap.
 // ---------------------------------------------------------------------------
 __global__ void k_sample(SampleArgs a) {
   pdl_trigger();
@@ -677,6 +684,9 @@ __global__ void k_sample(SampleArgs a) {
   extern __shared__ float ssm[];
   float* lc_s = ssm;                                             // [canvas]
   int* un_s = reinterpret_cast<int*>(ssm + a.canvas);            // [canvas]
+  float* h_s = ssm + 2 * a.canvas;                               // [canvas] entropy, by position
+  float* hr_s = ssm + 3 * a.canvas;                              // [canvas] entropy, by confidence rank
+  __shared__ int stop_s;
   const int slot = blockIdx.x;
   const int req = a.req[slot];
   const int i = threadIdx.x;
@@ -694,10 +704,11 @@ __global__ void k_sample(SampleArgs a) {
     if (H != H || lc != lc) atomicOr(a.err, DG_DEVERR_NAN);
     lc_s[i] = lc;
     un_s[i] = !acc;
+    h_s[i] = H;
   }
   const int nU = __syncthreads_count(valid && !acc);
-  const int n_top = min(a.min_accept, nU);
   const bool force = a.step[slot] >= a.max_steps;
+  // rank among the positions not yet accepted: descending logconf, ties to the lower position
   int rank = 0;
   if (valid && !acc) {
     for (int j = 0; j < C; ++j) {
@@ -705,7 +716,39 @@ __global__ void k_sample(SampleArgs a) {
       rank += (un_s[j] && (o > lc || (o == lc && j < i))) ? 1 : 0;
     }
   }
-  const bool take = valid && !acc && (force || H <= a.thr || rank < n_top);
+  bool take;
+  if (a.mode == DG_SAMPLER_ENTROPY_BUDGET) {
+    // converged: every open position kept its previous argmax and their mean
+    // entropy (fp64, summed in position order) is below stop_entropy
+    int* prev = a.prev_argmax + (size_t)req * C;
+    const bool same = !valid || acc || (a.step[slot] > 1 && prev[i] == am);
+    const int all_same = __syncthreads_and(same);
+    if (valid && !acc) hr_s[rank] = H;
+    if (i == 0) {
+      double sum = 0.0;
+      for (int j = 0; j < C; ++j)
+        if (un_s[j]) sum += (double)h_s[j];
+      stop_s = nU > 0 && all_same && sum / (double)nU < (double)a.stop_entropy;
+    }
+    __syncthreads();
+    // running entropy of the rank-ordered open positions (fp64, in rank
+    // order): a position is taken when no earlier prefix beyond the first
+    // position went over the budget
+    bool within = false;
+    if (valid && !acc) {
+      double cum = 0.0;
+      within = true;
+      for (int r = 0; r <= rank; ++r) {
+        cum += (double)hr_s[r];
+        if (r > 0 && cum > (double)a.budget) within = false;
+      }
+    }
+    take = valid && !acc && (force || stop_s || within);
+    if (valid) prev[i] = am;
+  } else {
+    const int n_top = min(a.min_accept, nU);
+    take = valid && !acc && (force || H <= a.thr || rank < n_top);
+  }
   if (take) {
     if (am < 0 || am >= a.vocab) {
       atomicOr(a.err, DG_DEVERR_TOKEN);
@@ -725,7 +768,7 @@ cudaError_t run_sample(const SampleArgs& a, cudaStream_t st) {
   if (a.n_slots == 0) return cudaSuccess;
   const int threads = (a.canvas + 31) / 32 * 32;
   {
-    const cudaError_t e_ = launch_pdl(k_sample, dim3(a.n_slots), dim3(threads), (size_t)a.canvas * 8, st, a);
+    const cudaError_t e_ = launch_pdl(k_sample, dim3(a.n_slots), dim3(threads), (size_t)a.canvas * 16, st, a);
     if (e_ != cudaSuccess) return e_;
   }
   return cudaGetLastError();

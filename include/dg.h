@@ -16,12 +16,13 @@
  *     re-randomised; a converged canvas is committed to the KV cache and the next
  *     canvas opens ("DiffusionGemma hits ~1,500 TPS", section "How the sampler
  *     actually works").
- * Sampler rule implemented: a position not yet accepted is accepted when its
+ * Sampler rule (default, DG_SAMPLER_THRESHOLD): a position not yet accepted is accepted when its
  * entropy is <= entropy_thresh nats, or when it is among the min_accept most
  * confident (highest log max-probability, ties to the lower position) of the
  * positions not yet accepted; at step max_steps every remaining position is
  * accepted.  Rejected positions get tok(seed, block, step, position) from
  * Philox-4x32-10 (key = seed, counter = (position, step, block, request)).
+ * The pages' entropy-budget rule is available as DG_SAMPLER_ENTROPY_BUDGET.
  *
  * Conventions for every entry point:
  *   - All device pointers are caller-owned and must stay valid while the handle
@@ -70,7 +71,21 @@ typedef struct dg_config {
   float entropy_thresh;/* nats (1.0) */
   float rope_theta;    /* 10000 */
   float norm_eps;      /* 1e-6 */
+  int sampler;         /* DG_SAMPLER_THRESHOLD (the rule above) or DG_SAMPLER_ENTROPY_BUDGET */
+  float entropy_budget;/* budget rule: nats of entropy accepted per step (0.1) */
+  float stop_entropy;  /* budget rule: converged below this mean entropy (0.005) */
 } dg_config;
+
+/* Sampler rules.  DG_SAMPLER_ENTROPY_BUDGET follows the pages' default sampler
+ * ("DiffusionGemma hits ~1,500 TPS", "How the sampler actually works"): the
+ * positions not yet accepted are taken from most to least confident while the
+ * running sum of their entropies (fp64, in that order) stays within
+ * entropy_budget, and at least the most confident one; when every such
+ * position keeps the argmax it had at the previous step and their mean
+ * entropy is below stop_entropy, all of them are accepted (the canvas has
+ * converged); at step max_steps all are accepted.  Candidates are argmax. */
+#define DG_SAMPLER_THRESHOLD 0
+#define DG_SAMPLER_ENTROPY_BUDGET 1
 
 /* Device pointers to one layer's weights.  bf16 tensors are row-major
  * "out x in"; gains are fp32.

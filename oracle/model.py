@@ -129,16 +129,20 @@ class Oracle:
         cache.length += canvas.shape[0]
 
     def denoise_step(self, cache: Cache, canvas, accepted, *, seed: int, block: int, step: int,
-                     request: int = 0, stats=None):
-        """One step: pass over the canvas (unless `stats` is given), then the sampler.
-        Returns (canvas, accepted, remaining, stats)."""
+                     request: int = 0, stats=None, prev_argmax=None):
+        """One step: pass over the canvas (unless `stats` is given), then the sampler
+        (the configuration's rule; `prev_argmax` = the previous step's argmax, for
+        the entropy-budget rule).  Returns (canvas, accepted, remaining, stats)."""
         c = self.cfg
         if stats is None:
             stats = self.forward(canvas, cache, want_stats=True)
         canvas, accepted, remaining = sample_step(
             canvas, accepted, stats["argmax"], stats["entropy"], stats["logconf"], seed=seed,
             block=block, step=step, vocab=c.vocab, entropy_thresh=c.entropy_thresh,
-            min_accept=c.min_accept, max_steps=c.max_steps, request=request)
+            min_accept=c.min_accept, max_steps=c.max_steps, request=request,
+            rule="budget" if getattr(c, "sampler", 0) == 1 else "threshold",
+            entropy_budget=getattr(c, "entropy_budget", 0.1), stop_entropy=getattr(c, "stop_entropy", 0.005),
+            prev_argmax=prev_argmax)
         return canvas, accepted, remaining, stats
 
     def open_canvas(self, *, seed: int, block: int, request: int = 0):
@@ -157,10 +161,12 @@ class Oracle:
         for b in range(n_out // c.canvas):
             canvas, accepted = self.open_canvas(seed=seed, block=b, request=request)
             s = 0
+            prev = None
             while True:
                 s += 1
-                canvas, accepted, rem, _ = self.denoise_step(cache, canvas, accepted, seed=seed,
-                                                             block=b, step=s, request=request)
+                canvas, accepted, rem, st = self.denoise_step(cache, canvas, accepted, seed=seed, block=b,
+                                                              step=s, request=request, prev_argmax=prev)
+                prev = st["argmax"]
                 if rem == 0:
                     break
             steps.append(s)

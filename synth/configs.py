@@ -33,6 +33,9 @@ class ModelConfig:
     entropy_thresh: float = 1.0
     rope_theta: float = 10000.0
     norm_eps: float = 1e-6
+    sampler: int = 0               # 0: entropy threshold + min_accept; 1: the pages' entropy budget
+    entropy_budget: float = 0.1
+    stop_entropy: float = 0.005
 
     @property
     def qkv_rows(self) -> int:

@@ -131,3 +131,50 @@ def test_sampler_step_cap_forces_acceptance(tiny_handle):
     tok, mask, _, _ = tiny_handle.get_canvas(req)
     assert mask.cpu().numpy().all() and tiny_handle.read_remaining(req) == 0
     np.testing.assert_array_equal(tok.cpu().numpy(), am)
+
+
+@pytest.fixture(scope="module")
+def budget_handle(dgmod):
+    w = to_device(make_weights(TINY, seed=0))
+    h = dgmod.DG(TINY.with_(sampler=1), w, max_requests=2, kv_capacity=1024)
+    yield h
+    h.close()
+
+
+@pytest.mark.parametrize("case", ["budget", "converge"])
+def test_entropy_budget_sampler_bitwise(budget_handle, case):
+    """The pages' entropy-budget rule from identical fp32 statistics: canvas,
+    mask and remaining match the oracle exactly at every step.  "budget": small
+    entropies spread so the running sum crosses 0.1 mid-canvas; "converge": the
+    argmax repeats with tiny entropies from step 3, so the canvas converges."""
+    C, V = TINY.canvas, TINY.vocab
+    req, seed = 1, 5 if case == "budget" else 6
+    budget_handle.open_canvas(req, seed, 0)
+    canvas, acc = OS.init_canvas(C, seed=seed, block=0, vocab=V, request=req)
+    rng = np.random.default_rng(17 if case == "budget" else 18)
+    am_fixed = rng.integers(0, V, size=C).astype(np.int32)
+    prev = None
+    for step in range(1, TINY.max_steps + 1):
+        if case == "budget":
+            H = rng.choice([0.0, 0.004, 0.01, 0.03, 2.0], size=C).astype(np.float32)
+            am = rng.integers(0, V, size=C).astype(np.int32)
+        else:
+            H = np.full(C, 1e-4 if step >= 3 else 0.5, dtype=np.float32)
+            am = am_fixed
+        lc = np.round(rng.normal(-5.0, 0.3, size=C), 2).astype(np.float32)
+        budget_handle.op_sample(req, torch.from_numpy(H).cuda(), torch.from_numpy(lc).cuda(),
+                                torch.from_numpy(am).cuda(), step)
+        canvas, acc, rem = OS.sample_step(canvas, acc, am, H.astype(np.float64), lc.astype(np.float64), seed=seed,
+                                          block=0, step=step, vocab=V, entropy_thresh=TINY.entropy_thresh,
+                                          min_accept=TINY.min_accept, max_steps=TINY.max_steps, request=req,
+                                          rule="budget", entropy_budget=0.1, stop_entropy=0.005, prev_argmax=prev)
+        prev = am
+        tok, mask, _, _ = budget_handle.get_canvas(req)
+        np.testing.assert_array_equal(tok.cpu().numpy(), canvas)
+        np.testing.assert_array_equal(mask.cpu().numpy().astype(bool), acc)
+        assert budget_handle.read_remaining(req) == rem
+        if rem == 0:
+            break
+    if case == "converge":
+        assert step == 3 and rem == 0
+    budget_handle.sync()

@@ -92,3 +92,80 @@ def test_min_accept_larger_than_remaining():
     acc[[2, 7]] = False
     got = S.accept_set(np.full(10, 5.0), np.zeros(10), acc, 1.0, 22)
     assert set(np.nonzero(got)[0]) == {2, 7}
+
+
+# --- entropy-budget rule ----------------------------------------------------
+
+def _budget_brute(H, lc, acc, budget):
+    """The budget rule restated as a search: the largest k such that the k most
+    confident open positions have total entropy (accumulated one by one)
+    within the budget at every prefix past the first; at least one."""
+    U = [i for i in range(len(H)) if not acc[i]]
+    order = sorted(U, key=lambda i: (-lc[i], i))
+    b = float(np.float32(budget))
+    best = 1 if order else 0
+    for k in range(2, len(order) + 1):
+        prefix_ok = True
+        s = 0.0
+        for r in range(k):
+            s += float(H[order[r]])
+            if r > 0 and s > b:
+                prefix_ok = False
+        if prefix_ok:
+            best = k
+    A = np.zeros(len(H), dtype=bool)
+    A[order[:best]] = True
+    return A
+
+
+def test_budget_rule_against_search():
+    rng = np.random.default_rng(11)
+    for trial in range(400):
+        n = int(rng.integers(1, 9))
+        H = rng.choice([0.0, 0.01, 0.02, 0.05, 0.08, 0.3], size=n)
+        lc = rng.choice([-1.0, -0.5, -0.2], size=n)         # ties
+        acc = rng.random(n) < 0.3
+        budget = float(rng.choice([0.0, 0.05, 0.1, 0.2]))
+        got = S.accept_set_budget(H, lc, acc, np.zeros(n, int), None, budget, 0.005)
+        np.testing.assert_array_equal(got, _budget_brute(H, lc, acc, budget), err_msg=f"trial {trial}")
+        if (~acc).any():
+            assert got[~acc].sum() >= 1          # progress every step
+        assert not (got & acc).any()             # frozen positions stay out
+
+
+def test_budget_rule_zero_budget_takes_one_per_step():
+    """Entropies above a zero budget: exactly one position (the most confident)
+    per step, so a canvas of n takes n steps unless the cap comes first."""
+    n, V = 10, 50
+    H = np.full(n, 2.0)
+    lc = -np.arange(n, dtype=float) * 0.1
+    canvas, acc = S.init_canvas(n, seed=3, block=0, vocab=V)
+    am = np.arange(n)
+    for step in range(1, n + 1):
+        canvas, acc, rem = S.sample_step(canvas, acc, am, H, lc, seed=3, block=0, step=step, vocab=V,
+                                         entropy_thresh=1.0, min_accept=22, max_steps=100, rule="budget",
+                                         entropy_budget=0.0, stop_entropy=0.005)
+        assert rem == n - step and acc[:step].all() and not acc[step:].any()
+
+
+def test_budget_rule_convergence_and_cap():
+    n, V = 8, 50
+    H = np.full(n, 1e-4)
+    lc = np.zeros(n)
+    am = np.arange(n) + 5
+    acc = np.zeros(n, bool)
+    # low mean entropy but no previous step: only the budget applies (all fit: 8e-4 <= 0.1)
+    A = S.accept_set_budget(H, lc, acc, am, None, 0.0, 0.005)
+    assert A.sum() == 1
+    # same argmax as the previous step and mean entropy 1e-4 < 0.005: converged
+    A = S.accept_set_budget(H, lc, acc, am, am.copy(), 0.0, 0.005)
+    assert A.all()
+    # one position changed its argmax: not converged
+    prev = am.copy()
+    prev[3] += 1
+    assert S.accept_set_budget(H, lc, acc, am, prev, 0.0, 0.005).sum() == 1
+    # mean entropy at the threshold is not below it
+    H2 = np.full(n, float(np.float32(0.005)))
+    assert S.accept_set_budget(H2, lc, acc, am, am, 0.0, 0.005).sum() == 1
+    # the step cap takes everything
+    assert S.accept_set_budget(np.full(n, 9.0), lc, acc, am, None, 0.0, 0.005, force_all=True).all()
