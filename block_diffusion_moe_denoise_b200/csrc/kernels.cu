@@ -271,9 +271,11 @@ cudaError_t run_topk(const float* logits, int T, int E, int k, int* idx, float* 
 }
 
 // ---------------------------------------------------------------------------
-// Expert grouping (single CTA): per-expert counts, exclusive offsets, the row
-// of every (token, slot) pair in expert-grouped order (tokens ascending inside
-// an expert, via per-expert token bitmasks), and the GEMM tile lists.
+// Expert grouping (single CTA, the operation-level entry point): per-expert
+// counts, exclusive offsets and the row of every (token, slot) pair in
+// expert-grouped order (tokens ascending inside an expert, via per-expert token
+// bitmasks).  The decoder pass uses k_group_gather, which also builds the GEMM
+// tile lists and gathers the rows.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024) k_group(GroupArgs a) {
   pdl_trigger();
@@ -283,8 +285,7 @@ __global__ void __launch_bounds__(1024) k_group(GroupArgs a) {
   const int MW = (T + 31) >> 5;
   int* cnt = gsm;                 // [E]
   int* off = cnt + E;             // [E+1]
-  int* toff = off + E + 1;        // [E+1]
-  unsigned* mask = reinterpret_cast<unsigned*>(toff + E + 1);  // [E][MW]
+  unsigned* mask = reinterpret_cast<unsigned*>(off + E + 1);  // [E][MW]
   const int tid = threadIdx.x;
   for (int i = tid; i < E; i += blockDim.x) cnt[i] = 0;
   for (int i = tid; i < E * MW; i += blockDim.x) mask[i] = 0u;
@@ -303,21 +304,13 @@ __global__ void __launch_bounds__(1024) k_group(GroupArgs a) {
   __syncthreads();
   if (tid == 0) {
     off[0] = 0;
-    toff[0] = 0;
-    for (int e = 0; e < E; ++e) {
-      off[e + 1] = off[e] + cnt[e];
-      toff[e + 1] = toff[e] + (cnt[e] + kExpertRows - 1) / kExpertRows;
-    }
+    for (int e = 0; e < E; ++e) off[e + 1] = off[e] + cnt[e];
     if (a.route_stats) {
       int touched = 0;
       for (int e = 0; e < E; ++e) touched += cnt[e] > 0;
       atomicAdd(&a.route_stats[0], (unsigned long long)touched);
       atomicAdd(&a.route_stats[1], 1ull);
     }
-    const int egu = toff[E] * a.FJ, ed = toff[E] * a.MD;
-    if (egu > a.egu_cap || ed > a.ed_cap) atomicOr(a.err, DG_DEVERR_CAPACITY);
-    *a.egu_count = min(egu, a.egu_cap);
-    *a.ed_count = min(ed, a.ed_cap);
   }
   __syncthreads();
   for (int e = tid; e < E; e += blockDim.x) {
@@ -338,22 +331,11 @@ __global__ void __launch_bounds__(1024) k_group(GroupArgs a) {
     a.row_weight[row] = a.w[p];
     a.row_pair[row] = p;
   }
-  for (int e = tid; e < E; e += blockDim.x) {
-    const int n_nt = toff[e + 1] - toff[e];
-    for (int nt = 0; nt < n_nt; ++nt) {
-      const int base_g = (toff[e] + nt) * a.FJ;
-      for (int j = 0; j < a.FJ; ++j)
-        if (base_g + j < a.egu_cap) a.egu_tiles[base_g + j] = make_int4(e, j, nt, 0);
-      const int base_d = (toff[e] + nt) * a.MD;
-      for (int m = 0; m < a.MD; ++m)
-        if (base_d + m < a.ed_cap) a.ed_tiles[base_d + m] = make_int4(e, m, nt, 0);
-    }
-  }
 }
 
 cudaError_t run_group(const GroupArgs& a, cudaStream_t st) {
   const int MW = (a.T + 31) >> 5;
-  const size_t smem = (size_t)(3 * a.E + 2 + a.E * MW) * sizeof(int);
+  const size_t smem = (size_t)(2 * a.E + 1 + a.E * MW) * sizeof(int);
   static size_t configured = 0;
   if (smem > configured) {
     cudaError_t e = cudaFuncSetAttribute(k_group, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
