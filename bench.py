@@ -6,9 +6,10 @@ Workload (default "generate"): the full synthetic 30-layer MoE stack (d 2816,
 weights, N(0, 0.02)), batch 1, a 4096-token uniform-random prompt prefilled
 into the KV cache, then 256-token canvases.  One benchmark step is one canvas:
 open (Philox init), denoising steps until every position is accepted (12 with
-the >=22-most-confident rule), commit.  Canvases cycle through blocks 0..3 at
+the >=22-most-confident rule), commit.  The commit's decoder pass runs inside
+the next canvas's first denoising step.  Canvases cycle through blocks 0..3 at
 KV positions 4096, 4352, 4608, 4864 (4096 in / 1024 out), the KV length being
-reset to 4096 every fourth canvas.
+reset to 4096 every fourth canvas (which runs the pending commit on its own).
 
   value       output tokens/s of the whole job (inputs resident in HBM),
               device-timed with CUDA events, max over ranks
@@ -18,7 +19,7 @@ reset to 4096 every fourth canvas.
               measured HBM copy bandwidth
   cpu_baseline  the fp64 oracle on the host cores, on a bounded sample
 
-`--impl reference` times the oracle alone (the reference arm of this build).
+`--impl reference` times the fp64 oracle alone on the host cores.
 Multi-GPU: independent replicas, one per rank (no data-path collective).
 """
 from __future__ import annotations

@@ -183,7 +183,7 @@ class DG:
         check(self.lib.dg_op_lm_head(self.h, _ptr(x), T, _ptr(stats), _ptr(am), _ptr(logits)), "dg_op_lm_head")
         return stats, am, logits
 
-    KERNEL_CLASSES = ("embed", "rmsnorm", "qkv", "attention", "oproj", "router", "group", "gather",
+    KERNEL_CLASSES = ("embed", "rmsnorm", "qkv", "attention", "oproj", "group",
                       "experts_gate_up", "experts_down", "shared_gate_up", "shared_down", "lm_head", "lm_combine",
                       "sample", "other")
 

@@ -193,11 +193,12 @@ struct KernelProfiler {
   }
 };
 
-const char* const kKernelClass[] = {"embed", "rmsnorm", "qkv", "attention", "oproj", "router", "group", "gather",
+const char* const kKernelClass[] = {"embed", "rmsnorm", "qkv", "attention", "oproj", "group",
                                     "experts_gate_up", "experts_down", "shared_gate_up", "shared_down", "lm_head",
                                     "lm_combine", "sample", "other"};
-enum KClass { K_EMBED, K_RMSNORM, K_QKV, K_ATTN, K_OPROJ, K_ROUTER, K_GROUP, K_GATHER, K_EGU, K_ED, K_SGU, K_SD,
-              K_LM, K_LMC, K_SAMPLE, K_OTHER };
+enum KClass { K_EMBED, K_RMSNORM, K_QKV, K_ATTN, K_OPROJ, K_GROUP, K_EGU, K_ED, K_SGU, K_SD, K_LM, K_LMC, K_SAMPLE,
+              K_OTHER, K_NCLASS };
+static_assert(K_NCLASS <= 16, "profiler tables hold 16 classes");
 
 struct dg_handle {
   dg_config cfg;
@@ -1015,7 +1016,7 @@ int dg_profile(dg_handle* h, int enable) {
   if (!h) return DG_E_ARG;
   h->prof.flush();
   if (enable < 0) {
-    for (int i = 0; i < 16; ++i) {
+    for (int i = 0; i < K_NCLASS; ++i) {
       h->prof.total_ms[i] = 0.0;
       h->prof.count[i] = 0;
     }
@@ -1028,7 +1029,7 @@ int dg_profile(dg_handle* h, int enable) {
 int dg_profile_read(dg_handle* h, const char* kernel, double* total_ms, int64_t* launches) {
   if (!h || !kernel) return DG_E_ARG;
   h->prof.flush();
-  for (int i = 0; i < 16; ++i)
+  for (int i = 0; i < K_NCLASS; ++i)
     if (strcmp(kernel, kKernelClass[i]) == 0) {
       if (total_ms) *total_ms = h->prof.total_ms[i];
       if (launches) *launches = h->prof.count[i];

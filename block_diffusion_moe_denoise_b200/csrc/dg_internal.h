@@ -138,7 +138,6 @@ cudaError_t run_group(const GroupArgs& a, cudaStream_t st);
 // set, plus the gather of u rows into xp; clears all of `mask_next`
 cudaError_t run_route(const bf16* u, int d, bf16* xp, unsigned* mask, unsigned* mask_next, int MW,
                       const GroupArgs& a, cudaStream_t st);
-cudaError_t run_gather(const bf16* u, const int* row_token, int rows, int d, bf16* xp, cudaStream_t st);
 cudaError_t run_lm_combine(const float4* part, int G, int MT, int T, float* stats, int* argmax, int* err,
                            cudaStream_t st);
 struct SampleArgs {

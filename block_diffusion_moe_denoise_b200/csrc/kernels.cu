@@ -508,30 +508,6 @@ cudaError_t run_route(const bf16* u, int d, bf16* xp, unsigned* mask, unsigned* 
 }
 
 // ---------------------------------------------------------------------------
-// Gather token rows into expert-grouped order: xp[row] = u[row_token[row]].
-// ---------------------------------------------------------------------------
-__global__ void k_gather(const bf16* __restrict__ u, const int* __restrict__ row_token, int rows, int d,
-                         bf16* __restrict__ xp) {
-  pdl_trigger();
-  pdl_wait();
-  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= rows) return;
-  const uint4* src = reinterpret_cast<const uint4*>(u + (size_t)row_token[row] * d);
-  uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)row * d);
-  for (int c = lane; c < d / 8; c += 32) dst[c] = src[c];
-}
-
-cudaError_t run_gather(const bf16* u, const int* row_token, int rows, int d, bf16* xp, cudaStream_t st) {
-  if (rows == 0) return cudaSuccess;
-  {
-    const cudaError_t e_ = launch_pdl(k_gather, dim3((rows + 7) / 8), dim3(256), 0, st, u, row_token, rows, d, xp);
-    if (e_ != cudaSuccess) return e_;
-  }
-  return cudaGetLastError();
-}
-
-// ---------------------------------------------------------------------------
 // Merge of the LM head's per-CTA partials, in CTA order:
 //   m = max, s = sum e^(z-m), t = sum e^(z-m)(z-m), argmax lowest id on ties.
 //   logZ = m + ln s, H = ln s - t/s, logconf = -ln s.

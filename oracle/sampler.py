@@ -4,11 +4,11 @@ The pages' loop ([P2] §"How the sampler actually works"): after the
 bidirectional pass, take a candidate token at every position, accept positions
 from most to least confident, re-randomise the rejected ones for the next
 step, and stop when the canvas has converged or at a step cap.  Accepted
-tokens are kept ([P2] §"What DiffusionGemma is": the model "accepts the tokens
-it is confident about, re-randomizes the rest").
+tokens stay fixed while the others are drawn again ([P2] §"What DiffusionGemma
+is").
 
-Rule used here (the workload's sampler rule, which replaces the pages'
-cumulative entropy budget of 0.1):
+Default rule (the workload's sampler rule; the pages' cumulative entropy
+budget of 0.1 is the second rule below):
   U = positions not yet accepted;
   A = {i in U : H_i <= entropy_thresh}
       union the min(min_accept, |U|) positions of U with the highest logconf
