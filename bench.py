@@ -147,11 +147,13 @@ def step_work(cfg, kv_len: int, T: int, n_touched: float):
 # ---------------------------------------------------------------------------
 # oracle baseline (host cores)
 # ---------------------------------------------------------------------------
-def oracle_sample(reps: int = 1, warm: int = 0):
+def oracle_sample(reps: int = 1, warm: int = 0, min_seconds: float = 0.0):
     """Time the fp64 oracle on a bounded sample of the workload: one of the 30
     layers of a denoising step over a 256-token canvas with a 4096-token
     prefix, plus the LM head over 1/16 of the vocabulary; scaled to a canvas
-    (12 steps of 30 layers + LM head, one 30-layer commit)."""
+    (12 steps of 30 layers + LM head, one 30-layer commit).  Runs `warm`
+    untimed and at least `reps` timed repetitions, more until `min_seconds` of
+    timed work have accumulated."""
     import numpy as np
     from oracle import layers as OL
     from oracle.model import Oracle
@@ -173,7 +175,8 @@ def oracle_sample(reps: int = 1, warm: int = 0):
     k, v = make_kv_prefix(FULL, PROMPT, seed=1)
     ora = Oracle(cfg1, {"embed": emb_rows, "final_norm": np.ones(FULL.d_model), "layers": [lw]})
     times = []
-    for it in range(warm + reps):
+    it = 0
+    while it < warm + reps or (sum(t[3] for t in times) < min_seconds and it < warm + 1000):
         cache = ora.new_cache(PROMPT + 256)
         cache.K[0][:, :PROMPT] = to_f64(k)
         cache.V[0][:, :PROMPT] = to_f64(v)
@@ -191,11 +194,12 @@ def oracle_sample(reps: int = 1, warm: int = 0):
             t_step = FULL.n_layers * t_layer + t_lm
             t_canvas = 12 * t_step + FULL.n_layers * t_layer
             times.append((256.0 / t_canvas, t_canvas, t_step, t1 - t0 + t2 - t1))
+        it += 1
     tok_s = sum(t[0] for t in times) / len(times)
     return {"value": tok_s, "unit": "tok/s", "cores": threads, "kind": "oracle",
             "sample": f"fp64 oracle: 1 of 30 layers of one denoising step (256-token canvas, 4096-token KV prefix) "
                       f"+ LM head on 1/16 of the vocab, scaled to 12 steps + 1 commit per 256-token canvas; "
-                      f"mean of {reps} timed repetitions ({sum(t[3] for t in times):.1f} s of CPU work)",
+                      f"mean of {len(times)} timed repetitions ({sum(t[3] for t in times):.1f} s of CPU work)",
             "ms_per_denoise_step": 1e3 * sum(t[2] for t in times) / len(times),
             "ms_per_canvas": 1e3 * sum(t[1] for t in times) / len(times),
             "sample_seconds": sum(t[3] for t in times) / len(times)}
@@ -429,7 +433,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        s = oracle_sample(reps=5, warm=1)
+        s = oracle_sample(reps=3, warm=1, min_seconds=10.0)
         cpu = {k: s[k] for k in ("value", "unit", "cores", "kind", "sample")}
 
     line = {
