@@ -13,9 +13,10 @@
 //              transposed so both MMAs read K-major operands); a K slot is
 //              refilled as soon as the S MMA that read it completes, a V slot
 //              once its PV MMA completes
-//   warp 1     MMA issuer: S = Q K^T into one of two TMEM buffers (N = 64, Q
-//              read from tensor memory), O += P V^T into TMEM (N = D); S(j+1)
-//              is issued before PV(j)
+//   warp 1     S issuer: S = Q K^T into one of two TMEM buffers (N = 64, Q read
+//              from tensor memory)
+//   warp 7     P V issuer: O += P V^T into TMEM (N = D); two issuing threads keep
+//              the S stream from waiting behind P V and the other way round
 //   warps 2-5  one query row per thread: Q row into tensor memory, then per
 //              tile the exp2-domain online softmax on the S row read from TMEM,
 //              P row (bf16) written into the swizzled shared tile PV reads.
@@ -33,7 +34,8 @@ constexpr int kAK = 64;         // keys per tile
 constexpr int kAStages = 3;     // K/V ring depth
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int kVWarp = 6;                 // V^T producer
-constexpr int kAttnThreads = 32 * (kVWarp + 1);
+constexpr int kPVWarp = 7;                // issuer of the P V MMAs
+constexpr int kAttnThreads = 32 * (kPVWarp + 1);
 
 // Tensor memory (512 columns): O fp32 in [0, D), the two S buffers at 256 and
 // 320, Q (bf16 pairs, the A operand of S = Q K^T) in [384, 384 + D/2).
@@ -172,16 +174,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
       }
     }
   } else if (warp == 1) {
+    // S MMAs: S(j) as soon as its S buffer is free and its K tile landed,
+    // independently of the P V stream (separate issuing thread)
     if (lane == 0 && n_tiles > 0) {
       const uint32_t idesc_s = umma_idesc_bf16(128, kAK);
-      const uint32_t idesc_o = umma_idesc_bf16(128, D);
-      const uint32_t p0 = smem_u32(sP);
       bool ok = mbar_wait_bounded(q_ready, 0, abort_flag, err);
-      // S(j) = Q K_j^T into S buffer j%2
-      auto issue_s = [&](int j) -> bool {
+      for (int j = 0; ok && j < n_tiles; ++j) {
         const int b = j & 1, stage = j % kAStages;
-        if (!mbar_wait_bounded(&s_empty[b], ((j >> 1) & 1) ^ 1, abort_flag, err)) return false;
-        if (!mbar_wait_bounded(&k_full[stage], (j / kAStages) & 1, abort_flag, err)) return false;
+        if (!mbar_wait_bounded(&s_empty[b], ((j >> 1) & 1) ^ 1, abort_flag, err)) break;
+        if (!mbar_wait_bounded(&k_full[stage], (j / kAStages) & 1, abort_flag, err)) break;
         tc_fence_after();
         const uint32_t k0 = smem_u32(sK + (size_t)stage * S::kK);
 #pragma unroll
@@ -192,11 +193,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
                          umma_sdesc_k128(k0 + kb * (kAK * 128) + 32 * k), idesc_s, (kb | k) != 0 ? 1u : 0u);
         umma_commit(&k_empty[stage]);
         umma_commit(&s_full[b]);
-        return true;
-      };
-      if (ok) ok = issue_s(0);
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        if (j + 1 < n_tiles && !issue_s(j + 1)) break;
+      }
+    }
+  } else if (warp == kPVWarp) {
+    // O += P(j) V(j)^T as soon as the softmax has written P(j)
+    if (lane == 0 && n_tiles > 0) {
+      const uint32_t idesc_o = umma_idesc_bf16(128, D);
+      const uint32_t p0 = smem_u32(sP);
+      for (int j = 0; j < n_tiles; ++j) {
         const int b = j & 1, stage = j % kAStages;
         if (!mbar_wait_bounded(&v_full[stage], (j / kAStages) & 1, abort_flag, err)) break;
         if (!mbar_wait_bounded(&p_full[b], (j >> 1) & 1, abort_flag, err)) break;
