@@ -20,7 +20,7 @@ constexpr int kSplitCap = 8;
 // A prefill pass carries up to this many consecutive 256-token segments of one
 // request (block-causal: each attends to the cache before it and to itself),
 // so the weights are streamed once per group instead of once per segment.
-constexpr int kPrefillSlots = 4;
+constexpr int kPrefillSlots = DG_MAX_REQUESTS;
 
 // Passes carry at most this many canvas-sized slots.
 int pass_slots(int max_req) { return max_req > kPrefillSlots ? max_req : kPrefillSlots; }

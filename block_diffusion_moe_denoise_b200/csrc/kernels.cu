@@ -497,7 +497,7 @@ __global__ void __launch_bounds__(256) k_group_gather(GroupArgs a, const unsigne
 
 cudaError_t run_route(const bf16* u, int d, bf16* xp, unsigned* mask, unsigned* mask_next, int MW,
                       const GroupArgs& a, cudaStream_t st) {
-  if (a.T < 1 || a.T > 1024 || a.E > 256 || MW * 32 < a.T) return cudaErrorInvalidValue;
+  if (a.T < 1 || a.T > DG_MAX_REQUESTS * 256 || a.E > 256 || MW * 32 < a.T) return cudaErrorInvalidValue;
   const int P = a.T * a.k;
   const int grid = (P + 7) / 8 < 148 ? (P + 7) / 8 : 148;
   {

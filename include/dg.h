@@ -127,7 +127,7 @@ const char* dg_strerror(int code);
 /* Append `n` prompt tokens (device int32 array) to request `req`'s KV cache:
  * the decoder runs over segments of `canvas` tokens counted from the first
  * token; each segment attends to all earlier positions and bidirectionally to
- * itself.  Up to four full segments share one decoder pass (block-causal
+ * itself.  Up to eight full segments share one decoder pass (block-causal
  * slots), with a result bit-identical to one segment per call.  Fails with
  * DG_E_STATE while a canvas is open, DG_E_CAPACITY if the cache would
  * overflow. */
