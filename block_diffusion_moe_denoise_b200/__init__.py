@@ -34,7 +34,7 @@ def config_struct(cfg) -> dg_config:
                      cfg.top_k, cfg.ffn_expert, cfg.ffn_shared, cfg.vocab, cfg.canvas, cfg.max_steps,
                      cfg.min_accept, cfg.entropy_thresh, cfg.rope_theta, cfg.norm_eps,
                      getattr(cfg, "sampler", 0), getattr(cfg, "entropy_budget", 0.1),
-                     getattr(cfg, "stop_entropy", 0.005))
+                     getattr(cfg, "stop_entropy", 0.005), getattr(cfg, "temperature", 0.0))
 
 
 def philox_tokens(seed: int, block: int, step: int, request: int, pos0: int, n: int, vocab: int,
@@ -182,6 +182,17 @@ class DG:
         logits = torch.empty((T, self.cfg.vocab), dtype=torch.float32, device=dev) if want_logits else None
         check(self.lib.dg_op_lm_head(self.h, _ptr(x), T, _ptr(stats), _ptr(am), _ptr(logits)), "dg_op_lm_head")
         return stats, am, logits
+
+    def op_lm_sample(self, x: torch.Tensor, temperature: float, seed: int, block: int, step: int, request: int = 0):
+        """dg_op_lm_sample: LM-head statistics and drawn candidates of rows = positions 0..T-1."""
+        T = x.shape[0]
+        dev = x.device
+        stats = torch.empty((T, 4), dtype=torch.float32, device=dev)
+        am = torch.empty(T, dtype=torch.int32, device=dev)
+        cand = torch.empty(T, dtype=torch.int32, device=dev)
+        check(self.lib.dg_op_lm_sample(self.h, _ptr(x), T, temperature, seed, block, step, request, _ptr(stats),
+                                       _ptr(am), _ptr(cand)), "dg_op_lm_sample")
+        return stats, am, cand
 
     KERNEL_CLASSES = ("embed", "rmsnorm", "qkv", "attention", "oproj", "group",
                       "experts_gate_up", "experts_down", "shared_gate_up", "shared_down", "lm_head", "lm_combine",

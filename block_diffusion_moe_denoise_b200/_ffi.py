@@ -18,7 +18,8 @@ class dg_config(C.Structure):
                                        "top_k", "ffn_expert", "ffn_shared", "vocab", "canvas", "max_steps",
                                        "min_accept")] + \
                [("entropy_thresh", C.c_float), ("rope_theta", C.c_float), ("norm_eps", C.c_float),
-                ("sampler", C.c_int), ("entropy_budget", C.c_float), ("stop_entropy", C.c_float)]
+                ("sampler", C.c_int), ("entropy_budget", C.c_float), ("stop_entropy", C.c_float),
+                ("temperature", C.c_float)]
 
 
 class dg_layer_weights(C.Structure):
@@ -65,6 +66,8 @@ _SIGS = {
                                     C.c_void_p]),
     "dg_op_sample": (C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int]),
     "dg_op_lm_head": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p]),
+    "dg_op_lm_sample": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int, C.c_float, C.c_uint64, C.c_int, C.c_int, C.c_int,
+                                  C.c_void_p, C.c_void_p, C.c_void_p]),
     "dg_profile": (C.c_int, [C.c_void_p, C.c_int]),
     "dg_profile_read": (C.c_int, [C.c_void_p, C.c_char_p, C.POINTER(C.c_double), C.POINTER(C.c_int64)]),
     "dg_launch_count": (C.c_int64, [C.c_void_p]),

@@ -260,3 +260,31 @@ DG_DEVINL float warp_max(float v) {
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
   return v;
 }
+
+// ---------------------------------------------------------------------------
+// Philox-4x32-10 (Salmon et al., SC'11): ten rounds of two 32x32->64-bit
+// multiplies with the high halves XORed into the odd words and the round key,
+// key bumped by the Weyl constants between rounds.  Returns all four words.
+// ---------------------------------------------------------------------------
+DG_DEVINL uint4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3, uint32_t k0, uint32_t k1) {
+  constexpr uint32_t M0 = 0xD2511F53u, M1 = 0xCD9E8D57u, W0 = 0x9E3779B9u, W1 = 0xBB67AE85u;
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    if (r > 0) {
+      k0 += W0;
+      k1 += W1;
+    }
+    const uint32_t lo0 = M0 * c0, hi0 = __umulhi(M0, c0);
+    const uint32_t lo1 = M1 * c2, hi1 = __umulhi(M1, c2);
+    const uint32_t n0 = hi1 ^ c1 ^ k0, n2 = hi0 ^ c3 ^ k1;
+    c0 = n0;
+    c1 = lo1;
+    c2 = n2;
+    c3 = lo0;
+  }
+  return make_uint4(c0, c1, c2, c3);
+}
+
+// A 32-bit word as an odd multiple of 2^-24 in (0, 1): (2 (w >> 9) + 1) / 2^24,
+// exact in float32 and never 0 or 1.
+DG_DEVINL float word_uniform(uint32_t w) { return (float)(2u * (w >> 9) + 1u) * 5.9604644775390625e-8f; }

@@ -66,6 +66,7 @@ bool config_ok(const dg_config* c) {
   if (c->max_steps < 1 || c->min_accept < 0) return false;
   if (c->sampler != DG_SAMPLER_THRESHOLD && c->sampler != DG_SAMPLER_ENTROPY_BUDGET) return false;
   if (c->sampler == DG_SAMPLER_ENTROPY_BUDGET && !(c->entropy_budget >= 0.f && c->stop_entropy >= 0.f)) return false;
+  if (!(c->temperature >= 0.f && c->temperature <= 1e30f)) return false;
   return true;
 }
 
@@ -106,6 +107,8 @@ void make_plan(const dg_config* c, int max_req, long long cap_user, Plan* p) {
   p->add("lm_part", (size_t)kLmGridMax * Tcap * 16);
   p->add("stats", (size_t)Tcap * 16);
   p->add("argmax", (size_t)Tcap * 4);
+  p->add("draw", (size_t)max_req * c->canvas * (c->vocab / 256) * 8);
+  p->add("cand", (size_t)max_req * c->canvas * 4);
   p->add("canvas", (size_t)max_req * c->canvas * 4);
   p->add("commit_tok", (size_t)max_req * c->canvas * 4);
   p->add("prev_argmax", (size_t)max_req * c->canvas * 4);
@@ -260,7 +263,7 @@ namespace {
 // One decoder pass over the slots of `s`.  With want_lm, the final norm and
 // the LM head run over the first lm_rows tokens only (lm_rows < 0: all).
 int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layers, bool qkv_only_last, bool want_lm,
-             float* logits, int lm_rows = -1) {
+             float* logits, int lm_rows = -1, const DrawKeys* keys = nullptr, float temperature = 0.f) {
   const dg_config& c = h->cfg;
   const int T = s.n * s.Tr;
   const int TL = lm_rows < 0 ? T : lm_rows;
@@ -471,11 +474,17 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     la.part = h->B<float4>("lm_part");
     la.logits = logits;
     la.err = err;
+    const bool draw = keys != nullptr && temperature > 0.f;
+    la.inv_tau = draw ? 1.0f / temperature : 1.0f;
+    la.draw = draw ? h->B<float2>("draw") : nullptr;
+    memset(&la.keys, 0, sizeof(la.keys));
+    if (draw) la.keys = *keys;
     int grid = 0;
     LAUNCH(h, K_LM, 1, run_lm_head(la, &grid, st));
     LAUNCH(h, K_LMC, 1,
            run_lm_combine(h->B<float4>("lm_part"), grid, (TL + 127) / 128, TL, h->B<float>("stats"),
-                          h->B<int>("argmax"), err, st));
+                          h->B<int>("argmax"), err, st, la.draw, (int)(c.vocab / 256), draw ? keys : nullptr,
+                          draw ? h->B<int>("cand") : nullptr));
   } else if (pending_k || pending_parts) {
     // a pass stopped after a full layer: fold its expert outputs into x
     LAUNCH(h, K_RMSNORM, 1,
@@ -713,7 +722,7 @@ int dg_open_canvas(dg_handle* h, int req, uint64_t seed, int block) {
 }
 
 static int sample_slots(dg_handle* h, int n_req, const int* reqs, const float* entropy, const float* logconf,
-                        int stride, const int* argmax, const int* steps) {
+                        int stride, const int* argmax, const int* steps, const int* cand = nullptr) {
   const dg_config& c = h->cfg;
   SampleArgs a;
   memset(&a, 0, sizeof(a));
@@ -738,6 +747,7 @@ static int sample_slots(dg_handle* h, int n_req, const int* reqs, const float* e
   a.logconf = logconf;
   a.stride = stride;
   a.argmax = argmax;
+  a.cand = cand;
   a.canvas_tok = h->B<int>("canvas");
   a.mask = h->B<unsigned char>("mask");
   a.remaining = h->B<int>("remaining");
@@ -787,11 +797,25 @@ int dg_denoise_step(dg_handle* h, int n_req, const int* reqs, int32_t* d_remaini
       ++j;
     }
   }
-  int rc = run_pass(h, ids, s, h->cfg.n_layers, false, true, nullptr, n_req * C);
+  // candidate draw keys of the canvas slots (LM-head rows slot * C + position)
+  DrawKeys keys;
+  memset(&keys, 0, sizeof(keys));
+  keys.canvas = C;
+  for (int i = 0; i < n_req; ++i) {
+    const ReqState& r = h->req[reqs[i]];
+    keys.req[i] = reqs[i];
+    keys.block[i] = r.block;
+    keys.step[i] = steps[i];
+    keys.seed[i] = r.seed;
+  }
+  const bool draw = h->cfg.temperature > 0.f;
+  int rc = run_pass(h, ids, s, h->cfg.n_layers, false, true, nullptr, n_req * C, draw ? &keys : nullptr,
+                    h->cfg.temperature);
   if (rc != DG_OK) return rc;
   for (int i = 0; i < n_req; ++i) h->req[reqs[i]].pending = false;
   float* stats = h->B<float>("stats");
-  rc = sample_slots(h, n_req, reqs, stats, stats + 1, 4, h->B<int>("argmax"), steps);
+  rc = sample_slots(h, n_req, reqs, stats, stats + 1, 4, h->B<int>("argmax"), steps,
+                    draw ? h->B<int>("cand") : nullptr);
   if (rc != DG_OK) return rc;
   for (int i = 0; i < n_req; ++i) {
     h->req[reqs[i]].step = steps[i];
@@ -990,6 +1014,45 @@ int dg_op_lm_head(dg_handle* h, const float* d_x, int T, float* d_stats, int32_t
   int grid = 0;
   CK(run_lm_head(la, &grid, h->st));
   CK(run_lm_combine(la.part, grid, (T + 127) / 128, T, h->B<float>("stats"), h->B<int>("argmax"), la.err, h->st));
+  if (d_stats) CK(cudaMemcpyAsync(d_stats, h->B<float>("stats"), (size_t)T * 16, cudaMemcpyDeviceToDevice, h->st));
+  if (d_argmax) CK(cudaMemcpyAsync(d_argmax, h->B<int>("argmax"), (size_t)T * 4, cudaMemcpyDeviceToDevice, h->st));
+  return DG_OK;
+}
+
+int dg_op_lm_sample(dg_handle* h, const float* d_x, int T, float temperature, uint64_t seed, int block, int step,
+                    int request, float* d_stats, int32_t* d_argmax, int32_t* d_cand) {
+  if (!h || !d_x || !d_cand || T < 1 || T > h->cfg.canvas || !(temperature > 0.f && temperature <= 1e30f) ||
+      block < 0 || step < 0 || request < 0 || request >= h->max_req)
+    return DG_E_ARG;
+  const dg_config& c = h->cfg;
+  float* x = h->B<float>("x");
+  CK(cudaMemcpyAsync(x, d_x, (size_t)T * c.d_model * 4, cudaMemcpyDeviceToDevice, h->st));
+  CK(run_rmsnorm(x, h->final_norm, T, c.d_model, c.norm_eps, h->B<bf16>("hn"), h->st));
+  DrawKeys keys;
+  memset(&keys, 0, sizeof(keys));
+  keys.canvas = c.canvas;
+  keys.req[0] = request;
+  keys.block[0] = block;
+  keys.step[0] = step;
+  keys.seed[0] = seed;
+  LmArgs la;
+  la.tm_x = &h->tm_hn;
+  la.tm_embed = &h->tm_embed;
+  la.T = T;
+  la.d = c.d_model;
+  la.num_sms = h->num_sms < kLmGridMax ? h->num_sms : kLmGridMax;
+  la.V = c.vocab;
+  la.part = h->B<float4>("lm_part");
+  la.logits = nullptr;
+  la.err = h->B<int>("err");
+  la.inv_tau = 1.0f / temperature;
+  la.draw = h->B<float2>("draw");
+  la.keys = keys;
+  int grid = 0;
+  CK(run_lm_head(la, &grid, h->st));
+  CK(run_lm_combine(la.part, grid, (T + 127) / 128, T, h->B<float>("stats"), h->B<int>("argmax"), la.err, h->st,
+                    la.draw, (int)(c.vocab / 256), &keys, h->B<int>("cand")));
+  CK(cudaMemcpyAsync(d_cand, h->B<int>("cand"), (size_t)T * 4, cudaMemcpyDeviceToDevice, h->st));
   if (d_stats) CK(cudaMemcpyAsync(d_stats, h->B<float>("stats"), (size_t)T * 16, cudaMemcpyDeviceToDevice, h->st));
   if (d_argmax) CK(cudaMemcpyAsync(d_argmax, h->B<int>("argmax"), (size_t)T * 4, cudaMemcpyDeviceToDevice, h->st));
   return DG_OK;

@@ -79,6 +79,16 @@ struct SharedArgs {
   unsigned* mask;     // [E][MW] per-expert token bitmasks, zero on entry
   int* err;
 };
+// Keys of the candidate draw: LM-head row r is position r % canvas of slot
+// r / canvas, drawn with that slot's (seed, block, step, request).
+struct DrawKeys {
+  int canvas;
+  int req[DG_MAX_REQUESTS];
+  int block[DG_MAX_REQUESTS];
+  int step[DG_MAX_REQUESTS];
+  unsigned long long seed[DG_MAX_REQUESTS];
+};
+
 struct LmArgs {
   const CUtensorMap* tm_x;
   const CUtensorMap* tm_embed;
@@ -87,6 +97,10 @@ struct LmArgs {
   float4* part;
   float* logits;
   int* err;
+  // candidate draw (draw == nullptr: argmax candidates only)
+  float inv_tau = 1.f;       // 1 / temperature
+  float2* draw = nullptr;    // [T][V/256]: (log-mass of the tile at 1/temperature, drawn id in the tile)
+  DrawKeys keys = {};
 };
 
 cudaError_t run_qkv(const QkvArgs& a, cudaStream_t st);
@@ -138,8 +152,12 @@ cudaError_t run_group(const GroupArgs& a, cudaStream_t st);
 // set, plus the gather of u rows into xp; clears all of `mask_next`
 cudaError_t run_route(const bf16* u, int d, bf16* xp, unsigned* mask, unsigned* mask_next, int MW,
                       const GroupArgs& a, cudaStream_t st);
+// Merge of the LM head's per-CTA partials into per-row statistics; with
+// `draw` (the per-tile records of a candidate draw, NV tiles per row) also the
+// row-level pick of the tile, whose drawn id goes to cand[row].
 cudaError_t run_lm_combine(const float4* part, int G, int MT, int T, float* stats, int* argmax, int* err,
-                           cudaStream_t st);
+                           cudaStream_t st, const float2* draw = nullptr, int NV = 0, const DrawKeys* keys = nullptr,
+                           int* cand = nullptr);
 struct SampleArgs {
   int n_slots, canvas, vocab, min_accept, max_steps;
   float thr;
@@ -154,6 +172,7 @@ struct SampleArgs {
   const float* logconf;   // [slot*canvas + i] * stride
   int stride;             // floats between consecutive positions
   const int* argmax;      // [slot*canvas + i]
+  const int* cand;        // [slot*canvas + i] drawn candidates, or nullptr (argmax candidates)
   int* canvas_tok;        // [req][canvas]
   unsigned char* mask;    // [req][canvas]
   int* remaining;         // [req]

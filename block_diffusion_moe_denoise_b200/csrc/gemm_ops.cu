@@ -545,6 +545,12 @@ struct P_SGU : ProblemBase {
 // per token tile, the running (max m, argmax a, s = sum e^(z-m),
 // t = sum e^(z-m)(z-m)) in shared memory across the CTA's tiles; the CTA's
 // partial is written at the end and merged across CTAs by k_lm_combine.
+//
+// Candidate draw (draw != nullptr), the tile level of a two-level draw from
+// softmax(z / temperature): for its row and the tile's 256 ids the thread sums
+// w_v = exp(z_v/tau - max/tau), picks the first id whose running sum reaches
+// u * sum (u from Philox, keyed by the row's slot), and stores the tile's
+// log-mass max/tau + ln(sum) with that id.  k_lm_combine picks the tile.
 // ---------------------------------------------------------------------------
 struct LmStat {
   float m, s, t;
@@ -563,12 +569,57 @@ struct P_LM : ProblemBase {
     float4* part;    // [gridDim.x][MT*128]
     float* logits;   // optional [T, V]
     int* err;
+    float inv_tau;
+    float2* draw;    // optional [T][NV]
+    DrawKeys keys;
   };
   DG_DEVINL static void prefetch(const Params& p) {
     tma_prefetch_desc(&p.tmX);
     tma_prefetch_desc(&p.tmE);
   }
   DG_DEVINL static int num_tiles(const Params& p) { return p.MT * p.NV; }
+  DG_DEVINL static float draw_weight(float z, float inv_tau, float mt) {
+    return exp2f((z * inv_tau - mt) * 1.4426950408889634f);
+  }
+  // Tile level of the candidate draw (all threads of the warp take part: the
+  // TMEM loads are warp-collective); tm / ta = the tile's max logit and its column.
+  DG_DEVINL static void draw_tile(const Params& p, const Tile& t, uint32_t taddr, int tok, bool ok, float tm,
+                                  int ta) {
+    const float it = p.inv_tau;
+    const float mt = tm * it;
+    float s = 0.f;
+    for (int c0 = 0; c0 < 256; c0 += 32) {
+      float z[32];
+      tmem_ld16(taddr + c0, z);
+      tmem_ld16(taddr + c0 + 16, z + 16);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) s += draw_weight(z[i], it, mt);
+    }
+    float u = 0.5f;
+    if (ok) {
+      const int slot = tok / p.keys.canvas, pos = tok - slot * p.keys.canvas;
+      const unsigned long long seed = p.keys.seed[slot];
+      u = word_uniform(philox4x32_10((uint32_t)pos, (uint32_t)p.keys.step[slot], (uint32_t)p.keys.block[slot],
+                                     (uint32_t)p.keys.req[slot] + 256u * (uint32_t)(t.b + 1), (uint32_t)seed,
+                                     (uint32_t)(seed >> 32))
+                           .x);
+    }
+    const float target = u * s;
+    float cum = 0.f;
+    int cand = -1;
+    for (int c0 = 0; c0 < 256; c0 += 32) {
+      float z[32];
+      tmem_ld16(taddr + c0, z);
+      tmem_ld16(taddr + c0 + 16, z + 16);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        cum += draw_weight(z[i], it, mt);
+        if (cand < 0 && cum >= target) cand = c0 + i;
+      }
+    }
+    if (cand < 0) cand = ta;  // rounding left the running sum short of the target
+    if (ok) p.draw[(size_t)tok * p.NV + t.b] = make_float2(mt + logf(s), __int_as_float(t.b * 256 + cand));
+  }
   DG_DEVINL static Tile tile(const Params& p, int v) {
     Tile t;
     t.valid = 1;
@@ -600,6 +651,8 @@ struct P_LM : ProblemBase {
     const int tok = t.a * 128 + row;
     const bool ok = tok < p.T;
     constexpr float kLog2e = 1.4426950408889634f;
+    float tm = -INFINITY;  // this tile's max logit and its column
+    int ta = 0;
     for (int c0 = 0; c0 < 256; c0 += 32) {
       float z[32];
       tmem_ld16(taddr + c0, z);
@@ -626,6 +679,10 @@ struct P_LM : ProblemBase {
         r.m = cm;
         r.a = t.b * 256 + c0 + ca;
       }
+      if (cm > tm) {
+        tm = cm;
+        ta = c0 + ca;
+      }
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         const float dz = z[i] - r.m;
@@ -635,6 +692,7 @@ struct P_LM : ProblemBase {
       }
     }
     st[t.a * 128 + row] = r;
+    if (p.draw != nullptr) draw_tile(p, t, taddr, tok, ok, tm, ta);
   }
   DG_DEVINL static void finish(const Params& p, int row, uint8_t* ep) {
     const LmStat* st = reinterpret_cast<const LmStat*>(ep);
@@ -780,7 +838,12 @@ cudaError_t run_lm_head(const LmArgs& a, int* grid_out, cudaStream_t st) {
   p.part = a.part;
   p.logits = a.logits;
   p.err = a.err;
+  p.inv_tau = a.inv_tau;
+  p.draw = a.draw;
+  p.keys = a.keys;
   if (p.MT > P_LM::MT_MAX) return cudaErrorInvalidValue;
+  if (p.draw != nullptr && (p.keys.canvas < 1 || (p.T + p.keys.canvas - 1) / p.keys.canvas > DG_MAX_REQUESTS))
+    return cudaErrorInvalidValue;
   const int grid = grid_for(p.MT * p.NV, a.num_sms);
   *grid_out = grid;
   return launch_gemm<P_LM>(p, grid, st);

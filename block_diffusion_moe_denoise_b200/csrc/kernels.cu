@@ -1,6 +1,7 @@
 // CUDA-core kernels of the denoising pass: everything that is not a dense
 // contraction.  Warp-shuffle reductions, 16-byte vector loads/stores.
 #include <float.h>
+#include <string.h>
 
 #include "common.cuh"
 #include "dg_internal.h"
@@ -532,8 +533,13 @@ DG_DEVINL LmPart lm_merge(LmPart x, LmPart y) {
   return x;
 }
 
+// With `draw`: the row level of the candidate draw.  Lane l owns a contiguous
+// run of the row's tiles; the tile masses exp(lambda_j - max) are summed per
+// lane, scanned across lanes in lane order, and the tile whose running sum
+// first reaches u * total is picked (u = word 1 of the row's re-noise Philox
+// block); its drawn id is the candidate.
 __global__ void k_lm_combine(const float4* __restrict__ part, int G, int MT, int T, float* stats, int* argmax,
-                             int* err) {
+                             int* err, const float2* __restrict__ draw, int NV, DrawKeys keys, int* cand) {
   pdl_trigger();
   pdl_wait();
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -563,45 +569,80 @@ __global__ void k_lm_combine(const float4* __restrict__ part, int G, int MT, int
     reinterpret_cast<float4*>(stats)[t] = o;
     argmax[t] = r.a;
   }
+  if (draw == nullptr) return;
+  constexpr float kLog2e = 1.4426950408889634f;
+  const float2* dr = draw + (size_t)t * NV;
+  const int per = (NV + 31) / 32;
+  const int j0 = min(lane * per, NV), j1 = min(j0 + per, NV);
+  float M = -INFINITY;
+  for (int j = j0; j < j1; ++j) M = fmaxf(M, dr[j].x);
+  M = warp_max(M);
+  float cs = 0.f;
+  for (int j = j0; j < j1; ++j) cs += exp2f((dr[j].x - M) * kLog2e);
+  float incl = cs;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  const float total = __shfl_sync(0xffffffffu, incl, 31);
+  const int slot = t / keys.canvas, pos = t - slot * keys.canvas;
+  const unsigned long long seed = keys.seed[slot];
+  const float u = word_uniform(philox4x32_10((uint32_t)pos, (uint32_t)keys.step[slot], (uint32_t)keys.block[slot],
+                                             (uint32_t)keys.req[slot], (uint32_t)seed, (uint32_t)(seed >> 32))
+                                   .y);
+  const float target = u * total;
+  const unsigned hit = __ballot_sync(0xffffffffu, incl >= target && cs > 0.f);
+  const int L = hit ? __ffs(hit) - 1 : 31;
+  int J = -1;
+  if (lane == L) {
+    const float local = target - (incl - cs);
+    float cum = 0.f;
+    int last = -1;
+    for (int j = j0; j < j1; ++j) {
+      const float w = exp2f((dr[j].x - M) * kLog2e);
+      cum += w;
+      if (w > 0.f) last = j;
+      if (J < 0 && cum >= local) J = j;
+    }
+    if (J < 0) J = last;  // rounding left the running sum short of the target
+    if (J < 0) {
+      atomicOr(err, DG_DEVERR_NAN);
+      J = 0;
+    }
+    const int c = __float_as_int(dr[J].y);
+    if (c < 0 || c >= NV * 256) atomicOr(err, DG_DEVERR_TOKEN);
+    cand[t] = c;
+  }
 }
 
 cudaError_t run_lm_combine(const float4* part, int G, int MT, int T, float* stats, int* argmax, int* err,
-                           cudaStream_t st) {
+                           cudaStream_t st, const float2* draw, int NV, const DrawKeys* keys, int* cand) {
   if (T == 0) return cudaSuccess;
+  DrawKeys k;
+  memset(&k, 0, sizeof(k));
+  if (draw != nullptr) {
+    if (keys == nullptr || cand == nullptr || NV < 1 || keys->canvas < 1 ||
+        (T + keys->canvas - 1) / keys->canvas > DG_MAX_REQUESTS)
+      return cudaErrorInvalidValue;
+    k = *keys;
+  }
   {
-    const cudaError_t e_ = launch_pdl(k_lm_combine, dim3((T + 7) / 8), dim3(256), 0, st, part, G, MT, T, stats, argmax, err);
+    const cudaError_t e_ = launch_pdl(k_lm_combine, dim3((T + 7) / 8), dim3(256), 0, st, part, G, MT, T, stats, argmax,
+                                      err, draw, NV, k, cand);
     if (e_ != cudaSuccess) return e_;
   }
   return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------
-// Philox-4x32-10 (Salmon et al., SC'11): ten rounds of two 32x32->64-bit
-// multiplies with the high halves XORed into the odd words and the round key,
-// key bumped by the Weyl constants between rounds.
+// Re-noise token: word 0 of Philox-4x32-10 (common.cuh) at counter
+// (position, step, block, request), key = seed, mapped to [0, vocab) by
+// multiply-shift.
 // ---------------------------------------------------------------------------
-DG_DEVINL uint32_t philox_word0(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3, uint32_t k0, uint32_t k1) {
-  constexpr uint32_t M0 = 0xD2511F53u, M1 = 0xCD9E8D57u, W0 = 0x9E3779B9u, W1 = 0xBB67AE85u;
-#pragma unroll
-  for (int r = 0; r < 10; ++r) {
-    if (r > 0) {
-      k0 += W0;
-      k1 += W1;
-    }
-    const uint32_t lo0 = M0 * c0, hi0 = __umulhi(M0, c0);
-    const uint32_t lo1 = M1 * c2, hi1 = __umulhi(M1, c2);
-    const uint32_t n0 = hi1 ^ c1 ^ k0, n2 = hi0 ^ c3 ^ k1;
-    c0 = n0;
-    c1 = lo1;
-    c2 = n2;
-    c3 = lo0;
-  }
-  return c0;
-}
-
 DG_DEVINL int renoise_token(unsigned long long seed, int block, int step, uint32_t pos, int request, int vocab) {
-  const uint32_t x0 = philox_word0(pos, (uint32_t)step, (uint32_t)block, (uint32_t)request, (uint32_t)seed,
-                                   (uint32_t)(seed >> 32));
+  const uint32_t x0 = philox4x32_10(pos, (uint32_t)step, (uint32_t)block, (uint32_t)request, (uint32_t)seed,
+                                    (uint32_t)(seed >> 32)).x;
   return (int)(((unsigned long long)x0 * (unsigned long long)vocab) >> 32);
 }
 
@@ -712,7 +753,15 @@ __global__ void k_sample(SampleArgs a) {
       atomicOr(a.err, DG_DEVERR_TOKEN);
       am = 0;
     }
-    a.canvas_tok[(size_t)req * C + i] = am;
+    int tok = am;
+    if (a.cand != nullptr) {
+      tok = a.cand[p];
+      if (tok < 0 || tok >= a.vocab) {
+        atomicOr(a.err, DG_DEVERR_TOKEN);
+        tok = 0;
+      }
+    }
+    a.canvas_tok[(size_t)req * C + i] = tok;
     a.mask[(size_t)req * C + i] = 1;
   } else if (valid && !acc) {
     a.canvas_tok[(size_t)req * C + i] =

@@ -74,6 +74,7 @@ typedef struct dg_config {
   int sampler;         /* DG_SAMPLER_THRESHOLD (the rule above) or DG_SAMPLER_ENTROPY_BUDGET */
   float entropy_budget;/* budget rule: nats of entropy accepted per step (0.1) */
   float stop_entropy;  /* budget rule: converged below this mean entropy (0.005) */
+  float temperature;   /* 0: candidates are the argmax; > 0: drawn from softmax(logits / temperature) */
 } dg_config;
 
 /* Sampler rules.  DG_SAMPLER_ENTROPY_BUDGET follows the pages' default sampler
@@ -83,7 +84,20 @@ typedef struct dg_config {
  * entropy_budget, and at least the most confident one; when every such
  * position keeps the argmax it had at the previous step and their mean
  * entropy is below stop_entropy, all of them are accepted (the canvas has
- * converged); at step max_steps all are accepted.  Candidates are argmax. */
+ * converged); at step max_steps all are accepted.
+ *
+ * Candidates (both rules).  With temperature 0 the token accepted at a
+ * position is its argmax.  With temperature tau > 0 it is drawn from
+ * softmax(z / tau) of the position's logits z (the pages' "sample a candidate
+ * token at every position", same section), in two levels over tiles of 256
+ * consecutive vocabulary ids: a tile by the inverse CDF of the tile masses
+ * sum exp(z_v / tau) with u_row, then an id inside it by the inverse CDF of
+ * exp(z_v / tau) with u_tile; both levels in float32.  u = (2 (w >> 9) + 1) / 2^24
+ * of a Philox-4x32-10 word w (key = seed): u_row is word 1 of counter
+ * (position, step, block, request) (word 0 is the re-noise token), u_tile of
+ * tile j is word 0 of counter (position, step, block, request + 256 (j + 1)).
+ * Entropy and confidence stay those of softmax(z): the temperature shapes the
+ * draw only.  The draw adds two passes over each LM-head tile in its epilogue. */
 #define DG_SAMPLER_THRESHOLD 0
 #define DG_SAMPLER_ENTROPY_BUDGET 1
 

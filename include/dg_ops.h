@@ -46,6 +46,14 @@ int dg_op_sample(dg_handle* h, int req, const float* d_entropy, const float* d_l
  * is not NULL the fp32 logits [T, vocab] are written too. */
 int dg_op_lm_head(dg_handle* h, const float* d_x, int T, float* d_stats, int32_t* d_argmax, float* d_logits);
 
+/* dg_op_lm_head plus the candidate draw of dg.h ("Candidates"): rows 0..T-1
+ * (T <= canvas) are positions 0..T-1 of request `request` at (seed, block,
+ * step); `temperature` > 0 overrides the configuration's.  d_cand [T] int32
+ * receives the drawn ids; d_stats and d_argmax (may be NULL) as in
+ * dg_op_lm_head.  Does not touch the request's canvas. */
+int dg_op_lm_sample(dg_handle* h, const float* d_x, int T, float temperature, uint64_t seed, int block, int step,
+                    int request, float* d_stats, int32_t* d_argmax, int32_t* d_cand);
+
 /* Run the decoder over `T` tokens (device ids) of request `req` at positions
  * [L, L+T) without advancing L, stopping after `n_layers` layers (the K/V of
  * those layers are written to the cache slots).  The intermediates of the last
@@ -59,7 +67,8 @@ int dg_debug_forward(dg_handle* h, int req, const int32_t* d_tokens, int T, int 
  * "counts" i32 [E]; "offsets" i32 [E+1];
  * "pair_row" i32 [T*k]; "row_pair" i32 [T*k]; "hp" bf16 [T*k, fe];
  * "yp" f32 [T*k, d]; "hs" bf16 [T, fs]; "stats" f32 [Tcap][4];
- * "argmax" i32 [Tcap]; "canvas" i32 [max_req, canvas]; "mask" u8 [...];
+ * "argmax" i32 [Tcap]; "cand" i32 [max_req * canvas] drawn candidates;
+ * "canvas" i32 [max_req, canvas]; "mask" u8 [...];
  * "remaining" i32 [max_req]; "route_stats" u64 [2] = (sum over router launches
  * of the number of experts that received a token, number of launches).
  * Returns DG_E_ARG for an unknown name. */

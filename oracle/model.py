@@ -30,7 +30,7 @@ from dataclasses import dataclass, field
 import numpy as np
 
 from . import layers as L_
-from .sampler import init_canvas, sample_step
+from .sampler import DRAW_TILE, candidate_uniforms, draw_candidates, init_canvas, sample_step
 
 
 @dataclass
@@ -136,13 +136,19 @@ class Oracle:
         c = self.cfg
         if stats is None:
             stats = self.forward(canvas, cache, want_stats=True)
+        cand = None
+        tau = getattr(c, "temperature", 0.0)
+        if tau > 0:
+            n = stats["logits"].shape[0]
+            u_row, u_tile = candidate_uniforms(seed, block, step, np.arange(n), c.vocab // DRAW_TILE, request)
+            cand, _ = draw_candidates(stats["logits"], tau, u_row, u_tile)
         canvas, accepted, remaining = sample_step(
             canvas, accepted, stats["argmax"], stats["entropy"], stats["logconf"], seed=seed,
             block=block, step=step, vocab=c.vocab, entropy_thresh=c.entropy_thresh,
             min_accept=c.min_accept, max_steps=c.max_steps, request=request,
             rule="budget" if getattr(c, "sampler", 0) == 1 else "threshold",
             entropy_budget=getattr(c, "entropy_budget", 0.1), stop_entropy=getattr(c, "stop_entropy", 0.005),
-            prev_argmax=prev_argmax)
+            prev_argmax=prev_argmax, candidates=cand)
         return canvas, accepted, remaining, stats
 
     def open_canvas(self, *, seed: int, block: int, request: int = 0):

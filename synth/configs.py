@@ -36,6 +36,7 @@ class ModelConfig:
     sampler: int = 0               # 0: entropy threshold + min_accept; 1: the pages' entropy budget
     entropy_budget: float = 0.1
     stop_entropy: float = 0.005
+    temperature: float = 0.0       # 0: argmax candidates; > 0: candidates drawn from softmax(z / temperature)
 
     @property
     def qkv_rows(self) -> int:

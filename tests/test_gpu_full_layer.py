@@ -147,3 +147,25 @@ def test_public_step_matches_debug_pass(setup):
     np.testing.assert_array_equal(tok.cpu().numpy()[m], am.cpu().numpy()[m])
     t = tok.cpu().numpy()
     assert t.min() >= 0 and t.max() < CFG.vocab
+
+
+def test_lm_sample_full_vocab_sampled_rows(setup):
+    """The candidate draw at the full LM-head shape (vocab 262144 = 1024 tiles,
+    the benchmark's grid) on exact-logit inputs: sampled rows equal the
+    oracle's draw wherever the targets lie more than 3e-5 from an interval edge."""
+    import block_diffusion_moe_denoise_b200 as dgm
+    from .test_gpu_ops import _exact_lm_inputs, _oracle_draw
+    E, x = _exact_lm_inputs(CFG.vocab, CFG.d_model, CFG.canvas, 32, seed=43)
+    w = dict(setup["w"])
+    w["embed"] = E
+    h = dgm.DG(CFG, w, max_requests=1, kv_capacity=CFG.canvas)
+    tau, seed, block, step = 0.7, 1234, 1, 4
+    _, am, cand = h.op_lm_sample(x, tau, seed, block, step, 0)
+    h.sync()
+    rows = list(range(0, CFG.canvas, 8)) + [CFG.canvas - 1]
+    (c_o, margin), z = _oracle_draw(E, x, rows, CFG.norm_eps, tau, seed, block, step, 0)
+    sel = margin > 3e-5
+    assert sel.sum() >= 0.75 * len(rows), sel.sum()
+    np.testing.assert_array_equal(cand.cpu().numpy()[rows][sel], c_o[sel])
+    np.testing.assert_array_equal(am.cpu().numpy()[rows], np.argmax(z, axis=1))
+    h.close()

@@ -178,3 +178,55 @@ def test_entropy_budget_sampler_bitwise(budget_handle, case):
     if case == "converge":
         assert step == 3 and rem == 0
     budget_handle.sync()
+
+
+# ---- candidate draw at a temperature (LM-head epilogue + combine) ---------------------------
+
+def _exact_lm_inputs(V, d, T, nz_inv, seed):
+    """Inputs whose logits every summation order computes exactly: embedding rows
+    with entries in {-1/4, 0, 1/4} (nonzero with probability 1/nz_inv) and hidden
+    rows of +-1 (the final RMSNorm with unit gain maps them to +-1 after bf16
+    rounding), so z = sum of +-1/4 terms is exact in fp32 and fp64 alike."""
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+    sign = torch.randint(0, 2, (V, d), generator=g, device="cuda", dtype=torch.int8) * 2 - 1
+    keep = torch.randint(0, nz_inv, (V, d), generator=g, device="cuda", dtype=torch.int16) == 0
+    E = (sign * keep).to(torch.bfloat16) * 0.25
+    x = (torch.randint(0, 2, (T, d), generator=g, device="cuda", dtype=torch.int8) * 2 - 1).to(torch.float32)
+    return E, x
+
+
+def _oracle_draw(E, x, rows, eps, tau, seed, block, step, request):
+    """Oracle logits (fp64, in vocabulary chunks) and the oracle's candidate draw for `rows`."""
+    xn = OL.rms_norm(x[rows].cpu().double().numpy(), np.ones(x.shape[1]), eps)
+    V = E.shape[0]
+    z = np.empty((len(rows), V))
+    for v0 in range(0, V, 32768):
+        z[:, v0:v0 + 32768] = xn @ E[v0:v0 + 32768].to(torch.float32).cpu().double().numpy().T
+    u_row, u_tile = OS.candidate_uniforms(seed, block, step, np.asarray(rows), V // OS.DRAW_TILE, request)
+    return OS.draw_candidates(z, tau, u_row, u_tile), z
+
+
+def test_lm_sample_bitwise_on_exact_logits(dgmod):
+    """Drawn candidates equal the oracle's draw for every row whose targets lie
+    more than 3e-5 (relative) from an interval edge: the logits are exact on
+    both sides, so only float32 sums of the draw itself differ from fp64.  The
+    statistics and argmax equal those of the plain LM-head entry point."""
+    cfg = TINY.with_(n_layers=1, d_model=512, vocab=32768)
+    w = to_device(make_weights(cfg, seed=0))
+    E, x = _exact_lm_inputs(cfg.vocab, cfg.d_model, cfg.canvas, 8, seed=41)
+    w["embed"] = E
+    h = dgmod.DG(cfg, w, max_requests=2, kv_capacity=1024)
+    tau, seed, block, step, req = 0.7, 2**33 + 17, 2, 3, 1
+    stats, am, cand = h.op_lm_sample(x, tau, seed, block, step, req)
+    stats0, am0, _ = h.op_lm_head(x)
+    h.sync()
+    assert torch.equal(stats, stats0) and torch.equal(am, am0)
+    rows = list(range(cfg.canvas))
+    (c_o, margin), z = _oracle_draw(E, x, rows, cfg.norm_eps, tau, seed, block, step, req)
+    sel = margin > 3e-5
+    assert sel.sum() >= 0.85 * len(rows), sel.sum()
+    np.testing.assert_array_equal(cand.cpu().numpy()[sel], c_o[sel])
+    assert (cand.cpu().numpy() != am.cpu().numpy()).sum() > 20      # the draw is not the argmax
+    np.testing.assert_array_equal(am.cpu().numpy(), np.argmax(z, axis=1))
+    h.close()

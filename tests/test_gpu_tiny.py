@@ -358,3 +358,37 @@ def test_generate_free_running(model):
     print(f"free-running generation: token match {match:.3f}, first divergence at {first}")
     assert (got[:256] == ref[:256]).mean() > 0.2
     h.close()
+
+
+def test_temperature_step_draws_candidates(model):
+    """A denoising step with temperature 0.7: the accept mask and the re-noised
+    tokens equal those of the temperature-0 step (the temperature shapes the
+    draw only), accepted positions hold the drawn candidates, and the step is
+    deterministic."""
+    dgm, wd, _ = model
+
+    def run(tau):
+        h = dgm.DG(CFG.with_(temperature=tau), wd, max_requests=2, kv_capacity=1024)
+        h.prefill(1, make_tokens(CFG, 200, seed=31).cuda())
+        h.open_canvas(1, 9, 0)
+        h.denoise_step([1])
+        tok, mask, stats, am = h.get_canvas(1)
+        cand = h.debug_buffer("cand", torch.int32, (CFG.canvas,)).clone()
+        h.sync()
+        out = [t.cpu().numpy() for t in (tok, mask, stats, am, cand)]
+        h.close()
+        return out
+
+    tok0, mask0, st0, am0, _ = run(0.0)
+    tok1, mask1, st1, am1, cand1 = run(0.7)
+    tok2, _, _, _, _ = run(0.7)
+    np.testing.assert_array_equal(mask0, mask1)
+    np.testing.assert_array_equal(st0, st1)
+    acc = mask1.astype(bool)
+    assert acc.sum() >= CFG.min_accept
+    np.testing.assert_array_equal(tok1[~acc], tok0[~acc])
+    np.testing.assert_array_equal(tok1[acc], cand1[acc])
+    np.testing.assert_array_equal(tok0[acc], am0[acc])
+    assert (cand1 != am1).mean() > 0.5          # near-flat random-weight logits: the draw is rarely the argmax
+    assert np.all((cand1 >= 0) & (cand1 < CFG.vocab))
+    np.testing.assert_array_equal(tok1, tok2)

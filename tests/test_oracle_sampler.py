@@ -169,3 +169,118 @@ def test_budget_rule_convergence_and_cap():
     assert S.accept_set_budget(H2, lc, acc, am, am, 0.0, 0.005).sum() == 1
     # the step cap takes everything
     assert S.accept_set_budget(np.full(n, 9.0), lc, acc, am, None, 0.0, 0.005, force_all=True).all()
+
+
+# ---- candidate draw at a temperature ------------------------------------------------------
+
+def _brute_two_level(weights, tile, u_row, u_tile):
+    """The two-level inverse-CDF pick in exact rational arithmetic on integer weights."""
+    from fractions import Fraction
+    w = [int(v) for v in weights]
+    n_t = len(w) // tile
+    masses = [sum(w[j * tile:(j + 1) * tile]) for j in range(n_t)]
+    tgt = Fraction(u_row) * sum(masses)
+    cum, J = 0, None
+    for j, m in enumerate(masses):
+        cum += m
+        if cum >= tgt:
+            J = j
+            break
+    seg = w[J * tile:(J + 1) * tile]
+    tgt2 = Fraction(u_tile[J]) * sum(seg)
+    cum = 0
+    for i, v in enumerate(seg):
+        cum += v
+        if cum >= tgt2:
+            return J * tile + i
+    raise AssertionError("unreachable")
+
+
+def test_draw_matches_exact_rational_brute_force():
+    """Integer weights w_v = exp(z_v / tau): the fp64 draw must pick the id the exact
+    rational inverse CDF picks, for every uniform pair away from an interval edge."""
+    rng = np.random.default_rng(3)
+    tile, V = 4, 16
+    for trial in range(300):
+        w = rng.integers(1, 9, size=V)
+        w[rng.random(V) < 0.2] = rng.integers(20, 40)          # a few heavy ids
+        tau = [1.0, 0.5, 2.0][trial % 3]                        # exact in float32
+        z = tau * np.log(w.astype(np.float64))
+        u_row = S.uniform_from_word(rng.integers(0, 2**32, size=1, dtype=np.uint64))
+        u_tile = S.uniform_from_word(rng.integers(0, 2**32, size=(1, V // tile), dtype=np.uint64))
+        cand, margin = S.draw_candidates(z[None, :], tau, u_row, u_tile, tile=tile)
+        if margin[0] < 1e-9:
+            continue
+        assert cand[0] == _brute_two_level(w, tile, u_row[0], u_tile[0])
+
+
+def test_draw_frequencies_follow_the_tempered_softmax():
+    """Many independent draws of one row: the id frequencies match softmax(z / tau)
+    (chi-square over the ids with an expected count >= 5, the rest lumped)."""
+    rng = np.random.default_rng(4)
+    V, tau, n = 1024, 0.7, 30000
+    z = rng.normal(0.0, 1.5, size=V)
+    p = np.exp(z / tau - (z / tau).max())
+    p /= p.sum()
+    u_row = S.uniform_from_word(rng.integers(0, 2**32, size=n, dtype=np.uint64))
+    u_tile = S.uniform_from_word(rng.integers(0, 2**32, size=(n, V // 256), dtype=np.uint64))
+    cand, _ = S.draw_candidates(np.broadcast_to(z, (n, V)), tau, u_row, u_tile)
+    counts = np.bincount(cand, minlength=V).astype(np.float64)
+    exp_c = n * p
+    big = exp_c >= 5
+    obs = np.append(counts[big], counts[~big].sum())
+    ex = np.append(exp_c[big], exp_c[~big].sum())
+    chi2 = ((obs - ex) ** 2 / ex).sum()
+    dof = obs.size - 1
+    assert chi2 < dof + 6 * np.sqrt(2 * dof), (chi2, dof)
+    # the tile level alone: four tiles, their masses
+    tile_obs = counts.reshape(4, 256).sum(1)
+    tile_p = p.reshape(4, 256).sum(1)
+    assert np.all(np.abs(tile_obs - n * tile_p) < 5 * np.sqrt(n * tile_p * (1 - tile_p)) + 1)
+
+
+def test_draw_special_cases():
+    # a dominant logit is drawn for any uniforms; a tiny temperature gives the argmax
+    z = np.zeros((3, 512))
+    z[0, 300] = 80.0
+    z[1] = np.linspace(-1, 1, 512)
+    z[2] = np.linspace(1, -1, 512)
+    u_row = np.array([2.0 ** -24, 0.5, 1 - 2.0 ** -24])
+    u_tile = np.tile(np.array([[2.0 ** -24, 1 - 2.0 ** -24]]), (3, 1))
+    cand, _ = S.draw_candidates(z, 1.0, u_row, u_tile)
+    assert cand[0] == 300
+    cand, _ = S.draw_candidates(z, 1e-4, u_row, u_tile)
+    np.testing.assert_array_equal(cand, [300, 511, 0])
+    # u -> 0 takes the first id of positive mass, u -> 1 the last
+    flat = np.zeros((1, 512))
+    assert S.draw_candidates(flat, 0.7, np.array([2.0 ** -24]), np.array([[2.0 ** -24, 0.5]]))[0][0] == 0
+    assert S.draw_candidates(flat, 0.7, np.array([1 - 2.0 ** -24]), np.array([[0.5, 1 - 2.0 ** -24]]))[0][0] == 511
+
+
+def test_uniforms_and_their_counters():
+    w = np.array([0, 1, 511, 512, 2**31, 2**32 - 1], dtype=np.uint64)
+    u = S.uniform_from_word(w)
+    np.testing.assert_array_equal(u, [2.0 ** -24, 2.0 ** -24, 2.0 ** -24, 3 * 2.0 ** -24, 0.5 + 2.0 ** -24,
+                                      1 - 2.0 ** -24])
+    assert np.all(u.astype(np.float32).astype(np.float64) == u)      # exact in float32
+    # row uniform = word 1 of the re-noise block, tile j = word 0 at request + 256 (j + 1)
+    from oracle.philox import philox4, seed_key
+    seed, block, step, req = 0x1234_5678_9ABC, 3, 5, 2
+    u_row, u_tile = S.candidate_uniforms(seed, block, step, [0, 7, 255], 3, request=req)
+    k = seed_key(seed)
+    for i, pos in enumerate([0, 7, 255]):
+        assert u_row[i] == S.uniform_from_word(philox4((pos, step, block, req), k, 32, 10)[1])
+        for j in range(3):
+            assert u_tile[i, j] == S.uniform_from_word(philox4((pos, step, block, req + 256 * (j + 1)), k, 32, 10)[0])
+
+
+def test_sample_step_writes_candidates():
+    n, V = 30, 64
+    canvas, acc = S.init_canvas(n, seed=2, block=0, vocab=V)
+    H = np.full(n, 9.0)
+    lc = -np.arange(n, dtype=np.float64)
+    am = np.arange(n) % V
+    cand = (np.arange(n) * 7 + 3) % V
+    c2, a2, _ = S.sample_step(canvas, acc, am, H, lc, seed=2, block=0, step=1, vocab=V, entropy_thresh=1.0,
+                              min_accept=5, max_steps=12, candidates=cand)
+    np.testing.assert_array_equal(c2[a2], cand[a2])
