@@ -8,11 +8,15 @@ from synth import to_f64
 
 def oracle_weights(w: dict) -> dict:
     """float64 copies of a synth weight dict (exact upcast of bf16/fp32 values)."""
-    return {
+    out = {
         "embed": to_f64(w["embed"]),
         "final_norm": to_f64(w["final_norm"]),
         "layers": [{k: to_f64(v) for k, v in lw.items()} for lw in w["layers"]],
     }
+    for name in ("sc_gate", "sc_up", "sc_down"):
+        if name in w:
+            out[name] = to_f64(w[name])
+    return out
 
 
 def rel_l2(a, b) -> float:

@@ -154,7 +154,7 @@ def test_lm_sample_full_vocab_sampled_rows(setup):
     the benchmark's grid) on exact-logit inputs: sampled rows equal the
     oracle's draw wherever the targets lie more than 3e-5 from an interval edge."""
     import block_diffusion_moe_denoise_b200 as dgm
-    from .test_gpu_ops import _exact_lm_inputs, _oracle_draw
+    from .test_gpu_ops import _assert_argmax_lowest_tied, _exact_lm_inputs, _oracle_draw
     E, x = _exact_lm_inputs(CFG.vocab, CFG.d_model, CFG.canvas, 32, seed=43)
     w = dict(setup["w"])
     w["embed"] = E
@@ -167,5 +167,5 @@ def test_lm_sample_full_vocab_sampled_rows(setup):
     sel = margin > 3e-5
     assert sel.sum() >= 0.75 * len(rows), sel.sum()
     np.testing.assert_array_equal(cand.cpu().numpy()[rows][sel], c_o[sel])
-    np.testing.assert_array_equal(am.cpu().numpy()[rows], np.argmax(z, axis=1))
+    _assert_argmax_lowest_tied(am.cpu().numpy()[rows], z)
     h.close()

@@ -207,6 +207,15 @@ def _oracle_draw(E, x, rows, eps, tau, seed, block, step, request):
     return OS.draw_candidates(z, tau, u_row, u_tile), z
 
 
+def _assert_argmax_lowest_tied(am, z):
+    """The logits here take few distinct values (multiples of 1/4), so the maximum
+    is often shared; the kernel takes the lowest id among the ids within 1e-6 of
+    it (fp64 rounding of the oracle's sums only separates exact ties)."""
+    for r in range(z.shape[0]):
+        tied = np.nonzero(z[r] >= z[r].max() - 1e-6)[0]
+        assert am[r] == tied.min(), (r, am[r], tied[:8])
+
+
 def test_lm_sample_bitwise_on_exact_logits(dgmod):
     """Drawn candidates equal the oracle's draw for every row whose targets lie
     more than 3e-5 (relative) from an interval edge: the logits are exact on
@@ -228,5 +237,5 @@ def test_lm_sample_bitwise_on_exact_logits(dgmod):
     assert sel.sum() >= 0.85 * len(rows), sel.sum()
     np.testing.assert_array_equal(cand.cpu().numpy()[sel], c_o[sel])
     assert (cand.cpu().numpy() != am.cpu().numpy()).sum() > 20      # the draw is not the argmax
-    np.testing.assert_array_equal(am.cpu().numpy(), np.argmax(z, axis=1))
+    _assert_argmax_lowest_tied(am.cpu().numpy(), z)
     h.close()
