@@ -34,7 +34,8 @@ def config_struct(cfg) -> dg_config:
                      cfg.top_k, cfg.ffn_expert, cfg.ffn_shared, cfg.vocab, cfg.canvas, cfg.max_steps,
                      cfg.min_accept, cfg.entropy_thresh, cfg.rope_theta, cfg.norm_eps,
                      getattr(cfg, "sampler", 0), getattr(cfg, "entropy_budget", 0.1),
-                     getattr(cfg, "stop_entropy", 0.005), getattr(cfg, "temperature", 0.0))
+                     getattr(cfg, "stop_entropy", 0.005), getattr(cfg, "temperature", 0.0),
+                     getattr(cfg, "ffn_selfcond", 0), getattr(cfg, "selfcond_topk", 8))
 
 
 def philox_tokens(seed: int, block: int, step: int, request: int, pos0: int, n: int, vocab: int,
@@ -75,7 +76,8 @@ class DG:
                 "attn_norm", "w_qkv", "w_o", "ffn_norm", "w_router", "w_gate", "w_up", "w_down", "ws_gate",
                 "ws_up", "ws_down")])
         self._layers = layers
-        self.c_w = dg_weights(weights["embed"].data_ptr(), weights["final_norm"].data_ptr(), layers)
+        sc = [weights[n].data_ptr() if n in weights else None for n in ("sc_gate", "sc_up", "sc_down")]
+        self.c_w = dg_weights(weights["embed"].data_ptr(), weights["final_norm"].data_ptr(), layers, *sc)
         nbytes = lib.dg_workspace_size(C.byref(self.c_cfg), max_requests, kv_capacity)
         if nbytes == 0:
             raise DGError(-1, "dg_workspace_size")
@@ -194,9 +196,18 @@ class DG:
                                        _ptr(am), _ptr(cand)), "dg_op_lm_sample")
         return stats, am, cand
 
+    def op_selfcond(self, request: int, x: torch.Tensor):
+        """dg_op_selfcond: the self-conditioning term [T, d] of hidden rows x and the
+        top entries (p [T, 8] f32, ids [T, 8] i32; entries past selfcond_topk undefined)."""
+        T, d = x.shape
+        sc = torch.empty((T, d), dtype=torch.float32, device=x.device)
+        top = torch.empty((T, 8, 2), dtype=torch.float32, device=x.device)
+        check(self.lib.dg_op_selfcond(self.h, request, _ptr(x), T, _ptr(sc), _ptr(top)), "dg_op_selfcond")
+        return sc, top[..., 0], top.view(torch.int32)[..., 1]
+
     KERNEL_CLASSES = ("embed", "rmsnorm", "qkv", "attention", "oproj", "group",
                       "experts_gate_up", "experts_down", "shared_gate_up", "shared_down", "lm_head", "lm_combine",
-                      "sample", "other")
+                      "sample", "selfcond", "other")
 
     def profile(self, enable: int):
         check(self.lib.dg_profile(self.h, enable), "dg_profile")

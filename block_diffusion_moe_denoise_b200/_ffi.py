@@ -19,7 +19,7 @@ class dg_config(C.Structure):
                                        "min_accept")] + \
                [("entropy_thresh", C.c_float), ("rope_theta", C.c_float), ("norm_eps", C.c_float),
                 ("sampler", C.c_int), ("entropy_budget", C.c_float), ("stop_entropy", C.c_float),
-                ("temperature", C.c_float)]
+                ("temperature", C.c_float), ("ffn_selfcond", C.c_int), ("selfcond_topk", C.c_int)]
 
 
 class dg_layer_weights(C.Structure):
@@ -28,7 +28,8 @@ class dg_layer_weights(C.Structure):
 
 
 class dg_weights(C.Structure):
-    _fields_ = [("embed", C.c_void_p), ("final_norm", C.c_void_p), ("layers", C.POINTER(dg_layer_weights))]
+    _fields_ = [("embed", C.c_void_p), ("final_norm", C.c_void_p), ("layers", C.POINTER(dg_layer_weights)),
+                ("sc_gate", C.c_void_p), ("sc_up", C.c_void_p), ("sc_down", C.c_void_p)]
 
 
 class DGError(RuntimeError):
@@ -66,6 +67,7 @@ _SIGS = {
                                     C.c_void_p]),
     "dg_op_sample": (C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int]),
     "dg_op_lm_head": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p]),
+    "dg_op_selfcond": (C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p]),
     "dg_op_lm_sample": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int, C.c_float, C.c_uint64, C.c_int, C.c_int, C.c_int,
                                   C.c_void_p, C.c_void_p, C.c_void_p]),
     "dg_profile": (C.c_int, [C.c_void_p, C.c_int]),

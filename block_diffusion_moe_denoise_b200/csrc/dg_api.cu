@@ -37,6 +37,7 @@ struct ReqState {
   unsigned long long seed = 0;
   bool open = false;
   int last_slot = 0;
+  bool sc_valid = false;  // "sc_top" holds this canvas's previous-step self-conditioning state
 };
 
 // Offsets of every buffer inside the caller's workspace.
@@ -67,6 +68,8 @@ bool config_ok(const dg_config* c) {
   if (c->sampler != DG_SAMPLER_THRESHOLD && c->sampler != DG_SAMPLER_ENTROPY_BUDGET) return false;
   if (c->sampler == DG_SAMPLER_ENTROPY_BUDGET && !(c->entropy_budget >= 0.f && c->stop_entropy >= 0.f)) return false;
   if (!(c->temperature >= 0.f && c->temperature <= 1e30f)) return false;
+  if (c->ffn_selfcond < 0 || c->ffn_selfcond % 64 != 0) return false;
+  if (c->ffn_selfcond > 0 && (c->selfcond_topk < 1 || c->selfcond_topk > 8)) return false;
   return true;
 }
 
@@ -109,6 +112,12 @@ void make_plan(const dg_config* c, int max_req, long long cap_user, Plan* p) {
   p->add("argmax", (size_t)Tcap * 4);
   p->add("draw", (size_t)max_req * c->canvas * (c->vocab / 256) * 8);
   p->add("cand", (size_t)max_req * c->canvas * 4);
+  {
+    const bool sc = c->ffn_selfcond > 0;
+    p->add("sc_part", sc ? (size_t)kLmGridMax * max_req * c->canvas * 8 * 8 : 64);
+    p->add("sc_top", sc ? (size_t)max_req * c->canvas * 8 * 8 : 64);
+    p->add("hs_sc", sc ? (size_t)Tcap * c->ffn_selfcond * 2 : 64);
+  }
   p->add("canvas", (size_t)max_req * c->canvas * 4);
   p->add("commit_tok", (size_t)max_req * c->canvas * 4);
   p->add("prev_argmax", (size_t)max_req * c->canvas * 4);
@@ -198,9 +207,9 @@ struct KernelProfiler {
 
 const char* const kKernelClass[] = {"embed", "rmsnorm", "qkv", "attention", "oproj", "group",
                                     "experts_gate_up", "experts_down", "shared_gate_up", "shared_down", "lm_head",
-                                    "lm_combine", "sample", "other"};
+                                    "lm_combine", "sample", "selfcond", "other"};
 enum KClass { K_EMBED, K_RMSNORM, K_QKV, K_ATTN, K_OPROJ, K_GROUP, K_EGU, K_ED, K_SGU, K_SD, K_LM, K_LMC, K_SAMPLE,
-              K_OTHER, K_NCLASS };
+              K_SC, K_OTHER, K_NCLASS };
 static_assert(K_NCLASS <= 16, "profiler tables hold 16 classes");
 
 struct dg_handle {
@@ -221,6 +230,7 @@ struct dg_handle {
   long long kv_req_stride = 0, kv_layer_stride = 0;
   std::vector<LayerMaps> maps;
   CUtensorMap tm_hn, tm_o, tm_u, tm_xp, tm_hp, tm_hs, tm_embed, tm_k, tm_vt;
+  CUtensorMap tm_sc_gate, tm_sc_up, tm_sc_down, tm_hs_sc;  // self-conditioning MLP and its hidden rows
   long long cap_user = 0;  // capacity the caller asked for (cap is rounded up to 64)
   ReqState req[DG_MAX_REQUESTS];
   int mask_flip = 0;  // which of the two routing bitmask buffers the next layer uses
@@ -263,7 +273,8 @@ namespace {
 // One decoder pass over the slots of `s`.  With want_lm, the final norm and
 // the LM head run over the first lm_rows tokens only (lm_rows < 0: all).
 int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layers, bool qkv_only_last, bool want_lm,
-             float* logits, int lm_rows = -1, const DrawKeys* keys = nullptr, float temperature = 0.f) {
+             float* logits, int lm_rows = -1, const DrawKeys* keys = nullptr, float temperature = 0.f,
+             const SelfCondArgs* sc = nullptr) {
   const dg_config& c = h->cfg;
   const int T = s.n * s.Tr;
   const int TL = lm_rows < 0 ? T : lm_rows;
@@ -285,6 +296,42 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
   // reason as the attention key splits
   const int so = wpart_splits(d, s.Tr, c.n_q_heads * D, h->num_sms);
   const int ss = wpart_splits(d, s.Tr, c.ffn_shared, h->num_sms);
+  if (sc != nullptr) {
+    // self-conditioning: soft embeddings -> gated MLP; its split-K partials are
+    // added to the token embeddings by the first layer's norm kernel
+    SelfCondArgs ea = *sc;
+    ea.T = T;
+    ea.out = h->B<bf16>("u");
+    LAUNCH(h, K_SC, 1, run_selfcond_embed(ea, st));
+    SharedArgs ga;
+    memset(&ga, 0, sizeof(ga));
+    ga.tm_u = &h->tm_u;
+    ga.tm_gate = &h->tm_sc_gate;
+    ga.tm_up = &h->tm_sc_up;
+    ga.tm_router = nullptr;
+    ga.T = T;
+    ga.d = d;
+    ga.fs = c.ffn_selfcond;
+    ga.num_sms = h->num_sms;
+    ga.E = 0;
+    ga.hs = h->B<bf16>("hs_sc");
+    ga.err = err;
+    LAUNCH(h, K_SC, 1, run_shared_gate_up(ga, st));
+    const int sp = wpart_splits(d, s.Tr, c.ffn_selfcond, h->num_sms);
+    WpartArgs da;
+    da.tm_w = &h->tm_sc_down;
+    da.tm_x = &h->tm_hs_sc;
+    da.T = T;
+    da.Tcap = h->Tcap;
+    da.d = d;
+    da.K = c.ffn_selfcond;
+    da.splits = sp;
+    da.num_sms = h->num_sms;
+    da.part = part;
+    da.err = err;
+    LAUNCH(h, K_SC, 1, run_wpart(da, st));
+    pending_parts = sp;
+  }
   for (int l = 0; l < n_layers; ++l) {
     const dg_layer_weights& w = h->lw[l];
     const LayerMaps& m = h->maps[l];
@@ -475,16 +522,22 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     la.logits = logits;
     la.err = err;
     const bool draw = keys != nullptr && temperature > 0.f;
+    const bool keep_sc = keys != nullptr && c.ffn_selfcond > 0;  // record this step's state for the next
     la.inv_tau = draw ? 1.0f / temperature : 1.0f;
     la.draw = draw ? h->B<float2>("draw") : nullptr;
     memset(&la.keys, 0, sizeof(la.keys));
     if (draw) la.keys = *keys;
+    la.sc_part = keep_sc ? h->B<float2>("sc_part") : nullptr;
     int grid = 0;
     LAUNCH(h, K_LM, 1, run_lm_head(la, &grid, st));
     LAUNCH(h, K_LMC, 1,
            run_lm_combine(h->B<float4>("lm_part"), grid, (TL + 127) / 128, TL, h->B<float>("stats"),
                           h->B<int>("argmax"), err, st, la.draw, (int)(c.vocab / 256), draw ? keys : nullptr,
                           draw ? h->B<int>("cand") : nullptr));
+    if (keep_sc)
+      LAUNCH(h, K_SC, 1,
+             run_selfcond_topk(la.sc_part, grid, TL, h->B<float>("stats"), *keys, c.selfcond_topk,
+                               h->B<float2>("sc_top"), err, st));
   } else if (pending_k || pending_parts) {
     // a pass stopped after a full layer: fold its expert outputs into x
     LAUNCH(h, K_RMSNORM, 1,
@@ -612,6 +665,14 @@ int dg_init(const dg_config* cfg, const dg_weights* wts, int max_requests, int64
     ok = ok && make_map(&h->tm_k, h->B<bf16>("kv"), D, kv_elems / D, 64);
     ok = ok && make_map(&h->tm_vt, h->B<bf16>("kv"), h->cap, kv_elems / h->cap, D);
   }
+  if (c.ffn_selfcond > 0) {
+    const int f = c.ffn_selfcond;
+    ok = ok && wts->sc_gate && wts->sc_up && wts->sc_down;
+    ok = ok && make_map(&h->tm_sc_gate, wts->sc_gate, d, f, 32);
+    ok = ok && make_map(&h->tm_sc_up, wts->sc_up, d, f, 32);
+    ok = ok && make_map(&h->tm_sc_down, wts->sc_down, f, d, 128);
+    ok = ok && make_map(&h->tm_hs_sc, h->B<bf16>("hs_sc"), f, h->Tcap, 256);
+  }
   if (!ok) {
     delete h;
     return DG_E_ARG;
@@ -718,6 +779,7 @@ int dg_open_canvas(dg_handle* h, int req, uint64_t seed, int block) {
   r.seed = seed;
   r.block = block;
   r.step = 0;
+  r.sc_valid = false;
   return DG_OK;
 }
 
@@ -809,10 +871,34 @@ int dg_denoise_step(dg_handle* h, int n_req, const int* reqs, int32_t* d_remaini
     keys.seed[i] = r.seed;
   }
   const bool draw = h->cfg.temperature > 0.f;
-  int rc = run_pass(h, ids, s, h->cfg.n_layers, false, true, nullptr, n_req * C, draw ? &keys : nullptr,
-                    h->cfg.temperature);
+  const bool selfcond = h->cfg.ffn_selfcond > 0;
+  // self-conditioning input of the canvas slots whose request has a previous
+  // step of this canvas (slots past n_req, the commit slots, get none)
+  SelfCondArgs sca;
+  memset(&sca, 0, sizeof(sca));
+  bool any_sc = false;
+  if (selfcond) {
+    sca.canvas = C;
+    sca.d = h->cfg.d_model;
+    sca.vocab = h->cfg.vocab;
+    sca.K = h->cfg.selfcond_topk;
+    sca.n_slots = n_req;
+    sca.top = h->B<float2>("sc_top");
+    sca.embed = h->embed;
+    sca.err = h->B<int>("err");
+    for (int i = 0; i < n_req; ++i) {
+      sca.req[i] = reqs[i];
+      sca.on[i] = h->req[reqs[i]].sc_valid ? 1 : 0;
+      any_sc = any_sc || sca.on[i];
+    }
+  }
+  int rc = run_pass(h, ids, s, h->cfg.n_layers, false, true, nullptr, n_req * C,
+                    (draw || selfcond) ? &keys : nullptr, h->cfg.temperature, any_sc ? &sca : nullptr);
   if (rc != DG_OK) return rc;
-  for (int i = 0; i < n_req; ++i) h->req[reqs[i]].pending = false;
+  for (int i = 0; i < n_req; ++i) {
+    h->req[reqs[i]].pending = false;
+    h->req[reqs[i]].sc_valid = selfcond;
+  }
   float* stats = h->B<float>("stats");
   rc = sample_slots(h, n_req, reqs, stats, stats + 1, 4, h->B<int>("argmax"), steps,
                     draw ? h->B<int>("cand") : nullptr);
@@ -1055,6 +1141,86 @@ int dg_op_lm_sample(dg_handle* h, const float* d_x, int T, float temperature, ui
   CK(cudaMemcpyAsync(d_cand, h->B<int>("cand"), (size_t)T * 4, cudaMemcpyDeviceToDevice, h->st));
   if (d_stats) CK(cudaMemcpyAsync(d_stats, h->B<float>("stats"), (size_t)T * 16, cudaMemcpyDeviceToDevice, h->st));
   if (d_argmax) CK(cudaMemcpyAsync(d_argmax, h->B<int>("argmax"), (size_t)T * 4, cudaMemcpyDeviceToDevice, h->st));
+  return DG_OK;
+}
+
+int dg_op_selfcond(dg_handle* h, int request, const float* d_x, int T, float* d_sc, void* d_top) {
+  if (!h || !d_x || !d_sc || T < 1 || T > h->cfg.canvas || !req_ok(h, request)) return DG_E_ARG;
+  const dg_config& c = h->cfg;
+  if (c.ffn_selfcond <= 0) return DG_E_ARG;
+  const int d = c.d_model;
+  float* x = h->B<float>("x");
+  int* err = h->B<int>("err");
+  CK(cudaMemcpyAsync(x, d_x, (size_t)T * d * 4, cudaMemcpyDeviceToDevice, h->st));
+  CK(run_rmsnorm(x, h->final_norm, T, d, c.norm_eps, h->B<bf16>("hn"), h->st));
+  DrawKeys keys;
+  memset(&keys, 0, sizeof(keys));
+  keys.canvas = c.canvas;
+  keys.req[0] = request;
+  LmArgs la;
+  la.tm_x = &h->tm_hn;
+  la.tm_embed = &h->tm_embed;
+  la.T = T;
+  la.d = d;
+  la.num_sms = h->num_sms < kLmGridMax ? h->num_sms : kLmGridMax;
+  la.V = c.vocab;
+  la.part = h->B<float4>("lm_part");
+  la.logits = nullptr;
+  la.err = err;
+  la.sc_part = h->B<float2>("sc_part");
+  int grid = 0;
+  CK(run_lm_head(la, &grid, h->st));
+  CK(run_lm_combine(la.part, grid, (T + 127) / 128, T, h->B<float>("stats"), h->B<int>("argmax"), err, h->st));
+  float2* top = h->B<float2>("sc_top");
+  CK(run_selfcond_topk(la.sc_part, grid, T, h->B<float>("stats"), keys, c.selfcond_topk, top, err, h->st));
+  if (d_top)
+    CK(cudaMemcpyAsync(d_top, top + (size_t)request * c.canvas * 8, (size_t)T * 8 * sizeof(float2),
+                       cudaMemcpyDeviceToDevice, h->st));
+  // the pass's self-conditioning prologue on rows 0..T-1 as slot 0
+  SelfCondArgs ea;
+  memset(&ea, 0, sizeof(ea));
+  ea.canvas = c.canvas;
+  ea.T = T;
+  ea.d = d;
+  ea.vocab = c.vocab;
+  ea.K = c.selfcond_topk;
+  ea.n_slots = 1;
+  ea.req[0] = request;
+  ea.on[0] = 1;
+  ea.top = top;
+  ea.embed = h->embed;
+  ea.out = h->B<bf16>("u");
+  ea.err = err;
+  CK(run_selfcond_embed(ea, h->st));
+  SharedArgs ga;
+  memset(&ga, 0, sizeof(ga));
+  ga.tm_u = &h->tm_u;
+  ga.tm_gate = &h->tm_sc_gate;
+  ga.tm_up = &h->tm_sc_up;
+  ga.T = T;
+  ga.d = d;
+  ga.fs = c.ffn_selfcond;
+  ga.num_sms = h->num_sms;
+  ga.hs = h->B<bf16>("hs_sc");
+  ga.err = err;
+  CK(run_shared_gate_up(ga, h->st));
+  const int sp = wpart_splits(d, T, c.ffn_selfcond, h->num_sms);
+  WpartArgs da;
+  da.tm_w = &h->tm_sc_down;
+  da.tm_x = &h->tm_hs_sc;
+  da.T = T;
+  da.Tcap = h->Tcap;
+  da.d = d;
+  da.K = c.ffn_selfcond;
+  da.splits = sp;
+  da.num_sms = h->num_sms;
+  da.part = h->B<float>("part");
+  da.err = err;
+  CK(run_wpart(da, h->st));
+  // sum of the partials (fold into a zeroed residual, no norm)
+  CK(cudaMemsetAsync(x, 0, (size_t)T * d * 4, h->st));
+  CK(run_residual_norm(x, nullptr, nullptr, 0, da.part, sp, h->Tcap, nullptr, T, d, c.norm_eps, nullptr, h->st));
+  CK(cudaMemcpyAsync(d_sc, x, (size_t)T * d * 4, cudaMemcpyDeviceToDevice, h->st));
   return DG_OK;
 }
 

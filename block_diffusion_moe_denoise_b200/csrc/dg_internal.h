@@ -101,6 +101,7 @@ struct LmArgs {
   float inv_tau = 1.f;       // 1 / temperature
   float2* draw = nullptr;    // [T][V/256]: (log-mass of the tile at 1/temperature, drawn id in the tile)
   DrawKeys keys = {};
+  float2* sc_part = nullptr; // self-conditioning: per-CTA top-8 logits [grid][T][8] (logit, id bits)
 };
 
 cudaError_t run_qkv(const QkvArgs& a, cudaStream_t st);
@@ -158,6 +159,25 @@ cudaError_t run_route(const bf16* u, int d, bf16* xp, unsigned* mask, unsigned* 
 cudaError_t run_lm_combine(const float4* part, int G, int MT, int T, float* stats, int* argmax, int* err,
                            cudaStream_t st, const float2* draw = nullptr, int NV = 0, const DrawKeys* keys = nullptr,
                            int* cand = nullptr);
+// Self-conditioning state: merge the LM head's per-CTA top-8 lists (sc_part,
+// [G][T][8]) per row into the row's top-K softmax entries, written as (p, id
+// bits) to sc_top[(keys.req[slot] * keys.canvas + pos) * 8 + k], k < K.  The
+// rows' log-partitions come from `stats` (written by run_lm_combine).
+cudaError_t run_selfcond_topk(const float2* sc_part, int G, int T, const float* stats, const DrawKeys& keys, int K,
+                              float2* sc_top, int* err, cudaStream_t st);
+// Soft embeddings of the self-conditioning input: row r (slot r / canvas,
+// position r % canvas) gets sum_k p_k E[id_k] over its request's sc_top entries
+// when on[slot], else zeros; rows T..: untouched.  out: bf16 [T, d].
+struct SelfCondArgs {
+  int canvas, T, d, vocab, K, n_slots;
+  int req[DG_MAX_REQUESTS];
+  int on[DG_MAX_REQUESTS];
+  const float2* top;      // [max_req][canvas][8]
+  const bf16* embed;      // [vocab, d]
+  bf16* out;              // [T, d]
+  int* err;
+};
+cudaError_t run_selfcond_embed(const SelfCondArgs& a, cudaStream_t st);
 struct SampleArgs {
   int n_slots, canvas, vocab, min_accept, max_steps;
   float thr;

@@ -424,20 +424,23 @@ struct P_SGU : ProblemBase {
     tma_prefetch_desc(&p.tmX);
     tma_prefetch_desc(&p.tmG);
     tma_prefetch_desc(&p.tmU);
-    tma_prefetch_desc(&p.tmR);
+    if (p.E > 0) tma_prefetch_desc(&p.tmR);
   }
-  DG_DEVINL static int num_tiles(const Params& p) { return p.MT * (p.FJ + 1); }
+  // E == 0: a plain gated MLP (no router tile), as used for self-conditioning
+  DG_DEVINL static int router_tiles(const Params& p) { return p.E > 0 ? p.MT : 0; }
+  DG_DEVINL static int num_tiles(const Params& p) { return router_tiles(p) + p.MT * p.FJ; }
   DG_DEVINL static Tile tile(const Params& p, int v) {
     Tile t;
     t.valid = 1;
     t.nk = p.nk;
-    if (v < p.MT) {
+    const int R = router_tiles(p);
+    if (v < R) {
       t.a = v;
       t.b = -1;  // router tile
       t.n_mma = p.E;
     } else {
-      t.a = (v - p.MT) % p.MT;
-      t.b = (v - p.MT) / p.MT;
+      t.a = (v - R) % p.MT;
+      t.b = (v - R) / p.MT;
       t.n_mma = 2 * kHid;
     }
     return t;
@@ -551,16 +554,41 @@ struct P_SGU : ProblemBase {
 // w_v = exp(z_v/tau - max/tau), picks the first id whose running sum reaches
 // u * sum (u from Philox, keyed by the row's slot), and stores the tile's
 // log-mass max/tau + ln(sum) with that id.  k_lm_combine picks the tile.
+//
+// Self-conditioning (sc_part != nullptr): each thread also keeps its row's
+// SC_K largest logits (ties to the lower id) over the CTA's tiles in shared
+// memory; the grid is a multiple of MT so that a CTA only sees one token tile
+// (mt = blockIdx.x % MT).  The CTA's lists go to sc_part and are merged by
+// k_lm_combine.
 // ---------------------------------------------------------------------------
 struct LmStat {
   float m, s, t;
   int a;
 };
 
+// Sorted insertion into a descending top-8 list.  Values arrive in ascending
+// id order, so the strict comparisons keep the lower id ahead of an equal one.
+DG_DEVINL void top8_insert(float (&tv)[8], int (&ti)[8], float v, int id) {
+  if (v > tv[7]) {
+    bool gt[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) gt[r] = v > tv[r];
+#pragma unroll
+    for (int r = 7; r > 0; --r) {
+      tv[r] = gt[r] ? (gt[r - 1] ? tv[r - 1] : v) : tv[r];
+      ti[r] = gt[r] ? (gt[r - 1] ? ti[r - 1] : id) : ti[r];
+    }
+    tv[0] = gt[0] ? v : tv[0];
+    ti[0] = gt[0] ? id : ti[0];
+  }
+}
+
 struct P_LM : ProblemBase {
   static constexpr int BN = 256, STAGES = 4, B_STAGE = BN * 128, TMEM_COLS = 512;
   static constexpr int MT_MAX = 8;
-  static constexpr int EP_SMEM = MT_MAX * 128 * (int)sizeof(LmStat);
+  static constexpr int SC_K = 8;
+  static constexpr int STAT_SMEM = MT_MAX * 128 * (int)sizeof(LmStat);
+  static constexpr int EP_SMEM = STAT_SMEM + 128 * SC_K * 8;
   struct Params {
     CUtensorMap tmX;  // final-normed tokens [Tcap, d]
     CUtensorMap tmE;  // embedding [V, d]
@@ -572,6 +600,7 @@ struct P_LM : ProblemBase {
     float inv_tau;
     float2* draw;    // optional [T][NV]
     DrawKeys keys;
+    float2* sc_part; // optional [gridDim.x][T][SC_K] (logit, id as int bits)
   };
   DG_DEVINL static void prefetch(const Params& p) {
     tma_prefetch_desc(&p.tmX);
@@ -641,9 +670,16 @@ struct P_LM : ProblemBase {
     load_x(p, t, kb, sa, sb, bar);
     load_w(p, t, kb, sa, sb, bar);
   }
+  DG_DEVINL static float2* sc_list(uint8_t* ep, int row) {
+    return reinterpret_cast<float2*>(ep + STAT_SMEM) + row * SC_K;
+  }
   DG_DEVINL static void epilogue_init(const Params& p, int row, uint8_t* ep) {
     LmStat* st = reinterpret_cast<LmStat*>(ep);
     for (int mt = 0; mt < p.MT; ++mt) st[mt * 128 + row] = LmStat{-INFINITY, 0.f, 0.f, 0x7fffffff};
+    if (p.sc_part != nullptr) {
+      float2* l = sc_list(ep, row);
+      for (int r = 0; r < SC_K; ++r) l[r] = make_float2(-INFINITY, __int_as_float(0x7fffffff));
+    }
   }
   DG_DEVINL static void epilogue(const Params& p, const Tile& t, uint32_t taddr, int, int, int row, uint8_t* ep) {
     LmStat* st = reinterpret_cast<LmStat*>(ep);
@@ -653,10 +689,25 @@ struct P_LM : ProblemBase {
     constexpr float kLog2e = 1.4426950408889634f;
     float tm = -INFINITY;  // this tile's max logit and its column
     int ta = 0;
+    const bool sc = p.sc_part != nullptr;
+    float tv[SC_K];
+    int ti[SC_K];
+    if (sc) {
+      const float2* l = sc_list(ep, row);
+#pragma unroll
+      for (int r = 0; r < SC_K; ++r) {
+        tv[r] = l[r].x;
+        ti[r] = __float_as_int(l[r].y);
+      }
+    }
     for (int c0 = 0; c0 < 256; c0 += 32) {
       float z[32];
       tmem_ld16(taddr + c0, z);
       tmem_ld16(taddr + c0 + 16, z + 16);
+      if (sc) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) top8_insert(tv, ti, z[i], t.b * 256 + c0 + i);
+      }
       if (p.logits != nullptr && ok) {
         float* dst = p.logits + (size_t)tok * p.V + (size_t)t.b * 256 + c0;
 #pragma unroll
@@ -692,6 +743,11 @@ struct P_LM : ProblemBase {
       }
     }
     st[t.a * 128 + row] = r;
+    if (sc) {
+      float2* l = sc_list(ep, row);
+#pragma unroll
+      for (int r2 = 0; r2 < SC_K; ++r2) l[r2] = make_float2(tv[r2], __int_as_float(ti[r2]));
+    }
     if (p.draw != nullptr) draw_tile(p, t, taddr, tok, ok, tm, ta);
   }
   DG_DEVINL static void finish(const Params& p, int row, uint8_t* ep) {
@@ -699,6 +755,14 @@ struct P_LM : ProblemBase {
     for (int mt = 0; mt < p.MT; ++mt) {
       const LmStat r = st[mt * 128 + row];
       p.part[((size_t)blockIdx.x * p.MT + mt) * 128 + row] = make_float4(r.m, r.s, r.t, __int_as_float(r.a));
+    }
+    if (p.sc_part != nullptr) {
+      const int tok = (blockIdx.x % p.MT) * 128 + row;
+      if (tok < p.T) {
+        const float2* l = sc_list(ep, row);
+        float2* dst = p.sc_part + ((size_t)blockIdx.x * p.T + tok) * SC_K;
+        for (int r = 0; r < SC_K; ++r) dst[r] = l[r];
+      }
     }
   }
 };
@@ -751,7 +815,10 @@ int wpart_splits(int d, int T, int K, int num_sms) {
   const int nk = K / 64;
   if (s > nk) s = nk;
   if (s > kMaxPartSplits) s = kMaxPartSplits;
-  return s < 1 ? 1 : s;
+  if (s < 1) return 1;
+  // every split must own at least one k-block (an empty split writes no partial)
+  const int per = (nk + s - 1) / s;
+  return (nk + per - 1) / per;
 }
 
 cudaError_t run_wpart(const WpartArgs& a, cudaStream_t st) {
@@ -803,12 +870,14 @@ cudaError_t run_experts_down(const ExpertArgs& a, cudaStream_t st) {
 }
 
 cudaError_t run_shared_gate_up(const SharedArgs& a, cudaStream_t st) {
-  if (a.E < 16 || a.E > P_SGU::BN || a.E % 16 != 0 || a.k < 1 || a.k > 8) return cudaErrorInvalidValue;
+  if (a.E != 0 && (a.E < 16 || a.E > P_SGU::BN || a.E % 16 != 0 || a.k < 1 || a.k > 8 || a.tm_router == nullptr))
+    return cudaErrorInvalidValue;
+  if (a.fs % P_SGU::kHid != 0) return cudaErrorInvalidValue;
   P_SGU::Params g;
   g.tmX = *a.tm_u;
   g.tmG = *a.tm_gate;
   g.tmU = *a.tm_up;
-  g.tmR = *a.tm_router;
+  g.tmR = a.E > 0 ? *a.tm_router : *a.tm_gate;  // unused without a router
   g.T = a.T;
   g.nk = a.d / 64;
   g.MT = (a.T + 127) / 128;
@@ -823,7 +892,7 @@ cudaError_t run_shared_gate_up(const SharedArgs& a, cudaStream_t st) {
   g.w = a.w;
   g.mask = a.mask;
   g.err = a.err;
-  return launch_gemm<P_SGU>(g, grid_for(g.MT * (g.FJ + 1), a.num_sms), st);
+  return launch_gemm<P_SGU>(g, grid_for(g.MT * (g.FJ + (a.E > 0 ? 1 : 0)), a.num_sms), st);
 }
 
 cudaError_t run_lm_head(const LmArgs& a, int* grid_out, cudaStream_t st) {
@@ -841,10 +910,13 @@ cudaError_t run_lm_head(const LmArgs& a, int* grid_out, cudaStream_t st) {
   p.inv_tau = a.inv_tau;
   p.draw = a.draw;
   p.keys = a.keys;
+  p.sc_part = a.sc_part;
   if (p.MT > P_LM::MT_MAX) return cudaErrorInvalidValue;
   if (p.draw != nullptr && (p.keys.canvas < 1 || (p.T + p.keys.canvas - 1) / p.keys.canvas > DG_MAX_REQUESTS))
     return cudaErrorInvalidValue;
-  const int grid = grid_for(p.MT * p.NV, a.num_sms);
+  int grid = grid_for(p.MT * p.NV, a.num_sms);
+  if (p.sc_part != nullptr) grid = grid / p.MT * p.MT;  // one token tile per CTA
+  if (grid < 1) return cudaErrorInvalidValue;
   *grid_out = grid;
   return launch_gemm<P_LM>(p, grid, st);
 }

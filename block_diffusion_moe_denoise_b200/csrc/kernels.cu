@@ -636,6 +636,146 @@ cudaError_t run_lm_combine(const float4* part, int G, int MT, int T, float* stat
 }
 
 // ---------------------------------------------------------------------------
+// Self-conditioning.  k_selfcond_topk: one warp per LM-head row merges the
+// per-CTA top-8 logit lists (lane l takes CTAs l, l+32, ...; then K rounds of
+// a warp-wide max, ties to the lower id) and stores the K largest softmax
+// entries p = exp(z - logZ) with their ids in the row's request slot.
+// k_selfcond_embed: one CTA per pass row, 8 columns per thread, accumulates
+// sum_k p_k E[id_k] in fp32 (k ascending) and stores bf16.
+// ---------------------------------------------------------------------------
+DG_DEVINL void sc_insert(float (&tv)[8], int (&ti)[8], float v, int id) {
+  // list sorted by (value descending, id ascending); gt[r]: the new entry goes before entry r
+  bool gt[8];
+#pragma unroll
+  for (int r = 0; r < 8; ++r) gt[r] = v > tv[r] || (v == tv[r] && id < ti[r]);
+  if (!gt[7]) return;
+#pragma unroll
+  for (int r = 7; r > 0; --r) {
+    tv[r] = gt[r] ? (gt[r - 1] ? tv[r - 1] : v) : tv[r];
+    ti[r] = gt[r] ? (gt[r - 1] ? ti[r - 1] : id) : ti[r];
+  }
+  tv[0] = gt[0] ? v : tv[0];
+  ti[0] = gt[0] ? id : ti[0];
+}
+
+__global__ void k_selfcond_topk(const float2* __restrict__ sc_part, int G, int T, const float* __restrict__ stats,
+                                DrawKeys keys, int K, float2* sc_top, int* err) {
+  pdl_trigger();
+  pdl_wait();
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+  float tv[8];
+  int ti[8];
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    tv[r] = -INFINITY;
+    ti[r] = 0x7fffffff;
+  }
+  for (int c = lane; c < G; c += 32) {
+    const float2* l = sc_part + ((size_t)c * T + t) * 8;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const float2 e = l[r];
+      sc_insert(tv, ti, e.x, __float_as_int(e.y));
+    }
+  }
+  const float4 st = reinterpret_cast<const float4*>(stats)[t];  // (entropy, logconf, max, logZ)
+  const float logZ = st.w;
+  const int slot = t / keys.canvas, pos = t - slot * keys.canvas;
+  float2* out = sc_top + ((size_t)keys.req[slot] * keys.canvas + pos) * 8;
+  for (int k = 0; k < K; ++k) {
+    float bv = tv[0];
+    int bi = ti[0];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ov > bv || (ov == bv && oi < bi)) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    if (tv[0] == bv && ti[0] == bi) {  // this lane held it: pop
+#pragma unroll
+      for (int r = 0; r < 7; ++r) {
+        tv[r] = tv[r + 1];
+        ti[r] = ti[r + 1];
+      }
+      tv[7] = -INFINITY;
+      ti[7] = 0x7fffffff;
+    }
+    if (lane == 0) {
+      const float pk = expf(bv - logZ);
+      if (bi < 0 || bi == 0x7fffffff || pk != pk) atomicOr(err, DG_DEVERR_NAN);
+      out[k] = make_float2(pk, __int_as_float(bi));
+    }
+  }
+}
+
+cudaError_t run_selfcond_topk(const float2* sc_part, int G, int T, const float* stats, const DrawKeys& keys, int K,
+                              float2* sc_top, int* err, cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+  if (K < 1 || K > 8 || keys.canvas < 1 || (T + keys.canvas - 1) / keys.canvas > DG_MAX_REQUESTS)
+    return cudaErrorInvalidValue;
+  {
+    const cudaError_t e_ = launch_pdl(k_selfcond_topk, dim3((T + 7) / 8), dim3(256), 0, st, sc_part, G, T, stats,
+                                      keys, K, sc_top, err);
+    if (e_ != cudaSuccess) return e_;
+  }
+  return cudaGetLastError();
+}
+
+__global__ void k_selfcond_embed(const __grid_constant__ SelfCondArgs a) {
+  pdl_trigger();
+  pdl_wait();
+  const int r = blockIdx.x;
+  const int slot = r / a.canvas, pos = r - slot * a.canvas;
+  const bool on = slot < a.n_slots && a.on[slot];
+  const float2* top = on ? a.top + ((size_t)a.req[slot] * a.canvas + pos) * 8 : nullptr;
+  for (int c = threadIdx.x; c < a.d / 8; c += blockDim.x) {
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    if (on) {
+      for (int k = 0; k < a.K; ++k) {
+        const float2 e = top[k];
+        const int id = __float_as_int(e.y);
+        if (id < 0 || id >= a.vocab) {
+          if (c == threadIdx.x) atomicOr(a.err, DG_DEVERR_TOKEN);
+          continue;
+        }
+        const uint4 v = *reinterpret_cast<const uint4*>(a.embed + (size_t)id * a.d + c * 8);
+        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = __bfloat1622float2(b2[i]);
+          acc[2 * i] = fmaf(e.x, f.x, acc[2 * i]);
+          acc[2 * i + 1] = fmaf(e.x, f.y, acc[2 * i + 1]);
+        }
+      }
+    }
+    uint4 o;
+    o.x = pack_bf16x2(acc[0], acc[1]);
+    o.y = pack_bf16x2(acc[2], acc[3]);
+    o.z = pack_bf16x2(acc[4], acc[5]);
+    o.w = pack_bf16x2(acc[6], acc[7]);
+    *reinterpret_cast<uint4*>(a.out + (size_t)r * a.d + c * 8) = o;
+  }
+}
+
+cudaError_t run_selfcond_embed(const SelfCondArgs& a, cudaStream_t st) {
+  if (a.T == 0) return cudaSuccess;
+  if (a.d % 8 != 0 || a.K < 1 || a.K > 8 || a.canvas < 1 || a.n_slots > DG_MAX_REQUESTS) return cudaErrorInvalidValue;
+  const int threads = a.d / 8 < 512 ? (a.d / 8 + 31) / 32 * 32 : 512;
+  {
+    const cudaError_t e_ = launch_pdl(k_selfcond_embed, dim3(a.T), dim3(threads), 0, st, a);
+    if (e_ != cudaSuccess) return e_;
+  }
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
 // Re-noise token: word 0 of Philox-4x32-10 (common.cuh) at counter
 // (position, step, block, request), key = seed, mapped to [0, vocab) by
 // multiply-shift.

@@ -75,7 +75,21 @@ typedef struct dg_config {
   float entropy_budget;/* budget rule: nats of entropy accepted per step (0.1) */
   float stop_entropy;  /* budget rule: converged below this mean entropy (0.005) */
   float temperature;   /* 0: candidates are the argmax; > 0: drawn from softmax(logits / temperature) */
+  int ffn_selfcond;    /* self-conditioning gated-MLP width, a multiple of 64 (0: no self-conditioning) */
+  int selfcond_topk;   /* softmax entries per position fed back, 1..8 (8) */
 } dg_config;
+
+/* Self-conditioning (pages: "DiffusionGemma hits ~1,500 TPS", "How the sampler
+ * actually works": the previous step's softmax is fed back through a small
+ * gated MLP; its shape is not published, so this reading is the library's).
+ * At every denoising step after the first of a canvas, each canvas position
+ * adds to its token embedding
+ *   sc = sc_down (silu(sc_gate e) * (sc_up e)),  e = sum_k p_k E[id_k],
+ * where (p_k, id_k) are the selfcond_topk largest entries (ties to the lower
+ * id) of the softmax of that position's logits at the request's previous
+ * denoising step (not renormalised) and E is the tied embedding.  The first
+ * step of a canvas (after dg_open_canvas), prefill and commit passes have no
+ * such term.  dg_set_canvas keeps the request's previous-step state. */
 
 /* Sampler rules.  DG_SAMPLER_ENTROPY_BUDGET follows the pages' default sampler
  * ("DiffusionGemma hits ~1,500 TPS", "How the sampler actually works"): the
@@ -118,6 +132,9 @@ typedef struct dg_weights {
   const void* embed;
   const void* final_norm;
   const dg_layer_weights* layers;
+  /* self-conditioning MLP (NULL unless ffn_selfcond > 0): sc_gate, sc_up
+   * [ffn_selfcond, d], sc_down [d, ffn_selfcond], bf16, 16-byte aligned */
+  const void *sc_gate, *sc_up, *sc_down;
 } dg_weights;
 
 typedef struct dg_handle dg_handle;

@@ -54,6 +54,15 @@ int dg_op_lm_head(dg_handle* h, const float* d_x, int T, float* d_stats, int32_t
 int dg_op_lm_sample(dg_handle* h, const float* d_x, int T, float temperature, uint64_t seed, int block, int step,
                     int request, float* d_stats, int32_t* d_argmax, int32_t* d_cand);
 
+/* The self-conditioning term of dg.h from given fp32 hidden rows d_x [T, d]
+ * (T <= canvas) of a previous step: final RMSNorm + tied LM head, the
+ * selfcond_topk largest softmax entries per row, the soft embeddings and the
+ * gated MLP.  d_sc [T, d] f32 receives the term; d_top (may be NULL) receives
+ * [T][8] pairs of 32-bit words (p as f32, id as int32), entries k >=
+ * selfcond_topk undefined.  Uses and overwrites request `request`'s
+ * self-conditioning state.  DG_E_ARG without self-conditioning. */
+int dg_op_selfcond(dg_handle* h, int request, const float* d_x, int T, float* d_sc, void* d_top);
+
 /* Run the decoder over `T` tokens (device ids) of request `req` at positions
  * [L, L+T) without advancing L, stopping after `n_layers` layers (the K/V of
  * those layers are written to the cache slots).  The intermediates of the last
@@ -68,6 +77,7 @@ int dg_debug_forward(dg_handle* h, int req, const int32_t* d_tokens, int T, int 
  * "pair_row" i32 [T*k]; "row_pair" i32 [T*k]; "hp" bf16 [T*k, fe];
  * "yp" f32 [T*k, d]; "hs" bf16 [T, fs]; "stats" f32 [Tcap][4];
  * "argmax" i32 [Tcap]; "cand" i32 [max_req * canvas] drawn candidates;
+ * "sc_top" f32/i32 pairs [max_req][canvas][8] self-conditioning state;
  * "canvas" i32 [max_req, canvas]; "mask" u8 [...];
  * "remaining" i32 [max_req]; "route_stats" u64 [2] = (sum over router launches
  * of the number of experts that received a token, number of launches).
@@ -79,7 +89,8 @@ int dg_debug_buffer(const dg_handle* h, const char* name, size_t* offset, size_t
  * totals.  dg_profile_read (synchronising) returns the summed elapsed ms and
  * launch count of one class: "embed", "rmsnorm", "qkv", "attention", "oproj",
  * "group", "experts_gate_up", "experts_down", "shared_gate_up" (with the
- * router), "shared_down", "lm_head", "lm_combine", "sample", "other". */
+ * router), "shared_down", "lm_head", "lm_combine", "sample", "selfcond",
+ * "other". */
 int dg_profile(dg_handle* h, int enable);
 int dg_profile_read(dg_handle* h, const char* kernel, double* total_ms, int64_t* launches);
 

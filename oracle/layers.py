@@ -135,3 +135,33 @@ def lm_head_stats(xn: np.ndarray, E_tok: np.ndarray):
     H = -(p * logp).sum(axis=-1)
     logconf = m - logZ
     return dict(argmax=a.astype(np.int64), max=m, logZ=logZ, entropy=H, logconf=logconf, logits=z)
+
+
+def topk_probs(z: np.ndarray, k: int):
+    """Per row, the k largest entries of softmax(z) (ties to the lower id) and their ids.
+    Returns (p [T, k], ids [T, k]) in descending probability order."""
+    z = np.asarray(z, dtype=np.float64)
+    m = z.max(axis=-1, keepdims=True)
+    e = np.exp(z - m)
+    p = e / e.sum(axis=-1, keepdims=True)
+    order = np.argsort(-z, axis=-1, kind="stable")[:, :k]     # stable: equal logits keep id order
+    return np.take_along_axis(p, order, axis=-1), order.astype(np.int64)
+
+
+def soft_embedding(p: np.ndarray, ids: np.ndarray, E_tok: np.ndarray) -> np.ndarray:
+    """sum_k p[t, k] E[ids[t, k]] per row: the embedding expected under the given
+    (truncated) distribution."""
+    return np.einsum("tk,tkd->td", p, E_tok[ids])
+
+
+def self_condition(z_prev: np.ndarray, E_tok: np.ndarray, wg: np.ndarray, wu: np.ndarray, wd: np.ndarray,
+                   k: int) -> np.ndarray:
+    """Self-conditioning term added to the canvas embeddings ([P2] "How the sampler
+    actually works": the previous step's softmax goes back through a small gated
+    MLP).  Reading (the pages give no shape): the previous step's softmax at each
+    position, truncated to its k largest entries (not renormalised), is turned
+    into the expected embedding under it, and a gated MLP of the shared expert's
+    form maps that to the residual stream."""
+    p, ids = topk_probs(z_prev, k)
+    return swiglu(soft_embedding(p, ids, E_tok), wg, wu, wd)
+

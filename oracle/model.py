@@ -21,7 +21,11 @@ Readings where the pages are silent:
     first prompt token (the last one may be shorter): each segment attends to
     everything before it and bidirectionally to itself, so commit(C) and
     prefill(C) produce identical caches;
-  * embedding rows are used unscaled; the LM head is tied to the embedding.
+  * embedding rows are used unscaled; the LM head is tied to the embedding;
+  * self-conditioning (when the model has it) adds a term computed from the
+    previous denoising step's logits of the same canvas to the canvas token
+    embeddings (see layers.self_condition); a canvas's first step has none,
+    and prefill and commit passes never have it.
 """
 from __future__ import annotations
 
@@ -53,6 +57,7 @@ class Oracle:
         `layers`: a list of per-layer dicts, or a callable l -> dict (names as in
         synth.weights)."""
         self.cfg = cfg
+        self._weights = weights
         self.embed = weights["embed"]
         self.final_norm = weights["final_norm"]
         self._layers = weights["layers"]
@@ -69,9 +74,10 @@ class Oracle:
 
     # ---- one pass over a segment -------------------------------------------------
     def forward(self, tokens, cache: Cache, want_stats: bool = True, trace: Trace | None = None,
-                n_layers: int | None = None):
+                n_layers: int | None = None, sc=None):
         """Run the decoder over `tokens` at positions [L, L+T), writing their K/V to
-        the cache slots [L, L+T).  Returns LM-head statistics (or None)."""
+        the cache slots [L, L+T).  `sc` ([T, d]) is added to the token embeddings
+        (self-conditioning).  Returns LM-head statistics (or None)."""
         c = self.cfg
         tokens = np.asarray(tokens, dtype=np.int64)
         T = tokens.shape[0]
@@ -79,6 +85,8 @@ class Oracle:
         Hq, Hkv, D = c.n_q_heads, c.n_kv_heads, c.head_dim
         pos = L + np.arange(T)
         x = self.embed[tokens].astype(np.float64)
+        if sc is not None:
+            x = x + sc
         for l in range(c.n_layers if n_layers is None else n_layers):
             w = self.layer(l)
             rec = {"x_in": x.copy()} if trace is not None else None
@@ -128,14 +136,24 @@ class Oracle:
         self.forward(canvas, cache, want_stats=False)
         cache.length += canvas.shape[0]
 
+    def self_condition(self, prev_logits):
+        """Self-conditioning term from the previous step's logits (None at a canvas's
+        first step, or when the model has none)."""
+        c = self.cfg
+        if prev_logits is None or getattr(c, "ffn_selfcond", 0) <= 0:
+            return None
+        w = self._weights
+        return L_.self_condition(prev_logits, self.embed, w["sc_gate"], w["sc_up"], w["sc_down"], c.selfcond_topk)
+
     def denoise_step(self, cache: Cache, canvas, accepted, *, seed: int, block: int, step: int,
-                     request: int = 0, stats=None, prev_argmax=None):
+                     request: int = 0, stats=None, prev_argmax=None, prev_logits=None):
         """One step: pass over the canvas (unless `stats` is given), then the sampler
         (the configuration's rule; `prev_argmax` = the previous step's argmax, for
-        the entropy-budget rule).  Returns (canvas, accepted, remaining, stats)."""
+        the entropy-budget rule; `prev_logits` = the previous step's logits, for
+        self-conditioning).  Returns (canvas, accepted, remaining, stats)."""
         c = self.cfg
         if stats is None:
-            stats = self.forward(canvas, cache, want_stats=True)
+            stats = self.forward(canvas, cache, want_stats=True, sc=self.self_condition(prev_logits))
         cand = None
         tau = getattr(c, "temperature", 0.0)
         if tau > 0:
@@ -167,12 +185,14 @@ class Oracle:
         for b in range(n_out // c.canvas):
             canvas, accepted = self.open_canvas(seed=seed, block=b, request=request)
             s = 0
-            prev = None
+            prev = prev_logits = None
             while True:
                 s += 1
                 canvas, accepted, rem, st = self.denoise_step(cache, canvas, accepted, seed=seed, block=b,
-                                                              step=s, request=request, prev_argmax=prev)
+                                                              step=s, request=request, prev_argmax=prev,
+                                                              prev_logits=prev_logits)
                 prev = st["argmax"]
+                prev_logits = st["logits"]
                 if rem == 0:
                     break
             steps.append(s)

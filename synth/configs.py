@@ -37,6 +37,8 @@ class ModelConfig:
     entropy_budget: float = 0.1
     stop_entropy: float = 0.005
     temperature: float = 0.0       # 0: argmax candidates; > 0: candidates drawn from softmax(z / temperature)
+    ffn_selfcond: int = 0          # self-conditioning gated-MLP width (0: off)
+    selfcond_topk: int = 8         # softmax entries of the previous step fed back per position
 
     @property
     def qkv_rows(self) -> int:

@@ -21,6 +21,10 @@ Weight layout (row-major, "out x in" like a linear layer):
     ws_gate   [f_s, d]
     ws_up     [f_s, d]
     ws_down   [d, f_s]
+  self-conditioning (when ffn_selfcond > 0):
+    sc_gate   [f_sc, d]
+    sc_up     [f_sc, d]
+    sc_down   [d, f_sc]
 """
 from __future__ import annotations
 
@@ -32,6 +36,7 @@ _TENSOR_IDS = {
     "embed": 1, "final_norm": 2, "attn_norm": 3, "w_qkv": 4, "w_o": 5, "ffn_norm": 6,
     "w_router": 7, "w_gate": 8, "w_up": 9, "w_down": 10, "ws_gate": 11, "ws_up": 12,
     "ws_down": 13, "kv_k": 14, "kv_v": 15, "prompt": 16, "canvas": 17,
+    "sc_gate": 18, "sc_up": 19, "sc_down": 20,
 }
 
 LAYER_TENSORS = ("attn_norm", "w_qkv", "w_o", "ffn_norm", "w_router", "w_gate", "w_up",
@@ -91,11 +96,21 @@ def make_layer(cfg: ModelConfig, layer: int, seed: int = 0, device="cpu", std=0.
 
 def make_weights(cfg: ModelConfig, seed: int = 0, device="cpu", std=0.02, gain_std=0.0) -> dict:
     """All weights of the model as bf16 tensors (fp32 norm gains) on `device`."""
-    return {
+    w = {
         "embed": _normal_bf16((cfg.vocab, cfg.d_model), tensor_seed(seed, -1, "embed"), device, std),
         "final_norm": _gain((cfg.d_model,), tensor_seed(seed, -1, "final_norm"), device, gain_std),
         "layers": [make_layer(cfg, l, seed, device, std, gain_std) for l in range(cfg.n_layers)],
     }
+    if getattr(cfg, "ffn_selfcond", 0) > 0:
+        w.update(make_selfcond(cfg, seed, device, std))
+    return w
+
+
+def make_selfcond(cfg: ModelConfig, seed: int = 0, device="cpu", std=0.02) -> dict:
+    """The self-conditioning MLP's weights (sc_gate, sc_up, sc_down) as bf16 tensors."""
+    f, d = cfg.ffn_selfcond, cfg.d_model
+    return {name: _normal_bf16(shape, tensor_seed(seed, -1, name), device, std)
+            for name, shape in (("sc_gate", (f, d)), ("sc_up", (f, d)), ("sc_down", (d, f)))}
 
 
 def make_kv_prefix(cfg: ModelConfig, n_pos: int, seed: int = 1, device="cpu", layer: int = 0):

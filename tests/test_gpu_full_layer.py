@@ -169,3 +169,27 @@ def test_lm_sample_full_vocab_sampled_rows(setup):
     np.testing.assert_array_equal(cand.cpu().numpy()[rows][sel], c_o[sel])
     _assert_argmax_lowest_tied(am.cpu().numpy()[rows], z)
     h.close()
+
+
+def test_selfcond_op_full_vocab_sampled_rows(setup):
+    """The self-conditioning term at the full LM-head shape (vocab 262144, the
+    benchmark's grid; MLP width 1024) on exact-logit inputs, sampled rows."""
+    import block_diffusion_moe_denoise_b200 as dgm
+    from synth import make_selfcond
+    from .gpu_common import REL_L2, rel_l2
+    from .test_gpu_ops import _exact_lm_inputs, _exact_z, _oracle_selfcond
+    cfg = CFG.with_(ffn_selfcond=1024, selfcond_topk=8)
+    E, x = _exact_lm_inputs(cfg.vocab, cfg.d_model, cfg.canvas, 32, seed=53)
+    w = dict(setup["w"])
+    w["embed"] = E
+    w.update(make_selfcond(cfg, seed=5, device="cuda"))
+    h = dgm.DG(cfg, w, max_requests=1, kv_capacity=cfg.canvas)
+    sc, p, ids = h.op_selfcond(0, x)
+    h.sync()
+    rows = list(range(0, cfg.canvas, 16)) + [cfg.canvas - 1]
+    z = _exact_z(E, x, rows, cfg.norm_eps)
+    p_o, ids_o, sc_o = _oracle_selfcond(z, E, w, cfg.selfcond_topk)
+    np.testing.assert_array_equal(ids.cpu().numpy()[rows], ids_o)
+    np.testing.assert_allclose(p.cpu().numpy()[rows], p_o, rtol=1e-4)
+    assert rel_l2(sc.cpu().double().numpy()[rows], sc_o) < REL_L2
+    h.close()

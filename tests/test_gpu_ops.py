@@ -239,3 +239,56 @@ def test_lm_sample_bitwise_on_exact_logits(dgmod):
     assert (cand.cpu().numpy() != am.cpu().numpy()).sum() > 20      # the draw is not the argmax
     _assert_argmax_lowest_tied(am.cpu().numpy(), z)
     h.close()
+
+
+# ---- self-conditioning term -------------------------------------------------------------------
+
+def _exact_z(E, x, rows, eps):
+    """Oracle logits of the exact-logit inputs with their ties intact: the normed
+    rows are +-m (one magnitude m), so z = m/4 * (signs @ 4E^T), an integer
+    matrix product that fp64 computes exactly in any summation order."""
+    xn = OL.rms_norm(x[rows].cpu().double().numpy(), np.ones(x.shape[1]), eps)
+    m = np.abs(xn[0, 0])
+    assert np.all(np.abs(xn) == m)
+    V = E.shape[0]
+    z = np.empty((len(rows), V))
+    for v0 in range(0, V, 32768):
+        E4 = (E[v0:v0 + 32768].to(torch.float32) * 4).cpu().double().numpy()
+        z[:, v0:v0 + 32768] = np.sign(xn) @ E4.T
+    return z * (m / 4)
+
+
+def _oracle_selfcond(z, E, w, k):
+    """The oracle's self-conditioning term of logits z, reading only the embedding
+    rows the top-k entries name."""
+    p, ids = OL.topk_probs(z, k)
+    uniq = np.unique(ids)
+    E_sub = E[torch.from_numpy(uniq).to(E.device)].to(torch.float32).cpu().double().numpy()
+    e = OL.soft_embedding(p, np.searchsorted(uniq, ids), E_sub)
+    f64 = lambda t: t.to(torch.float32).cpu().double().numpy()
+    return p, ids, OL.swiglu(e, f64(w["sc_gate"]), f64(w["sc_up"]), f64(w["sc_down"]))
+
+
+def test_selfcond_op_on_exact_logits(dgmod):
+    """The self-conditioning term from hidden rows: the top-8 ids equal the
+    oracle's exactly (exact logits, ties to the lower id), their probabilities to
+    float32 rounding, and the term itself within the bf16 tolerance (the soft
+    embedding and the MLP's hidden rows are bf16 GEMM inputs)."""
+    from .gpu_common import REL_L2, rel_l2
+    cfg = TINY.with_(n_layers=1, d_model=512, vocab=32768, ffn_selfcond=256, selfcond_topk=8)
+    w = to_device(make_weights(cfg, seed=0))
+    E, x = _exact_lm_inputs(cfg.vocab, cfg.d_model, cfg.canvas, 8, seed=47)
+    w["embed"] = E
+    h = dgmod.DG(cfg, w, max_requests=2, kv_capacity=1024)
+    sc, p, ids = h.op_selfcond(1, x)
+    h.sync()
+    rows = list(range(cfg.canvas))
+    z = _exact_z(E, x, rows, cfg.norm_eps)
+    p_o, ids_o, sc_o = _oracle_selfcond(z, E, w, cfg.selfcond_topk)
+    np.testing.assert_array_equal(ids.cpu().numpy(), ids_o)
+    np.testing.assert_allclose(p.cpu().numpy(), p_o, rtol=1e-4)
+    assert rel_l2(sc.cpu().double().numpy(), sc_o) < REL_L2
+    # the state of request 1 now holds these entries
+    top = h.debug_buffer("sc_top", torch.float32, (2, cfg.canvas, 8, 2))[1]
+    assert torch.equal(top[..., 0], p)
+    h.close()

@@ -392,3 +392,56 @@ def test_temperature_step_draws_candidates(model):
     assert (cand1 != am1).mean() > 0.5          # near-flat random-weight logits: the draw is rarely the argmax
     assert np.all((cand1 >= 0) & (cand1 < CFG.vocab))
     np.testing.assert_array_equal(tok1, tok2)
+
+
+def test_selfcond_teacher_forced_steps():
+    """Self-conditioning in the denoising loop (MLP width 256, top 8).  Step 1
+    has no term, so its statistics equal those of the same model without
+    self-conditioning bit for bit.  Step 2 starts both sides from the oracle's
+    canvas; the GPU feeds back its own step-1 softmax, the oracle its own, and
+    the step-2 statistics agree within the logit tolerance (positions whose
+    step-1 8th and 9th logits are within 0.05, or whose routing is ambiguous,
+    excluded).  Embedding and MLP weights are scaled up so that the softmax is
+    peaked and the term moves the statistics well beyond that tolerance."""
+    import block_diffusion_moe_denoise_b200 as dgm
+    cfg = CFG.with_(ffn_selfcond=256, selfcond_topk=8)
+    w = make_weights(cfg, seed=0, gain_std=0.1)
+    for n in ("embed", "sc_gate", "sc_up", "sc_down"):
+        w[n] = (w[n].float() * 10).to(torch.bfloat16)
+    ora = Oracle(cfg, oracle_weights(w))
+    wd = to_device(w)
+    wd.update({n: w[n].cuda() for n in ("sc_gate", "sc_up", "sc_down")})
+    h = dgm.DG(cfg, wd, max_requests=2, kv_capacity=1024)
+    h0 = dgm.DG(CFG, wd, max_requests=2, kv_capacity=1024)
+    prompt = make_tokens(cfg, 128, seed=0)
+    for hh in (h, h0):
+        hh.prefill(0, prompt.cuda())
+        hh.open_canvas(0, 3, 0)
+        hh.denoise_step([0])
+    _, _, g1, _ = h.get_canvas(0)
+    _, _, g1_plain, _ = h0.get_canvas(0)
+    h.sync()
+    h0.sync()
+    assert torch.equal(g1, g1_plain)
+    cache = ora.new_cache(128 + 256)
+    ora.prefill(cache, prompt.numpy())
+    canvas, acc = ora.open_canvas(seed=3, block=0)
+    st1 = ora.forward(canvas, cache)
+    ncanvas, nacc, _, _ = ora.denoise_step(cache, canvas, acc, seed=3, block=0, step=1, stats=st1)
+    h.set_canvas(0, torch.from_numpy(ncanvas.astype(np.int32)).cuda(),
+                 torch.from_numpy(nacc.astype(np.uint8)).cuda(), 1)
+    h.denoise_step([0])
+    _, _, g2, _ = h.get_canvas(0)
+    h.sync()
+    tr = Trace()
+    st2 = ora.forward(ncanvas, cache, trace=tr, sc=ora.self_condition(st1["logits"]))
+    st2_plain = ora.forward(ncanvas, cache)
+    zs = np.sort(st1["logits"], axis=1)
+    keep = ~ambiguous_tokens(tr.layers, cfg.top_k) & (zs[:, -8] - zs[:, -9] > 0.05)
+    assert keep.sum() > 0.7 * cfg.canvas, keep.sum()
+    gs = g2.cpu().numpy().astype(np.float64)
+    assert np.max(np.abs(gs[keep, 2] - st2["max"][keep])) < LOGIT_MAX_ABS
+    assert rel_l2(gs[keep, 0], st2["entropy"][keep]) < REL_L2
+    assert np.max(np.abs(st2["max"] - st2_plain["max"])) > 10 * LOGIT_MAX_ABS      # the term matters
+    h.close()
+    h0.close()

@@ -57,9 +57,15 @@ def test_host_validation_without_gpu(lib):
     assert L.dg_workspace_size(ctypes.byref(config_struct(TINY)), 9, 1024) == 0
     assert L.dg_workspace_size(ctypes.byref(config_struct(TINY.with_(temperature=-0.5))), 1, 1024) == 0
     assert L.dg_workspace_size(ctypes.byref(config_struct(TINY.with_(temperature=0.7))), 1, 1024) > 0
+    assert L.dg_workspace_size(ctypes.byref(config_struct(TINY.with_(ffn_selfcond=100))), 1, 1024) == 0
+    assert L.dg_workspace_size(ctypes.byref(config_struct(TINY.with_(ffn_selfcond=256, selfcond_topk=9))), 1,
+                               1024) == 0
+    n0 = L.dg_workspace_size(ctypes.byref(config_struct(TINY)), 1, 1024)
+    assert L.dg_workspace_size(ctypes.byref(config_struct(TINY.with_(ffn_selfcond=256))), 1, 1024) > n0
     assert L.dg_strerror(-3) == b"KV capacity or workspace too small"
     # entry points reject bad arguments before touching the device
     assert L.dg_op_route_topk(None, 4, 300, 2, None, None, None) == -1
     assert L.dg_op_philox_tokens(1, 0, 0, 0, 0, 10, 0, None, None) == -1
     assert L.dg_prefill(None, 0, None, 0) == -1
     assert L.dg_op_lm_sample(None, None, 4, 0.7, 1, 0, 1, 0, None, None, None) == -1
+    assert L.dg_op_selfcond(None, 0, None, 4, None, None) == -1

@@ -258,3 +258,81 @@ def test_layer_bruteforce(use_rope):
         assert st["argmax"][t] == ref["argmax"]
         assert abs(st["entropy"][t] - ref["entropy"]) < 1e-10
         assert abs(st["logconf"][t] - ref["logconf"]) < 1e-10
+
+
+# ---- self-conditioning -----------------------------------------------------------------------
+
+def test_topk_probs_bruteforce_with_ties():
+    rng = _rng(30)
+    for _ in range(200):
+        z = rng.choice([-1.0, 0.0, 0.5, 2.0, 2.0, 3.0], size=(1, 12))
+        k = int(rng.integers(1, 9))
+        p, ids = L.topk_probs(z, k)
+        ref = sorted(range(12), key=lambda i: (-z[0, i], i))[:k]      # value descending, lower id first
+        assert ids[0].tolist() == ref
+        full = np.exp(z[0]) / np.exp(z[0]).sum()
+        np.testing.assert_allclose(p[0], full[ref], rtol=1e-14)
+
+
+def test_soft_embedding_closed_forms():
+    rng = _rng(31)
+    V, d = 10, 6
+    E = rng.normal(size=(V, d))
+    z = rng.normal(size=(3, V))
+    # k = V: the full expectation of the embedding under softmax(z)
+    p, ids = L.topk_probs(z, V)
+    sm = np.exp(z) / np.exp(z).sum(axis=1, keepdims=True)
+    np.testing.assert_allclose(L.soft_embedding(p, ids, E), sm @ E, rtol=1e-12)
+    # a dominant logit: the embedding of that id
+    zd = np.zeros((1, V))
+    zd[0, 7] = 60.0
+    p, ids = L.topk_probs(zd, 3)
+    np.testing.assert_allclose(L.soft_embedding(p, ids, E)[0], E[7], atol=1e-20)
+    # two equal dominant logits: half of each (k = 2), half of the lower id alone (k = 1)
+    zt = np.zeros((1, V))
+    zt[0, [2, 5]] = 60.0
+    p, ids = L.topk_probs(zt, 2)
+    np.testing.assert_allclose(L.soft_embedding(p, ids, E)[0], 0.5 * (E[2] + E[5]), rtol=1e-12)
+    p, ids = L.topk_probs(zt, 1)
+    np.testing.assert_allclose(L.soft_embedding(p, ids, E)[0], 0.5 * E[2], rtol=1e-12)
+
+
+def test_self_condition_invariances():
+    rng = _rng(32)
+    V, d, f, k = 16, 8, 12, 4
+    E = rng.normal(size=(V, d))
+    wg, wu, wd = rng.normal(size=(f, d)), rng.normal(size=(f, d)), rng.normal(size=(d, f))
+    z = rng.normal(size=(5, V))
+    out = L.self_condition(z, E, wg, wu, wd, k)
+    # a constant added to a row's logits changes nothing (softmax shift invariance)
+    np.testing.assert_allclose(L.self_condition(z + 3.7, E, wg, wu, wd, k), out, rtol=1e-10)
+    # relabelling the vocabulary (logits and embedding rows together) changes nothing
+    perm = rng.permutation(V)
+    np.testing.assert_allclose(L.self_condition(z[:, perm], E[perm], wg, wu, wd, k), out, rtol=1e-10)
+    # with a dominant logit the term is the gated MLP of that token's embedding
+    zd = np.full((1, V), -50.0)
+    zd[0, 11] = 50.0
+    np.testing.assert_allclose(L.self_condition(zd, E, wg, wu, wd, k)[0], L.swiglu(E[11:12], wg, wu, wd)[0],
+                               rtol=1e-12)
+    # a zero-mass input gives a zero term (no biases)
+    np.testing.assert_array_equal(L.swiglu(np.zeros((1, d)), wg, wu, wd), np.zeros((1, d)))
+
+
+def test_self_conditioning_enters_only_after_the_first_step():
+    cfg = TOY.with_(ffn_selfcond=8, selfcond_topk=3)
+    w = oracle_weights(make_weights(cfg, seed=3))
+    ora = Oracle(cfg, w)
+    toks = np.arange(cfg.canvas) % cfg.vocab
+    c1 = ora.new_cache(32)
+    c2 = ora.new_cache(32)
+    st_plain = ora.forward(toks, c1)
+    st_none = ora.forward(toks, c2, sc=ora.self_condition(None))
+    np.testing.assert_array_equal(st_plain["logits"], st_none["logits"])
+    sc = ora.self_condition(st_plain["logits"])
+    assert sc.shape == (cfg.canvas, cfg.d_model) and np.abs(sc).max() > 0
+    from oracle.model import Trace
+    tr = Trace()
+    st_sc = ora.forward(toks, ora.new_cache(32), sc=sc, trace=tr)
+    # the term is added to the token embeddings at the first layer's input
+    np.testing.assert_array_equal(tr.layers[0]["x_in"], w["embed"][toks] + sc)
+    assert np.abs(st_sc["logits"] - st_plain["logits"]).max() > 1e-12
