@@ -637,7 +637,9 @@ cudaError_t run_lm_combine(const float4* part, int G, int MT, int T, float* stat
 
 // ---------------------------------------------------------------------------
 // Self-conditioning.  k_selfcond_topk: one warp per LM-head row merges the
-// per-CTA top-8 logit lists (lane l takes CTAs l, l+32, ...; then K rounds of
+// top-8 logit lists of the CTAs that saw the row (the grid is a multiple of
+// the token-tile count MT and CTA c handles tile c % MT; lane l takes the
+// l-th, (l+32)-th, ... of them), then K rounds of
 // a warp-wide max, ties to the lower id) and stores the K largest softmax
 // entries p = exp(z - logZ) with their ids in the row's request slot.
 // k_selfcond_embed: one CTA per pass row, 8 columns per thread, accumulates
@@ -672,7 +674,9 @@ __global__ void k_selfcond_topk(const float2* __restrict__ sc_part, int G, int T
     tv[r] = -INFINITY;
     ti[r] = 0x7fffffff;
   }
-  for (int c = lane; c < G; c += 32) {
+  // only the CTAs of this row's token tile wrote it (CTA c holds tile c % MT)
+  const int MT = (T + 127) / 128;
+  for (int c = t / 128 + lane * MT; c < G; c += 32 * MT) {
     const float2* l = sc_part + ((size_t)c * T + t) * 8;
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
