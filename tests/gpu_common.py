@@ -19,11 +19,15 @@ LOGIT_MAX_ABS = 5e-2
 
 
 def to_device(w: dict, device="cuda") -> dict:
-    return {
+    out = {
         "embed": w["embed"].to(device),
         "final_norm": w["final_norm"].to(device),
         "layers": [{k: v.to(device).contiguous() for k, v in lw.items()} for lw in w["layers"]],
     }
+    for name in ("sc_gate", "sc_up", "sc_down"):
+        if name in w:
+            out[name] = w[name].to(device).contiguous()
+    return out
 
 
 def np64(t: torch.Tensor) -> np.ndarray:

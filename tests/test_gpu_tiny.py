@@ -399,18 +399,19 @@ def test_selfcond_teacher_forced_steps():
     has no term, so its statistics equal those of the same model without
     self-conditioning bit for bit.  Step 2 starts both sides from the oracle's
     canvas; the GPU feeds back its own step-1 softmax, the oracle its own, and
-    the step-2 statistics agree within the logit tolerance (positions whose
-    step-1 8th and 9th logits are within 0.05, or whose routing is ambiguous,
-    excluded).  Embedding and MLP weights are scaled up so that the softmax is
-    peaked and the term moves the statistics well beyond that tolerance."""
+    the step-2 statistics agree within the logit tolerance (positions with
+    ambiguous routing excluded).  The embedding (x3) and MLP (x5) weights are
+    scaled so that the softmax is peaked (step-1 entropy ~0.2 nats: the entries
+    past the 8th carry almost no mass, so the GPU's and the oracle's top-8 may
+    differ there without effect) and the term moves the statistics well beyond
+    the tolerance."""
     import block_diffusion_moe_denoise_b200 as dgm
     cfg = CFG.with_(ffn_selfcond=256, selfcond_topk=8)
     w = make_weights(cfg, seed=0, gain_std=0.1)
-    for n in ("embed", "sc_gate", "sc_up", "sc_down"):
-        w[n] = (w[n].float() * 10).to(torch.bfloat16)
+    for n, f in (("embed", 3), ("sc_gate", 5), ("sc_up", 5), ("sc_down", 5)):
+        w[n] = (w[n].float() * f).to(torch.bfloat16)
     ora = Oracle(cfg, oracle_weights(w))
     wd = to_device(w)
-    wd.update({n: w[n].cuda() for n in ("sc_gate", "sc_up", "sc_down")})
     h = dgm.DG(cfg, wd, max_requests=2, kv_capacity=1024)
     h0 = dgm.DG(CFG, wd, max_requests=2, kv_capacity=1024)
     prompt = make_tokens(cfg, 128, seed=0)
@@ -436,12 +437,13 @@ def test_selfcond_teacher_forced_steps():
     tr = Trace()
     st2 = ora.forward(ncanvas, cache, trace=tr, sc=ora.self_condition(st1["logits"]))
     st2_plain = ora.forward(ncanvas, cache)
-    zs = np.sort(st1["logits"], axis=1)
-    keep = ~ambiguous_tokens(tr.layers, cfg.top_k) & (zs[:, -8] - zs[:, -9] > 0.05)
-    assert keep.sum() > 0.7 * cfg.canvas, keep.sum()
+    keep = ~ambiguous_tokens(tr.layers, cfg.top_k)
+    assert keep.sum() > 0.8 * cfg.canvas, keep.sum()
     gs = g2.cpu().numpy().astype(np.float64)
     assert np.max(np.abs(gs[keep, 2] - st2["max"][keep])) < LOGIT_MAX_ABS
     assert rel_l2(gs[keep, 0], st2["entropy"][keep]) < REL_L2
-    assert np.max(np.abs(st2["max"] - st2_plain["max"])) > 10 * LOGIT_MAX_ABS      # the term matters
+    # the term matters: without it the statistics are far outside the tolerance
+    assert np.max(np.abs(st2["max"] - st2_plain["max"])) > 5 * LOGIT_MAX_ABS
+    assert rel_l2(st2_plain["entropy"], st2["entropy"]) > 5 * REL_L2
     h.close()
     h0.close()
