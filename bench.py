@@ -52,6 +52,10 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--canvas-vocab", type=int, default=0,
                     help="layer workload: draw canvas ids from this many distinct tokens (concentrates routing)")
+    ap.add_argument("--temperature", type=float, default=0.0,
+                    help="variant: candidates drawn from softmax(logits / T) instead of the argmax")
+    ap.add_argument("--selfcond", type=int, default=0,
+                    help="variant: self-conditioning gated MLP of this width (top-8 softmax fed back)")
     return ap.parse_args()
 
 
@@ -270,9 +274,14 @@ def workload_config(cfg, workload, world):
     else:
         name = ("generate: 30 layers d2816, 16q/8kv heads x256, 128 experts top-8 + shared 2112, vocab 262144, "
                 "4096-token prompt prefilled, canvases of 256 (12 steps + commit), blocks 0-3, batch 1")
-    return {"workload": name, "canvas": cfg.canvas, "kv_prefix": PROMPT, "batch": 1,
-            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-            "l2": "inputs larger than L2: every step streams ~50 GB of weights (no flush needed)"}
+    out = {"workload": name, "canvas": cfg.canvas, "kv_prefix": PROMPT, "batch": 1,
+           "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+           "l2": "inputs larger than L2: every step streams ~50 GB of weights (no flush needed)"}
+    if getattr(cfg, "temperature", 0.0) > 0:
+        out["temperature"] = cfg.temperature
+    if getattr(cfg, "ffn_selfcond", 0) > 0:
+        out["selfcond"] = {"ffn": cfg.ffn_selfcond, "topk": cfg.selfcond_topk}
+    return out
 
 
 # ---------------------------------------------------------------------------
@@ -292,6 +301,7 @@ def main():
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     cfg = FULL if args.workload == "generate" else LAYER
+    cfg = cfg.with_(temperature=args.temperature, ffn_selfcond=args.selfcond)
     hbm_gbs, bf16_tf, bf16_tf_sus, peak_kind = measured_peaks()
 
     w = make_weights(cfg, seed=0, device=dev)
