@@ -56,6 +56,8 @@ def parse():
                     help="variant: candidates drawn from softmax(logits / T) instead of the argmax")
     ap.add_argument("--selfcond", type=int, default=0,
                     help="variant: self-conditioning gated MLP of this width (top-8 softmax fed back)")
+    ap.add_argument("--fp8-experts", action="store_true",
+                    help="variant: routed-expert weights as E4M3 codes with per-row scales (W8A8 expert GEMMs)")
     return ap.parse_args()
 
 
@@ -129,9 +131,10 @@ def expert_gate_up_bytes(cfg, n_touched: float, T: int) -> float:
     """Bytes one routed-expert gate|up launch must move: the gate and up
     weights of every expert some token is routed to, the grouped token rows
     read, the SwiGLU hidden rows written."""
-    w = n_touched * 2 * cfg.ffn_expert * cfg.d_model * 2
+    eb = 1 if getattr(cfg, "expert_fp8", 0) else 2          # E4M3 codes or bf16
+    w = n_touched * 2 * cfg.ffn_expert * (cfg.d_model * eb + (4 if eb == 1 else 0))
     rows = T * cfg.top_k
-    return w + rows * cfg.d_model * 2 + rows * cfg.ffn_expert * 2
+    return w + rows * (cfg.d_model * eb + (4 if eb == 1 else 0)) + rows * cfg.ffn_expert * 2
 
 
 def step_work(cfg, kv_len: int, T: int, n_touched: float):
@@ -139,7 +142,8 @@ def step_work(cfg, kv_len: int, T: int, n_touched: float):
     experts and all dense weights once, the KV prefix read, per-token FLOPs."""
     d, D = cfg.d_model, cfg.head_dim
     attn_w = cfg.qkv_rows * d + d * cfg.n_q_heads * D
-    per_layer_w = attn_w + n_touched * 3 * cfg.ffn_expert * d + 3 * cfg.ffn_shared * d + cfg.n_experts * d
+    eb = 0.5 if getattr(cfg, "expert_fp8", 0) else 1.0      # expert weights: E4M3 codes or bf16
+    per_layer_w = attn_w + eb * n_touched * 3 * cfg.ffn_expert * d + 3 * cfg.ffn_shared * d + cfg.n_experts * d
     weights = (cfg.n_layers * per_layer_w + cfg.vocab * d) * 2
     kv = cfg.n_layers * 2 * cfg.n_kv_heads * (kv_len + T) * D * 2
     act = cfg.n_layers * T * (cfg.top_k * (3 * d + cfg.ffn_expert) * 2 + 12 * d * 4)
@@ -281,6 +285,8 @@ def workload_config(cfg, workload, world):
         out["temperature"] = cfg.temperature
     if getattr(cfg, "ffn_selfcond", 0) > 0:
         out["selfcond"] = {"ffn": cfg.ffn_selfcond, "topk": cfg.selfcond_topk}
+    if getattr(cfg, "expert_fp8", 0):
+        out["experts"] = "e4m3 weights with per-row fp32 scales, per-row e4m3 activations (W8A8)"
     return out
 
 
@@ -301,7 +307,8 @@ def main():
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     cfg = FULL if args.workload == "generate" else LAYER
-    cfg = cfg.with_(temperature=args.temperature, ffn_selfcond=args.selfcond)
+    cfg = cfg.with_(temperature=args.temperature, ffn_selfcond=args.selfcond,
+                    expert_fp8=1 if args.fp8_experts else 0)
     hbm_gbs, bf16_tf, bf16_tf_sus, peak_kind = measured_peaks()
 
     w = make_weights(cfg, seed=0, device=dev)
@@ -462,7 +469,7 @@ def main():
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": "bf16+e4m3" if getattr(cfg, "expert_fp8", 0) else "bf16",
         "data": "synthetic (seeded N(0,0.02) bf16 weights, uniform token ids)",
         "config": workload_config(cfg, args.workload, world),
         "roofline": {"kernel": "experts_gate_up (routed-expert gate|up GEMM + SwiGLU)", "bound": "hbm",

@@ -35,7 +35,8 @@ def config_struct(cfg) -> dg_config:
                      cfg.min_accept, cfg.entropy_thresh, cfg.rope_theta, cfg.norm_eps,
                      getattr(cfg, "sampler", 0), getattr(cfg, "entropy_budget", 0.1),
                      getattr(cfg, "stop_entropy", 0.005), getattr(cfg, "temperature", 0.0),
-                     getattr(cfg, "ffn_selfcond", 0), getattr(cfg, "selfcond_topk", 8))
+                     getattr(cfg, "ffn_selfcond", 0), getattr(cfg, "selfcond_topk", 8),
+                     getattr(cfg, "expert_fp8", 0))
 
 
 def philox_tokens(seed: int, block: int, step: int, request: int, pos0: int, n: int, vocab: int,
@@ -72,9 +73,9 @@ class DG:
         self.stream = stream or torch.cuda.current_stream(device)
         layers = (dg_layer_weights * cfg.n_layers)()
         for i, lw in enumerate(weights["layers"]):
-            layers[i] = dg_layer_weights(*[lw[n].data_ptr() for n in (
+            layers[i] = dg_layer_weights(*[lw[n].data_ptr() if n in lw else None for n in (
                 "attn_norm", "w_qkv", "w_o", "ffn_norm", "w_router", "w_gate", "w_up", "w_down", "ws_gate",
-                "ws_up", "ws_down")])
+                "ws_up", "ws_down", "w_gate_scale", "w_up_scale", "w_down_scale")])
         self._layers = layers
         sc = [weights[n].data_ptr() if n in weights else None for n in ("sc_gate", "sc_up", "sc_down")]
         self.c_w = dg_weights(weights["embed"].data_ptr(), weights["final_norm"].data_ptr(), layers, *sc)

@@ -19,12 +19,14 @@ class dg_config(C.Structure):
                                        "min_accept")] + \
                [("entropy_thresh", C.c_float), ("rope_theta", C.c_float), ("norm_eps", C.c_float),
                 ("sampler", C.c_int), ("entropy_budget", C.c_float), ("stop_entropy", C.c_float),
-                ("temperature", C.c_float), ("ffn_selfcond", C.c_int), ("selfcond_topk", C.c_int)]
+                ("temperature", C.c_float), ("ffn_selfcond", C.c_int), ("selfcond_topk", C.c_int),
+                ("expert_fp8", C.c_int)]
 
 
 class dg_layer_weights(C.Structure):
     _fields_ = [(n, C.c_void_p) for n in ("attn_norm", "w_qkv", "w_o", "ffn_norm", "w_router", "w_gate", "w_up",
-                                          "w_down", "ws_gate", "ws_up", "ws_down")]
+                                          "w_down", "ws_gate", "ws_up", "ws_down", "w_gate_scale", "w_up_scale",
+                                          "w_down_scale")]
 
 
 class dg_weights(C.Structure):

@@ -145,6 +145,18 @@ DG_DEVINL void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32
       : "memory");
 }
 
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, E4M3 inputs (K = 32 per
+// instruction, the same 32 bytes of each 128-byte row as a bf16 K = 16 step),
+// fp32 accumulator.
+DG_DEVINL void umma_e4m3(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // D[tmem] (+)= A[tmem] * B[smem desc]^T: A (M = 128 rows, one per lane, bf16
 // pairs per 32-bit column, K-major) read from tensor memory.
 DG_DEVINL void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
@@ -168,6 +180,16 @@ DG_DEVINL uint32_t umma_idesc_bf16(uint32_t m, uint32_t n) {
   return (1u << 4)            // D format: f32
          | (1u << 7)          // A format: bf16
          | (1u << 10)         // B format: bf16
+         | ((n >> 3) << 17)   // N >> 3
+         | ((m >> 4) << 24);  // M >> 4
+}
+
+// Instruction descriptor for kind::f8f6f4 with E4M3 A/B (format code 0), fp32 D,
+// both K-major, M = 128, N = n (multiple of 16, 16..256).
+DG_DEVINL uint32_t umma_idesc_e4m3(uint32_t m, uint32_t n) {
+  return (1u << 4)            // D format: f32
+         | (0u << 7)          // A format: e4m3
+         | (0u << 10)         // B format: e4m3
          | ((n >> 3) << 17)   // N >> 3
          | ((m >> 4) << 24);  // M >> 4
 }

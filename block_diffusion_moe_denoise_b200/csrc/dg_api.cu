@@ -70,6 +70,7 @@ bool config_ok(const dg_config* c) {
   if (!(c->temperature >= 0.f && c->temperature <= 1e30f)) return false;
   if (c->ffn_selfcond < 0 || c->ffn_selfcond % 64 != 0) return false;
   if (c->ffn_selfcond > 0 && (c->selfcond_topk < 1 || c->selfcond_topk > 8)) return false;
+  if (c->expert_fp8 != 0 && c->expert_fp8 != 1) return false;
   return true;
 }
 
@@ -118,6 +119,13 @@ void make_plan(const dg_config* c, int max_req, long long cap_user, Plan* p) {
     p->add("sc_top", sc ? (size_t)max_req * c->canvas * 8 * 8 : 64);
     p->add("hs_sc", sc ? (size_t)Tcap * c->ffn_selfcond * 2 : 64);
   }
+  {
+    const bool f8 = c->expert_fp8 != 0;
+    p->add("xq", f8 ? (size_t)rows * d : 64);
+    p->add("xs", f8 ? (size_t)rows * 4 : 64);
+    p->add("hq", f8 ? (size_t)rows * c->ffn_expert : 64);
+    p->add("hsq", f8 ? (size_t)rows * 4 : 64);
+  }
   p->add("canvas", (size_t)max_req * c->canvas * 4);
   p->add("commit_tok", (size_t)max_req * c->canvas * 4);
   p->add("prev_argmax", (size_t)max_req * c->canvas * 4);
@@ -160,6 +168,21 @@ bool make_map(CUtensorMap* m, const void* base, long long K, long long rows, int
   cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   cuuint32_t es[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D byte tensor [rows, K] (E4M3 codes, K contiguous) read in boxes of 128 x
+// box_rows bytes with the 128-byte swizzle; out-of-range elements read as zeros.
+bool make_map_u8(CUtensorMap* m, const void* base, long long K, long long rows, int box_rows) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  if ((reinterpret_cast<uintptr_t>(base) & 15) != 0 || K % 16 != 0) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)K};
+  cuuint32_t box[2] = {128, (cuuint32_t)box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -231,6 +254,7 @@ struct dg_handle {
   std::vector<LayerMaps> maps;
   CUtensorMap tm_hn, tm_o, tm_u, tm_xp, tm_hp, tm_hs, tm_embed, tm_k, tm_vt;
   CUtensorMap tm_sc_gate, tm_sc_up, tm_sc_down, tm_hs_sc;  // self-conditioning MLP and its hidden rows
+  CUtensorMap tm_xq, tm_hq;                                // FP8 experts: token and hidden codes
   long long cap_user = 0;  // capacity the caller asked for (cap is rounded up to 64)
   ReqState req[DG_MAX_REQUESTS];
   int mask_flip = 0;  // which of the two routing bitmask buffers the next layer uses
@@ -468,7 +492,10 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     ga.ed_count = h->B<int>("tile_counts") + 1;
     ga.route_stats = h->B<unsigned long long>("route_stats");
     ga.err = err;
-    LAUNCH(h, K_GROUP, 1, run_route(h->B<bf16>("u"), d, h->B<bf16>("xp"), mask_cur, mask_nxt, MW, ga, st));
+    const bool f8 = c.expert_fp8 != 0;
+    LAUNCH(h, K_GROUP, 1,
+           run_route(h->B<bf16>("u"), d, h->B<bf16>("xp"), mask_cur, mask_nxt, MW, ga, st,
+                     f8 ? h->B<uint8_t>("xq") : nullptr, f8 ? h->B<float>("xs") : nullptr));
 
     ExpertArgs ea;
     ea.tm_gate = &m.gate;
@@ -489,8 +516,22 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     ea.hp = h->B<bf16>("hp");
     ea.yp = yp;
     ea.err = err;
-    LAUNCH(h, K_EGU, 1, run_experts_gate_up(ea, st));
-    LAUNCH(h, K_ED, 1, run_experts_down(ea, st));
+    if (f8) {
+      // E4M3 weight codes and token rows; the SwiGLU rows are quantised per row before down
+      ea.tm_xp = &h->tm_xq;
+      ea.tm_hp = &h->tm_hq;
+      ea.s_gate = (const float*)w.w_gate_scale;
+      ea.s_up = (const float*)w.w_up_scale;
+      ea.s_down = (const float*)w.w_down_scale;
+      ea.s_x = h->B<float>("xs");
+      ea.s_h = h->B<float>("hsq");
+      LAUNCH(h, K_EGU, 1, run_experts_gate_up_fp8(ea, st));
+      LAUNCH(h, K_ED, 1, run_quant_rows(ea.hp, c.ffn_expert, T * k, h->B<uint8_t>("hq"), h->B<float>("hsq"), st));
+      LAUNCH(h, K_ED, 1, run_experts_down_fp8(ea, st));
+    } else {
+      LAUNCH(h, K_EGU, 1, run_experts_gate_up(ea, st));
+      LAUNCH(h, K_ED, 1, run_experts_down(ea, st));
+    }
 
     WpartArgs da;
     da.tm_w = &m.sdown;
@@ -645,9 +686,16 @@ int dg_init(const dg_config* cfg, const dg_weights* wts, int max_requests, int64
     ok = ok && w.attn_norm && w.ffn_norm && w.w_router;
     ok = ok && make_map(&m.qkv, w.w_qkv, d, qkv_rows, 64);
     ok = ok && make_map(&m.o, w.w_o, (long long)c.n_q_heads * D, d, 128);
-    ok = ok && make_map(&m.gate, w.w_gate, d, E * c.ffn_expert, 64);
-    ok = ok && make_map(&m.up, w.w_up, d, E * c.ffn_expert, 64);
-    ok = ok && make_map(&m.down, w.w_down, c.ffn_expert, E * d, 128);
+    if (c.expert_fp8) {
+      ok = ok && w.w_gate_scale && w.w_up_scale && w.w_down_scale;
+      ok = ok && make_map_u8(&m.gate, w.w_gate, d, E * c.ffn_expert, 64);
+      ok = ok && make_map_u8(&m.up, w.w_up, d, E * c.ffn_expert, 64);
+      ok = ok && make_map_u8(&m.down, w.w_down, c.ffn_expert, E * d, 128);
+    } else {
+      ok = ok && make_map(&m.gate, w.w_gate, d, E * c.ffn_expert, 64);
+      ok = ok && make_map(&m.up, w.w_up, d, E * c.ffn_expert, 64);
+      ok = ok && make_map(&m.down, w.w_down, c.ffn_expert, E * d, 128);
+    }
     ok = ok && make_map(&m.sgate, w.ws_gate, d, c.ffn_shared, 32);
     ok = ok && make_map(&m.sup, w.ws_up, d, c.ffn_shared, 32);
     ok = ok && make_map(&m.router, w.w_router, d, E, (int)E);
@@ -664,6 +712,10 @@ int dg_init(const dg_config* cfg, const dg_weights* wts, int max_requests, int64
     const long long kv_elems = (long long)max_requests * h->kv_req_stride;
     ok = ok && make_map(&h->tm_k, h->B<bf16>("kv"), D, kv_elems / D, 64);
     ok = ok && make_map(&h->tm_vt, h->B<bf16>("kv"), h->cap, kv_elems / h->cap, D);
+  }
+  if (c.expert_fp8) {
+    ok = ok && make_map_u8(&h->tm_xq, h->B<uint8_t>("xq"), d, rows, kExpertRows);
+    ok = ok && make_map_u8(&h->tm_hq, h->B<uint8_t>("hq"), c.ffn_expert, rows, kExpertRows);
   }
   if (c.ffn_selfcond > 0) {
     const int f = c.ffn_selfcond;

@@ -67,6 +67,8 @@ struct ExpertArgs {
   bf16* hp;
   float* yp;
   int* err;
+  // FP8 experts: per-row scales of the weight codes and of the token / hidden codes
+  const float *s_gate = nullptr, *s_up = nullptr, *s_down = nullptr, *s_x = nullptr, *s_h = nullptr;
 };
 struct SharedArgs {
   const CUtensorMap *tm_u, *tm_gate, *tm_up, *tm_router;
@@ -109,6 +111,8 @@ int wpart_splits(int d, int T, int K, int num_sms);
 cudaError_t run_wpart(const WpartArgs& a, cudaStream_t st);
 cudaError_t run_experts_gate_up(const ExpertArgs& a, cudaStream_t st);
 cudaError_t run_experts_down(const ExpertArgs& a, cudaStream_t st);
+cudaError_t run_experts_gate_up_fp8(const ExpertArgs& a, cudaStream_t st);
+cudaError_t run_experts_down_fp8(const ExpertArgs& a, cudaStream_t st);
 cudaError_t run_shared_gate_up(const SharedArgs& a, cudaStream_t st);
 cudaError_t run_lm_head(const LmArgs& a, int* grid_out, cudaStream_t st);
 size_t gemm_smem_bytes_max();
@@ -152,7 +156,10 @@ cudaError_t run_group(const GroupArgs& a, cudaStream_t st);
 // the workspace so the layout never changes between passes) the router epilogue
 // set, plus the gather of u rows into xp; clears all of `mask_next`
 cudaError_t run_route(const bf16* u, int d, bf16* xp, unsigned* mask, unsigned* mask_next, int MW,
-                      const GroupArgs& a, cudaStream_t st);
+                      const GroupArgs& a, cudaStream_t st, uint8_t* xq = nullptr, float* xs = nullptr);
+// Per-row E4M3 quantisation of bf16 rows [rows, n] (n % 8 == 0, n <= 4096):
+// codes [rows, n] and fp32 scales [rows] (E4M3(x * 448 / amax), amax / 448).
+cudaError_t run_quant_rows(const bf16* in, int n, int rows, uint8_t* out, float* scale, cudaStream_t st);
 // Merge of the LM head's per-CTA partials into per-row statistics; with
 // `draw` (the per-tile records of a candidate draw, NV tiles per row) also the
 // row-level pick of the tile, whose drawn id goes to cand[row].

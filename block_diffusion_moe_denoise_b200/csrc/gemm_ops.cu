@@ -392,6 +392,147 @@ struct P_ED : ProblemBase {
 };
 
 // ---------------------------------------------------------------------------
+// FP8 (E4M3) routed experts: the same tiles as P_EGU / P_ED with E4M3 weight
+// codes (one fp32 scale per weight row) and E4M3 token rows (one fp32 scale per
+// grouped row); a k-block is 128 elements (one 128-byte row), so a tile has
+// half the k-blocks of its bf16 form.  The accumulator holds
+// sum decode(q_w) decode(q_x); the epilogue applies both scales.
+// ---------------------------------------------------------------------------
+struct P_EGU8 : ProblemBase {
+  static constexpr bool F8 = true;
+  static constexpr int BN = kExpertRows, STAGES = 4, KB = 2, B_STAGE = BN * 128, TMEM_COLS = 128;
+  static constexpr int EP_SMEM = 64 * 17 * 4;
+  struct Params {
+    CUtensorMap tmG;  // w_gate codes as [E*fe, d] bytes
+    CUtensorMap tmU;  // w_up codes as [E*fe, d] bytes
+    CUtensorMap tmX;  // grouped token codes [rows_cap, d] bytes, 64-row boxes
+    int nk, fe;
+    const int4* tiles;
+    const int* n_tiles;
+    const int* counts;
+    const int* offsets;
+    const float* sg;    // [E*fe] gate row scales
+    const float* su;    // [E*fe] up row scales
+    const float* sx;    // [rows] token row scales
+    __nv_bfloat16* hp;  // [rows_cap, fe]
+    int* err;
+  };
+  DG_DEVINL static void prefetch(const Params& p) {
+    tma_prefetch_desc(&p.tmG);
+    tma_prefetch_desc(&p.tmU);
+    tma_prefetch_desc(&p.tmX);
+  }
+  DG_DEVINL static int num_tiles(const Params& p) { return *p.n_tiles; }
+  DG_DEVINL static Tile tile(const Params& p, int v) {
+    const int4 tt = p.tiles[v];
+    Tile t;
+    t.a = tt.x;
+    t.b = tt.y;
+    const int nt = tt.z;
+    const int n_valid = min(BN, p.counts[t.a] - nt * BN);
+    t.valid = n_valid > 0;
+    t.c = n_valid;
+    t.d = p.offsets[t.a] + nt * BN;
+    t.nk = p.nk;
+    t.n_mma = round_up16(n_valid);
+    return t;
+  }
+  DG_DEVINL static uint32_t tx_bytes(const Params&, const Tile&) { return kAStage + B_STAGE; }
+  DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
+    const int r = t.a * p.fe + t.b * 64;
+    tma_load_2d(sa, &p.tmG, kb * 128, r, bar);
+    tma_load_2d(sa + 64 * 128, &p.tmU, kb * 128, r, bar);
+    tma_load_2d(sb, &p.tmX, kb * 128, t.d, bar);
+  }
+  DG_DEVINL static void epilogue(const Params& p, const Tile& t, uint32_t taddr, int, int, int row, uint8_t* ep) {
+    float* xch = reinterpret_cast<float*>(ep);
+    const int r = t.a * p.fe + t.b * 64 + (row & 63);
+    const float sw = row < 64 ? p.sg[r] : p.su[r];
+    for (int c0 = 0; c0 < t.n_mma; c0 += 16) {
+      float v[16];
+      tmem_ld16(taddr + c0, v);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) v[i] = c0 + i < t.c ? v[i] * sw * p.sx[t.d + c0 + i] : 0.f;
+      if (row >= 64) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) xch[(row - 64) * 17 + i] = v[i];
+      }
+      named_bar_sync(1, 128);
+      if (row < 64) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int c = c0 + i;
+          if (c < t.c) {
+            const float h = silu_f(v[i]) * xch[row * 17 + i];
+            p.hp[(size_t)(t.d + c) * p.fe + t.b * 64 + row] = f2bf(h);
+          }
+        }
+      }
+      named_bar_sync(1, 128);
+    }
+  }
+};
+
+struct P_ED8 : ProblemBase {
+  static constexpr bool F8 = true;
+  static constexpr int BN = kExpertRows, STAGES = 4, KB = 2, B_STAGE = BN * 128, TMEM_COLS = 128;
+  struct Params {
+    CUtensorMap tmW;  // w_down codes as [E*d, fe] bytes
+    CUtensorMap tmH;  // hidden codes [rows_cap, fe] bytes, 64-row boxes
+    int nk, d;
+    const int4* tiles;
+    const int* n_tiles;
+    const int* counts;
+    const int* offsets;
+    const float* sw;   // [E*d] down row scales
+    const float* sh;   // [rows] hidden row scales
+    const float* row_weight;
+    float* yp;  // [rows_cap, d]
+    int* err;
+  };
+  DG_DEVINL static void prefetch(const Params& p) {
+    tma_prefetch_desc(&p.tmW);
+    tma_prefetch_desc(&p.tmH);
+  }
+  DG_DEVINL static int num_tiles(const Params& p) { return *p.n_tiles; }
+  DG_DEVINL static Tile tile(const Params& p, int v) {
+    const int4 tt = p.tiles[v];
+    Tile t;
+    t.a = tt.x;
+    t.b = tt.y;
+    const int nt = tt.z;
+    const int n_valid = min(BN, p.counts[t.a] - nt * BN);
+    t.valid = n_valid > 0;
+    t.c = n_valid;
+    t.d = p.offsets[t.a] + nt * BN;
+    t.nk = p.nk;
+    t.n_mma = round_up16(n_valid);
+    return t;
+  }
+  DG_DEVINL static uint32_t tx_bytes(const Params&, const Tile&) { return kAStage + B_STAGE; }
+  DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
+    tma_load_2d(sa, &p.tmW, kb * 128, t.a * p.d + t.b * 128, bar);
+    tma_load_2d(sb, &p.tmH, kb * 128, t.d, bar);
+  }
+  DG_DEVINL static void epilogue(const Params& p, const Tile& t, uint32_t taddr, int, int, int row, uint8_t*) {
+    const int f = t.b * 128 + row;
+    const float sw = p.sw[(size_t)t.a * p.d + f];
+    for (int c0 = 0; c0 < t.n_mma; c0 += 16) {
+      float v[16];
+      tmem_ld16(taddr + c0, v);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int c = c0 + i;
+        if (c < t.c) {
+          const int r = t.d + c;
+          p.yp[(size_t)r * p.d + f] = p.row_weight[r] * (v[i] * sw * p.sh[r]);
+        }
+      }
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------
 // Shared expert gate|up + SwiGLU, and the router, in one launch (both read the
 // FFN-normed token rows).  Tokens are the 128-row operand.
 //   router tile (mt):     N = E router rows; the epilogue thread owning a token
@@ -853,6 +994,43 @@ cudaError_t run_experts_gate_up(const ExpertArgs& a, cudaStream_t st) {
   return launch_gemm<P_EGU>(g, a.num_sms, st);
 }
 
+cudaError_t run_experts_gate_up_fp8(const ExpertArgs& a, cudaStream_t st) {
+  P_EGU8::Params g;
+  g.tmG = *a.tm_gate;
+  g.tmU = *a.tm_up;
+  g.tmX = *a.tm_xp;
+  g.nk = (a.d + 127) / 128;
+  g.fe = a.fe;
+  g.tiles = a.egu_tiles;
+  g.n_tiles = a.egu_count;
+  g.counts = a.counts;
+  g.offsets = a.offsets;
+  g.sg = a.s_gate;
+  g.su = a.s_up;
+  g.sx = a.s_x;
+  g.hp = a.hp;
+  g.err = a.err;
+  return launch_gemm<P_EGU8>(g, a.num_sms, st);
+}
+
+cudaError_t run_experts_down_fp8(const ExpertArgs& a, cudaStream_t st) {
+  P_ED8::Params dn;
+  dn.tmW = *a.tm_down;
+  dn.tmH = *a.tm_hp;
+  dn.nk = (a.fe + 127) / 128;
+  dn.d = a.d;
+  dn.tiles = a.ed_tiles;
+  dn.n_tiles = a.ed_count;
+  dn.counts = a.counts;
+  dn.offsets = a.offsets;
+  dn.sw = a.s_down;
+  dn.sh = a.s_h;
+  dn.row_weight = a.row_weight;
+  dn.yp = a.yp;
+  dn.err = a.err;
+  return launch_gemm<P_ED8>(dn, a.num_sms, st);
+}
+
 cudaError_t run_experts_down(const ExpertArgs& a, cudaStream_t st) {
   P_ED::Params dn;
   dn.tmW = *a.tm_down;
@@ -928,6 +1106,8 @@ size_t gemm_smem_bytes_max() {
   m = m > GemmSmem<P_ED>::total ? m : GemmSmem<P_ED>::total;
   m = m > GemmSmem<P_SGU>::total ? m : GemmSmem<P_SGU>::total;
   m = m > GemmSmem<P_LM>::total ? m : GemmSmem<P_LM>::total;
+  m = m > GemmSmem<P_EGU8>::total ? m : GemmSmem<P_EGU8>::total;
+  m = m > GemmSmem<P_ED8>::total ? m : GemmSmem<P_ED8>::total;
   return m;
 }
 

@@ -1,5 +1,6 @@
 // CUDA-core kernels of the denoising pass: everything that is not a dense
 // contraction.  Warp-shuffle reductions, 16-byte vector loads/stores.
+#include <cuda_fp8.h>
 #include <float.h>
 #include <string.h>
 
@@ -373,6 +374,77 @@ DG_DEVINL int warp_excl_scan8(int* vals8, int lane) {
 }
 
 // ---------------------------------------------------------------------------
+// Per-row E4M3 quantisation by one warp (row of n bf16 values, n % 8 == 0,
+// n <= 4096): amax = max |x|; codes = E4M3(x * (448 / amax)) rounded to
+// nearest even with saturation; scale = amax / 448 (both divisions and the
+// product IEEE round-to-nearest in fp32); a zero row gives zero codes and
+// scale 0.
+// ---------------------------------------------------------------------------
+DG_DEVINL void quant_row_warp(const bf16* __restrict__ src, int n, uint8_t* __restrict__ dst, float* scale,
+                              int lane) {
+  constexpr int kMaxChunks = 16;  // 4096 / 8 / 32
+  const int n8 = n / 8;
+  uint4 r[kMaxChunks];
+  float amax = 0.f;
+#pragma unroll
+  for (int b = 0; b < kMaxChunks; ++b) {
+    const int c = lane + 32 * b;
+    if (c < n8) {
+      r[b] = reinterpret_cast<const uint4*>(src)[c];
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&r[b]);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(h2[i]);
+        amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+      }
+    }
+  }
+  amax = warp_max(amax);
+  const bool nz = amax > 0.f;
+  const float s_inv = nz ? __fdiv_rn(448.f, amax) : 0.f;
+#pragma unroll
+  for (int b = 0; b < kMaxChunks; ++b) {
+    const int c = lane + 32 * b;
+    if (c < n8) {
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&r[b]);
+      uint32_t w[2];
+#pragma unroll
+      for (int i = 0; i < 4; i += 2) {
+        const float2 f0 = __bfloat1622float2(h2[i]), f1 = __bfloat1622float2(h2[i + 1]);
+        const __nv_fp8x2_storage_t q0 =
+            __nv_cvt_float2_to_fp8x2(make_float2(__fmul_rn(f0.x, s_inv), __fmul_rn(f0.y, s_inv)), __NV_SATFINITE,
+                                     __NV_E4M3);
+        const __nv_fp8x2_storage_t q1 =
+            __nv_cvt_float2_to_fp8x2(make_float2(__fmul_rn(f1.x, s_inv), __fmul_rn(f1.y, s_inv)), __NV_SATFINITE,
+                                     __NV_E4M3);
+        w[i / 2] = (uint32_t)q0 | ((uint32_t)q1 << 16);
+      }
+      reinterpret_cast<uint2*>(dst)[c] = make_uint2(w[0], w[1]);
+    }
+  }
+  if (lane == 0) *scale = nz ? __fdiv_rn(amax, 448.f) : 0.f;
+}
+
+__global__ void k_quant_rows(const bf16* __restrict__ in, int n, int rows, uint8_t* __restrict__ out,
+                             float* __restrict__ scale) {
+  pdl_trigger();
+  pdl_wait();
+  const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (r >= rows) return;
+  quant_row_warp(in + (size_t)r * n, n, out + (size_t)r * n, scale + r, threadIdx.x & 31);
+}
+
+cudaError_t run_quant_rows(const bf16* in, int n, int rows, uint8_t* out, float* scale, cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  if (n % 8 != 0 || n > 4096) return cudaErrorInvalidValue;
+  {
+    const cudaError_t e_ = launch_pdl(k_quant_rows, dim3((rows + 7) / 8), dim3(256), 0, st, in, n, rows, out, scale);
+    if (e_ != cudaSuccess) return e_;
+  }
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
 // Routing after the router GEMM (every CTA): per-expert counts from the token
 // bitmasks the router epilogue set and their
 // exclusive scans (tiny, recomputed by each CTA); CTA 0 publishes counts,
@@ -384,7 +456,8 @@ DG_DEVINL int warp_excl_scan8(int* vals8, int lane) {
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k_group_gather(GroupArgs a, const unsigned* __restrict__ mask,
                                                       unsigned* __restrict__ mask_next, int MW,
-                                                      const bf16* __restrict__ u, int d, bf16* __restrict__ xp) {
+                                                      const bf16* __restrict__ u, int d, bf16* __restrict__ xp,
+                                                      uint8_t* __restrict__ xq, float* __restrict__ xs) {
   pdl_trigger();
   pdl_wait();
   __shared__ int cnt[256];
@@ -481,6 +554,10 @@ __global__ void __launch_bounds__(256) k_group_gather(GroupArgs a, const unsigne
       a.row_weight[row] = a.w[p];
       a.row_pair[row] = p;
     }
+    if (xq != nullptr) {  // FP8 experts: the row is quantised on the way (same codes for every copy)
+      quant_row_warp(u + (size_t)t * d, d, xq + (size_t)row * d, xs + row, lane);
+      continue;
+    }
     const uint4* src = reinterpret_cast<const uint4*>(u + (size_t)t * d);
     uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)row * d);
     const int n16 = d / 8;
@@ -497,12 +574,14 @@ __global__ void __launch_bounds__(256) k_group_gather(GroupArgs a, const unsigne
 }
 
 cudaError_t run_route(const bf16* u, int d, bf16* xp, unsigned* mask, unsigned* mask_next, int MW,
-                      const GroupArgs& a, cudaStream_t st) {
+                      const GroupArgs& a, cudaStream_t st, uint8_t* xq, float* xs) {
   if (a.T < 1 || a.T > DG_MAX_REQUESTS * 256 || a.E > 256 || MW * 32 < a.T) return cudaErrorInvalidValue;
+  if (xq != nullptr && (d % 8 != 0 || d > 4096 || xs == nullptr)) return cudaErrorInvalidValue;
   const int P = a.T * a.k;
   const int grid = (P + 7) / 8 < 148 ? (P + 7) / 8 : 148;
   {
-    const cudaError_t e_ = launch_pdl(k_group_gather, dim3(grid), dim3(256), 0, st, a, mask, mask_next, MW, u, d, xp);
+    const cudaError_t e_ = launch_pdl(k_group_gather, dim3(grid), dim3(256), 0, st, a, mask, mask_next, MW, u, d, xp, xq,
+                                      xs);
     if (e_ != cudaSuccess) return e_;
   }
   return cudaGetLastError();

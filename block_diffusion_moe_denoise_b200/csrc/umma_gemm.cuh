@@ -157,7 +157,8 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
         if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1, abort_flag, err)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem + acc * P::BN;
-        const uint32_t idesc = umma_idesc_bf16(128, (uint32_t)t.n_mma);
+        const uint32_t idesc =
+            P::F8 ? umma_idesc_e4m3(128, (uint32_t)t.n_mma) : umma_idesc_bf16(128, (uint32_t)t.n_mma);
         bool ok = true;
         for (int kb = 0; kb < t.nk; kb += P::KB) {
           const int nsub = t.nk - kb < P::KB ? t.nk - kb : P::KB;
@@ -169,9 +170,14 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
           for (int j = 0; j < P::KB; ++j) {
             if (j < nsub) {
 #pragma unroll
-              for (int k = 0; k < 4; ++k)
-                umma_bf16(d_tmem, umma_sdesc_k128(a0 + j * kAStage + 32 * k),
-                          umma_sdesc_k128(b0 + j * P::B_STAGE + 32 * k), idesc, (kb | j | k) != 0 ? 1u : 0u);
+              for (int k = 0; k < 4; ++k) {
+                const uint64_t ad = umma_sdesc_k128(a0 + j * kAStage + 32 * k);
+                const uint64_t bd = umma_sdesc_k128(b0 + j * P::B_STAGE + 32 * k);
+                if constexpr (P::F8)
+                  umma_e4m3(d_tmem, ad, bd, idesc, (kb | j | k) != 0 ? 1u : 0u);
+                else
+                  umma_bf16(d_tmem, ad, bd, idesc, (kb | j | k) != 0 ? 1u : 0u);
+              }
             }
           }
           umma_commit(&empty[stage]);
@@ -218,6 +224,7 @@ struct ProblemBase {
   static constexpr int EP_SMEM = 0;
   static constexpr bool PRELOAD = false;  // true: static tiles, load_w / load_x split of load
   static constexpr int KB = 1;            // k-blocks per ring stage
+  static constexpr bool F8 = false;       // E4M3 operands (kind::f8f6f4): a k-block is 128 elements
   template <class Params>
   DG_DEVINL static void epilogue_init(const Params&, int, uint8_t*) {}
   template <class Params>

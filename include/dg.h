@@ -77,7 +77,20 @@ typedef struct dg_config {
   float temperature;   /* 0: candidates are the argmax; > 0: drawn from softmax(logits / temperature) */
   int ffn_selfcond;    /* self-conditioning gated-MLP width, a multiple of 64 (0: no self-conditioning) */
   int selfcond_topk;   /* softmax entries per position fed back, 1..8 (8) */
+  int expert_fp8;      /* 1: routed-expert weights are E4M3 codes with per-row scales (W8A8 GEMMs); 0: bf16 */
 } dg_config;
+
+/* FP8 routed experts (expert_fp8 = 1; the pages name FP8 and NVFP4
+ * checkpoints of the model without giving the scheme; this W8A8 reading is
+ * the library's).  w_gate, w_up and w_down hold E4M3 codes (one byte each, same
+ * shapes as the bf16 form) whose rows are scaled by w_gate_scale [E, fe],
+ * w_up_scale [E, fe] and w_down_scale [E, d] (fp32): W = decode(q) * scale.
+ * The token rows entering gate|up and the SwiGLU rows entering down are
+ * quantised per row: codes = E4M3(x * (448 / amax)) (round to nearest even,
+ * saturating), scale = amax / 448, amax = max |x| (fp32; a zero row gives
+ * zeros).  The tensor cores multiply the codes (kind::f8f6f4, fp32
+ * accumulation) and the epilogues apply both scales.  Everything else stays
+ * bf16. */
 
 /* Self-conditioning (pages: "DiffusionGemma hits ~1,500 TPS", "How the sampler
  * actually works": the previous step's softmax is fed back through a small
@@ -124,6 +137,7 @@ typedef struct dg_config {
 typedef struct dg_layer_weights {
   const void *attn_norm, *w_qkv, *w_o, *ffn_norm, *w_router;
   const void *w_gate, *w_up, *w_down, *ws_gate, *ws_up, *ws_down;
+  const void *w_gate_scale, *w_up_scale, *w_down_scale; /* fp32 row scales (expert_fp8 only, else NULL) */
 } dg_layer_weights;
 
 /* embed [vocab, d] bf16 (tied with the LM head), final_norm [d] f32,

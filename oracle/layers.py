@@ -100,6 +100,22 @@ def routed_experts(u: np.ndarray, idx: np.ndarray, w: np.ndarray, Wg, Wu, Wd) ->
     return y
 
 
+def routed_experts_fp8(u: np.ndarray, idx: np.ndarray, w: np.ndarray, Wg, Wu, Wd) -> np.ndarray:
+    """routed_experts with FP8 expert GEMMs (oracle/quant.py): the weights are the
+    dequantised E4M3 weights; each token's row is quantised per row before
+    gate|up, and each SwiGLU row before down."""
+    from .quant import fake_quant_rows
+    T, d = u.shape
+    out = np.zeros((T, d))
+    xq = fake_quant_rows(u)
+    for t in range(T):
+        for j in range(idx.shape[1]):
+            e = idx[t, j]
+            h = silu(xq[t] @ Wg[e].T) * (xq[t] @ Wu[e].T)
+            out[t] += w[t, j] * (fake_quant_rows(h[None, :])[0] @ Wd[e].T)
+    return out
+
+
 def histogram_and_permutation(idx: np.ndarray, n_experts: int):
     """Counts per expert, exclusive-scan offsets and the (token, slot) pairs
     grouped by expert, ordered by token inside each expert.

@@ -105,7 +105,8 @@ class Oracle:
             u = L_.rms_norm(x, w["ffn_norm"], c.norm_eps)
             r = u @ w["w_router"].T
             idx, wts = L_.route(r, c.top_k)
-            y = L_.routed_experts(u, idx, wts, w["w_gate"], w["w_up"], w["w_down"])
+            experts = L_.routed_experts_fp8 if getattr(c, "expert_fp8", 0) else L_.routed_experts
+            y = experts(u, idx, wts, w["w_gate"], w["w_up"], w["w_down"])
             ys = L_.swiglu(u, w["ws_gate"], w["ws_up"], w["ws_down"])
             if rec is not None:
                 rec.update(h=h, q=q, k=k, v=v, o=o, x_attn=x.copy(), u=u, router_logits=r,

@@ -39,6 +39,7 @@ class ModelConfig:
     temperature: float = 0.0       # 0: argmax candidates; > 0: candidates drawn from softmax(z / temperature)
     ffn_selfcond: int = 0          # self-conditioning gated-MLP width (0: off)
     selfcond_topk: int = 8         # softmax entries of the previous step fed back per position
+    expert_fp8: int = 0            # 1: routed-expert weights E4M3 with per-row scales, W8A8 GEMMs
 
     @property
     def qkv_rows(self) -> int:

@@ -21,6 +21,10 @@ Weight layout (row-major, "out x in" like a linear layer):
     ws_gate   [f_s, d]
     ws_up     [f_s, d]
     ws_down   [d, f_s]
+  FP8 checkpoint form (when expert_fp8): w_gate, w_up, w_down hold E4M3 codes
+    (uint8) of the bf16 draws divided by one float32 scale per output row
+    (largest magnitude -> 448), with w_gate_scale [E, f_e], w_up_scale [E, f_e],
+    w_down_scale [E, d]; the checkpoint is an input, like the bf16 weights.
   self-conditioning (when ffn_selfcond > 0):
     sc_gate   [f_sc, d]
     sc_up     [f_sc, d]
@@ -91,7 +95,26 @@ def make_layer(cfg: ModelConfig, layer: int, seed: int = 0, device="cpu", std=0.
             w[name] = _gain(shapes[name], s, device, gain_std)
         else:
             w[name] = _normal_bf16(shapes[name], s, device, std)
+    if getattr(cfg, "expert_fp8", 0):
+        for name in ("w_gate", "w_up", "w_down"):
+            w[name], w[name + "_scale"] = _to_e4m3_rows(w[name])
     return w
+
+
+def _to_e4m3_rows(t):
+    """E4M3 codes (uint8) and float32 per-row scales of a bf16 tensor (rows = last dim)."""
+    out = torch.empty(t.shape, dtype=torch.uint8, device=t.device)
+    scale = torch.empty(t.shape[:-1], dtype=torch.float32, device=t.device)
+    step = 1024
+    for e in range(t.shape[0]):
+        for r0 in range(0, t.shape[1], step):
+            x = t[e, r0:r0 + step].float()
+            amax = x.abs().amax(dim=-1)
+            sc = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+            q = (x / sc[:, None]).clamp(-448.0, 448.0).to(torch.float8_e4m3fn)
+            out[e, r0:r0 + step] = q.view(torch.uint8)
+            scale[e, r0:r0 + step] = torch.where(amax > 0, sc, torch.zeros_like(sc))
+    return out, scale
 
 
 def make_weights(cfg: ModelConfig, seed: int = 0, device="cpu", std=0.02, gain_std=0.0) -> dict:

@@ -11,11 +11,25 @@ def oracle_weights(w: dict) -> dict:
     out = {
         "embed": to_f64(w["embed"]),
         "final_norm": to_f64(w["final_norm"]),
-        "layers": [{k: to_f64(v) for k, v in lw.items()} for lw in w["layers"]],
+        "layers": [_layer_f64(lw) for lw in w["layers"]],
     }
     for name in ("sc_gate", "sc_up", "sc_down"):
         if name in w:
             out[name] = to_f64(w[name])
+    return out
+
+
+def _layer_f64(lw: dict) -> dict:
+    """float64 layer weights; FP8 expert weights (codes + per-row scales) dequantised exactly."""
+    from oracle.quant import e4m3_decode
+    out = {}
+    for k, v in lw.items():
+        if k.endswith("_scale"):
+            continue
+        if k + "_scale" in lw:
+            out[k] = e4m3_decode(v.cpu().numpy()) * to_f64(lw[k + "_scale"])[..., None]
+        else:
+            out[k] = to_f64(v)
     return out
 
 
