@@ -71,6 +71,7 @@ bool config_ok(const dg_config* c) {
   if (c->ffn_selfcond < 0 || c->ffn_selfcond % 64 != 0) return false;
   if (c->ffn_selfcond > 0 && (c->selfcond_topk < 1 || c->selfcond_topk > 8)) return false;
   if (c->expert_fp8 != 0 && c->expert_fp8 != 1) return false;
+  if (c->expert_fp8 && c->ffn_expert > 4096) return false;  // one warp quantises a row in registers
   return true;
 }
 
