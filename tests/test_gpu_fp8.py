@@ -53,11 +53,18 @@ def _buffers(h, cfg, T):
 
 
 def _check_quant(rows: torch.Tensor, codes: torch.Tensor, scale: torch.Tensor):
+    """Codes equal the library's E4M3 conversion; a value that rounds to zero may
+    carry either sign (the library keeps the sign of zero, the kernel's
+    conversion may not), so zeros compare by value."""
     x = rows.float()
     amax = x.abs().amax(dim=1)
     s_inv = 448.0 / amax
     ref = (x * s_inv[:, None]).to(torch.float8_e4m3fn).view(torch.uint8)
-    assert torch.equal(codes, ref)
+    same = (codes == ref) | (((codes & 0x7F) == 0) & ((ref & 0x7F) == 0))
+    if not bool(same.all()):
+        bad = (~same).nonzero()[:8]
+        info = [(int(r), int(c), float(x[r, c] * s_inv[r]), int(codes[r, c]), int(ref[r, c])) for r, c in bad.tolist()]
+        raise AssertionError(f"{int((~same).sum())} codes differ, e.g. (row, col, scaled value, kernel, library): {info}")
     assert torch.equal(scale, amax / 448.0)
 
 
@@ -65,16 +72,23 @@ def _check_gemms(cfg, lw, b, rows):
     """hp and yp of the sampled grouped rows against float64 products of the
     GEMMs' own codes and scales."""
     off = b["offsets"].cpu().numpy()
+    cache = {}
+
+    def weights(e):
+        if e not in cache:
+            cache[e] = [_decode(lw[n][e]) * lw[n + "_scale"][e].double().cpu().numpy()[:, None]
+                        for n in ("w_gate", "w_up", "w_down")]
+        return cache[e]
+
     for r in rows:
         e = int(np.searchsorted(off, r, side="right") - 1)
+        Wg, Wu, Wd = weights(e)
         x = _decode(b["xq"][r]) * float(b["xs"][r])
-        g = (_decode(lw["w_gate"][e]) * lw["w_gate_scale"][e].double().cpu().numpy()[:, None]) @ x
-        u = (_decode(lw["w_up"][e]) * lw["w_up_scale"][e].double().cpu().numpy()[:, None]) @ x
+        g, u = Wg @ x, Wu @ x
         hp_ref = g / (1 + np.exp(-g)) * u
         assert rel_l2(np64(b["hp"][r]), hp_ref) < 1e-2, r
         hrow = _decode(b["hq"][r]) * float(b["hs"][r])
-        y_ref = float(b["row_weight"][r]) * (
-            (_decode(lw["w_down"][e]) * lw["w_down_scale"][e].double().cpu().numpy()[:, None]) @ hrow)
+        y_ref = float(b["row_weight"][r]) * (Wd @ hrow)
         assert rel_l2(np64(b["yp"][r]), y_ref) < 1e-4, r
 
 
