@@ -412,7 +412,8 @@ def main():
     egu_avg_ms = egu_ms / max(1, egu_n)
     achieved = egu_bytes / (egu_avg_ms * 1e-3) / 1e9
     traffic = None
-    tpath = os.path.join(ROOT, "profiles", "experts_gate_up_traffic.json")
+    tname = "experts_gate_up_fp8_traffic.json" if getattr(cfg, "expert_fp8", 0) else "experts_gate_up_traffic.json"
+    tpath = os.path.join(ROOT, "profiles", tname)
     if os.path.exists(tpath):
         try:
             tj = json.load(open(tpath))
@@ -472,7 +473,8 @@ def main():
         "dtype": "bf16+e4m3" if getattr(cfg, "expert_fp8", 0) else "bf16",
         "data": "synthetic (seeded N(0,0.02) bf16 weights, uniform token ids)",
         "config": workload_config(cfg, args.workload, world),
-        "roofline": {"kernel": "experts_gate_up (routed-expert gate|up GEMM + SwiGLU)", "bound": "hbm",
+        "roofline": {"kernel": ("experts_gate_up (routed-expert gate|up GEMM + SwiGLU"
+                                + (", E4M3 W8A8)" if getattr(cfg, "expert_fp8", 0) else ")")), "bound": "hbm",
                      "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s", "frac": achieved / hbm_gbs,
                      "traffic": traffic, "algorithmic_bytes_per_launch": egu_bytes,
                      "avg_launch_ms": egu_avg_ms, "peak_source": f"{peak_kind} HBM copy (MEASURED_PEAKS.json)"},
