@@ -553,33 +553,51 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     LAUNCH(h, K_RMSNORM, 1,
            run_residual_norm(x, yp, pair_row, pending_k, part, pending_parts, h->Tcap, h->final_norm, TL, d,
                              c.norm_eps, hn, st));
-    LmArgs la;
-    la.tm_x = &h->tm_hn;
-    la.tm_embed = &h->tm_embed;
-    la.T = TL;
-    la.d = d;
-    la.num_sms = h->num_sms < kLmGridMax ? h->num_sms : kLmGridMax;
-    la.V = c.vocab;
-    la.part = h->B<float4>("lm_part");
-    la.logits = logits;
-    la.err = err;
     const bool draw = keys != nullptr && temperature > 0.f;
     const bool keep_sc = keys != nullptr && c.ffn_selfcond > 0;  // record this step's state for the next
-    la.inv_tau = draw ? 1.0f / temperature : 1.0f;
-    la.draw = draw ? h->B<float2>("draw") : nullptr;
-    memset(&la.keys, 0, sizeof(la.keys));
-    if (draw) la.keys = *keys;
-    la.sc_part = keep_sc ? h->B<float2>("sc_part") : nullptr;
-    int grid = 0;
-    LAUNCH(h, K_LM, 1, run_lm_head(la, &grid, st));
-    LAUNCH(h, K_LMC, 1,
-           run_lm_combine(h->B<float4>("lm_part"), grid, (TL + 127) / 128, TL, h->B<float>("stats"),
-                          h->B<int>("argmax"), err, st, la.draw, (int)(c.vocab / 256), draw ? keys : nullptr,
-                          draw ? h->B<int>("cand") : nullptr));
-    if (keep_sc)
-      LAUNCH(h, K_SC, 1,
-             run_selfcond_topk(la.sc_part, grid, TL, h->B<float>("stats"), *keys, c.selfcond_topk,
-                               h->B<float2>("sc_top"), err, st));
+    const int NV = (int)(c.vocab / 256);
+    // chunks of whole slots of at most kLmRowsMax rows; each chunk's draw keys
+    // start at its first slot, so all row indexing inside a chunk is local
+    const int chunk = kLmRowsMax / s.Tr * s.Tr;
+    for (int r0 = 0; r0 < TL; r0 += chunk) {
+      const int n = TL - r0 < chunk ? TL - r0 : chunk;
+      DrawKeys ck;
+      memset(&ck, 0, sizeof(ck));
+      if (keys != nullptr) {
+        const int slot0 = r0 / s.Tr;
+        ck.canvas = keys->canvas;
+        for (int i = 0; slot0 + i < DG_MAX_REQUESTS; ++i) {
+          ck.req[i] = keys->req[slot0 + i];
+          ck.block[i] = keys->block[slot0 + i];
+          ck.step[i] = keys->step[slot0 + i];
+          ck.seed[i] = keys->seed[slot0 + i];
+        }
+      }
+      LmArgs la;
+      la.tm_x = &h->tm_hn;
+      la.tm_embed = &h->tm_embed;
+      la.row0 = r0;
+      la.T = n;
+      la.d = d;
+      la.num_sms = h->num_sms < kLmGridMax ? h->num_sms : kLmGridMax;
+      la.V = c.vocab;
+      la.part = h->B<float4>("lm_part");
+      la.logits = logits ? logits + (size_t)r0 * c.vocab : nullptr;
+      la.err = err;
+      la.inv_tau = draw ? 1.0f / temperature : 1.0f;
+      la.draw = draw ? h->B<float2>("draw") + (size_t)r0 * NV : nullptr;
+      if (draw) la.keys = ck;
+      la.sc_part = keep_sc ? h->B<float2>("sc_part") : nullptr;
+      float* stats = h->B<float>("stats") + (size_t)r0 * 4;
+      int grid = 0;
+      LAUNCH(h, K_LM, 1, run_lm_head(la, &grid, st));
+      LAUNCH(h, K_LMC, 1,
+             run_lm_combine(h->B<float4>("lm_part"), grid, (n + 127) / 128, n, stats, h->B<int>("argmax") + r0, err,
+                            st, la.draw, NV, draw ? &ck : nullptr, draw ? h->B<int>("cand") + r0 : nullptr));
+      if (keep_sc)
+        LAUNCH(h, K_SC, 1,
+               run_selfcond_topk(la.sc_part, grid, n, stats, ck, c.selfcond_topk, h->B<float2>("sc_top"), err, st));
+    }
   } else if (pending_k || pending_parts) {
     // a pass stopped after a full layer: fold its expert outputs into x
     LAUNCH(h, K_RMSNORM, 1,

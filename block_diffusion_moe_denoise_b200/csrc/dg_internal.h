@@ -91,6 +91,10 @@ struct DrawKeys {
   unsigned long long seed[DG_MAX_REQUESTS];
 };
 
+// Rows one LM-head launch covers (its per-CTA statistics hold 8 token tiles);
+// larger passes run the LM head in chunks of whole slots.
+constexpr int kLmRowsMax = 1024;
+
 struct LmArgs {
   const CUtensorMap* tm_x;
   const CUtensorMap* tm_embed;
@@ -104,6 +108,7 @@ struct LmArgs {
   float2* draw = nullptr;    // [T][V/256]: (log-mass of the tile at 1/temperature, drawn id in the tile)
   DrawKeys keys = {};
   float2* sc_part = nullptr; // self-conditioning: per-CTA top-8 logits [grid][T][8] (logit, id bits)
+  int row0 = 0;              // first row of tm_x this launch reads (its rows are row0 .. row0+T-1)
 };
 
 cudaError_t run_qkv(const QkvArgs& a, cudaStream_t st);

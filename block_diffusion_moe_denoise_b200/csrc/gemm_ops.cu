@@ -742,6 +742,7 @@ struct P_LM : ProblemBase {
     float2* draw;    // optional [T][NV]
     DrawKeys keys;
     float2* sc_part; // optional [gridDim.x][T][SC_K] (logit, id as int bits)
+    int row0;        // row of tmX holding this launch's row 0
   };
   DG_DEVINL static void prefetch(const Params& p) {
     tma_prefetch_desc(&p.tmX);
@@ -805,7 +806,7 @@ struct P_LM : ProblemBase {
     tma_load_2d(sb, &p.tmE, kb * 64, t.b * 256, bar);
   }
   DG_DEVINL static void load_x(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t, uint64_t* bar) {
-    tma_load_2d(sa, &p.tmX, kb * 64, t.a * 128, bar);
+    tma_load_2d(sa, &p.tmX, kb * 64, p.row0 + t.a * 128, bar);
   }
   DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
     load_x(p, t, kb, sa, sb, bar);
@@ -1089,7 +1090,9 @@ cudaError_t run_lm_head(const LmArgs& a, int* grid_out, cudaStream_t st) {
   p.draw = a.draw;
   p.keys = a.keys;
   p.sc_part = a.sc_part;
-  if (p.MT > P_LM::MT_MAX) return cudaErrorInvalidValue;
+  p.row0 = a.row0;
+  static_assert(P_LM::MT_MAX * 128 == kLmRowsMax, "LM-head chunk size");
+  if (p.MT > P_LM::MT_MAX || a.row0 < 0) return cudaErrorInvalidValue;
   if (p.draw != nullptr && (p.keys.canvas < 1 || (p.T + p.keys.canvas - 1) / p.keys.canvas > DG_MAX_REQUESTS))
     return cudaErrorInvalidValue;
   int grid = grid_for(p.MT * p.NV, a.num_sms);

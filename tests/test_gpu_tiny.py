@@ -447,3 +447,35 @@ def test_selfcond_teacher_forced_steps():
     assert rel_l2(st2_plain["entropy"], st2["entropy"]) > 5 * REL_L2
     h.close()
     h0.close()
+
+
+def test_eight_requests_in_one_step(model):
+    """A step over eight requests (2,048 canvas rows: the LM head runs in two
+    chunks of four slots) gives each request the statistics it gets alone, and
+    with a temperature the drawn tokens too."""
+    dgm, wd, _ = model
+    for tau in (0.0, 0.7):
+        cfg = CFG.with_(temperature=tau)
+        h = dgm.DG(cfg, wd, max_requests=8, kv_capacity=1024)
+        h1 = dgm.DG(cfg, wd, max_requests=8, kv_capacity=1024)
+        for r in range(8):
+            for hh in (h, h1):
+                hh.prefill(r, make_tokens(CFG, 64 + 16 * r, seed=40 + r).cuda())
+                hh.open_canvas(r, 11 + r, 0)
+        h.denoise_step(list(range(8)))
+        for r in range(8):
+            h1.denoise_step([r])
+        for r in range(8):
+            tok, mask, st, am = h.get_canvas(r)
+            tok1, mask1, st1, am1 = h1.get_canvas(r)
+            np.testing.assert_allclose(st.cpu().numpy(), st1.cpu().numpy(), rtol=1e-5, atol=1e-5)
+            assert torch.equal(mask, mask1) and torch.equal(am, am1), r
+            if tau > 0:
+                # a draw can move only where a batched logit moved it across an interval edge
+                assert (tok != tok1).float().mean() < 0.02, r
+            else:
+                assert torch.equal(tok, tok1), r
+        h.sync()
+        h1.sync()
+        h.close()
+        h1.close()
