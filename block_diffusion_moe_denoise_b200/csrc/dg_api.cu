@@ -37,6 +37,7 @@ struct ReqState {
   unsigned long long seed = 0;
   bool open = false;
   int last_slot = 0;
+  long long stats_seq = -1;  // LM-head pass whose statistics are this request's last step
   bool sc_valid = false;  // "sc_top" holds this canvas's previous-step self-conditioning state
 };
 
@@ -259,6 +260,7 @@ struct dg_handle {
   long long cap_user = 0;  // capacity the caller asked for (cap is rounded up to 64)
   ReqState req[DG_MAX_REQUESTS];
   int mask_flip = 0;  // which of the two routing bitmask buffers the next layer uses
+  long long lm_seq = 0;  // LM-head passes so far: the "stats" / "argmax" buffers hold the latest
 
   template <class T>
   T* B(const char* name) const {
@@ -550,6 +552,7 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     pending_parts = ss;
   }
   if (want_lm) {
+    ++h->lm_seq;
     LAUNCH(h, K_RMSNORM, 1,
            run_residual_norm(x, yp, pair_row, pending_k, part, pending_parts, h->Tcap, h->final_norm, TL, d,
                              c.norm_eps, hn, st));
@@ -977,6 +980,7 @@ int dg_denoise_step(dg_handle* h, int n_req, const int* reqs, int32_t* d_remaini
   for (int i = 0; i < n_req; ++i) {
     h->req[reqs[i]].step = steps[i];
     h->req[reqs[i]].last_slot = i;
+    h->req[reqs[i]].stats_seq = h->lm_seq;
     if (d_remaining)
       CK(cudaMemcpyAsync(d_remaining + i, h->B<int>("remaining") + reqs[i], 4, cudaMemcpyDeviceToDevice, h->st));
   }
@@ -1067,12 +1071,24 @@ int dg_get_canvas(dg_handle* h, int req, int32_t* d_tokens, uint8_t* d_mask, flo
   if (d_mask)
     CK(cudaMemcpyAsync(d_mask, h->B<unsigned char>("mask") + (size_t)req * C, (size_t)C, cudaMemcpyDeviceToDevice,
                        h->st));
-  if (d_stats)
-    CK(cudaMemcpyAsync(d_stats, h->B<float>("stats") + (size_t)r.last_slot * C * 4, (size_t)C * 16,
-                       cudaMemcpyDeviceToDevice, h->st));
-  if (d_argmax)
-    CK(cudaMemcpyAsync(d_argmax, h->B<int>("argmax") + (size_t)r.last_slot * C, (size_t)C * 4,
-                       cudaMemcpyDeviceToDevice, h->st));
+  // the statistics buffers hold the latest LM-head pass only: another
+  // request's step, an LM-head operation or a full debug pass since this
+  // request's last step has overwritten them (NaN / -1 then)
+  const bool current = r.stats_seq == h->lm_seq;
+  if (d_stats) {
+    if (current)
+      CK(cudaMemcpyAsync(d_stats, h->B<float>("stats") + (size_t)r.last_slot * C * 4, (size_t)C * 16,
+                         cudaMemcpyDeviceToDevice, h->st));
+    else
+      CK(cudaMemsetAsync(d_stats, 0xFF, (size_t)C * 16, h->st));
+  }
+  if (d_argmax) {
+    if (current)
+      CK(cudaMemcpyAsync(d_argmax, h->B<int>("argmax") + (size_t)r.last_slot * C, (size_t)C * 4,
+                         cudaMemcpyDeviceToDevice, h->st));
+    else
+      CK(cudaMemsetAsync(d_argmax, 0xFF, (size_t)C * 4, h->st));
+  }
   return DG_OK;
 }
 
@@ -1168,6 +1184,7 @@ int dg_op_lm_head(dg_handle* h, const float* d_x, int T, float* d_stats, int32_t
   la.part = h->B<float4>("lm_part");
   la.logits = d_logits;
   la.err = h->B<int>("err");
+  ++h->lm_seq;
   int grid = 0;
   CK(run_lm_head(la, &grid, h->st));
   CK(run_lm_combine(la.part, grid, (T + 127) / 128, T, h->B<float>("stats"), h->B<int>("argmax"), la.err, h->st));
@@ -1205,6 +1222,7 @@ int dg_op_lm_sample(dg_handle* h, const float* d_x, int T, float temperature, ui
   la.inv_tau = 1.0f / temperature;
   la.draw = h->B<float2>("draw");
   la.keys = keys;
+  ++h->lm_seq;
   int grid = 0;
   CK(run_lm_head(la, &grid, h->st));
   CK(run_lm_combine(la.part, grid, (T + 127) / 128, T, h->B<float>("stats"), h->B<int>("argmax"), la.err, h->st,
@@ -1239,6 +1257,7 @@ int dg_op_selfcond(dg_handle* h, int request, const float* d_x, int T, float* d_
   la.logits = nullptr;
   la.err = err;
   la.sc_part = h->B<float2>("sc_part");
+  ++h->lm_seq;
   int grid = 0;
   CK(run_lm_head(la, &grid, h->st));
   CK(run_lm_combine(la.part, grid, (T + 127) / 128, T, h->B<float>("stats"), h->B<int>("argmax"), err, h->st));

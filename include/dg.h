@@ -228,7 +228,10 @@ int dg_generate(dg_handle* h, int req, const int32_t* h_prompt, int n_prompt, in
 /* Copy the open canvas of `req`: tokens [canvas] int32, accepted mask [canvas]
  * u8 (1 = frozen), and the last step's statistics for its positions:
  * d_stats [canvas][4] f32 = (entropy nats, log max-probability, max logit,
- * log-partition), d_argmax [canvas] int32.  Any output pointer may be NULL. */
+ * log-partition), d_argmax [canvas] int32.  Any output pointer may be NULL.
+ * The statistics are kept for the latest LM-head pass of the handle only: if
+ * another denoising step, an LM-head operation or a full debug pass ran after
+ * this request's last step, d_stats is filled with NaN and d_argmax with -1. */
 int dg_get_canvas(dg_handle* h, int req, int32_t* d_tokens, uint8_t* d_mask, float* d_stats, int32_t* d_argmax);
 
 /* Replace the open canvas of `req` (tokens, accepted mask) and its step counter. */

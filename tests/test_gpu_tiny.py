@@ -463,11 +463,15 @@ def test_eight_requests_in_one_step(model):
                 hh.prefill(r, make_tokens(CFG, 64 + 16 * r, seed=40 + r).cuda())
                 hh.open_canvas(r, 11 + r, 0)
         h.denoise_step(list(range(8)))
+        alone = []
         for r in range(8):
             h1.denoise_step([r])
+            alone.append([t.clone() for t in h1.get_canvas(r)])   # statistics of the latest pass only
+        _, _, stale, stale_am = h1.get_canvas(0)
+        assert torch.isnan(stale).all() and (stale_am == -1).all()
         for r in range(8):
             tok, mask, st, am = h.get_canvas(r)
-            tok1, mask1, st1, am1 = h1.get_canvas(r)
+            tok1, mask1, st1, am1 = alone[r]
             # logits are bit-identical; the LM head's per-row sums merge its
             # vocabulary tiles in a grid-dependent order (last-bit differences)
             np.testing.assert_allclose(st.cpu().numpy(), st1.cpu().numpy(), rtol=1e-5, atol=1e-5)
