@@ -124,6 +124,21 @@ class ClockSampler:
                 "samples": len(loaded), "power_w_max": max(r[2] for r in rows)}
 
 
+def kernel_source_digest(problem: str) -> str:
+    """sha256 over the source a routed-expert GEMM is built from: its problem
+    struct in gemm_ops.cu, the GEMM engine and the shared device helpers.  A
+    stored ncu traffic ratio is used only while this digest is unchanged."""
+    import hashlib
+    csrc = os.path.join(ROOT, "block_diffusion_moe_denoise_b200", "csrc")
+    text = open(os.path.join(csrc, "gemm_ops.cu")).read()
+    start = text.index(f"struct {problem} : ProblemBase {{")
+    body = text[start:text.index("\n};\n", start) + 4]
+    h = hashlib.sha256(body.encode())
+    for f in ("umma_gemm.cuh", "common.cuh"):
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()
+
+
 # ---------------------------------------------------------------------------
 # algorithmic work
 # ---------------------------------------------------------------------------
@@ -417,13 +432,11 @@ def main():
     if os.path.exists(tpath):
         try:
             tj = json.load(open(tpath))
-            import hashlib
-            src = open(os.path.join(ROOT, "block_diffusion_moe_denoise_b200", "csrc", "gemm_ops.cu"), "rb").read()
-            src += open(os.path.join(ROOT, "block_diffusion_moe_denoise_b200", "csrc", "umma_gemm.cuh"), "rb").read()
+            src = kernel_source_digest("P_EGU8" if getattr(cfg, "expert_fp8", 0) else "P_EGU")
             # The capture is a smaller case (one layer, 124 experts touched); DRAM
             # traffic grows in proportion to the expert weights streamed, so it is
             # scaled to this launch by its algorithmic bytes.
-            if tj.get("source_sha256") == hashlib.sha256(src).hexdigest():
+            if tj.get("source_sha256") == src:
                 traffic = tj["traffic_per_algorithmic_byte"] * egu_bytes
         except Exception:
             traffic = None
