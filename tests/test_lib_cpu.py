@@ -69,3 +69,37 @@ def test_host_validation_without_gpu(lib):
     assert L.dg_prefill(None, 0, None, 0) == -1
     assert L.dg_op_lm_sample(None, None, 4, 0.7, 1, 0, 1, 0, None, None, None) == -1
     assert L.dg_op_selfcond(None, 0, None, 4, None, None) == -1
+
+
+def _c_struct_fields(name):
+    """(field, C type) in declaration order of `typedef struct name {...} name;` in dg.h."""
+    src = open(os.path.join(ROOT, "include", "dg.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    body = re.search(r"typedef struct " + name + r" \{(.*?)\} " + name + ";", src, flags=re.S).group(1)
+    out = []
+    for decl in body.split(";"):
+        decl = decl.strip()
+        if not decl:
+            continue
+        m = re.match(r"(const\s+)?(int|float|void|int64_t|const dg_layer_weights)\s*(.*)", decl, flags=re.S)
+        base = ("const " if m.group(1) else "") + m.group(2)
+        for part in m.group(3).split(","):
+            part = part.strip()
+            ptr = part.startswith("*")
+            out.append((part.lstrip("*").strip(), base + ("*" if ptr else "")))
+    return out
+
+
+def test_ctypes_structs_match_the_header():
+    """The binding's ctypes structures declare the header's fields, in order, with
+    matching types (an ABI drift check that needs no GPU)."""
+    import ctypes as C
+    from block_diffusion_moe_denoise_b200 import _ffi
+    ctype = {"int": C.c_int, "float": C.c_float, "const void*": C.c_void_p}
+    for name, cls in (("dg_config", _ffi.dg_config), ("dg_layer_weights", _ffi.dg_layer_weights)):
+        fields = _c_struct_fields(name)
+        assert [f for f, _ in fields] == [f for f, _ in cls._fields_], name
+        for (f, t), (_, ct) in zip(fields, cls._fields_):
+            assert ctype[t] is ct, (name, f, t)
+    w = _c_struct_fields("dg_weights")
+    assert [f for f, _ in w] == [f for f, _ in _ffi.dg_weights._fields_]
