@@ -23,7 +23,10 @@ Pages cited (by title; the section follows in each citation):
 
 Where the pages are silent the plainest reading is taken; each reading is named
 where it is used.  Pinned by tests/test_oracle_*.py (brute force, closed forms,
-invariants, a library cross-check of the Philox round structure).  Model-level
+invariants, a library cross-check of the Philox round structure, of the E4M3
+codec against the library float8 type, an exact rational brute force and a
+chi-square test of the candidate draw, closed forms and invariances of the
+self-conditioning term).  Model-level
 end-to-end values have no printed worked example in the pages: that level is
 pinned only through the invariants (frozen tokens, >= min_accept accepted per
 step, convergence within the step cap, commit == prefill, permutation

@@ -1,7 +1,8 @@
 """FP8 (E4M3) expert weights and activations.
 
 The pages name FP8 and NVFP4 checkpoints of the model ([P2] "Serve it with
-vLLM"; [P1] and [P4] on the quantised variants) without giving the scheme.
+vLLM") and a quantised model that fits 18 GB ([P1] "26B MoE Architecture, but
+Only 3.8B Activated"; [P4] "What's new") without giving the scheme.
 Reading taken (the common W8A8 form): expert weights are stored as E4M3 codes
 with one float32 scale per output row (W = decode(q) * scale); the expert
 inputs -- the normalised token rows entering gate|up and the SwiGLU rows
