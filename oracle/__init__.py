@@ -32,4 +32,4 @@ pinned only through the invariants (frozen tokens, >= min_accept accepted per
 step, convergence within the step cap, commit == prefill, permutation
 equivariance) and through the per-part pins.
 """
-from . import layers, model, philox, sampler  # noqa: F401
+from . import layers, model, philox, quant, sampler  # noqa: F401
