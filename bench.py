@@ -463,7 +463,9 @@ def main():
                "steps_per_canvas": gen_steps}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    # the oracle sample is the headline workload's; the variants have none
+    variant = args.temperature > 0 or args.selfcond > 0 or args.fp8_experts
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not variant:
         s = oracle_sample(reps=3, warm=1, min_seconds=10.0)
         cpu = {k: s[k] for k in ("value", "unit", "cores", "kind", "sample")}
 

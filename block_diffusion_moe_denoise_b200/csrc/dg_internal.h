@@ -81,8 +81,9 @@ struct SharedArgs {
   unsigned* mask;     // [E][MW] per-expert token bitmasks, zero on entry
   int* err;
 };
-// Keys of the candidate draw: LM-head row r is position r % canvas of slot
-// r / canvas, drawn with that slot's (seed, block, step, request).
+// Per-slot keys of the LM-head rows: row r is position r % canvas of slot
+// r / canvas.  The candidate draw uses the slot's (seed, block, step,
+// request); the self-conditioning state is stored under its request.
 struct DrawKeys {
   int canvas;
   int req[DG_MAX_REQUESTS];
