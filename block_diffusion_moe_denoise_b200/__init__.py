@@ -22,6 +22,42 @@ def _ptr(t):
     return None if t is None else C.c_void_p(t.data_ptr())
 
 
+def _check(t, name: str, dtype, device: bool, numel: int | None = None, shape=None):
+    """Reject, before any C call, a tensor the C ABI cannot take: host memory
+    where device memory is expected (or the reverse), another element type, a
+    non-contiguous view, or fewer elements than the call reads.  A wrong
+    pointer would otherwise reach a kernel as an out-of-range address."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor")
+    if bool(t.is_cuda) != device:
+        raise ValueError(f"{name}: expected {'device (CUDA)' if device else 'host'} memory, got {t.device}")
+    dtypes = dtype if isinstance(dtype, tuple) else (dtype,)
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name}: expected dtype {' or '.join(str(d) for d in dtypes)}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous tensor")
+    if numel is not None and t.numel() < numel:
+        raise ValueError(f"{name}: expected at least {numel} elements, got {t.numel()}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t
+
+
+def _dev(t, name: str, dtype, numel: int | None = None, shape=None, optional: bool = False):
+    """Device pointer of a checked CUDA tensor (None for an optional None)."""
+    if t is None and optional:
+        return None
+    return C.c_void_p(_check(t, name, dtype, True, numel, shape).data_ptr())
+
+
+def _host(t, name: str, dtype, numel: int | None = None):
+    """Host pointer of a checked CPU tensor."""
+    return C.c_void_p(_check(t, name, dtype, False, numel).data_ptr())
+
+
+_F32, _I32, _U8, _BF16 = torch.float32, torch.int32, torch.uint8, torch.bfloat16
+
+
 def _stream(stream):
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -41,14 +77,14 @@ def config_struct(cfg) -> dg_config:
 
 def philox_tokens(seed: int, block: int, step: int, request: int, pos0: int, n: int, vocab: int,
                   out: torch.Tensor, stream=None) -> None:
-    check(_ffi.load().dg_op_philox_tokens(seed, block, step, request, pos0, n, vocab, _ptr(out), _stream(stream)),
-          "dg_op_philox_tokens")
+    check(_ffi.load().dg_op_philox_tokens(seed, block, step, request, pos0, n, vocab, _dev(out, "out", _I32, n),
+                                          _stream(stream)), "dg_op_philox_tokens")
 
 
 def route_topk(logits: torch.Tensor, k: int, idx: torch.Tensor, w: torch.Tensor, stream=None) -> None:
     T, E = logits.shape
-    check(_ffi.load().dg_op_route_topk(_ptr(logits), T, E, k, _ptr(idx), _ptr(w), _stream(stream)),
-          "dg_op_route_topk")
+    check(_ffi.load().dg_op_route_topk(_dev(logits, "logits", _F32), T, E, k, _dev(idx, "idx", _I32, T * k),
+                                       _dev(w, "w", _F32, T * k), _stream(stream)), "dg_op_route_topk")
 
 
 def lm_head_noalloc(x: torch.Tensor, final_norm: torch.Tensor, embed: torch.Tensor, norm_eps: float,
@@ -56,9 +92,10 @@ def lm_head_noalloc(x: torch.Tensor, final_norm: torch.Tensor, embed: torch.Tens
     """dg_op_lm_head_noalloc: LM-head statistics with the library's built-in
     scratch (no workspace, no allocation inside)."""
     T, d = x.shape
-    check(_ffi.load().dg_op_lm_head_noalloc(_ptr(x), _ptr(final_norm), _ptr(embed), T, d, embed.shape[0], norm_eps,
-                                            _ptr(stats), _ptr(argmax), _ptr(err), _stream(stream)),
-          "dg_op_lm_head_noalloc")
+    check(_ffi.load().dg_op_lm_head_noalloc(
+        _dev(x, "x", _F32), _dev(final_norm, "final_norm", _F32, d), _dev(embed, "embed", _BF16), T, d,
+        embed.shape[0], norm_eps, _dev(stats, "stats", _F32, T * 4), _dev(argmax, "argmax", _I32, T),
+        _dev(err, "err", _I32, 1, optional=True), _stream(stream)), "dg_op_lm_head_noalloc")
 
 
 class DG:
@@ -71,14 +108,26 @@ class DG:
         self.c_cfg = config_struct(cfg)
         self.weights = weights            # keep the tensors alive
         self.stream = stream or torch.cuda.current_stream(device)
+        if len(weights["layers"]) != cfg.n_layers:
+            raise ValueError(f"weights: {len(weights['layers'])} layers for a {cfg.n_layers}-layer configuration")
+        fp8 = bool(getattr(cfg, "expert_fp8", 0))
         layers = (dg_layer_weights * cfg.n_layers)()
         for i, lw in enumerate(weights["layers"]):
-            layers[i] = dg_layer_weights(*[lw[n].data_ptr() if n in lw else None for n in (
-                "attn_norm", "w_qkv", "w_o", "ffn_norm", "w_router", "w_gate", "w_up", "w_down", "ws_gate",
-                "ws_up", "ws_down", "w_gate_scale", "w_up_scale", "w_down_scale")])
+            ptrs = []
+            for n in ("attn_norm", "w_qkv", "w_o", "ffn_norm", "w_router", "w_gate", "w_up", "w_down", "ws_gate",
+                      "ws_up", "ws_down", "w_gate_scale", "w_up_scale", "w_down_scale"):
+                if n.endswith("_scale") and not fp8:
+                    ptrs.append(None)
+                    continue
+                dt = _F32 if n.endswith("norm") or n.endswith("_scale") else (
+                    _U8 if fp8 and n in ("w_gate", "w_up", "w_down") else _BF16)
+                ptrs.append(_check(lw[n], f"layers[{i}].{n}", dt, True).data_ptr())
+            layers[i] = dg_layer_weights(*ptrs)
         self._layers = layers
-        sc = [weights[n].data_ptr() if n in weights else None for n in ("sc_gate", "sc_up", "sc_down")]
-        self.c_w = dg_weights(weights["embed"].data_ptr(), weights["final_norm"].data_ptr(), layers, *sc)
+        sc = [_check(weights[n], n, _BF16, True).data_ptr() if getattr(cfg, "ffn_selfcond", 0) > 0 else None
+              for n in ("sc_gate", "sc_up", "sc_down")]
+        self.c_w = dg_weights(_check(weights["embed"], "embed", _BF16, True).data_ptr(),
+                              _check(weights["final_norm"], "final_norm", _F32, True).data_ptr(), layers, *sc)
         nbytes = lib.dg_workspace_size(C.byref(self.c_cfg), max_requests, kv_capacity)
         if nbytes == 0:
             raise DGError(-1, "dg_workspace_size")
@@ -106,10 +155,12 @@ class DG:
 
     # ---- the C ABI, same names ----
     def prefill(self, req: int, tokens: torch.Tensor):
-        check(self.lib.dg_prefill(self.h, req, _ptr(tokens), tokens.numel()), "dg_prefill")
+        check(self.lib.dg_prefill(self.h, req, _dev(tokens, "tokens", _I32), tokens.numel()), "dg_prefill")
 
     def set_kv(self, req: int, layer: int, pos0: int, k: torch.Tensor, v: torch.Tensor):
-        check(self.lib.dg_set_kv(self.h, req, layer, pos0, k.shape[1], _ptr(k), _ptr(v)), "dg_set_kv")
+        shape = (self.cfg.n_kv_heads, k.shape[1] if k.dim() == 3 else -1, self.cfg.head_dim)
+        check(self.lib.dg_set_kv(self.h, req, layer, pos0, shape[1], _dev(k, "k", _BF16, shape=shape),
+                                 _dev(v, "v", _BF16, shape=shape)), "dg_set_kv")
 
     def get_kv(self, req: int, layer: int, pos0: int, n: int):
         c = self.cfg
@@ -129,7 +180,9 @@ class DG:
 
     def denoise_step(self, reqs, d_remaining: torch.Tensor | None = None):
         arr = (C.c_int * len(reqs))(*reqs)
-        check(self.lib.dg_denoise_step(self.h, len(reqs), arr, _ptr(d_remaining)), "dg_denoise_step")
+        check(self.lib.dg_denoise_step(self.h, len(reqs), arr,
+                                       _dev(d_remaining, "d_remaining", _I32, len(reqs), optional=True)),
+              "dg_denoise_step")
 
     def read_remaining(self, req: int) -> int:
         r = C.c_int32()
@@ -142,8 +195,8 @@ class DG:
     def generate(self, req: int, prompt_host: torch.Tensor, n_out: int, seed: int, out_host: torch.Tensor):
         n_blocks = n_out // self.cfg.canvas
         steps = (C.c_int * max(1, n_blocks))()
-        check(self.lib.dg_generate(self.h, req, C.c_void_p(prompt_host.data_ptr()), prompt_host.numel(), n_out, seed,
-                                   C.c_void_p(out_host.data_ptr()), steps), "dg_generate")
+        check(self.lib.dg_generate(self.h, req, _host(prompt_host, "prompt_host", _I32), prompt_host.numel(), n_out,
+                                   seed, _host(out_host, "out_host", _I32, n_out), steps), "dg_generate")
         return list(steps)[:n_blocks]
 
     def get_canvas(self, req: int):
@@ -157,7 +210,9 @@ class DG:
         return tok, mask, stats, am
 
     def set_canvas(self, req: int, tokens: torch.Tensor, mask: torch.Tensor, step: int):
-        check(self.lib.dg_set_canvas(self.h, req, _ptr(tokens), _ptr(mask), step), "dg_set_canvas")
+        C_ = self.cfg.canvas
+        check(self.lib.dg_set_canvas(self.h, req, _dev(tokens, "tokens", _I32, C_), _dev(mask, "mask", _U8, C_), step),
+              "dg_set_canvas")
 
     def sync(self):
         check(self.lib.dg_sync(self.h), "dg_sync")
@@ -170,12 +225,15 @@ class DG:
         counts = torch.empty(E, dtype=torch.int32, device=dev)
         offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
         perm = torch.empty(idx.numel(), dtype=torch.int32, device=dev)
-        check(self.lib.dg_op_route_group(self.h, _ptr(idx), _ptr(w), T, _ptr(counts), _ptr(offsets), _ptr(perm)),
-              "dg_op_route_group")
+        k = self.cfg.top_k
+        check(self.lib.dg_op_route_group(self.h, _dev(idx, "idx", _I32, shape=(T, k)), _dev(w, "w", _F32, shape=(T, k)),
+                                         T, _ptr(counts), _ptr(offsets), _ptr(perm)), "dg_op_route_group")
         return counts, offsets, perm
 
     def op_sample(self, req: int, entropy, logconf, argmax, step: int):
-        check(self.lib.dg_op_sample(self.h, req, _ptr(entropy), _ptr(logconf), _ptr(argmax), step), "dg_op_sample")
+        C_ = self.cfg.canvas
+        check(self.lib.dg_op_sample(self.h, req, _dev(entropy, "entropy", _F32, C_), _dev(logconf, "logconf", _F32, C_),
+                                    _dev(argmax, "argmax", _I32, C_), step), "dg_op_sample")
 
     def op_lm_head(self, x: torch.Tensor, want_logits: bool = False):
         T = x.shape[0]
@@ -183,7 +241,8 @@ class DG:
         stats = torch.empty((T, 4), dtype=torch.float32, device=dev)
         am = torch.empty(T, dtype=torch.int32, device=dev)
         logits = torch.empty((T, self.cfg.vocab), dtype=torch.float32, device=dev) if want_logits else None
-        check(self.lib.dg_op_lm_head(self.h, _ptr(x), T, _ptr(stats), _ptr(am), _ptr(logits)), "dg_op_lm_head")
+        check(self.lib.dg_op_lm_head(self.h, _dev(x, "x", _F32, shape=(T, self.cfg.d_model)), T, _ptr(stats), _ptr(am),
+                                     _ptr(logits)), "dg_op_lm_head")
         return stats, am, logits
 
     def op_lm_sample(self, x: torch.Tensor, temperature: float, seed: int, block: int, step: int, request: int = 0):
@@ -193,8 +252,8 @@ class DG:
         stats = torch.empty((T, 4), dtype=torch.float32, device=dev)
         am = torch.empty(T, dtype=torch.int32, device=dev)
         cand = torch.empty(T, dtype=torch.int32, device=dev)
-        check(self.lib.dg_op_lm_sample(self.h, _ptr(x), T, temperature, seed, block, step, request, _ptr(stats),
-                                       _ptr(am), _ptr(cand)), "dg_op_lm_sample")
+        check(self.lib.dg_op_lm_sample(self.h, _dev(x, "x", _F32, shape=(T, self.cfg.d_model)), T, temperature, seed,
+                                       block, step, request, _ptr(stats), _ptr(am), _ptr(cand)), "dg_op_lm_sample")
         return stats, am, cand
 
     def op_selfcond(self, request: int, x: torch.Tensor):
@@ -203,7 +262,8 @@ class DG:
         T, d = x.shape
         sc = torch.empty((T, d), dtype=torch.float32, device=x.device)
         top = torch.empty((T, 8, 2), dtype=torch.float32, device=x.device)
-        check(self.lib.dg_op_selfcond(self.h, request, _ptr(x), T, _ptr(sc), _ptr(top)), "dg_op_selfcond")
+        check(self.lib.dg_op_selfcond(self.h, request, _dev(x, "x", _F32, shape=(T, self.cfg.d_model)), T, _ptr(sc),
+                                      _ptr(top)), "dg_op_selfcond")
         return sc, top[..., 0], top.view(torch.int32)[..., 1]
 
     KERNEL_CLASSES = ("embed", "rmsnorm", "qkv", "attention", "oproj", "group",
@@ -225,7 +285,8 @@ class DG:
         return self.lib.dg_launch_count(self.h)
 
     def debug_forward(self, req: int, tokens: torch.Tensor, n_layers: int):
-        check(self.lib.dg_debug_forward(self.h, req, _ptr(tokens), tokens.numel(), n_layers), "dg_debug_forward")
+        check(self.lib.dg_debug_forward(self.h, req, _dev(tokens, "tokens", _I32), tokens.numel(), n_layers),
+              "dg_debug_forward")
 
     def token_capacity(self) -> int:
         """Rows of the per-pass token buffers (the middle extent of "q")."""

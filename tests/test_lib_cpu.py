@@ -103,3 +103,47 @@ def test_ctypes_structs_match_the_header():
             assert ctype[t] is ct, (name, f, t)
     w = _c_struct_fields("dg_weights")
     assert [f for f, _ in w] == [f for f, _ in _ffi.dg_weights._fields_]
+
+
+def test_binding_rejects_unusable_tensors_before_any_call():
+    """Host memory where the C ABI wants device memory, a wrong element type, a
+    non-contiguous view or too few elements raise in Python, before any C call
+    could hand a bad address to a kernel."""
+    import torch
+    import block_diffusion_moe_denoise_b200 as dgm
+    from block_diffusion_moe_denoise_b200 import _check, _host
+    from synth import TINY
+
+    class NoCalls:                       # a library whose every entry point fails the test
+        def __getattr__(self, name):
+            def call(*args):
+                raise AssertionError(f"{name} was called")
+            return call
+
+    h = object.__new__(dgm.DG)          # no device here: only the argument checks run
+    h.cfg, h.lib, h.h = TINY, NoCalls(), None
+    with pytest.raises(ValueError, match="device"):
+        h.prefill(0, torch.zeros(16, dtype=torch.int32))
+    with pytest.raises(ValueError, match="device"):
+        h.set_canvas(0, torch.zeros(256, dtype=torch.int32), torch.zeros(256, dtype=torch.uint8), 1)
+    with pytest.raises(ValueError, match="device"):
+        h.op_lm_head(torch.zeros((4, TINY.d_model)))
+    import block_diffusion_moe_denoise_b200._ffi as ffi
+    real_load = ffi.load
+    ffi.load = lambda: NoCalls()
+    try:
+        with pytest.raises(ValueError, match="device"):
+            dgm.philox_tokens(1, 0, 0, 0, 0, 8, 64, torch.zeros(8, dtype=torch.int32), stream=object())
+    finally:
+        ffi.load = real_load
+    # host buffers of dg_generate
+    p = torch.zeros(32, dtype=torch.int32)
+    assert _host(p, "p", torch.int32, 32).value == p.data_ptr()
+    with pytest.raises(ValueError, match="dtype"):
+        _host(torch.zeros(32, dtype=torch.int64), "p", torch.int32)
+    with pytest.raises(ValueError, match="contiguous"):
+        _host(torch.zeros((8, 8), dtype=torch.int32)[:, ::2], "p", torch.int32)
+    with pytest.raises(ValueError, match="at least"):
+        _host(p, "out", torch.int32, 64)
+    with pytest.raises(ValueError, match="shape"):
+        _check(torch.zeros((2, 3)), "k", torch.float32, False, shape=(3, 2))
