@@ -117,3 +117,36 @@ def test_tiny_generation_takes_twelve_steps():
         if rem == 0:
             break
     assert rems == [256 - 22 * i for i in range(1, 12)] + [0]
+
+
+@pytest.mark.parametrize("variant", [dict(temperature=0.7), dict(ffn_selfcond=32, selfcond_topk=4),
+                                     dict(expert_fp8=1), dict(sampler=1),
+                                     dict(temperature=0.7, ffn_selfcond=32, expert_fp8=1, sampler=1)])
+def test_generation_invariants_of_the_variants(variant):
+    """Every configuration knob keeps the loop's invariants: deterministic for a
+    seed, at most max_steps steps per canvas, ids in range, and frozen tokens stay
+    frozen step to step."""
+    cfg = SMALL.with_(**variant)
+    ora = Oracle(cfg, oracle_weights(make_weights(cfg, seed=1, std=0.15, gain_std=0.1)))
+    rng = np.random.default_rng(5)
+    prompt = rng.integers(0, cfg.vocab, 45)
+    out, steps = ora.generate(prompt, 2 * cfg.canvas, seed=9)
+    out2, steps2 = ora.generate(prompt, 2 * cfg.canvas, seed=9)
+    np.testing.assert_array_equal(out, out2)
+    assert steps == steps2 and all(1 <= s <= cfg.max_steps for s in steps)
+    assert out.min() >= 0 and out.max() < cfg.vocab
+    # frozen tokens persist through one canvas
+    cache = ora.new_cache(45 + cfg.canvas)
+    ora.prefill(cache, prompt)
+    canvas, acc = ora.open_canvas(seed=9, block=0)
+    prev = prev_logits = None
+    for s in range(1, cfg.max_steps + 1):
+        frozen = canvas[acc].copy()
+        before = acc.copy()
+        canvas, acc, rem, st = ora.denoise_step(cache, canvas, acc, seed=9, block=0, step=s, prev_argmax=prev,
+                                                prev_logits=prev_logits)
+        np.testing.assert_array_equal(canvas[before], frozen)
+        prev, prev_logits = st["argmax"], st["logits"]
+        if rem == 0:
+            break
+    assert rem == 0
