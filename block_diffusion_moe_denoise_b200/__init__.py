@@ -15,7 +15,7 @@ import torch
 from . import _ffi
 from ._ffi import DGError, check, dg_config, dg_layer_weights, dg_weights  # noqa: F401
 
-__all__ = ["DG", "DGError", "config_struct", "lm_head_noalloc", "philox_tokens", "route_topk"]
+__all__ = ["DG", "DGError", "config_struct", "lm_head_noalloc", "philox_tokens", "route_topk", "weight_shapes"]
 
 
 def _ptr(t):
@@ -91,11 +91,32 @@ def lm_head_noalloc(x: torch.Tensor, final_norm: torch.Tensor, embed: torch.Tens
                     stats: torch.Tensor, argmax: torch.Tensor, err: torch.Tensor | None = None, stream=None) -> None:
     """dg_op_lm_head_noalloc: LM-head statistics with the library's built-in
     scratch (no workspace, no allocation inside)."""
+    if not isinstance(x, torch.Tensor) or x.dim() != 2:
+        raise ValueError("x: expected a 2-D [T, d_model] tensor")
+    if not isinstance(embed, torch.Tensor) or embed.dim() != 2:
+        raise ValueError("embed: expected a 2-D [vocab, d_model] tensor")
     T, d = x.shape
+    V = embed.shape[0]
     check(_ffi.load().dg_op_lm_head_noalloc(
-        _dev(x, "x", _F32), _dev(final_norm, "final_norm", _F32, d), _dev(embed, "embed", _BF16), T, d,
-        embed.shape[0], norm_eps, _dev(stats, "stats", _F32, T * 4), _dev(argmax, "argmax", _I32, T),
+        _dev(x, "x", _F32, shape=(T, d)), _dev(final_norm, "final_norm", _F32, shape=(d,)),
+        _dev(embed, "embed", _BF16, shape=(V, d)), T, d, V, norm_eps, _dev(stats, "stats", _F32, T * 4), _dev(argmax, "argmax", _I32, T),
         _dev(err, "err", _I32, 1, optional=True), _stream(stream)), "dg_op_lm_head_noalloc")
+
+
+def weight_shapes(cfg) -> dict:
+    """The shape dg_init reads for every weight tensor of a configuration (dg.h,
+    dg_layer_weights / dg_weights): a tensor of another shape is rejected before
+    the C call, since its TMA descriptors would reach past its end."""
+    d, D, E = cfg.d_model, cfg.head_dim, cfg.n_experts
+    fe, fs, fsc = cfg.ffn_expert, cfg.ffn_shared, getattr(cfg, "ffn_selfcond", 0)
+    return {
+        "embed": (cfg.vocab, d), "final_norm": (d,),
+        "attn_norm": (d,), "w_qkv": ((cfg.n_q_heads + 2 * cfg.n_kv_heads) * D, d), "w_o": (d, cfg.n_q_heads * D),
+        "ffn_norm": (d,), "w_router": (E, d), "w_gate": (E, fe, d), "w_up": (E, fe, d), "w_down": (E, d, fe),
+        "ws_gate": (fs, d), "ws_up": (fs, d), "ws_down": (d, fs),
+        "w_gate_scale": (E, fe), "w_up_scale": (E, fe), "w_down_scale": (E, d),
+        "sc_gate": (fsc, d), "sc_up": (fsc, d), "sc_down": (d, fsc),
+    }
 
 
 class DG:
@@ -111,6 +132,7 @@ class DG:
         if len(weights["layers"]) != cfg.n_layers:
             raise ValueError(f"weights: {len(weights['layers'])} layers for a {cfg.n_layers}-layer configuration")
         fp8 = bool(getattr(cfg, "expert_fp8", 0))
+        shapes = weight_shapes(cfg)
         layers = (dg_layer_weights * cfg.n_layers)()
         for i, lw in enumerate(weights["layers"]):
             ptrs = []
@@ -121,13 +143,14 @@ class DG:
                     continue
                 dt = _F32 if n.endswith("norm") or n.endswith("_scale") else (
                     _U8 if fp8 and n in ("w_gate", "w_up", "w_down") else _BF16)
-                ptrs.append(_check(lw[n], f"layers[{i}].{n}", dt, True).data_ptr())
+                ptrs.append(_check(lw[n], f"layers[{i}].{n}", dt, True, shape=shapes[n]).data_ptr())
             layers[i] = dg_layer_weights(*ptrs)
         self._layers = layers
-        sc = [_check(weights[n], n, _BF16, True).data_ptr() if getattr(cfg, "ffn_selfcond", 0) > 0 else None
-              for n in ("sc_gate", "sc_up", "sc_down")]
-        self.c_w = dg_weights(_check(weights["embed"], "embed", _BF16, True).data_ptr(),
-                              _check(weights["final_norm"], "final_norm", _F32, True).data_ptr(), layers, *sc)
+        sc = [_check(weights[n], n, _BF16, True, shape=shapes[n]).data_ptr()
+              if getattr(cfg, "ffn_selfcond", 0) > 0 else None for n in ("sc_gate", "sc_up", "sc_down")]
+        self.c_w = dg_weights(_check(weights["embed"], "embed", _BF16, True, shape=shapes["embed"]).data_ptr(),
+                              _check(weights["final_norm"], "final_norm", _F32, True,
+                                     shape=shapes["final_norm"]).data_ptr(), layers, *sc)
         nbytes = lib.dg_workspace_size(C.byref(self.c_cfg), max_requests, kv_capacity)
         if nbytes == 0:
             raise DGError(-1, "dg_workspace_size")

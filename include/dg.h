@@ -153,12 +153,15 @@ typedef struct dg_weights {
 
 typedef struct dg_handle dg_handle;
 
-/* Bytes of device workspace dg_init needs for up to `max_requests` requests
+/* (No counterpart in the pages: workspace sizing is the library's own, so that
+ * the caller owns every device buffer.)
+ * Bytes of device workspace dg_init needs for up to `max_requests` requests
  * denoised together, each with a KV cache of `kv_capacity` positions
  * (prompt + committed canvases + one open canvas).  0 on invalid input. */
 size_t dg_workspace_size(const dg_config* cfg, int max_requests, int64_t kv_capacity);
 
-/* Create a handle.  `workspace` is a device buffer of at least
+/* (No counterpart in the pages: handle set-up.)
+ * Create a handle.  `workspace` is a device buffer of at least
  * dg_workspace_size(...) bytes, 1024-byte aligned, owned by the caller (it
  * holds the KV cache); `stream` is a cudaStream_t (NULL = legacy default).
  * Builds the TMA descriptors for every weight and activation buffer.
@@ -166,10 +169,19 @@ size_t dg_workspace_size(const dg_config* cfg, int max_requests, int64_t kv_capa
 int dg_init(const dg_config* cfg, const dg_weights* weights, int max_requests, int64_t kv_capacity,
             void* workspace, size_t workspace_bytes, void* stream, dg_handle** out);
 
+/* (No counterpart in the pages.)  Release the handle (host state only; the
+ * caller frees its device buffers); NULL is ignored. */
 void dg_destroy(dg_handle* h);
+/* (No counterpart in the pages.)  Static name of a DG_* return code. */
 const char* dg_strerror(int code);
 
-/* Append `n` prompt tokens (device int32 array) to request `req`'s KV cache:
+/* Defined by: "DiffusionGemma Hits 1,000 Tokens per Second--But Its Benchmarks Reveal the Real Tradeoff",
+ * section "How diffusion text generation changes the bottleneck" (committed
+ * blocks live in the key-value cache and condition the next canvas), and
+ * section "The speed numbers and the hardware they require" of the same page
+ * (the serving example prefills the prompt in chunks).  Reading: the prompt is cached
+ * by the same segment pass as a committed canvas.
+ * Append `n` prompt tokens (device int32 array) to request `req`'s KV cache:
  * the decoder runs over segments of `canvas` tokens counted from the first
  * token; each segment attends to all earlier positions and bidirectionally to
  * itself.  Up to eight full segments share one decoder pass (block-causal
@@ -178,7 +190,8 @@ const char* dg_strerror(int code);
  * overflow. */
 int dg_prefill(dg_handle* h, int req, const int32_t* d_tokens, int n);
 
-/* Write synthetic committed K/V: positions [pos0, pos0+n) of layer `layer`
+/* (No counterpart in the pages: KV inspection and synthetic prefixes.)
+ * Write synthetic committed K/V: positions [pos0, pos0+n) of layer `layer`
  * from device arrays k, v of shape [n_kv_heads, n, head_dim] bf16 (post-RoPE
  * keys).  Does not change the KV length.  Like dg_get_kv, dg_set_kv_len,
  * dg_prefill and dg_debug_forward, it first runs a deferred commit pass of
@@ -190,12 +203,22 @@ int dg_get_kv(dg_handle* h, int req, int layer, int64_t pos0, int64_t n, void* d
 int dg_set_kv_len(dg_handle* h, int req, int64_t len);
 int64_t dg_kv_len(const dg_handle* h, int req);
 
-/* Open canvas number `block` of request `req`: every position gets
+/* Defined by: "DiffusionGemma hits ~1,500 TPS on one H100: when a diffusion LLM beats autoregressive serving",
+ * section "What DiffusionGemma is" (each canvas starts as a scratch pad of
+ * random tokens).
+ * Open canvas number `block` of request `req`: every position gets
  * tok(seed, block, 0, position), nothing accepted.  DG_E_CAPACITY if the canvas
  * does not fit after the committed positions. */
 int dg_open_canvas(dg_handle* h, int req, uint64_t seed, int block);
 
-/* One denoising step for `n_req` requests (host array `reqs`), denoised
+/* Defined by: "DiffusionGemma hits ~1,500 TPS on one H100: when a diffusion LLM beats autoregressive serving",
+ * sections "What DiffusionGemma is" (a bidirectional decoder pass over all 256
+ * positions, accept the confident tokens, re-randomise the rest) and "How
+ * the sampler actually works" (the per-step procedure and the stop rule);
+ * the pass's MoE routing: "DiffusionGemma Hits 1,000 Tokens per Second--But Its Benchmarks Reveal the Real Tradeoff",
+ * section "The speed numbers and the hardware they require" (128 experts,
+ * eight active plus one shared).
+ * One denoising step for `n_req` requests (host array `reqs`), denoised
  * together: one bidirectional pass over their canvases (tokens routed
  * together), LM-head statistics, then the accept / re-noise rule.  Each canvas
  * writes its own K/V into cache slots [L, L+canvas) as scratch; L is unchanged.
@@ -203,10 +226,16 @@ int dg_open_canvas(dg_handle* h, int req, uint64_t seed, int block);
  * (device int32, may be NULL) and is readable with dg_read_remaining. */
 int dg_denoise_step(dg_handle* h, int n_req, const int* reqs, int32_t* d_remaining);
 
-/* Synchronising read of a request's remaining count (host). */
+/* (No counterpart in the pages.)  Synchronising read of a request's remaining
+ * count (host). */
 int dg_read_remaining(dg_handle* h, int req, int32_t* remaining);
 
-/* Commit request `req`'s converged canvas: the decoder runs over the final
+/* Defined by: "DiffusionGemma Hits 1,000 Tokens per Second--But Its Benchmarks Reveal the Real Tradeoff",
+ * section "How diffusion text generation changes the bottleneck" (a completed
+ * block is committed to the key-value cache before the next canvas opens),
+ * and "DiffusionGemma hits ~1,500 TPS on one H100: when a diffusion LLM beats autoregressive serving", section "What DiffusionGemma
+ * is" (finished blocks are committed to the KV cache).
+ * Commit request `req`'s converged canvas: the decoder runs over the final
  * canvas tokens at [L, L+canvas), writing their K/V, and L advances by canvas
  * (dg_kv_len reports the new length at once).  The pass itself is deferred:
  * it joins the request's next dg_denoise_step as an extra block-causal slot
@@ -217,7 +246,11 @@ int dg_read_remaining(dg_handle* h, int req, int32_t* remaining);
  * == 0); committing earlier commits the current tokens as they are. */
 int dg_commit_block(dg_handle* h, int req);
 
-/* Whole generation with HOST buffers: copy `n_prompt` prompt ids from host,
+/* Defined by: "DiffusionGemma hits ~1,500 TPS on one H100: when a diffusion LLM beats autoregressive serving",
+ * sections "What DiffusionGemma is" (canvas after canvas until the output is
+ * complete) and "The specs that matter for serving" (the measured setup: 4096
+ * input and 1024 output tokens at batch 1).
+ * Whole generation with HOST buffers: copy `n_prompt` prompt ids from host,
  * prefill, then n_out/canvas canvases (each denoised until nothing remains,
  * at most max_steps steps, then committed), copying the output ids to host
  * `h_out` [n_out].  steps_taken (host, may be NULL) receives the step count of
@@ -225,7 +258,10 @@ int dg_commit_block(dg_handle* h, int req);
 int dg_generate(dg_handle* h, int req, const int32_t* h_prompt, int n_prompt, int n_out, uint64_t seed,
                 int32_t* h_out, int* steps_taken);
 
-/* Copy the open canvas of `req`: tokens [canvas] int32, accepted mask [canvas]
+/* Defined by: "DiffusionGemma hits ~1,500 TPS on one H100: when a diffusion LLM beats autoregressive serving",
+ * section "How the sampler actually works" (the canvas, which positions are
+ * accepted, and the per-position entropy and confidence the rule reads).
+ * Copy the open canvas of `req`: tokens [canvas] int32, accepted mask [canvas]
  * u8 (1 = frozen), and the last step's statistics for its positions:
  * d_stats [canvas][4] f32 = (entropy nats, log max-probability, max logit,
  * log-partition), d_argmax [canvas] int32.  Any output pointer may be NULL.
@@ -234,10 +270,12 @@ int dg_generate(dg_handle* h, int req, const int32_t* h_prompt, int n_prompt, in
  * this request's last step, d_stats is filled with NaN and d_argmax with -1. */
 int dg_get_canvas(dg_handle* h, int req, int32_t* d_tokens, uint8_t* d_mask, float* d_stats, int32_t* d_argmax);
 
-/* Replace the open canvas of `req` (tokens, accepted mask) and its step counter. */
+/* (No counterpart in the pages: teacher forcing for tests.)
+ * Replace the open canvas of `req` (tokens, accepted mask) and its step counter. */
 int dg_set_canvas(dg_handle* h, int req, const int32_t* d_tokens, const uint8_t* d_mask, int step);
 
-/* Wait for all enqueued work; DG_E_DEVICE if a kernel flagged an error (the
+/* (No counterpart in the pages.)
+ * Wait for all enqueued work; DG_E_DEVICE if a kernel flagged an error (the
  * error word is then cleared), DG_E_CUDA on a CUDA error. */
 int dg_sync(dg_handle* h);
 

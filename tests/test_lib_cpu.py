@@ -147,3 +147,68 @@ def test_binding_rejects_unusable_tensors_before_any_call():
         _host(p, "out", torch.int32, 64)
     with pytest.raises(ValueError, match="shape"):
         _check(torch.zeros((2, 3)), "k", torch.float32, False, shape=(3, 2))
+
+
+def _host_as_device(monkeypatch):
+    """Let the binding's tensor checks accept host tensors as if they were device
+    memory, so the remaining checks (dtype, shape, element count) run on a
+    machine without a GPU; and make every library entry point fail the test."""
+    import block_diffusion_moe_denoise_b200 as dgm
+    import block_diffusion_moe_denoise_b200._ffi as ffi
+    real = dgm._check
+
+    def check(t, name, dtype, device, numel=None, shape=None):
+        return real(t, name, dtype, bool(getattr(t, "is_cuda", False)), numel, shape)
+
+    class NoCalls:
+        def __getattr__(self, name):
+            def call(*args):
+                raise AssertionError(f"{name} was called")
+            return call
+
+    monkeypatch.setattr(dgm, "_check", check)
+    monkeypatch.setattr(ffi, "load", lambda: NoCalls())
+    return dgm
+
+
+def test_binding_rejects_wrong_weight_shapes_before_init(monkeypatch):
+    """A weight of the wrong shape (here one expert row short, or an output
+    projection one head narrow) raises in dg_init's binding before any C call: its TMA
+    descriptors would otherwise reach past the end of the tensor."""
+    import torch
+    from synth import TINY, make_weights
+    dgm = _host_as_device(monkeypatch)
+    w = make_weights(TINY, seed=0)
+    for name, bad in (("w_gate", lambda t: t[:, :-1].contiguous()), ("w_o", lambda t: t[:, :-64].contiguous()),
+                      ("ws_down", lambda t: t[:-64].contiguous())):
+        ww = {"embed": w["embed"], "final_norm": w["final_norm"],
+              "layers": [dict(lw) for lw in w["layers"]]}
+        ww["layers"][1][name] = bad(ww["layers"][1][name])
+        with pytest.raises(ValueError, match=rf"layers\[1\]\.{name}: expected shape"):
+            dgm.DG(TINY, ww, max_requests=1, kv_capacity=512, stream=object())
+    ww = {"embed": w["embed"][:, :128].contiguous(), "final_norm": w["final_norm"], "layers": w["layers"]}
+    with pytest.raises(ValueError, match="embed: expected shape"):
+        dgm.DG(TINY, ww, max_requests=1, kv_capacity=512, stream=object())
+    shapes = dgm.weight_shapes(TINY)
+    for name, t in w["layers"][0].items():
+        assert tuple(t.shape) == shapes[name], name
+
+
+def test_noalloc_binding_rejects_mismatched_embedding(monkeypatch):
+    """dg_op_lm_head_noalloc reads embed as [vocab, d_model] rows of x's width:
+    a narrower or 1-D embedding, or a 1-D x, raises before any C call."""
+    import torch
+    dgm = _host_as_device(monkeypatch)
+    T, d, V = 8, 256, 1024
+    x = torch.zeros((T, d))
+    g = torch.ones(d)
+    st, am = torch.zeros((T, 4)), torch.zeros(T, dtype=torch.int32)
+    with pytest.raises(ValueError, match="embed: expected shape"):
+        dgm.lm_head_noalloc(x, g, torch.zeros((V, d - 64), dtype=torch.bfloat16), 1e-6, st, am, stream=object())
+    with pytest.raises(ValueError, match="2-D"):
+        dgm.lm_head_noalloc(x, g, torch.zeros(V * d, dtype=torch.bfloat16), 1e-6, st, am, stream=object())
+    with pytest.raises(ValueError, match="2-D"):
+        dgm.lm_head_noalloc(x.view(-1), g, torch.zeros((V, d), dtype=torch.bfloat16), 1e-6, st, am, stream=object())
+    with pytest.raises(ValueError, match="final_norm: expected shape"):
+        dgm.lm_head_noalloc(x, torch.ones(d + 64), torch.zeros((V, d), dtype=torch.bfloat16), 1e-6, st, am,
+                            stream=object())
