@@ -37,6 +37,8 @@ sys.path.insert(0, ROOT)
 
 PROMPT = 4096
 N_OUT = 1024
+LONG_PREFIX = 65536
+LONG_REQUESTS = 4
 SEED = 1234
 METRIC = "output tok/s at batch 1 (4096 in / 1024 out), full synthetic 30-layer MoE stack; ms/denoise step"
 
@@ -47,7 +49,9 @@ def parse():
     ap.add_argument("--steps", type=int, default=8)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="generate", choices=["generate", "layer"])
+    ap.add_argument("--workload", default="generate", choices=["generate", "layer", "long"],
+                    help="generate: the headline (4096 in / 1024 out); layer: one full-shape layer; long: four "
+                         "requests with 65536-token KV prefixes denoised together (one step over 1024 canvas tokens)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--canvas-vocab", type=int, default=0,
@@ -152,19 +156,26 @@ def expert_gate_up_bytes(cfg, n_touched: float, T: int) -> float:
     return w + rows * (cfg.d_model * eb + (4 if eb == 1 else 0)) + rows * cfg.ffn_expert * 2
 
 
-def step_work(cfg, kv_len: int, T: int, n_touched: float):
-    """(bytes, flops) of one denoising step: every weight of the touched
-    experts and all dense weights once, the KV prefix read, per-token FLOPs."""
+def step_work(cfg, kv_len: int, T: int, n_touched: float, n_req: int = 1):
+    """(bytes, flops) of one denoising step over n_req requests of T canvas
+    tokens each: every weight of the touched experts and all dense weights
+    once, each request's KV prefix read, per-token FLOPs."""
     d, D = cfg.d_model, cfg.head_dim
     attn_w = cfg.qkv_rows * d + d * cfg.n_q_heads * D
     eb = 0.5 if getattr(cfg, "expert_fp8", 0) else 1.0      # expert weights: E4M3 codes or bf16
     per_layer_w = attn_w + eb * n_touched * 3 * cfg.ffn_expert * d + 3 * cfg.ffn_shared * d + cfg.n_experts * d
     weights = (cfg.n_layers * per_layer_w + cfg.vocab * d) * 2
-    kv = cfg.n_layers * 2 * cfg.n_kv_heads * (kv_len + T) * D * 2
-    act = cfg.n_layers * T * (cfg.top_k * (3 * d + cfg.ffn_expert) * 2 + 12 * d * 4)
+    kv = n_req * cfg.n_layers * 2 * cfg.n_kv_heads * (kv_len + T) * D * 2
+    act = n_req * cfg.n_layers * T * (cfg.top_k * (3 * d + cfg.ffn_expert) * 2 + 12 * d * 4)
     active = cfg.active_params_per_token()
-    flops = 2 * T * active + cfg.n_layers * 4 * cfg.n_q_heads * T * (kv_len + T) * D
+    flops = n_req * (2 * T * active + cfg.n_layers * attention_flops_per_layer(cfg, kv_len, T))
     return weights + kv + act, flops
+
+
+def attention_flops_per_layer(cfg, kv_len: int, T: int) -> float:
+    """FLOPs of one request's canvas attention in one layer: Q K^T and P V over
+    kv_len + T keys for T queries of every query head."""
+    return 4.0 * cfg.n_q_heads * T * (kv_len + T) * cfg.head_dim
 
 
 # ---------------------------------------------------------------------------
@@ -228,6 +239,44 @@ def oracle_sample(reps: int = 1, warm: int = 0, min_seconds: float = 0.0):
             "sample_seconds": sum(t[3] for t in times) / len(times)}
 
 
+def oracle_full_step(w, dev):
+    """Time ONE whole denoising step of the fp64 oracle at the full shape: all 30
+    layers over a 256-token canvas with a 4096-token synthetic N(0, 1) KV prefix
+    per layer, then the LM head over the full vocabulary (configs of the full
+    synthetic stack).  The weights are the benchmark's device tensors, widened
+    to fp64 one layer at a time (the whole stack would need ~200 GB in fp64);
+    the time spent widening them is measured and left out, so the figure is the
+    oracle's arithmetic.  Returns seconds for the step and for its 30 layers."""
+    import numpy as np
+    from oracle.model import Oracle
+    from synth import FULL, make_kv_prefix, make_tokens, to_f64
+    widen = [0.0]
+
+    def layer(l):
+        t0 = time.perf_counter()
+        out = {n: to_f64(t) for n, t in w["layers"][l].items()}
+        widen[0] += time.perf_counter() - t0
+        return out
+
+    ora = Oracle(FULL, {"embed": to_f64(w["embed"]), "final_norm": to_f64(w["final_norm"]), "layers": layer})
+    cache = ora.new_cache(PROMPT + FULL.canvas)
+    for l in range(FULL.n_layers):
+        k, v = make_kv_prefix(FULL, PROMPT, seed=1, device=dev, layer=l)
+        cache.K[l][:, :PROMPT] = to_f64(k)
+        cache.V[l][:, :PROMPT] = to_f64(v)
+    cache.length = PROMPT
+    tok = make_tokens(FULL, FULL.canvas, seed=2, name="canvas").numpy().astype(np.int64)
+    t0 = time.perf_counter()
+    ora.forward(tok, cache, want_stats=False)
+    t_layers = time.perf_counter() - t0 - widen[0]
+    from oracle import layers as OL
+    xn = np.random.default_rng(0).standard_normal((FULL.canvas, FULL.d_model))
+    t1 = time.perf_counter()
+    OL.lm_head_stats(OL.rms_norm(xn, ora.final_norm, FULL.norm_eps), ora.embed)
+    t_lm = time.perf_counter() - t1
+    return t_layers + t_lm, t_layers
+
+
 # ---------------------------------------------------------------------------
 # distributed plumbing (replicas)
 # ---------------------------------------------------------------------------
@@ -287,6 +336,14 @@ def run_reference(args, world):
 
 
 def workload_config(cfg, workload, world):
+    if workload == "long":
+        out = {"workload": ("long: 30 layers d2816, 16q/8kv heads x256, 128 experts top-8 + shared 2112, vocab "
+                            "262144; 4 requests, each a 65536-token synthetic KV prefix (N(0,1) bf16) and its own "
+                            "256-token canvas, denoised together (1024 canvas tokens per step)"),
+               "canvas": cfg.canvas, "kv_prefix": LONG_PREFIX, "batch": LONG_REQUESTS,
+               "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+               "l2": "inputs larger than L2: every step streams ~50 GB of weights and ~65 GB of KV"}
+        return out
     if workload == "layer":
         name = ("layer: one decoder layer at full shape + LM head over 262144, one denoising step, "
                 "4096-token synthetic KV prefix, 256-token canvas, batch 1")
@@ -321,15 +378,16 @@ def main():
     from synth import FULL, LAYER, make_kv_prefix, make_tokens, make_weights
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    cfg = FULL if args.workload == "generate" else LAYER
+    cfg = LAYER if args.workload == "layer" else FULL
     cfg = cfg.with_(temperature=args.temperature, ffn_selfcond=args.selfcond,
                     expert_fp8=1 if args.fp8_experts else 0)
     hbm_gbs, bf16_tf, bf16_tf_sus, peak_kind = measured_peaks()
 
     w = make_weights(cfg, seed=0, device=dev)
     torch.cuda.synchronize()
-    cap = PROMPT + N_OUT if args.workload == "generate" else PROMPT + cfg.canvas
-    h = dgm.DG(cfg, w, max_requests=1, kv_capacity=cap, device=dev)
+    n_req = LONG_REQUESTS if args.workload == "long" else 1
+    cap = {"generate": PROMPT + N_OUT, "layer": PROMPT + cfg.canvas, "long": LONG_PREFIX + cfg.canvas}[args.workload]
+    h = dgm.DG(cfg, w, max_requests=n_req, kv_capacity=cap, device=dev)
     st = h.stream
     prompt = make_tokens(cfg, PROMPT, seed=0)
 
@@ -363,6 +421,27 @@ def main():
             if record:
                 seg_steps.append((e0, e1))
                 steps_per.append(n)
+    elif args.workload == "long":
+        # four requests, each with its own synthetic committed prefix in every layer
+        for r in range(n_req):
+            for l in range(cfg.n_layers):
+                k, v = make_kv_prefix(cfg, LONG_PREFIX, seed=10 + r, device=dev, layer=l)
+                h.set_kv(r, l, 0, k, v)
+                del k, v
+            h.set_kv_len(r, LONG_PREFIX)
+        torch.cuda.synchronize()
+        prefill_ms = None
+
+        def one_step(i, record=False):
+            if i % cfg.max_steps == 0:
+                for r in range(n_req):
+                    h.open_canvas(r, SEED + r, 0)
+            e0 = ev() if record else None
+            h.denoise_step(list(range(n_req)))
+            e1 = ev() if record else None
+            if record:
+                seg_steps.append((e0, e1))
+                steps_per.append(1)
     else:
         k, v = make_kv_prefix(cfg, PROMPT, seed=1, device=dev)
         h.set_kv(0, 0, 0, k, v)
@@ -405,7 +484,7 @@ def main():
     elapsed = start.elapsed_time(end)
     launches = h.launch_count() - launches0
     h.sync()
-    toks_per_step = cfg.canvas if args.workload == "generate" else cfg.canvas / 12.0
+    toks_per_step = cfg.canvas if args.workload == "generate" else n_req * cfg.canvas / 12.0
     value, elapsed_max = job_throughput(toks_per_step * args.steps, elapsed, world)
     step_ms = sum(a.elapsed_time(b) for a, b in seg_steps)
     n_steps = sum(steps_per)
@@ -443,7 +522,8 @@ def main():
     total_prof = sum(v[0] for v in prof.values()) or 1.0
     kernels = {k: {"ms": round(v[0], 4), "launches": v[1], "share": round(v[0] / total_prof, 4)}
                for k, v in prof.items() if v[1] > 0}
-    sbytes, sflops = step_work(cfg, PROMPT + 384 if args.workload == "generate" else PROMPT, T, n_touched)
+    kv_step = {"generate": PROMPT + 384, "layer": PROMPT, "long": LONG_PREFIX}[args.workload]
+    sbytes, sflops = step_work(cfg, kv_step, T, n_touched, n_req)
     t_roof_ms = max(sbytes / (hbm_gbs * 1e9), sflops / (bf16_tf * 1e12)) * 1e3
 
     e2e = None
@@ -464,11 +544,41 @@ def main():
 
     cpu = None
     # the oracle sample is the headline workload's; the variants have none
-    variant = args.temperature > 0 or args.selfcond > 0 or args.fp8_experts
+    variant = args.temperature > 0 or args.selfcond > 0 or args.fp8_experts or args.workload == "long"
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not variant:
-        s = oracle_sample(reps=3, warm=1, min_seconds=10.0)
-        cpu = {k: s[k] for k in ("value", "unit", "cores", "kind", "sample")}
+        if args.workload == "generate":
+            # one whole 30-layer step of the oracle, measured once; a canvas is 12
+            # such steps plus a commit (the step's 30 layers without the LM head)
+            t_step, t_layers = oracle_full_step(w, dev)
+            t_canvas = 12 * t_step + t_layers
+            s = oracle_sample(reps=1, warm=0)
+            cpu = {"value": 256.0 / t_canvas, "unit": "tok/s", "cores": s["cores"], "kind": "oracle",
+                   "sample": (f"fp64 oracle, one whole denoising step measured: 30 layers over a 256-token canvas "
+                              f"with a 4096-token KV prefix ({t_layers:.1f} s) + LM head over 262144 "
+                              f"({t_step - t_layers:.1f} s), scaled to 12 steps + 1 commit per canvas; the "
+                              f"one-layer extrapolation gives {s['value']:.3f} tok/s"),
+                   "ms_per_denoise_step": 1e3 * t_step}
+        else:
+            s = oracle_sample(reps=3, warm=1, min_seconds=10.0)
+            cpu = {k: s[k] for k in ("value", "unit", "cores", "kind", "sample")}
 
+    roofline = {"kernel": ("experts_gate_up (routed-expert gate|up GEMM + SwiGLU"
+                           + (", E4M3 W8A8)" if getattr(cfg, "expert_fp8", 0) else ")")), "bound": "hbm",
+                "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s", "frac": achieved / hbm_gbs,
+                "traffic": traffic, "algorithmic_bytes_per_launch": egu_bytes,
+                "avg_launch_ms": egu_avg_ms, "peak_source": f"{peak_kind} HBM copy (MEASURED_PEAKS.json)"}
+    if args.workload == "long":
+        # the dominant kernel of the long-context step is the canvas attention
+        # (k_attn_tc + its split combine, one "attention" class launch pair per layer)
+        at_ms, at_n = prof["attention"]
+        at_layers = max(1, at_n // 2)
+        at_flops = n_req * attention_flops_per_layer(cfg, LONG_PREFIX, T)
+        at_avg = at_ms / at_layers
+        tf = at_flops / (at_avg * 1e-3) / 1e12
+        roofline = {"kernel": "attention (k_attn_tc + split-KV combine, per layer: 4 requests x 65792 keys)",
+                    "bound": "tensor", "achieved": tf, "peak": bf16_tf, "unit": "TFLOP/s", "frac": tf / bf16_tf,
+                    "traffic": None, "algorithmic_flops_per_launch": at_flops, "avg_launch_ms": at_avg,
+                    "peak_source": f"{peak_kind} bf16 dense burst (MEASURED_PEAKS.json)"}
     line = {
         "metric": METRIC,
         "value": value,
@@ -488,11 +598,7 @@ def main():
         "dtype": "bf16+e4m3" if getattr(cfg, "expert_fp8", 0) else "bf16",
         "data": "synthetic (seeded N(0,0.02) bf16 weights, uniform token ids)",
         "config": workload_config(cfg, args.workload, world),
-        "roofline": {"kernel": ("experts_gate_up (routed-expert gate|up GEMM + SwiGLU"
-                                + (", E4M3 W8A8)" if getattr(cfg, "expert_fp8", 0) else ")")), "bound": "hbm",
-                     "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s", "frac": achieved / hbm_gbs,
-                     "traffic": traffic, "algorithmic_bytes_per_launch": egu_bytes,
-                     "avg_launch_ms": egu_avg_ms, "peak_source": f"{peak_kind} HBM copy (MEASURED_PEAKS.json)"},
+        "roofline": roofline,
         "step_roofline": {"bytes": sbytes, "flops": sflops, "bound": "hbm" if sbytes / hbm_gbs > sflops / bf16_tf / 1e3
                           else "tensor", "t_roof_ms": t_roof_ms, "frac": t_roof_ms / ms_denoise,
                           "experts_touched_per_layer": round(n_touched, 2)},

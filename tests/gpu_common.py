@@ -115,3 +115,57 @@ def argmax_agreement(gpu_argmax, ora_logits, keep=None, min_rate=0.95):
     rate = float(agree.mean()) if agree.size else 1.0
     assert rate >= min_rate, (rate, int(counted.sum()))
     return int(counted.sum()), int((~agree).sum()), rate
+
+
+def routing_divergence(gpu_idx_layers, ora_logits_layers, ora_idx_layers, k: int):
+    """Where the GPU's routing first leaves the oracle's, and a check that it only
+    ever leaves it at a near-tie.
+
+    Top-k routing is discontinuous, so a token whose k-th and (k+1)-th oracle
+    router logits are nearly tied may pick a different expert on the GPU, whose
+    router logits carry the bf16 rounding noise of the residual stream; both
+    choices are then correct to the precision of the inputs.  For every token
+    this returns the first layer at which the GPU's set of experts differs from
+    the oracle's (the number of layers if never).  At that layer the GPU's
+    choice must be a valid top-k set within the ambiguity margin
+    delta = ROUTER_GAP_REL * RMS(oracle router logits of the layer): every
+    expert it picked has an oracle logit at least the largest oracle logit of
+    the experts it did not pick minus delta.  Anything else is a routing bug
+    and fails here.  After its first divergence a token's hidden state follows
+    another (equally valid) branch, so value comparisons use the tokens that
+    have not diverged up to the compared layer."""
+    n_layers = len(gpu_idx_layers)
+    T = gpu_idx_layers[0].shape[0]
+    first = np.full(T, n_layers)
+    for l in range(n_layers):
+        r = np.asarray(ora_logits_layers[l], dtype=np.float64)
+        delta = ROUTER_GAP_REL * np.sqrt(np.mean(r * r))
+        for t in np.nonzero(first == n_layers)[0]:
+            g = set(int(e) for e in gpu_idx_layers[l][t])
+            if g == set(int(e) for e in ora_idx_layers[l][t]):
+                continue
+            first[t] = l
+            picked = np.array(sorted(g))
+            others = np.array([e for e in range(r.shape[1]) if e not in g])
+            assert len(g) == k, (l, t, sorted(g))
+            lo, hi = r[t, picked].min(), r[t, others].max()
+            assert lo >= hi - delta, (f"layer {l} token {t}: GPU experts {sorted(g)} are not a top-{k} set within "
+                                      f"{delta:.3g} of the oracle logits (lowest picked {lo:.5g}, highest other {hi:.5g})")
+    return first
+
+
+# Upper bound on the share of tokens a test may leave out of its value
+# comparisons for routing reasons.  Tests that exclude the oracle's near-tie
+# tokens (the tiny model: ~4.5% per layer) allow 20%; tests that exclude only
+# the tokens whose GPU routing actually left the oracle's (routing_divergence;
+# ~5% of a full-shape layer) allow 10%.
+MAX_EXCLUDED_NEAR_TIES = 0.20
+MAX_EXCLUDED_DIVERGED = 0.10
+
+
+def assert_excluded_fraction(excluded, bound: float, what: str) -> float:
+    excluded = np.asarray(excluded, dtype=bool)
+    frac = float(excluded.mean()) if excluded.size else 0.0
+    print(f"{what}: {int(excluded.sum())} of {excluded.size} tokens excluded ({frac:.1%}, bound {bound:.0%})")
+    assert frac <= bound, (what, frac, bound)
+    return frac

@@ -11,7 +11,8 @@ from oracle.model import Oracle, Trace
 from oracle import sampler as OS
 from synth import LAYER, make_kv_prefix, make_weights, to_f64
 
-from .gpu_common import LOGIT_MAX_ABS, REL_L2, ambiguous_tokens, argmax_agreement, np64, rel_l2, routing_match
+from .gpu_common import (LOGIT_MAX_ABS, MAX_EXCLUDED_DIVERGED, REL_L2, argmax_agreement, assert_excluded_fraction,
+                         np64, rel_l2, routing_divergence)
 
 pytestmark = [pytest.mark.gpu,
               pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
@@ -70,10 +71,9 @@ def test_moe_path(setup):
     h, rec, ora = setup["h"], setup["tr"], setup["ora"]
     T, d, k = CFG.canvas, CFG.d_model, CFG.top_k
     idx = h.debug_buffer("idx", torch.int32, (T, k)).cpu().numpy()
-    same = routing_match(idx, rec["idx"])
-    amb = ambiguous_tokens([rec], k)
-    assert same[~amb].all(), np.nonzero(~same & ~amb)
-    print(f"full layer: {amb.sum()} routing-ambiguous tokens, {(~same).sum()} re-routed")
+    # every token whose GPU routing differs from the oracle's must be a near-tie
+    same = routing_divergence([idx], [rec["router_logits"]], [rec["idx"]], k) == 1
+    assert_excluded_fraction(~same, MAX_EXCLUDED_DIVERGED, "full layer, routed differently at a near-tie")
     counts = h.debug_buffer("counts", torch.int32, (CFG.n_experts,)).cpu().numpy()
     assert counts.sum() == T * k and (counts == np.bincount(idx.ravel(), minlength=CFG.n_experts)).all()
     pair_row = h.debug_buffer("pair_row", torch.int32, (T * k,)).cpu().numpy()
@@ -117,14 +117,16 @@ def test_lm_head_sampled_rows(setup):
     h, rec, ora = setup["h"], setup["tr"], setup["ora"]
     stats = h.debug_buffer("stats", torch.float32, (256, 4)).cpu().numpy().astype(np.float64)
     am = h.debug_buffer("argmax", torch.int32, (256,)).cpu().numpy()
-    amb = ambiguous_tokens([rec], CFG.top_k)
-    rows = np.random.default_rng(1).choice(np.nonzero(~amb)[0], 24, replace=False)
+    idx = h.debug_buffer("idx", torch.int32, (256, CFG.top_k)).cpu().numpy()
+    same = routing_divergence([idx], [rec["router_logits"]], [rec["idx"]], CFG.top_k) == 1
+    assert_excluded_fraction(~same, MAX_EXCLUDED_DIVERGED, "full layer LM head, routed differently at a near-tie")
+    rows = np.random.default_rng(1).choice(np.nonzero(same)[0], 32, replace=False)
     xn = OL.rms_norm(rec["x_out"][rows], ora.final_norm, CFG.norm_eps)
     ref = OL.lm_head_stats(xn, ora.embed)
     assert np.max(np.abs(stats[rows, 2] - ref["max"])) < LOGIT_MAX_ABS
     assert np.max(np.abs(stats[rows, 3] - ref["logZ"])) < LOGIT_MAX_ABS
     assert rel_l2(stats[rows, 0], ref["entropy"]) < REL_L2
-    n, bad, rate = argmax_agreement(am[rows], ref["logits"], min_rate=0.9)
+    n, bad, rate = argmax_agreement(am[rows], ref["logits"], min_rate=0.95)
     print(f"full layer argmax: {n} rows with margin > 1e-2, {bad} differ ({rate:.3f})")
 
 

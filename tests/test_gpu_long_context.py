@@ -14,7 +14,8 @@ import torch
 from oracle import layers as OL
 from synth import LAYER, make_kv_prefix, make_weights, to_f64
 
-from .gpu_common import LOGIT_MAX_ABS, REL_L2, ROUTER_GAP_REL, argmax_agreement, np64, rel_l2, router_gap
+from .gpu_common import (LOGIT_MAX_ABS, MAX_EXCLUDED_NEAR_TIES, REL_L2, argmax_agreement, assert_excluded_fraction,
+                         np64, rel_l2, routing_divergence)
 
 pytestmark = [pytest.mark.gpu,
               pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
@@ -45,6 +46,7 @@ def setup():
                o=np64(h.debug_buffer("o", torch.bfloat16, (Tcap, CFG.n_q_heads * CFG.head_dim))),
                stats=h.debug_buffer("stats", torch.float32, (Tcap, 4)).cpu().numpy().astype(np.float64),
                argmax=h.debug_buffer("argmax", torch.int32, (Tcap,)).cpu().numpy(),
+               idx=h.debug_buffer("idx", torch.int32, (Tcap, CFG.top_k)).cpu().numpy(),
                remaining=[h.read_remaining(r) for r in range(N_REQ)])
     yield out
     h.close()
@@ -92,36 +94,44 @@ def test_sampled_attention_rows_over_65k_keys(setup):
 
 
 def test_sampled_lm_head_statistics(setup):
-    """Whole layer + LM head for sampled tokens of every request: the attention
+    """Whole layer + LM head for 32 sampled tokens (8 per request): the attention
     of each sampled token over its request's 65,792 keys, then its MoE and the
-    full-vocabulary statistics."""
+    full-vocabulary statistics.  A sampled token whose GPU routing differs from
+    the oracle's must be a near-tie and is left out (counted; at most 20% of
+    so small a sample, against ~5% expected);
+    on the rest, max logit within the logit bound and argmax equal where the
+    oracle's margin exceeds twice it, at a rate >= 95% where it exceeds 1e-2."""
     c = CFG
     lw = {n: to_f64(t) for n, t in setup["w"]["layers"][0].items()}
     embed = setup["w"]["embed"]
     rng = np.random.default_rng(1)
-    rows, xns = [], []
+    rows, xns, rls, oidx = [], [], [], []
     for r in range(N_REQ):
         x, q, k, v = _oracle_canvas_qkv(setup["w"]["layers"][0], embed, setup["canv"][r], L_PREFIX)
         kp, vp = setup["kvs"][r]
         Kall = [np.concatenate([to_f64(kp[g]), k[:, g]], 0) for g in range(c.n_kv_heads)]
         Vall = [np.concatenate([to_f64(vp[g]), v[:, g]], 0) for g in range(c.n_kv_heads)]
-        for t in rng.choice(c.canvas, 2, replace=False):
+        for t in rng.choice(c.canvas, 8, replace=False):
             o = OL.attention(q[t:t + 1], np.stack(Kall), np.stack(Vall))[0]
             xa = x[t] + o.reshape(-1) @ lw["w_o"].T
             u = OL.rms_norm(xa[None], lw["ffn_norm"], c.norm_eps)
             rl = u @ lw["w_router"].T
-            if router_gap(rl, c.top_k)[0] < ROUTER_GAP_REL * np.sqrt(np.mean(rl * rl)):
-                continue                                   # routing-ambiguous token
             idx, wts = OL.route(rl, c.top_k)
             y = OL.routed_experts(u, idx, wts, lw["w_gate"], lw["w_up"], lw["w_down"])
             xo = xa + y[0] + OL.swiglu(u, lw["ws_gate"], lw["ws_up"], lw["ws_down"])[0]
             xns.append(OL.rms_norm(xo[None], to_f64(setup["w"]["final_norm"]), c.norm_eps)[0])
+            rls.append(rl[0])
+            oidx.append(idx[0])
             rows.append(r * c.canvas + t)
-    assert len(rows) >= 4
-    XN = np.stack(xns)
+    rows = np.array(rows)
+    same = routing_divergence([setup["idx"][rows]], [np.stack(rls)], [np.stack(oidx)], c.top_k) == 1
+    assert_excluded_fraction(~same, MAX_EXCLUDED_NEAR_TIES, "long context, sampled tokens routed differently")
+    assert same.sum() >= 16
+    XN = np.stack(xns)[same]
+    rows = rows[same]
     ref_logits = np.concatenate([XN @ to_f64(embed[i:i + 32768]).T for i in range(0, c.vocab, 32768)], axis=1)
     ref_max = ref_logits.max(axis=1)
     st, am = setup["stats"], setup["argmax"]
     assert np.max(np.abs(st[rows, 2] - ref_max)) < LOGIT_MAX_ABS
-    n, bad, rate = argmax_agreement(am[rows], ref_logits, min_rate=0.75)
+    n, bad, rate = argmax_agreement(am[rows], ref_logits, min_rate=0.95)
     print(f"long context: {len(rows)} sampled tokens, argmax {n - bad}/{n} at margin > 1e-2")

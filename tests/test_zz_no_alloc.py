@@ -10,9 +10,10 @@ import numpy as np
 import pytest
 import torch
 
+from oracle import layers as OL
 from synth import TINY, make_weights
 
-from .gpu_common import to_device
+from .gpu_common import LOGIT_MAX_ABS, REL_L2, argmax_agreement, rel_l2, to_device
 
 pytestmark = [pytest.mark.gpu,
               pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
@@ -51,4 +52,54 @@ def test_noalloc_rejects_sizes_beyond_its_limit():
     am = torch.empty(257, dtype=torch.int32, device="cuda")
     with pytest.raises(DGError) as ei:
         dgm.lm_head_noalloc(x, g, e, cfg.norm_eps, stats, am)
+    assert ei.value.code == -1
+
+
+def test_noalloc_at_its_limits_matches_oracle():
+    """The documented limits themselves: T = 256 tokens of width d_model = 4096
+    fill the array's row region exactly (the padded token count equals the
+    maximum).  Two calls in a row (the second on other rows) agree with the
+    fp64 oracle's LM-head statistics within the bf16 bounds, and the first is
+    reproduced bit for bit when repeated after the second."""
+    import block_diffusion_moe_denoise_b200 as dgm
+    T, d, V = 256, 4096, 4096
+    g = torch.Generator(device="cuda")
+    g.manual_seed(5)
+    embed = (0.02 * torch.randn((V, d), generator=g, device="cuda")).to(torch.bfloat16)
+    gain = 1.0 + 0.1 * torch.randn(d, generator=g, device="cuda")
+    xs = [torch.randn((T, d), generator=g, device="cuda") for _ in range(2)]
+    E64, g64 = embed.double().cpu().numpy(), gain.double().cpu().numpy()
+    outs = []
+    for x in xs + xs[:1]:
+        stats = torch.empty((T, 4), dtype=torch.float32, device="cuda")
+        am = torch.empty(T, dtype=torch.int32, device="cuda")
+        err = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+        dgm.lm_head_noalloc(x, gain, embed, 1e-6, stats, am, err)
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0
+        outs.append((stats.clone(), am.clone()))
+    for x, (stats, am) in zip(xs, outs):
+        ref = OL.lm_head_stats(OL.rms_norm(x.double().cpu().numpy(), g64, 1e-6), E64)
+        st = stats.cpu().numpy().astype(np.float64)
+        assert np.max(np.abs(st[:, 2] - ref["max"])) < LOGIT_MAX_ABS
+        assert np.max(np.abs(st[:, 3] - ref["logZ"])) < LOGIT_MAX_ABS
+        assert rel_l2(st[:, 0], ref["entropy"]) < REL_L2
+        argmax_agreement(am.cpu().numpy(), ref["logits"])
+    assert torch.equal(outs[0][0], outs[2][0]) and torch.equal(outs[0][1], outs[2][1])
+
+
+@pytest.mark.parametrize("d", [4160, 4032 + 32, 200])
+def test_noalloc_rejects_widths_beyond_its_limit(d):
+    """A row width above DG_NOALLOC_MAX_DMODEL or not a multiple of 64 returns
+    DG_E_ARG before any work is enqueued."""
+    import block_diffusion_moe_denoise_b200 as dgm
+    from block_diffusion_moe_denoise_b200._ffi import DGError
+    T, V = 8, 1024
+    x = torch.zeros((T, d), dtype=torch.float32, device="cuda")
+    g = torch.ones(d, dtype=torch.float32, device="cuda")
+    e = torch.zeros((V, d), dtype=torch.bfloat16, device="cuda")
+    stats = torch.empty((T, 4), dtype=torch.float32, device="cuda")
+    am = torch.empty(T, dtype=torch.int32, device="cuda")
+    with pytest.raises(DGError) as ei:
+        dgm.lm_head_noalloc(x, g, e, 1e-6, stats, am)
     assert ei.value.code == -1
