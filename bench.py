@@ -569,9 +569,9 @@ def main():
                 "avg_launch_ms": egu_avg_ms, "peak_source": f"{peak_kind} HBM copy (MEASURED_PEAKS.json)"}
     if args.workload == "long":
         # the dominant kernel of the long-context step is the canvas attention
-        # (k_attn_tc + its split combine, one "attention" class launch pair per layer)
+        # (k_attn_tc + its split-KV combine, timed together once per layer)
         at_ms, at_n = prof["attention"]
-        at_layers = max(1, at_n // 2)
+        at_layers = max(1, at_n)   # one profiled record per layer (attention + its combine)
         at_flops = n_req * attention_flops_per_layer(cfg, LONG_PREFIX, T)
         at_avg = at_ms / at_layers
         tf = at_flops / (at_avg * 1e-3) / 1e12

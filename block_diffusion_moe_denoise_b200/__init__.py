@@ -291,7 +291,7 @@ class DG:
 
     KERNEL_CLASSES = ("embed", "rmsnorm", "qkv", "attention", "oproj", "group",
                       "experts_gate_up", "experts_down", "shared_gate_up", "shared_down", "lm_head", "lm_combine",
-                      "sample", "selfcond", "other")
+                      "sample", "selfcond", "other", "router")
 
     def profile(self, enable: int):
         check(self.lib.dg_profile(self.h, enable), "dg_profile")
@@ -310,6 +310,13 @@ class DG:
     def debug_forward(self, req: int, tokens: torch.Tensor, n_layers: int):
         check(self.lib.dg_debug_forward(self.h, req, _dev(tokens, "tokens", _I32), tokens.numel(), n_layers),
               "dg_debug_forward")
+
+    def debug_forward_hidden(self, req: int, tokens: torch.Tensor, x: torch.Tensor, layer0: int, n_layers: int):
+        """dg_debug_forward_hidden: layers layer0.. from the residual stream x [T, d_model] f32."""
+        T = tokens.numel()
+        check(self.lib.dg_debug_forward_hidden(self.h, req, _dev(tokens, "tokens", _I32),
+                                               _dev(x, "x", _F32, shape=(T, self.cfg.d_model)), T, layer0, n_layers),
+              "dg_debug_forward_hidden")
 
     def token_capacity(self) -> int:
         """Rows of the per-pass token buffers (the middle extent of "q")."""

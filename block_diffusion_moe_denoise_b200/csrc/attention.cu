@@ -225,19 +225,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
     const int t = slot * a.Tr + (valid ? qr % a.Tr : 0);
     // Q row -> tensor memory lane `row`, bf16 pairs in columns kTmQ + [0, D/2)
     {
+      // the row's loads go out in groups of 16 x 16 bytes (all in flight at
+      // once), then into tensor memory: two memory round trips for D = 256
       const uint4* src = reinterpret_cast<const uint4*>(a.q + ((size_t)h * a.q_T + t) * D);
+      constexpr int kGroup = D / 32 < 4 ? D / 32 : 4;  // 16-column TMEM stores per group
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t r[16];
+      for (int c0 = 0; c0 < D / 32; c0 += kGroup) {
+        uint4 v[kGroup * 4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint4 v = valid ? src[c * 4 + i] : make_uint4(0, 0, 0, 0);
-          r[4 * i] = v.x;
-          r[4 * i + 1] = v.y;
-          r[4 * i + 2] = v.z;
-          r[4 * i + 3] = v.w;
+        for (int i = 0; i < kGroup * 4; ++i) v[i] = valid ? src[c0 * 4 + i] : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int c = 0; c < kGroup; ++c) {
+          uint32_t r[16];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            r[4 * i] = v[c * 4 + i].x;
+            r[4 * i + 1] = v[c * 4 + i].y;
+            r[4 * i + 2] = v[c * 4 + i].z;
+            r[4 * i + 3] = v[c * 4 + i].w;
+          }
+          tmem_st16_raw(tm_q + lane_off + (c0 + c) * 16, r);
         }
-        tmem_st16_raw(tm_q + lane_off + c * 16, r);
       }
       tmem_st_wait();
       tc_fence_before();

@@ -69,6 +69,15 @@ int dg_op_selfcond(dg_handle* h, int request, const float* d_x, int T, float* d_
  * layer run stay in the workspace; dg_debug_buffer locates them. */
 int dg_debug_forward(dg_handle* h, int req, const int32_t* d_tokens, int T, int n_layers);
 
+/* dg_debug_forward starting inside the stack: the residual stream entering
+ * layer `layer0` is d_x [T, d_model] f32 (device) instead of the embeddings of
+ * d_tokens (which still fix nothing but the pass's shape), and layers layer0 ..
+ * layer0 + n_layers - 1 run (their K/V written to the cache slots [L, L+T));
+ * the LM head runs when the last layer of the stack is among them.  Lets a
+ * test give one deep layer the oracle's own input. */
+int dg_debug_forward_hidden(dg_handle* h, int req, const int32_t* d_tokens, const float* d_x, int T, int layer0,
+                            int n_layers);
+
 /* Byte offset and size, inside the workspace, of a named internal buffer:
  * "x" f32 [T, d] residual stream; "hn" bf16 [T, d] normed input of the last
  * projection; "q" bf16 [Hq, Tcap, D]; "o" bf16 [T, Hq*D]; "u" bf16 [T, d];
@@ -88,9 +97,10 @@ int dg_debug_buffer(const dg_handle* h, const char* name, size_t* offset, size_t
  * stream around every launch of the pass, enable=0 stops, enable=-1 clears the
  * totals.  dg_profile_read (synchronising) returns the summed elapsed ms and
  * launch count of one class: "embed", "rmsnorm", "qkv", "attention", "oproj",
- * "group", "experts_gate_up", "experts_down", "shared_gate_up" (with the
- * router), "shared_down", "lm_head", "lm_combine", "sample", "selfcond",
- * "other". */
+ * "group", "experts_gate_up", "experts_down" (with bf16 experts these two also
+ * run the shared expert's tiles), "router" (bf16 experts), "shared_gate_up"
+ * (FP8 experts: the shared expert's gate|up with the router), "shared_down"
+ * (FP8 experts), "lm_head", "lm_combine", "sample", "selfcond", "other". */
 int dg_profile(dg_handle* h, int enable);
 int dg_profile_read(dg_handle* h, const char* kernel, double* total_ms, int64_t* launches);
 

@@ -117,7 +117,8 @@ def argmax_agreement(gpu_argmax, ora_logits, keep=None, min_rate=0.95):
     return int(counted.sum()), int((~agree).sum()), rate
 
 
-def routing_divergence(gpu_idx_layers, ora_logits_layers, ora_idx_layers, k: int):
+def routing_divergence(gpu_idx_layers, ora_logits_layers, ora_idx_layers, k: int, gpu_logits_layers=None,
+                       noise_sigmas: float = 8.0):
     """Where the GPU's routing first leaves the oracle's, and a check that it only
     ever leaves it at a near-tie.
 
@@ -133,13 +134,24 @@ def routing_divergence(gpu_idx_layers, ora_logits_layers, ora_idx_layers, k: int
     the experts it did not pick minus delta.  Anything else is a routing bug
     and fails here.  After its first divergence a token's hidden state follows
     another (equally valid) branch, so value comparisons use the tokens that
-    have not diverged up to the compared layer."""
+    have not diverged up to the compared layer.
+
+    Deep in a stack the residual stream carries the rounding of every earlier
+    layer, so the GPU's router-logit noise grows with depth.  When the GPU's
+    router logits of every layer are given, the margin at layer l is at least
+    noise_sigmas times sigma_l, the RMS difference between the GPU's and the
+    oracle's router logits over the tokens still on the oracle's routing (the
+    measured noise at that depth)."""
     n_layers = len(gpu_idx_layers)
     T = gpu_idx_layers[0].shape[0]
     first = np.full(T, n_layers)
     for l in range(n_layers):
         r = np.asarray(ora_logits_layers[l], dtype=np.float64)
         delta = ROUTER_GAP_REL * np.sqrt(np.mean(r * r))
+        if gpu_logits_layers is not None:
+            on = first == n_layers
+            dg = np.asarray(gpu_logits_layers[l], dtype=np.float64)[on] - r[on]
+            delta = max(delta, noise_sigmas * float(np.sqrt(np.mean(dg * dg))))
         for t in np.nonzero(first == n_layers)[0]:
             g = set(int(e) for e in gpu_idx_layers[l][t])
             if g == set(int(e) for e in ora_idx_layers[l][t]):
