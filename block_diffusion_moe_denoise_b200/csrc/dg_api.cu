@@ -27,8 +27,6 @@ int pass_slots(int max_req) { return max_req > kPrefillSlots ? max_req : kPrefil
 
 struct LayerMaps {
   CUtensorMap qkv, o, gate, up, down, sgate, sup, sdown, router;
-  CUtensorMap gate128, up128;                     // bf16 expert gate / up rows in 128-row boxes
-  CUtensorMap sgate64, sgate128, sup64, sup128;   // shared gate / up rows as tiles of the expert kernel
 };
 
 struct ReqState {
@@ -80,23 +78,13 @@ bool config_ok(const dg_config* c) {
 
 long long round_cap(long long cap) { return (cap + 63) / 64 * 64; }
 
-// Tiles the shared expert adds to the routed-expert lists of a pass of T tokens.
-long long shared_egu_tiles(const dg_config* c, int T) {
-  return (long long)((c->ffn_shared + 63) / 64) * ((T + kEguRows - 1) / kEguRows);
-}
-long long shared_ed_tiles(const dg_config* c, int T) {
-  return (long long)(c->d_model / 128) * ((T + kEdRows - 1) / kEdRows);
-}
-
 void make_plan(const dg_config* c, int max_req, long long cap_user, Plan* p) {
   const long long cap = round_cap(cap_user);
   const int T = pass_slots(max_req) * c->canvas;
   const int Tcap = (T + 127) / 128 * 128;
   const long long rows = (long long)T * c->top_k;
   const int D = c->head_dim, d = c->d_model;
-  // token tiles: at most one partial tile per expert plus the full ones
-  const long long n_ntg = c->n_experts + (rows + kEguRows - 1) / kEguRows;
-  const long long n_ntd = c->n_experts + (rows + kEdRows - 1) / kEdRows;
+  const long long n_nt = c->n_experts + (rows + kExpertRows - 1) / kExpertRows;
   p->add("err", 64);
   p->add("kv", (size_t)max_req * c->n_layers * 2 * c->n_kv_heads * (size_t)cap * D * 2);
   p->add("x", (size_t)Tcap * d * 4);
@@ -114,8 +102,8 @@ void make_plan(const dg_config* c, int max_req, long long cap_user, Plan* p) {
   p->add("row_pair", (size_t)rows * 4);
   p->add("tile_counts", 64);
   p->add("route_stats", 64);
-  p->add("egu_tiles", (size_t)(n_ntg * (c->ffn_expert / 64) + shared_egu_tiles(c, T)) * 16);
-  p->add("ed_tiles", (size_t)(n_ntd * (d / 128) + shared_ed_tiles(c, T)) * 16);
+  p->add("egu_tiles", (size_t)n_nt * (c->ffn_expert / 64) * 16);
+  p->add("ed_tiles", (size_t)n_nt * (d / 128) * 16);
   p->add("xp", (size_t)rows * d * 2);
   p->add("hp", (size_t)rows * c->ffn_expert * 2);
   p->add("yp", (size_t)rows * d * 4);
@@ -152,8 +140,6 @@ void make_plan(const dg_config* c, int max_req, long long cap_user, Plan* p) {
   p->add("router_logits", (size_t)Tcap * c->n_experts * 4);
   p->add("part", (size_t)kMaxPartSplits * Tcap * d * 4);
   p->add("route_mask", (size_t)2 * c->n_experts * ((T + 31) / 32) * 4);
-  p->add("router_part", (size_t)(Tcap / 128) * kRouterSplits * 128 * c->n_experts * 4);
-  p->add("router_counter", (size_t)(Tcap / 128) * 4);
   p->add("prompt", (size_t)cap_user * 4);
 }
 
@@ -246,9 +232,9 @@ struct KernelProfiler {
 
 const char* const kKernelClass[] = {"embed", "rmsnorm", "qkv", "attention", "oproj", "group",
                                     "experts_gate_up", "experts_down", "shared_gate_up", "shared_down", "lm_head",
-                                    "lm_combine", "sample", "selfcond", "other", "router"};
+                                    "lm_combine", "sample", "selfcond", "other"};
 enum KClass { K_EMBED, K_RMSNORM, K_QKV, K_ATTN, K_OPROJ, K_GROUP, K_EGU, K_ED, K_SGU, K_SD, K_LM, K_LMC, K_SAMPLE,
-              K_SC, K_OTHER, K_ROUTER, K_NCLASS };
+              K_SC, K_OTHER, K_NCLASS };
 static_assert(K_NCLASS <= 16, "profiler tables hold 16 classes");
 
 struct dg_handle {
@@ -268,11 +254,9 @@ struct dg_handle {
   int egu_cap = 0, ed_cap = 0;
   long long kv_req_stride = 0, kv_layer_stride = 0;
   std::vector<LayerMaps> maps;
-  CUtensorMap tm_hn, tm_o, tm_u, tm_hs, tm_embed, tm_k, tm_vt;
-  CUtensorMap tm_u_tile, tm_hs_tile;                      // u and hs in token-tile boxes of the expert kernels
-  CUtensorMap tm_xp[2], tm_hp[3];                         // grouped expert rows: 64/128(/256)-row boxes
+  CUtensorMap tm_hn, tm_o, tm_u, tm_xp, tm_hp, tm_hs, tm_embed, tm_k, tm_vt;
   CUtensorMap tm_sc_gate, tm_sc_up, tm_sc_down, tm_hs_sc;  // self-conditioning MLP and its hidden rows
-  CUtensorMap tm_xq[2], tm_hq[3];                          // FP8 experts: token and hidden codes
+  CUtensorMap tm_xq, tm_hq;                                // FP8 experts: token and hidden codes
   long long cap_user = 0;  // capacity the caller asked for (cap is rounded up to 64)
   ReqState req[DG_MAX_REQUESTS];
   int mask_flip = 0;  // which of the two routing bitmask buffers the next layer uses
@@ -492,45 +476,15 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     sa.w = h->B<float>("w");
     sa.mask = mask_cur;
     sa.err = err;
-    const bool f8 = c.expert_fp8 != 0;
-    // with the shared expert merged (bf16 experts, kSharedInExperts) the router
-    // runs alone (split-K) and the shared expert joins the routed-expert
-    // launches as extra tiles; otherwise the shared gate|up runs in the
-    // router's launch and its down projection split-K
-    const bool merged = !f8 && kSharedInExperts;
-    const int MTr = (T + 127) / 128;
-    const int rsplit = kRouterSplits < d / 64 ? kRouterSplits : d / 64;
-    if (!merged) {
-      LAUNCH(h, K_SGU, 1, run_shared_gate_up(sa, st));
-    } else {
-      RouterArgs ra;
-      ra.tm_u = &h->tm_u;
-      ra.tm_router = &m.router;
-      ra.T = T;
-      ra.d = d;
-      ra.E = c.n_experts;
-      ra.k = k;
-      ra.MW = MW;
-      ra.splits = rsplit;
-      ra.part = h->B<float>("router_part");
-      ra.counter = h->B<unsigned>("router_counter");
-      ra.logits = sa.logits;
-      ra.idx = sa.idx;
-      ra.w = sa.w;
-      ra.mask = mask_cur;
-      ra.err = err;
-      LAUNCH(h, K_ROUTER, 1, run_router(ra, st));
-    }
+    LAUNCH(h, K_SGU, 1, run_shared_gate_up(sa, st));
     GroupArgs ga;
     ga.idx = h->B<int>("idx");
     ga.w = h->B<float>("w");
     ga.T = T;
     ga.k = k;
     ga.E = c.n_experts;
-    // hidden-unit blocks per expert of the gate|up tiles: 128 units (bf16), 64 (FP8)
-    ga.FJ = f8 ? c.ffn_expert / 64 : (c.ffn_expert + 64 * kEguAcc - 1) / (64 * kEguAcc);
-    // output-feature blocks per expert of the down tiles: 128 x kEdAcc (bf16), 128 (FP8)
-    ga.MD = f8 ? d / 128 : d / (128 * kEdAcc);
+    ga.FJ = c.ffn_expert / 64;
+    ga.MD = d / 128;
     ga.egu_cap = h->egu_cap;
     ga.ed_cap = h->ed_cap;
     ga.counts = h->B<int>("counts");
@@ -545,27 +499,17 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     ga.ed_count = h->B<int>("tile_counts") + 1;
     ga.route_stats = h->B<unsigned long long>("route_stats");
     ga.err = err;
-    if (merged) {
-      ga.sh_fj = (c.ffn_shared + 64 * kEguAcc - 1) / (64 * kEguAcc);
-      ga.sh_ntg = (T + kEguRows - 1) / kEguRows;
-      ga.sh_md = d / (128 * kEdAcc);
-      ga.sh_ntd = (T + kEdRows - 1) / kEdRows;
-      ga.router_counter = h->B<unsigned>("router_counter");
-      ga.router_mt = MTr;
-    }
+    const bool f8 = c.expert_fp8 != 0;
     LAUNCH(h, K_GROUP, 1,
            run_route(h->B<bf16>("u"), d, h->B<bf16>("xp"), mask_cur, mask_nxt, MW, ga, st,
                      f8 ? h->B<uint8_t>("xq") : nullptr, f8 ? h->B<float>("xs") : nullptr));
 
     ExpertArgs ea;
-    ea.tm_gate[0] = &m.gate;
-    ea.tm_gate[1] = &m.gate128;
-    ea.tm_up[0] = &m.up;
-    ea.tm_up[1] = &m.up128;
-    ea.tm_xp[0] = &h->tm_xp[0];
-    ea.tm_xp[1] = &h->tm_xp[1];
+    ea.tm_gate = &m.gate;
+    ea.tm_up = &m.up;
+    ea.tm_xp = &h->tm_xp;
     ea.tm_down = &m.down;
-    for (int i = 0; i < 3; ++i) ea.tm_hp[i] = &h->tm_hp[i];
+    ea.tm_hp = &h->tm_hp;
     ea.d = d;
     ea.fe = c.ffn_expert;
     ea.num_sms = h->num_sms;
@@ -581,9 +525,8 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     ea.err = err;
     if (f8) {
       // E4M3 weight codes and token rows; the SwiGLU rows are quantised per row before down
-      ea.tm_xp[0] = &h->tm_xq[0];
-      ea.tm_xp[1] = &h->tm_xq[1];
-      for (int i = 0; i < 3; ++i) ea.tm_hp[i] = &h->tm_hq[i];
+      ea.tm_xp = &h->tm_xq;
+      ea.tm_hp = &h->tm_hq;
       ea.s_gate = (const float*)w.w_gate_scale;
       ea.s_up = (const float*)w.w_up_scale;
       ea.s_down = (const float*)w.w_down_scale;
@@ -592,24 +535,6 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
       LAUNCH(h, K_EGU, 1, run_experts_gate_up_fp8(ea, st));
       LAUNCH(h, K_ED, 1, run_quant_rows(ea.hp, c.ffn_expert, T * k, h->B<uint8_t>("hq"), h->B<float>("hsq"), st));
       LAUNCH(h, K_ED, 1, run_experts_down_fp8(ea, st));
-    } else if (merged) {
-      ea.E = c.n_experts;
-      ea.T = T;
-      ea.fs = c.ffn_shared;
-      ea.tm_sgate[0] = &m.sgate64;
-      ea.tm_sgate[1] = &m.sgate128;
-      ea.tm_sup[0] = &m.sup64;
-      ea.tm_sup[1] = &m.sup128;
-      ea.tm_u = &h->tm_u_tile;
-      ea.tm_sdown = &m.sdown;
-      ea.tm_hs = &h->tm_hs_tile;
-      ea.hs = h->B<bf16>("hs");
-      ea.ys = part;  // the shared expert's output rows, slice 0 of the partial buffer
-      LAUNCH(h, K_EGU, 1, run_experts_gate_up(ea, st));
-      LAUNCH(h, K_ED, 1, run_experts_down(ea, st));
-      pending_k = k;
-      pending_parts = 1;
-      continue;
     } else {
       LAUNCH(h, K_EGU, 1, run_experts_gate_up(ea, st));
       LAUNCH(h, K_ED, 1, run_experts_down(ea, st));
@@ -773,10 +698,9 @@ int dg_init(const dg_config* cfg, const dg_weights* wts, int max_requests, int64
   h->kv_layer_stride = 2ll * c.n_kv_heads * h->cap * D;
   h->kv_req_stride = h->kv_layer_stride * c.n_layers;
   const long long rows = (long long)h->T_max * c.top_k;
-  const long long n_ntg = c.n_experts + (rows + kEguRows - 1) / kEguRows;
-  const long long n_ntd = c.n_experts + (rows + kEdRows - 1) / kEdRows;
-  h->egu_cap = (int)(n_ntg * (c.ffn_expert / 64) + shared_egu_tiles(&c, h->T_max));
-  h->ed_cap = (int)(n_ntd * (d / 128) + shared_ed_tiles(&c, h->T_max));
+  const long long n_nt = c.n_experts + (rows + kExpertRows - 1) / kExpertRows;
+  h->egu_cap = (int)(n_nt * (c.ffn_expert / 64));
+  h->ed_cap = (int)(n_nt * (d / 128));
 
   bool ok = true;
   const int qkv_rows = (c.n_q_heads + 2 * c.n_kv_heads) * D;
@@ -796,30 +720,19 @@ int dg_init(const dg_config* cfg, const dg_weights* wts, int max_requests, int64
     } else {
       ok = ok && make_map(&m.gate, w.w_gate, d, E * c.ffn_expert, 64);
       ok = ok && make_map(&m.up, w.w_up, d, E * c.ffn_expert, 64);
-      ok = ok && make_map(&m.gate128, w.w_gate, d, E * c.ffn_expert, 128);
-      ok = ok && make_map(&m.up128, w.w_up, d, E * c.ffn_expert, 128);
       ok = ok && make_map(&m.down, w.w_down, c.ffn_expert, E * d, 128);
     }
     ok = ok && make_map(&m.sgate, w.ws_gate, d, c.ffn_shared, 32);
     ok = ok && make_map(&m.sup, w.ws_up, d, c.ffn_shared, 32);
-    ok = ok && make_map(&m.sgate64, w.ws_gate, d, c.ffn_shared, 64);
-    ok = ok && make_map(&m.sgate128, w.ws_gate, d, c.ffn_shared, 128);
-    ok = ok && make_map(&m.sup64, w.ws_up, d, c.ffn_shared, 64);
-    ok = ok && make_map(&m.sup128, w.ws_up, d, c.ffn_shared, 128);
     ok = ok && make_map(&m.router, w.w_router, d, E, (int)E);
     ok = ok && make_map(&m.sdown, w.ws_down, c.ffn_shared, d, 128);
   }
   ok = ok && make_map(&h->tm_hn, h->B<bf16>("hn"), d, h->Tcap, 128);
   ok = ok && make_map(&h->tm_o, h->B<bf16>("o"), (long long)c.n_q_heads * D, h->Tcap, 256);
   ok = ok && make_map(&h->tm_u, h->B<bf16>("u"), d, h->Tcap, 128);
-  ok = ok && make_map(&h->tm_xp[0], h->B<bf16>("xp"), d, rows, 64);
-  ok = ok && make_map(&h->tm_xp[1], h->B<bf16>("xp"), d, rows, 128);
-  ok = ok && make_map(&h->tm_hp[0], h->B<bf16>("hp"), c.ffn_expert, rows, 64);
-  ok = ok && make_map(&h->tm_hp[1], h->B<bf16>("hp"), c.ffn_expert, rows, 128);
-  ok = ok && make_map(&h->tm_hp[2], h->B<bf16>("hp"), c.ffn_expert, rows, 256);
+  ok = ok && make_map(&h->tm_xp, h->B<bf16>("xp"), d, rows, kExpertRows);
+  ok = ok && make_map(&h->tm_hp, h->B<bf16>("hp"), c.ffn_expert, rows, kExpertRows);
   ok = ok && make_map(&h->tm_hs, h->B<bf16>("hs"), c.ffn_shared, h->Tcap, 256);
-  ok = ok && make_map(&h->tm_u_tile, h->B<bf16>("u"), d, h->Tcap, kEguRows);
-  ok = ok && make_map(&h->tm_hs_tile, h->B<bf16>("hs"), c.ffn_shared, h->Tcap, kEdRows);
   ok = ok && make_map(&h->tm_embed, h->embed, d, c.vocab, 256);
   {
     const long long kv_elems = (long long)max_requests * h->kv_req_stride;
@@ -827,11 +740,8 @@ int dg_init(const dg_config* cfg, const dg_weights* wts, int max_requests, int64
     ok = ok && make_map(&h->tm_vt, h->B<bf16>("kv"), h->cap, kv_elems / h->cap, D);
   }
   if (c.expert_fp8) {
-    ok = ok && make_map_u8(&h->tm_xq[0], h->B<uint8_t>("xq"), d, rows, 64);
-    ok = ok && make_map_u8(&h->tm_xq[1], h->B<uint8_t>("xq"), d, rows, 128);
-    ok = ok && make_map_u8(&h->tm_hq[0], h->B<uint8_t>("hq"), c.ffn_expert, rows, 64);
-    ok = ok && make_map_u8(&h->tm_hq[1], h->B<uint8_t>("hq"), c.ffn_expert, rows, 128);
-    ok = ok && make_map_u8(&h->tm_hq[2], h->B<uint8_t>("hq"), c.ffn_expert, rows, 256);
+    ok = ok && make_map_u8(&h->tm_xq, h->B<uint8_t>("xq"), d, rows, kExpertRows);
+    ok = ok && make_map_u8(&h->tm_hq, h->B<uint8_t>("hq"), c.ffn_expert, rows, kExpertRows);
   }
   if (c.ffn_selfcond > 0) {
     const int f = c.ffn_selfcond;
@@ -853,8 +763,6 @@ int dg_init(const dg_config* cfg, const dg_weights* wts, int max_requests, int64
       cudaMemsetAsync(h->B<int>("err"), 0, 64, h->st) != cudaSuccess ||
       cudaMemsetAsync(h->B<int>("route_stats"), 0, 64, h->st) != cudaSuccess ||
       cudaMemsetAsync(h->B<int>("route_mask"), 0, h->plan.buf.at("route_mask").second, h->st) != cudaSuccess ||
-      cudaMemsetAsync(h->B<int>("router_counter"), 0, h->plan.buf.at("router_counter").second, h->st) !=
-          cudaSuccess ||
       cudaMemsetAsync(h->B<bf16>("kv"), 0, h->plan.buf.at("kv").second, h->st) != cudaSuccess ||
       cudaMemsetAsync(h->B<int>("remaining"), 0, (size_t)max_requests * 4, h->st) != cudaSuccess ||
       cudaStreamSynchronize(h->st) != cudaSuccess) {

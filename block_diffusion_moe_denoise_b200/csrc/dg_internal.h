@@ -46,22 +46,7 @@ struct QkvArgs {
   int* err;
 };
 constexpr int kMaxPartSplits = 8;
-// Token rows per routed-expert GEMM tile (the MMA's N).  The expert GEMMs
-// stream weights from HBM, and their speed is set by the weight bytes each SM
-// keeps in flight; a narrow token tile leaves most of the shared-memory ring
-// to the weights (measured on B200: 128- and 256-row token tiles were slower
-// than 64 for both GEMMs of the benchmark's routing).
-constexpr int kEguRows = 64;
-constexpr int kEdRows = 64;
-// Accumulators (weight tiles of 128 rows) per tile of the bf16 expert GEMMs:
-// gate|up with 2 holds 128 hidden units (gate and up rows in separate tiles),
-// with 1 holds 64 (gate and up rows stacked in one tile); down with 2 holds
-// 256 output features, with 1 holds 128.
-constexpr int kEguAcc = 2;
-constexpr int kEdAcc = 2;
-// The shared expert: in the routed-expert launches as extra tiles (the router
-// then runs alone), or in the router's launch with its down projection split-K.
-constexpr bool kSharedInExperts = true;
+constexpr int kExpertRows = 64;  // token rows per routed-expert GEMM tile
 struct WpartArgs {
   const CUtensorMap* tm_w;  // weights [d, K], 128-row boxes
   const CUtensorMap* tm_x;  // activations [Tcap, K], 256-row boxes
@@ -70,11 +55,7 @@ struct WpartArgs {
   int* err;
 };
 struct ExpertArgs {
-  const CUtensorMap* tm_gate[2];  // expert gate rows [E*fe, d]: 64-row boxes, 128-row boxes (bf16 only)
-  const CUtensorMap* tm_up[2];    // expert up rows, likewise
-  const CUtensorMap* tm_down;
-  const CUtensorMap* tm_xp[2];  // grouped token rows, 64- and 128-row boxes
-  const CUtensorMap* tm_hp[3];  // grouped SwiGLU rows, 64-, 128- and 256-row boxes
+  const CUtensorMap *tm_gate, *tm_up, *tm_xp, *tm_down, *tm_hp;
   int d, fe, num_sms;
   const int4* egu_tiles;
   const int* egu_count;
@@ -88,31 +69,7 @@ struct ExpertArgs {
   int* err;
   // FP8 experts: per-row scales of the weight codes and of the token / hidden codes
   const float *s_gate = nullptr, *s_up = nullptr, *s_down = nullptr, *s_x = nullptr, *s_h = nullptr;
-  // shared expert as extra tiles of the bf16 kernels (expert id E); the tile
-  // lists from the grouping kernel hold its tiles when shared_tiles is set
-  int E = 0, T = 0, fs = 0;
-  const CUtensorMap* tm_sgate[2] = {nullptr, nullptr};  // ws_gate, 64/128-row boxes
-  const CUtensorMap* tm_sup[2] = {nullptr, nullptr};    // ws_up, 64/128-row boxes
-  const CUtensorMap* tm_u = nullptr;                    // normed tokens [Tcap, d], kEguRows-row boxes
-  const CUtensorMap* tm_sdown = nullptr;                // ws_down [d, fs], 128-row boxes
-  const CUtensorMap* tm_hs = nullptr;                   // shared SwiGLU rows [Tcap, fs], kEdRows-row boxes
-  bf16* hs = nullptr;                                   // [Tcap, fs]
-  float* ys = nullptr;                                  // [Tcap, d] shared-expert output
 };
-// Router alone (split-K, last-arriving CTA of a token tile reduces and picks
-// the top-k): tokens [Tcap, d] x w_router [E, d]^T.
-struct RouterArgs {
-  const CUtensorMap *tm_u, *tm_router;
-  int T, d, E, k, MW, splits;
-  float* part;        // [MT][splits][128][E]
-  unsigned* counter;  // [MT], zero between launches
-  float* logits;      // [Tcap, E]
-  int* idx;           // [T, k]
-  float* w;           // [T, k]
-  unsigned* mask;     // [E][MW], zero on entry
-  int* err;
-};
-constexpr int kRouterSplits = 4;
 struct SharedArgs {
   const CUtensorMap *tm_u, *tm_gate, *tm_up, *tm_router;
   int T, d, fs, num_sms;
@@ -163,7 +120,6 @@ cudaError_t run_experts_down(const ExpertArgs& a, cudaStream_t st);
 cudaError_t run_experts_gate_up_fp8(const ExpertArgs& a, cudaStream_t st);
 cudaError_t run_experts_down_fp8(const ExpertArgs& a, cudaStream_t st);
 cudaError_t run_shared_gate_up(const SharedArgs& a, cudaStream_t st);
-cudaError_t run_router(const RouterArgs& a, cudaStream_t st);
 cudaError_t run_lm_head(const LmArgs& a, int* grid_out, cudaStream_t st);
 size_t gemm_smem_bytes_max();
 
@@ -200,11 +156,6 @@ struct GroupArgs {
   int* ed_count;
   unsigned long long* route_stats;  // [0] += experts touched, [1] += launches (may be null)
   int* err;
-  // shared-expert tiles at the head of the lists (0: none): hidden blocks x
-  // token tiles of the gate|up kernel, feature blocks x token tiles of down
-  int sh_fj = 0, sh_ntg = 0, sh_md = 0, sh_ntd = 0;
-  unsigned* router_counter = nullptr;  // arrival counters of the router launch, cleared here
-  int router_mt = 0;
 };
 cudaError_t run_group(const GroupArgs& a, cudaStream_t st);
 // the grouping above from the token bitmasks `mask` ([E][MW] words, MW fixed by

@@ -261,225 +261,135 @@ struct P_WPART : ProblemBase {
 };
 
 // ---------------------------------------------------------------------------
-// Routed experts, gate|up + SwiGLU.  Tile (e, j, nt): hidden units j*128..+127
-// of expert e (the last block of an expert may hold fewer: 704 = 5*128 + 64)
-// for its tokens nt*kEguRows.. (rows of the expert-grouped buffer, at most
-// kEguRows = 128: the MMA's N).  Two accumulators per tile (NACC = 2): A tile
-// 0 holds the 128 W_gate rows, A tile 1 the W_up rows of the same hidden
-// units, so a hidden unit's gate and up values land in the same TMEM lane and
-// the SwiGLU needs no exchange between threads.  An expert with many tokens
-// takes few wide tiles, so its weights are streamed fewer times and each
-// k-block's barrier round trip carries four times the MMA work of a 64 x 64
-// tile.  Weight rows of a partial last block come in 64-row boxes (no bytes
-// of the next expert are fetched; the stale upper half of the A tile feeds
-// accumulator lanes the epilogue ignores); token rows in 64-row boxes when
-// the tile has no more.
+// Routed experts, gate|up + SwiGLU.  Tile (e, j, nt): hidden units j*64..+63 of
+// expert e for its tokens nt*64..+63 (rows of the expert-grouped buffer).
+// A rows 0..63 = W_gate rows, 64..127 = W_up rows of the same hidden units.
 // ---------------------------------------------------------------------------
-DG_DEVINL int rows_box(int n_valid) { return n_valid <= 64 ? 64 : (n_valid <= 128 ? 128 : 256); }
-
-//
-// The shared expert runs in the same launch as extra tiles (expert id E, all
-// T tokens of the pass, read straight from the normed rows u; hidden blocks of
-// the shared width fs; SwiGLU rows to hs): its gate|up weights stream while
-// the routed tiles run, instead of in a launch of their own.  The grouping
-// kernel puts these tiles first in the list.
-template <int NA>
-struct P_EGU_T : ProblemBase {
-  // NA = 2: hidden blocks of 128 units, gate and up rows in two A tiles / two
-  // accumulators.  NA = 1: hidden blocks of 64 units, A rows 0..63 = W_gate and
-  // 64..127 = W_up of the same units in one accumulator; the epilogue pairs the
-  // two halves through shared memory.
-  static constexpr int NACC = NA;
-  static constexpr int UNITS = NA == 2 ? 128 : 64;  // hidden units per tile
-  static constexpr int BN = kEguRows, STAGES = NA == 2 ? 5 : 4, KB = NA == 2 ? 1 : 2, B_STAGE = BN * 128;
-  static constexpr int TMEM_COLS = 2 * NACC * BN;
-  static constexpr int EP_SMEM = NA == 2 ? 0 : 64 * 17 * 4;
+struct P_EGU : ProblemBase {
+  static constexpr int BN = kExpertRows, STAGES = 4, KB = 2, B_STAGE = BN * 128, TMEM_COLS = 128;
+  static constexpr int EP_SMEM = 64 * 17 * 4;
   struct Params {
-    CUtensorMap tmG[2];   // w_gate as [E*fe, d]: 64- and 128-row boxes
-    CUtensorMap tmU[2];   // w_up   as [E*fe, d]: 64- and 128-row boxes
-    CUtensorMap tmX[2];   // expert-grouped tokens [rows_cap, d], 64- and 128-row boxes
-    CUtensorMap tmSG[2];  // shared ws_gate [fs, d]: 64- and 128-row boxes
-    CUtensorMap tmSU[2];  // shared ws_up [fs, d]: 64- and 128-row boxes
-    CUtensorMap tmXS;     // normed tokens u [Tcap, d], BN-row boxes
-    int nk, fe, E, T, fs;
+    CUtensorMap tmG;  // w_gate as [E*fe, d]
+    CUtensorMap tmU;  // w_up   as [E*fe, d]
+    CUtensorMap tmX;  // expert-grouped tokens [rows_cap, d], 64-row boxes
+    int nk, fe;
     const int4* tiles;
     const int* n_tiles;
     const int* counts;
     const int* offsets;
     __nv_bfloat16* hp;  // [rows_cap, fe]
-    __nv_bfloat16* hs;  // [Tcap, fs] shared SwiGLU rows
     int* err;
   };
   DG_DEVINL static void prefetch(const Params& p) {
-    for (int i = 0; i < 2; ++i) {
-      tma_prefetch_desc(&p.tmG[i]);
-      tma_prefetch_desc(&p.tmU[i]);
-      tma_prefetch_desc(&p.tmX[i]);
-      tma_prefetch_desc(&p.tmSG[i]);
-      tma_prefetch_desc(&p.tmSU[i]);
-    }
-    tma_prefetch_desc(&p.tmXS);
+    tma_prefetch_desc(&p.tmG);
+    tma_prefetch_desc(&p.tmU);
+    tma_prefetch_desc(&p.tmX);
   }
   DG_DEVINL static int num_tiles(const Params& p) { return *p.n_tiles; }
   DG_DEVINL static Tile tile(const Params& p, int v) {
     const int4 tt = p.tiles[v];
     Tile t;
-    t.a = tt.x;  // expert (E: the shared expert)
-    t.b = tt.y;  // hidden block of UNITS units
+    t.a = tt.x;  // expert
+    t.b = tt.y;  // hidden-unit block
     const int nt = tt.z;
-    const bool sh = t.a == p.E;
-    const int n_valid = min(BN, (sh ? p.T : p.counts[t.a]) - nt * BN);
+    const int n_valid = min(BN, p.counts[t.a] - nt * BN);
     t.valid = n_valid > 0;
     t.c = n_valid;
-    t.d = (sh ? 0 : p.offsets[t.a]) + nt * BN;           // first token row (u) / grouped row (xp)
-    t.e = min(UNITS, (sh ? p.fs : p.fe) - t.b * UNITS);  // hidden units of this block
+    t.d = p.offsets[t.a] + nt * BN;  // first grouped row
     t.nk = p.nk;
     t.n_mma = round_up16(n_valid);
     return t;
   }
-  DG_DEVINL static uint32_t tx_bytes(const Params& p, const Tile& t) {
-    const uint32_t xb = t.a == p.E ? (uint32_t)BN : (uint32_t)rows_box(t.c);
-    const uint32_t wrows = NA == 2 ? (t.e <= 64 ? 64u : 128u) : 64u;  // rows per weight box
-    return 2u * wrows * 128u + xb * 128u;
-  }
+  DG_DEVINL static uint32_t tx_bytes(const Params&, const Tile&) { return kAStage + B_STAGE; }
   DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
-    const int wb = NA == 2 && t.e > 64 ? 1 : 0;
-    const uint32_t su = NA == 2 ? sa + kAStage : sa + 64 * 128;  // up rows: second A tile / lower half
-    const bool sh = t.a == p.E;
-    const int r = sh ? t.b * UNITS : t.a * p.fe + t.b * UNITS;
-    tma_load_2d(sa, sh ? &p.tmSG[wb] : &p.tmG[wb], kb * 64, r, bar);
-    tma_load_2d(su, sh ? &p.tmSU[wb] : &p.tmU[wb], kb * 64, r, bar);
-    tma_load_2d(sb, sh ? &p.tmXS : &p.tmX[t.c <= 64 ? 0 : 1], kb * 64, t.d, bar);
+    const int r = t.a * p.fe + t.b * 64;
+    tma_load_2d(sa, &p.tmG, kb * 64, r, bar);
+    tma_load_2d(sa + 64 * 128, &p.tmU, kb * 64, r, bar);
+    tma_load_2d(sb, &p.tmX, kb * 64, t.d, bar);
   }
   DG_DEVINL static void epilogue(const Params& p, const Tile& t, uint32_t taddr, int, int, int row, uint8_t* ep) {
-    const bool sh = t.a == p.E;
-    const int ld = sh ? p.fs : p.fe;
-    if constexpr (NA == 2) {
-      const bool live = row < t.e;
-      __nv_bfloat16* dst = (sh ? p.hs : p.hp) + (size_t)t.d * ld + t.b * UNITS + row;
-      for (int c0 = 0; c0 < t.n_mma; c0 += 16) {
-        float g[16], u[16];
-        tmem_ld16(taddr + c0, g);
-        tmem_ld16(taddr + BN + c0, u);
-        if (live) {
+    float* xch = reinterpret_cast<float*>(ep);
+    for (int c0 = 0; c0 < t.n_mma; c0 += 16) {
+      float v[16];
+      tmem_ld16(taddr + c0, v);
+      if (row >= 64) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            if (c0 + i < t.c) dst[(size_t)(c0 + i) * ld] = f2bf(silu_f(g[i]) * u[i]);
+        for (int i = 0; i < 16; ++i) xch[(row - 64) * 17 + i] = v[i];
+      }
+      named_bar_sync(1, 128);
+      if (row < 64) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int c = c0 + i;
+          if (c < t.c) {
+            const float h = silu_f(v[i]) * xch[row * 17 + i];
+            p.hp[(size_t)(t.d + c) * p.fe + t.b * 64 + row] = f2bf(h);
+          }
         }
       }
-    } else {
-      float* xch = reinterpret_cast<float*>(ep);
-      __nv_bfloat16* dst = (sh ? p.hs : p.hp) + (size_t)t.d * ld + t.b * UNITS + row;
-      for (int c0 = 0; c0 < t.n_mma; c0 += 16) {
-        float v[16];
-        tmem_ld16(taddr + c0, v);
-        if (row >= 64) {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) xch[(row - 64) * 17 + i] = v[i];
-        }
-        named_bar_sync(1, 128);
-        if (row < 64) {
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            if (c0 + i < t.c) dst[(size_t)(c0 + i) * ld] = f2bf(silu_f(v[i]) * xch[row * 17 + i]);
-        }
-        named_bar_sync(1, 128);
-      }
+      named_bar_sync(1, 128);
     }
   }
 };
-using P_EGU = P_EGU_T<kEguAcc>;
 
 // ---------------------------------------------------------------------------
-// Routed experts, down projection.  Tile (e, m, nt): output features
-// m*256..+255 of expert e (two accumulators of 128 W_down rows each, NACC = 2,
-// so one B tile of SwiGLU rows serves twice the weight rows) for its grouped
-// rows nt*kEdRows..; each row scaled by its gate weight.
+// Routed experts, down projection.  Tile (e, m, nt): output features m*128..+127
+// of expert e for its grouped rows nt*64..+63; each row scaled by its gate weight.
 // ---------------------------------------------------------------------------
-//
-// The shared expert's down projection runs in the same launch (expert id E:
-// W_sd rows against the shared SwiGLU rows hs of all T tokens, K = fs; its
-// fp32 output rows go to ys, added with weight 1 by the next norm kernel).
-// Its tiles have the longest K chain and come first in the list.
-template <int NA>
-struct P_ED_T : ProblemBase {
-  static constexpr int NACC = NA;  // 128-feature blocks per tile against one B tile
-  static constexpr int FB = 128 * NA;  // output features per tile
-  static constexpr int BN = kEdRows, STAGES = NA == 2 ? 5 : 4, KB = NA == 2 ? 1 : 2, B_STAGE = BN * 128;
-  static constexpr int TMEM_COLS = 2 * NACC * BN;
+struct P_ED : ProblemBase {
+  static constexpr int BN = kExpertRows, STAGES = 4, KB = 2, B_STAGE = BN * 128, TMEM_COLS = 128;
   struct Params {
-    CUtensorMap tmW;     // w_down as [E*d, fe], 128-row boxes
-    CUtensorMap tmH[3];  // hidden [rows_cap, fe], 64-, 128- and 256-row boxes
-    CUtensorMap tmSW;    // shared ws_down [d, fs], 128-row boxes
-    CUtensorMap tmHS;    // shared SwiGLU rows hs [Tcap, fs], BN-row boxes
-    int nk, d, E, T, nks;
+    CUtensorMap tmW;  // w_down as [E*d, fe]
+    CUtensorMap tmH;  // hidden [rows_cap, fe], 64-row boxes
+    int nk, d;
     const int4* tiles;
     const int* n_tiles;
     const int* counts;
     const int* offsets;
     const float* row_weight;
     float* yp;  // [rows_cap, d]
-    float* ys;  // [Tcap, d] shared-expert output
     int* err;
   };
   DG_DEVINL static void prefetch(const Params& p) {
     tma_prefetch_desc(&p.tmW);
-    for (int i = 0; i < 3; ++i) tma_prefetch_desc(&p.tmH[i]);
-    tma_prefetch_desc(&p.tmSW);
-    tma_prefetch_desc(&p.tmHS);
+    tma_prefetch_desc(&p.tmH);
   }
   DG_DEVINL static int num_tiles(const Params& p) { return *p.n_tiles; }
   DG_DEVINL static Tile tile(const Params& p, int v) {
     const int4 tt = p.tiles[v];
     Tile t;
-    t.a = tt.x;  // expert (E: the shared expert)
-    t.b = tt.y;  // block of FB output features (NACC accumulators of 128)
+    t.a = tt.x;  // expert
+    t.b = tt.y;  // 128-feature block
     const int nt = tt.z;
-    const bool sh = t.a == p.E;
-    const int n_valid = min(BN, (sh ? p.T : p.counts[t.a]) - nt * BN);
+    const int n_valid = min(BN, p.counts[t.a] - nt * BN);
     t.valid = n_valid > 0;
     t.c = n_valid;
-    t.d = (sh ? 0 : p.offsets[t.a]) + nt * BN;
-    t.nk = sh ? p.nks : p.nk;
+    t.d = p.offsets[t.a] + nt * BN;
+    t.nk = p.nk;
     t.n_mma = round_up16(n_valid);
     return t;
   }
-  DG_DEVINL static uint32_t tx_bytes(const Params& p, const Tile& t) {
-    return NACC * kAStage + (t.a == p.E ? BN : rows_box(t.c)) * 128;
-  }
+  DG_DEVINL static uint32_t tx_bytes(const Params&, const Tile&) { return kAStage + B_STAGE; }
   DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
-    const bool sh = t.a == p.E;
-    const int r = sh ? t.b * FB : t.a * p.d + t.b * FB;
-#pragma unroll
-    for (int ai = 0; ai < NACC; ++ai)
-      tma_load_2d(sa + ai * kAStage, sh ? &p.tmSW : &p.tmW, kb * 64, r + ai * 128, bar);
-    tma_load_2d(sb, sh ? &p.tmHS : &p.tmH[t.c <= 64 ? 0 : (t.c <= 128 ? 1 : 2)], kb * 64, t.d, bar);
+    tma_load_2d(sa, &p.tmW, kb * 64, t.a * p.d + t.b * 128, bar);
+    tma_load_2d(sb, &p.tmH, kb * 64, t.d, bar);
   }
   DG_DEVINL static void epilogue(const Params& p, const Tile& t, uint32_t taddr, int, int, int row, uint8_t*) {
-    const bool sh = t.a == p.E;
+    const int f = t.b * 128 + row;
+    for (int c0 = 0; c0 < t.n_mma; c0 += 16) {
+      float v[16];
+      tmem_ld16(taddr + c0, v);
 #pragma unroll
-    for (int ai = 0; ai < NACC; ++ai) {
-      const int f = t.b * FB + ai * 128 + row;
-      for (int c0 = 0; c0 < t.n_mma; c0 += 16) {
-        float v[16];
-        tmem_ld16(taddr + ai * BN + c0, v);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int c = c0 + i;
-          if (c < t.c) {
-            const int r = t.d + c;
-            if (sh)
-              p.ys[(size_t)r * p.d + f] = v[i];
-            else
-              p.yp[(size_t)r * p.d + f] = p.row_weight[r] * v[i];
-          }
+      for (int i = 0; i < 16; ++i) {
+        const int c = c0 + i;
+        if (c < t.c) {
+          const int r = t.d + c;
+          p.yp[(size_t)r * p.d + f] = p.row_weight[r] * v[i];
         }
       }
     }
   }
 };
-
-using P_ED = P_ED_T<kEdAcc>;
 
 // ---------------------------------------------------------------------------
 // FP8 (E4M3) routed experts: the same tiles as P_EGU / P_ED with E4M3 weight
@@ -490,12 +400,12 @@ using P_ED = P_ED_T<kEdAcc>;
 // ---------------------------------------------------------------------------
 struct P_EGU8 : ProblemBase {
   static constexpr bool F8 = true;
-  static constexpr int BN = kEguRows, STAGES = 4, KB = 2, B_STAGE = BN * 128, TMEM_COLS = 2 * BN;
+  static constexpr int BN = kExpertRows, STAGES = 4, KB = 2, B_STAGE = BN * 128, TMEM_COLS = 128;
   static constexpr int EP_SMEM = 64 * 17 * 4;
   struct Params {
-    CUtensorMap tmG;     // w_gate codes as [E*fe, d] bytes
-    CUtensorMap tmU;     // w_up codes as [E*fe, d] bytes
-    CUtensorMap tmX[2];  // grouped token codes [rows_cap, d] bytes, 64- and 128-row boxes
+    CUtensorMap tmG;  // w_gate codes as [E*fe, d] bytes
+    CUtensorMap tmU;  // w_up codes as [E*fe, d] bytes
+    CUtensorMap tmX;  // grouped token codes [rows_cap, d] bytes, 64-row boxes
     int nk, fe;
     const int4* tiles;
     const int* n_tiles;
@@ -510,8 +420,7 @@ struct P_EGU8 : ProblemBase {
   DG_DEVINL static void prefetch(const Params& p) {
     tma_prefetch_desc(&p.tmG);
     tma_prefetch_desc(&p.tmU);
-    tma_prefetch_desc(&p.tmX[0]);
-    tma_prefetch_desc(&p.tmX[1]);
+    tma_prefetch_desc(&p.tmX);
   }
   DG_DEVINL static int num_tiles(const Params& p) { return *p.n_tiles; }
   DG_DEVINL static Tile tile(const Params& p, int v) {
@@ -528,12 +437,12 @@ struct P_EGU8 : ProblemBase {
     t.n_mma = round_up16(n_valid);
     return t;
   }
-  DG_DEVINL static uint32_t tx_bytes(const Params&, const Tile& t) { return kAStage + rows_box(t.c) * 128; }
+  DG_DEVINL static uint32_t tx_bytes(const Params&, const Tile&) { return kAStage + B_STAGE; }
   DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
     const int r = t.a * p.fe + t.b * 64;
     tma_load_2d(sa, &p.tmG, kb * 128, r, bar);
     tma_load_2d(sa + 64 * 128, &p.tmU, kb * 128, r, bar);
-    tma_load_2d(sb, &p.tmX[t.c <= 64 ? 0 : 1], kb * 128, t.d, bar);
+    tma_load_2d(sb, &p.tmX, kb * 128, t.d, bar);
   }
   DG_DEVINL static void epilogue(const Params& p, const Tile& t, uint32_t taddr, int, int, int row, uint8_t* ep) {
     float* xch = reinterpret_cast<float*>(ep);
@@ -566,10 +475,10 @@ struct P_EGU8 : ProblemBase {
 
 struct P_ED8 : ProblemBase {
   static constexpr bool F8 = true;
-  static constexpr int BN = kEdRows, STAGES = 4, KB = 2, B_STAGE = BN * 128, TMEM_COLS = 2 * BN;
+  static constexpr int BN = kExpertRows, STAGES = 4, KB = 2, B_STAGE = BN * 128, TMEM_COLS = 128;
   struct Params {
-    CUtensorMap tmW;     // w_down codes as [E*d, fe] bytes
-    CUtensorMap tmH[3];  // hidden codes [rows_cap, fe] bytes, 64-, 128- and 256-row boxes
+    CUtensorMap tmW;  // w_down codes as [E*d, fe] bytes
+    CUtensorMap tmH;  // hidden codes [rows_cap, fe] bytes, 64-row boxes
     int nk, d;
     const int4* tiles;
     const int* n_tiles;
@@ -583,7 +492,7 @@ struct P_ED8 : ProblemBase {
   };
   DG_DEVINL static void prefetch(const Params& p) {
     tma_prefetch_desc(&p.tmW);
-    for (int i = 0; i < 3; ++i) tma_prefetch_desc(&p.tmH[i]);
+    tma_prefetch_desc(&p.tmH);
   }
   DG_DEVINL static int num_tiles(const Params& p) { return *p.n_tiles; }
   DG_DEVINL static Tile tile(const Params& p, int v) {
@@ -600,10 +509,10 @@ struct P_ED8 : ProblemBase {
     t.n_mma = round_up16(n_valid);
     return t;
   }
-  DG_DEVINL static uint32_t tx_bytes(const Params&, const Tile& t) { return kAStage + rows_box(t.c) * 128; }
+  DG_DEVINL static uint32_t tx_bytes(const Params&, const Tile&) { return kAStage + B_STAGE; }
   DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
     tma_load_2d(sa, &p.tmW, kb * 128, t.a * p.d + t.b * 128, bar);
-    tma_load_2d(sb, &p.tmH[t.c <= 64 ? 0 : (t.c <= 128 ? 1 : 2)], kb * 128, t.d, bar);
+    tma_load_2d(sb, &p.tmH, kb * 128, t.d, bar);
   }
   DG_DEVINL static void epilogue(const Params& p, const Tile& t, uint32_t taddr, int, int, int row, uint8_t*) {
     const int f = t.b * 128 + row;
@@ -774,152 +683,6 @@ struct P_SGU : ProblemBase {
   }
 };
 
-// Sorted insertion into a descending top-8 list.  Values arrive in ascending
-// id order, so the strict comparisons keep the lower id ahead of an equal one.
-DG_DEVINL void top8_insert(float (&tv)[8], int (&ti)[8], float v, int id) {
-  if (v > tv[7]) {
-    bool gt[8];
-#pragma unroll
-    for (int r = 0; r < 8; ++r) gt[r] = v > tv[r];
-#pragma unroll
-    for (int r = 7; r > 0; --r) {
-      tv[r] = gt[r] ? (gt[r - 1] ? tv[r - 1] : v) : tv[r];
-      ti[r] = gt[r] ? (gt[r - 1] ? ti[r - 1] : id) : ti[r];
-    }
-    tv[0] = gt[0] ? v : tv[0];
-    ti[0] = gt[0] ? id : ti[0];
-  }
-}
-
-// ---------------------------------------------------------------------------
-// Router logits r = u W_r^T with the top-k, the renormalised softmax of the
-// picked logits and the per-expert token bitmasks (the routing rule of the
-// shared-expert kernel's router tile, split so that it no longer runs as one
-// long chain).  Tokens are the 128-row operand and the E router rows the N
-// side; the 64-column k-blocks of d are split into S slices, one CTA per
-// (token tile, slice).  Every CTA writes its fp32 partial [128][E]; the last
-// CTA of a token tile to finish (an arrival counter per token tile) sums the
-// S partials in slice order -- the same order whoever arrives last, so the
-// logits are deterministic -- and runs the top-k.  The counter is put back to
-// zero by that CTA (and by the grouping kernel that follows, should a CTA have
-// given up on a bounded wait).
-// ---------------------------------------------------------------------------
-struct P_ROUTER : ProblemBase {
-  static constexpr int BN = 128, STAGES = 3, KB = 2, B_STAGE = BN * 128, TMEM_COLS = 256;
-  static constexpr int EP_SMEM = 16;
-  struct Params {
-    CUtensorMap tmX;    // normed tokens u [Tcap, d], 128-row boxes
-    CUtensorMap tmR;    // w_router [E, d], E-row boxes
-    int T, nk, MT, S, E, k, MW;
-    float* part;        // [MT][S][128][E] fp32 partial logits
-    unsigned* counter;  // [MT] arrivals of the current launch (zero between launches)
-    float* logits;      // [Tcap, E]
-    int* idx;           // [T, k]
-    float* w;           // [T, k]
-    unsigned* mask;     // [E][MW] token bitmasks (zero on entry)
-    int* err;
-  };
-  static constexpr bool PRELOAD = true;
-  DG_DEVINL static void prefetch(const Params& p) {
-    tma_prefetch_desc(&p.tmX);
-    tma_prefetch_desc(&p.tmR);
-  }
-  DG_DEVINL static int num_tiles(const Params& p) { return p.MT * p.S; }
-  DG_DEVINL static Tile tile(const Params& p, int v) {
-    Tile t;
-    t.a = v % p.MT;  // token tile
-    t.c = v / p.MT;  // K slice
-    const int per = (p.nk + p.S - 1) / p.S;
-    t.d = t.c * per;
-    t.nk = min(per, p.nk - t.d);
-    t.valid = t.nk > 0;
-    t.n_mma = p.E;
-    return t;
-  }
-  DG_DEVINL static uint32_t tx_bytes(const Params& p, const Tile&) { return kAStage + p.E * 128; }
-  DG_DEVINL static void load_w(const Params& p, const Tile& t, int kb, uint32_t, uint32_t sb, uint64_t* bar) {
-    tma_load_2d(sb, &p.tmR, (t.d + kb) * 64, 0, bar);
-  }
-  DG_DEVINL static void load_x(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t, uint64_t* bar) {
-    tma_load_2d(sa, &p.tmX, (t.d + kb) * 64, t.a * 128, bar);
-  }
-  DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
-    load_x(p, t, kb, sa, sb, bar);
-    load_w(p, t, kb, sa, sb, bar);
-  }
-  DG_DEVINL static void epilogue(const Params& p, const Tile& t, uint32_t taddr, int, int, int row, uint8_t* ep) {
-    volatile int* last = reinterpret_cast<volatile int*>(ep);
-    const int E = p.E;
-    float4* mine = reinterpret_cast<float4*>(p.part + (((size_t)t.a * p.S + t.c) * 128 + row) * E);
-    for (int c0 = 0; c0 < E; c0 += 16) {
-      float z[16];
-      tmem_ld16(taddr + c0, z);
-#pragma unroll
-      for (int i = 0; i < 16; i += 4) mine[(c0 + i) / 4] = make_float4(z[i], z[i + 1], z[i + 2], z[i + 3]);
-    }
-    __threadfence();
-    named_bar_sync(1, 128);
-    if (row == 0) *last = atomicAdd(&p.counter[t.a], 1u) == (unsigned)(p.S - 1);
-    named_bar_sync(1, 128);
-    const bool is_last = *last != 0;
-    named_bar_sync(1, 128);  // every thread has read the flag before the next tile may rewrite it
-    if (!is_last) return;
-    __threadfence();
-    const int tok = t.a * 128 + row;
-    const bool ok = tok < p.T;
-    float tv[8];
-    int ti[8];
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      tv[r] = -INFINITY;
-      ti[r] = 0x7fffffff;
-    }
-    const float* base = p.part + ((size_t)t.a * p.S * 128 + row) * E;
-    for (int c0 = 0; c0 < E; c0 += 16) {
-      float z[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) z[i] = 0.f;
-      for (int s2 = 0; s2 < p.S; ++s2) {  // slice order
-        const float4* src = reinterpret_cast<const float4*>(base + (size_t)s2 * 128 * E + c0);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float4 v = __ldcg(src + i);
-          z[4 * i] += v.x;
-          z[4 * i + 1] += v.y;
-          z[4 * i + 2] += v.z;
-          z[4 * i + 3] += v.w;
-        }
-      }
-      if (!ok) continue;
-      float4* lg = reinterpret_cast<float4*>(p.logits + (size_t)tok * E + c0);
-#pragma unroll
-      for (int i = 0; i < 16; i += 4) lg[i / 4] = make_float4(z[i], z[i + 1], z[i + 2], z[i + 3]);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) top8_insert(tv, ti, z[i], c0 + i);
-    }
-    if (row == 0) p.counter[t.a] = 0u;
-    if (!ok) return;
-    float ex[8], sum = 0.f;
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      ex[r] = r < p.k ? expf(tv[r] - tv[0]) : 0.f;
-      sum += ex[r];
-    }
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      if (r < p.k) {
-        const bool valid = (unsigned)ti[r] < (unsigned)E;  // fewer than k picks only with NaN logits
-        p.idx[(size_t)tok * p.k + r] = valid ? ti[r] : -1;
-        p.w[(size_t)tok * p.k + r] = ex[r] / sum;
-        if (valid)
-          atomicOr(&p.mask[(size_t)ti[r] * p.MW + (tok >> 5)], 1u << (tok & 31));
-        else
-          atomicOr(p.err, DG_DEVERR_NAN);
-      }
-    }
-  }
-};
-
 // ---------------------------------------------------------------------------
 // LM head with fused online statistics.  Tile (mt, vt): tokens mt*128..+127,
 // vocab rows vt*256..+255.  Each epilogue thread owns one token row and keeps,
@@ -943,6 +706,23 @@ struct LmStat {
   float m, s, t;
   int a;
 };
+
+// Sorted insertion into a descending top-8 list.  Values arrive in ascending
+// id order, so the strict comparisons keep the lower id ahead of an equal one.
+DG_DEVINL void top8_insert(float (&tv)[8], int (&ti)[8], float v, int id) {
+  if (v > tv[7]) {
+    bool gt[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) gt[r] = v > tv[r];
+#pragma unroll
+    for (int r = 7; r > 0; --r) {
+      tv[r] = gt[r] ? (gt[r - 1] ? tv[r - 1] : v) : tv[r];
+      ti[r] = gt[r] ? (gt[r - 1] ? ti[r - 1] : id) : ti[r];
+    }
+    tv[0] = gt[0] ? v : tv[0];
+    ti[0] = gt[0] ? id : ti[0];
+  }
+}
 
 struct P_LM : ProblemBase {
   static constexpr int BN = 256, STAGES = 4, B_STAGE = BN * 128, TMEM_COLS = 512;
@@ -1201,19 +981,9 @@ cudaError_t run_wpart(const WpartArgs& a, cudaStream_t st) {
 
 cudaError_t run_experts_gate_up(const ExpertArgs& a, cudaStream_t st) {
   P_EGU::Params g;
-  for (int i = 0; i < 2; ++i) {
-    g.tmG[i] = *a.tm_gate[i];
-    g.tmU[i] = *a.tm_up[i];
-    g.tmSG[i] = a.tm_sgate[i] ? *a.tm_sgate[i] : *a.tm_gate[i];  // unused without shared tiles
-    g.tmSU[i] = a.tm_sup[i] ? *a.tm_sup[i] : *a.tm_up[i];
-  }
-  g.tmXS = a.tm_u ? *a.tm_u : *a.tm_xp[0];
-  g.E = a.tm_u ? a.E : -1;
-  g.T = a.T;
-  g.fs = a.fs;
-  g.hs = a.hs;
-  g.tmX[0] = *a.tm_xp[0];
-  g.tmX[1] = *a.tm_xp[1];
+  g.tmG = *a.tm_gate;
+  g.tmU = *a.tm_up;
+  g.tmX = *a.tm_xp;
   g.nk = a.d / 64;
   g.fe = a.fe;
   g.tiles = a.egu_tiles;
@@ -1227,10 +997,9 @@ cudaError_t run_experts_gate_up(const ExpertArgs& a, cudaStream_t st) {
 
 cudaError_t run_experts_gate_up_fp8(const ExpertArgs& a, cudaStream_t st) {
   P_EGU8::Params g;
-  g.tmG = *a.tm_gate[0];
-  g.tmU = *a.tm_up[0];
-  g.tmX[0] = *a.tm_xp[0];
-  g.tmX[1] = *a.tm_xp[1];
+  g.tmG = *a.tm_gate;
+  g.tmU = *a.tm_up;
+  g.tmX = *a.tm_xp;
   g.nk = (a.d + 127) / 128;
   g.fe = a.fe;
   g.tiles = a.egu_tiles;
@@ -1248,7 +1017,7 @@ cudaError_t run_experts_gate_up_fp8(const ExpertArgs& a, cudaStream_t st) {
 cudaError_t run_experts_down_fp8(const ExpertArgs& a, cudaStream_t st) {
   P_ED8::Params dn;
   dn.tmW = *a.tm_down;
-  for (int i = 0; i < 3; ++i) dn.tmH[i] = *a.tm_hp[i];
+  dn.tmH = *a.tm_hp;
   dn.nk = (a.fe + 127) / 128;
   dn.d = a.d;
   dn.tiles = a.ed_tiles;
@@ -1266,13 +1035,7 @@ cudaError_t run_experts_down_fp8(const ExpertArgs& a, cudaStream_t st) {
 cudaError_t run_experts_down(const ExpertArgs& a, cudaStream_t st) {
   P_ED::Params dn;
   dn.tmW = *a.tm_down;
-  dn.tmSW = a.tm_sdown ? *a.tm_sdown : *a.tm_down;  // unused without shared tiles
-  dn.tmHS = a.tm_hs ? *a.tm_hs : *a.tm_hp[0];
-  dn.E = a.tm_sdown ? a.E : -1;
-  dn.T = a.T;
-  dn.nks = a.fs / 64;
-  dn.ys = a.ys;
-  for (int i = 0; i < 3; ++i) dn.tmH[i] = *a.tm_hp[i];
+  dn.tmH = *a.tm_hp;
   dn.nk = a.fe / 64;
   dn.d = a.d;
   dn.tiles = a.ed_tiles;
@@ -1311,31 +1074,6 @@ cudaError_t run_shared_gate_up(const SharedArgs& a, cudaStream_t st) {
   return launch_gemm<P_SGU>(g, grid_for(g.MT * (g.FJ + (a.E > 0 ? 1 : 0)), a.num_sms), st);
 }
 
-cudaError_t run_router(const RouterArgs& a, cudaStream_t st) {
-  if (a.E < 16 || a.E > P_ROUTER::BN || a.E % 16 != 0 || a.k < 1 || a.k > 8 || a.splits < 1) return cudaErrorInvalidValue;
-  P_ROUTER::Params p;
-  p.tmX = *a.tm_u;
-  p.tmR = *a.tm_router;
-  p.T = a.T;
-  p.nk = a.d / 64;
-  p.MT = (a.T + 127) / 128;
-  p.S = a.splits;
-  p.E = a.E;
-  p.k = a.k;
-  p.MW = a.MW;
-  p.part = a.part;
-  p.counter = a.counter;
-  p.logits = a.logits;
-  p.idx = a.idx;
-  p.w = a.w;
-  p.mask = a.mask;
-  p.err = a.err;
-  // every slice must own at least one k-block (the last arriver waits for all S)
-  const int per = (p.nk + p.S - 1) / p.S;
-  if ((p.S - 1) * per >= p.nk) return cudaErrorInvalidValue;
-  return launch_gemm<P_ROUTER>(p, p.MT * p.S, st);
-}
-
 cudaError_t run_lm_head(const LmArgs& a, int* grid_out, cudaStream_t st) {
   P_LM::Params p;
   p.tmX = *a.tm_x;
@@ -1364,13 +1102,6 @@ cudaError_t run_lm_head(const LmArgs& a, int* grid_out, cudaStream_t st) {
   return launch_gemm<P_LM>(p, grid, st);
 }
 
-static_assert(GemmSmem<P_QKV>::total <= 227 * 1024 && GemmSmem<P_WPART>::total <= 227 * 1024 &&
-                  GemmSmem<P_EGU>::total <= 227 * 1024 && GemmSmem<P_ED>::total <= 227 * 1024 &&
-                  GemmSmem<P_SGU>::total <= 227 * 1024 && GemmSmem<P_LM>::total <= 227 * 1024 &&
-                  GemmSmem<P_EGU8>::total <= 227 * 1024 && GemmSmem<P_ED8>::total <= 227 * 1024 &&
-                  GemmSmem<P_ROUTER>::total <= 227 * 1024,
-              "a GEMM problem's shared memory exceeds the per-CTA limit");
-
 size_t gemm_smem_bytes_max() {
   size_t m = GemmSmem<P_QKV>::total;
   m = m > GemmSmem<P_WPART>::total ? m : GemmSmem<P_WPART>::total;
@@ -1380,7 +1111,6 @@ size_t gemm_smem_bytes_max() {
   m = m > GemmSmem<P_LM>::total ? m : GemmSmem<P_LM>::total;
   m = m > GemmSmem<P_EGU8>::total ? m : GemmSmem<P_EGU8>::total;
   m = m > GemmSmem<P_ED8>::total ? m : GemmSmem<P_ED8>::total;
-  m = m > GemmSmem<P_ROUTER>::total ? m : GemmSmem<P_ROUTER>::total;
   return m;
 }
 

@@ -462,8 +462,7 @@ __global__ void __launch_bounds__(256) k_group_gather(GroupArgs a, const unsigne
   pdl_wait();
   __shared__ int cnt[256];
   __shared__ int off[257];
-  __shared__ int toff[257];   // gate|up token tiles before expert e
-  __shared__ int doff[257];   // down token tiles before expert e
+  __shared__ int toff[257];
   const int E = a.E, T = a.T, k = a.k, P = T * k;
   const int used = (T + 31) >> 5;  // words of each expert's mask this pass can have set
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -474,32 +473,28 @@ __global__ void __launch_bounds__(256) k_group_gather(GroupArgs a, const unsigne
   }
   __syncthreads();
   if (warp == 0) {
-    int v[8], tv[8], dv[8];
+    int v[8], tv[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int e = lane * 8 + i;
       v[i] = e < E ? cnt[e] : 0;
-      tv[i] = e < E ? (cnt[e] + kEguRows - 1) / kEguRows : 0;
-      dv[i] = e < E ? (cnt[e] + kEdRows - 1) / kEdRows : 0;
+      tv[i] = e < E ? (cnt[e] + kExpertRows - 1) / kExpertRows : 0;
     }
     const int tot = warp_excl_scan8(v, lane);
     const int ttot = warp_excl_scan8(tv, lane);
-    const int dtot = warp_excl_scan8(dv, lane);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int e = lane * 8 + i;
       if (e < E) {
         off[e] = v[i];
         toff[e] = tv[i];
-        doff[e] = dv[i];
       }
     }
     if (lane == 0) {
       off[E] = tot;
       toff[E] = ttot;
-      doff[E] = dtot;
       if (blockIdx.x == 0) {
-        const int egu = a.sh_fj * a.sh_ntg + ttot * a.FJ, ed = a.sh_md * a.sh_ntd + dtot * a.MD;
+        const int egu = ttot * a.FJ, ed = ttot * a.MD;
         if (egu > a.egu_cap || ed > a.ed_cap || tot != P) atomicOr(a.err, DG_DEVERR_CAPACITY);
         *a.egu_count = min(egu, a.egu_cap);
         *a.ed_count = min(ed, a.ed_cap);
@@ -520,25 +515,17 @@ __global__ void __launch_bounds__(256) k_group_gather(GroupArgs a, const unsigne
       if (lane == 0) atomicAdd(&a.route_stats[0], (unsigned long long)touched);
       if (tid == 0) atomicAdd(&a.route_stats[1], 1ull);
     }
-    // the shared expert's tiles first (expert id E; all tokens of the pass):
-    // the down tiles have the longest K chain, so they start on the first CTAs
-    const int shg = a.sh_fj * a.sh_ntg, shd = a.sh_md * a.sh_ntd;
-    for (int i = tid; i < shg; i += blockDim.x)
-      if (i < a.egu_cap) a.egu_tiles[i] = make_int4(E, i % a.sh_fj, i / a.sh_fj, 0);
-    for (int i = tid; i < shd; i += blockDim.x)
-      if (i < a.ed_cap) a.ed_tiles[i] = make_int4(E, i % a.sh_md, i / a.sh_md, 0);
-    for (int i = tid; i < a.router_mt; i += blockDim.x) a.router_counter[i] = 0u;
     for (int e = warp; e < E; e += blockDim.x >> 5) {
-      const int n_g = toff[e + 1] - toff[e], n_d = doff[e + 1] - doff[e];
-      for (int i = lane; i < n_g * a.FJ; i += 32) {
-        const int nt = i / a.FJ, r = i % a.FJ;
-        const int slot = shg + (toff[e] + nt) * a.FJ + r;
-        if (slot < a.egu_cap) a.egu_tiles[slot] = make_int4(e, r, nt, 0);
-      }
-      for (int i = lane; i < n_d * a.MD; i += 32) {
-        const int nt = i / a.MD, r = i % a.MD;
-        const int slot = shd + (doff[e] + nt) * a.MD + r;
-        if (slot < a.ed_cap) a.ed_tiles[slot] = make_int4(e, r, nt, 0);
+      const int n_nt = toff[e + 1] - toff[e];
+      for (int i = lane; i < n_nt * (a.FJ + a.MD); i += 32) {
+        const int nt = i / (a.FJ + a.MD), r = i % (a.FJ + a.MD);
+        if (r < a.FJ) {
+          const int slot = (toff[e] + nt) * a.FJ + r;
+          if (slot < a.egu_cap) a.egu_tiles[slot] = make_int4(e, r, nt, 0);
+        } else {
+          const int slot = (toff[e] + nt) * a.MD + (r - a.FJ);
+          if (slot < a.ed_cap) a.ed_tiles[slot] = make_int4(e, r - a.FJ, nt, 0);
+        }
       }
     }
   }
@@ -571,26 +558,25 @@ __global__ void __launch_bounds__(256) k_group_gather(GroupArgs a, const unsigne
       quant_row_warp(u + (size_t)t * d, d, xq + (size_t)row * d, xs + row, lane);
       continue;
     }
-    // the row copy: every 16-byte chunk of the row in flight at once (d <= 4096:
-    // at most 16 chunks per lane), then the stores
     const uint4* src = reinterpret_cast<const uint4*>(u + (size_t)t * d);
     uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)row * d);
     const int n16 = d / 8;
-    constexpr int kChunks = 16;
-    uint4 r[kChunks];
+    for (int c0 = lane; c0 < n16; c0 += 32 * 4) {
+      uint4 r[4];
 #pragma unroll
-    for (int b = 0; b < kChunks; ++b)
-      if (lane + b * 32 < n16) r[b] = src[lane + b * 32];
+      for (int b = 0; b < 4; ++b)
+        if (c0 + b * 32 < n16) r[b] = src[c0 + b * 32];
 #pragma unroll
-    for (int b = 0; b < kChunks; ++b)
-      if (lane + b * 32 < n16) dst[lane + b * 32] = r[b];
+      for (int b = 0; b < 4; ++b)
+        if (c0 + b * 32 < n16) dst[c0 + b * 32] = r[b];
+    }
   }
 }
 
 cudaError_t run_route(const bf16* u, int d, bf16* xp, unsigned* mask, unsigned* mask_next, int MW,
                       const GroupArgs& a, cudaStream_t st, uint8_t* xq, float* xs) {
   if (a.T < 1 || a.T > DG_MAX_REQUESTS * 256 || a.E > 256 || MW * 32 < a.T) return cudaErrorInvalidValue;
-  if (d % 8 != 0 || d > 4096 || (xq != nullptr && xs == nullptr)) return cudaErrorInvalidValue;
+  if (xq != nullptr && (d % 8 != 0 || d > 4096 || xs == nullptr)) return cudaErrorInvalidValue;
   const int P = a.T * a.k;
   const int grid = (P + 7) / 8 < 148 ? (P + 7) / 8 : 148;
   {

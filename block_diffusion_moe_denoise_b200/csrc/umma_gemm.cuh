@@ -17,10 +17,6 @@
 // of one tile overlaps the main loop of the next.  Tiles are assigned
 // statically (tile v to CTA v mod gridDim.x), so every role walks the same list.
 //
-// A problem may keep NACC accumulators per tile (default 1): each k-block then
-// holds NACC A tiles (rows of NACC weight matrices) against one B tile, and
-// accumulator i of a tile lives in TMEM columns [i*BN, (i+1)*BN) of the tile's
-// buffer (the double buffer advances by NACC*BN columns).
 // A problem class P supplies: BN, STAGES, KB, B_STAGE (bytes per k-block), EP_SMEM (bytes),
 // TMEM_COLS, Params, num_tiles(), tile(), tx_bytes(), load(), epilogue(),
 // finish(), epilogue_prefetch() (called before the accumulator wait, so an
@@ -45,8 +41,7 @@ constexpr int kAStage = 128 * 128;  // 128 rows x 128 bytes
 template <class P>
 struct GemmSmem {
   static constexpr int kStages = P::STAGES;
-  static constexpr size_t a_kb = (size_t)P::NACC * kAStage;  // A bytes per k-block
-  static constexpr size_t a_stage = (size_t)P::KB * a_kb;
+  static constexpr size_t a_stage = (size_t)P::KB * kAStage;
   static constexpr size_t b_stage = (size_t)P::KB * P::B_STAGE;
   static constexpr size_t a_off = 0;
   static constexpr size_t b_off = a_off + (size_t)kStages * a_stage;
@@ -114,7 +109,7 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
               const int nsub = t0.nk - kb < P::KB ? t0.nk - kb : P::KB;
               mbar_arrive_expect_tx(&full[st], P::tx_bytes(p, t0) * (uint32_t)nsub);
               for (int j = 0; j < nsub; ++j)
-                P::load_w(p, t0, kb + j, smem_u32(sA + st * S::a_stage + (size_t)j * S::a_kb),
+                P::load_w(p, t0, kb + j, smem_u32(sA + st * S::a_stage + (size_t)j * kAStage),
                           smem_u32(sB + st * S::b_stage + (size_t)j * P::B_STAGE), &full[st]);
             }
           }
@@ -135,13 +130,13 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
           if (pre > 0) {  // slot already armed and holding its weight tiles
             --pre;
             for (int j = 0; j < nsub; ++j)
-              P::load_x(p, t, kb + j, smem_u32(sa + (size_t)j * S::a_kb), smem_u32(sb + (size_t)j * P::B_STAGE),
+              P::load_x(p, t, kb + j, smem_u32(sa + (size_t)j * kAStage), smem_u32(sb + (size_t)j * P::B_STAGE),
                         &full[stage]);
           } else {
             if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, err)) { ok = false; break; }
             mbar_arrive_expect_tx(&full[stage], tx * (uint32_t)nsub);
             for (int j = 0; j < nsub; ++j)
-              P::load(p, t, kb + j, smem_u32(sa + (size_t)j * S::a_kb), smem_u32(sb + (size_t)j * P::B_STAGE),
+              P::load(p, t, kb + j, smem_u32(sa + (size_t)j * kAStage), smem_u32(sb + (size_t)j * P::B_STAGE),
                       &full[stage]);
           }
           if (++stage == P::STAGES) { stage = 0; phase ^= 1; }
@@ -161,7 +156,7 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
         if (!t.valid) continue;
         if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1, abort_flag, err)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem + acc * (P::NACC * P::BN);
+        const uint32_t d_tmem = tmem + acc * P::BN;
         const uint32_t idesc =
             P::F8 ? umma_idesc_e4m3(128, (uint32_t)t.n_mma) : umma_idesc_bf16(128, (uint32_t)t.n_mma);
         bool ok = true;
@@ -176,16 +171,12 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
             if (j < nsub) {
 #pragma unroll
               for (int k = 0; k < 4; ++k) {
+                const uint64_t ad = umma_sdesc_k128(a0 + j * kAStage + 32 * k);
                 const uint64_t bd = umma_sdesc_k128(b0 + j * P::B_STAGE + 32 * k);
-#pragma unroll
-                for (int ai = 0; ai < P::NACC; ++ai) {
-                  const uint64_t ad = umma_sdesc_k128(a0 + (uint32_t)(j * S::a_kb + ai * kAStage) + 32 * k);
-                  const uint32_t dt = d_tmem + (uint32_t)(ai * P::BN);
-                  if constexpr (P::F8)
-                    umma_e4m3(dt, ad, bd, idesc, (kb | j | k) != 0 ? 1u : 0u);
-                  else
-                    umma_bf16(dt, ad, bd, idesc, (kb | j | k) != 0 ? 1u : 0u);
-                }
+                if constexpr (P::F8)
+                  umma_e4m3(d_tmem, ad, bd, idesc, (kb | j | k) != 0 ? 1u : 0u);
+                else
+                  umma_bf16(d_tmem, ad, bd, idesc, (kb | j | k) != 0 ? 1u : 0u);
               }
             }
           }
@@ -211,7 +202,7 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
       P::epilogue_prefetch(p, t, row);
       if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, err)) break;
       tc_fence_after();
-      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + acc * (P::NACC * P::BN);
+      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + acc * P::BN;
       P::epilogue(p, t, taddr, q, lane, row, ep_smem);
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
@@ -234,7 +225,6 @@ struct ProblemBase {
   static constexpr bool PRELOAD = false;  // true: static tiles, load_w / load_x split of load
   static constexpr int KB = 1;            // k-blocks per ring stage
   static constexpr bool F8 = false;       // E4M3 operands (kind::f8f6f4): a k-block is 128 elements
-  static constexpr int NACC = 1;          // accumulators (A tiles) per tile
   template <class Params>
   DG_DEVINL static void epilogue_init(const Params&, int, uint8_t*) {}
   template <class Params>
