@@ -152,9 +152,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
         mbar_arrive_expect_tx(&k_full[st], S::kK);
         const uint32_t k_dst = smem_u32(sK + (size_t)st * S::kK);
         const int key0 = k_begin + j * kAK;
-#pragma unroll
-        for (int kb = 0; kb < D / 64; ++kb)
-          tma_load_2d(k_dst + kb * (kAK * 128), &a.tm_k, kb * 64, (int)(krow0 + key0), &k_full[st]);
+        // the tiled K cache holds the 64 keys x D dims of a tile as D
+        // consecutive 128-byte rows: one box, [D/64][64 keys][128 B] in smem
+        tma_load_2d(k_dst, &a.tm_k, 0, (int)((krow0 + key0) * (D / 64)), &k_full[st]);
         return true;
       };
       auto load_v = [&](int j) -> bool {

@@ -269,6 +269,19 @@ DG_DEVINL void named_bar_sync(int id, int nthreads) {
 }
 
 // ---------------------------------------------------------------------------
+// K cache layout.  Per (request, layer, KV head) the keys are stored in tiles
+// of 64 positions, and inside a tile by 64-dimension block:
+//   [cap / 64][D / 64][64 positions][64 dims]
+// so one 64-position K tile of every dimension is a single contiguous run of
+// D rows of 128 bytes -- one TMA box instead of D / 64 of them -- that lands
+// in shared memory as the [D / 64][64][128 B] operand the S MMAs read.
+// Element offset of (position, dim) from the head's base; cap % 64 == 0.
+// ---------------------------------------------------------------------------
+DG_DEVINL size_t k_tile_offset(long long pos, int dim, int D) {
+  return (size_t)(pos >> 6) * 64 * D + (size_t)(dim >> 6) * 4096 + (size_t)(pos & 63) * 64 + (dim & 63);
+}
+
+// ---------------------------------------------------------------------------
 // misc
 // ---------------------------------------------------------------------------
 DG_DEVINL float warp_sum(float v) {

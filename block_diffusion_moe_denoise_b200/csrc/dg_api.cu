@@ -140,6 +140,7 @@ void make_plan(const dg_config* c, int max_req, long long cap_user, Plan* p) {
   p->add("router_logits", (size_t)Tcap * c->n_experts * 4);
   p->add("part", (size_t)kMaxPartSplits * Tcap * d * 4);
   p->add("route_mask", (size_t)2 * c->n_experts * ((T + 31) / 32) * 4);
+  p->add("sched", 64);
   p->add("prompt", (size_t)cap_user * 4);
 }
 
@@ -499,6 +500,7 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     ga.ed_count = h->B<int>("tile_counts") + 1;
     ga.route_stats = h->B<unsigned long long>("route_stats");
     ga.err = err;
+    ga.sched = h->B<int>("sched");
     const bool f8 = c.expert_fp8 != 0;
     LAUNCH(h, K_GROUP, 1,
            run_route(h->B<bf16>("u"), d, h->B<bf16>("xp"), mask_cur, mask_nxt, MW, ga, st,
@@ -523,6 +525,7 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     ea.hp = h->B<bf16>("hp");
     ea.yp = yp;
     ea.err = err;
+    ea.sched = h->B<int>("sched");
     if (f8) {
       // E4M3 weight codes and token rows; the SwiGLU rows are quantised per row before down
       ea.tm_xp = &h->tm_xq;
@@ -736,7 +739,9 @@ int dg_init(const dg_config* cfg, const dg_weights* wts, int max_requests, int64
   ok = ok && make_map(&h->tm_embed, h->embed, d, c.vocab, 256);
   {
     const long long kv_elems = (long long)max_requests * h->kv_req_stride;
-    ok = ok && make_map(&h->tm_k, h->B<bf16>("kv"), D, kv_elems / D, 64);
+    // K in the tiled layout: rows of 64 dims, a tile of 64 keys = D rows
+    ok = ok && kv_elems / 64 < (1ll << 31);
+    ok = ok && make_map(&h->tm_k, h->B<bf16>("kv"), 64, kv_elems / 64, D);
     ok = ok && make_map(&h->tm_vt, h->B<bf16>("kv"), h->cap, kv_elems / h->cap, D);
   }
   if (c.expert_fp8) {
@@ -763,6 +768,7 @@ int dg_init(const dg_config* cfg, const dg_weights* wts, int max_requests, int64
       cudaMemsetAsync(h->B<int>("err"), 0, 64, h->st) != cudaSuccess ||
       cudaMemsetAsync(h->B<int>("route_stats"), 0, 64, h->st) != cudaSuccess ||
       cudaMemsetAsync(h->B<int>("route_mask"), 0, h->plan.buf.at("route_mask").second, h->st) != cudaSuccess ||
+      cudaMemsetAsync(h->B<int>("sched"), 0, 64, h->st) != cudaSuccess ||
       cudaMemsetAsync(h->B<bf16>("kv"), 0, h->plan.buf.at("kv").second, h->st) != cudaSuccess ||
       cudaMemsetAsync(h->B<int>("remaining"), 0, (size_t)max_requests * 4, h->st) != cudaSuccess ||
       cudaStreamSynchronize(h->st) != cudaSuccess) {

@@ -69,6 +69,7 @@ struct ExpertArgs {
   int* err;
   // FP8 experts: per-row scales of the weight codes and of the token / hidden codes
   const float *s_gate = nullptr, *s_up = nullptr, *s_down = nullptr, *s_x = nullptr, *s_h = nullptr;
+  int* sched = nullptr;  // [2] tile counters of the gate|up and down launches (zeroed by the grouping kernel)
 };
 struct SharedArgs {
   const CUtensorMap *tm_u, *tm_gate, *tm_up, *tm_router;
@@ -156,6 +157,7 @@ struct GroupArgs {
   int* ed_count;
   unsigned long long* route_stats;  // [0] += experts touched, [1] += launches (may be null)
   int* err;
+  int* sched = nullptr;             // [2] tile counters of the expert GEMMs that follow, zeroed here
 };
 cudaError_t run_group(const GroupArgs& a, cudaStream_t st);
 // the grouping above from the token bitmasks `mask` ([E][MW] words, MW fixed by
@@ -219,7 +221,7 @@ cudaError_t run_kv_copy(bf16* cache_k, bf16* cache_v, int Hkv, long long cap, in
 
 // ---- attention (attention.cu) ----
 struct AttnArgs {
-  CUtensorMap tm_k;   // whole KV area as rows of D elements, 64 x 64 boxes
+  CUtensorMap tm_k;   // whole KV area as rows of 64 elements, boxes of D rows (one tiled 64-key K tile)
   CUtensorMap tm_vt;  // whole KV area as rows of cap elements, 64 x D boxes
   const bf16* q;      // [Hq][q_T][D]
   int q_T;

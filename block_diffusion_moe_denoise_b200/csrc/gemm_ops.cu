@@ -140,7 +140,9 @@ struct P_QKV : ProblemBase {
     const int D = p.D, half = D >> 1;
     int kind, tb, r0, r1;
     rows_of(p, t.b, kind, tb, r0, r1);
-    __nv_bfloat16* kbase = p.kv + (size_t)req * p.kv_req_stride + (size_t)pos * D;
+    // K: tiled cache layout (k_tile_offset); kpos = this position's row inside
+    // its 64-position tile, block j of the dimensions 4096 elements further
+    __nv_bfloat16* kbase = p.kv + (size_t)req * p.kv_req_stride + k_tile_offset(pos, 0, D);
     const size_t head_stride = (size_t)p.kv_cap * D;
     if (kind == 2) {
       // V is cached transposed, [Hkv][D][cap]: consecutive tokens of a warp
@@ -161,6 +163,7 @@ struct P_QKV : ProblemBase {
     if (D == 64) {
       for (int hh = 0; hh < 2; ++hh) {
         const int head = tb * 2 + hh;
+        // one 64-dim block: the tiled K row is contiguous like the q row
         __nv_bfloat16* dst = kind == 0 ? p.q + ((size_t)head * p.q_T + tok) * D : kbase + (size_t)head * head_stride;
         for (int c = 0; c < 32; c += 16) {
           float x1[16], x2[16], y1[16], y2[16];
@@ -180,7 +183,11 @@ struct P_QKV : ProblemBase {
     }
     const int j = D == 256 ? (tb & 1) : 0;
     const int head = D == 256 ? (tb >> 1) : tb;
+    // dims j*64.. and half + j*64..: q rows are plain; K rows are 64-dim blocks
+    // 4096 elements apart (tiled layout)
     __nv_bfloat16* dst = kind == 0 ? p.q + ((size_t)head * p.q_T + tok) * D : kbase + (size_t)head * head_stride;
+    const size_t o1 = kind == 0 ? (size_t)j * 64 : (size_t)j * 4096;
+    const size_t o2 = kind == 0 ? (size_t)(half + j * 64) : (size_t)((half >> 6) + j) * 4096;
     for (int c = 0; c < 64; c += 16) {
       float x1[16], x2[16], y1[16], y2[16];
       tmem_ld16(taddr + c, x1);
@@ -190,8 +197,8 @@ struct P_QKV : ProblemBase {
 #pragma unroll
         for (int i = 0; i < 16; ++i) cs[i] = cs_row[j * 64 + c + i];
         rotate16(x1, x2, cs, y1, y2);
-        store_bf16x16(dst + j * 64 + c, y1);
-        store_bf16x16(dst + half + j * 64 + c, y2);
+        store_bf16x16(dst + o1 + c, y1);
+        store_bf16x16(dst + o2 + c, y2);
       }
     }
   }
@@ -267,7 +274,9 @@ struct P_WPART : ProblemBase {
 // ---------------------------------------------------------------------------
 struct P_EGU : ProblemBase {
   static constexpr int BN = kExpertRows, STAGES = 4, KB = 2, B_STAGE = BN * 128, TMEM_COLS = 128;
-  static constexpr int EP_SMEM = 64 * 17 * 4;
+  static constexpr int kXchBytes = 64 * 17 * 4;
+  static constexpr int EP_SMEM = kXchBytes + BN * 64 * 2;
+  static constexpr bool DYNAMIC = true;
   struct Params {
     CUtensorMap tmG;  // w_gate as [E*fe, d]
     CUtensorMap tmU;  // w_up   as [E*fe, d]
@@ -278,6 +287,7 @@ struct P_EGU : ProblemBase {
     const int* counts;
     const int* offsets;
     __nv_bfloat16* hp;  // [rows_cap, fe]
+    int* sched;  // tile counter (zeroed by the grouping kernel)
     int* err;
   };
   DG_DEVINL static void prefetch(const Params& p) {
@@ -307,8 +317,13 @@ struct P_EGU : ProblemBase {
     tma_load_2d(sa + 64 * 128, &p.tmU, kb * 64, r, bar);
     tma_load_2d(sb, &p.tmX, kb * 64, t.d, bar);
   }
-  DG_DEVINL static void epilogue(const Params& p, const Tile& t, uint32_t taddr, int, int, int row, uint8_t* ep) {
+  // The SwiGLU rows are transposed through shared memory: the 64 gate-row
+  // threads each hold one hidden unit of 16 tokens per chunk; staged as
+  // [token][64 units] they leave as full 128-byte row segments of hp (one
+  // coalesced store per warp and token) instead of 2-byte stores per thread.
+  DG_DEVINL static void epilogue(const Params& p, const Tile& t, uint32_t taddr, int, int lane, int row, uint8_t* ep) {
     float* xch = reinterpret_cast<float*>(ep);
+    __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(ep + kXchBytes);  // [BN tokens][64 units]
     for (int c0 = 0; c0 < t.n_mma; c0 += 16) {
       float v[16];
       tmem_ld16(taddr + c0, v);
@@ -319,16 +334,18 @@ struct P_EGU : ProblemBase {
       named_bar_sync(1, 128);
       if (row < 64) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int c = c0 + i;
-          if (c < t.c) {
-            const float h = silu_f(v[i]) * xch[row * 17 + i];
-            p.hp[(size_t)(t.d + c) * p.fe + t.b * 64 + row] = f2bf(h);
-          }
-        }
+        for (int i = 0; i < 16; ++i) stage[(c0 + i) * 64 + row] = f2bf(silu_f(v[i]) * xch[row * 17 + i]);
       }
       named_bar_sync(1, 128);
     }
+    // row segments: token c, units 2*lane, 2*lane+1 (one warp per token)
+    const int w = row >> 5;
+    const uint32_t* st32 = reinterpret_cast<const uint32_t*>(stage);
+    for (int c = w; c < t.c; c += 4) {
+      uint32_t* dst = reinterpret_cast<uint32_t*>(p.hp + (size_t)(t.d + c) * p.fe + t.b * 64);
+      dst[lane] = st32[c * 32 + lane];
+    }
+    named_bar_sync(1, 128);  // the staging tile is free for the next tile
   }
 };
 
@@ -338,6 +355,7 @@ struct P_EGU : ProblemBase {
 // ---------------------------------------------------------------------------
 struct P_ED : ProblemBase {
   static constexpr int BN = kExpertRows, STAGES = 4, KB = 2, B_STAGE = BN * 128, TMEM_COLS = 128;
+  static constexpr bool DYNAMIC = true;
   struct Params {
     CUtensorMap tmW;  // w_down as [E*d, fe]
     CUtensorMap tmH;  // hidden [rows_cap, fe], 64-row boxes
@@ -348,6 +366,7 @@ struct P_ED : ProblemBase {
     const int* offsets;
     const float* row_weight;
     float* yp;  // [rows_cap, d]
+    int* sched;  // tile counter (zeroed by the grouping kernel)
     int* err;
   };
   DG_DEVINL static void prefetch(const Params& p) {
@@ -402,6 +421,7 @@ struct P_EGU8 : ProblemBase {
   static constexpr bool F8 = true;
   static constexpr int BN = kExpertRows, STAGES = 4, KB = 2, B_STAGE = BN * 128, TMEM_COLS = 128;
   static constexpr int EP_SMEM = 64 * 17 * 4;
+  static constexpr bool DYNAMIC = true;
   struct Params {
     CUtensorMap tmG;  // w_gate codes as [E*fe, d] bytes
     CUtensorMap tmU;  // w_up codes as [E*fe, d] bytes
@@ -415,6 +435,7 @@ struct P_EGU8 : ProblemBase {
     const float* su;    // [E*fe] up row scales
     const float* sx;    // [rows] token row scales
     __nv_bfloat16* hp;  // [rows_cap, fe]
+    int* sched;  // tile counter (zeroed by the grouping kernel)
     int* err;
   };
   DG_DEVINL static void prefetch(const Params& p) {
@@ -476,6 +497,7 @@ struct P_EGU8 : ProblemBase {
 struct P_ED8 : ProblemBase {
   static constexpr bool F8 = true;
   static constexpr int BN = kExpertRows, STAGES = 4, KB = 2, B_STAGE = BN * 128, TMEM_COLS = 128;
+  static constexpr bool DYNAMIC = true;
   struct Params {
     CUtensorMap tmW;  // w_down codes as [E*d, fe] bytes
     CUtensorMap tmH;  // hidden codes [rows_cap, fe] bytes, 64-row boxes
@@ -488,6 +510,7 @@ struct P_ED8 : ProblemBase {
     const float* sh;   // [rows] hidden row scales
     const float* row_weight;
     float* yp;  // [rows_cap, d]
+    int* sched;  // tile counter (zeroed by the grouping kernel)
     int* err;
   };
   DG_DEVINL static void prefetch(const Params& p) {
@@ -992,6 +1015,7 @@ cudaError_t run_experts_gate_up(const ExpertArgs& a, cudaStream_t st) {
   g.offsets = a.offsets;
   g.hp = a.hp;
   g.err = a.err;
+  g.sched = a.sched;
   return launch_gemm<P_EGU>(g, a.num_sms, st);
 }
 
@@ -1011,6 +1035,7 @@ cudaError_t run_experts_gate_up_fp8(const ExpertArgs& a, cudaStream_t st) {
   g.sx = a.s_x;
   g.hp = a.hp;
   g.err = a.err;
+  g.sched = a.sched;
   return launch_gemm<P_EGU8>(g, a.num_sms, st);
 }
 
@@ -1029,6 +1054,7 @@ cudaError_t run_experts_down_fp8(const ExpertArgs& a, cudaStream_t st) {
   dn.row_weight = a.row_weight;
   dn.yp = a.yp;
   dn.err = a.err;
+  dn.sched = a.sched + 1;
   return launch_gemm<P_ED8>(dn, a.num_sms, st);
 }
 
@@ -1045,6 +1071,7 @@ cudaError_t run_experts_down(const ExpertArgs& a, cudaStream_t st) {
   dn.row_weight = a.row_weight;
   dn.yp = a.yp;
   dn.err = a.err;
+  dn.sched = a.sched + 1;
   return launch_gemm<P_ED>(dn, a.num_sms, st);
 }
 

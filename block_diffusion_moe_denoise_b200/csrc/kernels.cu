@@ -529,6 +529,8 @@ __global__ void __launch_bounds__(256) k_group_gather(GroupArgs a, const unsigne
       }
     }
   }
+  // the expert GEMMs that follow draw their tiles from these counters
+  if (blockIdx.x == 0 && tid < 2 && a.sched != nullptr) a.sched[tid] = 0;
   // clear the other mask buffer, sliced across CTAs
   for (int i = blockIdx.x * blockDim.x + tid; i < E * MW; i += gridDim.x * blockDim.x) mask_next[i] = 0u;
   // this CTA's pairs, one warp per pair
@@ -1005,8 +1007,8 @@ cudaError_t run_sample(const SampleArgs& a, cudaStream_t st) {
 }
 
 // ---------------------------------------------------------------------------
-// KV copy between the cache layout (K [Hkv][cap][D], V^T [Hkv][D][cap]) and
-// dense [Hkv][n][D] arrays, either direction.
+// KV copy between the cache layout (K tiled as in k_tile_offset per head,
+// V^T [Hkv][D][cap]) and dense [Hkv][n][D] arrays, either direction.
 // ---------------------------------------------------------------------------
 __global__ void k_k_copy(bf16* cache_k, int Hkv, long long cap, int D, long long pos0, long long n, const bf16* k_in,
                          bf16* k_out) {
@@ -1015,13 +1017,14 @@ __global__ void k_k_copy(bf16* cache_k, int Hkv, long long cap, int D, long long
   const long long r = blockIdx.x;  // (head, i)
   const int head = (int)(r / n);
   const long long i = r - (long long)head * n;
-  const size_t cache_off = ((size_t)head * cap + pos0 + i) * D;
+  const size_t head_off = (size_t)head * cap * D;
   const size_t dense_off = ((size_t)head * n + i) * D;
-  for (int c = threadIdx.x; c < D / 8; c += blockDim.x) {
+  for (int c = threadIdx.x; c < D / 8; c += blockDim.x) {  // 8 dims, inside one 64-dim block
+    const size_t cache_off = head_off + k_tile_offset(pos0 + i, c * 8, D);
     if (k_in)
-      reinterpret_cast<uint4*>(cache_k + cache_off)[c] = reinterpret_cast<const uint4*>(k_in + dense_off)[c];
+      *reinterpret_cast<uint4*>(cache_k + cache_off) = reinterpret_cast<const uint4*>(k_in + dense_off)[c];
     else
-      reinterpret_cast<uint4*>(k_out + dense_off)[c] = reinterpret_cast<const uint4*>(cache_k + cache_off)[c];
+      reinterpret_cast<uint4*>(k_out + dense_off)[c] = *reinterpret_cast<const uint4*>(cache_k + cache_off);
   }
 }
 

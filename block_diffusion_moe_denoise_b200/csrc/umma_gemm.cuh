@@ -23,6 +23,14 @@
 // epilogue can pull its inputs into L1 while the main loop runs), and, with
 // PRELOAD, load_w()/load_x(): the weight and activation halves of load().
 // Every wait is bounded (see mbar_wait_bounded).
+//
+// Tile scheduling.  By default tile v goes to CTA v mod gridDim.x.  A problem
+// with DYNAMIC = true instead hands out tiles from a global counter (p.sched,
+// zero at launch): the producer thread takes the next index with an atomic
+// add and publishes it through a small shared-memory ring that the MMA thread
+// and the epilogue threads read in the same order, so a CTA that drew cheap
+// tiles simply takes more of them (the expert GEMMs, whose tiles differ in
+// cost and do not divide evenly over the SMs).
 #pragma once
 
 #include "common.cuh"
@@ -37,6 +45,7 @@ struct Tile {
 };
 
 constexpr int kAStage = 128 * 128;  // 128 rows x 128 bytes
+constexpr int kSchedRing = 8;       // tile indices in flight between the roles (DYNAMIC)
 
 template <class P>
 struct GemmSmem {
@@ -47,12 +56,13 @@ struct GemmSmem {
   static constexpr size_t b_off = a_off + (size_t)kStages * a_stage;
   static constexpr size_t ep_off = b_off + (size_t)kStages * b_stage;
   static constexpr size_t bar_off = (ep_off + P::EP_SMEM + 15) & ~(size_t)15;
-  static constexpr size_t misc_off = bar_off + (2 * kStages + 4) * 8;
-  static constexpr size_t total = misc_off + 16 + 1024;  // + alignment slack
+  static constexpr size_t misc_off = bar_off + (2 * kStages + 4 + 2 * kSchedRing) * 8;
+  static constexpr size_t total = misc_off + 16 + 4 * kSchedRing + 1024;  // + alignment slack
 };
 
 template <class P>
 __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ typename P::Params p) {
+  static_assert(!(P::PRELOAD && P::DYNAMIC), "a preloaded first tile needs the static schedule");
   using S = GemmSmem<P>;
   extern __shared__ uint8_t dyn_smem[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~(uintptr_t)1023);
@@ -63,8 +73,11 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
   uint64_t* empty = full + P::STAGES;
   uint64_t* tfull = empty + P::STAGES;
   uint64_t* tempty = tfull + 2;
+  uint64_t* sched_full = tempty + 2;                 // [kSchedRing], DYNAMIC only
+  uint64_t* sched_empty = sched_full + kSchedRing;   // [kSchedRing]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + S::misc_off);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base + S::misc_off + 4);
+  volatile int* sched_tile = reinterpret_cast<volatile int*>(base + S::misc_off + 16);  // [kSchedRing]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -78,6 +91,11 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], 128);
     }
+    if constexpr (P::DYNAMIC)
+      for (int r = 0; r < kSchedRing; ++r) {
+        mbar_init(&sched_full[r], 1);
+        mbar_init(&sched_empty[r], 129);  // the MMA thread and the 128 epilogue threads
+      }
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -118,7 +136,15 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
       pdl_wait();
       const int n_tiles = P::num_tiles(p);
       uint32_t stage = 0, phase = 0;
-      for (int v = blockIdx.x; v < n_tiles; v += gridDim.x) {
+      for (int i = 0, v = blockIdx.x;; ++i, v += gridDim.x) {
+        if constexpr (P::DYNAMIC) {
+          const int slot = i % kSchedRing;
+          if (!mbar_wait_bounded(&sched_empty[slot], ((i / kSchedRing) & 1) ^ 1, abort_flag, err)) break;
+          v = atomicAdd(p.sched, 1);
+          sched_tile[slot] = v;
+          mbar_arrive(&sched_full[slot]);
+        }
+        if (v >= n_tiles) break;
         const Tile t = P::tile(p, v);
         if (!t.valid) continue;
         const uint32_t tx = P::tx_bytes(p, t);
@@ -151,7 +177,14 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
     const int n_tiles = P::num_tiles(p);
     if (lane == 0) {
       uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
-      for (int v = blockIdx.x; v < n_tiles; v += gridDim.x) {
+      for (int i = 0, v = blockIdx.x;; ++i, v += gridDim.x) {
+        if constexpr (P::DYNAMIC) {
+          const int slot = i % kSchedRing;
+          if (!mbar_wait_bounded(&sched_full[slot], (i / kSchedRing) & 1, abort_flag, err)) break;
+          v = sched_tile[slot];
+          mbar_arrive(&sched_empty[slot]);
+        }
+        if (v >= n_tiles) break;
         const Tile t = P::tile(p, v);
         if (!t.valid) continue;
         if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1, abort_flag, err)) break;
@@ -196,7 +229,14 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
     const int row = q * 32 + lane;     // accumulator row (M index) owned by this thread
     P::epilogue_init(p, row, ep_smem);
     uint32_t acc = 0, acc_phase = 0;
-    for (int v = blockIdx.x; v < n_tiles; v += gridDim.x) {
+    for (int i = 0, v = blockIdx.x;; ++i, v += gridDim.x) {
+      if constexpr (P::DYNAMIC) {
+        const int slot = i % kSchedRing;
+        if (!mbar_wait_bounded(&sched_full[slot], (i / kSchedRing) & 1, abort_flag, err)) break;
+        v = sched_tile[slot];
+        mbar_arrive(&sched_empty[slot]);
+      }
+      if (v >= n_tiles) break;
       const Tile t = P::tile(p, v);
       if (!t.valid) continue;
       P::epilogue_prefetch(p, t, row);
@@ -225,6 +265,7 @@ struct ProblemBase {
   static constexpr bool PRELOAD = false;  // true: static tiles, load_w / load_x split of load
   static constexpr int KB = 1;            // k-blocks per ring stage
   static constexpr bool F8 = false;       // E4M3 operands (kind::f8f6f4): a k-block is 128 elements
+  static constexpr bool DYNAMIC = false;  // tiles from the global counter p.sched (see above)
   template <class Params>
   DG_DEVINL static void epilogue_init(const Params&, int, uint8_t*) {}
   template <class Params>
