@@ -33,6 +33,7 @@ constexpr int kAQ = 128;        // query rows per CTA
 constexpr int kAK = 64;         // keys per tile
 constexpr int kAStages = 3;     // K/V ring depth
 constexpr float kRescaleLog2 = 8.0f;
+constexpr int kMaxSplits = 8;   // key splits of one query tile (also the largest cluster)
 constexpr int kVWarp = 6;                 // V^T producer
 constexpr int kPVWarp = 7;                // issuer of the P V MMAs
 constexpr int kAttnThreads = 32 * (kPVWarp + 1);
@@ -49,6 +50,10 @@ struct AttnSmem {
   static constexpr size_t k_off = 0;
   static constexpr size_t v_off = k_off + (size_t)kAStages * kK;
   static constexpr size_t p_off = v_off + (size_t)kAStages * kV;
+  // after the last MMA the K and V rings hold the finished O rows (fp32,
+  // 128 x D) and, with the cluster merge, each row's (max, sum) behind them
+  static constexpr size_t ml_off = k_off + (size_t)kAQ * D * 4;
+  static_assert(ml_off + kAQ * 8 <= p_off, "O staging exceeds the K and V rings");
   static constexpr size_t bar_off = p_off + 2 * (size_t)kP;
   static constexpr int kBars = 4 * kAStages + 9;
   static constexpr size_t misc_off = bar_off + kBars * 8;
@@ -67,6 +72,31 @@ DG_DEVINL void tmem_st16_raw(uint32_t taddr, const uint32_t* r) {
 }
 
 DG_DEVINL void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Distributed shared memory of the CTAs of a cluster.
+DG_DEVINL uint32_t dsmem_addr(uint32_t local_addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_addr), "r"(rank));
+  return r;
+}
+DG_DEVINL float4 ld_dsmem_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+DG_DEVINL float2 ld_dsmem_f2(uint32_t addr) {
+  float2 v;
+  asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr) : "memory");
+  return v;
+}
+// Every thread of every CTA of the cluster; orders this CTA's earlier shared
+// memory writes before the other CTAs' later reads of them.
+DG_DEVINL void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
 
 template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_constant__ AttnArgs a) {
@@ -99,6 +129,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
   if ((int)blockIdx.z >= n_split) {  // this slot uses fewer key splits
     pdl_trigger();
     pdl_wait();
+    if (a.cluster) {  // not launched this way (uniform splits), but never leave a cluster waiting
+      float2* ml = reinterpret_cast<float2*>(base + S::ml_off);
+      if (threadIdx.x < kAQ) ml[threadIdx.x] = make_float2(-INFINITY, 0.f);
+      __syncthreads();
+      cluster_sync_all();
+      cluster_sync_all();
+    }
     return;
   }
   int per = (n_keys + n_split - 1) / n_split;
@@ -329,38 +366,71 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
     if (ok && n_tiles > 0 &&
         mbar_wait_bounded(&pv_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, abort_flag, err)) {
       tc_fence_after();
-      if (n_split == 1) {
-        const float inv = l > 0.f ? 1.f / l : 0.f;
-        uint4* dst = reinterpret_cast<uint4*>(a.o + (size_t)t * a.Hq * D + (size_t)h * D);
-        for (int c = 0; c < D; c += 16) {
-          float o[16];
-          tmem_ld16(tm_o + lane_off + c, o);
-          if (valid) {
-            uint4 u0, u1;
-            u0.x = pack_bf16x2(o[0] * inv, o[1] * inv);
-            u0.y = pack_bf16x2(o[2] * inv, o[3] * inv);
-            u0.z = pack_bf16x2(o[4] * inv, o[5] * inv);
-            u0.w = pack_bf16x2(o[6] * inv, o[7] * inv);
-            u1.x = pack_bf16x2(o[8] * inv, o[9] * inv);
-            u1.y = pack_bf16x2(o[10] * inv, o[11] * inv);
-            u1.z = pack_bf16x2(o[12] * inv, o[13] * inv);
-            u1.w = pack_bf16x2(o[14] * inv, o[15] * inv);
-            dst[c / 8] = u0;
-            dst[c / 8 + 1] = u1;
+      // Each warp stages its 32 finished rows in shared memory (the K and V
+      // rings: every MMA that read them has completed) and then writes them
+      // row by row, each lane storing 16 consecutive bytes of the row, so every
+      // store instruction covers whole 128-byte lines.  Chunk c of local row i
+      // is kept at position c ^ (i mod nch) (conflict-free both ways).
+      const bool direct = n_split == 1;
+      const bool merge = a.cluster != 0;
+      const int nch = direct ? D / 8 : D / 4;  // 16-byte chunks per output row (bf16 / fp32)
+      uint4* stg = reinterpret_cast<uint4*>(sK) + (size_t)q * 32 * (D / 4);
+      const float inv = direct ? (l > 0.f ? 1.f / l : 0.f) : 1.f;
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 64) {
+        uint32_t r[4][16];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) tmem_ld16_issue(tm_o + lane_off + c0 + 16 * u, r[u]);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) tmem_ld_wait16(r[u]);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int col = c0 + 16 * u;
+          if (direct) {
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              uint4 w;
+              const uint32_t* x = r[u] + 8 * hh;
+              w.x = pack_bf16x2(__uint_as_float(x[0]) * inv, __uint_as_float(x[1]) * inv);
+              w.y = pack_bf16x2(__uint_as_float(x[2]) * inv, __uint_as_float(x[3]) * inv);
+              w.z = pack_bf16x2(__uint_as_float(x[4]) * inv, __uint_as_float(x[5]) * inv);
+              w.w = pack_bf16x2(__uint_as_float(x[6]) * inv, __uint_as_float(x[7]) * inv);
+              const int ch = col / 8 + hh;
+              stg[lane * nch + (ch ^ (lane & (nch - 1)))] = w;
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int ch = col / 4 + i;
+              stg[lane * nch + (ch ^ (lane & (nch - 1)))] =
+                  make_uint4(r[u][4 * i], r[u][4 * i + 1], r[u][4 * i + 2], r[u][4 * i + 3]);
+            }
           }
         }
-      } else {
-        const size_t prow_i = ((size_t)blockIdx.z * a.Hq + h) * a.q_T + t;
-        float4* dst = reinterpret_cast<float4*>(a.part_o + prow_i * D);
-        for (int c = 0; c < D; c += 16) {
-          float o[16];
-          tmem_ld16(tm_o + lane_off + c, o);
-          if (valid)
-#pragma unroll
-            for (int i = 0; i < 16; i += 4) dst[(c + i) / 4] = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
-        }
-        if (valid) a.part_ml[prow_i] = make_float2(m_used, l);
       }
+      __syncwarp();
+      if (!merge) {
+        // each lane knows its own row's destination; the warp writes row i from lane i's pointer
+        unsigned long long my_dst = 0ull;
+        if (valid)
+          my_dst = direct ? reinterpret_cast<unsigned long long>(a.o + (size_t)t * a.Hq * D + (size_t)h * D)
+                          : reinterpret_cast<unsigned long long>(
+                                a.part_o + (((size_t)blockIdx.z * a.Hq + h) * a.q_T + t) * D);
+#pragma unroll 4
+        for (int i = 0; i < 32; ++i) {
+          uint4* dst = reinterpret_cast<uint4*>(__shfl_sync(0xffffffffu, my_dst, i));
+          if (dst == nullptr) continue;
+          for (int c = lane; c < nch; c += 32) dst[c] = stg[i * nch + (c ^ (i & (nch - 1)))];
+        }
+      }
+      if (merge) {
+        reinterpret_cast<float2*>(base + S::ml_off)[row] = make_float2(m_used, l);
+      } else if (!direct && valid) {
+        const size_t prow_i = ((size_t)blockIdx.z * a.Hq + h) * a.q_T + t;
+        a.part_ml[prow_i] = make_float2(m_used, l);
+      }
+    } else if (a.cluster) {  // no keys in this split (or an aborted wait): zero weight in the merge
+      reinterpret_cast<float2*>(base + S::ml_off)[row] = make_float2(-INFINITY, 0.f);
     } else if (n_tiles == 0 && n_split > 1 && valid) {
       const size_t prow_i = ((size_t)blockIdx.z * a.Hq + h) * a.q_T + t;
       a.part_ml[prow_i] = make_float2(-INFINITY, 0.f);
@@ -371,6 +441,92 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (a.cluster) {
+    // The n_split CTAs of this query tile (one cluster) have staged their
+    // partial O rows and (max, sum); CTA z merges rows [z*rp, (z+1)*rp) from all
+    // of them, as O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s with M the
+    // largest max, in split order, and writes them in bf16.
+    cluster_sync_all();
+    if (warp >= 2 && warp <= 5) {
+      const int q = warp & 3;
+      const int ns = gridDim.z;
+      const int rp = (kAQ + ns - 1) / ns;
+      const int i0 = (int)blockIdx.z * rp, i1 = min(kAQ, i0 + rp);
+      const uint32_t stg = smem_u32(base + S::k_off), mls = smem_u32(base + S::ml_off);
+      // per merged row: the split weights 2^(m_s - M), 1 / L and the output row.
+      // The arithmetic (and its order) is that of k_attn_combine, so a query
+      // tile's result does not depend on which of the two merges it took.
+      float* wsm = reinterpret_cast<float*>(base + S::p_off);  // [kAQ][kMaxSplits + 1]
+      bf16** osm = reinterpret_cast<bf16**>(base + S::p_off + kAQ * (kMaxSplits + 1) * 4);  // [kAQ]
+      const int row = q * 32 + lane;
+      if (row >= i0 && row < i1) {
+        float2 ml[kMaxSplits];
+#pragma unroll
+        for (int s2 = 0; s2 < kMaxSplits; ++s2)
+          ml[s2] = s2 < ns ? ld_dsmem_f2(dsmem_addr(mls + row * 8, s2)) : make_float2(-INFINITY, 0.f);
+        float M = -INFINITY;
+#pragma unroll
+        for (int s2 = 0; s2 < kMaxSplits; ++s2) M = fmaxf(M, ml[s2].y > 0.f ? ml[s2].x : -INFINITY);
+        float w[kMaxSplits], x[kMaxSplits];
+#pragma unroll
+        for (int s2 = 0; s2 < kMaxSplits; ++s2) {
+          w[s2] = ml[s2].y > 0.f ? exp2f(ml[s2].x - M) : 0.f;
+          x[s2] = __fmul_rn(w[s2], ml[s2].y);
+        }
+        // the combine kernel's butterfly sum over lanes 0..7 (the other lanes hold 0)
+        const float L = __fadd_rn(__fadd_rn(__fadd_rn(x[0], x[4]), __fadd_rn(x[2], x[6])),
+                                  __fadd_rn(__fadd_rn(x[1], x[5]), __fadd_rn(x[3], x[7])));
+#pragma unroll
+        for (int s2 = 0; s2 < kMaxSplits; ++s2) wsm[row * (kMaxSplits + 1) + s2] = w[s2];
+        wsm[row * (kMaxSplits + 1) + kMaxSplits] = L > 0.f ? 1.f / L : 0.f;
+        const int qr = r0 + row;  // the output row (h, t) of merged row `row`
+        const int hr = g * G + (qr < rows ? qr / a.Tr : 0), tr = slot * a.Tr + (qr < rows ? qr % a.Tr : 0);
+        osm[row] = a.o + (size_t)tr * a.Hq * D + (size_t)hr * D;
+      }
+      named_bar_sync(1, 128);  // the four softmax warps
+      constexpr int nch = D / 4;   // 16-byte chunks of an fp32 row
+      constexpr int kRows = 2;     // rows merged side by side (loads in flight)
+#pragma unroll 1
+      for (int ib = i0 + q; ib < i1; ib += 4 * kRows) {
+#pragma unroll
+        for (int c0 = 0; c0 < nch; c0 += 32) {
+          const int c = c0 + lane;
+          float4 v[kRows][kMaxSplits];
+          float wr[kRows][kMaxSplits];
+#pragma unroll
+          for (int rr = 0; rr < kRows; ++rr) {
+            const int i = ib + 4 * rr;
+#pragma unroll
+            for (int s2 = 0; s2 < kMaxSplits; ++s2) {
+              wr[rr][s2] = (i < i1 && r0 + i < rows) ? wsm[i * (kMaxSplits + 1) + s2] : 0.f;
+              if (s2 < ns && wr[rr][s2] != 0.f && c < nch)
+                v[rr][s2] = ld_dsmem_f4(
+                    dsmem_addr(stg + (uint32_t)(i * nch + (c ^ (i & 31 & (nch - 1)))) * 16u, s2));
+            }
+          }
+#pragma unroll
+          for (int rr = 0; rr < kRows; ++rr) {
+            const int i = ib + 4 * rr;
+            if (i >= i1 || r0 + i >= rows || c >= nch) continue;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int s2 = 0; s2 < kMaxSplits; ++s2)
+              if (s2 < ns && wr[rr][s2] != 0.f) {
+                acc.x = __fmaf_rn(wr[rr][s2], v[rr][s2].x, acc.x);
+                acc.y = __fmaf_rn(wr[rr][s2], v[rr][s2].y, acc.y);
+                acc.z = __fmaf_rn(wr[rr][s2], v[rr][s2].z, acc.z);
+                acc.w = __fmaf_rn(wr[rr][s2], v[rr][s2].w, acc.w);
+              }
+            const float inv = wsm[i * (kMaxSplits + 1) + kMaxSplits];
+            reinterpret_cast<uint2*>(osm[i])[c] = make_uint2(pack_bf16x2(__fmul_rn(acc.x, inv), __fmul_rn(acc.y, inv)),
+                                                             pack_bf16x2(__fmul_rn(acc.z, inv), __fmul_rn(acc.w, inv)));
+          }
+        }
+      }
+    }
+    __syncwarp();
+    cluster_sync_all();  // no CTA leaves while another still reads its shared memory
+  }
   if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
@@ -378,8 +534,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
 // One warp per (token, head); lane s reads split s's (max, sum), each lane then
 // owns 8 consecutive output elements and loads every split's values at once.
 // Tokens of slots that used a single split were written by the attention kernel.
-constexpr int kMaxSplits = 8;
-
 struct SlotSplits {
   int s[DG_MAX_REQUESTS];
 };
@@ -400,9 +554,10 @@ __global__ void k_attn_combine(const float* __restrict__ part_o, const float2* _
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
   const float wl = ml.y > 0.f ? exp2f(ml.x - M) : 0.f;
-  float L = wl * ml.y;
+  // explicit roundings: the in-kernel cluster merge repeats exactly these operations
+  float L = __fmul_rn(wl, ml.y);
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+  for (int off = 16; off > 0; off >>= 1) L = __fadd_rn(L, __shfl_xor_sync(0xffffffffu, L, off));
   float wts[kMaxSplits];
 #pragma unroll
   for (int s = 0; s < kMaxSplits; ++s) wts[s] = __shfl_sync(0xffffffffu, wl, s);
@@ -420,21 +575,21 @@ __global__ void k_attn_combine(const float* __restrict__ part_o, const float2* _
 #pragma unroll
   for (int s = 0; s < kMaxSplits; ++s)
     if (s < n_split && wts[s] != 0.f) {
-      acc[0] += wts[s] * va[s].x;
-      acc[1] += wts[s] * va[s].y;
-      acc[2] += wts[s] * va[s].z;
-      acc[3] += wts[s] * va[s].w;
-      acc[4] += wts[s] * vb[s].x;
-      acc[5] += wts[s] * vb[s].y;
-      acc[6] += wts[s] * vb[s].z;
-      acc[7] += wts[s] * vb[s].w;
+      acc[0] = __fmaf_rn(wts[s], va[s].x, acc[0]);
+      acc[1] = __fmaf_rn(wts[s], va[s].y, acc[1]);
+      acc[2] = __fmaf_rn(wts[s], va[s].z, acc[2]);
+      acc[3] = __fmaf_rn(wts[s], va[s].w, acc[3]);
+      acc[4] = __fmaf_rn(wts[s], vb[s].x, acc[4]);
+      acc[5] = __fmaf_rn(wts[s], vb[s].y, acc[5]);
+      acc[6] = __fmaf_rn(wts[s], vb[s].z, acc[6]);
+      acc[7] = __fmaf_rn(wts[s], vb[s].w, acc[7]);
     }
   const float inv = L > 0.f ? 1.f / L : 0.f;
   uint4 u;
-  u.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
-  u.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
-  u.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
-  u.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
+  u.x = pack_bf16x2(__fmul_rn(acc[0], inv), __fmul_rn(acc[1], inv));
+  u.y = pack_bf16x2(__fmul_rn(acc[2], inv), __fmul_rn(acc[3], inv));
+  u.z = pack_bf16x2(__fmul_rn(acc[4], inv), __fmul_rn(acc[5], inv));
+  u.w = pack_bf16x2(__fmul_rn(acc[6], inv), __fmul_rn(acc[7], inv));
   *reinterpret_cast<uint4*>(o + (size_t)t * Hq * D + (size_t)h * D + c) = u;
 }
 
@@ -451,6 +606,14 @@ static cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st) {
   }
   const int G = a.Hq / a.Hkv;
   dim3 grid((G * a.Tr + kAQ - 1) / kAQ, a.Hkv * a.n_slots, a.n_split);
+  if (a.cluster) {  // the key splits of a query tile merge in-kernel (uniform splits only)
+    for (int i = 0; i < a.n_slots; ++i)
+      if (a.slot_split[i] != a.n_split) return cudaErrorInvalidValue;
+    const cudaError_t e_ = launch_pdl_cluster(k_attn_tc<D>, dim3(grid), dim3(kAttnThreads), smem, st,
+                                              (unsigned)a.n_split, a);
+    if (e_ != cudaSuccess) return e_;
+    return cudaGetLastError();
+  }
   {
     const cudaError_t e_ = launch_pdl(k_attn_tc<D>, dim3(grid), dim3(kAttnThreads), smem, st, a);
     if (e_ != cudaSuccess) return e_;

@@ -434,7 +434,13 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     aa.part_ml = h->B<float2>("attn_ml");
     aa.scale = 1.0f / sqrtf((float)D);
     aa.err = err;
-    LAUNCH(h, K_ATTN, aa.n_split > 1 ? 2 : 1, run_attention(aa, st));
+    // With the same key split in every slot the splits of a query tile run as
+    // one thread-block cluster and merge through distributed shared memory;
+    // otherwise their partials go through global memory and k_attn_combine.
+    bool uniform = aa.n_split > 1;
+    for (int i = 0; i < s.n; ++i) uniform = uniform && aa.slot_split[i] == aa.n_split;
+    aa.cluster = uniform ? 1 : 0;
+    LAUNCH(h, K_ATTN, aa.n_split > 1 && !aa.cluster ? 2 : 1, run_attention(aa, st));
 
     WpartArgs oa;
     oa.tm_w = &m.o;

@@ -32,6 +32,27 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
+// The same launch as thread-block clusters of cluster_z CTAs along z.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                      unsigned cluster_z, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 1;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = cluster_z;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // ---- arguments of the tcgen05 GEMM launchers (gemm_ops.cu) ----
 struct QkvArgs {
   const CUtensorMap* tm_x;  // normed tokens [Tcap, d]
@@ -236,6 +257,9 @@ struct AttnArgs {
   int slot_split[DG_MAX_REQUESTS];     // key splits of each slot (1 = direct output)
   float* part_o;     // [n_split][Hq][q_T][D]
   float2* part_ml;   // [n_split][Hq][q_T]
+  int cluster;       // 1: every slot has n_split key splits, which form one thread-block
+                     // cluster per query tile and merge through distributed shared memory
+                     // (part_o / part_ml unused)
   float scale;
   int* err;
 };
