@@ -73,31 +73,6 @@ DG_DEVINL void tmem_st16_raw(uint32_t taddr, const uint32_t* r) {
 
 DG_DEVINL void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-// Distributed shared memory of the CTAs of a cluster.
-DG_DEVINL uint32_t dsmem_addr(uint32_t local_addr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_addr), "r"(rank));
-  return r;
-}
-DG_DEVINL float4 ld_dsmem_f4(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(addr)
-               : "memory");
-  return v;
-}
-DG_DEVINL float2 ld_dsmem_f2(uint32_t addr) {
-  float2 v;
-  asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr) : "memory");
-  return v;
-}
-// Every thread of every CTA of the cluster; orders this CTA's earlier shared
-// memory writes before the other CTAs' later reads of them.
-DG_DEVINL void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
 template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_constant__ AttnArgs a) {
   using S = AttnSmem<D>;
@@ -610,7 +585,7 @@ static cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st) {
     for (int i = 0; i < a.n_slots; ++i)
       if (a.slot_split[i] != a.n_split) return cudaErrorInvalidValue;
     const cudaError_t e_ = launch_pdl_cluster(k_attn_tc<D>, dim3(grid), dim3(kAttnThreads), smem, st,
-                                              (unsigned)a.n_split, a);
+                                              dim3(1, 1, a.n_split), a);
     if (e_ != cudaSuccess) return e_;
     return cudaGetLastError();
   }

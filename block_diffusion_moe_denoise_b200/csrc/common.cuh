@@ -126,6 +126,37 @@ DG_DEVINL void tma_prefetch_desc(const CUtensorMap* map) {
 }
 
 // ---------------------------------------------------------------------------
+// Distributed shared memory of the CTAs of a cluster.
+DG_DEVINL uint32_t dsmem_addr(uint32_t local_addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_addr), "r"(rank));
+  return r;
+}
+DG_DEVINL float4 ld_dsmem_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+DG_DEVINL float ld_dsmem_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+DG_DEVINL float2 ld_dsmem_f2(uint32_t addr) {
+  float2 v;
+  asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr) : "memory");
+  return v;
+}
+// Every thread of every CTA of the cluster; orders this CTA's earlier shared
+// memory writes before the other CTAs' later reads of them.
+DG_DEVINL void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
 // tcgen05: tensor memory allocation, MMA, commit, loads, fences
 // ---------------------------------------------------------------------------
 DG_DEVINL void tmem_alloc(uint32_t* dst_smem_slot, uint32_t ncols) {  // whole warp

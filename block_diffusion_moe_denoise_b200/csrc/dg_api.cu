@@ -106,7 +106,7 @@ void make_plan(const dg_config* c, int max_req, long long cap_user, Plan* p) {
   p->add("ed_tiles", (size_t)n_nt * (d / 128) * 16);
   p->add("xp", (size_t)rows * d * 2);
   p->add("hp", (size_t)rows * c->ffn_expert * 2);
-  p->add("yp", (size_t)rows * d * 4);
+  p->add("yp", (size_t)rows * d * 2);
   p->add("hs", (size_t)Tcap * c->ffn_shared * 2);
   p->add("attn_o", (size_t)kSplitCap * c->n_q_heads * Tcap * D * 4);
   p->add("attn_ml", (size_t)kSplitCap * c->n_q_heads * Tcap * 8);
@@ -319,7 +319,7 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
                    h->B<double>("inv_freq"), D / 2, h->B<float2>("rope"), err, st));
   // the routed outputs and the shared-expert partials of layer l are summed
   // into x by the norm kernel of layer l+1 (or the final norm)
-  float* yp = h->B<float>("yp");
+  bf16* yp = h->B<bf16>("yp");
   const int* pair_row = h->B<int>("pair_row");
   float* part = h->B<float>("part");
   int pending_k = 0, pending_parts = 0;

@@ -32,10 +32,10 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
-// The same launch as thread-block clusters of cluster_z CTAs along z.
+// The same launch as thread-block clusters of the given shape.
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
-                                      unsigned cluster_z, Args... args) {
+                                      dim3 cluster, Args... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -45,9 +45,9 @@ inline cudaError_t launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   attr[1].id = cudaLaunchAttributeClusterDimension;
-  attr[1].val.clusterDim.x = 1;
-  attr[1].val.clusterDim.y = 1;
-  attr[1].val.clusterDim.z = cluster_z;
+  attr[1].val.clusterDim.x = cluster.x;
+  attr[1].val.clusterDim.y = cluster.y;
+  attr[1].val.clusterDim.z = cluster.z;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kernel, args...);
@@ -86,7 +86,7 @@ struct ExpertArgs {
   const int* offsets;
   const float* row_weight;
   bf16* hp;
-  float* yp;
+  bf16* yp;  // gate-weighted routed outputs, bf16
   int* err;
   // FP8 experts: per-row scales of the weight codes and of the token / hidden codes
   const float *s_gate = nullptr, *s_up = nullptr, *s_down = nullptr, *s_x = nullptr, *s_h = nullptr;
@@ -158,7 +158,7 @@ cudaError_t run_embed(const int* const* ids, const SlotInfo& s, const bf16* embe
                       int* tok_req, const double* inv_freq, int half, float2* rope, int* err, cudaStream_t st);
 // x[t] += sum_j yp[pair_row[t*k+j]] + sum_s part[s][t]; then (if an output is
 // given) the RMSNorm of x[t] with gain g as bf16
-cudaError_t run_residual_norm(float* x, const float* yp, const int* pair_row, int k, const float* part, int n_part,
+cudaError_t run_residual_norm(float* x, const bf16* yp, const int* pair_row, int k, const float* part, int n_part,
                               int Tcap, const float* g, int T, int d, float eps, bf16* out, cudaStream_t st);
 cudaError_t run_rmsnorm(const float* x, const float* g, int T, int d, float eps, bf16* out, cudaStream_t st);
 cudaError_t run_topk(const float* logits, int T, int E, int k, int* idx, float* w, cudaStream_t st);

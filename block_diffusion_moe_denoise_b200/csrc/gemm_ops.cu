@@ -365,7 +365,7 @@ struct P_ED : ProblemBase {
     const int* counts;
     const int* offsets;
     const float* row_weight;
-    float* yp;  // [rows_cap, d]
+    bf16* yp;   // [rows_cap, d], gate-weighted expert outputs
     int* sched;  // tile counter (zeroed by the grouping kernel)
     int* err;
   };
@@ -403,7 +403,7 @@ struct P_ED : ProblemBase {
         const int c = c0 + i;
         if (c < t.c) {
           const int r = t.d + c;
-          p.yp[(size_t)r * p.d + f] = p.row_weight[r] * v[i];
+          p.yp[(size_t)r * p.d + f] = __float2bfloat16_rn(p.row_weight[r] * v[i]);
         }
       }
     }
@@ -509,7 +509,7 @@ struct P_ED8 : ProblemBase {
     const float* sw;   // [E*d] down row scales
     const float* sh;   // [rows] hidden row scales
     const float* row_weight;
-    float* yp;  // [rows_cap, d]
+    bf16* yp;   // [rows_cap, d], gate-weighted expert outputs
     int* sched;  // tile counter (zeroed by the grouping kernel)
     int* err;
   };
@@ -548,7 +548,7 @@ struct P_ED8 : ProblemBase {
         const int c = c0 + i;
         if (c < t.c) {
           const int r = t.d + c;
-          p.yp[(size_t)r * p.d + f] = p.row_weight[r] * (v[i] * sw * p.sh[r]);
+          p.yp[(size_t)r * p.d + f] = __float2bfloat16_rn(p.row_weight[r] * (v[i] * sw * p.sh[r]));
         }
       }
     }

@@ -116,7 +116,10 @@ cudaError_t run_rmsnorm(const float* x, const float* g, int T, int d, float eps,
 // The routed experts' outputs (slot order) and the split-K partials (slice
 // order) are added in a fixed order, so the result is deterministic.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(512) k_residual_norm(float* __restrict__ x, const float* __restrict__ yp,
+// One CTA per SM at most by registers on purpose: the GEMM launched after it
+// (programmatic dependent launch) must find room on every SM to become
+// resident and start its weight loads while this kernel still runs.
+__global__ void __launch_bounds__(512) k_residual_norm(float* __restrict__ x, const bf16* __restrict__ yp,
                                                         const int* __restrict__ pair_row, int k,
                                                         const float* __restrict__ part, int n_part,
                                                         size_t part_stride, const float* __restrict__ g, int d,
@@ -134,20 +137,23 @@ __global__ void __launch_bounds__(512) k_residual_norm(float* __restrict__ x, co
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     v[h] = xr[c + h];
-    float4 y[8], q[kMaxPartSplits];
+    uint2 y[8];  // 4 bf16
+    float4 q[kMaxPartSplits];
 #pragma unroll
     for (int j = 0; j < 8; ++j)
-      if (j < k) y[j] = reinterpret_cast<const float4*>(yp + (size_t)rows[j] * d)[c + h];
+      if (j < k) y[j] = reinterpret_cast<const uint2*>(yp + (size_t)rows[j] * d)[c + h];
 #pragma unroll
     for (int j = 0; j < kMaxPartSplits; ++j)
       if (j < n_part) q[j] = reinterpret_cast<const float4*>(part + j * part_stride + (size_t)t * d)[c + h];
 #pragma unroll
     for (int j = 0; j < 8; ++j)
       if (j < k) {
-        v[h].x += y[j].x;
-        v[h].y += y[j].y;
-        v[h].z += y[j].z;
-        v[h].w += y[j].w;
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&y[j].x));
+        const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&y[j].y));
+        v[h].x += a.x;
+        v[h].y += a.y;
+        v[h].z += b.x;
+        v[h].w += b.y;
       }
 #pragma unroll
     for (int j = 0; j < kMaxPartSplits; ++j)
@@ -189,7 +195,7 @@ __global__ void __launch_bounds__(512) k_residual_norm(float* __restrict__ x, co
   reinterpret_cast<uint4*>(out + (size_t)t * d)[threadIdx.x] = o;
 }
 
-cudaError_t run_residual_norm(float* x, const float* yp, const int* pair_row, int k, const float* part, int n_part,
+cudaError_t run_residual_norm(float* x, const bf16* yp, const int* pair_row, int k, const float* part, int n_part,
                               int Tcap, const float* g, int T, int d, float eps, bf16* out, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
   if (n_part > kMaxPartSplits || k > 8 || d % 256 != 0 || d > 4096) return cudaErrorInvalidValue;
@@ -454,7 +460,8 @@ cudaError_t run_quant_rows(const bf16* in, int n, int rows, uint8_t* out, float*
 // row into the expert-grouped buffer.  It also clears the other mask buffer
 // (used by the previous layer, read by nobody now) for the next layer.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) k_group_gather(GroupArgs a, const unsigned* __restrict__ mask,
+template <bool kF8>
+__global__ void __launch_bounds__(512) k_group_gather(GroupArgs a, const unsigned* __restrict__ mask,
                                                       unsigned* __restrict__ mask_next, int MW,
                                                       const bf16* __restrict__ u, int d, bf16* __restrict__ xp,
                                                       uint8_t* __restrict__ xq, float* __restrict__ xs) {
@@ -556,20 +563,21 @@ __global__ void __launch_bounds__(256) k_group_gather(GroupArgs a, const unsigne
       a.row_weight[row] = a.w[p];
       a.row_pair[row] = p;
     }
-    if (xq != nullptr) {  // FP8 experts: the row is quantised on the way (same codes for every copy)
+    if constexpr (kF8) {  // FP8 experts: the row is quantised on the way (same codes for every copy)
       quant_row_warp(u + (size_t)t * d, d, xq + (size_t)row * d, xs + row, lane);
       continue;
     }
+    // rows of up to 3072 features in flight at once (12 chunks of 16 bytes per lane)
     const uint4* src = reinterpret_cast<const uint4*>(u + (size_t)t * d);
     uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)row * d);
     const int n16 = d / 8;
-    for (int c0 = lane; c0 < n16; c0 += 32 * 4) {
-      uint4 r[4];
+    for (int c0 = lane; c0 < n16; c0 += 32 * 12) {
+      uint4 r[12];
 #pragma unroll
-      for (int b = 0; b < 4; ++b)
+      for (int b = 0; b < 12; ++b)
         if (c0 + b * 32 < n16) r[b] = src[c0 + b * 32];
 #pragma unroll
-      for (int b = 0; b < 4; ++b)
+      for (int b = 0; b < 12; ++b)
         if (c0 + b * 32 < n16) dst[c0 + b * 32] = r[b];
     }
   }
@@ -579,11 +587,14 @@ cudaError_t run_route(const bf16* u, int d, bf16* xp, unsigned* mask, unsigned* 
                       const GroupArgs& a, cudaStream_t st, uint8_t* xq, float* xs) {
   if (a.T < 1 || a.T > DG_MAX_REQUESTS * 256 || a.E > 256 || MW * 32 < a.T) return cudaErrorInvalidValue;
   if (xq != nullptr && (d % 8 != 0 || d > 4096 || xs == nullptr)) return cudaErrorInvalidValue;
+  // one pair per warp where the GPU allows (16 warps per CTA, one CTA per SM)
   const int P = a.T * a.k;
-  const int grid = (P + 7) / 8 < 148 ? (P + 7) / 8 : 148;
+  const int grid = (P + 15) / 16 < 148 ? (P + 15) / 16 : 148;
   {
-    const cudaError_t e_ = launch_pdl(k_group_gather, dim3(grid), dim3(256), 0, st, a, mask, mask_next, MW, u, d, xp, xq,
-                                      xs);
+    const cudaError_t e_ = xq != nullptr ? launch_pdl(k_group_gather<true>, dim3(grid), dim3(512), 0, st, a, mask,
+                                                      mask_next, MW, u, d, xp, xq, xs)
+                                         : launch_pdl(k_group_gather<false>, dim3(grid), dim3(512), 0, st, a, mask,
+                                                      mask_next, MW, u, d, xp, xq, xs);
     if (e_ != cudaSuccess) return e_;
   }
   return cudaGetLastError();

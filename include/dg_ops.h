@@ -84,7 +84,7 @@ int dg_debug_forward_hidden(dg_handle* h, int req, const int32_t* d_tokens, cons
  * "router_logits" f32 [T, E]; "idx" i32 [T, k]; "w" f32 [T, k];
  * "counts" i32 [E]; "offsets" i32 [E+1];
  * "pair_row" i32 [T*k]; "row_pair" i32 [T*k]; "hp" bf16 [T*k, fe];
- * "yp" f32 [T*k, d]; "hs" bf16 [T, fs]; "stats" f32 [Tcap][4];
+ * "yp" bf16 [T*k, d]; "hs" bf16 [T, fs]; "stats" f32 [Tcap][4];
  * "argmax" i32 [Tcap]; "cand" i32 [max_req * canvas] drawn candidates;
  * "sc_top" f32/i32 pairs [max_req][canvas][8] self-conditioning state;
  * "canvas" i32 [max_req, canvas]; "mask" u8 [...];

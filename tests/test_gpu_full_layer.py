@@ -77,7 +77,7 @@ def test_moe_path(setup):
     counts = h.debug_buffer("counts", torch.int32, (CFG.n_experts,)).cpu().numpy()
     assert counts.sum() == T * k and (counts == np.bincount(idx.ravel(), minlength=CFG.n_experts)).all()
     pair_row = h.debug_buffer("pair_row", torch.int32, (T * k,)).cpu().numpy()
-    yp = np64(h.debug_buffer("yp", torch.float32, (T * k, d)))
+    yp = np64(h.debug_buffer("yp", torch.bfloat16, (T * k, d)))
     W = ora.layer(0)
     rng = np.random.default_rng(0)
     got, ref = [], []

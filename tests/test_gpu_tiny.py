@@ -155,7 +155,7 @@ def test_layer_intermediates(model, T):
     # expert hidden / weighted outputs, per (token, slot) pair in grouped order
     pair_row = h.debug_buffer("pair_row", torch.int32, (T * k,)).cpu().numpy()
     hp = np64(h.debug_buffer("hp", torch.bfloat16, (T * k, CFG.ffn_expert)))
-    yp = np64(h.debug_buffer("yp", torch.float32, (T * k, d)))
+    yp = np64(h.debug_buffer("yp", torch.bfloat16, (T * k, d)))
     W = ora.layer(0)
     got_h, ref_h, got_y, ref_y = [], [], [], []
     for t in np.nonzero(same)[0]:
