@@ -128,16 +128,17 @@ class ClockSampler:
                 "samples": len(loaded), "power_w_max": max(r[2] for r in rows)}
 
 
-def kernel_source_digest(problem: str) -> str:
+def kernel_source_digest(*problems: str) -> str:
     """sha256 over the source a routed-expert GEMM is built from: its problem
-    struct in gemm_ops.cu, the GEMM engine and the shared device helpers.  A
+    structs in gemm_ops.cu, the GEMM engine and the shared device helpers.  A
     stored ncu traffic ratio is used only while this digest is unchanged."""
     import hashlib
     csrc = os.path.join(ROOT, "block_diffusion_moe_denoise_b200", "csrc")
     text = open(os.path.join(csrc, "gemm_ops.cu")).read()
-    start = text.index(f"struct {problem} : ProblemBase {{")
-    body = text[start:text.index("\n};\n", start) + 4]
-    h = hashlib.sha256(body.encode())
+    h = hashlib.sha256()
+    for problem in problems:
+        start = text.index(f"struct {problem} : ProblemBase {{")
+        h.update(text[start:text.index("\n};\n", start) + 4].encode())
     for f in ("umma_gemm.cuh", "common.cuh"):
         h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()
@@ -154,6 +155,16 @@ def expert_gate_up_bytes(cfg, n_touched: float, T: int) -> float:
     w = n_touched * 2 * cfg.ffn_expert * (cfg.d_model * eb + (4 if eb == 1 else 0))
     rows = T * cfg.top_k
     return w + rows * (cfg.d_model * eb + (4 if eb == 1 else 0)) + rows * cfg.ffn_expert * 2
+
+
+def expert_bytes(cfg, n_touched: float, T: int) -> float:
+    """Bytes the fused bf16 routed-expert launch (gate|up, SwiGLU, down) must
+    move: all three weight matrices of every expert some token is routed to,
+    the grouped token rows read, the SwiGLU rows written and read back, the
+    gate-weighted outputs written (bf16)."""
+    rows = T * cfg.top_k
+    w = n_touched * 3 * cfg.ffn_expert * cfg.d_model * 2
+    return w + rows * cfg.d_model * 2 * 2 + rows * cfg.ffn_expert * 2 * 2
 
 
 def step_work(cfg, kv_len: int, T: int, n_touched: float, n_req: int = 1):
@@ -501,17 +512,19 @@ def main():
     # experts that received at least one token, averaged over every layer of the profiled step
     n_touched = float((rs1[0] - rs0[0]) / max(1, int(rs1[1] - rs0[1])))
     T = cfg.canvas
-    egu_ms, egu_n = prof["experts_gate_up"]
-    egu_bytes = expert_gate_up_bytes(cfg, n_touched, T)
+    fp8 = bool(getattr(cfg, "expert_fp8", 0))
+    # dominant kernel: the fused routed-expert launch (bf16), or the FP8 experts' gate|up launch
+    egu_ms, egu_n = prof["experts_gate_up" if fp8 else "experts"]
+    egu_bytes = expert_gate_up_bytes(cfg, n_touched, T) if fp8 else expert_bytes(cfg, n_touched, T)
     egu_avg_ms = egu_ms / max(1, egu_n)
     achieved = egu_bytes / (egu_avg_ms * 1e-3) / 1e9
     traffic = None
-    tname = "experts_gate_up_fp8_traffic.json" if getattr(cfg, "expert_fp8", 0) else "experts_gate_up_traffic.json"
+    tname = "experts_gate_up_fp8_traffic.json" if fp8 else "experts_traffic.json"
     tpath = os.path.join(ROOT, "profiles", tname)
     if os.path.exists(tpath):
         try:
             tj = json.load(open(tpath))
-            src = kernel_source_digest("P_EGU8" if getattr(cfg, "expert_fp8", 0) else "P_EGU")
+            src = kernel_source_digest("P_EGU8") if fp8 else kernel_source_digest("P_EGU", "P_ED", "P_EXP")
             # The capture is a smaller case (one layer, 124 experts touched); DRAM
             # traffic grows in proportion to the expert weights streamed, so it is
             # scaled to this launch by its algorithmic bytes.
@@ -562,8 +575,8 @@ def main():
             s = oracle_sample(reps=3, warm=1, min_seconds=10.0)
             cpu = {k: s[k] for k in ("value", "unit", "cores", "kind", "sample")}
 
-    roofline = {"kernel": ("experts_gate_up (routed-expert gate|up GEMM + SwiGLU"
-                           + (", E4M3 W8A8)" if getattr(cfg, "expert_fp8", 0) else ")")), "bound": "hbm",
+    roofline = {"kernel": ("experts_gate_up (routed-expert gate|up GEMM + SwiGLU, E4M3 W8A8)" if fp8 else
+                           "experts (routed-expert gate|up GEMM + SwiGLU + down GEMM, one launch)"), "bound": "hbm",
                 "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s", "frac": achieved / hbm_gbs,
                 "traffic": traffic, "algorithmic_bytes_per_launch": egu_bytes,
                 "avg_launch_ms": egu_avg_ms, "peak_source": f"{peak_kind} HBM copy (MEASURED_PEAKS.json)"}

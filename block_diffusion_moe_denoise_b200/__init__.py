@@ -291,7 +291,7 @@ class DG:
 
     KERNEL_CLASSES = ("embed", "rmsnorm", "qkv", "attention", "oproj", "group",
                       "experts_gate_up", "experts_down", "shared_gate_up", "shared_down", "lm_head", "lm_combine",
-                      "sample", "selfcond", "other")
+                      "sample", "selfcond", "other", "experts")
 
     def profile(self, enable: int):
         check(self.lib.dg_profile(self.h, enable), "dg_profile")

@@ -110,6 +110,37 @@ DG_DEVINL bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, volatile int* a
   }
 }
 
+// Wait (bounded like mbar_wait_bounded) until the counter reaches target;
+// acquire ordering, then a proxy fence so that TMA loads issued afterwards see
+// the data the counted writers stored before their release.
+DG_DEVINL bool counter_wait_bounded(const int* ctr, int target, volatile int* abort, int* err) {
+  auto load = [&]() {
+    int v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+    return v;
+  };
+  if (load() < target) {
+    const uint64_t t0 = globaltimer_ns();
+    while (load() < target) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > DG_WAIT_LIMIT_NS) {
+        *abort = 1;
+        if (err) atomicOr(err, DG_DEVERR_TIMEOUT);
+        return false;
+      }
+      __nanosleep(64);
+    }
+  }
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  return true;
+}
+
+// Release side of counter_wait_bounded for data written by this thread.
+DG_DEVINL void counter_release_fence() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  __threadfence();
+}
+
 // ---------------------------------------------------------------------------
 // TMA (bulk tensor copies global -> shared, completion on an mbarrier)
 // ---------------------------------------------------------------------------

@@ -141,6 +141,7 @@ void make_plan(const dg_config* c, int max_req, long long cap_user, Plan* p) {
   p->add("part", (size_t)kMaxPartSplits * Tcap * d * 4);
   p->add("route_mask", (size_t)2 * c->n_experts * ((T + 31) / 32) * 4);
   p->add("sched", 64);
+  p->add("ready", (size_t)n_nt * 4);
   p->add("prompt", (size_t)cap_user * 4);
 }
 
@@ -233,9 +234,11 @@ struct KernelProfiler {
 
 const char* const kKernelClass[] = {"embed", "rmsnorm", "qkv", "attention", "oproj", "group",
                                     "experts_gate_up", "experts_down", "shared_gate_up", "shared_down", "lm_head",
-                                    "lm_combine", "sample", "selfcond", "other"};
+                                    "lm_combine", "sample", "selfcond", "other", "experts"};
+// K_EXP: the fused routed-expert launch (gate|up, SwiGLU and down); K_EGU /
+// K_ED: the two launches of the FP8 experts
 enum KClass { K_EMBED, K_RMSNORM, K_QKV, K_ATTN, K_OPROJ, K_GROUP, K_EGU, K_ED, K_SGU, K_SD, K_LM, K_LMC, K_SAMPLE,
-              K_SC, K_OTHER, K_NCLASS };
+              K_SC, K_OTHER, K_EXP, K_NCLASS };
 static_assert(K_NCLASS <= 16, "profiler tables hold 16 classes");
 
 struct dg_handle {
@@ -507,6 +510,7 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     ga.route_stats = h->B<unsigned long long>("route_stats");
     ga.err = err;
     ga.sched = h->B<int>("sched");
+    ga.ready = h->B<int>("ready");
     const bool f8 = c.expert_fp8 != 0;
     LAUNCH(h, K_GROUP, 1,
            run_route(h->B<bf16>("u"), d, h->B<bf16>("xp"), mask_cur, mask_nxt, MW, ga, st,
@@ -545,8 +549,8 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
       LAUNCH(h, K_ED, 1, run_quant_rows(ea.hp, c.ffn_expert, T * k, h->B<uint8_t>("hq"), h->B<float>("hsq"), st));
       LAUNCH(h, K_ED, 1, run_experts_down_fp8(ea, st));
     } else {
-      LAUNCH(h, K_EGU, 1, run_experts_gate_up(ea, st));
-      LAUNCH(h, K_ED, 1, run_experts_down(ea, st));
+      ea.ready = h->B<int>("ready");
+      LAUNCH(h, K_EXP, 1, run_experts(ea, st));
     }
 
     WpartArgs da;

@@ -91,6 +91,7 @@ struct ExpertArgs {
   // FP8 experts: per-row scales of the weight codes and of the token / hidden codes
   const float *s_gate = nullptr, *s_up = nullptr, *s_down = nullptr, *s_x = nullptr, *s_h = nullptr;
   int* sched = nullptr;  // [2] tile counters of the gate|up and down launches (zeroed by the grouping kernel)
+  int* ready = nullptr;  // [token tiles] per-token-tile gate|up completions of run_experts (zeroed likewise)
 };
 struct SharedArgs {
   const CUtensorMap *tm_u, *tm_gate, *tm_up, *tm_router;
@@ -137,8 +138,8 @@ struct LmArgs {
 cudaError_t run_qkv(const QkvArgs& a, cudaStream_t st);
 int wpart_splits(int d, int T, int K, int num_sms);
 cudaError_t run_wpart(const WpartArgs& a, cudaStream_t st);
-cudaError_t run_experts_gate_up(const ExpertArgs& a, cudaStream_t st);
-cudaError_t run_experts_down(const ExpertArgs& a, cudaStream_t st);
+// gate|up and down of the bf16 routed experts in one launch (needs a.ready, a.sched)
+cudaError_t run_experts(const ExpertArgs& a, cudaStream_t st);
 cudaError_t run_experts_gate_up_fp8(const ExpertArgs& a, cudaStream_t st);
 cudaError_t run_experts_down_fp8(const ExpertArgs& a, cudaStream_t st);
 cudaError_t run_shared_gate_up(const SharedArgs& a, cudaStream_t st);
@@ -179,6 +180,7 @@ struct GroupArgs {
   unsigned long long* route_stats;  // [0] += experts touched, [1] += launches (may be null)
   int* err;
   int* sched = nullptr;             // [2] tile counters of the expert GEMMs that follow, zeroed here
+  int* ready = nullptr;             // [token tiles] counters of the fused expert launch, zeroed here
 };
 cudaError_t run_group(const GroupArgs& a, cudaStream_t st);
 // the grouping above from the token bitmasks `mask` ([E][MW] words, MW fixed by

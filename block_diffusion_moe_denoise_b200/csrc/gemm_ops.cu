@@ -268,8 +268,9 @@ struct P_WPART : ProblemBase {
 };
 
 // ---------------------------------------------------------------------------
-// Routed experts, gate|up + SwiGLU.  Tile (e, j, nt): hidden units j*64..+63 of
-// expert e for its tokens nt*64..+63 (rows of the expert-grouped buffer).
+// Routed experts, gate|up + SwiGLU (the first tile kind of P_EXP below).
+// Tile (e, j, nt): hidden units j*64..+63 of expert e for its tokens
+// nt*64..+63 (rows of the expert-grouped buffer).
 // A rows 0..63 = W_gate rows, 64..127 = W_up rows of the same hidden units.
 // ---------------------------------------------------------------------------
 struct P_EGU : ProblemBase {
@@ -350,7 +351,8 @@ struct P_EGU : ProblemBase {
 };
 
 // ---------------------------------------------------------------------------
-// Routed experts, down projection.  Tile (e, m, nt): output features m*128..+127
+// Routed experts, down projection (the second tile kind of P_EXP below).
+// Tile (e, m, nt): output features m*128..+127
 // of expert e for its grouped rows nt*64..+63; each row scaled by its gate weight.
 // ---------------------------------------------------------------------------
 struct P_ED : ProblemBase {
@@ -407,6 +409,76 @@ struct P_ED : ProblemBase {
         }
       }
     }
+  }
+};
+
+// ---------------------------------------------------------------------------
+// Routed experts, gate|up + SwiGLU and down projection in one persistent
+// launch: the tile queue holds every gate|up tile (in expert order) and then
+// every down tile (in expert order).  A down tile reads the SwiGLU rows of one
+// token tile of its expert, which that token tile's FJ gate|up tiles write;
+// each of their epilogues adds one to ready[tt] (tt: the token tile's index
+// over all experts) once its rows are stored, and the producer of the down
+// tile waits for FJ before loading them.  All gate|up tiles come first in the
+// queue, so no wait depends on a tile not yet taken (see the engine header).
+// The down tiles of the first experts start while the last gate|up tiles
+// still run: no gate|up tail and down ramp between two launches.
+// ---------------------------------------------------------------------------
+struct P_EXP : ProblemBase {
+  static constexpr int BN = kExpertRows, STAGES = 4, KB = 2, B_STAGE = BN * 128, TMEM_COLS = 128;
+  static constexpr int EP_SMEM = P_EGU::EP_SMEM;
+  static constexpr bool DYNAMIC = true;
+  static constexpr bool ACQUIRE = true;
+  static_assert(P_EGU::BN == BN && P_ED::BN == BN && P_EGU::KB == KB && P_ED::KB == KB &&
+                    P_EGU::B_STAGE == B_STAGE && P_ED::B_STAGE == B_STAGE,
+                "gate|up and down tiles share the ring layout");
+  struct Params {
+    P_EGU::Params gu;
+    P_ED::Params dn;
+    int* ready;  // [token tiles] finished gate|up tiles per token tile (zeroed by the grouping kernel)
+    int FJ;      // gate|up tiles per token tile (fe / 64)
+    int* sched;  // tile counter (zeroed by the grouping kernel)
+    int* err;
+  };
+  DG_DEVINL static void prefetch(const Params& p) {
+    P_EGU::prefetch(p.gu);
+    P_ED::prefetch(p.dn);
+  }
+  DG_DEVINL static int num_tiles(const Params& p) { return *p.gu.n_tiles + *p.dn.n_tiles; }
+  DG_DEVINL static Tile tile(const Params& p, int v) {
+    const int ng = *p.gu.n_tiles;
+    Tile t;
+    if (v < ng) {
+      t = P_EGU::tile(p.gu, v);
+      t.e = 0;
+      t.f = p.gu.tiles[v].w;
+    } else {
+      t = P_ED::tile(p.dn, v - ng);
+      t.e = 1;
+      t.f = p.dn.tiles[v - ng].w;
+    }
+    return t;
+  }
+  DG_DEVINL static uint32_t tx_bytes(const Params&, const Tile&) { return kAStage + B_STAGE; }
+  DG_DEVINL static bool acquire(const Params& p, const Tile& t, volatile int* abort, int* err) {
+    return t.e == 0 || counter_wait_bounded(p.ready + t.f, p.FJ, abort, err);
+  }
+  DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
+    if (t.e == 0)
+      P_EGU::load(p.gu, t, kb, sa, sb, bar);
+    else
+      P_ED::load(p.dn, t, kb, sa, sb, bar);
+  }
+  DG_DEVINL static void epilogue(const Params& p, const Tile& t, uint32_t taddr, int q, int lane, int row,
+                                 uint8_t* ep) {
+    if (t.e != 0) {
+      P_ED::epilogue(p.dn, t, taddr, q, lane, row, ep);
+      return;
+    }
+    P_EGU::epilogue(p.gu, t, taddr, q, lane, row, ep);
+    counter_release_fence();   // this thread's SwiGLU rows are visible to the TMA loads of the down tiles
+    named_bar_sync(3, 128);    // ... every thread's
+    if (row == 0) atomicAdd(p.ready + t.f, 1);
   }
 };
 
@@ -1002,23 +1074,6 @@ cudaError_t run_wpart(const WpartArgs& a, cudaStream_t st) {
   return launch_gemm<P_WPART>(p, grid_for(p.MT * p.NT * p.S, a.num_sms), st);
 }
 
-cudaError_t run_experts_gate_up(const ExpertArgs& a, cudaStream_t st) {
-  P_EGU::Params g;
-  g.tmG = *a.tm_gate;
-  g.tmU = *a.tm_up;
-  g.tmX = *a.tm_xp;
-  g.nk = a.d / 64;
-  g.fe = a.fe;
-  g.tiles = a.egu_tiles;
-  g.n_tiles = a.egu_count;
-  g.counts = a.counts;
-  g.offsets = a.offsets;
-  g.hp = a.hp;
-  g.err = a.err;
-  g.sched = a.sched;
-  return launch_gemm<P_EGU>(g, a.num_sms, st);
-}
-
 cudaError_t run_experts_gate_up_fp8(const ExpertArgs& a, cudaStream_t st) {
   P_EGU8::Params g;
   g.tmG = *a.tm_gate;
@@ -1058,21 +1113,38 @@ cudaError_t run_experts_down_fp8(const ExpertArgs& a, cudaStream_t st) {
   return launch_gemm<P_ED8>(dn, a.num_sms, st);
 }
 
-cudaError_t run_experts_down(const ExpertArgs& a, cudaStream_t st) {
-  P_ED::Params dn;
-  dn.tmW = *a.tm_down;
-  dn.tmH = *a.tm_hp;
-  dn.nk = a.fe / 64;
-  dn.d = a.d;
-  dn.tiles = a.ed_tiles;
-  dn.n_tiles = a.ed_count;
-  dn.counts = a.counts;
-  dn.offsets = a.offsets;
-  dn.row_weight = a.row_weight;
-  dn.yp = a.yp;
-  dn.err = a.err;
-  dn.sched = a.sched + 1;
-  return launch_gemm<P_ED>(dn, a.num_sms, st);
+cudaError_t run_experts(const ExpertArgs& a, cudaStream_t st) {
+  if (a.ready == nullptr || a.sched == nullptr) return cudaErrorInvalidValue;
+  P_EXP::Params x;
+  x.gu.tmG = *a.tm_gate;
+  x.gu.tmU = *a.tm_up;
+  x.gu.tmX = *a.tm_xp;
+  x.gu.nk = a.d / 64;
+  x.gu.fe = a.fe;
+  x.gu.tiles = a.egu_tiles;
+  x.gu.n_tiles = a.egu_count;
+  x.gu.counts = a.counts;
+  x.gu.offsets = a.offsets;
+  x.gu.hp = a.hp;
+  x.gu.err = a.err;
+  x.gu.sched = a.sched;
+  x.dn.tmW = *a.tm_down;
+  x.dn.tmH = *a.tm_hp;
+  x.dn.nk = a.fe / 64;
+  x.dn.d = a.d;
+  x.dn.tiles = a.ed_tiles;
+  x.dn.n_tiles = a.ed_count;
+  x.dn.counts = a.counts;
+  x.dn.offsets = a.offsets;
+  x.dn.row_weight = a.row_weight;
+  x.dn.yp = a.yp;
+  x.dn.err = a.err;
+  x.dn.sched = a.sched;
+  x.ready = a.ready;
+  x.FJ = a.fe / 64;
+  x.sched = a.sched;
+  x.err = a.err;
+  return launch_gemm<P_EXP>(x, a.num_sms, st);
 }
 
 cudaError_t run_shared_gate_up(const SharedArgs& a, cudaStream_t st) {
@@ -1134,6 +1206,7 @@ size_t gemm_smem_bytes_max() {
   m = m > GemmSmem<P_WPART>::total ? m : GemmSmem<P_WPART>::total;
   m = m > GemmSmem<P_EGU>::total ? m : GemmSmem<P_EGU>::total;
   m = m > GemmSmem<P_ED>::total ? m : GemmSmem<P_ED>::total;
+  m = m > GemmSmem<P_EXP>::total ? m : GemmSmem<P_EXP>::total;
   m = m > GemmSmem<P_SGU>::total ? m : GemmSmem<P_SGU>::total;
   m = m > GemmSmem<P_LM>::total ? m : GemmSmem<P_LM>::total;
   m = m > GemmSmem<P_EGU8>::total ? m : GemmSmem<P_EGU8>::total;

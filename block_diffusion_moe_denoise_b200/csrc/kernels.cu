@@ -526,18 +526,23 @@ __global__ void __launch_bounds__(512) k_group_gather(GroupArgs a, const unsigne
       const int n_nt = toff[e + 1] - toff[e];
       for (int i = lane; i < n_nt * (a.FJ + a.MD); i += 32) {
         const int nt = i / (a.FJ + a.MD), r = i % (a.FJ + a.MD);
+        // .w: the token tile's index over all experts (its readiness counter)
         if (r < a.FJ) {
           const int slot = (toff[e] + nt) * a.FJ + r;
-          if (slot < a.egu_cap) a.egu_tiles[slot] = make_int4(e, r, nt, 0);
+          if (slot < a.egu_cap) a.egu_tiles[slot] = make_int4(e, r, nt, toff[e] + nt);
         } else {
           const int slot = (toff[e] + nt) * a.MD + (r - a.FJ);
-          if (slot < a.ed_cap) a.ed_tiles[slot] = make_int4(e, r - a.FJ, nt, 0);
+          if (slot < a.ed_cap) a.ed_tiles[slot] = make_int4(e, r - a.FJ, nt, toff[e] + nt);
         }
       }
     }
   }
   // the expert GEMMs that follow draw their tiles from these counters
   if (blockIdx.x == 0 && tid < 2 && a.sched != nullptr) a.sched[tid] = 0;
+  if (blockIdx.x == 0 && a.ready != nullptr) {
+    const int n_tt = min(toff[E], a.egu_cap / max(1, a.FJ));  // token tiles the lists can hold
+    for (int i = tid; i < n_tt; i += blockDim.x) a.ready[i] = 0;
+  }
   // clear the other mask buffer, sliced across CTAs
   for (int i = blockIdx.x * blockDim.x + tid; i < E * MW; i += gridDim.x * blockDim.x) mask_next[i] = 0u;
   // this CTA's pairs, one warp per pair

@@ -31,6 +31,13 @@
 // and the epilogue threads read in the same order, so a CTA that drew cheap
 // tiles simply takes more of them (the expert GEMMs, whose tiles differ in
 // cost and do not divide evenly over the SMs).
+//
+// Dependent tiles.  With ACQUIRE = true the producer calls P::acquire(p, t)
+// before loading a tile; it may wait (bounded) for data that earlier tiles of
+// the same launch write.  Every wait ends as long as the tiles it depends on
+// come earlier in the tile order: a dequeued tile is fully loaded before its
+// producer takes the next index, and the MMA and epilogue roles never wait on
+// the producer's later tiles.
 #pragma once
 
 #include "common.cuh"
@@ -41,7 +48,7 @@ struct Tile {
   int valid;
   int nk;     // k-blocks of 64
   int n_mma;  // MMA N (multiple of 16, <= BN)
-  int a, b, c, d, e;  // problem-specific coordinates
+  int a, b, c, d, e, f;  // problem-specific coordinates
 };
 
 constexpr int kAStage = 128 * 128;  // 128 rows x 128 bytes
@@ -147,6 +154,9 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
         if (v >= n_tiles) break;
         const Tile t = P::tile(p, v);
         if (!t.valid) continue;
+        // a tile whose operands another tile of this launch produces waits for them
+        if constexpr (P::ACQUIRE)
+          if (!P::acquire(p, t, abort_flag, err)) break;
         const uint32_t tx = P::tx_bytes(p, t);
         bool ok = true;
         for (int kb = 0; kb < t.nk; kb += P::KB) {
@@ -266,12 +276,15 @@ struct ProblemBase {
   static constexpr int KB = 1;            // k-blocks per ring stage
   static constexpr bool F8 = false;       // E4M3 operands (kind::f8f6f4): a k-block is 128 elements
   static constexpr bool DYNAMIC = false;  // tiles from the global counter p.sched (see above)
+  static constexpr bool ACQUIRE = false;  // acquire(): the producer waits before loading a tile
   template <class Params>
   DG_DEVINL static void epilogue_init(const Params&, int, uint8_t*) {}
   template <class Params>
   DG_DEVINL static void finish(const Params&, int, uint8_t*) {}
   template <class Params>
   DG_DEVINL static void epilogue_prefetch(const Params&, const Tile&, int) {}
+  template <class Params>
+  DG_DEVINL static bool acquire(const Params&, const Tile&, volatile int*, int*) { return true; }
   template <class Params>
   DG_DEVINL static void load_w(const Params&, const Tile&, int, uint32_t, uint32_t, uint64_t*) {}
   template <class Params>

@@ -97,9 +97,10 @@ int dg_debug_buffer(const dg_handle* h, const char* name, size_t* offset, size_t
  * stream around every launch of the pass, enable=0 stops, enable=-1 clears the
  * totals.  dg_profile_read (synchronising) returns the summed elapsed ms and
  * launch count of one class: "embed", "rmsnorm", "qkv", "attention", "oproj",
- * "group", "experts_gate_up", "experts_down", "shared_gate_up" (with the
- * router), "shared_down", "lm_head", "lm_combine", "sample", "selfcond",
- * "other". */
+ * "group", "experts" (the bf16 routed experts: gate|up, SwiGLU and down in one
+ * launch), "experts_gate_up" and "experts_down" (the two launches of the FP8
+ * experts), "shared_gate_up" (with the router), "shared_down", "lm_head",
+ * "lm_combine", "sample", "selfcond", "other". */
 int dg_profile(dg_handle* h, int enable);
 int dg_profile_read(dg_handle* h, const char* kernel, double* total_ms, int64_t* launches);
 
