@@ -245,7 +245,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
       for (int c0 = 0; c0 < D / 32; c0 += kGroup) {
         uint4 v[kGroup * 4];
 #pragma unroll
-        for (int i = 0; i < kGroup * 4; ++i) v[i] = valid ? src[c0 * 4 + i] : make_uint4(0, 0, 0, 0);
+        for (int i = 0; i < kGroup * 4; ++i) v[i] = valid ? __ldcg(src + c0 * 4 + i) : make_uint4(0, 0, 0, 0);
 #pragma unroll
         for (int c = 0; c < kGroup; ++c) {
           uint32_t r[16];
@@ -524,7 +524,7 @@ __global__ void k_attn_combine(const float* __restrict__ part_o, const float2* _
   const int n_split = splits.s[t / Tr];
   if (n_split == 1) return;  // written directly by the attention kernel
   float2 ml = make_float2(-INFINITY, 0.f);
-  if (lane < n_split) ml = part_ml[((size_t)lane * Hq + h) * q_T + t];
+  if (lane < n_split) ml = __ldcg(part_ml + ((size_t)lane * Hq + h) * q_T + t);
   float M = ml.y > 0.f ? ml.x : -INFINITY;
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
@@ -543,8 +543,8 @@ __global__ void k_attn_combine(const float* __restrict__ part_o, const float2* _
   for (int s = 0; s < kMaxSplits; ++s)
     if (s < n_split && wts[s] != 0.f) {
       const float4* src = reinterpret_cast<const float4*>(part_o + (((size_t)s * Hq + h) * q_T + t) * D + c);
-      va[s] = src[0];
-      vb[s] = src[1];
+      va[s] = __ldcg(src);
+      vb[s] = __ldcg(src + 1);
     }
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll

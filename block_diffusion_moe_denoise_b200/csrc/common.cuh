@@ -27,7 +27,13 @@ enum : int {
 // successor be scheduled (pdl_trigger) and then waits for the predecessor to
 // complete and its writes to be visible (pdl_wait) before touching anything
 // the predecessor produced.  Every CTA waits unconditionally, so completion
-// stays transitive along the stream.
+// stays transitive along the stream.  A kernel that starts early this way can
+// still find lines of a buffer in its SM's L1 that are older than what its
+// predecessors wrote there (measured: the residual norm, reading the shared
+// expert's output written by the routed-expert launch, picked up stale values
+// in about one canvas segment in four); CUDA-core kernels therefore read
+// data produced earlier in the pass with ld.global.cg (__ldcg, L2 only).  TMA
+// loads do not go through L1.
 DG_DEVINL void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 DG_DEVINL void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 

@@ -258,7 +258,7 @@ struct dg_handle {
   int egu_cap = 0, ed_cap = 0;
   long long kv_req_stride = 0, kv_layer_stride = 0;
   std::vector<LayerMaps> maps;
-  CUtensorMap tm_hn, tm_o, tm_u, tm_xp, tm_hp, tm_hs, tm_embed, tm_k, tm_vt;
+  CUtensorMap tm_hn, tm_o, tm_u, tm_xp, tm_hp, tm_hs, tm_hs64, tm_embed, tm_k, tm_vt;
   CUtensorMap tm_sc_gate, tm_sc_up, tm_sc_down, tm_hs_sc;  // self-conditioning MLP and its hidden rows
   CUtensorMap tm_xq, tm_hq;                                // FP8 experts: token and hidden codes
   long long cap_user = 0;  // capacity the caller asked for (cap is rounded up to 64)
@@ -550,7 +550,17 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
       LAUNCH(h, K_ED, 1, run_experts_down_fp8(ea, st));
     } else {
       ea.ready = h->B<int>("ready");
+      // the shared expert's down projection runs as tiles of the same launch,
+      // unsplit along K: one fp32 slice for the residual norm
+      ea.tm_sdown = &m.sdown;
+      ea.tm_hs64 = &h->tm_hs64;
+      ea.T = T;
+      ea.sd_K = c.ffn_shared;
+      ea.sd_part = part;
       LAUNCH(h, K_EXP, 1, run_experts(ea, st));
+      pending_k = k;
+      pending_parts = 1;
+      continue;
     }
 
     WpartArgs da;
@@ -746,6 +756,7 @@ int dg_init(const dg_config* cfg, const dg_weights* wts, int max_requests, int64
   ok = ok && make_map(&h->tm_xp, h->B<bf16>("xp"), d, rows, kExpertRows);
   ok = ok && make_map(&h->tm_hp, h->B<bf16>("hp"), c.ffn_expert, rows, kExpertRows);
   ok = ok && make_map(&h->tm_hs, h->B<bf16>("hs"), c.ffn_shared, h->Tcap, 256);
+  ok = ok && make_map(&h->tm_hs64, h->B<bf16>("hs"), c.ffn_shared, h->Tcap, kExpertRows);
   ok = ok && make_map(&h->tm_embed, h->embed, d, c.vocab, 256);
   {
     const long long kv_elems = (long long)max_requests * h->kv_req_stride;

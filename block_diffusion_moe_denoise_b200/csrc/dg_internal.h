@@ -92,6 +92,11 @@ struct ExpertArgs {
   const float *s_gate = nullptr, *s_up = nullptr, *s_down = nullptr, *s_x = nullptr, *s_h = nullptr;
   int* sched = nullptr;  // [2] tile counters of the gate|up and down launches (zeroed by the grouping kernel)
   int* ready = nullptr;  // [token tiles] per-token-tile gate|up completions of run_experts (zeroed likewise)
+  // run_experts only: the shared expert's down projection as extra tiles of the
+  // same launch (tm_sdown == nullptr: none), output [T][d] fp32 into sd_part
+  const CUtensorMap *tm_sdown = nullptr, *tm_hs64 = nullptr;
+  int T = 0, sd_K = 0;
+  float* sd_part = nullptr;
 };
 struct SharedArgs {
   const CUtensorMap *tm_u, *tm_gate, *tm_up, *tm_router;

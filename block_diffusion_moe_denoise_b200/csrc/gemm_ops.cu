@@ -413,9 +413,13 @@ struct P_ED : ProblemBase {
 };
 
 // ---------------------------------------------------------------------------
-// Routed experts, gate|up + SwiGLU and down projection in one persistent
-// launch: the tile queue holds every gate|up tile (in expert order) and then
-// every down tile (in expert order).  A down tile reads the SwiGLU rows of one
+// Routed experts, gate|up + SwiGLU and down projection, and the shared
+// expert's down projection, in one persistent launch.  The tile queue holds
+// every gate|up tile (in expert order), then the shared-down tiles (128
+// output features x 64 tokens over the whole shared hidden width, written
+// straight to the fp32 partial the residual norm adds), then every down tile
+// (in expert order): CTAs that finish gate|up work take shared-down tiles
+// while the first down tiles' inputs are completed.  A down tile reads the SwiGLU rows of one
 // token tile of its expert, which that token tile's FJ gate|up tiles write;
 // each of their epilogues adds one to ready[tt] (tt: the token tile's index
 // over all experts) once its rows are stored, and the producer of the down
@@ -435,6 +439,11 @@ struct P_EXP : ProblemBase {
   struct Params {
     P_EGU::Params gu;
     P_ED::Params dn;
+    CUtensorMap tmSW;  // shared-expert down weights [d, fs], 128-row boxes
+    CUtensorMap tmHS;  // shared SwiGLU rows [Tcap, fs], 64-row boxes
+    int n_sd;          // shared-down tiles: (d / 128) x ceil(T / 64), 0 = none
+    int sd_nk, sd_fb, T, d;
+    float* part;       // [Tcap][d] shared-expert output (fp32)
     int* ready;  // [token tiles] finished gate|up tiles per token tile (zeroed by the grouping kernel)
     int FJ;      // gate|up tiles per token tile (fe / 64)
     int* sched;  // tile counter (zeroed by the grouping kernel)
@@ -443,8 +452,13 @@ struct P_EXP : ProblemBase {
   DG_DEVINL static void prefetch(const Params& p) {
     P_EGU::prefetch(p.gu);
     P_ED::prefetch(p.dn);
+    if (p.n_sd > 0) {
+      tma_prefetch_desc(&p.tmSW);
+      tma_prefetch_desc(&p.tmHS);
+    }
   }
-  DG_DEVINL static int num_tiles(const Params& p) { return *p.gu.n_tiles + *p.dn.n_tiles; }
+  DG_DEVINL static int num_tiles(const Params& p) { return *p.gu.n_tiles + p.n_sd + *p.dn.n_tiles; }
+  // kinds: e = 0 gate|up, 1 down, 2 shared down
   DG_DEVINL static Tile tile(const Params& p, int v) {
     const int ng = *p.gu.n_tiles;
     Tile t;
@@ -452,27 +466,53 @@ struct P_EXP : ProblemBase {
       t = P_EGU::tile(p.gu, v);
       t.e = 0;
       t.f = p.gu.tiles[v].w;
+    } else if (v < ng + p.n_sd) {
+      const int u = v - ng;
+      t.a = u % p.sd_fb;  // 128-feature block
+      t.b = u / p.sd_fb;  // 64-token tile
+      t.c = min(BN, p.T - t.b * BN);
+      t.valid = t.c > 0;
+      t.d = 0;
+      t.e = 2;
+      t.f = 0;
+      t.nk = p.sd_nk;
+      t.n_mma = round_up16(t.c);
     } else {
-      t = P_ED::tile(p.dn, v - ng);
+      t = P_ED::tile(p.dn, v - ng - p.n_sd);
       t.e = 1;
-      t.f = p.dn.tiles[v - ng].w;
+      t.f = p.dn.tiles[v - ng - p.n_sd].w;
     }
     return t;
   }
   DG_DEVINL static uint32_t tx_bytes(const Params&, const Tile&) { return kAStage + B_STAGE; }
   DG_DEVINL static bool acquire(const Params& p, const Tile& t, volatile int* abort, int* err) {
-    return t.e == 0 || counter_wait_bounded(p.ready + t.f, p.FJ, abort, err);
+    return t.e != 1 || counter_wait_bounded(p.ready + t.f, p.FJ, abort, err);
   }
   DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
-    if (t.e == 0)
+    if (t.e == 0) {
       P_EGU::load(p.gu, t, kb, sa, sb, bar);
-    else
+    } else if (t.e == 1) {
       P_ED::load(p.dn, t, kb, sa, sb, bar);
+    } else {
+      tma_load_2d(sa, &p.tmSW, kb * 64, t.a * 128, bar);
+      tma_load_2d(sb, &p.tmHS, kb * 64, t.b * BN, bar);
+    }
   }
   DG_DEVINL static void epilogue(const Params& p, const Tile& t, uint32_t taddr, int q, int lane, int row,
                                  uint8_t* ep) {
-    if (t.e != 0) {
+    if (t.e == 1) {
       P_ED::epilogue(p.dn, t, taddr, q, lane, row, ep);
+      return;
+    }
+    if (t.e == 2) {  // thread = output feature, columns = tokens
+      float* dst = p.part + t.a * 128 + row;
+      for (int c0 = 0; c0 < t.n_mma; c0 += 16) {
+        float v[16];
+        tmem_ld16(taddr + c0, v);
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (c0 + j < t.c) dst[(size_t)(t.b * BN + c0 + j) * p.d] = v[j];
+      }
       return;
     }
     P_EGU::epilogue(p.gu, t, taddr, q, lane, row, ep);
@@ -1140,6 +1180,22 @@ cudaError_t run_experts(const ExpertArgs& a, cudaStream_t st) {
   x.dn.yp = a.yp;
   x.dn.err = a.err;
   x.dn.sched = a.sched;
+  x.n_sd = 0;
+  x.sd_nk = x.sd_fb = 0;
+  x.T = a.T;
+  x.d = a.d;
+  x.part = a.sd_part;
+  if (a.tm_sdown != nullptr) {  // the shared expert's down projection rides along
+    if (a.sd_K % 64 != 0 || a.d % 128 != 0 || a.T < 1 || a.sd_part == nullptr) return cudaErrorInvalidValue;
+    x.tmSW = *a.tm_sdown;
+    x.tmHS = *a.tm_hs64;
+    x.sd_fb = a.d / 128;
+    x.sd_nk = a.sd_K / 64;
+    x.n_sd = x.sd_fb * ((a.T + P_EXP::BN - 1) / P_EXP::BN);
+  } else {
+    x.tmSW = *a.tm_down;  // unused
+    x.tmHS = *a.tm_hp;
+  }
   x.ready = a.ready;
   x.FJ = a.fe / 64;
   x.sched = a.sched;

@@ -85,7 +85,7 @@ __global__ void k_rmsnorm(const float* __restrict__ x, const float* __restrict__
   const float4* xr = reinterpret_cast<const float4*>(x + (size_t)row * d);
   float ss = 0.f;
   for (int c = lane; c < d / 4; c += 32) {
-    const float4 v = xr[c];
+    const float4 v = __ldcg(xr + c);
     ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
   }
   ss = warp_sum(ss);
@@ -93,7 +93,7 @@ __global__ void k_rmsnorm(const float* __restrict__ x, const float* __restrict__
   const float4* g4 = reinterpret_cast<const float4*>(g);
   uint2* o = reinterpret_cast<uint2*>(out + (size_t)row * d);
   for (int c = lane; c < d / 4; c += 32) {
-    const float4 v = xr[c];
+    const float4 v = __ldcg(xr + c);
     const float4 w = g4[c];
     o[c] = make_uint2(pack_bf16x2(v.x * rs * w.x, v.y * rs * w.y), pack_bf16x2(v.z * rs * w.z, v.w * rs * w.w));
   }
@@ -132,19 +132,19 @@ __global__ void __launch_bounds__(512) k_residual_norm(float* __restrict__ x, co
   float4* xr = reinterpret_cast<float4*>(x + (size_t)t * d);
   int rows[8];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) rows[j] = j < k ? pair_row[(size_t)t * k + j] : 0;
+  for (int j = 0; j < 8; ++j) rows[j] = j < k ? __ldcg(pair_row + (size_t)t * k + j) : 0;
   float4 v[2];
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    v[h] = xr[c + h];
+    v[h] = __ldcg(xr + c + h);
     uint2 y[8];  // 4 bf16
     float4 q[kMaxPartSplits];
 #pragma unroll
     for (int j = 0; j < 8; ++j)
-      if (j < k) y[j] = reinterpret_cast<const uint2*>(yp + (size_t)rows[j] * d)[c + h];
+      if (j < k) y[j] = __ldcg(reinterpret_cast<const uint2*>(yp + (size_t)rows[j] * d) + c + h);
 #pragma unroll
     for (int j = 0; j < kMaxPartSplits; ++j)
-      if (j < n_part) q[j] = reinterpret_cast<const float4*>(part + j * part_stride + (size_t)t * d)[c + h];
+      if (j < n_part) q[j] = __ldcg(reinterpret_cast<const float4*>(part + j * part_stride + (size_t)t * d) + c + h);
 #pragma unroll
     for (int j = 0; j < 8; ++j)
       if (j < k) {
@@ -475,7 +475,7 @@ __global__ void __launch_bounds__(512) k_group_gather(GroupArgs a, const unsigne
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   for (int e = tid; e < E; e += blockDim.x) {
     int c = 0;
-    for (int wi = 0; wi < used; ++wi) c += __popc(mask[(size_t)e * MW + wi]);
+    for (int wi = 0; wi < used; ++wi) c += __popc(__ldcg(mask + (size_t)e * MW + wi));
     cnt[e] = c;
   }
   __syncthreads();
@@ -549,14 +549,15 @@ __global__ void __launch_bounds__(512) k_group_gather(GroupArgs a, const unsigne
   const int per = (P + gridDim.x - 1) / gridDim.x;
   const int p0 = blockIdx.x * per, p1 = min(P, p0 + per);
   for (int p = p0 + warp; p < p1; p += blockDim.x >> 5) {
-    const int e = a.idx[p];
+    const int e = __ldcg(a.idx + p);
     const int t = p / k;
     int rank = 0;
     if (e >= 0 && e < E) {
       const unsigned* m = mask + (size_t)e * MW;
       const int wt = t >> 5;
       for (int wi = lane; wi <= wt; wi += 32) {
-        const unsigned bits = wi < wt ? m[wi] : (m[wi] & ((1u << (t & 31)) - 1u));
+        const unsigned mw = __ldcg(m + wi);
+        const unsigned bits = wi < wt ? mw : (mw & ((1u << (t & 31)) - 1u));
         rank += __popc(bits);
       }
       rank = warp_sum_int(rank);
@@ -565,7 +566,7 @@ __global__ void __launch_bounds__(512) k_group_gather(GroupArgs a, const unsigne
     if (lane == 0) {
       a.pair_row[p] = row;
       a.row_token[row] = t;
-      a.row_weight[row] = a.w[p];
+      a.row_weight[row] = __ldcg(a.w + p);
       a.row_pair[row] = p;
     }
     if constexpr (kF8) {  // FP8 experts: the row is quantised on the way (same codes for every copy)
@@ -580,7 +581,7 @@ __global__ void __launch_bounds__(512) k_group_gather(GroupArgs a, const unsigne
       uint4 r[12];
 #pragma unroll
       for (int b = 0; b < 12; ++b)
-        if (c0 + b * 32 < n16) r[b] = src[c0 + b * 32];
+        if (c0 + b * 32 < n16) r[b] = __ldcg(src + c0 + b * 32);
 #pragma unroll
       for (int b = 0; b < 12; ++b)
         if (c0 + b * 32 < n16) dst[c0 + b * 32] = r[b];
@@ -645,7 +646,7 @@ __global__ void k_lm_combine(const float4* __restrict__ part, int G, int MT, int
   const size_t stride = (size_t)MT * 128;
   LmPart r{-INFINITY, 0.f, 0.f, 0x7fffffff};
   for (int c = lane; c < G; c += 32) {
-    const float4 v = part[(size_t)c * stride + t];
+    const float4 v = __ldcg(part + (size_t)c * stride + t);
     if (v.y != v.y) atomicOr(err, DG_DEVERR_NAN);
     r = lm_merge(r, LmPart{v.x, v.y, v.z, __float_as_int(v.w)});
   }
