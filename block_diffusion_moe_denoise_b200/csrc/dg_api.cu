@@ -258,7 +258,7 @@ struct dg_handle {
   int egu_cap = 0, ed_cap = 0;
   long long kv_req_stride = 0, kv_layer_stride = 0;
   std::vector<LayerMaps> maps;
-  CUtensorMap tm_hn, tm_o, tm_u, tm_xp, tm_hp, tm_hs, tm_hs64, tm_embed, tm_k, tm_vt;
+  CUtensorMap tm_hn, tm_o, tm_u, tm_u64, tm_xp, tm_hp, tm_hs, tm_hs64, tm_embed, tm_k, tm_vt;
   CUtensorMap tm_sc_gate, tm_sc_up, tm_sc_down, tm_hs_sc;  // self-conditioning MLP and its hidden rows
   CUtensorMap tm_xq, tm_hq;                                // FP8 experts: token and hidden codes
   long long cap_user = 0;  // capacity the caller asked for (cap is rounded up to 64)
@@ -470,6 +470,7 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     // shared expert gate|up + router logits, top-k and token bitmasks
     SharedArgs sa;
     sa.tm_u = &h->tm_u;
+    sa.tm_u64 = &h->tm_u64;
     sa.tm_gate = &m.sgate;
     sa.tm_up = &m.sup;
     sa.tm_router = &m.router;
@@ -753,6 +754,7 @@ int dg_init(const dg_config* cfg, const dg_weights* wts, int max_requests, int64
   ok = ok && make_map(&h->tm_hn, h->B<bf16>("hn"), d, h->Tcap, 128);
   ok = ok && make_map(&h->tm_o, h->B<bf16>("o"), (long long)c.n_q_heads * D, h->Tcap, 256);
   ok = ok && make_map(&h->tm_u, h->B<bf16>("u"), d, h->Tcap, 128);
+  ok = ok && make_map(&h->tm_u64, h->B<bf16>("u"), d, h->Tcap, 64);
   ok = ok && make_map(&h->tm_xp, h->B<bf16>("xp"), d, rows, kExpertRows);
   ok = ok && make_map(&h->tm_hp, h->B<bf16>("hp"), c.ffn_expert, rows, kExpertRows);
   ok = ok && make_map(&h->tm_hs, h->B<bf16>("hs"), c.ffn_shared, h->Tcap, 256);

@@ -687,7 +687,9 @@ struct P_SGU : ProblemBase {
     CUtensorMap tmG;  // ws_gate [fs, d], 32-row boxes
     CUtensorMap tmU;  // ws_up [fs, d], 32-row boxes
     CUtensorMap tmR;  // w_router [E, d], E-row boxes
+    CUtensorMap tmX64;  // normed tokens, 64-row boxes (router tiles of 64 tokens)
     int T, nk, MT, FJ, fs, E, k, MW;
+    int RH;             // 1: a router tile covers 64 tokens (see router_tiles)
     __nv_bfloat16* hs;  // [Tcap, fs]
     float* logits;      // [Tcap, E]
     int* idx;           // [T, k]
@@ -702,8 +704,14 @@ struct P_SGU : ProblemBase {
     tma_prefetch_desc(&p.tmU);
     if (p.E > 0) tma_prefetch_desc(&p.tmR);
   }
-  // E == 0: a plain gated MLP (no router tile), as used for self-conditioning
-  DG_DEVINL static int router_tiles(const Params& p) { return p.E > 0 ? p.MT : 0; }
+  // E == 0: a plain gated MLP (no router tile), as used for self-conditioning.
+  // With RH a router tile takes 64 tokens (one 64-row box in the first half of
+  // the A stage; MMA rows 64..127 are ignored): it then streams 64 + E rows per
+  // k-block, no more than a shared tile's 128 + 2 * kHid, instead of 128 + E,
+  // so the router no longer outlasts the shared tiles.
+  DG_DEVINL static int router_tiles(const Params& p) {
+    return p.E > 0 ? (p.RH ? (p.T + 63) / 64 : p.MT) : 0;
+  }
   DG_DEVINL static int num_tiles(const Params& p) { return router_tiles(p) + p.MT * p.FJ; }
   DG_DEVINL static Tile tile(const Params& p, int v) {
     Tile t;
@@ -722,7 +730,7 @@ struct P_SGU : ProblemBase {
     return t;
   }
   DG_DEVINL static uint32_t tx_bytes(const Params& p, const Tile& t) {
-    return kAStage + (t.b < 0 ? p.E : 2 * kHid) * 128;
+    return (t.b < 0 && p.RH ? kAStage / 2 : kAStage) + (t.b < 0 ? p.E : 2 * kHid) * 128;
   }
   DG_DEVINL static void load_w(const Params& p, const Tile& t, int kb, uint32_t, uint32_t sb, uint64_t* bar) {
     if (t.b < 0) {
@@ -733,14 +741,17 @@ struct P_SGU : ProblemBase {
     }
   }
   DG_DEVINL static void load_x(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t, uint64_t* bar) {
-    tma_load_2d(sa, &p.tmX, kb * 64, t.a * 128, bar);
+    if (t.b < 0 && p.RH)
+      tma_load_2d(sa, &p.tmX64, kb * 64, t.a * 64, bar);
+    else
+      tma_load_2d(sa, &p.tmX, kb * 64, t.a * 128, bar);
   }
   DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
     load_x(p, t, kb, sa, sb, bar);
     load_w(p, t, kb, sa, sb, bar);
   }
-  DG_DEVINL static void router_epilogue(const Params& p, int tok, uint32_t taddr) {
-    const bool ok = tok < p.T;
+  DG_DEVINL static void router_epilogue(const Params& p, int tok, bool row_valid, uint32_t taddr) {
+    const bool ok = row_valid && tok < p.T;
     float tv[8];
     int ti[8];
 #pragma unroll
@@ -798,11 +809,14 @@ struct P_SGU : ProblemBase {
     }
   }
   DG_DEVINL static void epilogue(const Params& p, const Tile& t, uint32_t taddr, int, int, int row, uint8_t*) {
-    const int tok = t.a * 128 + row;
     if (t.b < 0) {
-      router_epilogue(p, tok, taddr);
+      if (p.RH)
+        router_epilogue(p, t.a * 64 + row, row < 64, taddr);
+      else
+        router_epilogue(p, t.a * 128 + row, true, taddr);
       return;
     }
+    const int tok = t.a * 128 + row;
     const bool ok = tok < p.T;
     for (int c0 = 0; c0 < kHid; c0 += 16) {
       float g[16], u[16];
@@ -1226,7 +1240,11 @@ cudaError_t run_shared_gate_up(const SharedArgs& a, cudaStream_t st) {
   g.w = a.w;
   g.mask = a.mask;
   g.err = a.err;
-  return launch_gemm<P_SGU>(g, grid_for(g.MT * (g.FJ + (a.E > 0 ? 1 : 0)), a.num_sms), st);
+  // router tiles of 64 tokens when they and the shared tiles still fit in one wave
+  g.RH = (a.E > 0 && a.tm_u64 != nullptr && (a.T + 63) / 64 + g.MT * g.FJ <= a.num_sms) ? 1 : 0;
+  g.tmX64 = g.RH ? *a.tm_u64 : *a.tm_u;
+  const int router = a.E > 0 ? (g.RH ? (a.T + 63) / 64 : g.MT) : 0;  // P_SGU::router_tiles
+  return launch_gemm<P_SGU>(g, grid_for(router + g.MT * g.FJ, a.num_sms), st);
 }
 
 cudaError_t run_lm_head(const LmArgs& a, int* grid_out, cudaStream_t st) {
