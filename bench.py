@@ -49,7 +49,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=8)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="generate", choices=["generate", "layer", "long"],
+    ap.add_argument("--workload", default="generate", choices=["generate", "layer", "long", "long_layer"],
                     help="generate: the headline (4096 in / 1024 out); layer: one full-shape layer; long: four "
                          "requests with 65536-token KV prefixes denoised together (one step over 1024 canvas tokens)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -158,13 +158,17 @@ def expert_gate_up_bytes(cfg, n_touched: float, T: int) -> float:
 
 
 def expert_bytes(cfg, n_touched: float, T: int) -> float:
-    """Bytes the fused bf16 routed-expert launch (gate|up, SwiGLU, down) must
-    move: all three weight matrices of every expert some token is routed to,
-    the grouped token rows read, the SwiGLU rows written and read back, the
-    gate-weighted outputs written (bf16)."""
+    """Bytes the fused bf16 expert launch must move: all three weight matrices
+    of every routed expert some token is routed to, the grouped token rows
+    read, the SwiGLU rows written and read back, the gate-weighted outputs
+    written (bf16); and for the shared expert's down projection riding in the
+    same launch its weights, its SwiGLU rows read (bf16) and its output
+    written (fp32)."""
     rows = T * cfg.top_k
     w = n_touched * 3 * cfg.ffn_expert * cfg.d_model * 2
-    return w + rows * cfg.d_model * 2 * 2 + rows * cfg.ffn_expert * 2 * 2
+    routed = w + rows * cfg.d_model * 2 * 2 + rows * cfg.ffn_expert * 2 * 2
+    shared = cfg.ffn_shared * cfg.d_model * 2 + T * cfg.ffn_shared * 2 + T * cfg.d_model * 4
+    return routed + shared
 
 
 def step_work(cfg, kv_len: int, T: int, n_touched: float, n_req: int = 1):
@@ -355,6 +359,13 @@ def workload_config(cfg, workload, world):
                "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                "l2": "inputs larger than L2: every step streams ~50 GB of weights and ~65 GB of KV"}
         return out
+    if workload == "long_layer":
+        return {"workload": ("long_layer: one decoder layer at full shape + LM head over 262144; 4 requests, each a "
+                             "65536-token synthetic KV prefix and its own 256-token canvas (the long-context step "
+                             "cut to one layer, for profiling)"),
+                "canvas": cfg.canvas, "kv_prefix": LONG_PREFIX, "batch": LONG_REQUESTS,
+                "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                "l2": "inputs larger than L2: ~2.2 GB of KV per step"}
     if workload == "layer":
         name = ("layer: one decoder layer at full shape + LM head over 262144, one denoising step, "
                 "4096-token synthetic KV prefix, 256-token canvas, batch 1")
@@ -389,15 +400,17 @@ def main():
     from synth import FULL, LAYER, make_kv_prefix, make_tokens, make_weights
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    cfg = LAYER if args.workload == "layer" else FULL
+    cfg = LAYER if args.workload in ("layer", "long_layer") else FULL
     cfg = cfg.with_(temperature=args.temperature, ffn_selfcond=args.selfcond,
                     expert_fp8=1 if args.fp8_experts else 0)
     hbm_gbs, bf16_tf, bf16_tf_sus, peak_kind = measured_peaks()
 
     w = make_weights(cfg, seed=0, device=dev)
     torch.cuda.synchronize()
-    n_req = LONG_REQUESTS if args.workload == "long" else 1
-    cap = {"generate": PROMPT + N_OUT, "layer": PROMPT + cfg.canvas, "long": LONG_PREFIX + cfg.canvas}[args.workload]
+    long_ctx = args.workload in ("long", "long_layer")
+    n_req = LONG_REQUESTS if long_ctx else 1
+    cap = {"generate": PROMPT + N_OUT, "layer": PROMPT + cfg.canvas, "long": LONG_PREFIX + cfg.canvas,
+           "long_layer": LONG_PREFIX + cfg.canvas}[args.workload]
     h = dgm.DG(cfg, w, max_requests=n_req, kv_capacity=cap, device=dev)
     st = h.stream
     prompt = make_tokens(cfg, PROMPT, seed=0)
@@ -432,7 +445,7 @@ def main():
             if record:
                 seg_steps.append((e0, e1))
                 steps_per.append(n)
-    elif args.workload == "long":
+    elif long_ctx:
         # four requests, each with its own synthetic committed prefix in every layer
         for r in range(n_req):
             for l in range(cfg.n_layers):
@@ -535,7 +548,7 @@ def main():
     total_prof = sum(v[0] for v in prof.values()) or 1.0
     kernels = {k: {"ms": round(v[0], 4), "launches": v[1], "share": round(v[0] / total_prof, 4)}
                for k, v in prof.items() if v[1] > 0}
-    kv_step = {"generate": PROMPT + 384, "layer": PROMPT, "long": LONG_PREFIX}[args.workload]
+    kv_step = {"generate": PROMPT + 384, "layer": PROMPT, "long": LONG_PREFIX, "long_layer": LONG_PREFIX}[args.workload]
     sbytes, sflops = step_work(cfg, kv_step, T, n_touched, n_req)
     t_roof_ms = max(sbytes / (hbm_gbs * 1e9), sflops / (bf16_tf * 1e12)) * 1e3
 
@@ -557,7 +570,7 @@ def main():
 
     cpu = None
     # the oracle sample is the headline workload's; the variants have none
-    variant = args.temperature > 0 or args.selfcond > 0 or args.fp8_experts or args.workload == "long"
+    variant = args.temperature > 0 or args.selfcond > 0 or args.fp8_experts or long_ctx
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not variant:
         if args.workload == "generate":
             # one whole 30-layer step of the oracle, measured once; a canvas is 12
@@ -580,15 +593,15 @@ def main():
                 "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s", "frac": achieved / hbm_gbs,
                 "traffic": traffic, "algorithmic_bytes_per_launch": egu_bytes,
                 "avg_launch_ms": egu_avg_ms, "peak_source": f"{peak_kind} HBM copy (MEASURED_PEAKS.json)"}
-    if args.workload == "long":
+    if long_ctx:
         # the dominant kernel of the long-context step is the canvas attention
-        # (k_attn_tc + its split-KV combine, timed together once per layer)
+        # (k_attn_tc, with its split-KV merge in-kernel, once per layer)
         at_ms, at_n = prof["attention"]
         at_layers = max(1, at_n)   # one profiled record per layer (attention + its combine)
         at_flops = n_req * attention_flops_per_layer(cfg, LONG_PREFIX, T)
         at_avg = at_ms / at_layers
         tf = at_flops / (at_avg * 1e-3) / 1e12
-        roofline = {"kernel": "attention (k_attn_tc + split-KV combine, per layer: 4 requests x 65792 keys)",
+        roofline = {"kernel": "attention (k_attn_tc, split-KV merge in its clusters, per layer: 4 requests x 65792 keys)",
                     "bound": "tensor", "achieved": tf, "peak": bf16_tf, "unit": "TFLOP/s", "frac": tf / bf16_tf,
                     "traffic": None, "algorithmic_flops_per_launch": at_flops, "avg_launch_ms": at_avg,
                     "peak_source": f"{peak_kind} bf16 dense burst (MEASURED_PEAKS.json)"}
