@@ -404,6 +404,9 @@ def main():
     cfg = cfg.with_(temperature=args.temperature, ffn_selfcond=args.selfcond,
                     expert_fp8=1 if args.fp8_experts else 0)
     hbm_gbs, bf16_tf, bf16_tf_sus, peak_kind = measured_peaks()
+    # a whole step, and a kernel timed inside it, run long enough to settle at the
+    # power-capped clock: the sustained bf16 figure is their tensor peak
+    bf16_tf_step = bf16_tf_sus or bf16_tf
 
     w = make_weights(cfg, seed=0, device=dev)
     torch.cuda.synchronize()
@@ -550,7 +553,7 @@ def main():
                for k, v in prof.items() if v[1] > 0}
     kv_step = {"generate": PROMPT + 384, "layer": PROMPT, "long": LONG_PREFIX, "long_layer": LONG_PREFIX}[args.workload]
     sbytes, sflops = step_work(cfg, kv_step, T, n_touched, n_req)
-    t_roof_ms = max(sbytes / (hbm_gbs * 1e9), sflops / (bf16_tf * 1e12)) * 1e3
+    t_roof_ms = max(sbytes / (hbm_gbs * 1e9), sflops / (bf16_tf_step * 1e12)) * 1e3
 
     e2e = None
     if args.workload == "generate" and not args.no_e2e:
@@ -602,9 +605,9 @@ def main():
         at_avg = at_ms / at_layers
         tf = at_flops / (at_avg * 1e-3) / 1e12
         roofline = {"kernel": "attention (k_attn_tc, split-KV merge in its clusters, per layer: 4 requests x 65792 keys)",
-                    "bound": "tensor", "achieved": tf, "peak": bf16_tf, "unit": "TFLOP/s", "frac": tf / bf16_tf,
+                    "bound": "tensor", "achieved": tf, "peak": bf16_tf_step, "unit": "TFLOP/s", "frac": tf / bf16_tf_step,
                     "traffic": None, "algorithmic_flops_per_launch": at_flops, "avg_launch_ms": at_avg,
-                    "peak_source": f"{peak_kind} bf16 dense burst (MEASURED_PEAKS.json)"}
+                    "peak_source": f"{peak_kind} bf16 dense sustained (MEASURED_PEAKS.json): a kernel inside a long step"}
     line = {
         "metric": METRIC,
         "value": value,
@@ -625,7 +628,7 @@ def main():
         "data": "synthetic (seeded N(0,0.02) bf16 weights, uniform token ids)",
         "config": workload_config(cfg, args.workload, world),
         "roofline": roofline,
-        "step_roofline": {"bytes": sbytes, "flops": sflops, "bound": "hbm" if sbytes / hbm_gbs > sflops / bf16_tf / 1e3
+        "step_roofline": {"bytes": sbytes, "flops": sflops, "bound": "hbm" if sbytes / hbm_gbs > sflops / bf16_tf_step / 1e3
                           else "tensor", "t_roof_ms": t_roof_ms, "frac": t_roof_ms / ms_denoise,
                           "experts_touched_per_layer": round(n_touched, 2)},
         "kernels": kernels,
