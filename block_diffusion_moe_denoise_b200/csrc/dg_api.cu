@@ -258,7 +258,7 @@ struct dg_handle {
   int egu_cap = 0, ed_cap = 0;
   long long kv_req_stride = 0, kv_layer_stride = 0;
   std::vector<LayerMaps> maps;
-  CUtensorMap tm_hn, tm_o, tm_u, tm_u64, tm_xp, tm_hp, tm_hs, tm_hs64, tm_embed, tm_k, tm_vt;
+  CUtensorMap tm_hn, tm_o, tm_o128, tm_u, tm_u64, tm_xp, tm_hp, tm_hs, tm_hs64, tm_embed, tm_k, tm_vt;
   CUtensorMap tm_sc_gate, tm_sc_up, tm_sc_down, tm_hs_sc;  // self-conditioning MLP and its hidden rows
   CUtensorMap tm_xq, tm_hq;                                // FP8 experts: token and hidden codes
   long long cap_user = 0;  // capacity the caller asked for (cap is rounded up to 64)
@@ -394,6 +394,7 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     qa.q = h->B<bf16>("q");
     qa.kv = kv_l;
     qa.err = err;
+    qa.pair = 1;  // M = 256 tiles over CTA pairs
     LAUNCH(h, K_QKV, 1, run_qkv(qa, st));
     if (qkv_only_last && l == c.n_layers - 1) break;
 
@@ -456,6 +457,7 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     oa.num_sms = h->num_sms;
     oa.part = part;
     oa.err = err;
+    oa.tm_x128 = &h->tm_o128;  // CTA pairs
     LAUNCH(h, K_OPROJ, 1, run_wpart(oa, st));
     // x += attention output projection; FFN RMSNorm -> bf16 rows u
     LAUNCH(h, K_RMSNORM, 1,
@@ -753,6 +755,7 @@ int dg_init(const dg_config* cfg, const dg_weights* wts, int max_requests, int64
   }
   ok = ok && make_map(&h->tm_hn, h->B<bf16>("hn"), d, h->Tcap, 128);
   ok = ok && make_map(&h->tm_o, h->B<bf16>("o"), (long long)c.n_q_heads * D, h->Tcap, 256);
+  ok = ok && make_map(&h->tm_o128, h->B<bf16>("o"), (long long)c.n_q_heads * D, h->Tcap, 128);
   ok = ok && make_map(&h->tm_u, h->B<bf16>("u"), d, h->Tcap, 128);
   ok = ok && make_map(&h->tm_u64, h->B<bf16>("u"), d, h->Tcap, 64);
   ok = ok && make_map(&h->tm_xp, h->B<bf16>("xp"), d, rows, kExpertRows);

@@ -65,6 +65,7 @@ struct QkvArgs {
   bf16* q;
   bf16* kv;
   int* err;
+  int pair = 0;  // 1: M = 256 tiles over CTA pairs (P_QKV2)
 };
 constexpr int kMaxPartSplits = 8;
 constexpr int kExpertRows = 64;  // token rows per routed-expert GEMM tile
@@ -74,6 +75,7 @@ struct WpartArgs {
   int T, Tcap, d, K, splits, num_sms;
   float* part;              // [splits][Tcap][d]
   int* err;
+  const CUtensorMap* tm_x128 = nullptr;  // the activations in 128-row boxes: CTA pairs (P_WPART2)
 };
 struct ExpertArgs {
   const CUtensorMap *tm_gate, *tm_up, *tm_xp, *tm_down, *tm_hp;

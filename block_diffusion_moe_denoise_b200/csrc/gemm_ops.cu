@@ -204,6 +204,47 @@ struct P_QKV : ProblemBase {
   }
 };
 
+// The QKV projection as M = 256 tiles over CTA pairs: a pair covers two token
+// tiles (256 tokens) against one 128-column tile of W_qkv; each CTA loads its
+// own 128 tokens and one of the column tile's two 64-row weight boxes, so the
+// token rows stream through each SM once per 128 columns instead of the
+// weight rows and token rows both (a quarter less traffic per SM).  The
+// epilogue (each CTA: its 128 tokens x 128 columns) is P_QKV's.
+struct P_QKV2 : P_QKV {
+  static constexpr bool PAIR = true;
+  // a CTA's B slot holds its 64 rows only: 48 KB per stage, four stages
+  static constexpr int STAGES = 4, B_STAGE = BN * 128 / 2;
+  DG_DEVINL static int num_tiles(const Params& p) { return ((p.MT + 1) / 2) * p.NT; }
+  DG_DEVINL static Tile tile(const Params& p, int v) {
+    Tile t;
+    t.valid = 1;
+    t.nk = p.nk;
+    t.n_mma = BN;
+    const int mt2 = (p.MT + 1) / 2;
+    t.a = v % mt2;  // pair of token tiles
+    t.b = v / mt2;  // 128-column tile of W_qkv
+    return t;
+  }
+  DG_DEVINL static Tile local(const Params&, Tile t, int rank) {
+    t.a = 2 * t.a + rank;  // this CTA's token tile
+    t.half = rank;         // and weight box
+    return t;
+  }
+  DG_DEVINL static uint32_t tx_bytes(const Params&, const Tile&) { return kAStage + B_STAGE; }
+  DG_DEVINL static void load_w(const Params& p, const Tile& t, int kb, uint32_t, uint32_t sb, uint64_t* bar) {
+    int kind, tb, r0, r1;
+    rows_of(p, t.b, kind, tb, r0, r1);
+    tma_load_2d_pair(sb, &p.tmB, kb * 64, t.half ? r1 : r0, bar);
+  }
+  DG_DEVINL static void load_x(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t, uint64_t* bar) {
+    tma_load_2d_pair(sa, &p.tmA, kb * 64, t.a * 128, bar);
+  }
+  DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
+    load_x(p, t, kb, sa, sb, bar);
+    load_w(p, t, kb, sa, sb, bar);
+  }
+};
+
 // ---------------------------------------------------------------------------
 // Split-K weight-row GEMM with fp32 partial output, shared by the output
 // projection and the shared expert's down projection:
@@ -264,6 +305,47 @@ struct P_WPART : ProblemBase {
         if (tok < p.T) dst[(size_t)tok * p.d] = v[j];
       }
     }
+  }
+};
+
+// P_WPART as M = 256 tiles over CTA pairs: a pair covers two 128-feature tiles
+// against one 256-token tile (one K slice); each CTA loads its own 128 weight
+// rows and half of the tokens (128 rows), a third less traffic per SM than a
+// single-CTA tile.  Each CTA's accumulator is its 128 features x all 256
+// tokens, so the epilogue is P_WPART's.  Needs an even number of feature tiles.
+struct P_WPART2 : P_WPART {
+  static constexpr bool PAIR = true;
+  static constexpr int STAGES = 6, B_STAGE = BN * 128 / 2;  // 32 KB per stage and CTA
+  DG_DEVINL static int num_tiles(const Params& p) { return (p.MT / 2) * p.NT * p.S; }
+  DG_DEVINL static Tile tile(const Params& p, int v) {
+    Tile t;
+    const int mt2 = p.MT / 2;
+    t.a = v % mt2;  // pair of feature tiles
+    const int rest = v / mt2;
+    t.b = rest % p.NT;  // token tile
+    t.c = rest / p.NT;  // K slice
+    const int per = (p.nk + p.S - 1) / p.S;
+    t.d = t.c * per;
+    t.nk = min(per, p.nk - t.d);
+    t.valid = t.nk > 0;
+    t.n_mma = BN;  // the full token tile; columns past T are not stored
+    return t;
+  }
+  DG_DEVINL static Tile local(const Params&, Tile t, int rank) {
+    t.a = 2 * t.a + rank;  // this CTA's feature tile
+    t.half = rank;         // and half of the token tile
+    return t;
+  }
+  DG_DEVINL static uint32_t tx_bytes(const Params&, const Tile&) { return kAStage + B_STAGE; }
+  DG_DEVINL static void load_w(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t, uint64_t* bar) {
+    tma_load_2d_pair(sa, &p.tmA, (t.d + kb) * 64, t.a * 128, bar);
+  }
+  DG_DEVINL static void load_x(const Params& p, const Tile& t, int kb, uint32_t, uint32_t sb, uint64_t* bar) {
+    tma_load_2d_pair(sb, &p.tmB, (t.d + kb) * 64, t.b * BN + t.half * (BN / 2), bar);  // 128-row boxes
+  }
+  DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
+    load_w(p, t, kb, sa, sb, bar);
+    load_x(p, t, kb, sa, sb, bar);
   }
 };
 
@@ -1071,7 +1153,10 @@ static cudaError_t launch_gemm(const typename P::Params& p, int grid, cudaStream
     configured = true;
   }
   if (grid <= 0) return cudaSuccess;
-  return launch_pdl(k_umma_gemm<P>, dim3(grid), dim3(192), smem, st, p);
+  if constexpr (P::PAIR)  // grid = 2 x pairs, launched as clusters of two
+    return launch_pdl_cluster(k_umma_gemm<P>, dim3(grid), dim3(192), smem, st, dim3(2, 1, 1), p);
+  else
+    return launch_pdl(k_umma_gemm<P>, dim3(grid), dim3(192), smem, st, p);
 }
 
 static int grid_for(int tiles, int sms) { return tiles < sms ? tiles : sms; }
@@ -1096,6 +1181,7 @@ cudaError_t run_qkv(const QkvArgs& a, cudaStream_t st) {
   p.q = a.q;
   p.kv = a.kv;
   p.err = a.err;
+  if (a.pair) return launch_gemm<P_QKV2>(p, 2 * grid_for(((p.MT + 1) / 2) * p.NT, a.num_sms / 2), st);
   return launch_gemm<P_QKV>(p, grid_for(p.MT * p.NT, a.num_sms), st);
 }
 
@@ -1125,6 +1211,10 @@ cudaError_t run_wpart(const WpartArgs& a, cudaStream_t st) {
   p.d = a.d;
   p.part = a.part;
   p.err = a.err;
+  if (a.tm_x128 != nullptr && p.MT % 2 == 0) {  // CTA pairs (the activations in 128-row boxes)
+    p.tmB = *a.tm_x128;
+    return launch_gemm<P_WPART2>(p, 2 * grid_for((p.MT / 2) * p.NT * p.S, a.num_sms / 2), st);
+  }
   return launch_gemm<P_WPART>(p, grid_for(p.MT * p.NT * p.S, a.num_sms), st);
 }
 
@@ -1281,6 +1371,8 @@ size_t gemm_smem_bytes_max() {
   m = m > GemmSmem<P_EGU>::total ? m : GemmSmem<P_EGU>::total;
   m = m > GemmSmem<P_ED>::total ? m : GemmSmem<P_ED>::total;
   m = m > GemmSmem<P_EXP>::total ? m : GemmSmem<P_EXP>::total;
+  m = m > GemmSmem<P_QKV2>::total ? m : GemmSmem<P_QKV2>::total;
+  m = m > GemmSmem<P_WPART2>::total ? m : GemmSmem<P_WPART2>::total;
   m = m > GemmSmem<P_SGU>::total ? m : GemmSmem<P_SGU>::total;
   m = m > GemmSmem<P_LM>::total ? m : GemmSmem<P_LM>::total;
   m = m > GemmSmem<P_EGU8>::total ? m : GemmSmem<P_EGU8>::total;

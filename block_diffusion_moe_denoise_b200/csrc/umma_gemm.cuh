@@ -32,6 +32,15 @@
 // tiles simply takes more of them (the expert GEMMs, whose tiles differ in
 // cost and do not divide evenly over the SMs).
 //
+// CTA pairs.  With PAIR = true the grid is launched as clusters of two CTAs
+// and one tile is an M = 256 MMA tile (tcgen05 .cta_group::2): each CTA loads
+// half of A (its 128 rows) and half of B (N/2 rows) into its own ring, both
+// halves completing on the even CTA's full barrier; the even CTA alone issues
+// the MMAs, whose commits arrive on the empty and accumulator barriers of
+// both; each CTA's epilogue reads its own 128 accumulator rows and releases
+// the accumulator on the even CTA's barrier.  P::local(t, rank) turns a pair
+// tile into the CTA's half (its tile coordinates and t.half).
+//
 // Dependent tiles.  With ACQUIRE = true the producer calls P::acquire(p, t)
 // before loading a tile; it may wait (bounded) for data that earlier tiles of
 // the same launch write.  Every wait ends as long as the tiles it depends on
@@ -49,6 +58,7 @@ struct Tile {
   int nk;     // k-blocks of 64
   int n_mma;  // MMA N (multiple of 16, <= BN)
   int a, b, c, d, e, f;  // problem-specific coordinates
+  int half;              // PAIR problems: this CTA's rank in its pair (0 issues the MMAs)
 };
 
 constexpr int kAStage = 128 * 128;  // 128 rows x 128 bytes
@@ -70,6 +80,7 @@ struct GemmSmem {
 template <class P>
 __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ typename P::Params p) {
   static_assert(!(P::PRELOAD && P::DYNAMIC), "a preloaded first tile needs the static schedule");
+  static_assert(!(P::PAIR && (P::DYNAMIC || P::F8)), "CTA pairs: static schedule, bf16");
   using S = GemmSmem<P>;
   extern __shared__ uint8_t dyn_smem[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~(uintptr_t)1023);
@@ -89,6 +100,16 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
+  // PAIR: rank in the pair; tiles are dealt to pairs
+  const uint32_t rank = P::PAIR ? cluster_ctarank() : 0;
+  const int unit = P::PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int n_units = P::PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+  auto tile_of = [&](int v) {
+    Tile t = P::tile(p, v);
+    if constexpr (P::PAIR) t = P::local(p, t, (int)rank);
+    return t;
+  };
+
   if (threadIdx.x == 0) {
     for (int s = 0; s < P::STAGES; ++s) {
       mbar_init(&full[s], 1);
@@ -96,7 +117,7 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 128);
+      mbar_init(&tempty[a], P::PAIR ? 256 : 128);  // the epilogue threads (of both CTAs of a pair)
     }
     if constexpr (P::DYNAMIC)
       for (int r = 0; r < kSchedRing; ++r) {
@@ -108,9 +129,15 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
     fence_proxy_async_smem();
   }
   if (warp == 0 && lane == 0) P::prefetch(p);
-  if (warp == 1) tmem_alloc(tmem_slot, P::TMEM_COLS);
+  if (warp == 1) {
+    if constexpr (P::PAIR)
+      tmem_alloc_pair(tmem_slot, P::TMEM_COLS);
+    else
+      tmem_alloc(tmem_slot, P::TMEM_COLS);
+  }
   tc_fence_before();
   __syncthreads();
+  if constexpr (P::PAIR) cluster_sync_all();  // the partner's barriers exist before anything signals them
   tc_fence_after();
   pdl_trigger();
   const uint32_t tmem = *tmem_slot;
@@ -124,15 +151,16 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
       // weight stream starts while the predecessor drains.
       int pre = 0;  // stages of the first tile armed before the wait
       if constexpr (P::PRELOAD) {
-        if ((int)blockIdx.x < P::num_tiles(p)) {
-          const Tile t0 = P::tile(p, blockIdx.x);
+        if (unit < P::num_tiles(p)) {
+          const Tile t0 = tile_of(unit);
           if (t0.valid) {
             const int n_st = (t0.nk + P::KB - 1) / P::KB;
             pre = n_st < P::STAGES ? n_st : P::STAGES;
             for (int st = 0; st < pre; ++st) {
               const int kb = st * P::KB;
               const int nsub = t0.nk - kb < P::KB ? t0.nk - kb : P::KB;
-              mbar_arrive_expect_tx(&full[st], P::tx_bytes(p, t0) * (uint32_t)nsub);
+              if (rank == 0)  // a pair's even CTA expects both halves
+                mbar_arrive_expect_tx(&full[st], P::tx_bytes(p, t0) * (uint32_t)nsub * (P::PAIR ? 2u : 1u));
               for (int j = 0; j < nsub; ++j)
                 P::load_w(p, t0, kb + j, smem_u32(sA + st * S::a_stage + (size_t)j * kAStage),
                           smem_u32(sB + st * S::b_stage + (size_t)j * P::B_STAGE), &full[st]);
@@ -143,7 +171,7 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
       pdl_wait();
       const int n_tiles = P::num_tiles(p);
       uint32_t stage = 0, phase = 0;
-      for (int i = 0, v = blockIdx.x;; ++i, v += gridDim.x) {
+      for (int i = 0, v = unit;; ++i, v += n_units) {
         if constexpr (P::DYNAMIC) {
           const int slot = i % kSchedRing;
           if (!mbar_wait_bounded(&sched_empty[slot], ((i / kSchedRing) & 1) ^ 1, abort_flag, err)) break;
@@ -152,7 +180,7 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
           mbar_arrive(&sched_full[slot]);
         }
         if (v >= n_tiles) break;
-        const Tile t = P::tile(p, v);
+        const Tile t = tile_of(v);
         if (!t.valid) continue;
         // a tile whose operands another tile of this launch produces waits for them
         if constexpr (P::ACQUIRE)
@@ -170,7 +198,7 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
                         &full[stage]);
           } else {
             if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, err)) { ok = false; break; }
-            mbar_arrive_expect_tx(&full[stage], tx * (uint32_t)nsub);
+            if (rank == 0) mbar_arrive_expect_tx(&full[stage], tx * (uint32_t)nsub * (P::PAIR ? 2u : 1u));
             for (int j = 0; j < nsub; ++j)
               P::load(p, t, kb + j, smem_u32(sa + (size_t)j * kAStage), smem_u32(sb + (size_t)j * P::B_STAGE),
                       &full[stage]);
@@ -185,9 +213,9 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
   } else if (warp == 1) {
     pdl_wait();
     const int n_tiles = P::num_tiles(p);
-    if (lane == 0) {
+    if (lane == 0 && rank == 0) {  // a pair's odd CTA issues no MMAs
       uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
-      for (int i = 0, v = blockIdx.x;; ++i, v += gridDim.x) {
+      for (int i = 0, v = unit;; ++i, v += n_units) {
         if constexpr (P::DYNAMIC) {
           const int slot = i % kSchedRing;
           if (!mbar_wait_bounded(&sched_full[slot], (i / kSchedRing) & 1, abort_flag, err)) break;
@@ -195,13 +223,14 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
           mbar_arrive(&sched_empty[slot]);
         }
         if (v >= n_tiles) break;
-        const Tile t = P::tile(p, v);
+        const Tile t = tile_of(v);
         if (!t.valid) continue;
         if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1, abort_flag, err)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem + acc * P::BN;
+        constexpr uint32_t kM = P::PAIR ? 256 : 128;
         const uint32_t idesc =
-            P::F8 ? umma_idesc_e4m3(128, (uint32_t)t.n_mma) : umma_idesc_bf16(128, (uint32_t)t.n_mma);
+            P::F8 ? umma_idesc_e4m3(kM, (uint32_t)t.n_mma) : umma_idesc_bf16(kM, (uint32_t)t.n_mma);
         bool ok = true;
         for (int kb = 0; kb < t.nk; kb += P::KB) {
           const int nsub = t.nk - kb < P::KB ? t.nk - kb : P::KB;
@@ -218,16 +247,24 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
                 const uint64_t bd = umma_sdesc_k128(b0 + j * P::B_STAGE + 32 * k);
                 if constexpr (P::F8)
                   umma_e4m3(d_tmem, ad, bd, idesc, (kb | j | k) != 0 ? 1u : 0u);
+                else if constexpr (P::PAIR)
+                  umma_bf16_pair(d_tmem, ad, bd, idesc, (kb | j | k) != 0 ? 1u : 0u);
                 else
                   umma_bf16(d_tmem, ad, bd, idesc, (kb | j | k) != 0 ? 1u : 0u);
               }
             }
           }
-          umma_commit(&empty[stage]);
+          if constexpr (P::PAIR)
+            umma_commit_pair(&empty[stage]);
+          else
+            umma_commit(&empty[stage]);
           if (++stage == P::STAGES) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
-        umma_commit(&tfull[acc]);
+        if constexpr (P::PAIR)
+          umma_commit_pair(&tfull[acc]);
+        else
+          umma_commit(&tfull[acc]);
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1;
       }
@@ -239,7 +276,7 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
     const int row = q * 32 + lane;     // accumulator row (M index) owned by this thread
     P::epilogue_init(p, row, ep_smem);
     uint32_t acc = 0, acc_phase = 0;
-    for (int i = 0, v = blockIdx.x;; ++i, v += gridDim.x) {
+    for (int i = 0, v = unit;; ++i, v += n_units) {
       if constexpr (P::DYNAMIC) {
         const int slot = i % kSchedRing;
         if (!mbar_wait_bounded(&sched_full[slot], (i / kSchedRing) & 1, abort_flag, err)) break;
@@ -247,7 +284,7 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
         mbar_arrive(&sched_empty[slot]);
       }
       if (v >= n_tiles) break;
-      const Tile t = P::tile(p, v);
+      const Tile t = tile_of(v);
       if (!t.valid) continue;
       P::epilogue_prefetch(p, t, row);
       if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, err)) break;
@@ -255,7 +292,10 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
       const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + acc * P::BN;
       P::epilogue(p, t, taddr, q, lane, row, ep_smem);
       tc_fence_before();
-      mbar_arrive(&tempty[acc]);
+      if (rank == 0)
+        mbar_arrive(&tempty[acc]);
+      else
+        mbar_arrive_remote(&tempty[acc], 0);  // the pair's MMAs are issued from the even CTA
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1;
     }
@@ -265,8 +305,14 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
   __syncwarp();
   tc_fence_before();
   __syncthreads();
+  if constexpr (P::PAIR) cluster_sync_all();  // the partner is done with both CTAs' memory
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, P::TMEM_COLS);
+  if (warp == 1) {
+    if constexpr (P::PAIR)
+      tmem_dealloc_pair(tmem, P::TMEM_COLS);
+    else
+      tmem_dealloc(tmem, P::TMEM_COLS);
+  }
 }
 
 // Default no-op hooks for problems that need none.
@@ -277,6 +323,12 @@ struct ProblemBase {
   static constexpr bool F8 = false;       // E4M3 operands (kind::f8f6f4): a k-block is 128 elements
   static constexpr bool DYNAMIC = false;  // tiles from the global counter p.sched (see above)
   static constexpr bool ACQUIRE = false;  // acquire(): the producer waits before loading a tile
+  static constexpr bool PAIR = false;     // M = 256 tiles over a cluster of two CTAs (see above)
+  template <class Params>
+  DG_DEVINL static Tile local(const Params&, Tile t, int rank) {
+    t.half = rank;
+    return t;
+  }
   template <class Params>
   DG_DEVINL static void epilogue_init(const Params&, int, uint8_t*) {}
   template <class Params>
