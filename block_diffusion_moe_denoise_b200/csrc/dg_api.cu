@@ -258,7 +258,7 @@ struct dg_handle {
   int egu_cap = 0, ed_cap = 0;
   long long kv_req_stride = 0, kv_layer_stride = 0;
   std::vector<LayerMaps> maps;
-  CUtensorMap tm_hn, tm_o, tm_o128, tm_u, tm_u64, tm_xp, tm_hp, tm_hs, tm_hs64, tm_embed, tm_k, tm_vt;
+  CUtensorMap tm_hn, tm_o, tm_o128, tm_u, tm_u64, tm_xp, tm_hp, tm_hs, tm_hs64, tm_embed, tm_embed128, tm_k, tm_vt;
   CUtensorMap tm_sc_gate, tm_sc_up, tm_sc_down, tm_hs_sc;  // self-conditioning MLP and its hidden rows
   CUtensorMap tm_xq, tm_hq;                                // FP8 experts: token and hidden codes
   long long cap_user = 0;  // capacity the caller asked for (cap is rounded up to 64)
@@ -621,6 +621,7 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
       la.draw = draw ? h->B<float2>("draw") + (size_t)r0 * NV : nullptr;
       if (draw) la.keys = ck;
       la.sc_part = keep_sc ? h->B<float2>("sc_part") : nullptr;
+      la.tm_embed128 = &h->tm_embed128;  // CTA pairs (unless the self-conditioning lists are kept)
       float* stats = h->B<float>("stats") + (size_t)r0 * 4;
       int grid = 0;
       LAUNCH(h, K_LM, 1, run_lm_head(la, &grid, st));
@@ -763,6 +764,7 @@ int dg_init(const dg_config* cfg, const dg_weights* wts, int max_requests, int64
   ok = ok && make_map(&h->tm_hs, h->B<bf16>("hs"), c.ffn_shared, h->Tcap, 256);
   ok = ok && make_map(&h->tm_hs64, h->B<bf16>("hs"), c.ffn_shared, h->Tcap, kExpertRows);
   ok = ok && make_map(&h->tm_embed, h->embed, d, c.vocab, 256);
+  ok = ok && make_map(&h->tm_embed128, h->embed, d, c.vocab, 128);
   {
     const long long kv_elems = (long long)max_requests * h->kv_req_stride;
     // K in the tiled layout: rows of 64 dims, a tile of 64 keys = D rows

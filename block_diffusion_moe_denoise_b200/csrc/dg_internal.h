@@ -141,6 +141,7 @@ struct LmArgs {
   DrawKeys keys = {};
   float2* sc_part = nullptr; // self-conditioning: per-CTA top-8 logits [grid][T][8] (logit, id bits)
   int row0 = 0;              // first row of tm_x this launch reads (its rows are row0 .. row0+T-1)
+  const CUtensorMap* tm_embed128 = nullptr;  // the embedding in 128-row boxes: CTA pairs (P_LM2)
 };
 
 cudaError_t run_qkv(const QkvArgs& a, cudaStream_t st);

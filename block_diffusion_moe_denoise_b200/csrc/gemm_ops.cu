@@ -1140,6 +1140,44 @@ struct P_LM : ProblemBase {
   }
 };
 
+// The LM head as M = 256 tiles over CTA pairs: a pair covers two token tiles
+// against one 256-row vocabulary tile; each CTA loads its 128 tokens and 128
+// of the vocabulary rows, and its accumulator holds its tokens x all 256
+// vocabulary columns, so P_LM's epilogue and statistics apply unchanged (a CTA
+// sees one token tile, the other's partial stays empty).  Not with the
+// self-conditioning lists (they assume a CTA sees one fixed token tile).
+struct P_LM2 : P_LM {
+  static constexpr bool PAIR = true;
+  static constexpr int STAGES = 6, B_STAGE = BN * 128 / 2;  // 32 KB per stage and CTA
+  DG_DEVINL static int num_tiles(const Params& p) { return ((p.MT + 1) / 2) * p.NV; }
+  DG_DEVINL static Tile tile(const Params& p, int v) {
+    Tile t;
+    t.valid = 1;
+    t.nk = p.nk;
+    t.n_mma = BN;
+    const int mt2 = (p.MT + 1) / 2;
+    t.a = v % mt2;  // pair of token tiles
+    t.b = v / mt2;  // vocabulary tile
+    return t;
+  }
+  DG_DEVINL static Tile local(const Params&, Tile t, int rank) {
+    t.a = 2 * t.a + rank;
+    t.half = rank;
+    return t;
+  }
+  DG_DEVINL static uint32_t tx_bytes(const Params&, const Tile&) { return kAStage + B_STAGE; }
+  DG_DEVINL static void load_w(const Params& p, const Tile& t, int kb, uint32_t, uint32_t sb, uint64_t* bar) {
+    tma_load_2d_pair(sb, &p.tmE, kb * 64, t.b * 256 + t.half * 128, bar);  // 128-row boxes
+  }
+  DG_DEVINL static void load_x(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t, uint64_t* bar) {
+    tma_load_2d_pair(sa, &p.tmX, kb * 64, p.row0 + t.a * 128, bar);
+  }
+  DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
+    load_x(p, t, kb, sa, sb, bar);
+    load_w(p, t, kb, sa, sb, bar);
+  }
+};
+
 // ---------------------------------------------------------------------------
 // host launchers
 // ---------------------------------------------------------------------------
@@ -1358,6 +1396,13 @@ cudaError_t run_lm_head(const LmArgs& a, int* grid_out, cudaStream_t st) {
   if (p.MT > P_LM::MT_MAX || a.row0 < 0) return cudaErrorInvalidValue;
   if (p.draw != nullptr && (p.keys.canvas < 1 || (p.T + p.keys.canvas - 1) / p.keys.canvas > DG_MAX_REQUESTS))
     return cudaErrorInvalidValue;
+  if (a.tm_embed128 != nullptr && p.sc_part == nullptr) {  // CTA pairs
+    p.tmE = *a.tm_embed128;
+    const int grid = 2 * grid_for(((p.MT + 1) / 2) * p.NV, a.num_sms / 2);
+    if (grid < 2) return cudaErrorInvalidValue;
+    *grid_out = grid;
+    return launch_gemm<P_LM2>(p, grid, st);
+  }
   int grid = grid_for(p.MT * p.NV, a.num_sms);
   if (p.sc_part != nullptr) grid = grid / p.MT * p.MT;  // one token tile per CTA
   if (grid < 1) return cudaErrorInvalidValue;
@@ -1373,6 +1418,7 @@ size_t gemm_smem_bytes_max() {
   m = m > GemmSmem<P_EXP>::total ? m : GemmSmem<P_EXP>::total;
   m = m > GemmSmem<P_QKV2>::total ? m : GemmSmem<P_QKV2>::total;
   m = m > GemmSmem<P_WPART2>::total ? m : GemmSmem<P_WPART2>::total;
+  m = m > GemmSmem<P_LM2>::total ? m : GemmSmem<P_LM2>::total;
   m = m > GemmSmem<P_SGU>::total ? m : GemmSmem<P_SGU>::total;
   m = m > GemmSmem<P_LM>::total ? m : GemmSmem<P_LM>::total;
   m = m > GemmSmem<P_EGU8>::total ? m : GemmSmem<P_EGU8>::total;
