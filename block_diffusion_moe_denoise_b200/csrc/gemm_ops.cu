@@ -477,19 +477,39 @@ struct P_ED : ProblemBase {
     tma_load_2d(sa, &p.tmW, kb * 64, t.a * p.d + t.b * 128, bar);
     tma_load_2d(sb, &p.tmH, kb * 64, t.d, bar);
   }
-  DG_DEVINL static void epilogue(const Params& p, const Tile& t, uint32_t taddr, int, int, int row, uint8_t*) {
-    const int f = t.b * 128 + row;
+  // The accumulator (thread = output feature, columns = tokens) is transposed
+  // through shared memory 16 tokens at a time: staged fp32 as [token][128
+  // features], each warp then scales whole token rows by their gate weight and
+  // stores them as 256-byte row segments of yp (8 bytes per lane), instead of
+  // 2-byte stores per thread and token.
+  static constexpr int EP_SMEM = 16 * 128 * 4;
+  DG_DEVINL static void epilogue(const Params& p, const Tile& t, uint32_t taddr, int q, int lane, int row,
+                                 uint8_t* ep) {
+    float* stg = reinterpret_cast<float*>(ep);  // [16 tokens][128 features]
     for (int c0 = 0; c0 < t.n_mma; c0 += 16) {
+      float w[4];  // gate weights of the token rows this warp stores: c0 + q + 4 j
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int c = c0 + q + 4 * j;
+        w[j] = c < t.c ? __ldcg(p.row_weight + t.d + c) : 0.f;
+      }
       float v[16];
       tmem_ld16(taddr + c0, v);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int c = c0 + i;
+      for (int i = 0; i < 16; ++i) stg[i * 128 + row] = v[i];
+      named_bar_sync(1, 128);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int c = c0 + q + 4 * j;
         if (c < t.c) {
-          const int r = t.d + c;
-          p.yp[(size_t)r * p.d + f] = __float2bfloat16_rn(p.row_weight[r] * v[i]);
+          const float4 a = *reinterpret_cast<const float4*>(stg + (q + 4 * j) * 128 + 4 * lane);
+          uint2 o;
+          o.x = pack_bf16x2(w[j] * a.x, w[j] * a.y);
+          o.y = pack_bf16x2(w[j] * a.z, w[j] * a.w);
+          *reinterpret_cast<uint2*>(p.yp + (size_t)(t.d + c) * p.d + t.b * 128 + 4 * lane) = o;
         }
       }
+      named_bar_sync(1, 128);  // staging free for the next 16 tokens
     }
   }
 };
@@ -512,7 +532,7 @@ struct P_ED : ProblemBase {
 // ---------------------------------------------------------------------------
 struct P_EXP : ProblemBase {
   static constexpr int BN = kExpertRows, STAGES = 4, KB = 2, B_STAGE = BN * 128, TMEM_COLS = 128;
-  static constexpr int EP_SMEM = P_EGU::EP_SMEM;
+  static constexpr int EP_SMEM = P_EGU::EP_SMEM > P_ED::EP_SMEM ? P_EGU::EP_SMEM : P_ED::EP_SMEM;
   static constexpr bool DYNAMIC = true;
   static constexpr bool ACQUIRE = true;
   static_assert(P_EGU::BN == BN && P_ED::BN == BN && P_EGU::KB == KB && P_ED::KB == KB &&
@@ -1192,9 +1212,9 @@ static cudaError_t launch_gemm(const typename P::Params& p, int grid, cudaStream
   }
   if (grid <= 0) return cudaSuccess;
   if constexpr (P::PAIR)  // grid = 2 x pairs, launched as clusters of two
-    return launch_pdl_cluster(k_umma_gemm<P>, dim3(grid), dim3(192), smem, st, dim3(2, 1, 1), p);
+    return launch_pdl_cluster(k_umma_gemm<P>, dim3(grid), dim3(gemm_threads<P>()), smem, st, dim3(2, 1, 1), p);
   else
-    return launch_pdl(k_umma_gemm<P>, dim3(grid), dim3(192), smem, st, p);
+    return launch_pdl(k_umma_gemm<P>, dim3(grid), dim3(gemm_threads<P>()), smem, st, p);
 }
 
 static int grid_for(int tiles, int sms) { return tiles < sms ? tiles : sms; }

@@ -13,6 +13,7 @@
 //   warps 2..5          epilogue: tcgen05.ld of the accumulator rows they own
 //                       (warp w reads TMEM lanes 32*(w%4) .. +31) and the fused
 //                       problem-specific epilogue
+//   warp 6 (one lane)   DYNAMIC problems only: tile scheduler (see below)
 // The accumulator is double-buffered in TMEM (2 x BN columns) so the epilogue
 // of one tile overlaps the main loop of the next.  Tiles are assigned
 // statically (tile v to CTA v mod gridDim.x), so every role walks the same list.
@@ -26,11 +27,15 @@
 //
 // Tile scheduling.  By default tile v goes to CTA v mod gridDim.x.  A problem
 // with DYNAMIC = true instead hands out tiles from a global counter (p.sched,
-// zero at launch): the producer thread takes the next index with an atomic
-// add and publishes it through a small shared-memory ring that the MMA thread
-// and the epilogue threads read in the same order, so a CTA that drew cheap
-// tiles simply takes more of them (the expert GEMMs, whose tiles differ in
-// cost and do not divide evenly over the SMs).
+// zero at launch): a seventh warp (the scheduler, one lane) takes indices with
+// an atomic add, builds each tile's descriptor and publishes it through a
+// small shared-memory ring that the producer, the MMA thread and the epilogue
+// threads read in the same order, so a CTA that drew cheap tiles simply takes
+// more of them (the expert GEMMs, whose tiles differ in cost and do not divide
+// evenly over the SMs).  The atomic, the descriptor's dependent loads and any
+// dependency wait (below) take one to two microseconds of round trips to L2;
+// in a separate warp they overlap the producer's loads of the previous tile
+// instead of draining the ring between two short tiles.
 //
 // CTA pairs.  With PAIR = true the grid is launched as clusters of two CTAs
 // and one tile is an M = 256 MMA tile (tcgen05 .cta_group::2): each CTA loads
@@ -41,12 +46,15 @@
 // the accumulator on the even CTA's barrier.  P::local(t, rank) turns a pair
 // tile into the CTA's half (its tile coordinates and t.half).
 //
-// Dependent tiles.  With ACQUIRE = true the producer calls P::acquire(p, t)
-// before loading a tile; it may wait (bounded) for data that earlier tiles of
-// the same launch write.  Every wait ends as long as the tiles it depends on
-// come earlier in the tile order: a dequeued tile is fully loaded before its
-// producer takes the next index, and the MMA and epilogue roles never wait on
-// the producer's later tiles.
+// Dependent tiles.  With ACQUIRE = true P::acquire(p, t) runs before a tile is
+// loaded (in the scheduler, which then hands the tile on through the ring's
+// release/acquire barriers; in the producer with a static schedule); it may
+// wait (bounded) for data that earlier tiles of the same launch write.  Every wait ends as long as the tiles it depends on
+// come earlier in the tile order: a CTA processes its claimed tiles in claim
+// order and claims increasing indices, so every tile queued in front of a
+// tile X has a smaller index than X, and by induction over the index all of
+// them finish; the MMA and epilogue roles never wait on the producer's later
+// tiles.
 #pragma once
 
 #include "common.cuh"
@@ -62,7 +70,12 @@ struct Tile {
 };
 
 constexpr int kAStage = 128 * 128;  // 128 rows x 128 bytes
-constexpr int kSchedRing = 8;       // tile indices in flight between the roles (DYNAMIC)
+constexpr int kSchedRing = 3;       // tiles in flight between the scheduler and the other roles (DYNAMIC)
+
+// Threads of a block: producer, MMA and four epilogue warps, plus the scheduler
+// warp of DYNAMIC problems.
+template <class P>
+constexpr int gemm_threads() { return P::DYNAMIC ? 224 : 192; }
 
 template <class P>
 struct GemmSmem {
@@ -74,11 +87,11 @@ struct GemmSmem {
   static constexpr size_t ep_off = b_off + (size_t)kStages * b_stage;
   static constexpr size_t bar_off = (ep_off + P::EP_SMEM + 15) & ~(size_t)15;
   static constexpr size_t misc_off = bar_off + (2 * kStages + 4 + 2 * kSchedRing) * 8;
-  static constexpr size_t total = misc_off + 16 + 4 * kSchedRing + 1024;  // + alignment slack
+  static constexpr size_t total = misc_off + 16 + sizeof(Tile) * kSchedRing + 1024;  // + alignment slack
 };
 
 template <class P>
-__global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ typename P::Params p) {
+__global__ void __launch_bounds__(224, 1) k_umma_gemm(const __grid_constant__ typename P::Params p) {
   static_assert(!(P::PRELOAD && P::DYNAMIC), "a preloaded first tile needs the static schedule");
   static_assert(!(P::PAIR && (P::DYNAMIC || P::F8)), "CTA pairs: static schedule, bf16");
   using S = GemmSmem<P>;
@@ -95,7 +108,8 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
   uint64_t* sched_empty = sched_full + kSchedRing;   // [kSchedRing]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + S::misc_off);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base + S::misc_off + 4);
-  volatile int* sched_tile = reinterpret_cast<volatile int*>(base + S::misc_off + 16);  // [kSchedRing]
+  Tile* sched_tile = reinterpret_cast<Tile*>(base + S::misc_off + 16);  // [kSchedRing], DYNAMIC only;
+                                                                         // valid < 0 ends the list
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -122,7 +136,7 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
     if constexpr (P::DYNAMIC)
       for (int r = 0; r < kSchedRing; ++r) {
         mbar_init(&sched_full[r], 1);
-        mbar_init(&sched_empty[r], 129);  // the MMA thread and the 128 epilogue threads
+        mbar_init(&sched_empty[r], 130);  // the producer, the MMA thread and the 128 epilogue threads
       }
     *abort_flag = 0;
     fence_barrier_init();
@@ -172,19 +186,21 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
       const int n_tiles = P::num_tiles(p);
       uint32_t stage = 0, phase = 0;
       for (int i = 0, v = unit;; ++i, v += n_units) {
-        if constexpr (P::DYNAMIC) {
+        Tile t;
+        if constexpr (P::DYNAMIC) {  // descriptor (dependencies already met) from the scheduler
           const int slot = i % kSchedRing;
-          if (!mbar_wait_bounded(&sched_empty[slot], ((i / kSchedRing) & 1) ^ 1, abort_flag, err)) break;
-          v = atomicAdd(p.sched, 1);
-          sched_tile[slot] = v;
-          mbar_arrive(&sched_full[slot]);
+          if (!mbar_wait_bounded(&sched_full[slot], (i / kSchedRing) & 1, abort_flag, err)) break;
+          t = sched_tile[slot];
+          mbar_arrive(&sched_empty[slot]);
+          if (t.valid < 0) break;
+        } else {
+          if (v >= n_tiles) break;
+          t = tile_of(v);
+          // a tile whose operands another tile of this launch produces waits for them
+          if constexpr (P::ACQUIRE)
+            if (t.valid && !P::acquire(p, t, abort_flag, err)) break;
         }
-        if (v >= n_tiles) break;
-        const Tile t = tile_of(v);
         if (!t.valid) continue;
-        // a tile whose operands another tile of this launch produces waits for them
-        if constexpr (P::ACQUIRE)
-          if (!P::acquire(p, t, abort_flag, err)) break;
         const uint32_t tx = P::tx_bytes(p, t);
         bool ok = true;
         for (int kb = 0; kb < t.nk; kb += P::KB) {
@@ -216,14 +232,17 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
     if (lane == 0 && rank == 0) {  // a pair's odd CTA issues no MMAs
       uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
       for (int i = 0, v = unit;; ++i, v += n_units) {
+        Tile t;
         if constexpr (P::DYNAMIC) {
           const int slot = i % kSchedRing;
           if (!mbar_wait_bounded(&sched_full[slot], (i / kSchedRing) & 1, abort_flag, err)) break;
-          v = sched_tile[slot];
+          t = sched_tile[slot];
           mbar_arrive(&sched_empty[slot]);
+          if (t.valid < 0) break;
+        } else {
+          if (v >= n_tiles) break;
+          t = tile_of(v);
         }
-        if (v >= n_tiles) break;
-        const Tile t = tile_of(v);
         if (!t.valid) continue;
         if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1, abort_flag, err)) break;
         tc_fence_after();
@@ -269,7 +288,7 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
         if (acc == 0) acc_phase ^= 1;
       }
     }
-  } else {
+  } else if (warp < 6) {
     pdl_wait();
     const int n_tiles = P::num_tiles(p);
     const int q = warp & 3;            // TMEM lane quadrant of this warp
@@ -277,14 +296,17 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
     P::epilogue_init(p, row, ep_smem);
     uint32_t acc = 0, acc_phase = 0;
     for (int i = 0, v = unit;; ++i, v += n_units) {
+      Tile t;
       if constexpr (P::DYNAMIC) {
         const int slot = i % kSchedRing;
         if (!mbar_wait_bounded(&sched_full[slot], (i / kSchedRing) & 1, abort_flag, err)) break;
-        v = sched_tile[slot];
+        t = sched_tile[slot];
         mbar_arrive(&sched_empty[slot]);
+        if (t.valid < 0) break;
+      } else {
+        if (v >= n_tiles) break;
+        t = tile_of(v);
       }
-      if (v >= n_tiles) break;
-      const Tile t = tile_of(v);
       if (!t.valid) continue;
       P::epilogue_prefetch(p, t, row);
       if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, err)) break;
@@ -300,6 +322,29 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ ty
       if (acc == 0) acc_phase ^= 1;
     }
     P::finish(p, row, ep_smem);
+  } else {
+    // scheduler (DYNAMIC only): claim, describe, wait for dependencies, publish
+    pdl_wait();
+    if constexpr (P::DYNAMIC) {
+      if (lane == 0) {
+        const int n_tiles = P::num_tiles(p);
+        for (int i = 0;; ++i) {
+          const int slot = i % kSchedRing;
+          if (!mbar_wait_bounded(&sched_empty[slot], ((i / kSchedRing) & 1) ^ 1, abort_flag, err)) break;
+          const int v = atomicAdd(p.sched, 1);
+          Tile t{};
+          t.valid = -1;
+          if (v < n_tiles) {
+            t = tile_of(v);
+            if constexpr (P::ACQUIRE)
+              if (t.valid && !P::acquire(p, t, abort_flag, err)) t.valid = -1;  // abort: end the list
+          }
+          sched_tile[slot] = t;
+          mbar_arrive(&sched_full[slot]);
+          if (t.valid < 0) break;
+        }
+      }
+    }
   }
 
   __syncwarp();
