@@ -182,6 +182,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
       if (warp == 0) {
         for (int j = 0; ok && j < n_tiles; ++j) ok = load_k(j);
       } else {
+        // the Q rows and the first K tiles go first: V(0) is needed only after S(0) and its softmax
+        ok = n_tiles == 0 || mbar_wait_bounded(q_ready, 0, abort_flag, err);
         for (int j = 0; ok && j < n_tiles; ++j) ok = load_v(j);
       }
     }
@@ -422,8 +424,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
     // of them, as O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s with M the
     // largest max, in split order, and writes them in bf16.
     cluster_sync_all();
-    if (warp >= 2 && warp <= 5) {
-      const int q = warp & 3;
+    {
       const int ns = gridDim.z;
       const int rp = (kAQ + ns - 1) / ns;
       const int i0 = (int)blockIdx.z * rp, i1 = min(kAQ, i0 + rp);
@@ -433,8 +434,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
       // tile's result does not depend on which of the two merges it took.
       float* wsm = reinterpret_cast<float*>(base + S::p_off);  // [kAQ][kMaxSplits + 1]
       bf16** osm = reinterpret_cast<bf16**>(base + S::p_off + kAQ * (kMaxSplits + 1) * 4);  // [kAQ]
-      const int row = q * 32 + lane;
-      if (row >= i0 && row < i1) {
+      const int row = (warp & 3) * 32 + lane;
+      if (warp >= 2 && warp <= 5 && row >= i0 && row < i1) {
         float2 ml[kMaxSplits];
 #pragma unroll
         for (int s2 = 0; s2 < kMaxSplits; ++s2)
@@ -458,11 +459,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
         const int hr = g * G + (qr < rows ? qr / a.Tr : 0), tr = slot * a.Tr + (qr < rows ? qr % a.Tr : 0);
         osm[row] = a.o + (size_t)tr * a.Hq * D + (size_t)hr * D;
       }
-      named_bar_sync(1, 128);  // the four softmax warps
+      // the merge itself is bound by the latency of distributed-shared-memory
+      // loads: all eight warps take rows, doubling the loads in flight
+      __syncthreads();
       constexpr int nch = D / 4;   // 16-byte chunks of an fp32 row
       constexpr int kRows = 2;     // rows merged side by side (loads in flight)
+      constexpr int kWarps = kAttnThreads / 32;
 #pragma unroll 1
-      for (int ib = i0 + q; ib < i1; ib += 4 * kRows) {
+      for (int ib = i0 + warp; ib < i1; ib += kWarps * kRows) {
 #pragma unroll
         for (int c0 = 0; c0 < nch; c0 += 32) {
           const int c = c0 + lane;
@@ -470,7 +474,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
           float wr[kRows][kMaxSplits];
 #pragma unroll
           for (int rr = 0; rr < kRows; ++rr) {
-            const int i = ib + 4 * rr;
+            const int i = ib + kWarps * rr;
 #pragma unroll
             for (int s2 = 0; s2 < kMaxSplits; ++s2) {
               wr[rr][s2] = (i < i1 && r0 + i < rows) ? wsm[i * (kMaxSplits + 1) + s2] : 0.f;
@@ -481,7 +485,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
           }
 #pragma unroll
           for (int rr = 0; rr < kRows; ++rr) {
-            const int i = ib + 4 * rr;
+            const int i = ib + kWarps * rr;
             if (i >= i1 || r0 + i >= rows || c >= nch) continue;
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
