@@ -237,29 +237,48 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
     const bool valid = qr < rows;
     const int h = g * G + (valid ? qr / a.Tr : 0);
     const int t = slot * a.Tr + (valid ? qr % a.Tr : 0);
-    // Q row -> tensor memory lane `row`, bf16 pairs in columns kTmQ + [0, D/2)
+    // Q row -> tensor memory lane `row`, bf16 pairs in columns kTmQ + [0, D/2).
+    // The rows are read coalesced (kRW lanes per row, up to 256 bytes per row
+    // and instruction) and transposed through the P buffers (free until the
+    // first softmax) kRW 16-byte chunks per round: lane-per-row loads touched
+    // 32 sectors per instruction and were bound by the L2 request rate.
     {
-      // the row's loads go out in groups of 16 x 16 bytes (all in flight at
-      // once), then into tensor memory: two memory round trips for D = 256
-      const uint4* src = reinterpret_cast<const uint4*>(a.q + ((size_t)h * a.q_T + t) * D);
-      constexpr int kGroup = D / 32 < 4 ? D / 32 : 4;  // 16-column TMEM stores per group
+      constexpr int kNC = D / 8;                 // 16-byte chunks of a row
+      constexpr int kRW = kNC < 16 ? kNC : 16;   // chunks per round
+      constexpr int kRPI = 32 / kRW;             // rows per load instruction
+      static_assert(kRW % 4 == 0 && kNC % kRW == 0 && 4 * 32 * kRW * 16 <= 2 * S::kP, "Q staging");
+      const unsigned long long my_src =
+          valid ? reinterpret_cast<unsigned long long>(a.q + ((size_t)h * a.q_T + t) * D) : 0ull;
+      uint4* stq = reinterpret_cast<uint4*>(sP) + (size_t)q * 32 * kRW;  // this warp: [32 rows][kRW chunks]
+      const int cl = lane % kRW, rl = lane / kRW;
+#pragma unroll 1
+      for (int rd = 0; rd < kNC / kRW; ++rd) {
+        uint4 v[kRW];
 #pragma unroll
-      for (int c0 = 0; c0 < D / 32; c0 += kGroup) {
-        uint4 v[kGroup * 4];
+        for (int k = 0; k < kRW; ++k) {
+          const uint4* src = reinterpret_cast<const uint4*>(__shfl_sync(0xffffffffu, my_src, kRPI * k + rl));
+          v[k] = src != nullptr ? __ldcg(src + rd * kRW + cl) : make_uint4(0, 0, 0, 0);
+        }
 #pragma unroll
-        for (int i = 0; i < kGroup * 4; ++i) v[i] = valid ? __ldcg(src + c0 * 4 + i) : make_uint4(0, 0, 0, 0);
+        for (int k = 0; k < kRW; ++k) {
+          const int rk = kRPI * k + rl;
+          stq[rk * kRW + (cl ^ (rk % kRW))] = v[k];
+        }
+        __syncwarp();
 #pragma unroll
-        for (int c = 0; c < kGroup; ++c) {
+        for (int cg = 0; cg < kRW / 4; ++cg) {
           uint32_t r[16];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            r[4 * i] = v[c * 4 + i].x;
-            r[4 * i + 1] = v[c * 4 + i].y;
-            r[4 * i + 2] = v[c * 4 + i].z;
-            r[4 * i + 3] = v[c * 4 + i].w;
+          for (int u = 0; u < 4; ++u) {
+            const uint4 w = stq[lane * kRW + ((cg * 4 + u) ^ (lane % kRW))];
+            r[4 * u] = w.x;
+            r[4 * u + 1] = w.y;
+            r[4 * u + 2] = w.z;
+            r[4 * u + 3] = w.w;
           }
-          tmem_st16_raw(tm_q + lane_off + (c0 + c) * 16, r);
+          tmem_st16_raw(tm_q + lane_off + (rd * kRW + cg * 4) * 4, r);
         }
+        __syncwarp();
       }
       tmem_st_wait();
       tc_fence_before();
