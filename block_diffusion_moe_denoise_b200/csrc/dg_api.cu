@@ -759,8 +759,8 @@ int dg_init(const dg_config* cfg, const dg_weights* wts, int max_requests, int64
   ok = ok && make_map(&h->tm_o128, h->B<bf16>("o"), (long long)c.n_q_heads * D, h->Tcap, 128);
   ok = ok && make_map(&h->tm_u, h->B<bf16>("u"), d, h->Tcap, 128);
   ok = ok && make_map(&h->tm_u64, h->B<bf16>("u"), d, h->Tcap, 64);
-  ok = ok && make_map(&h->tm_xp, h->B<bf16>("xp"), d, rows, kExpertRows);
-  ok = ok && make_map(&h->tm_hp, h->B<bf16>("hp"), c.ffn_expert, rows, kExpertRows);
+  ok = ok && make_map(&h->tm_xp, h->B<bf16>("xp"), d, rows, kExpertBoxRows);
+  ok = ok && make_map(&h->tm_hp, h->B<bf16>("hp"), c.ffn_expert, rows, kExpertBoxRows);
   ok = ok && make_map(&h->tm_hs, h->B<bf16>("hs"), c.ffn_shared, h->Tcap, 256);
   ok = ok && make_map(&h->tm_hs64, h->B<bf16>("hs"), c.ffn_shared, h->Tcap, kExpertRows);
   ok = ok && make_map(&h->tm_embed, h->embed, d, c.vocab, 256);

@@ -68,7 +68,10 @@ struct QkvArgs {
   int pair = 0;  // 1: M = 256 tiles over CTA pairs (P_QKV2)
 };
 constexpr int kMaxPartSplits = 8;
-constexpr int kExpertRows = 64;  // token rows per routed-expert GEMM tile
+constexpr int kExpertRows = 64;       // token rows per FP8 routed-expert GEMM tile
+constexpr int kExpertTileRows = 128;  // token rows per bf16 routed-expert tile (and shared-down tile)
+constexpr int kExpertBoxRows = 64;    // rows per TMA box of the bf16 grouped rows (boxes of 16 rows,
+                                      // four times the copies, measured slower on B200)
 struct WpartArgs {
   const CUtensorMap* tm_w;  // weights [d, K], 128-row boxes
   const CUtensorMap* tm_x;  // activations [Tcap, K], 256-row boxes

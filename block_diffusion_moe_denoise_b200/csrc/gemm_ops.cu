@@ -352,18 +352,20 @@ struct P_WPART2 : P_WPART {
 // ---------------------------------------------------------------------------
 // Routed experts, gate|up + SwiGLU (the first tile kind of P_EXP below).
 // Tile (e, j, nt): hidden units j*64..+63 of expert e for its tokens
-// nt*64..+63 (rows of the expert-grouped buffer).
+// nt*128..+127 (rows of the expert-grouped buffer; the token rows are loaded
+// in 64-row boxes, one or two as the tile needs).  Tiles of 128 tokens read an
+// expert's weights once per 128 of its tokens.
 // A rows 0..63 = W_gate rows, 64..127 = W_up rows of the same hidden units.
 // ---------------------------------------------------------------------------
 struct P_EGU : ProblemBase {
-  static constexpr int BN = kExpertRows, STAGES = 4, KB = 2, B_STAGE = BN * 128, TMEM_COLS = 128;
+  static constexpr int BN = kExpertTileRows, STAGES = 3, KB = 2, B_STAGE = BN * 128, TMEM_COLS = 2 * BN;
   static constexpr int kXchBytes = 64 * 17 * 4;
   static constexpr int EP_SMEM = kXchBytes + BN * 64 * 2;
   static constexpr bool DYNAMIC = true;
   struct Params {
     CUtensorMap tmG;  // w_gate as [E*fe, d]
     CUtensorMap tmU;  // w_up   as [E*fe, d]
-    CUtensorMap tmX;  // expert-grouped tokens [rows_cap, d], 64-row boxes
+    CUtensorMap tmX;  // expert-grouped tokens [rows_cap, d], kExpertBoxRows-row boxes
     int nk, fe;
     const int4* tiles;
     const int* n_tiles;
@@ -393,12 +395,15 @@ struct P_EGU : ProblemBase {
     t.n_mma = round_up16(n_valid);
     return t;
   }
-  DG_DEVINL static uint32_t tx_bytes(const Params&, const Tile&) { return kAStage + B_STAGE; }
+  // the token rows in kExpertBoxRows-row boxes, as many as the tile needs
+  DG_DEVINL static uint32_t tx_bytes(const Params&, const Tile& t) {
+    return kAStage + (uint32_t)((t.n_mma + kExpertBoxRows - 1) / kExpertBoxRows) * kExpertBoxRows * 128;
+  }
   DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
     const int r = t.a * p.fe + t.b * 64;
     tma_load_2d(sa, &p.tmG, kb * 64, r, bar);
     tma_load_2d(sa + 64 * 128, &p.tmU, kb * 64, r, bar);
-    tma_load_2d(sb, &p.tmX, kb * 64, t.d, bar);
+    for (int i = 0; i < t.n_mma; i += kExpertBoxRows) tma_load_2d(sb + i * 128, &p.tmX, kb * 64, t.d + i, bar);
   }
   // The SwiGLU rows are transposed through shared memory: the 64 gate-row
   // threads each hold one hidden unit of 16 tokens per chunk; staged as
@@ -435,14 +440,14 @@ struct P_EGU : ProblemBase {
 // ---------------------------------------------------------------------------
 // Routed experts, down projection (the second tile kind of P_EXP below).
 // Tile (e, m, nt): output features m*128..+127
-// of expert e for its grouped rows nt*64..+63; each row scaled by its gate weight.
+// of expert e for its grouped rows nt*128..+127; each row scaled by its gate weight.
 // ---------------------------------------------------------------------------
 struct P_ED : ProblemBase {
-  static constexpr int BN = kExpertRows, STAGES = 4, KB = 2, B_STAGE = BN * 128, TMEM_COLS = 128;
+  static constexpr int BN = kExpertTileRows, STAGES = 3, KB = 2, B_STAGE = BN * 128, TMEM_COLS = 2 * BN;
   static constexpr bool DYNAMIC = true;
   struct Params {
     CUtensorMap tmW;  // w_down as [E*d, fe]
-    CUtensorMap tmH;  // hidden [rows_cap, fe], 64-row boxes
+    CUtensorMap tmH;  // hidden [rows_cap, fe], kExpertBoxRows-row boxes
     int nk, d;
     const int4* tiles;
     const int* n_tiles;
@@ -472,10 +477,12 @@ struct P_ED : ProblemBase {
     t.n_mma = round_up16(n_valid);
     return t;
   }
-  DG_DEVINL static uint32_t tx_bytes(const Params&, const Tile&) { return kAStage + B_STAGE; }
+  DG_DEVINL static uint32_t tx_bytes(const Params&, const Tile& t) {
+    return kAStage + (uint32_t)((t.n_mma + kExpertBoxRows - 1) / kExpertBoxRows) * kExpertBoxRows * 128;
+  }
   DG_DEVINL static void load(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t sb, uint64_t* bar) {
     tma_load_2d(sa, &p.tmW, kb * 64, t.a * p.d + t.b * 128, bar);
-    tma_load_2d(sb, &p.tmH, kb * 64, t.d, bar);
+    for (int i = 0; i < t.n_mma; i += kExpertBoxRows) tma_load_2d(sb + i * 128, &p.tmH, kb * 64, t.d + i, bar);
   }
   // The accumulator (thread = output feature, columns = tokens) is transposed
   // through shared memory 16 tokens at a time: staged fp32 as [token][128
@@ -518,7 +525,7 @@ struct P_ED : ProblemBase {
 // Routed experts, gate|up + SwiGLU and down projection, and the shared
 // expert's down projection, in one persistent launch.  The tile queue holds
 // every gate|up tile (in expert order), then the shared-down tiles (128
-// output features x 64 tokens over the whole shared hidden width, written
+// output features x 128 tokens over the whole shared hidden width, written
 // straight to the fp32 partial the residual norm adds), then every down tile
 // (in expert order): CTAs that finish gate|up work take shared-down tiles
 // while the first down tiles' inputs are completed.  A down tile reads the SwiGLU rows of one
@@ -531,7 +538,7 @@ struct P_ED : ProblemBase {
 // still run: no gate|up tail and down ramp between two launches.
 // ---------------------------------------------------------------------------
 struct P_EXP : ProblemBase {
-  static constexpr int BN = kExpertRows, STAGES = 4, KB = 2, B_STAGE = BN * 128, TMEM_COLS = 128;
+  static constexpr int BN = kExpertTileRows, STAGES = 3, KB = 2, B_STAGE = BN * 128, TMEM_COLS = 2 * BN;
   static constexpr int EP_SMEM = P_EGU::EP_SMEM > P_ED::EP_SMEM ? P_EGU::EP_SMEM : P_ED::EP_SMEM;
   static constexpr bool DYNAMIC = true;
   static constexpr bool ACQUIRE = true;
@@ -543,7 +550,7 @@ struct P_EXP : ProblemBase {
     P_ED::Params dn;
     CUtensorMap tmSW;  // shared-expert down weights [d, fs], 128-row boxes
     CUtensorMap tmHS;  // shared SwiGLU rows [Tcap, fs], 64-row boxes
-    int n_sd;          // shared-down tiles: (d / 128) x ceil(T / 64), 0 = none
+    int n_sd;          // shared-down tiles: (d / 128) x ceil(T / BN), 0 = none
     int sd_nk, sd_fb, T, d;
     float* part;       // [Tcap][d] shared-expert output (fp32)
     int* ready;  // [token tiles] finished gate|up tiles per token tile (zeroed by the grouping kernel)
@@ -571,7 +578,7 @@ struct P_EXP : ProblemBase {
     } else if (v < ng + p.n_sd) {
       const int u = v - ng;
       t.a = u % p.sd_fb;  // 128-feature block
-      t.b = u / p.sd_fb;  // 64-token tile
+      t.b = u / p.sd_fb;  // BN-token tile
       t.c = min(BN, p.T - t.b * BN);
       t.valid = t.c > 0;
       t.d = 0;
@@ -586,7 +593,11 @@ struct P_EXP : ProblemBase {
     }
     return t;
   }
-  DG_DEVINL static uint32_t tx_bytes(const Params&, const Tile&) { return kAStage + B_STAGE; }
+  DG_DEVINL static uint32_t tx_bytes(const Params& p, const Tile& t) {
+    if (t.e == 0) return P_EGU::tx_bytes(p.gu, t);
+    if (t.e == 1) return P_ED::tx_bytes(p.dn, t);
+    return kAStage + (uint32_t)((t.c + 63) / 64) * 64 * 128;  // shared down: 64-row boxes
+  }
   DG_DEVINL static bool acquire(const Params& p, const Tile& t, volatile int* abort, int* err) {
     return t.e != 1 || counter_wait_bounded(p.ready + t.f, p.FJ, abort, err);
   }
@@ -597,7 +608,7 @@ struct P_EXP : ProblemBase {
       P_ED::load(p.dn, t, kb, sa, sb, bar);
     } else {
       tma_load_2d(sa, &p.tmSW, kb * 64, t.a * 128, bar);
-      tma_load_2d(sb, &p.tmHS, kb * 64, t.b * BN, bar);
+      for (int i = 0; i < t.c; i += 64) tma_load_2d(sb + i * 128, &p.tmHS, kb * 64, t.b * BN + i, bar);
     }
   }
   DG_DEVINL static void epilogue(const Params& p, const Tile& t, uint32_t taddr, int q, int lane, int row,

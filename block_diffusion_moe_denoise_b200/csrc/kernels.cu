@@ -485,7 +485,8 @@ __global__ void __launch_bounds__(512) k_group_gather(GroupArgs a, const unsigne
     for (int i = 0; i < 8; ++i) {
       const int e = lane * 8 + i;
       v[i] = e < E ? cnt[e] : 0;
-      tv[i] = e < E ? (cnt[e] + kExpertRows - 1) / kExpertRows : 0;
+      constexpr int kTileRows = kF8 ? kExpertRows : kExpertTileRows;  // token rows per expert tile
+      tv[i] = e < E ? (cnt[e] + kTileRows - 1) / kTileRows : 0;
     }
     const int tot = warp_excl_scan8(v, lane);
     const int ttot = warp_excl_scan8(tv, lane);
