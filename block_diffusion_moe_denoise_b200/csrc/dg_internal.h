@@ -70,8 +70,9 @@ struct QkvArgs {
 constexpr int kMaxPartSplits = 8;
 constexpr int kExpertRows = 64;       // token rows per FP8 routed-expert GEMM tile
 constexpr int kExpertTileRows = 128;  // token rows per bf16 routed-expert tile (and shared-down tile)
-constexpr int kExpertBoxRows = 64;    // rows per TMA box of the bf16 grouped rows (boxes of 16 rows,
-                                      // four times the copies, measured slower on B200)
+constexpr int kExpertBoxRows = 64;    // rows per TMA box of the bf16 grouped rows (measured slower on
+                                      // B200: 16-row boxes throughout, and 32/16-row boxes for the rows
+                                      // past a tile's last full 64, though both move fewer bytes)
 struct WpartArgs {
   const CUtensorMap* tm_w;  // weights [d, K], 128-row boxes
   const CUtensorMap* tm_x;  // activations [Tcap, K], 256-row boxes
