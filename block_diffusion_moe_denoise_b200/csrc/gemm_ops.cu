@@ -762,20 +762,40 @@ struct P_ED8 : ProblemBase {
     tma_load_2d(sa, &p.tmW, kb * 128, t.a * p.d + t.b * 128, bar);
     tma_load_2d(sb, &p.tmH, kb * 128, t.d, bar);
   }
-  DG_DEVINL static void epilogue(const Params& p, const Tile& t, uint32_t taddr, int, int, int row, uint8_t*) {
-    const int f = t.b * 128 + row;
-    const float sw = p.sw[(size_t)t.a * p.d + f];
+  // Transposed through shared memory as in P_ED: thread = output feature
+  // stages v * (its weight row's scale), each warp then applies a token row's
+  // scale and gate weight and stores 256-byte row segments of yp.  The
+  // products are those of w_r * ((v * s_w) * s_h), in that order.
+  static constexpr int EP_SMEM = 16 * 128 * 4;
+  DG_DEVINL static void epilogue(const Params& p, const Tile& t, uint32_t taddr, int q, int lane, int row,
+                                 uint8_t* ep) {
+    float* stg = reinterpret_cast<float*>(ep);  // [16 tokens][128 features]
+    const float sw = p.sw[(size_t)t.a * p.d + t.b * 128 + row];
     for (int c0 = 0; c0 < t.n_mma; c0 += 16) {
+      float w[4], sh[4];  // gate weights and row scales of the token rows this warp stores: c0 + q + 4 j
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int c = c0 + q + 4 * j;
+        w[j] = c < t.c ? __ldcg(p.row_weight + t.d + c) : 0.f;
+        sh[j] = c < t.c ? __ldcg(p.sh + t.d + c) : 0.f;
+      }
       float v[16];
       tmem_ld16(taddr + c0, v);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int c = c0 + i;
+      for (int i = 0; i < 16; ++i) stg[i * 128 + row] = v[i] * sw;
+      named_bar_sync(1, 128);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int c = c0 + q + 4 * j;
         if (c < t.c) {
-          const int r = t.d + c;
-          p.yp[(size_t)r * p.d + f] = __float2bfloat16_rn(p.row_weight[r] * (v[i] * sw * p.sh[r]));
+          const float4 a = *reinterpret_cast<const float4*>(stg + (q + 4 * j) * 128 + 4 * lane);
+          uint2 o;
+          o.x = pack_bf16x2(w[j] * (a.x * sh[j]), w[j] * (a.y * sh[j]));
+          o.y = pack_bf16x2(w[j] * (a.z * sh[j]), w[j] * (a.w * sh[j]));
+          *reinterpret_cast<uint2*>(p.yp + (size_t)(t.d + c) * p.d + t.b * 128 + 4 * lane) = o;
         }
       }
+      named_bar_sync(1, 128);  // staging free for the next 16 tokens
     }
   }
 };
