@@ -404,6 +404,7 @@ def main():
     cfg = cfg.with_(temperature=args.temperature, ffn_selfcond=args.selfcond,
                     expert_fp8=1 if args.fp8_experts else 0)
     hbm_gbs, bf16_tf, bf16_tf_sus, peak_kind = measured_peaks()
+    peak_note = "MEASURED_PEAKS.json" if peak_kind == "measured" else "no MEASURED_PEAKS.json: the pool's earlier measurement"
     # a whole step, and a kernel timed inside it, run long enough to settle at the
     # power-capped clock: the sustained bf16 figure is their tensor peak
     bf16_tf_step = bf16_tf_sus or bf16_tf
@@ -595,7 +596,7 @@ def main():
                            "experts (routed-expert gate|up GEMM + SwiGLU + down GEMM, one launch)"), "bound": "hbm",
                 "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s", "frac": achieved / hbm_gbs,
                 "traffic": traffic, "algorithmic_bytes_per_launch": egu_bytes,
-                "avg_launch_ms": egu_avg_ms, "peak_source": f"{peak_kind} HBM copy (MEASURED_PEAKS.json)"}
+                "avg_launch_ms": egu_avg_ms, "peak_source": f"{peak_kind} HBM copy ({peak_note})"}
     if long_ctx:
         # the dominant kernel of the long-context step is the canvas attention
         # (k_attn_tc, with its split-KV merge in-kernel, once per layer)
@@ -607,7 +608,7 @@ def main():
         roofline = {"kernel": "attention (k_attn_tc, split-KV merge in its clusters, per layer: 4 requests x 65792 keys)",
                     "bound": "tensor", "achieved": tf, "peak": bf16_tf_step, "unit": "TFLOP/s", "frac": tf / bf16_tf_step,
                     "traffic": None, "algorithmic_flops_per_launch": at_flops, "avg_launch_ms": at_avg,
-                    "peak_source": f"{peak_kind} bf16 dense sustained (MEASURED_PEAKS.json): a kernel inside a long step"}
+                    "peak_source": f"{peak_kind} bf16 dense sustained ({peak_note}): a kernel inside a long step"}
     line = {
         "metric": METRIC,
         "value": value,
