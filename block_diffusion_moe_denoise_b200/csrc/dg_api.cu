@@ -258,12 +258,14 @@ struct dg_handle {
   int egu_cap = 0, ed_cap = 0;
   long long kv_req_stride = 0, kv_layer_stride = 0;
   std::vector<LayerMaps> maps;
+  CUtensorMap tm_u32;
   CUtensorMap tm_hn, tm_o, tm_o128, tm_u, tm_u64, tm_xp, tm_hp, tm_hs, tm_hs64, tm_embed, tm_embed128, tm_k, tm_vt;
   CUtensorMap tm_sc_gate, tm_sc_up, tm_sc_down, tm_hs_sc;  // self-conditioning MLP and its hidden rows
   CUtensorMap tm_xq, tm_hq;                                // FP8 experts: token and hidden codes
   long long cap_user = 0;  // capacity the caller asked for (cap is rounded up to 64)
   ReqState req[DG_MAX_REQUESTS];
   int mask_flip = 0;  // which of the two routing bitmask buffers the next layer uses
+  bool keep_router_logits = false;  // debug passes keep the router's fp32 logits for inspection
   long long lm_seq = 0;  // LM-head passes so far: the "stats" / "argmax" buffers hold the latest
 
   template <class T>
@@ -473,6 +475,7 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     SharedArgs sa;
     sa.tm_u = &h->tm_u;
     sa.tm_u64 = &h->tm_u64;
+    sa.tm_u32 = &h->tm_u32;
     sa.tm_gate = &m.sgate;
     sa.tm_up = &m.sup;
     sa.tm_router = &m.router;
@@ -484,7 +487,7 @@ int run_pass(dg_handle* h, const int* const* ids, const SlotInfo& s, int n_layer
     sa.k = k;
     sa.MW = MW;
     sa.hs = h->B<bf16>("hs");
-    sa.logits = h->B<float>("router_logits");
+    sa.logits = h->keep_router_logits ? h->B<float>("router_logits") : nullptr;  // nothing else reads them
     sa.idx = h->B<int>("idx");
     sa.w = h->B<float>("w");
     sa.mask = mask_cur;
@@ -759,6 +762,7 @@ int dg_init(const dg_config* cfg, const dg_weights* wts, int max_requests, int64
   ok = ok && make_map(&h->tm_o128, h->B<bf16>("o"), (long long)c.n_q_heads * D, h->Tcap, 128);
   ok = ok && make_map(&h->tm_u, h->B<bf16>("u"), d, h->Tcap, 128);
   ok = ok && make_map(&h->tm_u64, h->B<bf16>("u"), d, h->Tcap, 64);
+  ok = ok && make_map(&h->tm_u32, h->B<bf16>("u"), d, h->Tcap, 32);
   ok = ok && make_map(&h->tm_xp, h->B<bf16>("xp"), d, rows, kExpertBoxRows);
   ok = ok && make_map(&h->tm_hp, h->B<bf16>("hp"), c.ffn_expert, rows, kExpertBoxRows);
   ok = ok && make_map(&h->tm_hs, h->B<bf16>("hs"), c.ffn_shared, h->Tcap, 256);
@@ -1366,7 +1370,10 @@ int dg_debug_forward(dg_handle* h, int req, const int32_t* d_tokens, int T, int 
   s.req[0] = req;
   s.pos0[0] = (int)r.kv_len;
   const int* ids[1] = {d_tokens};
-  return run_pass(h, ids, s, n_layers, false, n_layers == h->cfg.n_layers, nullptr);
+  h->keep_router_logits = true;
+  const int rc2 = run_pass(h, ids, s, n_layers, false, n_layers == h->cfg.n_layers, nullptr);
+  h->keep_router_logits = false;
+  return rc2;
 }
 
 int dg_debug_forward_hidden(dg_handle* h, int req, const int32_t* d_tokens, const float* d_x, int T, int layer0,
@@ -1385,8 +1392,11 @@ int dg_debug_forward_hidden(dg_handle* h, int req, const int32_t* d_tokens, cons
   s.req[0] = req;
   s.pos0[0] = (int)r.kv_len;
   const int* ids[1] = {d_tokens};
-  return run_pass(h, ids, s, n_layers, false, layer0 + n_layers == h->cfg.n_layers, nullptr, -1, nullptr, 0.f,
-                  nullptr, layer0, d_x);
+  h->keep_router_logits = true;
+  const int rc2 = run_pass(h, ids, s, n_layers, false, layer0 + n_layers == h->cfg.n_layers, nullptr, -1, nullptr,
+                           0.f, nullptr, layer0, d_x);
+  h->keep_router_logits = false;
+  return rc2;
 }
 
 int dg_profile(dg_handle* h, int enable) {

@@ -107,6 +107,7 @@ struct ExpertArgs {
 struct SharedArgs {
   const CUtensorMap *tm_u, *tm_gate, *tm_up, *tm_router;
   const CUtensorMap* tm_u64;  // the normed tokens in 64-row boxes (router tiles of 64 tokens), or null
+  const CUtensorMap* tm_u32 = nullptr;  // ... in 32-row boxes (router tiles of 32 tokens), or null
   int T, d, fs, num_sms;
   int E, k, MW;       // router: experts (multiple of 16, <= 128), top-k, bitmask words per expert
   bf16* hs;

@@ -820,11 +820,11 @@ struct P_SGU : ProblemBase {
     CUtensorMap tmG;  // ws_gate [fs, d], 32-row boxes
     CUtensorMap tmU;  // ws_up [fs, d], 32-row boxes
     CUtensorMap tmR;  // w_router [E, d], E-row boxes
-    CUtensorMap tmX64;  // normed tokens, 64-row boxes (router tiles of 64 tokens)
+    CUtensorMap tmXR;   // normed tokens in RR-row boxes (the router tiles' token rows)
     int T, nk, MT, FJ, fs, E, k, MW;
-    int RH;             // 1: a router tile covers 64 tokens (see router_tiles)
+    int RR;             // tokens per router tile: 128, 64 or 32 (see router_tiles)
     __nv_bfloat16* hs;  // [Tcap, fs]
-    float* logits;      // [Tcap, E]
+    float* logits;      // [Tcap, E], or nullptr: not written
     int* idx;           // [T, k]
     float* w;           // [T, k]
     unsigned* mask;     // [E][MW] token bitmasks (zero on entry)
@@ -838,13 +838,11 @@ struct P_SGU : ProblemBase {
     if (p.E > 0) tma_prefetch_desc(&p.tmR);
   }
   // E == 0: a plain gated MLP (no router tile), as used for self-conditioning.
-  // With RH a router tile takes 64 tokens (one 64-row box in the first half of
-  // the A stage; MMA rows 64..127 are ignored): it then streams 64 + E rows per
-  // k-block, no more than a shared tile's 128 + 2 * kHid, instead of 128 + E,
-  // so the router no longer outlasts the shared tiles.
-  DG_DEVINL static int router_tiles(const Params& p) {
-    return p.E > 0 ? (p.RH ? (p.T + 63) / 64 : p.MT) : 0;
-  }
+  // A router tile takes RR tokens (one RR-row box at the start of the A stage;
+  // MMA rows RR..127 are ignored): with RR < 128 it streams RR + E rows per
+  // k-block, fewer than a shared tile's 128 + 2 * kHid, so the router tiles,
+  // whose top-k epilogue is longer, no longer outlast the shared tiles.
+  DG_DEVINL static int router_tiles(const Params& p) { return p.E > 0 ? (p.T + p.RR - 1) / p.RR : 0; }
   DG_DEVINL static int num_tiles(const Params& p) { return router_tiles(p) + p.MT * p.FJ; }
   DG_DEVINL static Tile tile(const Params& p, int v) {
     Tile t;
@@ -863,7 +861,7 @@ struct P_SGU : ProblemBase {
     return t;
   }
   DG_DEVINL static uint32_t tx_bytes(const Params& p, const Tile& t) {
-    return (t.b < 0 && p.RH ? kAStage / 2 : kAStage) + (t.b < 0 ? p.E : 2 * kHid) * 128;
+    return (t.b < 0 ? (uint32_t)p.RR * 128 : kAStage) + (t.b < 0 ? p.E : 2 * kHid) * 128;
   }
   DG_DEVINL static void load_w(const Params& p, const Tile& t, int kb, uint32_t, uint32_t sb, uint64_t* bar) {
     if (t.b < 0) {
@@ -874,8 +872,8 @@ struct P_SGU : ProblemBase {
     }
   }
   DG_DEVINL static void load_x(const Params& p, const Tile& t, int kb, uint32_t sa, uint32_t, uint64_t* bar) {
-    if (t.b < 0 && p.RH)
-      tma_load_2d(sa, &p.tmX64, kb * 64, t.a * 64, bar);
+    if (t.b < 0)
+      tma_load_2d(sa, &p.tmXR, kb * 64, t.a * p.RR, bar);
     else
       tma_load_2d(sa, &p.tmX, kb * 64, t.a * 128, bar);
   }
@@ -896,9 +894,11 @@ struct P_SGU : ProblemBase {
       float z[16];
       tmem_ld16(taddr + c0, z);
       if (!ok) continue;
-      float4* lg = reinterpret_cast<float4*>(p.logits + (size_t)tok * p.E + c0);
+      if (p.logits != nullptr) {  // kept for inspection only
+        float4* lg = reinterpret_cast<float4*>(p.logits + (size_t)tok * p.E + c0);
 #pragma unroll
-      for (int i = 0; i < 16; i += 4) lg[i / 4] = make_float4(z[i], z[i + 1], z[i + 2], z[i + 3]);
+        for (int i = 0; i < 16; i += 4) lg[i / 4] = make_float4(z[i], z[i + 1], z[i + 2], z[i + 3]);
+      }
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         // Experts arrive in ascending id order; strict comparisons keep the
@@ -943,10 +943,7 @@ struct P_SGU : ProblemBase {
   }
   DG_DEVINL static void epilogue(const Params& p, const Tile& t, uint32_t taddr, int, int, int row, uint8_t*) {
     if (t.b < 0) {
-      if (p.RH)
-        router_epilogue(p, t.a * 64 + row, row < 64, taddr);
-      else
-        router_epilogue(p, t.a * 128 + row, true, taddr);
+      router_epilogue(p, t.a * p.RR + row, row < p.RR, taddr);
       return;
     }
     const int tok = t.a * 128 + row;
@@ -1419,10 +1416,18 @@ cudaError_t run_shared_gate_up(const SharedArgs& a, cudaStream_t st) {
   g.w = a.w;
   g.mask = a.mask;
   g.err = a.err;
-  // router tiles of 64 tokens when they and the shared tiles still fit in one wave
-  g.RH = (a.E > 0 && a.tm_u64 != nullptr && (a.T + 63) / 64 + g.MT * g.FJ <= a.num_sms) ? 1 : 0;
-  g.tmX64 = g.RH ? *a.tm_u64 : *a.tm_u;
-  const int router = a.E > 0 ? (g.RH ? (a.T + 63) / 64 : g.MT) : 0;  // P_SGU::router_tiles
+  // router tiles of 32 or 64 tokens while they and the shared tiles still fit in one wave
+  const int shared_tiles = g.MT * g.FJ;
+  g.RR = 128;
+  g.tmXR = *a.tm_u;
+  if (a.E > 0 && a.tm_u32 != nullptr && (a.T + 31) / 32 + shared_tiles <= a.num_sms) {
+    g.RR = 32;
+    g.tmXR = *a.tm_u32;
+  } else if (a.E > 0 && a.tm_u64 != nullptr && (a.T + 63) / 64 + shared_tiles <= a.num_sms) {
+    g.RR = 64;
+    g.tmXR = *a.tm_u64;
+  }
+  const int router = a.E > 0 ? (a.T + g.RR - 1) / g.RR : 0;  // P_SGU::router_tiles
   return launch_gemm<P_SGU>(g, grid_for(router + g.MT * g.FJ, a.num_sms), st);
 }
 

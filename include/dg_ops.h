@@ -81,7 +81,8 @@ int dg_debug_forward_hidden(dg_handle* h, int req, const int32_t* d_tokens, cons
 /* Byte offset and size, inside the workspace, of a named internal buffer:
  * "x" f32 [T, d] residual stream; "hn" bf16 [T, d] normed input of the last
  * projection; "q" bf16 [Hq, Tcap, D]; "o" bf16 [T, Hq*D]; "u" bf16 [T, d];
- * "router_logits" f32 [T, E]; "idx" i32 [T, k]; "w" f32 [T, k];
+ * "router_logits" f32 [T, E] (written by the dg_debug_forward passes only);
+ * "idx" i32 [T, k]; "w" f32 [T, k];
  * "counts" i32 [E]; "offsets" i32 [E+1];
  * "pair_row" i32 [T*k]; "row_pair" i32 [T*k]; "hp" bf16 [T*k, fe];
  * "yp" bf16 [T*k, d]; "hs" bf16 [T, fs]; "stats" f32 [Tcap][4];
