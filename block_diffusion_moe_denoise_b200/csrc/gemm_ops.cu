@@ -524,16 +524,18 @@ struct P_ED : ProblemBase {
 // ---------------------------------------------------------------------------
 // Routed experts, gate|up + SwiGLU and down projection, and the shared
 // expert's down projection, in one persistent launch.  The tile queue holds
-// every gate|up tile (in expert order), then the shared-down tiles (128
-// output features x 128 tokens over the whole shared hidden width, written
-// straight to the fp32 partial the residual norm adds), then every down tile
-// (in expert order): CTAs that finish gate|up work take shared-down tiles
-// while the first down tiles' inputs are completed.  A down tile reads the SwiGLU rows of one
+// the shared-down tiles (128 output features x 128 tokens over the whole
+// shared hidden width, written straight to the fp32 partial the residual norm
+// adds; they depend on nothing in the launch), then every gate|up tile (in
+// expert order), then every down tile (in expert order).  (The shared-down
+// tiles queued between the gate|up and the down tiles, or among the down
+// tiles, measured slower on B200.)  A down tile reads the SwiGLU rows of one
 // token tile of its expert, which that token tile's FJ gate|up tiles write;
 // each of their epilogues adds one to ready[tt] (tt: the token tile's index
-// over all experts) once its rows are stored, and the producer of the down
-// tile waits for FJ before loading them.  All gate|up tiles come first in the
-// queue, so no wait depends on a tile not yet taken (see the engine header).
+// over all experts) once its rows are stored, and the scheduler waits for FJ
+// before handing the down tile on.  All gate|up tiles come before the down
+// tiles in the queue, so no wait depends on a tile not yet taken (see the
+// engine header).
 // The down tiles of the first experts start while the last gate|up tiles
 // still run: no gate|up tail and down ramp between two launches.
 // ---------------------------------------------------------------------------
@@ -571,12 +573,12 @@ struct P_EXP : ProblemBase {
   DG_DEVINL static Tile tile(const Params& p, int v) {
     const int ng = *p.gu.n_tiles;
     Tile t;
-    if (v < ng) {
-      t = P_EGU::tile(p.gu, v);
+    if (v >= p.n_sd && v < p.n_sd + ng) {
+      t = P_EGU::tile(p.gu, v - p.n_sd);
       t.e = 0;
-      t.f = p.gu.tiles[v].w;
-    } else if (v < ng + p.n_sd) {
-      const int u = v - ng;
+      t.f = p.gu.tiles[v - p.n_sd].w;
+    } else if (v < p.n_sd) {
+      const int u = v;
       t.a = u % p.sd_fb;  // 128-feature block
       t.b = u / p.sd_fb;  // BN-token tile
       t.c = min(BN, p.T - t.b * BN);

@@ -70,7 +70,8 @@ struct Tile {
 };
 
 constexpr int kAStage = 128 * 128;  // 128 rows x 128 bytes
-constexpr int kSchedRing = 3;       // tiles in flight between the scheduler and the other roles (DYNAMIC)
+constexpr int kSchedRing = 2;       // tiles in flight between the scheduler and the other roles (DYNAMIC);
+                                    // deeper rings claim tiles too far ahead (measured slower: 3, 4, 8)
 
 // Threads of a block: producer, MMA and four epilogue warps, plus the scheduler
 // warp of DYNAMIC problems.
